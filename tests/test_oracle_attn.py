@@ -1,0 +1,135 @@
+"""Pins of the oracle's sparse + sliding-window attention against textbook
+special cases (hackernews.kjhq.dev post 49735410, key point 2: local sliding
+windows plus global sparse retrieval; tldrocket.com "DeepSeek AI Released
+DeepSeek-V4.1-Flash ...", paragraph 2: a 128-token window in every layer)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import read_golden
+from fp4_sparse_attention_csa2_b200 import workloads as wl
+from harness import build_ref_cache
+
+E2M1 = {int(c, 16): float(v) for c, v in read_golden("e2m1_values.txt")}
+
+
+def _decode_rows_lib(cache, b, positions, D):
+    """Rows decoded without the oracle: golden E2M1 table x torch's E4M3 scale."""
+    out = np.zeros((len(positions), D))
+    for i, t in enumerate(positions):
+        row = cache.rows[cache.slot(b, int(t))]
+        sc = torch.from_numpy(row[D // 2:D // 2 + D // 16].copy()).view(torch.float8_e4m3fn).double().numpy()
+        codes = np.empty(D, dtype=np.int64)
+        codes[0::2] = row[:D // 2] & 0xF
+        codes[1::2] = row[:D // 2] >> 4
+        out[i] = np.array([E2M1[c] for c in codes]) * np.repeat(sc, 16)
+    return out
+
+
+def _numpy_attn(q_bf16, V, scale):
+    q = q_bf16.double().numpy()
+    z = scale * (q @ V.T)                                # [H, n]
+    p = torch.softmax(torch.from_numpy(z), dim=1).numpy()
+    lse = torch.logsumexp(torch.from_numpy(z), dim=1).numpy()
+    return p @ V, lse
+
+
+def _setup(L=700, T=1, **kw):
+    w = wl.scaled(wl.WORKLOADS["tiny4k"], L, T=T, **kw)
+    cache = build_ref_cache(w)
+    q = wl.layer_queries(w, 2)["q"]
+    return w, cache, q
+
+
+def test_topk_covering_context_equals_dense():
+    w, cache, q = _setup(700)
+    p = 699
+    topk = np.arange(p + 1, dtype=np.int32)[::-1].copy()
+    out, lse = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window)
+    dout, dlse = oracle.dense_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]))
+    V = _decode_rows_lib(cache, 0, range(p + 1), w.D)
+    nout, nlse = _numpy_attn(q[0, 0], V, 1 / np.sqrt(w.D))
+    assert np.allclose(out, dout, rtol=0, atol=1e-12) and np.allclose(lse, dlse, atol=1e-12)
+    assert np.allclose(out, nout, rtol=0, atol=1e-12) and np.allclose(lse, nlse, atol=1e-12)
+
+
+def test_empty_topk_is_dense_over_window():
+    w, cache, q = _setup(700)
+    topk = np.full(w.top_k, -1, dtype=np.int32)
+    out, lse = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window)
+    V = _decode_rows_lib(cache, 0, range(700 - w.window, 700), w.D)
+    nout, nlse = _numpy_attn(q[0, 0], V, 1 / np.sqrt(w.D))
+    assert np.allclose(out, nout, atol=1e-12) and np.allclose(lse, nlse, atol=1e-12)
+
+
+def test_sparse_plus_window_equals_numpy_over_union():
+    w, cache, q = _setup(900)
+    rng = np.random.default_rng(1)
+    topk = rng.choice(900, w.top_k, replace=False).astype(np.int32)
+    topk[:10] = -1
+    out, lse = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window, 0.07)
+    S = sorted(set(range(900 - w.window, 900)) | set(int(t) for t in topk if t >= 0))
+    V = _decode_rows_lib(cache, 0, S, w.D)
+    nout, nlse = _numpy_attn(q[0, 0], V, 0.07)
+    assert np.allclose(out, nout, atol=1e-12) and np.allclose(lse, nlse, atol=1e-12)
+    assert max(np.sum(topk >= 0), w.window) <= len(S) <= np.sum(topk >= 0) + w.window
+
+
+def test_invariant_under_permutation_and_window_duplicates():
+    w, cache, q = _setup(900)
+    rng = np.random.default_rng(2)
+    topk = rng.choice(700, w.top_k, replace=False).astype(np.int32)
+    base, blse = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window)
+    perm = rng.permutation(topk)
+    out, lse = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), perm, w.window)
+    assert np.array_equal(out, base) and np.array_equal(lse, blse)
+    dup = topk.copy()
+    dup[:20] = np.arange(880, 900)                    # window positions repeated in top-k
+    a, _ = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), dup, w.window)
+    b, _ = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk[20:].copy(), w.window)
+    assert np.array_equal(a, b)
+
+
+def test_window_shorter_than_context_start():
+    # p + 1 < W: the window is [0, p]
+    w, cache, q = _setup(50)
+    topk = np.full(w.top_k, -1, dtype=np.int32)
+    out, _ = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window)
+    dout, _ = oracle.dense_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]))
+    assert np.allclose(out, dout, atol=1e-12)
+
+
+def test_multi_token_causal():
+    # token j of T sees positions <= p_j = L - T + j only, in top-k and window
+    T = 4
+    w, cache, q = _setup(600, T=T)
+    topk = np.arange(600, dtype=np.int32)              # includes the later tokens' positions
+    for j in range(T):
+        out, _ = oracle.sparse_swa_attn(cache, 0, T, j, wl.bf16_bits(q[0, j]), topk, w.window)
+        dout, _ = oracle.dense_attn(cache, 0, T, j, wl.bf16_bits(q[0, j]))
+        assert np.allclose(out, dout, atol=1e-12)
+
+
+def test_out_of_range_index_is_an_error():
+    w, cache, q = _setup(300)
+    topk = np.zeros(w.top_k, dtype=np.int32)
+    topk[5] = 300
+    with pytest.raises(RuntimeError):
+        oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window)
+
+
+def test_paged_equals_contiguous():
+    base = wl.scaled(wl.WORKLOADS["batch32_paged"], 900, batch=3, lens=("uniform", 300, 900))
+    contig = wl.Workload(**{**base.__dict__, "paged": False, "name": "contig"})
+    cp = build_ref_cache(base)
+    cc = build_ref_cache(contig)
+    assert np.array_equal(cp.seq_lens, cc.seq_lens)
+    layers = [wl.layer_queries(base, l) for l in range(2)]
+    hl = [{k: wl.host_array(v) for k, v in L.items()} for L in layers]
+    rp = oracle.run_stack(cp, "FR", hl, 1, base.pool_k, base.top_k, base.window, base.q_idx_dtype)
+    rc = oracle.run_stack(cc, "FR", hl, 1, base.pool_k, base.top_k, base.window, base.q_idx_dtype)
+    for l in range(2):
+        for key in rp[l]:
+            assert np.array_equal(rp[l][key][1], rc[l][key][1])
+            assert np.array_equal(rp[l][key][2], rc[l][key][2])

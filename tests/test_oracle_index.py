@@ -1,0 +1,155 @@
+"""Pins of the oracle's indexer (Full / Reindex / Reuse selection) against
+library routines and the bounds the pages print: the candidate pool holds at
+most 16,384 positions and Reuse layers take the indices unchanged
+(tldrocket.com "DeepSeek AI Released DeepSeek-V4.1-Flash ...", paragraph 3;
+hackernews.kjhq.dev post 49735410, key point 2)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_sparse_attention_csa2_b200 import workloads as wl
+from harness import build_ref_cache, host_layer
+
+
+def _small(name, L, **kw):
+    return wl.scaled(wl.WORKLOADS[name], L, **kw)
+
+
+def _keys_f64(cache, b, n):
+    """Stored index keys of positions 0..n-1 decoded by the library (torch fp8)."""
+    slots = np.array([cache.slot(b, t) for t in range(n)])
+    k = cache.idx_keys[slots]
+    if cache.idx_key_dtype == oracle.E4M3:
+        return torch.from_numpy(k.copy()).view(torch.float8_e4m3fn).double().numpy()
+    return k.astype(np.float64)
+
+
+def _q_f64(q):
+    return q.double().numpy() if isinstance(q, torch.Tensor) else np.asarray(q, dtype=np.float64)
+
+
+@pytest.mark.parametrize("name,L", [("tiny4k", 1000), ("long64k", 3000)])
+def test_scores_equal_numpy_gemm_relu_weighted_sum(name, L):
+    w = _small(name, L)
+    cache = build_ref_cache(w, rows=False)
+    lay = wl.layer_queries(w, 0)
+    qi, hw = lay["q_idx"][0, 0], lay["w"][0, 0]
+    pos = np.arange(L, dtype=np.int32)
+    s = oracle.index_scores(cache, 0, pos, wl.host_array(qi), w.q_idx_dtype, hw.numpy())
+    K = _keys_f64(cache, 0, L)
+    want = np.maximum(K @ _q_f64(qi).T, 0.0) @ hw.double().numpy()   # BLAS GEMM
+    assert np.allclose(s, want, rtol=1e-12, atol=1e-12)
+
+
+def test_single_head_positive_dot_is_plain_dot():
+    w = _small("tiny4k", 300, H_I=1)
+    cache = build_ref_cache(w, rows=False)
+    q = torch.randn(1, 64, generator=torch.Generator().manual_seed(5))
+    K = _keys_f64(cache, 0, 300)
+    pos = np.arange(300, dtype=np.int32)
+    s = oracle.index_scores(cache, 0, pos, q.numpy(), oracle.F32, np.ones(1, np.float32))
+    dots = K @ q.double().numpy()[0]
+    assert np.allclose(s[dots > 0], dots[dots > 0], rtol=1e-13, atol=0)
+    assert np.all(s[dots <= 0] == 0)
+
+
+def test_select_top_equals_full_sort():
+    rng = np.random.default_rng(0)
+    for n, k in [(10, 3), (1000, 128), (5000, 5000), (50, 80)]:
+        s = rng.standard_normal(n)
+        s[rng.integers(0, n, n // 5)] = 0.5          # plenty of exact ties
+        got = oracle.select_top(s, None, k)
+        order = np.lexsort((np.arange(n), -s))       # score desc, position asc
+        want = np.full(k, -1, dtype=np.int32)
+        want[:min(k, n)] = order[:k]
+        assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_full_pool_and_topk_bounds(T):
+    w = _small("tiny4k", 2000, T=T)
+    cache = build_ref_cache(w, rows=False)
+    lay = wl.layer_queries(w, 0)
+    for j in range(T):
+        p = 2000 - T + j
+        pool, topk, s = oracle.index_full(cache, 0, T, j, wl.host_array(lay["q_idx"][0, j]), w.q_idx_dtype,
+                                          lay["w"][0, j].numpy(), w.pool_k, w.top_k, want_scores=True)
+        assert s.size == p + 1                                 # causal: t <= p_j only
+        assert np.sum(pool >= 0) == min(w.pool_k, p + 1)
+        assert np.sum(topk >= 0) == min(w.top_k, p + 1)
+        assert set(topk[topk >= 0]) <= set(pool[pool >= 0])   # k is a subset of K
+        assert pool.max() <= p
+        order = np.lexsort((np.arange(p + 1), -s))
+        assert np.array_equal(pool, order[:w.pool_k])
+
+
+def test_pool_shorter_than_k_is_padded():
+    w = _small("tiny4k", 100)
+    cache = build_ref_cache(w, rows=False)
+    lay = wl.layer_queries(w, 0)
+    pool, topk, _ = oracle.index_full(cache, 0, 1, 0, wl.host_array(lay["q_idx"][0, 0]), w.q_idx_dtype,
+                                      lay["w"][0, 0].numpy(), 512, 128)
+    assert np.sum(pool >= 0) == 100 and np.all(pool[100:] == -1)
+    assert np.sum(topk >= 0) == 100
+
+
+def test_pool_bound_16384():
+    w = _small("tiny4k", 100)
+    cache = build_ref_cache(w, rows=False)
+    lay = wl.layer_queries(w, 0)
+    with pytest.raises(RuntimeError):
+        oracle.index_full(cache, 0, 1, 0, wl.host_array(lay["q_idx"][0, 0]), w.q_idx_dtype,
+                          lay["w"][0, 0].numpy(), 16385, 128)
+    with pytest.raises(RuntimeError):
+        oracle.index_full(cache, 0, 1, 0, wl.host_array(lay["q_idx"][0, 0]), w.q_idx_dtype,
+                          lay["w"][0, 0].numpy(), 64, 128)
+
+
+def test_reindex_with_whole_context_pool_equals_full_selection():
+    # pool = every position (L <= K): Reindex == Full selection with the Reindex query
+    w = _small("long64k", 1500)
+    cache = build_ref_cache(w, rows=False)
+    l0, l1 = wl.layer_queries(w, 0), wl.layer_queries(w, 1)
+    pool, _, _ = oracle.index_full(cache, 0, 1, 0, wl.host_array(l0["q_idx"][0, 0]), w.q_idx_dtype,
+                                   l0["w"][0, 0].numpy(), w.pool_k, w.top_k)
+    assert np.sum(pool >= 0) == 1500
+    re_topk, _ = oracle.index_reindex(cache, 0, 1, 0, wl.host_array(l1["q_idx"][0, 0]), w.q_idx_dtype,
+                                      l1["w"][0, 0].numpy(), pool, w.top_k)
+    _, full_topk, _ = oracle.index_full(cache, 0, 1, 0, wl.host_array(l1["q_idx"][0, 0]), w.q_idx_dtype,
+                                        l1["w"][0, 0].numpy(), w.pool_k, w.top_k)
+    assert np.array_equal(re_topk, full_topk)
+
+
+def test_reindex_scores_only_the_pool():
+    w = _small("tiny4k", 3000)
+    cache = build_ref_cache(w, rows=False)
+    l0, l1 = wl.layer_queries(w, 0), wl.layer_queries(w, 1)
+    pool, _, _ = oracle.index_full(cache, 0, 1, 0, wl.host_array(l0["q_idx"][0, 0]), w.q_idx_dtype,
+                                   l0["w"][0, 0].numpy(), w.pool_k, w.top_k)
+    topk, s = oracle.index_reindex(cache, 0, 1, 0, wl.host_array(l1["q_idx"][0, 0]), w.q_idx_dtype,
+                                   l1["w"][0, 0].numpy(), pool, w.top_k, want_scores=True)
+    assert set(topk) <= set(pool)
+    order = np.lexsort((pool, -s))
+    assert np.array_equal(topk, pool[order[:w.top_k]])
+
+
+def test_planted_keys_are_selected():
+    # the planted positions (cosine 0.9 with the query direction) score far
+    # above the N(0,1) background, so every one of them lands in the top-k
+    w = _small("long64k", 8192)
+    cache = build_ref_cache(w, rows=False)
+    l0 = wl.layer_queries(w, 0)
+    _, planted = wl.index_keys(w, 0, 8192, l0["q_idx"][0, 0])
+    _, topk, _ = oracle.index_full(cache, 0, 1, 0, wl.host_array(l0["q_idx"][0, 0]), w.q_idx_dtype,
+                                   l0["w"][0, 0].numpy(), w.pool_k, w.top_k)
+    assert set(planted.tolist()) <= set(topk.tolist())
+
+
+def test_reuse_passes_indices_through_unchanged():
+    w = _small("tiny4k", 1200)
+    cache = build_ref_cache(w)
+    layers = [host_layer(wl.layer_queries(w, l)) for l in range(3)]
+    res = oracle.run_stack(cache, "FRU", layers, 1, w.pool_k, w.top_k, w.window, w.q_idx_dtype)
+    assert np.array_equal(res[1][(0, 0)][1], res[2][(0, 0)][1])
+    assert res[1][(0, 0)][1].tobytes() == res[2][(0, 0)][1].tobytes()
