@@ -1,0 +1,485 @@
+"""Benchmark: CSA2 decode layer-steps/s on the 1M-context stack, with the
+indexer kernel's HBM roofline fraction, an end-to-end number through the C ABI
+with host buffers, and the CPU oracle as a reported baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload ctx1m]
+
+One step = one decode step of the whole layer stack (ctx1m: Full, Reindex and
+six Reuse layers for one 1,048,576-token sequence).  The metric counts layer
+executions per second over all ranks.  Under torchrun every rank runs its own
+sequence (weak scaling over independent sequences, no data-path collective).
+"""
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp4_sparse_attention_csa2_b200 import workloads as wl  # noqa: E402
+
+METRIC = "CSA2 decode layer-steps/s at 1M ctx; FP4-KV achieved HBM GB/s vs 8 TB/s"
+PROFILE = os.path.join(ROOT, "profiles", "index_score_ctx1m.md")
+SCORE_SOURCES = ["fp4_sparse_attention_csa2_b200/csrc/index.cu", "fp4_sparse_attention_csa2_b200/csrc/common.cuh"]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], "measured"
+    return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """NVML sampling of SM clock and throttle reasons while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.02):
+        self.samples, self.reasons = [], set()
+        self.period = period
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- our arm
+def build_replicas(csa2, w, n_rep, seed, lens):
+    """One cache filled through csa2_kv_append_quant, then copied into n_rep
+    independent buffers (rotated so that no step finds its inputs in L2)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from harness import cache_geometry
+    n_slots, table, stride = cache_geometry(w, lens, seed)
+    base = csa2.Cache(w.batch, n_slots, w.D, w.D_I, w.row_stride, w.idx_key_dtype, lens, table, w.page_size, stride)
+    q0 = wl.layer_queries(w, 0, seed)["q_idx"]
+    sp = torch.zeros(1, dtype=torch.int32, device="cuda")
+    chunk = 1 << 16
+    for b in range(w.batch):
+        L = int(lens[b])
+        x = wl.latent(w, b, L, seed)
+        keys, _ = wl.index_keys(w, b, L, q0[b, w.T - 1], seed)
+        v = base.view(b)
+        for t0 in range(0, L, chunk):
+            sp.fill_(t0)
+            csa2.kv_append_quant(v, x[t0:t0 + chunk][None].cuda(), sp, keys[t0:t0 + chunk][None].cuda())
+        torch.cuda.synchronize()
+    reps = [base]
+    for _ in range(n_rep - 1):
+        c = csa2.Cache(w.batch, n_slots, w.D, w.D_I, w.row_stride, w.idx_key_dtype, lens, table, w.page_size,
+                       stride)
+        c.rows.copy_(base.rows)
+        c.idx_keys.copy_(base.idx_keys)
+        reps.append(c)
+    torch.cuda.synchronize()
+    return reps
+
+
+class Stack:
+    """Device buffers of one decode step and the C-ABI calls that run it."""
+
+    def __init__(self, csa2, w, layers, ws):
+        self.csa2, self.w, self.ws = csa2, w, ws
+        B, T = w.batch, w.T
+        self.layers = [{k: v.cuda() for k, v in L.items()} for L in layers]
+        self.pool = torch.zeros((B, T, w.pool_k), dtype=torch.int32, device="cuda")
+        self.topk = torch.zeros((B, T, w.top_k), dtype=torch.int32, device="cuda")
+        self.out = [torch.empty((B, T, w.H, w.D), dtype=torch.float32, device="cuda") for _ in w.pattern]
+        self.lse = [torch.empty((B, T, w.H), dtype=torch.float32, device="cuda") for _ in w.pattern]
+        self.modes = [{"F": csa2.FULL, "R": csa2.REINDEX, "U": csa2.REUSE}[m] for m in w.pattern]
+
+    def step(self, cache):
+        c = self.csa2
+        for l, m in enumerate(self.modes):
+            L = self.layers[l]
+            idx = m != c.REUSE
+            c.layer_step(cache, m, L["q"], self.topk, self.out[l], self.ws, self.w.window,
+                         q_idx=L["q_idx"] if idx else None, head_w=L["w"] if idx else None, pool_idx=self.pool,
+                         lse=self.lse[l], pool_k=self.w.pool_k)
+
+
+def kernel_nodes(graph):
+    """Number of kernel nodes in a captured CUDA graph (all of them are libcsa2's)."""
+    try:
+        import cuda.bindings.runtime as rt
+        g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(g, None, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(g, None, n)
+        k = 0
+        for nd in nodes:
+            err, t = rt.cudaGraphNodeGetType(nd)
+            if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                k += 1
+        return k
+    except Exception:
+        return None
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_hash):
+    """Per-launch DRAM bytes of the scoring kernel from the committed ncu
+    summary, if it was taken on the current source of that kernel."""
+    if not os.path.exists(PROFILE):
+        return None
+    vals = {}
+    with open(PROFILE) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("-"):
+                k, v = line.strip()[1:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_hash") != kernel_hash:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_ours(args, world, rank):
+    import fp4_sparse_attention_csa2_b200 as csa2
+    csa2.lib()
+    w = wl.WORKLOADS[args.workload]
+    seed = args.seed + rank
+    lens = wl.seq_lens(w, seed)
+    layers = [wl.layer_queries(w, l, seed) for l in range(len(w.pattern))]
+    reps = build_replicas(csa2, w, args.replicas, seed, lens)
+    n_ws = csa2.workspace_bytes(reps[0], w.T, w.H, w.pool_k, w.top_k, w.window)
+    ws = torch.empty(n_ws, dtype=torch.uint8, device="cuda")
+    csa2.workspace_init(ws)
+    stack = Stack(csa2, w, layers, ws)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            stack.step(reps[i % len(reps)])
+    stream.synchronize()
+    st = csa2.read_device_status(ws, stream)
+    if st != csa2.OK:
+        raise RuntimeError("device status after warm-up: " + csa2.status_string(st))
+
+    graphs = []
+    for r in reps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            stack.step(r)
+        graphs.append(g)
+    launches_per_step = kernel_nodes(graphs[0])
+    for g in graphs:  # graph warm-up
+        g.replay()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(K):
+                graphs[i % len(graphs)].replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    st = csa2.read_device_status(ws, stream)
+    if st != csa2.OK:
+        raise RuntimeError("device status after timing: " + csa2.status_string(st))
+    layer_steps = world * len(w.pattern) * K
+    value = layer_steps / (ms / 1e3)
+
+    # the dominant kernel (Full-layer scoring over every cached position) timed
+    # on its own: a graph of R launches over the rotating replicas
+    R = 3 * len(reps)
+    gs = torch.cuda.CUDAGraph()
+    L0 = stack.layers[0]
+    with torch.cuda.graph(gs, stream=stream, capture_error_mode="relaxed"):
+        for i in range(R):
+            csa2.index_scores(reps[i % len(reps)], L0["q_idx"], L0["w"], ws)
+    gs.replay()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps_k = max(3, min(50, K // 10))
+    with torch.cuda.stream(stream):
+        s0.record(stream)
+        for _ in range(reps_k):
+            gs.replay()
+        s1.record(stream)
+    torch.cuda.synchronize()
+    score_ms = s0.elapsed_time(s1) / (reps_k * R)
+    key_bytes = 64 if w.idx_key_dtype == wl.E4M3 else 256
+    alg_bytes = int(np.sum(lens.astype(np.int64))) * w.T * key_bytes if w.T == 1 else int(np.sum(lens)) * key_bytes
+    hbm, peak_kind = peaks()
+    achieved = alg_bytes / (score_ms / 1e3) / 1e9
+    traffic = profiled_traffic(source_hash(SCORE_SOURCES))
+
+    # end to end through the public API with host buffers: per step, copy the
+    # queries of every layer from pinned host memory, run the stack, read back
+    # every layer's output and log-sum-exp
+    host_in = [{k: v.pin_memory() for k, v in L.items()} for L in layers]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in stack.out]
+    host_lse = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in stack.lse]
+    h2d = sum(v.numel() * v.element_size() for l, L in enumerate(host_in) for k, v in L.items()
+              if k == "q" or w.pattern[l] != "U")
+    d2h = sum(o.numel() * o.element_size() for o in host_out + host_lse)
+    Ke = max(3, min(K, 100))
+    barrier(world)
+    torch.cuda.synchronize()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        x0.record(stream)
+        for i in range(Ke):
+            for l, L in enumerate(host_in):
+                for k, v in L.items():
+                    if k == "q" or w.pattern[l] != "U":
+                        stack.layers[l][k].copy_(v, non_blocking=True)
+            stack.step(reps[i % len(reps)])
+            for l in range(len(w.pattern)):
+                host_out[l].copy_(stack.out[l], non_blocking=True)
+                host_lse[l].copy_(stack.lse[l], non_blocking=True)
+            stream.synchronize()
+        x1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), world)
+    e2e_value = world * len(w.pattern) * Ke / (e2e_ms / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, seed, layers, budget_s=args.cpu_budget)
+
+    if rank == 0:
+        ms_step = ms / K
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "layer-steps/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp32-accum (E2M1/E4M3 storage, bf16 queries)",
+            "data": "synthetic (seeded N(0,1) latents and keys, planted positions; no dataset)",
+            "config": {"workload": w.name, "batch": w.batch, "context": int(lens.max()), "query_tokens": w.T,
+                       "layers": w.pattern, "heads": w.H, "dim": w.D, "indexer": "%dx%d" % (w.H_I, w.D_I),
+                       "pool_k": w.pool_k, "top_k": w.top_k, "window": w.window,
+                       "parallelism": "dp%d (independent sequences per rank)" % world,
+                       "l2": "%d rotating cache replicas, %.0f MB each (> 126 MB L2 together)" % (
+                           len(reps), (reps[0].rows.numel() + reps[0].idx_keys.numel() *
+                                       reps[0].idx_keys.element_size()) / 1e6),
+                       "timing": "CUDA graph per step, CUDA events, max over ranks"},
+            "roofline": {"kernel": "index scoring (Full layer, every cached position)", "bound": "hbm",
+                         "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": round(achieved / hbm, 4), "traffic": traffic,
+                         "algorithmic_bytes_per_launch": alg_bytes, "ms_per_launch": round(score_ms, 5),
+                         "frac_of_8TBps": round(achieved / 8000.0, 4)},
+            "step_bytes_algorithmic": step_bytes(w, lens),
+            "e2e": {"value": round(e2e_value, 1), "unit": "layer-steps/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": Ke,
+                    "path": "python binding -> C ABI csa2_layer_step per layer, pinned host buffers, sync per step"},
+            "gpu_launches": None if launches_per_step is None else launches_per_step * K,
+            "gpu_launches_per_step": launches_per_step,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        line["roofline"]["step_frac_of_8TBps"] = round(line["step_bytes_algorithmic"] / (ms_step / 1e3) / 8e12, 4)
+        print(json.dumps(line))
+        sys.stdout.flush()
+
+
+def step_bytes(w, lens):
+    """Algorithmic bytes of one step: index keys scored, pool keys rescored and
+    FP4 rows attended (upper bound |S| = window + top_k per query)."""
+    key = 64 if w.idx_key_dtype == wl.E4M3 else 256
+    L = lens.astype(np.int64)
+    full = int(np.sum(L)) * key
+    n_q = w.batch * w.T
+    re = n_q * min(w.pool_k, int(L.min())) * key
+    S = n_q * (w.window + w.top_k) * w.row_stride if w.row_stride == w.D // 2 + w.D // 16 else \
+        n_q * (w.window + w.top_k) * (w.D // 2 + w.D // 16)
+    n_f = w.pattern.count("F")
+    n_r = w.pattern.count("R")
+    return n_f * full + n_r * re + len(w.pattern) * S
+
+
+# --------------------------------------------------------------------------- the oracle
+def oracle_step_timer(w, seed, layers, budget_s, max_steps=1000, warmup=0):
+    """Time the CPU oracle on decode steps of the workload for about budget_s
+    seconds (setup -- key encoding, row quantisation -- excluded).  Returns
+    (layer-steps per second, steps run, seconds, sample description)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from harness import attended_positions, build_ref_cache, fill_ref_rows, host_layer
+    lens = wl.seq_lens(w, seed)
+    ref = build_ref_cache(w, seed=seed, rows=False, layers=layers, batches=[0])
+    hl = [host_layer(L) for L in layers]
+    lat = wl.latent(w, 0, int(lens[0]), seed)
+    # rows of every position any layer may attend: quantised once, untimed
+    j = w.T - 1
+    p = int(lens[0]) - w.T + j
+    pool, topk, _ = oracle.index_full(ref, 0, w.T, j, hl[0]["q_idx"][0, j], w.q_idx_dtype, hl[0]["w"][0, j],
+                                      w.pool_k, w.top_k)
+    need = attended_positions(topk, p, w.window)
+    for l, m in enumerate(w.pattern):
+        if m == "R":
+            tk, _ = oracle.index_reindex(ref, 0, w.T, j, hl[l]["q_idx"][0, j], w.q_idx_dtype, hl[l]["w"][0, j],
+                                         pool, w.top_k)
+            need |= attended_positions(tk, p, w.window)
+    fill_ref_rows(ref, w, 0, need, lat)
+    for _ in range(warmup):
+        oracle.run_stack(ref, w.pattern, hl, w.T, w.pool_k, w.top_k, w.window, w.q_idx_dtype, batches=[0],
+                         tokens=[j])
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.run_stack(ref, w.pattern, hl, w.T, w.pool_k, w.top_k, w.window, w.q_idx_dtype, batches=[0],
+                         tokens=[j])
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or steps >= max_steps:
+            break
+    sample = ("sequence 0, query token %d of the %s stack (%s): %d full decode step(s), single-threaded C "
+              "oracle, fp64" % (j, w.name, w.pattern, steps))
+    # one (sequence, token) of the batch; the metric's step covers batch*T of them
+    per_step = el / steps * (w.batch * w.T)
+    return len(w.pattern) / per_step, steps, el, sample
+
+
+def cpu_baseline(w, seed, layers, budget_s):
+    v, steps, el, sample = oracle_step_timer(w, seed, layers, budget_s)
+    return {"value": round(v, 4), "unit": "layer-steps/s", "cores": 1, "kind": "oracle", "sample": sample,
+            "seconds": round(el, 2)}
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: full decode steps of the workload on
+    the host cores until the step count or a fixed time budget is reached."""
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    layers = [wl.layer_queries(w, l, args.seed) for l in range(len(w.pattern))]
+    budget = min(args.ref_budget, 1e9)
+    v, steps, el, sample = oracle_step_timer(w, args.seed, layers, budget_s=budget, max_steps=args.steps,
+                                             warmup=min(args.warmup, 1))
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "layer-steps/s", "n_gpus": world,
+            "steps": steps, "warmup": min(args.warmup, 1), "ms_per_step": round(el / steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, same generator as the CUDA arm)",
+            "config": {"workload": w.name, "context": int(wl.seq_lens(w, args.seed).max()), "layers": w.pattern},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(v, 4)},
+            "e2e": {"value": round(v, 4), "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="ctx1m", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--replicas", type=int, default=3)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds of oracle work in the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, _ = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,225 @@
+"""Python binding of libcsa2 (include/csa2.h): the CSA2 decode-time attention
+step over an FP4 global KV cache on one B200.
+
+The binding only marshals arguments: torch tensors provide device memory and
+streams, every step of the path runs in the CUDA library.  Function names match
+the C ABI without the ``csa2_`` prefix.  There is no CPU fallback: without the
+built library every call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcsa2.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_BOUNDS = range(6)
+FULL, REINDEX, REUSE = 0, 1, 2
+F32, BF16, E4M3 = 0, 1, 2
+
+ABI_FUNCTIONS = (
+    "csa2_workspace_bytes", "csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
+    "csa2_index_reindex", "csa2_sparse_swa_attn", "csa2_layer_step", "csa2_read_device_status",
+    "csa2_status_string",
+)
+
+
+class CSA2Error(RuntimeError):
+    def __init__(self, code, what):
+        super().__init__("%s: %s" % (what, status_string(code)))
+        self.code = code
+
+
+class csa2_cache(ctypes.Structure):
+    _fields_ = [
+        ("kv_rows", ctypes.c_void_p), ("idx_keys", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p), ("batch", ctypes.c_int32), ("max_pages", ctypes.c_int32),
+        ("page_size", ctypes.c_int32), ("dim", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
+        ("row_stride", ctypes.c_int32), ("seq_stride_slots", ctypes.c_int64), ("n_slots", ctypes.c_int64),
+        ("idx_key_dtype", ctypes.c_int),
+    ]
+
+
+class csa2_layer_args(ctypes.Structure):
+    _fields_ = [
+        ("mode", ctypes.c_int), ("q", ctypes.c_void_p), ("q_idx", ctypes.c_void_p), ("q_idx_dtype", ctypes.c_int),
+        ("head_w", ctypes.c_void_p), ("T", ctypes.c_int), ("H", ctypes.c_int), ("H_I", ctypes.c_int),
+        ("pool_k", ctypes.c_int), ("top_k", ctypes.c_int), ("window", ctypes.c_int), ("sm_scale", ctypes.c_float),
+        ("pool_idx", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("lse", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libcsa2.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libcsa2.so is not built; run `python -m fp4_sparse_attention_csa2_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        cp = ctypes.POINTER(csa2_cache)
+        L.csa2_workspace_bytes.restype = sz
+        L.csa2_workspace_bytes.argtypes = [cp, i32, i32, i32, i32, i32]
+        L.csa2_workspace_init.argtypes = [vp, sz, vp]
+        L.csa2_kv_append_quant.argtypes = [cp, vp, vp, i32, vp, i32, vp, vp]
+        L.csa2_index_scores.argtypes = [cp, vp, i32, vp, i32, i32, vp, vp, sz, vp]
+        L.csa2_index_full.argtypes = [cp, vp, i32, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.csa2_index_reindex.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, vp, vp, sz, vp]
+        L.csa2_sparse_swa_attn.argtypes = [cp, vp, i32, i32, vp, i32, i32, ctypes.c_float, vp, vp, vp, sz, vp]
+        L.csa2_layer_step.argtypes = [cp, ctypes.POINTER(csa2_layer_args), vp, sz, vp]
+        L.csa2_read_device_status.argtypes = [vp, vp]
+        L.csa2_status_string.restype = ctypes.c_char_p
+        L.csa2_status_string.argtypes = [i32]
+        for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
+                     "csa2_index_reindex",
+                     "csa2_sparse_swa_attn", "csa2_layer_step", "csa2_read_device_status"):
+            getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(code):
+    return lib().csa2_status_string(int(code)).decode()
+
+
+def _check(code, what):
+    if code != OK:
+        raise CSA2Error(code, what)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Cache:
+    """The global cache of one stack on one device: FP4 rows, index keys, page
+    table and sequence lengths (all device tensors owned by this object)."""
+
+    def __init__(self, batch, n_slots, dim, idx_dim, row_stride, idx_key_dtype, seq_lens, page_table=None,
+                 page_size=64, seq_stride_slots=0, device="cuda"):
+        self.rows = torch.zeros((n_slots, row_stride), dtype=torch.uint8, device=device)
+        kd = torch.uint8 if idx_key_dtype == E4M3 else torch.float32
+        self.idx_keys = torch.zeros((n_slots, idx_dim), dtype=kd, device=device)
+        self.seq_lens = torch.as_tensor(seq_lens, dtype=torch.int32).to(device).contiguous()
+        self.page_table = None if page_table is None else \
+            torch.as_tensor(page_table, dtype=torch.int32).to(device).contiguous()
+        self.batch, self.dim, self.idx_dim, self.idx_key_dtype = batch, dim, idx_dim, idx_key_dtype
+        self.page_size, self.row_stride, self.n_slots = page_size, row_stride, n_slots
+        self.seq_stride_slots = seq_stride_slots
+        self.c = csa2_cache(
+            self.rows.data_ptr(), self.idx_keys.data_ptr(),
+            None if self.page_table is None else self.page_table.data_ptr(), self.seq_lens.data_ptr(), batch,
+            0 if self.page_table is None else self.page_table.shape[1], page_size, dim, idx_dim, row_stride,
+            seq_stride_slots, n_slots, idx_key_dtype)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+    def view(self, b):
+        """A batch-1 cache of sequence b sharing this cache's memory."""
+        v = _View()
+        c = self.c
+        if self.page_table is None:
+            st = self.seq_stride_slots
+            v.c = csa2_cache(c.kv_rows + b * st * self.row_stride,
+                             c.idx_keys + b * st * self.idx_dim * self.idx_keys.element_size(), None,
+                             c.seq_lens + 4 * b, 1, 0, c.page_size, c.dim, c.idx_dim, c.row_stride, st, st,
+                             c.idx_key_dtype)
+        else:
+            v.c = csa2_cache(c.kv_rows, c.idx_keys, c.page_table + 4 * b * c.max_pages, c.seq_lens + 4 * b, 1,
+                             c.max_pages, c.page_size, c.dim, c.idx_dim, c.row_stride, 0, c.n_slots,
+                             c.idx_key_dtype)
+        v.owner = self
+        return v
+
+    @property
+    def capacity(self):
+        return self.page_table.shape[1] * self.page_size if self.page_table is not None else self.seq_stride_slots
+
+
+class _View:
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def workspace_bytes(cache, T, H, pool_k, top_k, window):
+    n = lib().csa2_workspace_bytes(cache.ref, T, H, pool_k, top_k, window)
+    if n == 0:
+        raise CSA2Error(ERR_INVALID_ARG, "workspace_bytes")
+    return n
+
+
+def workspace_init(ws, stream=None):
+    _check(lib().csa2_workspace_init(_p(ws), ws.numel() * ws.element_size(), _stream(stream)), "workspace_init")
+
+
+def kv_append_quant(cache, x, start_pos, idx_new=None, ws=None, stream=None):
+    """x: bf16 [B, n_new, dim]; idx_new: bf16/fp32 [B, n_new, idx_dim]; start_pos: int32 [B] (device)."""
+    dt = F32 if (idx_new is not None and idx_new.dtype == torch.float32) else BF16
+    _check(lib().csa2_kv_append_quant(cache.ref, _p(x), _p(idx_new), dt, _p(start_pos), x.shape[1], _p(ws),
+                                      _stream(stream)), "kv_append_quant")
+
+
+def _qdt(q_idx):
+    return F32 if q_idx.dtype == torch.float32 else BF16
+
+
+def index_scores(cache, q_idx, head_w, ws, scores=None, stream=None):
+    """Full-layer scores of every visible position: into `scores` (fp32
+    [B, T, capacity]) or, when None, into the workspace."""
+    B, T, H_I, _ = q_idx.shape
+    _check(lib().csa2_index_scores(cache.ref, _p(q_idx), _qdt(q_idx), _p(head_w), T, H_I, _p(scores), _p(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)), "index_scores")
+
+
+def index_full(cache, q_idx, head_w, pool_k, top_k, pool_idx, topk_idx, ws, stream=None):
+    """q_idx [B, T, H_I, idx_dim]; head_w fp32 [B, T, H_I]; writes pool_idx [B, T, pool_k], topk_idx [B, T, top_k]."""
+    B, T, H_I, _ = q_idx.shape
+    _check(lib().csa2_index_full(cache.ref, _p(q_idx), _qdt(q_idx), _p(head_w), T, H_I, pool_k, top_k, _p(pool_idx),
+                                 _p(topk_idx), _p(ws), ws.numel() * ws.element_size(), _stream(stream)), "index_full")
+
+
+def index_reindex(cache, q_idx, head_w, pool_idx, top_k, topk_idx, ws, stream=None):
+    B, T, H_I, _ = q_idx.shape
+    _check(lib().csa2_index_reindex(cache.ref, _p(q_idx), _qdt(q_idx), _p(head_w), T, H_I, _p(pool_idx),
+                                    pool_idx.shape[-1], top_k, _p(topk_idx), _p(ws), ws.numel() * ws.element_size(),
+                                    _stream(stream)), "index_reindex")
+
+
+def sparse_swa_attn(cache, q, topk_idx, window, out, lse=None, ws=None, sm_scale=0.0, stream=None):
+    """q bf16 [B, T, H, dim]; topk_idx int32 [B, T, top_k]; out fp32 [B, T, H, dim]; lse fp32 [B, T, H]."""
+    B, T, H, _ = q.shape
+    top_k = topk_idx.shape[-1] if topk_idx is not None else 0
+    _check(lib().csa2_sparse_swa_attn(cache.ref, _p(q), T, H, _p(topk_idx), top_k, window, sm_scale, _p(out), _p(lse),
+                                      _p(ws), ws.numel() * ws.element_size(), _stream(stream)), "sparse_swa_attn")
+
+
+def layer_step(cache, mode, q, topk_idx, out, ws, window, q_idx=None, head_w=None, pool_idx=None, lse=None,
+               pool_k=0, sm_scale=0.0, stream=None):
+    B, T, H, _ = q.shape
+    H_I = q_idx.shape[2] if q_idx is not None else 0
+    a = csa2_layer_args(mode, q.data_ptr(), None if q_idx is None else q_idx.data_ptr(),
+                        _qdt(q_idx) if q_idx is not None else BF16,
+                        None if head_w is None else head_w.data_ptr(), T, H, H_I,
+                        pool_k or (pool_idx.shape[-1] if pool_idx is not None else 0), topk_idx.shape[-1], window,
+                        sm_scale, None if pool_idx is None else pool_idx.data_ptr(), topk_idx.data_ptr(),
+                        out.data_ptr(), None if lse is None else lse.data_ptr())
+    _check(lib().csa2_layer_step(cache.ref, ctypes.byref(a), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "layer_step")
+
+
+def read_device_status(ws, stream=None):
+    """Synchronise and return (then clear) the sticky device status code."""
+    return lib().csa2_read_device_status(_p(ws), _stream(stream))

@@ -1,0 +1,309 @@
+// Host side of the libcsa2 C ABI: argument validation, workspace layout and
+// kernel dispatch.  Every entry point validates on the host, then only
+// enqueues work on the caller's stream.
+#include <cmath>
+#include <cstring>
+
+#include "../../include/csa2.h"
+#include "kernels.h"
+
+using namespace csa2;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxPool = 16384;  // candidate pool bound, tldrocket.com page, paragraph 3
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int64_t capacity(const csa2_cache* c) {
+    return c->page_table ? (int64_t)c->max_pages * c->page_size : c->seq_stride_slots;
+}
+
+csa2_status check_cache(const csa2_cache* c) {
+    if (!c || !c->kv_rows || !c->idx_keys || !c->seq_lens) return CSA2_ERR_INVALID_ARG;
+    if (!aligned16(c->kv_rows) || !aligned16(c->idx_keys) || !aligned4(c->seq_lens)) return CSA2_ERR_INVALID_ARG;
+    if (c->page_table && !aligned4(c->page_table)) return CSA2_ERR_INVALID_ARG;
+    if (c->batch < 1 || c->batch > 65535 || c->n_slots < 1) return CSA2_ERR_INVALID_ARG;
+    if (c->dim < 32 || c->dim % 32) return CSA2_ERR_INVALID_ARG;
+    if (c->dim > 512) return CSA2_ERR_UNSUPPORTED;
+    if (c->idx_dim != 64) return CSA2_ERR_UNSUPPORTED;
+    if (c->row_stride < c->dim / 2 + c->dim / 16 || c->row_stride % 16) return CSA2_ERR_INVALID_ARG;
+    if (c->idx_key_dtype != CSA2_E4M3 && c->idx_key_dtype != CSA2_F32) return CSA2_ERR_INVALID_ARG;
+    if (c->page_table) {
+        if (c->max_pages < 1 || c->page_size < 64 || c->page_size % 64) return CSA2_ERR_INVALID_ARG;
+        if (c->n_slots % c->page_size) return CSA2_ERR_INVALID_ARG;
+    } else {
+        if (c->seq_stride_slots < 64 || c->seq_stride_slots % 64) return CSA2_ERR_INVALID_ARG;
+        if (c->seq_stride_slots * (int64_t)c->batch > c->n_slots) return CSA2_ERR_INVALID_ARG;
+    }
+    if (capacity(c) > (int64_t)1 << 30) return CSA2_ERR_UNSUPPORTED;
+    return CSA2_OK;
+}
+
+DevCache dev_cache(const csa2_cache* c) {
+    DevCache d;
+    d.rows = c->kv_rows;
+    d.keys = c->idx_keys;
+    d.page_table = c->page_table;
+    d.seq_lens = c->seq_lens;
+    d.batch = c->batch;
+    d.max_pages = c->max_pages;
+    d.page_size = c->page_size;
+    d.dim = c->dim;
+    d.idx_dim = c->idx_dim;
+    d.row_stride = c->row_stride;
+    d.seq_stride = c->seq_stride_slots;
+    d.n_slots = c->n_slots;
+    d.cap = capacity(c);
+    d.key_dtype = c->idx_key_dtype == CSA2_E4M3 ? 2 : 0;
+    return d;
+}
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+// Workspace layout (byte offsets, each section 256-byte aligned):
+//   status word | full-layer scores | radix histograms | radix counters |
+//   candidates 1 | candidates 2 | pool scores | attention partials
+struct Layout {
+    size_t status, scores, hist, cnt, cand1, cand2, pscores, part_o, part_ml, total;
+    int64_t nseg, cap, cand_stride;
+    int nchunk;
+};
+
+bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int window, Layout* L) {
+    if (check_cache(c) != CSA2_OK || T < 1 || H < 1 || pool_k < 1 || top_k < 0 || window < 0) return false;
+    L->cap = capacity(c);
+    L->nseg = (int64_t)c->batch * T;
+    L->cand_stride = L->cap > pool_k ? L->cap : pool_k;
+    L->nchunk = (int)((window + top_k + attn_rows_per_chunk() - 1) / attn_rows_per_chunk());
+    if (L->nchunk < 1) L->nchunk = 1;
+    size_t off = 0;
+    L->status = off; off = align_up(off + 16);
+    L->scores = off; off = align_up(off + sizeof(float) * (size_t)(L->nseg * L->cap));
+    L->hist = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 3 * kRadixBins);
+    L->cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 4);
+    L->cand1 = off; off = align_up(off + sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
+    L->cand2 = off; off = align_up(off + sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
+    L->pscores = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * pool_k);
+    L->part_o = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * c->dim);
+    L->part_ml = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * 2);
+    L->total = off;
+    return true;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+SelWork sel_work(void* ws, const Layout& L) {
+    SelWork w;
+    w.hist = at<uint32_t>(ws, L.hist);
+    w.cnt = at<uint32_t>(ws, L.cnt);
+    w.cand1 = at<uint32_t>(ws, L.cand1);
+    w.cand2 = at<uint32_t>(ws, L.cand2);
+    w.cand_stride = L.cand_stride;
+    return w;
+}
+
+csa2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
+
+csa2_status check_ws(const csa2_cache* c, int T, int H, int pool_k, int top_k, int window, void* ws,
+                     size_t ws_bytes, Layout* L) {
+    if (!make_layout(c, T, H, pool_k, top_k, window, L)) return CSA2_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws) || ws_bytes < L->total) return CSA2_ERR_INVALID_ARG;
+    return CSA2_OK;
+}
+
+csa2_status check_index_args(const csa2_cache* c, const void* q_idx, csa2_dtype q_dtype, const float* head_w, int T,
+                             int H_I, int pool_k, int top_k) {
+    csa2_status s = check_cache(c);
+    if (s != CSA2_OK) return s;
+    if (!q_idx || !head_w || !aligned16(q_idx) || !aligned16(head_w)) return CSA2_ERR_INVALID_ARG;
+    if (T < 1 || H_I < 1 || H_I > 64 || T * H_I > 256) return CSA2_ERR_INVALID_ARG;
+    if (top_k < 1 || top_k > pool_k || pool_k > kMaxPool) return CSA2_ERR_INVALID_ARG;
+    if (c->idx_key_dtype == CSA2_E4M3 && q_dtype != CSA2_BF16) return CSA2_ERR_INVALID_ARG;
+    if (c->idx_key_dtype == CSA2_F32 && q_dtype != CSA2_F32) return CSA2_ERR_INVALID_ARG;
+    return CSA2_OK;
+}
+
+csa2_status topk_from_pool(const csa2_cache* c, const Layout& L, void* ws, const float* vals, int64_t vals_stride,
+                           int gather, const int32_t* pool_idx, int pool_k, int top_k, int32_t* topk_idx, int T,
+                           cudaStream_t st) {
+    SelSrc src;
+    src.vals = vals;
+    src.vals_stride = vals_stride;
+    src.ids = pool_idx;
+    src.ids_stride = pool_k;
+    src.gather = gather;
+    src.n = pool_k;
+    src.seq_lens = c->seq_lens;
+    src.T = T;
+    src.cap = L.cap;
+    return cuda_status(launch_select(src, sel_work(ws, L), (int)L.nseg, top_k, topk_idx, top_k, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t csa2_workspace_bytes(const csa2_cache* cache, int T, int H, int pool_k, int top_k, int window) {
+    Layout L;
+    if (!make_layout(cache, T, H, pool_k, top_k, window, &L)) return 0;
+    return L.total;
+}
+
+csa2_status csa2_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws || !aligned16(ws) || ws_bytes < 16) return CSA2_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+csa2_status csa2_kv_append_quant(const csa2_cache* cache, const void* x_bf16, const void* idx_new,
+                                 csa2_dtype idx_new_dtype, const int32_t* start_pos, int n_new, void* ws,
+                                 void* stream) {
+    csa2_status s = check_cache(cache);
+    if (s != CSA2_OK) return s;
+    if (!x_bf16 || !start_pos || !aligned16(x_bf16) || !aligned4(start_pos) || n_new < 0) return CSA2_ERR_INVALID_ARG;
+    if (idx_new && (!aligned16(idx_new) || (idx_new_dtype != CSA2_BF16 && idx_new_dtype != CSA2_F32)))
+        return CSA2_ERR_INVALID_ARG;
+    if (ws && !aligned16(ws)) return CSA2_ERR_INVALID_ARG;
+    if (n_new == 0) return CSA2_OK;
+    return cuda_status(launch_append_quant(dev_cache(cache), x_bf16, idx_new, idx_new_dtype == CSA2_F32 ? 1 : 0,
+                                           start_pos, n_new, static_cast<uint32_t*>(ws),
+                                           static_cast<cudaStream_t>(stream), num_sms()));
+}
+
+csa2_status csa2_index_scores(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
+                              int T, int H_I, float* scores, void* ws, size_t ws_bytes, void* stream) {
+    csa2_status s = check_index_args(cache, q_idx, q_dtype, head_w, T, H_I, 1, 1);
+    if (s != CSA2_OK) return s;
+    if (scores && !aligned16(scores)) return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(cache, T, 1, 1, 1, 0, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    return cuda_status(launch_score_full(dev_cache(cache), q_idx, q_dtype == CSA2_F32, head_w, T, H_I,
+                                         scores ? scores : at<float>(ws, L.scores), at<uint32_t>(ws, L.status),
+                                         static_cast<cudaStream_t>(stream), num_sms()));
+}
+
+csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
+                            int T, int H_I, int pool_k, int top_k, int32_t* pool_idx, int32_t* topk_idx, void* ws,
+                            size_t ws_bytes, void* stream) {
+    csa2_status s = check_index_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_k, top_k);
+    if (s != CSA2_OK) return s;
+    if (!pool_idx || !topk_idx || !aligned16(pool_idx) || !aligned16(topk_idx)) return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(cache, T, 1, pool_k, top_k, 0, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // every visible position scored into the workspace
+    s = csa2_index_scores(cache, q_idx, q_dtype, head_w, T, H_I, nullptr, ws, ws_bytes, stream);
+    if (s != CSA2_OK) return s;
+    float* scores = at<float>(ws, L.scores);
+    // the candidate pool: the pool_k best of all visible scores
+    SelSrc src;
+    src.vals = scores;
+    src.vals_stride = L.cap;
+    src.ids = nullptr;
+    src.ids_stride = 0;
+    src.gather = 0;
+    src.n = L.cap;
+    src.seq_lens = cache->seq_lens;
+    src.T = T;
+    src.cap = L.cap;
+    cudaError_t e = launch_select(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, pool_k, st);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    // this layer's top-k: the top_k best of the same scores, taken from the pool
+    return topk_from_pool(cache, L, ws, scores, L.cap, 1, pool_idx, pool_k, top_k, topk_idx, T, st);
+}
+
+csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
+                               int T, int H_I, const int32_t* pool_idx, int pool_k, int top_k, int32_t* topk_idx,
+                               void* ws, size_t ws_bytes, void* stream) {
+    csa2_status s = check_index_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_k, top_k);
+    if (s != CSA2_OK) return s;
+    if (!pool_idx || !topk_idx || !aligned16(pool_idx) || !aligned16(topk_idx)) return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(cache, T, 1, pool_k, top_k, 0, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevCache d = dev_cache(cache);
+    uint32_t* status = at<uint32_t>(ws, L.status);
+    float* ps = at<float>(ws, L.pscores);
+    cudaError_t e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, pool_idx, pool_k, ps, status, st);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    return topk_from_pool(cache, L, ws, ps, pool_k, 0, pool_idx, pool_k, top_k, topk_idx, T, st);
+}
+
+csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, int T, int H, const int32_t* topk_idx,
+                                 int top_k, int window, float sm_scale, float* out, float* lse, void* ws,
+                                 size_t ws_bytes, void* stream) {
+    csa2_status s = check_cache(cache);
+    if (s != CSA2_OK) return s;
+    if (!q_bf16 || !out || !aligned16(q_bf16) || !aligned16(out) || (lse && !aligned16(lse))) return CSA2_ERR_INVALID_ARG;
+    if (T < 1 || H < 1 || top_k < 0 || window < 0 || window > kMaxPool || top_k > kMaxPool) return CSA2_ERR_INVALID_ARG;
+    if (top_k > 0 && (!topk_idx || !aligned16(topk_idx))) return CSA2_ERR_INVALID_ARG;
+    if (H > 64) return CSA2_ERR_UNSUPPORTED;
+    if (!std::isfinite(sm_scale)) return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
+    AttnWork aw;
+    aw.part_o = at<float>(ws, L.part_o);
+    aw.part_ml = at<float>(ws, L.part_ml);
+    aw.nchunk = L.nchunk;
+    return cuda_status(launch_attention(dev_cache(cache), q_bf16, T, H, topk_idx, top_k, window, sm_scale, out, lse,
+                                        aw, at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream)));
+}
+
+csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* a, void* ws, size_t ws_bytes,
+                            void* stream) {
+    if (!a) return CSA2_ERR_INVALID_ARG;
+    csa2_status s = CSA2_OK;
+    if (a->mode == CSA2_FULL) {
+        s = csa2_index_full(cache, a->q_idx, a->q_idx_dtype, a->head_w, a->T, a->H_I, a->pool_k, a->top_k,
+                            a->pool_idx, a->topk_idx, ws, ws_bytes, stream);
+    } else if (a->mode == CSA2_REINDEX) {
+        s = csa2_index_reindex(cache, a->q_idx, a->q_idx_dtype, a->head_w, a->T, a->H_I, a->pool_idx, a->pool_k,
+                               a->top_k, a->topk_idx, ws, ws_bytes, stream);
+    } else if (a->mode != CSA2_REUSE) {
+        return CSA2_ERR_INVALID_ARG;
+    }
+    if (s != CSA2_OK) return s;
+    return csa2_sparse_swa_attn(cache, a->q, a->T, a->H, a->topk_idx, a->top_k, a->window, a->sm_scale, a->out, a->lse,
+                                ws, ws_bytes, stream);
+}
+
+csa2_status csa2_read_device_status(void* ws, void* stream) {
+    if (!ws || !aligned16(ws)) return CSA2_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(word), st) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (word & kStatusTimeout) return CSA2_ERR_TIMEOUT;
+    if (word & kStatusBounds) return CSA2_ERR_DEVICE_BOUNDS;
+    return CSA2_OK;
+}
+
+const char* csa2_status_string(csa2_status s) {
+    switch (s) {
+        case CSA2_OK: return "CSA2_OK";
+        case CSA2_ERR_INVALID_ARG: return "CSA2_ERR_INVALID_ARG";
+        case CSA2_ERR_UNSUPPORTED: return "CSA2_ERR_UNSUPPORTED";
+        case CSA2_ERR_CUDA: return "CSA2_ERR_CUDA";
+        case CSA2_ERR_TIMEOUT: return "CSA2_ERR_TIMEOUT";
+        case CSA2_ERR_DEVICE_BOUNDS: return "CSA2_ERR_DEVICE_BOUNDS";
+    }
+    return "CSA2_UNKNOWN_STATUS";
+}
+
+}  // extern "C"

@@ -1,0 +1,204 @@
+// Sparse + sliding-window attention over the FP4 global cache.
+//
+// Method: hackernews.kjhq.dev post 49735410, key point 2 (local sliding windows
+// plus global sparse retrieval, layers sharing one main KV and its Top-K
+// indices); tldrocket.com, "DeepSeek AI Released DeepSeek-V4.1-Flash with 1M
+// Context, FP4 KV Cache, and Cross-Layer Attention Reuse", paragraphs 2-4
+// (128-token window in every layer; E2M1 values with one E4M3 scale per 16
+// channels).
+//
+// Each (sequence, query token) owns a virtual list of W + k entries: the W
+// window positions p, p-1, ..., p-W+1 followed by its k top-k positions; a
+// top-k position that lies in the window, is -1 or is beyond p is masked, so
+// the attended set is window ∪ top-k without double counting.  The list is cut
+// into chunks of kRows entries; one CTA gathers the FP4 rows of its chunk,
+// dequantises them in shared memory and writes a partial (max, sum, unnormalised
+// output) per head.  A second kernel merges the partials (split softmax).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa2 {
+
+namespace {
+
+constexpr int kRows = 32;      // entries per CTA
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ int32_t entry_position(const int32_t* topk, int top_k, int window, int64_t p, int64_t L,
+                                                  int v, uint32_t* status) {
+    if (v < window) {
+        const int64_t t = p - v;
+        return t >= 0 ? (int32_t)t : -1;
+    }
+    const int32_t t = __ldg(topk + (v - window));
+    if (t < -1 || t >= L) { flag(status, kStatusBounds); return -1; }
+    if (t < 0 || t > p || t > p - window) return -1;   // padding, future, or already in the window
+    return t;
+}
+
+// grid (nchunk, batch*T); dynamic smem: H*(D+4) + kRows*(D+4) + H*kRows floats + kRows ints
+__global__ void __launch_bounds__(kThreads)
+k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, const int32_t* __restrict__ topk,
+               int top_k, int window, float scale, float* __restrict__ part_o, float* __restrict__ part_ml,
+               int nchunk, uint32_t* status) {
+    extern __shared__ float smem[];
+    const int D = c.dim;
+    const int DP = D + 4;
+    float* qs = smem;                      // [H][DP]
+    float* vs = qs + H * DP;               // [kRows][DP]
+    float* ps = vs + kRows * DP;           // [H][kRows]
+    int* pos = reinterpret_cast<int*>(ps + H * kRows);
+    const int seg = blockIdx.y, chunk = blockIdx.x;
+    const int b = seg / T, j = seg % T;
+    const int64_t L = seq_len(c, b, status);
+    const int64_t p = L - T + j;
+
+    if (threadIdx.x < kRows) {
+        const int v = chunk * kRows + threadIdx.x;
+        int32_t t = -1;
+        if (p >= 0 && v < window + top_k)
+            t = entry_position(topk + (int64_t)seg * top_k, top_k, window, p, L, v, status);
+        pos[threadIdx.x] = t;
+    }
+    const __nv_bfloat16* qg = q + (int64_t)seg * H * D;
+    for (int i = threadIdx.x; i < H * D; i += kThreads) qs[(i / D) * DP + i % D] = __bfloat162float(qg[i]);
+    __syncthreads();
+
+    // gather + dequantise: one thread per 16-channel block of one row
+    const int nblk = D >> 4;
+    for (int w = threadIdx.x; w < kRows * nblk; w += kThreads) {
+        const int r = w / nblk, blk = w % nblk;
+        float* dst = vs + r * DP + blk * 16;
+        const int32_t t = pos[r];
+        int64_t slot = t >= 0 ? slot_of(c, b, t) : -1;
+        if (t >= 0 && slot < 0) flag(status, kStatusBounds);
+        if (slot < 0) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) dst[k] = 0.0f;
+            continue;
+        }
+        const uint8_t* row = c.rows + slot * c.row_stride;
+        const uint2 codes = *reinterpret_cast<const uint2*>(row + blk * 8);
+        const float s = e4m3_to_float(row[(D >> 1) + blk]);
+        const uint32_t cw[2] = {codes.x, codes.y};
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 f = __half22float2(e2m1x2_to_half2((uint8_t)(cw[h] >> (8 * k))));
+                dst[h * 8 + 2 * k] = f.x * s;
+                dst[h * 8 + 2 * k + 1] = f.y * s;
+            }
+    }
+    __syncthreads();
+
+    // logits z[h][r] = scale * q_h . v_r ; thread (h, rg) handles rows rg, rg+4, ...
+    for (int w = threadIdx.x; w < H * 4; w += kThreads) {
+        const int h = w >> 2, rg = w & 3;
+        float acc[kRows / 4];
+#pragma unroll
+        for (int i = 0; i < kRows / 4; ++i) acc[i] = 0.0f;
+        const float* qh = qs + h * DP;
+        for (int d = 0; d < D; d += 4) {
+            const float4 qv = *reinterpret_cast<const float4*>(qh + d);
+#pragma unroll
+            for (int i = 0; i < kRows / 4; ++i) {
+                const float4 vv = *reinterpret_cast<const float4*>(vs + (rg + 4 * i) * DP + d);
+                acc[i] = fmaf(qv.x, vv.x, fmaf(qv.y, vv.y, fmaf(qv.z, vv.z, fmaf(qv.w, vv.w, acc[i]))));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kRows / 4; ++i) {
+            const int r = rg + 4 * i;
+            ps[h * kRows + r] = pos[r] >= 0 ? acc[i] * scale : -INFINITY;
+        }
+    }
+    __syncthreads();
+
+    // per-head partial softmax statistics over this chunk
+    float* ml = part_ml + ((int64_t)seg * nchunk + chunk) * H * 2;
+    for (int h = threadIdx.x; h < H; h += kThreads) {
+        float m = -INFINITY;
+        for (int r = 0; r < kRows; ++r) m = fmaxf(m, ps[h * kRows + r]);
+        float l = 0.0f;
+        for (int r = 0; r < kRows; ++r) {
+            const float e = m == -INFINITY ? 0.0f : __expf(ps[h * kRows + r] - m);
+            ps[h * kRows + r] = e;
+            l += e;
+        }
+        ml[2 * h] = m;
+        ml[2 * h + 1] = l;
+    }
+    __syncthreads();
+
+    // unnormalised partial output O[h][d] = sum_r e[h][r] v_r[d]
+    float* po = part_o + ((int64_t)seg * nchunk + chunk) * H * D;
+    const int D4 = D >> 2;
+    for (int w = threadIdx.x; w < H * D4; w += kThreads) {
+        const int h = w / D4, d = (w % D4) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < kRows; ++r) {
+            const float e = ps[h * kRows + r];
+            const float4 vv = *reinterpret_cast<const float4*>(vs + r * DP + d);
+            acc.x = fmaf(e, vv.x, acc.x);
+            acc.y = fmaf(e, vv.y, acc.y);
+            acc.z = fmaf(e, vv.z, acc.z);
+            acc.w = fmaf(e, vv.w, acc.w);
+        }
+        *reinterpret_cast<float4*>(po + (int64_t)h * D + d) = acc;
+    }
+}
+
+// grid (batch*T, H); block 128: merge the chunk partials of one head.
+__global__ void __launch_bounds__(128)
+k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk,
+               float* __restrict__ out, float* __restrict__ lse) {
+    const int seg = blockIdx.x, h = blockIdx.y;
+    __shared__ float s_w[1024];
+    __shared__ float s_stat[2];
+    if (threadIdx.x == 0) {
+        float m = -INFINITY;
+        for (int ch = 0; ch < nchunk; ++ch) m = fmaxf(m, part_ml[(((int64_t)seg * nchunk + ch) * H + h) * 2]);
+        float l = 0.0f;
+        for (int ch = 0; ch < nchunk; ++ch) {
+            const float* ml = part_ml + (((int64_t)seg * nchunk + ch) * H + h) * 2;
+            const float w = (m == -INFINITY || ml[0] == -INFINITY) ? 0.0f : __expf(ml[0] - m);
+            s_w[ch] = w;
+            l += w * ml[1];
+        }
+        s_stat[0] = m;
+        s_stat[1] = l;
+    }
+    __syncthreads();
+    const float l = s_stat[1];
+    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float acc = 0.0f;
+        for (int ch = 0; ch < nchunk; ++ch)
+            if (s_w[ch] != 0.0f) acc = fmaf(s_w[ch], part_o[(((int64_t)seg * nchunk + ch) * H + h) * D + d], acc);
+        out[((int64_t)seg * H + h) * D + d] = acc * inv;
+    }
+    if (lse && threadIdx.x == 0) lse[(int64_t)seg * H + h] = l > 0.0f ? s_stat[0] + logf(l) : -INFINITY;
+}
+
+}  // namespace
+
+int attn_rows_per_chunk() { return kRows; }
+
+cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
+                             int window, float sm_scale, float* out, float* lse, const AttnWork& aw,
+                             uint32_t* status, cudaStream_t st) {
+    const int D = c.dim;
+    const size_t smem = sizeof(float) * ((size_t)H * (D + 4) + (size_t)kRows * (D + 4) + (size_t)H * kRows) +
+                        sizeof(int) * kRows;
+    cudaError_t e = cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)aw.nchunk, (unsigned)(c.batch * T));
+    k_attn_partial<<<grid, kThreads, smem, st>>>(c, static_cast<const __nv_bfloat16*>(q), T, H, topk, top_k, window,
+                                                 sm_scale, aw.part_o, aw.part_ml, aw.nchunk, status);
+    k_attn_combine<<<dim3((unsigned)(c.batch * T), (unsigned)H), 128, 0, st>>>(D, H, aw.part_o, aw.part_ml,
+                                                                             aw.nchunk, out, lse);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,103 @@
+// Device-side helpers shared by the libcsa2 kernels (sm_100a).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace csa2 {
+
+// Sticky status bits ORed into the workspace status word by kernels.
+constexpr uint32_t kStatusBounds = 1u;
+constexpr uint32_t kStatusTimeout = 2u;
+
+// A by-value copy of csa2_cache plus the derived per-sequence capacity.
+struct DevCache {
+    uint8_t* rows;
+    void* keys;
+    const int32_t* page_table;
+    const int32_t* seq_lens;
+    int32_t batch, max_pages, page_size, dim, idx_dim, row_stride;
+    int64_t seq_stride, n_slots, cap;
+    int32_t key_dtype;  // 0 fp32, 2 e4m3
+};
+
+__device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
+    if (status) atomicOr(status, bit);
+}
+
+// Slot of position t of sequence b, or -1 when the page table points outside
+// the cache.  The caller guarantees 0 <= t < cap.
+__device__ __forceinline__ int64_t slot_of(const DevCache& c, int b, int64_t t) {
+    if (c.page_table) {
+        int64_t pg = t / c.page_size;
+        int32_t phys = __ldg(c.page_table + (int64_t)b * c.max_pages + pg);
+        int64_t s = (int64_t)phys * c.page_size + (t - pg * c.page_size);
+        return (phys < 0 || s >= c.n_slots) ? -1 : s;
+    }
+    return (int64_t)b * c.seq_stride + t;
+}
+
+// Valid length of sequence b clamped to the capacity (flags a longer one).
+__device__ __forceinline__ int64_t seq_len(const DevCache& c, int b, uint32_t* status) {
+    int64_t L = __ldg(c.seq_lens + b);
+    if (L > c.cap || L < 0) {
+        flag(status, kStatusBounds);
+        L = L < 0 ? 0 : c.cap;
+    }
+    return L;
+}
+
+// ---------------------------------------------------------------- conversions
+// E4M3 round-to-nearest-even, saturating: `hi` lands in the upper byte.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float hi, float lo) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Four E2M1 pairs (round-to-nearest-even, saturating) packed into 32 bits:
+// byte k holds x[2k] in its low nibble and x[2k+1] in its high nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float* x) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
+    return r;
+}
+
+// Two E4M3 bytes (low byte first) -> two halves; exact.
+__device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t v) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    __half2 h;
+    memcpy(&h, &r, 4);
+    return h;
+}
+
+__device__ __forceinline__ float e4m3_to_float(uint8_t v) {
+    return __low2float(e4m3x2_to_half2((uint16_t)v));
+}
+
+// Two E2M1 codes (one byte, low nibble first) -> two halves; exact.
+__device__ __forceinline__ __half2 e2m1x2_to_half2(uint8_t v) {
+    uint32_t r;
+    uint16_t in = v;
+    asm("{\n\t.reg .b8 b, u;\n\tmov.b16 {b, u}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(r) : "h"(in));
+    __half2 h;
+    memcpy(&h, &r, 4);
+    return h;
+}
+
+// Monotone map of fp32 onto uint32 (larger float -> larger key); -0 == +0.
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+    uint32_t u = __float_as_uint(f == 0.0f ? 0.0f : f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+}  // namespace csa2

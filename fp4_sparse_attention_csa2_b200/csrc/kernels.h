@@ -1,0 +1,65 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace csa2 {
+
+// Radix-select state of one workspace (see topk.cu).  Counts and histograms
+// are per segment (one segment = one (sequence, query token)).
+constexpr int kRadixBins = 2048;
+struct SelWork {
+    uint32_t* hist;   // [nseg][3][kRadixBins]
+    uint32_t* cnt;    // [nseg][4]: outputs, level-1 candidates, level-2 candidates, ties
+    uint32_t* cand1;  // [nseg][cand_stride]
+    uint32_t* cand2;  // [nseg][cand_stride]
+    int64_t cand_stride;
+};
+
+// Where the elements of one selection come from.
+//   ids == nullptr: element i is position i, valid for i <= p_j (Full scores).
+//   ids != nullptr: element i is position ids[seg*ids_stride + i], valid when
+//                   0 <= id <= p_j; its value is vals[seg*vals_stride + (gather ? id : i)].
+struct SelSrc {
+    const float* vals;
+    int64_t vals_stride;
+    const int32_t* ids;
+    int64_t ids_stride;
+    int gather;
+    int64_t n;                // elements per segment (upper bound)
+    const int32_t* seq_lens;  // for ids == nullptr
+    int T;
+    int64_t cap;
+};
+
+cudaError_t launch_append_quant(const DevCache& c, const void* x, const void* idx_new, int idx_new_f32,
+                                const int32_t* start_pos, int n_new, uint32_t* status, cudaStream_t st,
+                                int num_sms);
+
+// Full scoring: scores[(b*T + j) * cap + t] for t <= p_j.
+cudaError_t launch_score_full(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
+                              float* scores, uint32_t* status, cudaStream_t st, int num_sms);
+
+// Pool rescoring: scores[seg * pool_k + i] for pool entry i of segment seg.
+cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
+                              const int32_t* pool, int pool_k, float* scores, uint32_t* status, cudaStream_t st);
+
+// Top-n selection per segment into out[seg * out_stride + 0..n_out) (-1 padded).
+cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_out, int32_t* out,
+                          int64_t out_stride, cudaStream_t st);
+
+// Attention partials + combine.
+struct AttnWork {
+    float* part_o;    // [nseg][nchunk][H][D]
+    float* part_ml;   // [nseg][nchunk][H][2]
+    int nchunk;
+};
+int attn_rows_per_chunk();
+cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
+                             int window, float sm_scale, float* out, float* lse, const AttnWork& aw,
+                             uint32_t* status, cudaStream_t st);
+
+}  // namespace csa2

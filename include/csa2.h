@@ -1,0 +1,244 @@
+/*
+ * csa2.h -- C ABI of libcsa2: the CSA2 decode-time attention step over an FP4
+ * global KV cache, on one NVIDIA B200 (sm_100a).
+ *
+ * The method is described on these pages ("DeepSeek-V4.1-Flash: Pushing the
+ * Limits of KV Cache Compression"):
+ *   [TLDR]   tldrocket.com, "DeepSeek AI Released DeepSeek-V4.1-Flash with 1M
+ *            Context, FP4 KV Cache, and Cross-Layer Attention Reuse":
+ *            paragraph 2 (sliding window of 128 tokens in every layer),
+ *            paragraph 3 (Full / Reindex / Reuse layer roles; a Full layer
+ *            builds a candidate pool of up to 16,384 positions),
+ *            paragraph 4 (main KV as E2M1 values with one E4M3 scale per 16
+ *            channels, NVFP4 without the global scale).
+ *   [HN]     hackernews.kjhq.dev post 49735410, "key points" 2-3 (layers share
+ *            the main KV and Top-K indices; the hierarchical sparse indexer).
+ *   [FANOUT] fanout.sh daily lesson, "What you will learn" item 2 (modes share
+ *            global KV and sparse selections; queries and window stay
+ *            layer-local).
+ *
+ * Conventions for every call:
+ *  - All pointers inside csa2_cache and all tensor arguments are DEVICE
+ *    pointers owned by the caller; the library allocates and frees nothing.
+ *  - Every call only validates its arguments on the host and enqueues work on
+ *    `stream` (a cudaStream_t, NULL = legacy default stream); it never
+ *    synchronises, except csa2_read_device_status.
+ *  - Host-side validation failures return CSA2_ERR_INVALID_ARG (or
+ *    CSA2_ERR_UNSUPPORTED for legal but unimplemented shapes) before anything
+ *    is launched.  A failed launch returns CSA2_ERR_CUDA.
+ *  - Problems only the device can see (an index or page id out of range, a
+ *    sequence longer than the cache, a bounded wait that ran out) never trap:
+ *    the kernel skips the bad element and ORs a bit into a sticky status word
+ *    in the workspace, read back with csa2_read_device_status.
+ *  - The library keeps no mutable global state: calls on different streams
+ *    with different workspaces may run concurrently.
+ *  - Tensors are dense and row-major in the shapes given.  Pointers must be
+ *    16-byte aligned, except seq_lens, page_table and start_pos (4-byte):
+ *    a cache view of one sequence (page_table + b * max_pages, seq_lens + b)
+ *    is a valid cache.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of the shared library; everything else in it is hidden. */
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+typedef enum {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or bound */
+    CSA2_ERR_UNSUPPORTED = 2,   /* legal shape this build does not implement */
+    CSA2_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    CSA2_ERR_TIMEOUT = 4,       /* device: a bounded wait gave up */
+    CSA2_ERR_DEVICE_BOUNDS = 5  /* device: index / page / length out of range */
+} csa2_status;
+
+/* Layer roles, [TLDR] paragraph 3. */
+typedef enum { CSA2_FULL = 0, CSA2_REINDEX = 1, CSA2_REUSE = 2 } csa2_mode;
+
+typedef enum { CSA2_F32 = 0, CSA2_BF16 = 1, CSA2_E4M3 = 2 } csa2_dtype;
+
+/*
+ * The global cache shared by every layer of a stack ([HN] key point 2):
+ * one FP4 latent row per position (key and value for all heads) and one
+ * index key per position.
+ *
+ *   kv_rows    [n_slots][row_stride] bytes.  A row holds dim/2 code bytes (two
+ *              E2M1 codes per byte, channel 2j in the low nibble of byte j)
+ *              followed by dim/16 E4M3 scale bytes (one per 16 channels, no
+ *              global scale: [TLDR] paragraph 4).  Padding bytes are unused.
+ *   idx_keys   [n_slots][idx_dim] of idx_key_dtype (CSA2_E4M3 or CSA2_F32).
+ *   page_table [batch][max_pages] int32 physical page ids, or NULL for the
+ *              contiguous layout.  Position t of sequence b lives in slot
+ *              page_table[b][t / page_size] * page_size + t % page_size
+ *              (paged) or b * seq_stride_slots + t (contiguous).
+ *   seq_lens   [batch] int32, the number of valid positions L_b of each
+ *              sequence.  Read on the device, never written.
+ *
+ * Limits: dim % 32 == 0 and 32 <= dim <= 512; idx_dim == 64; row_stride >=
+ * dim/2 + dim/16 and a multiple of 16; page_size a multiple of 64 (paged);
+ * seq_stride_slots a multiple of 64 (contiguous).  The capacity of one
+ * sequence is max_pages * page_size (paged) or seq_stride_slots.
+ */
+typedef struct {
+    uint8_t* kv_rows;
+    void* idx_keys;
+    const int32_t* page_table;
+    const int32_t* seq_lens;
+    int32_t batch;
+    int32_t max_pages;
+    int32_t page_size;
+    int32_t dim;
+    int32_t idx_dim;
+    int32_t row_stride;
+    int64_t seq_stride_slots;
+    int64_t n_slots;
+    csa2_dtype idx_key_dtype;
+} csa2_cache;
+
+/*
+ * Bytes of device workspace the index and attention calls need for this cache
+ * with T query tokens per sequence, H attention heads, a pool of pool_k and a
+ * top-k of top_k positions, and a window of `window` positions.  Returns 0 on
+ * invalid arguments.  One workspace serves every call of a stack on one
+ * stream; it must be cleared once with csa2_workspace_init before first use.
+ */
+CSA2_API size_t csa2_workspace_bytes(const csa2_cache* cache, int T, int H, int pool_k, int top_k, int window);
+
+/* Zero the workspace (including the sticky device status word) on `stream`. */
+CSA2_API csa2_status csa2_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Quantise-on-append ([TLDR] paragraph 4).  For every sequence b and i <
+ * n_new, the bf16 latent x_bf16[b][i][0..dim) is written as the FP4 row of
+ * position start_pos[b] + i:
+ *     amax = max |x| over each 16-channel block,
+ *     s    = E4M3 round-to-nearest-even, saturating (fp32 amax / 6),
+ *     c_j  = E2M1 round-to-nearest-even, saturating (fp32 x_j / s), sign kept,
+ *            all codes 0 when s is 0.
+ * The divisions are IEEE binary32 divisions.  idx_new (nullable,
+ * [batch][n_new][idx_dim] of idx_new_dtype CSA2_BF16 or CSA2_F32) is stored as
+ * the position's index key: E4M3 (round-to-nearest-even, saturating) for an
+ * E4M3 cache, the fp32 value for an F32 cache.  start_pos is a device int32
+ * [batch] array; the call does not change seq_lens.  Inputs must be finite.
+ * ws (nullable) is a workspace whose sticky status word records positions
+ * outside the cache (those rows are skipped); with ws == NULL they are skipped
+ * silently.
+ */
+CSA2_API csa2_status csa2_kv_append_quant(const csa2_cache* cache, const void* x_bf16, const void* idx_new,
+                                 csa2_dtype idx_new_dtype, const int32_t* start_pos, int n_new,
+                                 void* ws, void* stream);
+
+/*
+ * Full-layer indexing ([TLDR] paragraph 3; [HN] key point 3).  Query token j
+ * of sequence b sits at p = seq_lens[b] - T + j and sees positions t <= p.
+ * Every visible position gets the score
+ *     s_t = sum_h head_w[b][j][h] * max(0, q_idx[b][j][h] . k_t)
+ * (fp32 accumulation), and
+ *     pool_idx[b][j][0..pool_k)  <- the min(pool_k, p+1) positions with the
+ *                                   largest s_t (the candidate pool),
+ *     topk_idx[b][j][0..top_k)   <- the min(top_k, p+1) largest of the same
+ *                                   scores (a subset of the pool),
+ * each as a set in unspecified order followed by -1 padding.  Ties at the
+ * cutoff are broken arbitrarily.  q_idx is [batch][T][H_I][idx_dim] of q_dtype
+ * (CSA2_BF16 with an E4M3 cache, CSA2_F32 with an F32 cache); head_w is fp32
+ * [batch][T][H_I].  Requires 1 <= top_k <= pool_k <= 16384, 1 <= H_I <= 64,
+ * T*H_I <= 256.
+ */
+CSA2_API csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
+                            const float* head_w, int T, int H_I, int pool_k, int top_k,
+                            int32_t* pool_idx, int32_t* topk_idx, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/*
+ * The scoring half of csa2_index_full on its own: s_t for every visible
+ * position t <= p of every (b, j), written to scores[(b*T + j)*capacity + t]
+ * (fp32; entries beyond p are left untouched).  With scores == NULL the
+ * scores go to the workspace, where csa2_index_full keeps them.  Same
+ * argument rules as csa2_index_full.
+ */
+CSA2_API csa2_status csa2_index_scores(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
+                                       const float* head_w, int T, int H_I, float* scores, void* ws,
+                                       size_t ws_bytes, void* stream);
+
+/*
+ * Reindex-layer indexing ([TLDR] paragraph 3, "rescore a shared candidate
+ * set").  For each (b, j), the valid entries of pool_idx[b][j][0..pool_k)
+ * (those >= 0; usually the pool of the last Full layer) are rescored with this
+ * layer's q_idx / head_w exactly as csa2_index_full scores, and topk_idx[b][j]
+ * receives the min(top_k, |pool|) best as a set followed by -1 padding.
+ * Pool entries > p or >= seq_lens[b] set CSA2_ERR_DEVICE_BOUNDS.
+ */
+CSA2_API csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
+                               const float* head_w, int T, int H_I, const int32_t* pool_idx,
+                               int pool_k, int top_k, int32_t* topk_idx, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/*
+ * Sparse + sliding-window attention ([HN] key point 2; [TLDR] paragraphs 2-3).
+ * For query token j of sequence b at p = seq_lens[b] - T + j, the attended set
+ * is S = window ∪ topk without double counting, with window = [max(0, p -
+ * window + 1), p]; topk entries that are -1 or > p are not attended.  With
+ * v_t the dequantised row of position t (value(code) * value(scale), used as
+ * both key and value for every head):
+ *     z_t   = sm_scale * q[b][j][h] . v_t          (sm_scale <= 0: 1/sqrt(dim))
+ *     out   = sum_{t in S} softmax(z)_t v_t        fp32 [batch][T][H][dim]
+ *     lse   = log sum_{t in S} exp(z_t)            fp32 [batch][T][H], nullable
+ * q is bf16 [batch][T][H][dim].  An empty S gives out = 0, lse = -inf.
+ * topk entries < -1 or >= seq_lens[b] set CSA2_ERR_DEVICE_BOUNDS.
+ */
+CSA2_API csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, int T, int H,
+                                 const int32_t* topk_idx, int top_k, int window, float sm_scale,
+                                 float* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * One layer of a CSA2 stack ([TLDR] paragraph 3; [FANOUT] item 2):
+ *   CSA2_FULL    csa2_index_full (writes pool_idx and topk_idx), then attention
+ *   CSA2_REINDEX csa2_index_reindex (reads pool_idx, writes topk_idx), then
+ *                attention
+ *   CSA2_REUSE   attention only, with topk_idx as given; no index buffer is
+ *                read or written other than topk_idx, which is only read.
+ */
+typedef struct {
+    csa2_mode mode;
+    const void* q;           /* bf16 [batch][T][H][dim] */
+    const void* q_idx;       /* [batch][T][H_I][idx_dim]; FULL / REINDEX only */
+    csa2_dtype q_idx_dtype;
+    const float* head_w;     /* [batch][T][H_I]; FULL / REINDEX only */
+    int T, H, H_I, pool_k, top_k, window;
+    float sm_scale;
+    int32_t* pool_idx;       /* [batch][T][pool_k] */
+    int32_t* topk_idx;       /* [batch][T][top_k] */
+    float* out;              /* [batch][T][H][dim] */
+    float* lse;              /* [batch][T][H] or NULL */
+} csa2_layer_args;
+
+CSA2_API csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* args, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then return the sticky device status recorded in the
+ * workspace (CSA2_OK, CSA2_ERR_DEVICE_BOUNDS or CSA2_ERR_TIMEOUT; the first
+ * error class found in that order of severity: TIMEOUT, then BOUNDS) and clear
+ * it.  Returns CSA2_ERR_CUDA if the synchronisation or copy fails.
+ */
+CSA2_API csa2_status csa2_read_device_status(void* ws, void* stream);
+
+/* A static, human-readable name for a status code. */
+CSA2_API const char* csa2_status_string(csa2_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA2_H */

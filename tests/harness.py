@@ -15,15 +15,16 @@ def cache_geometry(w, lens, seed=0):
     return w.batch * cap, None, cap
 
 
-def build_ref_cache(w, seed=0, lens=None, rows=True, layers=None):
-    """Oracle host cache with every position of every sequence written
-    (latent rows quantised by the oracle, index keys encoded by the oracle)."""
+def build_ref_cache(w, seed=0, lens=None, rows=True, layers=None, batches=None):
+    """Oracle host cache with every position of the sequences in `batches`
+    (default: all) written: index keys encoded by the oracle and, with rows=True,
+    latent rows quantised by the oracle."""
     lens = wl.seq_lens(w, seed) if lens is None else np.asarray(lens, dtype=np.int32)
     n_slots, table, stride = cache_geometry(w, lens, seed)
     cache = oracle.RefCache(w.batch, n_slots, w.D, w.D_I, w.row_stride, w.idx_key_dtype, lens,
                             page_table=table, page_size=w.page_size, seq_stride_slots=stride)
     q0 = (layers[0] if layers else wl.layer_queries(w, 0, seed))["q_idx"]
-    for b in range(w.batch):
+    for b in (range(w.batch) if batches is None else batches):
         L = int(lens[b])
         keys, _ = wl.index_keys(w, b, L, q0[b, w.T - 1], seed)
         x = wl.bf16_bits(wl.latent(w, b, L, seed)) if rows else None
@@ -56,3 +57,19 @@ def band_set_check(got, want_sorted, scores_by_pos, n_valid, rel=1e-5):
 def host_layer(layer):
     """A layer's query tensors as the oracle takes them (bf16 -> uint16 bits)."""
     return {k: wl.host_array(v) for k, v in layer.items()}
+
+
+def fill_ref_rows(ref, w, b, positions, latent_b):
+    """Quantise (with the oracle) the latent rows of the given positions of
+    sequence b into the oracle cache; latent_b is the bf16 [L_b, D] input."""
+    pos = np.unique(np.asarray([int(t) for t in positions if t >= 0], dtype=np.int64))
+    bits = wl.bf16_bits(latent_b)
+    for t in pos:
+        ref.write(b, int(t), bits[t:t + 1])
+
+
+def attended_positions(topk, p, window):
+    """Positions of window ∪ top-k for a query at p (the oracle's reading)."""
+    s = set(range(max(0, p - window + 1), p + 1))
+    s.update(int(t) for t in topk if 0 <= t <= p)
+    return s

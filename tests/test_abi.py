@@ -1,0 +1,88 @@
+"""The C-ABI library loads on a host without a GPU, exports every function
+include/csa2.h declares, and rejects bad arguments on the host before it
+launches anything (these calls never reach the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp4_sparse_attention_csa2_b200 as csa2
+from fp4_sparse_attention_csa2_b200 import build as _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "csa2.h")).read()
+    return re.findall(r"CSA2_API\s+[\w\s\*]+?\b(csa2_\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return csa2.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    assert set(names) == set(csa2.ABI_FUNCTIONS)
+    handle = ctypes.CDLL(csa2.LIB_PATH)
+    for n in names:
+        assert hasattr(handle, n), n
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["CSA2_OK", "CSA2_ERR_INVALID_ARG", "CSA2_ERR_UNSUPPORTED", "CSA2_ERR_CUDA",
+                                 "CSA2_ERR_TIMEOUT", "CSA2_ERR_DEVICE_BOUNDS"]):
+        assert csa2.status_string(code) == name
+
+
+def fake_cache(**kw):
+    d = dict(kv_rows=0x10000, idx_keys=0x20000, page_table=None, seq_lens=0x30000, batch=1, max_pages=0,
+             page_size=64, dim=512, idx_dim=64, row_stride=288, seq_stride_slots=1 << 20, n_slots=1 << 20,
+             idx_key_dtype=csa2.E4M3)
+    d.update(kw)
+    return csa2.csa2_cache(**d)
+
+
+def test_workspace_bytes_layout(lib):
+    c = fake_cache()
+    n = lib.csa2_workspace_bytes(ctypes.byref(c), 1, 64, 16384, 2048, 128)
+    # scores (4 MiB) + two candidate lists (8 MiB) + partials of 68 chunks x 64 x 512 fp32
+    assert n >= 4 * (1 << 20) * 3 + 68 * 64 * 512 * 4
+    assert n % 256 == 0
+    assert lib.csa2_workspace_bytes(ctypes.byref(fake_cache(dim=100)), 1, 64, 16384, 2048, 128) == 0
+    assert lib.csa2_workspace_bytes(ctypes.byref(fake_cache(row_stride=280)), 1, 64, 16384, 2048, 128) == 0
+    assert lib.csa2_workspace_bytes(None, 1, 64, 16384, 2048, 128) == 0
+
+
+@pytest.mark.parametrize("pool_k,top_k,H_I,T", [(16385, 128, 32, 1), (100, 200, 32, 1), (512, 0, 32, 1),
+                                                (512, 128, 65, 1), (512, 128, 32, 9)])
+def test_index_bounds_rejected_on_host(lib, pool_k, top_k, H_I, T):
+    c = fake_cache()
+    rc = lib.csa2_index_full(ctypes.byref(c), 0x40000, csa2.BF16, 0x50000, T, H_I, pool_k, top_k, 0x60000, 0x70000,
+                             0x80000, 1 << 40, None)
+    assert rc == csa2.ERR_INVALID_ARG
+
+
+def test_bad_pointers_rejected_on_host(lib):
+    c = fake_cache()
+    assert lib.csa2_index_full(ctypes.byref(c), None, csa2.BF16, 0x50000, 1, 32, 512, 128, 0x60000, 0x70000,
+                               0x80000, 1 << 40, None) == csa2.ERR_INVALID_ARG
+    assert lib.csa2_index_full(ctypes.byref(c), 0x40008, csa2.BF16, 0x50000, 1, 32, 512, 128, 0x60000, 0x70000,
+                               0x80000, 1 << 40, None) == csa2.ERR_INVALID_ARG
+    # wrong query dtype for an E4M3 cache
+    assert lib.csa2_index_full(ctypes.byref(c), 0x40000, csa2.F32, 0x50000, 1, 32, 512, 128, 0x60000, 0x70000,
+                               0x80000, 1 << 40, None) == csa2.ERR_INVALID_ARG
+    # workspace too small
+    assert lib.csa2_index_full(ctypes.byref(c), 0x40000, csa2.BF16, 0x50000, 1, 32, 512, 128, 0x60000, 0x70000,
+                               0x80000, 1024, None) == csa2.ERR_INVALID_ARG
+    assert lib.csa2_sparse_swa_attn(ctypes.byref(c), 0x40000, 1, 128, 0x60000, 2048, 128, 0.0, 0x70000, None,
+                                    0x80000, 1 << 40, None) == csa2.ERR_UNSUPPORTED
+    assert lib.csa2_kv_append_quant(ctypes.byref(fake_cache(dim=1024)), 0x40000, None, csa2.BF16, 0x50000, 8,
+                                    None, None) == csa2.ERR_UNSUPPORTED
+    bad_mode = csa2.csa2_layer_args(mode=7)
+    assert lib.csa2_layer_step(ctypes.byref(c), ctypes.byref(bad_mode), 0x80000, 1 << 40, None) == \
+        csa2.ERR_INVALID_ARG

@@ -1,0 +1,126 @@
+"""Indexer parity: Full-layer pool / top-k sets and Reindex top-k sets from the
+CUDA path against the oracle, exact outside the 1e-5 relative band around the
+cutoff score (tldrocket.com "DeepSeek AI Released DeepSeek-V4.1-Flash ...",
+paragraph 3; hackernews.kjhq.dev post 49735410, key points 2-3)."""
+import numpy as np
+import pytest
+import torch
+
+import fp4_sparse_attention_csa2_b200 as csa2
+import oracle
+from fp4_sparse_attention_csa2_b200 import workloads as wl
+from gpu_harness import build_gpu_cache, device_layer, new_ws
+from harness import band_set_check, build_ref_cache, host_layer
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("tiny4k", 4096, {}),
+    ("tiny4k", 333, {}),                        # L < pool: -1 padding
+    ("long64k", 20000, {}),
+    ("long64k", 5000, {"T": 3}),                # causal among 3 query tokens
+    ("batch32_paged", 30000, {"batch": 5}),     # paged, ragged lengths
+    ("append_mq", 9000, {"batch": 2}),          # T = 4
+]
+
+
+def _run_full(w, layer, cache, ws):
+    L = device_layer(layer)
+    pool = torch.full((w.batch, w.T, w.pool_k), -7, dtype=torch.int32, device="cuda")
+    topk = torch.full((w.batch, w.T, w.top_k), -7, dtype=torch.int32, device="cuda")
+    csa2.index_full(cache, L["q_idx"], L["w"], w.pool_k, w.top_k, pool, topk, ws)
+    return pool.cpu().numpy(), topk.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,L,kw", CASES)
+def test_full_pool_and_topk_sets(name, L, kw):
+    w = wl.scaled(wl.WORKLOADS[name], L, **kw)
+    layer = wl.layer_queries(w, 0)
+    ref = build_ref_cache(w, rows=False, layers=[layer])
+    dev = build_gpu_cache(w, q_idx0=layer["q_idx"])
+    ws = new_ws(dev, w)
+    pool, topk = _run_full(w, layer, dev, ws)
+    assert csa2.read_device_status(ws) == csa2.OK
+    hl = host_layer(layer)
+    for b in range(w.batch):
+        for j in range(w.T):
+            rp, rt, s = oracle.index_full(ref, b, w.T, j, hl["q_idx"][b, j], w.q_idx_dtype, hl["w"][b, j],
+                                          w.pool_k, w.top_k, want_scores=True)
+            band_set_check(pool[b, j], rp, lambda t: s[t], s.size)
+            band_set_check(topk[b, j], rt, lambda t: s[t], s.size)
+            # k is a subset of K on the device too
+            assert set(topk[b, j][topk[b, j] >= 0]) <= set(pool[b, j][pool[b, j] >= 0])
+
+
+@pytest.mark.parametrize("name,L,kw", CASES)
+def test_reindex_sets_on_oracle_pool(name, L, kw):
+    w = wl.scaled(wl.WORKLOADS[name], L, **kw)
+    l0, l1 = wl.layer_queries(w, 0), wl.layer_queries(w, 1)
+    ref = build_ref_cache(w, rows=False, layers=[l0])
+    dev = build_gpu_cache(w, q_idx0=l0["q_idx"])
+    ws = new_ws(dev, w)
+    h0, h1 = host_layer(l0), host_layer(l1)
+    pools = np.zeros((w.batch, w.T, w.pool_k), dtype=np.int32)
+    for b in range(w.batch):
+        for j in range(w.T):
+            pools[b, j], _, _ = oracle.index_full(ref, b, w.T, j, h0["q_idx"][b, j], w.q_idx_dtype, h0["w"][b, j],
+                                                  w.pool_k, w.top_k)
+    # shuffle the pool order: the device must not rely on it
+    rng = np.random.default_rng(3)
+    for b in range(w.batch):
+        for j in range(w.T):
+            pools[b, j] = rng.permutation(pools[b, j])
+    D1 = device_layer(l1)
+    topk = torch.full((w.batch, w.T, w.top_k), -7, dtype=torch.int32, device="cuda")
+    pool_d = torch.from_numpy(pools).cuda()
+    csa2.index_reindex(dev, D1["q_idx"], D1["w"], pool_d, w.top_k, topk, ws)
+    topk = topk.cpu().numpy()
+    assert csa2.read_device_status(ws) == csa2.OK
+    assert np.array_equal(pool_d.cpu().numpy(), pools)          # the pool is only read
+    for b in range(w.batch):
+        for j in range(w.T):
+            rt, s = oracle.index_reindex(ref, b, w.T, j, h1["q_idx"][b, j], w.q_idx_dtype, h1["w"][b, j],
+                                         pools[b, j], w.top_k, want_scores=True)
+            by_pos = {int(t): float(v) for t, v in zip(pools[b, j], s) if t >= 0}
+            band_set_check(topk[b, j], rt, lambda t: by_pos[t], len(by_pos))
+
+
+def test_all_equal_scores_select_exactly_k():
+    # every key is zero: all scores tie at 0, any min(K, p+1) distinct positions are right
+    w = wl.scaled(wl.WORKLOADS["long64k"], 40000)
+    cache = csa2.Cache(1, 40000 // 64 * 64 + 64, w.D, 64, w.row_stride, csa2.E4M3, [40000],
+                       seq_stride_slots=40000 // 64 * 64 + 64)
+    ws = new_ws(cache, w)
+    pool, topk = _run_full(w, wl.layer_queries(w, 0), cache, ws)
+    for arr, k in ((pool, w.pool_k), (topk, w.top_k)):
+        v = arr[0, 0]
+        assert np.all(v[:k] >= 0) and np.unique(v).size == k and v.max() < 40000
+
+
+def test_reuse_touches_no_index_buffer():
+    w = wl.scaled(wl.WORKLOADS["long64k"], 6000)
+    dev = build_gpu_cache(w)
+    ws = new_ws(dev, w)
+    rng = np.random.default_rng(0)
+    topk = torch.from_numpy(rng.choice(6000, (1, 1, w.top_k), replace=False).astype(np.int32)).cuda()
+    pool = torch.full((1, 1, w.pool_k), 12345, dtype=torch.int32, device="cuda")
+    before = (topk.clone(), pool.clone())
+    q = wl.layer_queries(w, 3)["q"].cuda()
+    out = torch.empty((1, 1, w.H, w.D), dtype=torch.float32, device="cuda")
+    csa2.layer_step(dev, csa2.REUSE, q, topk, out, ws, w.window, pool_idx=pool)
+    torch.cuda.synchronize()
+    assert torch.equal(topk, before[0]) and torch.equal(pool, before[1])
+
+
+def test_out_of_range_pool_entry_flags_status():
+    w = wl.scaled(wl.WORKLOADS["long64k"], 3000)
+    dev = build_gpu_cache(w)
+    ws = new_ws(dev, w)
+    l1 = device_layer(wl.layer_queries(w, 1))
+    pool = torch.arange(w.pool_k, dtype=torch.int32, device="cuda").view(1, 1, -1) % 3000
+    pool[0, 0, 5] = 3000                        # beyond p
+    pool[0, 0, 6] = -1
+    topk = torch.empty((1, 1, w.top_k), dtype=torch.int32, device="cuda")
+    csa2.index_reindex(dev, l1["q_idx"], l1["w"], pool, w.top_k, topk, ws)
+    assert csa2.read_device_status(ws) == csa2.ERR_DEVICE_BOUNDS
+    assert 3000 not in topk.cpu().numpy()
