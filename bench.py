@@ -187,15 +187,16 @@ def kernel_nodes(graph):
     try:
         import cuda.bindings.runtime as rt
         g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
-        err, _, n = rt.cudaGraphGetNodes(g, None, 0)
-        err, nodes, n = rt.cudaGraphGetNodes(g, None, n)
+        err, _, n = rt.cudaGraphGetNodes(g, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(g, n)
         k = 0
-        for nd in nodes:
+        for nd in nodes[:n]:
             err, t = rt.cudaGraphNodeGetType(nd)
             if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
                 k += 1
         return k
-    except Exception:
+    except Exception as e:  # counting is best effort; the JSON then says null
+        print("kernel node count unavailable: %r" % (e,), file=sys.stderr)
         return None
 
 
@@ -251,11 +252,13 @@ def run_ours(args, world, rank):
 
     graphs = []
     for r in reps:
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
             stack.step(r)
         graphs.append(g)
     launches_per_step = kernel_nodes(graphs[0])
+    for g in graphs:
+        g.instantiate()
     for g in graphs:  # graph warm-up
         g.replay()
     torch.cuda.synchronize()

@@ -149,6 +149,23 @@ csa2_status topk_from_pool(const csa2_cache* c, const Layout& L, void* ws, const
     return cuda_status(launch_select(src, sel_work(ws, L), (int)L.nseg, top_k, topk_idx, top_k, st));
 }
 
+// Scoring launch shared by csa2_index_scores and csa2_index_full: tensor cores
+// for E4M3 keys, CUDA cores for fp32 keys.  hist (nullable) receives the
+// level-1 radix histogram when the tensor-core kernel runs; returns whether it did.
+csa2_status launch_scores(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w, int T,
+                          int H_I, float* scores, uint32_t* hist, uint32_t* status, cudaStream_t st, bool* fused) {
+    DevCache d = dev_cache(cache);
+    *fused = false;
+    cudaError_t e;
+    if (score_full_tc_supported(d, T, H_I)) {
+        e = launch_score_full_tc(d, q_idx, head_w, T, H_I, scores, hist, status, st, num_sms());
+        *fused = hist != nullptr;
+    } else {
+        e = launch_score_full(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, scores, status, st, num_sms());
+    }
+    return cuda_status(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -187,9 +204,11 @@ csa2_status csa2_index_scores(const csa2_cache* cache, const void* q_idx, csa2_d
     Layout L;
     s = check_ws(cache, T, 1, 1, 1, 0, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
-    return cuda_status(launch_score_full(dev_cache(cache), q_idx, q_dtype == CSA2_F32, head_w, T, H_I,
-                                         scores ? scores : at<float>(ws, L.scores), at<uint32_t>(ws, L.status),
-                                         static_cast<cudaStream_t>(stream), num_sms()));
+    bool fused;
+    // the histogram section is scratch here (the same kernel as in csa2_index_full)
+    return launch_scores(cache, q_idx, q_dtype, head_w, T, H_I, scores ? scores : at<float>(ws, L.scores),
+                         at<uint32_t>(ws, L.hist), at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream),
+                         &fused);
 }
 
 csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
@@ -202,10 +221,14 @@ csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dty
     s = check_ws(cache, T, 1, pool_k, top_k, 0, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* hist = at<uint32_t>(ws, L.hist);
+    if (cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)L.nseg * 3 * kRadixBins, st) != cudaSuccess)
+        return CSA2_ERR_CUDA;
     // every visible position scored into the workspace
-    s = csa2_index_scores(cache, q_idx, q_dtype, head_w, T, H_I, nullptr, ws, ws_bytes, stream);
-    if (s != CSA2_OK) return s;
     float* scores = at<float>(ws, L.scores);
+    bool fused = false;
+    s = launch_scores(cache, q_idx, q_dtype, head_w, T, H_I, scores, hist, at<uint32_t>(ws, L.status), st, &fused);
+    if (s != CSA2_OK) return s;
     // the candidate pool: the pool_k best of all visible scores
     SelSrc src;
     src.vals = scores;
@@ -217,7 +240,7 @@ csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dty
     src.seq_lens = cache->seq_lens;
     src.T = T;
     src.cap = L.cap;
-    cudaError_t e = launch_select(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, pool_k, st);
+    cudaError_t e = launch_select(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, pool_k, st, fused);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
     // this layer's top-k: the top_k best of the same scores, taken from the pool
     return topk_from_pool(cache, L, ws, scores, L.cap, 1, pool_idx, pool_k, top_k, topk_idx, T, st);

@@ -155,30 +155,34 @@ k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __re
                float* __restrict__ out, float* __restrict__ lse) {
     const int seg = blockIdx.x, h = blockIdx.y;
     __shared__ float s_w[1024];
-    __shared__ float s_stat[2];
-    if (threadIdx.x == 0) {
-        float m = -INFINITY;
-        for (int ch = 0; ch < nchunk; ++ch) m = fmaxf(m, part_ml[(((int64_t)seg * nchunk + ch) * H + h) * 2]);
-        float l = 0.0f;
-        for (int ch = 0; ch < nchunk; ++ch) {
-            const float* ml = part_ml + (((int64_t)seg * nchunk + ch) * H + h) * 2;
-            const float w = (m == -INFINITY || ml[0] == -INFINITY) ? 0.0f : __expf(ml[0] - m);
-            s_w[ch] = w;
-            l += w * ml[1];
-        }
-        s_stat[0] = m;
-        s_stat[1] = l;
-    }
+    __shared__ float s_red[4];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    float m = -INFINITY;
+    for (int ch = tid; ch < nchunk; ch += 128) m = fmaxf(m, part_ml[(((int64_t)seg * nchunk + ch) * H + h) * 2]);
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_red[wid] = m;
     __syncthreads();
-    const float l = s_stat[1];
+    m = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+    __syncthreads();
+    float l = 0.0f;
+    for (int ch = tid; ch < nchunk; ch += 128) {
+        const float* ml = part_ml + (((int64_t)seg * nchunk + ch) * H + h) * 2;
+        const float w = (m == -INFINITY || ml[0] == -INFINITY) ? 0.0f : __expf(ml[0] - m);
+        s_w[ch] = w;
+        l += w * ml[1];
+    }
+    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) s_red[wid] = l;
+    __syncthreads();
+    l = s_red[0] + s_red[1] + s_red[2] + s_red[3];
     const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    for (int d = tid; d < D; d += blockDim.x) {
         float acc = 0.0f;
         for (int ch = 0; ch < nchunk; ++ch)
             if (s_w[ch] != 0.0f) acc = fmaf(s_w[ch], part_o[(((int64_t)seg * nchunk + ch) * H + h) * D + d], acc);
         out[((int64_t)seg * H + h) * D + d] = acc * inv;
     }
-    if (lse && threadIdx.x == 0) lse[(int64_t)seg * H + h] = l > 0.0f ? s_stat[0] + logf(l) : -INFINITY;
+    if (lse && tid == 0) lse[(int64_t)seg * H + h] = l > 0.0f ? m + logf(l) : -INFINITY;
 }
 
 }  // namespace

@@ -43,13 +43,21 @@ cudaError_t launch_append_quant(const DevCache& c, const void* x, const void* id
 cudaError_t launch_score_full(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
                               float* scores, uint32_t* status, cudaStream_t st, int num_sms);
 
+// Full scoring on tensor cores (E4M3 keys); also accumulates the level-1 radix
+// histogram of every (sequence, token) into hist when it is not null.
+bool score_full_tc_supported(const DevCache& c, int T, int H_I);
+cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* hw, int T, int H_I, float* scores,
+                                 uint32_t* hist, uint32_t* status, cudaStream_t st, int num_sms);
+
 // Pool rescoring: scores[seg * pool_k + i] for pool entry i of segment seg.
 cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
                               const int32_t* pool, int pool_k, float* scores, uint32_t* status, cudaStream_t st);
 
 // Top-n selection per segment into out[seg * out_stride + 0..n_out) (-1 padded).
+// hist_ready: the level-1 histogram was zeroed and accumulated by the scoring
+// kernel already (the counters are still cleared here).
 cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_out, int32_t* out,
-                          int64_t out_stride, cudaStream_t st);
+                          int64_t out_stride, cudaStream_t st, bool hist_ready = false);
 
 // Attention partials + combine.
 struct AttnWork {

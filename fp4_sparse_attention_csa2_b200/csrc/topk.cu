@@ -200,28 +200,58 @@ k_sel_pass(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_t
     const uint32_t* cand_in = LEVEL == 2 ? wk.cand1 + seg * wk.cand_stride : wk.cand2 + seg * wk.cand_stride;
     uint32_t* cand_out = LEVEL == 1 ? wk.cand1 + seg * wk.cand_stride : wk.cand2 + seg * wk.cand_stride;
 
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt_mask = (1u << lane) - 1u;
     for (int64_t base = (int64_t)blockIdx.x * kChunk; base < n_items; base += (int64_t)gridDim.x * kChunk) {
         const int64_t end = min(base + kChunk, n_items);
-        for (int64_t it = base + threadIdx.x; it < end; it += kThreads) {
-            const int64_t i = LEVEL == 1 ? it : (int64_t)cand_in[it];
-            Elem e = load_elem(src, seg, i, nvalid);
-            if (!e.valid) continue;
-            const uint32_t d = digit(e.key, LEVEL);
-            bool take = d > c;
-            if (d == c) {
-                if (LEVEL == 3) {
-                    take = atomicAdd(cnt + 3, 1u) < need_here;
-                } else if (!more) {
-                    take = true;
-                } else {
-                    const uint32_t k = atomicAdd(cnt + LEVEL, 1u);
-                    cand_out[k] = (uint32_t)i;
-                    atomicAdd(&hnext[digit(e.key, LEVEL + 1)], 1u);
+        for (int64_t it0 = base; it0 < end; it0 += kThreads) {
+            const int64_t it = it0 + threadIdx.x;
+            Elem e;
+            e.valid = false;
+            int64_t i = 0;
+            if (it < end) {
+                i = LEVEL == 1 ? it : (int64_t)cand_in[it];
+                e = load_elem(src, seg, i, nvalid);
+            }
+            const uint32_t d = e.valid ? digit(e.key, LEVEL) : 0u;
+            const bool eq = e.valid && d == c;
+            bool take = e.valid && d > c;
+            bool to_cand = false;
+            if (eq && LEVEL < 3) {
+                if (more) to_cand = true;   // resolved by the next digit
+                else take = true;           // exactly the missing number of them
+            }
+            // exact ties at the last level: the first `need_here` claimants win
+            if (LEVEL == 3) {
+                const uint32_t m = __ballot_sync(0xffffffffu, eq);
+                if (m) {
+                    const int leader = __ffs(m) - 1;
+                    uint32_t b0 = 0;
+                    if (lane == leader) b0 = atomicAdd(cnt + 3, (uint32_t)__popc(m));
+                    b0 = __shfl_sync(0xffffffffu, b0, leader);
+                    if (eq && b0 + __popc(m & lt_mask) < need_here) take = true;
                 }
             }
-            if (take) {
-                const uint32_t slot = atomicAdd(cnt, 1u);
-                o[slot] = e.id;
+            if (LEVEL < 3) {
+                const uint32_t m = __ballot_sync(0xffffffffu, to_cand);
+                if (m) {
+                    const int leader = __ffs(m) - 1;
+                    uint32_t b0 = 0;
+                    if (lane == leader) b0 = atomicAdd(cnt + LEVEL, (uint32_t)__popc(m));
+                    b0 = __shfl_sync(0xffffffffu, b0, leader);
+                    if (to_cand) {
+                        cand_out[b0 + __popc(m & lt_mask)] = (uint32_t)i;
+                        atomicAdd(&hnext[digit(e.key, LEVEL + 1)], 1u);
+                    }
+                }
+            }
+            const uint32_t mt = __ballot_sync(0xffffffffu, take);
+            if (mt) {
+                const int leader = __ffs(mt) - 1;
+                uint32_t b0 = 0;
+                if (lane == leader) b0 = atomicAdd(cnt, (uint32_t)__popc(mt));
+                b0 = __shfl_sync(0xffffffffu, b0, leader);
+                if (take) o[b0 + __popc(mt & lt_mask)] = e.id;
             }
         }
     }
@@ -236,14 +266,17 @@ k_sel_pass(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_t
 }  // namespace
 
 cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_out, int32_t* out,
-                          int64_t out_stride, cudaStream_t st) {
-    cudaError_t e = cudaMemsetAsync(wk.hist, 0, sizeof(uint32_t) * (size_t)nseg * 3 * kRadixBins, st);
-    if (e != cudaSuccess) return e;
+                          int64_t out_stride, cudaStream_t st, bool hist_ready) {
+    cudaError_t e;
+    if (!hist_ready) {
+        e = cudaMemsetAsync(wk.hist, 0, sizeof(uint32_t) * (size_t)nseg * 3 * kRadixBins, st);
+        if (e != cudaSuccess) return e;
+    }
     e = cudaMemsetAsync(wk.cnt, 0, sizeof(uint32_t) * (size_t)nseg * 4, st);
     if (e != cudaSuccess) return e;
     const unsigned chunks = (unsigned)((src.n + kChunk - 1) / kChunk);
     dim3 grid(chunks ? chunks : 1, (unsigned)nseg);
-    k_sel_hist<<<grid, kThreads, 0, st>>>(src, wk);
+    if (!hist_ready) k_sel_hist<<<grid, kThreads, 0, st>>>(src, wk);
     k_sel_pass<1><<<grid, kThreads, 0, st>>>(src, wk, n_out, out, out_stride);
     k_sel_pass<2><<<grid, kThreads, 0, st>>>(src, wk, n_out, out, out_stride);
     k_sel_pass<3><<<grid, kThreads, 0, st>>>(src, wk, n_out, out, out_stride);
