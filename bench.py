@@ -27,6 +27,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from fp4_sparse_attention_csa2_b200 import workloads as wl  # noqa: E402
+from fp4_sparse_attention_csa2_b200.runner import Stack, build_replicas  # noqa: E402
 
 METRIC = "CSA2 decode layer-steps/s at 1M ctx; FP4-KV achieved HBM GB/s vs 8 TB/s"
 PROFILE = os.path.join(ROOT, "profiles", "index_score_ctx1m.md")
@@ -129,59 +130,6 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- our arm
-def build_replicas(csa2, w, n_rep, seed, lens):
-    """One cache filled through csa2_kv_append_quant, then copied into n_rep
-    independent buffers (rotated so that no step finds its inputs in L2)."""
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from harness import cache_geometry
-    n_slots, table, stride = cache_geometry(w, lens, seed)
-    base = csa2.Cache(w.batch, n_slots, w.D, w.D_I, w.row_stride, w.idx_key_dtype, lens, table, w.page_size, stride)
-    q0 = wl.layer_queries(w, 0, seed)["q_idx"]
-    sp = torch.zeros(1, dtype=torch.int32, device="cuda")
-    chunk = 1 << 16
-    for b in range(w.batch):
-        L = int(lens[b])
-        x = wl.latent(w, b, L, seed)
-        keys, _ = wl.index_keys(w, b, L, q0[b, w.T - 1], seed)
-        v = base.view(b)
-        for t0 in range(0, L, chunk):
-            sp.fill_(t0)
-            csa2.kv_append_quant(v, x[t0:t0 + chunk][None].cuda(), sp, keys[t0:t0 + chunk][None].cuda())
-        torch.cuda.synchronize()
-    reps = [base]
-    for _ in range(n_rep - 1):
-        c = csa2.Cache(w.batch, n_slots, w.D, w.D_I, w.row_stride, w.idx_key_dtype, lens, table, w.page_size,
-                       stride)
-        c.rows.copy_(base.rows)
-        c.idx_keys.copy_(base.idx_keys)
-        reps.append(c)
-    torch.cuda.synchronize()
-    return reps
-
-
-class Stack:
-    """Device buffers of one decode step and the C-ABI calls that run it."""
-
-    def __init__(self, csa2, w, layers, ws):
-        self.csa2, self.w, self.ws = csa2, w, ws
-        B, T = w.batch, w.T
-        self.layers = [{k: v.cuda() for k, v in L.items()} for L in layers]
-        self.pool = torch.zeros((B, T, w.pool_k), dtype=torch.int32, device="cuda")
-        self.topk = torch.zeros((B, T, w.top_k), dtype=torch.int32, device="cuda")
-        self.out = [torch.empty((B, T, w.H, w.D), dtype=torch.float32, device="cuda") for _ in w.pattern]
-        self.lse = [torch.empty((B, T, w.H), dtype=torch.float32, device="cuda") for _ in w.pattern]
-        self.modes = [{"F": csa2.FULL, "R": csa2.REINDEX, "U": csa2.REUSE}[m] for m in w.pattern]
-
-    def step(self, cache):
-        c = self.csa2
-        for l, m in enumerate(self.modes):
-            L = self.layers[l]
-            idx = m != c.REUSE
-            c.layer_step(cache, m, L["q"], self.topk, self.out[l], self.ws, self.w.window,
-                         q_idx=L["q_idx"] if idx else None, head_w=L["w"] if idx else None, pool_idx=self.pool,
-                         lse=self.lse[l], pool_k=self.w.pool_k)
-
-
 def kernel_nodes(graph):
     """Number of kernel nodes in a captured CUDA graph (all of them are libcsa2's)."""
     try:
@@ -234,11 +182,11 @@ def run_ours(args, world, rank):
     seed = args.seed + rank
     lens = wl.seq_lens(w, seed)
     layers = [wl.layer_queries(w, l, seed) for l in range(len(w.pattern))]
-    reps = build_replicas(csa2, w, args.replicas, seed, lens)
+    reps = build_replicas(w, args.replicas, seed, lens)
     n_ws = csa2.workspace_bytes(reps[0], w.T, w.H, w.pool_k, w.top_k, w.window)
     ws = torch.empty(n_ws, dtype=torch.uint8, device="cuda")
     csa2.workspace_init(ws)
-    stack = Stack(csa2, w, layers, ws)
+    stack = Stack(w, layers, ws)
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
 

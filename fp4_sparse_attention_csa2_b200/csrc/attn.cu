@@ -189,20 +189,38 @@ k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __re
 
 int attn_rows_per_chunk() { return kRows; }
 
-cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
-                             int window, float sm_scale, float* out, float* lse, const AttnWork& aw,
-                             uint32_t* status, cudaStream_t st) {
-    const int D = c.dim;
-    const size_t smem = sizeof(float) * ((size_t)H * (D + 4) + (size_t)kRows * (D + 4) + (size_t)H * kRows) +
-                        sizeof(int) * kRows;
-    cudaError_t e = cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)aw.nchunk, (unsigned)(c.batch * T));
-    k_attn_partial<<<grid, kThreads, smem, st>>>(c, static_cast<const __nv_bfloat16*>(q), T, H, topk, top_k, window,
-                                                 sm_scale, aw.part_o, aw.part_ml, aw.nchunk, status);
-    k_attn_combine<<<dim3((unsigned)(c.batch * T), (unsigned)H), 128, 0, st>>>(D, H, aw.part_o, aw.part_ml,
+cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
+                                cudaStream_t st) {
+    k_attn_combine<<<dim3((unsigned)(c.batch * T), (unsigned)H), 128, 0, st>>>(c.dim, H, aw.part_o, aw.part_ml,
                                                                              aw.nchunk, out, lse);
     return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
+                             int window, float sm_scale, float* out, float* lse, const AttnWork& aw_in,
+                             uint32_t* status, cudaStream_t st) {
+    AttnWork aw = aw_in;
+    cudaError_t e;
+    if (attn_tc_supported(c, H)) {
+        const int rows = attn_tc_rows_per_chunk();
+        aw.nchunk = (window + top_k + rows - 1) / rows;
+        if (aw.nchunk < 1) aw.nchunk = 1;
+        e = launch_attention_tc(c, q, T, H, topk, top_k, window, sm_scale, aw, status, st);
+    } else {
+        const int D = c.dim;
+        aw.nchunk = (window + top_k + kRows - 1) / kRows;
+        if (aw.nchunk < 1) aw.nchunk = 1;
+        const size_t smem = sizeof(float) * ((size_t)H * (D + 4) + (size_t)kRows * (D + 4) + (size_t)H * kRows) +
+                            sizeof(int) * kRows;
+        e = cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        dim3 grid((unsigned)aw.nchunk, (unsigned)(c.batch * T));
+        k_attn_partial<<<grid, kThreads, smem, st>>>(c, static_cast<const __nv_bfloat16*>(q), T, H, topk, top_k,
+                                                     window, sm_scale, aw.part_o, aw.part_ml, aw.nchunk, status);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return e;
+    return launch_attn_combine(c, T, H, aw, out, lse, st);
 }
 
 }  // namespace csa2

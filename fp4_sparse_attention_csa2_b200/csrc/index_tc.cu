@@ -227,10 +227,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_full_tc(const Params p) {
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_f16_f32(kTile, p.NP);
             uint32_t g = 0, n = 0;
+            int cur_b = -1;
             bool ok = true;
             for (int64_t item = blockIdx.x; item < p.total_items && ok; item += gridDim.x) {
                 Item it;
                 if (!get_item(p, item, it)) continue;
+                if (it.b != cur_b) {
+                    // the query buffer of the previous sequence is free once its MMAs are done
+                    if (cur_b >= 0) { tc::mma_commit(&bars->b_free[n & 1]); ++n; }
+                    cur_b = it.b;
+                }
                 const uint32_t bq = tc::smem_u32(sB + (n & 1) * (p.NP * 128));
                 for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                     const int a = g % kA, acc = g & 1;
@@ -245,9 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_full_tc(const Params p) {
                     tc::mma_commit(&bars->a_empty[a]);
                     tc::mma_commit(&bars->acc_full[acc]);
                 }
-                if (!ok) break;
-                tc::mma_commit(&bars->b_free[n & 1]);
-                ++n;
             }
             if (!ok) flag(p.status, kStatusTimeout);
             tc::mma_commit(&bars->drain);
@@ -257,16 +260,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_full_tc(const Params p) {
         // converters: 128 threads
         const int tid = threadIdx.x - kWarpConv0 * 32;
         uint32_t g = 0, n = 0;
+        int cur_b = -1;
         bool ok = true;
         for (int64_t item = blockIdx.x; item < p.total_items && ok; item += gridDim.x) {
             Item it;
             if (!get_item(p, item, it)) continue;
-            const int qb = n & 1;
-            if (!tc::mbar_wait(&bars->b_free[qb], ((n >> 1) & 1) ^ 1) ||
-                !tc::mbar_wait(&bars->wq_free[qb], ((n >> 1) & 1) ^ 1)) { ok = false; break; }
-            prepare_queries(p, it.b, sB + qb * (p.NP * 128), sWq + qb * p.NP, tid);
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&bars->wq_ready[qb]);
+            if (it.b != cur_b) {
+                // a new sequence: stage its queries in the other buffer
+                if (cur_b >= 0) ++n;
+                cur_b = it.b;
+                const int qb = n & 1;
+                if (!tc::mbar_wait(&bars->b_free[qb], ((n >> 1) & 1) ^ 1) ||
+                    !tc::mbar_wait(&bars->wq_free[qb], ((n >> 1) & 1) ^ 1)) { ok = false; break; }
+                prepare_queries(p, it.b, sB + qb * (p.NP * 128), sWq + qb * p.NP, tid);
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(&bars->wq_ready[qb]);
+            }
             for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                 const int s = g % kRaw, a = g % kA;
                 if (!tc::mbar_wait(&bars->raw_full[s], (g / kRaw) & 1) ||
@@ -289,7 +298,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_full_tc(const Params p) {
                 tc::mbar_arrive(&bars->a_full[a]);
                 tc::mbar_arrive(&bars->raw_empty[s]);
             }
-            ++n;
         }
         if (!ok) flag(p.status, kStatusTimeout);
     } else {
@@ -326,16 +334,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_full_tc(const Params p) {
             const bool got = tc::mbar_wait(bar, parity);
             return __all_sync(0xffffffffu, got);
         };
+        const float* wq = sWq;
         for (int64_t item = blockIdx.x; item < p.total_items && ok; item += gridDim.x) {
             Item it;
             if (!get_item(p, item, it)) continue;
             if (it.b != cur_b) {
-                if (cur_b >= 0 && !flush(cur_b)) { ok = false; break; }
+                if (cur_b >= 0) {
+                    if (!flush(cur_b)) { ok = false; break; }
+                    tc::mbar_arrive(&bars->wq_free[n & 1]);
+                    ++n;
+                }
                 cur_b = it.b;
+                if (!warp_wait(&bars->wq_ready[n & 1], (n >> 1) & 1)) { ok = false; break; }
+                wq = sWq + (n & 1) * p.NP;
             }
-            const int qb = n & 1;
-            if (!warp_wait(&bars->wq_ready[qb], (n >> 1) & 1)) { ok = false; break; }
-            const float* wq = sWq + qb * p.NP;
             for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                 const int acc = g & 1;
                 if (!warp_wait(&bars->acc_full[acc], (g >> 1) & 1)) { ok = false; break; }
@@ -349,17 +361,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_full_tc(const Params p) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) s = fmaf(wq[c0 + i], fmaxf(v[i], 0.0f), s);
                     }
-                    if (t <= it.L - p.T + j) {
-                        p.scores[((int64_t)it.b * p.T + j) * p.c.cap + t] = s;
-                        if (p.hist) atomicAdd(&sHist[j * kRadixBins + (ordered_key(s) >> 21)], 1u);
+                    const bool vis = t <= it.L - p.T + j;
+                    if (vis) p.scores[((int64_t)it.b * p.T + j) * p.c.cap + t] = s;
+                    if (p.hist) {
+                        // lanes that hit the same bin add once (scores crowd into few bins)
+                        const uint32_t bin = vis ? (ordered_key(s) >> 21) : 0xFFFFFFFFu;
+                        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                        if (vis && lane == __ffs(peers) - 1)
+                            atomicAdd(&sHist[j * kRadixBins + bin], (uint32_t)__popc(peers));
                     }
                 }
                 tc::fence_before_sync();
                 tc::mbar_arrive(&bars->acc_empty[acc]);
             }
-            if (!ok) break;
-            tc::mbar_arrive(&bars->wq_free[qb]);
-            ++n;
         }
         if (ok && cur_b >= 0 && !flush(cur_b)) ok = false;
         if (!ok) flag(p.status, kStatusTimeout);

@@ -65,7 +65,13 @@ struct AttnWork {
     float* part_ml;   // [nseg][nchunk][H][2]
     int nchunk;
 };
-int attn_rows_per_chunk();
+int attn_rows_per_chunk();       // smallest chunk of any attention kernel (sizes the workspace)
+bool attn_tc_supported(const DevCache& c, int H);
+int attn_tc_rows_per_chunk();
+cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
+                                int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st);
+cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
+                                cudaStream_t st);
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
                              int window, float sm_scale, float* out, float* lse, const AttnWork& aw,
                              uint32_t* status, cudaStream_t st);

@@ -132,10 +132,27 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: fp16 A and B (K-major), fp32 accumulator, M x N.
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+// Shared-memory operand descriptor, MN-major, 128-byte swizzle: each 128-B row
+// holds 64 consecutive M (or N) elements of one k; 8 such rows (k .. k+7) form
+// a 1024-B atom.  lbo: bytes between atoms along M/N; sbo: bytes between
+// 8-row groups along K.  The start address must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// Instruction descriptor: fp16 A and B, fp32 accumulator, M x N; A and B
+// K-major unless a_mn / b_mn.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn = false, bool b_mn = false) {
     return (1u << 4)                                   // D format: f32
            | (0u << 7) | (0u << 10)                    // A, B format: f16
+           | (static_cast<uint32_t>(a_mn) << 15)       // A major-ness
+           | (static_cast<uint32_t>(b_mn) << 16)       // B major-ness
            | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }

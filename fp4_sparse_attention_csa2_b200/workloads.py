@@ -122,6 +122,16 @@ def page_table(w: Workload, lens, seed=0):
     return table, n_pages
 
 
+def cache_geometry(w: Workload, lens, seed=0):
+    """(n_slots, page_table | None, seq_stride_slots) of the cache that holds
+    sequences of these lengths."""
+    if w.paged:
+        table, n_pages = page_table(w, lens, seed)
+        return n_pages * w.page_size, table, 0
+    cap = capacity(w, lens)
+    return w.batch * cap, None, cap
+
+
 def latent(w: Workload, b, L, seed=0, t0=0):
     """bf16 N(0,1) latent rows [L - t0, D] for positions t0..L-1 of sequence b."""
     g = _gen(seed, 2, b)

@@ -6,13 +6,7 @@ import oracle
 from fp4_sparse_attention_csa2_b200 import workloads as wl
 
 
-def cache_geometry(w, lens, seed=0):
-    """(n_slots, page_table|None, seq_stride_slots) for a workload."""
-    if w.paged:
-        table, n_pages = wl.page_table(w, lens, seed)
-        return n_pages * w.page_size, table, 0
-    cap = wl.capacity(w, lens)
-    return w.batch * cap, None, cap
+cache_geometry = wl.cache_geometry
 
 
 def build_ref_cache(w, seed=0, lens=None, rows=True, layers=None, batches=None):
