@@ -110,18 +110,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     tc::fence_after_sync();
     const uint32_t tmem = misc->tmem_base;
 
+    // ---- gather: every load of this thread is issued before any is used
+    // item = (row, 16-byte code chunk = 32 channels); at most 8 items per thread
+    const int nchunk16 = D / 32;
+    const int n_items = kRows * nchunk16 / kThreads;
+    uint4 gcode[8];
+    uint16_t gscale[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (k < n_items) {
+            const int w = k * kThreads + tid;
+            const int r = w / nchunk16, cc = w - r * nchunk16;
+            const int32_t t = misc->pos[r];
+            const int64_t slot = t >= 0 ? slot_of(p.c, b, t) : -1;
+            if (t >= 0 && slot < 0) flag(p.status, kStatusBounds);
+            if (slot >= 0) {
+                const uint8_t* row = p.c.rows + slot * p.c.row_stride;
+                gcode[k] = __ldg(reinterpret_cast<const uint4*>(row + cc * 16));
+                gscale[k] = __ldg(reinterpret_cast<const uint16_t*>(row + (D >> 1) + 2 * cc));
+            } else {
+                gcode[k] = make_uint4(0u, 0u, 0u, 0u);
+                gscale[k] = 0;                                  // E4M3 zero scale: the row dequantises to 0
+            }
+        }
+    }
+
     // ---- queries: fp16 scaled by 2^e per head, K-major swizzled (4 threads per head)
     for (int w = tid; w < H * 4; w += kThreads) {
         const int h = w >> 2, part = w & 3;           // part: D/4 consecutive values
         const int span = D / 4;
         const __nv_bfloat16* src = p.q + ((int64_t)seg * H + h) * D + part * span;
-        float m = 0.0f;
-        for (int i = 0; i < span; i += 8) {
-            const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + i));
-            const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+        uint4 qv[16];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[k] << 16)), fabsf(__uint_as_float(wv[k] & 0xFFFF0000u))));
+        for (int i = 0; i < 16; ++i)
+            if (8 * i < span) qv[i] = __ldg(reinterpret_cast<const uint4*>(src + 8 * i));
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (8 * i < span) {
+                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[k] << 16)), fabsf(__uint_as_float(wv[k] & 0xFFFF0000u))));
+            }
         }
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
@@ -132,55 +163,48 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         }
         const float up = __uint_as_float((uint32_t)(127 + e) << 23);
         if (part == 0) misc->fac[h] = p.scale * __uint_as_float((uint32_t)(127 - e) << 23);
-        for (int i = 0; i < span; i += 8) {
-            const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + i));
-            const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-            uint32_t hv[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                __half2 hh = __floats2half2_rn(__uint_as_float(wv[k] << 16) * up,
-                                               __uint_as_float(wv[k] & 0xFFFF0000u) * up);
-                memcpy(&hv[k], &hh, 4);
+        for (int i = 0; i < 16; ++i) {
+            if (8 * i < span) {
+                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+                uint32_t hv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    __half2 hh = __floats2half2_rn(__uint_as_float(wv[k] << 16) * up,
+                                                   __uint_as_float(wv[k] & 0xFFFF0000u) * up);
+                    memcpy(&hv[k], &hh, 4);
+                }
+                const int d = part * span + 8 * i;        // 8 values: one 16-byte chunk
+                uint8_t* blk = sQ + (d >> 6) * (H * 128);
+                *reinterpret_cast<uint4*>(blk + tc::sw128_offset(h, (d & 63) >> 3)) =
+                    make_uint4(hv[0], hv[1], hv[2], hv[3]);
             }
-            const int d = part * span + i;            // 8 values: one 16-byte chunk
-            uint8_t* blk = sQ + (d >> 6) * (H * 128);
-            *reinterpret_cast<uint4*>(blk + tc::sw128_offset(h, (d & 63) >> 3)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
     }
 
-    // ---- gather + dequantise: item = (row, 16-byte code chunk = 32 channels)
-    const int nchunk16 = D / 32;
-    for (int w = tid; w < kRows * nchunk16; w += kThreads) {
-        const int r = w / nchunk16, cc = w - r * nchunk16;
-        const int32_t t = misc->pos[r];
-        int64_t slot = t >= 0 ? slot_of(p.c, b, t) : -1;
-        if (t >= 0 && slot < 0) flag(p.status, kStatusBounds);
-        uint4 out[4];
-        if (slot >= 0) {
-            const uint8_t* row = p.c.rows + slot * p.c.row_stride;
-            const uint4 codes = __ldg(reinterpret_cast<const uint4*>(row + cc * 16));
-            const uint16_t sc2 = __ldg(reinterpret_cast<const uint16_t*>(row + (D >> 1) + 2 * cc));
+    // ---- dequantise: value(code) * value(scale), exact in fp16, into the swizzled V tile
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (k < n_items) {
+            const int w = k * kThreads + tid;
+            const int r = w / nchunk16, cc = w - r * nchunk16;
             uint32_t s2;
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(sc2));
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(gscale[k]));
             const uint32_t s_lo = (s2 & 0xFFFFu) * 0x10001u;            // (s0, s0)
             const uint32_t s_hi = (s2 >> 16) * 0x10001u;                // (s1, s1)
-            const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+            const uint32_t cw[4] = {gcode[k].x, gcode[k].y, gcode[k].z, gcode[k].w};
             uint32_t hv[16];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int q = 0; q < 4; ++q)
 #pragma unroll
                 for (int bb = 0; bb < 4; ++bb)
-                    hv[4 * k + bb] = hmul2_u32(cvt_e2m1x2_f16x2(cw[k] >> (8 * bb)), k < 2 ? s_lo : s_hi);
+                    hv[4 * q + bb] = hmul2_u32(cvt_e2m1x2_f16x2(cw[q] >> (8 * bb)), q < 2 ? s_lo : s_hi);
+            uint8_t* blk = sV + (cc >> 1) * (kRows * 128);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) out[k] = make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
-        } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) out[k] = make_uint4(0u, 0u, 0u, 0u);
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(blk + tc::sw128_offset(r, 4 * (cc & 1) + q)) =
+                    make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
         }
-        uint8_t* blk = sV + (cc >> 1) * (kRows * 128);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(blk + tc::sw128_offset(r, 4 * (cc & 1) + k)) = out[k];
     }
     tc::fence_proxy_async_smem();
     __syncthreads();

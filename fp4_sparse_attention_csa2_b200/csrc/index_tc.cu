@@ -32,13 +32,13 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kItemTiles = 4;
-constexpr int kRaw = 8;
+constexpr int kRaw = 6;
 constexpr int kA = 2;
 constexpr int kRawBytes = kTile * 64;   // E4M3 keys of one tile
 constexpr int kABytes = kTile * 128;    // 128 rows x 64 fp16
 constexpr int kThreads = 320;
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpConv0 = 2, kWarpEpi0 = 6;
-constexpr uint32_t kDrainLimit = 1u << 24;
+constexpr uint32_t kDrainLimit = 65536;   // tries of the drain waits (x kSuspendNs)
 
 struct Params {
     DevCache c;
@@ -146,7 +146,7 @@ __device__ void prepare_queries(const Params& p, int b, uint8_t* bq, float* wq, 
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_score_full_tc(const Params p) {
+__global__ void __launch_bounds__(kThreads, 2) k_score_full_tc(const Params p) {
     extern __shared__ uint8_t smem_raw[];
     // operand tiles need 1024-byte alignment for the 128-byte swizzle
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -354,13 +354,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_full_tc(const Params p) {
                 tc::fence_after_sync();
                 const int64_t t = it.t0 + (int64_t)tl * kTile + row;
                 for (int j = 0; j < p.T; ++j) {
-                    float s = 0.0f;
+                    float s0 = 0.0f, s1 = 0.0f;
                     for (int c0 = j * p.HP; c0 < (j + 1) * p.HP; c0 += 16) {
                         float v[16];
                         tc::tmem_ld16(lane_addr + (uint32_t)(acc * p.NP + c0), v);
+                        const float4* w4 = reinterpret_cast<const float4*>(wq + c0);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) s = fmaf(wq[c0 + i], fmaxf(v[i], 0.0f), s);
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 ww = w4[i];
+                            s0 = fmaf(ww.x, fmaxf(v[4 * i], 0.0f), s0);
+                            s1 = fmaf(ww.y, fmaxf(v[4 * i + 1], 0.0f), s1);
+                            s0 = fmaf(ww.z, fmaxf(v[4 * i + 2], 0.0f), s0);
+                            s1 = fmaf(ww.w, fmaxf(v[4 * i + 3], 0.0f), s1);
+                        }
                     }
+                    const float s = s0 + s1;
                     const bool vis = t <= it.L - p.T + j;
                     if (vis) p.scores[((int64_t)it.b * p.T + j) * p.c.cap + t] = s;
                     if (p.hist) {
@@ -437,7 +445,7 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
     const size_t smem = off + 1024;  // room to align the base to 1024 B
     cudaError_t e = cudaFuncSetAttribute(k_score_full_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    int64_t grid = num_sms;
+    int64_t grid = 2 * (int64_t)num_sms;   // two CTAs per SM
     if (grid > p.total_items) grid = p.total_items;
     if (grid < 1) grid = 1;
     k_score_full_tc<<<(unsigned)grid, kThreads, smem, st>>>(p);

@@ -9,9 +9,11 @@
 namespace csa2 {
 namespace tc {
 
-// Iterations of try_wait before a wait gives up (each try_wait may suspend
-// for a hardware-defined interval, so this is well above any legal wait).
-constexpr uint32_t kWaitLimit = 1u << 22;
+// A waiting thread sleeps in try_wait for up to kSuspendNs per try (it wakes
+// as soon as the phase completes); after kWaitLimit tries (about 2 s) the wait
+// gives up.
+constexpr uint32_t kSuspendNs = 65536;
+constexpr uint32_t kWaitLimit = 32768;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -39,10 +41,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
