@@ -176,11 +176,24 @@ k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __re
     __syncthreads();
     l = s_red[0] + s_red[1] + s_red[2] + s_red[3];
     const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-    for (int d = tid; d < D; d += blockDim.x) {
-        float acc = 0.0f;
-        for (int ch = 0; ch < nchunk; ++ch)
-            if (s_w[ch] != 0.0f) acc = fmaf(s_w[ch], part_o[(((int64_t)seg * nchunk + ch) * H + h) * D + d], acc);
-        out[((int64_t)seg * H + h) * D + d] = acc * inv;
+    // every thread owns up to 4 channels; a masked chunk has weight 0 and a
+    // zero partial, so all loads are unconditional and independent
+    const float* base = part_o + ((int64_t)seg * nchunk * H + h) * D;
+    const int64_t cstride = (int64_t)H * D;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ch = 0; ch < nchunk; ++ch) {
+        const float w = s_w[ch];
+        const float* src = base + ch * cstride;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int d = tid + 128 * k;
+            if (d < D) acc[k] = fmaf(w, src[d], acc[k]);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int d = tid + 128 * k;
+        if (d < D) out[((int64_t)seg * H + h) * D + d] = acc[k] * inv;
     }
     if (lse && tid == 0) lse[(int64_t)seg * H + h] = l > 0.0f ? m + logf(l) : -INFINITY;
 }

@@ -5,18 +5,19 @@
 // Reuse", paragraph 3; hackernews.kjhq.dev post 49735410, key point 2, "Top-K
 // indices").
 //
-// The 32-bit key is split into three digits: bits 31..21, 20..10 and 9..0.
-//   hist pass : histogram of digit 1 over every valid element.
-//   level 1   : every CTA finds, from the histogram, the digit value c1 that
-//               holds the n-th largest key.  Elements above c1 are selected;
-//               elements equal to c1 are either all selected (when exactly the
-//               missing number of them exist) or appended to a candidate list
-//               and histogrammed on digit 2.
-//   level 2/3 : the same on the candidate list with the next digit; at level 3
-//               the remaining equal keys are exact ties and the first ones to
-//               claim a slot are selected.
-// Output order is unspecified; -1 pads the tail.  Every CTA re-derives the
-// thresholds from the (small) histograms, so no pass waits on another CTA.
+// The key is split into three digits: bits 31..21, 20..10 and 9..0.  For a
+// digit histogram h and a number `need` still to select, the threshold digit c
+// satisfies above(c) < need <= above(c) + h[c]; elements with a larger digit
+// are selected, elements with digit c go on to the next digit, and at the last
+// digit the remaining equal keys are exact ties of which the first claimants
+// win.  Output order is unspecified; -1 pads the tail.
+//
+//   large segments (Full layer, up to 1M scores): the level-1 histogram comes
+//     from the scoring kernel; a streaming pass (many CTAs per segment)
+//     selects above c1 and compacts the digit-c1 elements into a candidate
+//     list; one CTA per segment then resolves digits 2 and 3 on that list.
+//   small segments (<= 16,384: the top-k of a pool): one CTA per segment keeps
+//     every key in shared memory and resolves all three digits there.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,9 +25,10 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kPerThread = 16;
-constexpr int kChunk = kThreads * kPerThread;  // elements per CTA and pass
+constexpr int kPassThreads = 256;
+constexpr int kPassChunk = kPassThreads * 16;
+constexpr int kFinThreads = 1024;
+constexpr int kSmallMax = 16384;
 
 struct Elem {
     bool valid;
@@ -61,205 +63,309 @@ __device__ __forceinline__ uint32_t digit(uint32_t key, int level) {
     return level == 1 ? (key >> 21) : level == 2 ? ((key >> 10) & 0x7FFu) : (key & 0x3FFu);
 }
 
-// Block-wide: find c with above(c) < need <= above(c) + h[c], where above(c) is
-// the number of elements in bins > c.  Writes c and above(c) to out[0..1].
-// Requires 1 <= need <= sum(h).  256 threads, 2048 bins.
-__device__ void find_threshold(const uint32_t* __restrict__ h, uint32_t need, uint32_t* s_scan, uint32_t* out) {
-    const int tid = threadIdx.x;
-    // thread tid owns bins [2040 - 8*tid, 2047 - 8*tid] (thread 0: the top bins)
-    const int hi = kRadixBins - 1 - 8 * tid;
-    uint32_t local[8];
+// One warp: threshold digit of a 2048-bin histogram (global or shared).  Lane l
+// owns the 64 bins [2047 - 64 l - 63, 2047 - 64 l].  Returns (c, above(c)) in
+// every lane; requires 1 <= need <= sum(h).
+__device__ __forceinline__ uint2 warp_threshold(const uint32_t* h, uint32_t need) {
+    const int lane = threadIdx.x & 31;
+    const int hi = kRadixBins - 1 - 64 * lane;
     uint32_t sum = 0;
+#pragma unroll 16
+    for (int k = 0; k < 64; ++k) sum += h[hi - k];
+    uint32_t incl = sum;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) { local[k] = h[hi - k]; sum += local[k]; }
-    s_scan[tid] = sum;
-    __syncthreads();
-    // inclusive scan over 256 thread sums (Hillis-Steele)
-    for (int off = 1; off < kThreads; off <<= 1) {
-        uint32_t v = tid >= off ? s_scan[tid - off] : 0u;
-        __syncthreads();
-        s_scan[tid] += v;
-        __syncthreads();
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
     }
-    uint32_t above = tid ? s_scan[tid - 1] : 0u;   // elements in bins above this thread's range
-    if (above < need && need <= s_scan[tid]) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            if (above < need && need <= above + local[k]) {
-                out[0] = (uint32_t)(hi - k);
-                out[1] = above;
-                break;
-            }
-            above += local[k];
+    const uint32_t excl = incl - sum;
+    const bool mine = excl < need && need <= incl;
+    const int owner = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    uint2 r = make_uint2(0u, 0u);
+    if (mine) {
+        uint32_t above = excl;
+        for (int k = 0; k < 64; ++k) {
+            const uint32_t c = h[hi - k];
+            if (need <= above + c) { r = make_uint2((uint32_t)(hi - k), above); break; }
+            above += c;
         }
     }
-    __syncthreads();
+    r.x = __shfl_sync(0xffffffffu, r.x, owner & 31);
+    r.y = __shfl_sync(0xffffffffu, r.y, owner & 31);
+    return r;
 }
 
-__device__ uint32_t block_sum_hist(const uint32_t* __restrict__ h, uint32_t* s_red) {
+__device__ __forceinline__ uint32_t warp_sum_hist(const uint32_t* h) {
     uint32_t v = 0;
-    for (int i = threadIdx.x; i < kRadixBins; i += kThreads) v += h[i];
-    v = __reduce_add_sync(0xffffffffu, v);
-    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    uint32_t tot = 0;
-    for (int w = 0; w < kThreads / 32; ++w) tot += s_red[w];
-    __syncthreads();
-    return tot;
+    for (int i = threadIdx.x & 31; i < kRadixBins; i += 32) v += h[i];
+    return __reduce_add_sync(0xffffffffu, v);
 }
 
-// Thresholds of levels 1..level (shared with the block).
-struct Plan {
-    uint32_t need0;          // total to select: min(n_out, n_valid)
-    uint32_t c[4];           // c[l]: threshold digit at level l
-    uint32_t need[4];        // need[l]: still missing after taking digits > c[l]
-    uint32_t cnt_eq[4];      // hist_l[c_l]
-    bool direct[4];          // level l takes all of its equal-digit elements
-};
-
-__device__ void make_plan(const uint32_t* hist, int n_out, int level, Plan* p, uint32_t* s_scan, uint32_t* s_red,
-                          uint32_t* s_out) {
-    const uint32_t total = block_sum_hist(hist, s_red);
-    uint32_t need = total < (uint32_t)n_out ? total : (uint32_t)n_out;
-    if (threadIdx.x == 0) p->need0 = need;
-    for (int l = 1; l <= level; ++l) {
-        if (need == 0) {
-            if (threadIdx.x == 0) { p->c[l] = 0xFFFFFFFFu; p->need[l] = 0; p->cnt_eq[l] = 0; p->direct[l] = true; }
-            __syncthreads();
-            continue;
-        }
-        const uint32_t* h = hist + (l - 1) * kRadixBins;
-        find_threshold(h, need, s_scan, s_out);
-        const uint32_t c = s_out[0], above = s_out[1];
-        const uint32_t rem = need - above;
-        const uint32_t eq = h[c];
-        if (threadIdx.x == 0) {
-            p->c[l] = c;
-            p->cnt_eq[l] = eq;
-            p->direct[l] = (eq == rem) || l == 3;
-            p->need[l] = rem;
-        }
-        __syncthreads();
-        // elements equal at this level: all selected when `direct`, otherwise the
-        // next level needs `rem` of them; a direct level ends the search
-        need = p->direct[l] ? 0 : rem;
+// Warp-aggregated claim: the lanes with `pred` get consecutive values of *counter.
+__device__ __forceinline__ uint32_t warp_claim(bool pred, uint32_t* counter) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t m = __ballot_sync(0xffffffffu, pred);
+    uint32_t base = 0;
+    if (m) {
+        const int leader = __ffs(m) - 1;
+        if (lane == leader) base = atomicAdd(counter, (uint32_t)__popc(m));
+        base = __shfl_sync(0xffffffffu, base, leader);
     }
-    __syncthreads();
+    return base + __popc(m & ((1u << lane) - 1u));
 }
 
-__global__ void __launch_bounds__(kThreads)
-k_sel_hist(SelSrc src, SelWork wk) {
+// ---------------------------------------------------------------- large segments
+// Level-1 histogram, for sources that did not get one from the scoring kernel.
+__global__ void __launch_bounds__(kPassThreads) k_sel_hist(SelSrc src, SelWork wk) {
     __shared__ uint32_t h[kRadixBins];
     const int seg = blockIdx.y;
-    for (int i = threadIdx.x; i < kRadixBins; i += kThreads) h[i] = 0;
+    for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads) h[i] = 0;
     __syncthreads();
     const int64_t nvalid = n_valid_positions(src, seg);
-    const int64_t base = (int64_t)blockIdx.x * kChunk;
-    const int64_t end = min(base + kChunk, src.ids ? src.n : nvalid);
-    for (int64_t i = base + threadIdx.x; i < end; i += kThreads) {
+    const int64_t base = (int64_t)blockIdx.x * kPassChunk;
+    const int64_t end = min(base + kPassChunk, src.ids ? src.n : nvalid);
+    for (int64_t i = base + threadIdx.x; i < end; i += kPassThreads) {
         Elem e = load_elem(src, seg, i, nvalid);
         if (e.valid) atomicAdd(&h[digit(e.key, 1)], 1u);
     }
     __syncthreads();
     uint32_t* gh = wk.hist + (int64_t)seg * 3 * kRadixBins;
-    for (int i = threadIdx.x; i < kRadixBins; i += kThreads)
+    for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads)
         if (h[i]) atomicAdd(gh + i, h[i]);
 }
 
-template <int LEVEL>
-__global__ void __launch_bounds__(kThreads)
-k_sel_pass(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
-    __shared__ uint32_t s_scan[kThreads];
-    __shared__ uint32_t s_red[kThreads / 32];
-    __shared__ uint32_t s_out[2];
-    __shared__ Plan plan;
-    __shared__ uint32_t hnext[kRadixBins];
+// Level 1 over every element: select digit > c1, compact digit == c1.
+__global__ void __launch_bounds__(kPassThreads)
+k_sel_pass1(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    __shared__ uint32_t s_plan[3];   // c1, elements to select, take every digit-c1 element
+    __shared__ uint32_t h2[kRadixBins];
     const int seg = blockIdx.y;
-    const uint32_t* hist = wk.hist + (int64_t)seg * 3 * kRadixBins;
+    const uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
     uint32_t* cnt = wk.cnt + (int64_t)seg * 4;
-    make_plan(hist, n_out, LEVEL, &plan, s_scan, s_red, s_out);
-
-    int32_t* o = out + (int64_t)seg * out_stride;
-    if (LEVEL == 1 && blockIdx.x == 0)
-        for (int i = plan.need0 + threadIdx.x; i < n_out; i += kThreads) o[i] = -1;
-
-    // levels before this one must have left candidates for it
-    for (int l = 1; l < LEVEL; ++l)
-        if (plan.direct[l] || plan.need0 == 0) return;
-    if (plan.need0 == 0) return;
-
-    const bool more = !plan.direct[LEVEL];
-    if (more)
-        for (int i = threadIdx.x; i < kRadixBins; i += kThreads) hnext[i] = 0;
-    __syncthreads();
-
-    const uint32_t c = plan.c[LEVEL];
-    const uint32_t need_here = plan.need[LEVEL];
-    const int64_t nvalid = n_valid_positions(src, seg);
-    const int64_t n_items = LEVEL == 1 ? (src.ids ? src.n : nvalid) : (int64_t)plan.cnt_eq[LEVEL - 1];
-    const uint32_t* cand_in = LEVEL == 2 ? wk.cand1 + seg * wk.cand_stride : wk.cand2 + seg * wk.cand_stride;
-    uint32_t* cand_out = LEVEL == 1 ? wk.cand1 + seg * wk.cand_stride : wk.cand2 + seg * wk.cand_stride;
-
-    const int lane = threadIdx.x & 31;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int64_t base = (int64_t)blockIdx.x * kChunk; base < n_items; base += (int64_t)gridDim.x * kChunk) {
-        const int64_t end = min(base + kChunk, n_items);
-        for (int64_t it0 = base; it0 < end; it0 += kThreads) {
-            const int64_t it = it0 + threadIdx.x;
-            Elem e;
-            e.valid = false;
-            int64_t i = 0;
-            if (it < end) {
-                i = LEVEL == 1 ? it : (int64_t)cand_in[it];
-                e = load_elem(src, seg, i, nvalid);
-            }
-            const uint32_t d = e.valid ? digit(e.key, LEVEL) : 0u;
-            const bool eq = e.valid && d == c;
-            bool take = e.valid && d > c;
-            bool to_cand = false;
-            if (eq && LEVEL < 3) {
-                if (more) to_cand = true;   // resolved by the next digit
-                else take = true;           // exactly the missing number of them
-            }
-            // exact ties at the last level: the first `need_here` claimants win
-            if (LEVEL == 3) {
-                const uint32_t m = __ballot_sync(0xffffffffu, eq);
-                if (m) {
-                    const int leader = __ffs(m) - 1;
-                    uint32_t b0 = 0;
-                    if (lane == leader) b0 = atomicAdd(cnt + 3, (uint32_t)__popc(m));
-                    b0 = __shfl_sync(0xffffffffu, b0, leader);
-                    if (eq && b0 + __popc(m & lt_mask) < need_here) take = true;
-                }
-            }
-            if (LEVEL < 3) {
-                const uint32_t m = __ballot_sync(0xffffffffu, to_cand);
-                if (m) {
-                    const int leader = __ffs(m) - 1;
-                    uint32_t b0 = 0;
-                    if (lane == leader) b0 = atomicAdd(cnt + LEVEL, (uint32_t)__popc(m));
-                    b0 = __shfl_sync(0xffffffffu, b0, leader);
-                    if (to_cand) {
-                        cand_out[b0 + __popc(m & lt_mask)] = (uint32_t)i;
-                        atomicAdd(&hnext[digit(e.key, LEVEL + 1)], 1u);
-                    }
-                }
-            }
-            const uint32_t mt = __ballot_sync(0xffffffffu, take);
-            if (mt) {
-                const int leader = __ffs(mt) - 1;
-                uint32_t b0 = 0;
-                if (lane == leader) b0 = atomicAdd(cnt, (uint32_t)__popc(mt));
-                b0 = __shfl_sync(0xffffffffu, b0, leader);
-                if (take) o[b0 + __popc(mt & lt_mask)] = e.id;
-            }
+    if (threadIdx.x < 32) {
+        const uint32_t total = warp_sum_hist(h1);
+        const uint32_t need = total < (uint32_t)n_out ? total : (uint32_t)n_out;
+        uint2 t = make_uint2(0xFFFFFFFFu, 0u);
+        if (need > 0) t = warp_threshold(h1, need);
+        if (threadIdx.x == 0) {
+            s_plan[0] = t.x;
+            s_plan[1] = need;
+            s_plan[2] = need > 0 ? (h1[t.x] == need - t.y) : 1u;
         }
     }
-    if (LEVEL < 3 && more) {
+    for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads) h2[i] = 0;
+    __syncthreads();
+    const uint32_t c1 = s_plan[0], need0 = s_plan[1];
+    const bool take_eq = s_plan[2] != 0;
+    int32_t* o = out + (int64_t)seg * out_stride;
+    if (blockIdx.x == 0)
+        for (int i = need0 + threadIdx.x; i < n_out; i += kPassThreads) o[i] = -1;
+    if (need0 == 0) return;
+    const int64_t nvalid = n_valid_positions(src, seg);
+    const int64_t n_items = src.ids ? src.n : nvalid;
+    uint32_t* cand = wk.cand1 + seg * wk.cand_stride;
+    for (int64_t base = (int64_t)blockIdx.x * kPassChunk; base < n_items; base += (int64_t)gridDim.x * kPassChunk) {
+        const int64_t end = min(base + kPassChunk, n_items);
+        for (int64_t it0 = base; it0 < end; it0 += kPassThreads) {
+            const int64_t i = it0 + threadIdx.x;
+            Elem e;
+            e.valid = false;
+            if (i < end) e = load_elem(src, seg, i, nvalid);
+            const uint32_t d = e.valid ? digit(e.key, 1) : 0u;
+            const bool eq = e.valid && d == c1;
+            const bool take = e.valid && (d > c1 || (eq && take_eq));
+            const bool to_cand = eq && !take_eq;
+            const uint32_t cs = warp_claim(to_cand, cnt + 1);
+            if (to_cand) {
+                cand[cs] = (uint32_t)i;
+                atomicAdd(&h2[digit(e.key, 2)], 1u);
+            }
+            const uint32_t os = warp_claim(take, cnt);
+            if (take) o[os] = e.id;
+        }
+    }
+    if (take_eq) return;
+    __syncthreads();
+    uint32_t* gh2 = wk.hist + ((int64_t)seg * 3 + 1) * kRadixBins;
+    for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads)
+        if (h2[i]) atomicAdd(gh2 + i, h2[i]);
+}
+
+// Digits 2 and 3 of one segment's candidate list, one CTA.
+__global__ void __launch_bounds__(kFinThreads)
+k_sel_finish(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    __shared__ uint32_t h3[kRadixBins];
+    __shared__ uint32_t s_plan[6];
+    const int seg = blockIdx.x;
+    const uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
+    const uint32_t* h2 = h1 + kRadixBins;
+    uint32_t* cnt = wk.cnt + (int64_t)seg * 4;
+    for (int i = threadIdx.x; i < kRadixBins; i += kFinThreads) h3[i] = 0;
+    if (threadIdx.x < 32) {
+        const uint32_t total = warp_sum_hist(h1);
+        const uint32_t need = total < (uint32_t)n_out ? total : (uint32_t)n_out;
+        uint32_t run = 0, c2 = 0, need2 = 0, n_cand = 0;
+        if (need > 0) {
+            const uint2 t1 = warp_threshold(h1, need);
+            n_cand = h1[t1.x];
+            const uint32_t need1 = need - t1.y;
+            if (n_cand != need1) {                // level 1 left candidates
+                const uint2 t2 = warp_threshold(h2, need1);
+                c2 = t2.x;
+                need2 = need1 - t2.y;
+                run = 1;
+            }
+        }
+        if (threadIdx.x == 0) {
+            s_plan[0] = run;
+            s_plan[1] = c2;
+            s_plan[2] = need2;
+            s_plan[3] = n_cand;
+            s_plan[4] = run ? h2[c2] : 0;
+        }
+    }
+    __syncthreads();
+    if (!s_plan[0]) return;
+    const uint32_t c2 = s_plan[1], need2 = s_plan[2], n_cand = s_plan[3];
+    const bool take_eq2 = s_plan[4] == need2;
+    const uint32_t* cand = wk.cand1 + seg * wk.cand_stride;
+    uint32_t* cand2 = wk.cand2 + seg * wk.cand_stride;
+    int32_t* o = out + (int64_t)seg * out_stride;
+    const int64_t nvalid = n_valid_positions(src, seg);
+    // digit 2: select above c2, keep the digit-c2 candidates for digit 3
+    for (uint32_t it0 = 0; it0 < n_cand; it0 += kFinThreads) {
+        const uint32_t it = it0 + threadIdx.x;
+        Elem e;
+        e.valid = false;
+        uint32_t ci = 0;
+        if (it < n_cand) {
+            ci = cand[it];
+            e = load_elem(src, seg, ci, nvalid);
+        }
+        const uint32_t d = e.valid ? digit(e.key, 2) : 0u;
+        const bool eq = e.valid && d == c2;
+        const bool take = e.valid && (d > c2 || (eq && take_eq2));
+        const bool keep = eq && !take_eq2;
+        const uint32_t ks = warp_claim(keep, cnt + 2);
+        if (keep) {
+            cand2[ks] = ci;
+            atomicAdd(&h3[digit(e.key, 3)], 1u);
+        }
+        const uint32_t os = warp_claim(take, cnt);
+        if (take) o[os] = e.id;
+    }
+    if (take_eq2) return;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const uint2 t3 = warp_threshold(h3, need2);
+        if (threadIdx.x == 0) {
+            s_plan[1] = t3.x;
+            s_plan[2] = need2 - t3.y;
+            s_plan[3] = h2[c2];
+        }
+    }
+    __syncthreads();
+    const uint32_t c3 = s_plan[1], need3 = s_plan[2], n2 = s_plan[3];
+    for (uint32_t it0 = 0; it0 < n2; it0 += kFinThreads) {
+        const uint32_t it = it0 + threadIdx.x;
+        Elem e;
+        e.valid = false;
+        if (it < n2) e = load_elem(src, seg, cand2[it], nvalid);
+        const uint32_t d = e.valid ? digit(e.key, 3) : 0u;
+        const bool eq = e.valid && d == c3;
+        const uint32_t tie = warp_claim(eq, cnt + 3);
+        const bool take = e.valid && (d > c3 || (eq && tie < need3));
+        const uint32_t os = warp_claim(take, cnt);
+        if (take) o[os] = e.id;
+    }
+}
+
+// ---------------------------------------------------------------- small segments
+// Whole selection of one segment of at most kSmallMax elements in one CTA.
+__global__ void __launch_bounds__(kFinThreads)
+k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    extern __shared__ uint32_t sm[];
+    uint32_t* keys = sm;                        // [n]; 0 marks an invalid element
+    uint32_t* hist = sm + src.n;                // [kRadixBins]
+    __shared__ uint32_t s_plan[3];
+    __shared__ uint32_t s_cnt[2];
+    const int seg = blockIdx.x;
+    const int n = (int)src.n;
+    const int64_t nvalid = n_valid_positions(src, seg);
+    int32_t* o = out + (int64_t)seg * out_stride;
+    for (int i = threadIdx.x; i < kRadixBins; i += kFinThreads) hist[i] = 0;
+    if (threadIdx.x < 2) s_cnt[threadIdx.x] = 0;
+    __syncthreads();
+    uint32_t mine = 0;
+    for (int i = threadIdx.x; i < n; i += kFinThreads) {
+        Elem e = load_elem(src, seg, i, nvalid);
+        // the ordered key of a finite float is never 0
+        keys[i] = e.valid ? e.key : 0u;
+        if (e.valid) { atomicAdd(&hist[digit(e.key, 1)], 1u); ++mine; }
+    }
+    mine = __reduce_add_sync(0xffffffffu, mine);
+    if ((threadIdx.x & 31) == 0 && mine) atomicAdd(&s_cnt[1], mine);
+    __syncthreads();
+    const uint32_t total = s_cnt[1];
+    const uint32_t need0 = total < (uint32_t)n_out ? total : (uint32_t)n_out;
+    for (int i = need0 + threadIdx.x; i < n_out; i += kFinThreads) o[i] = -1;
+    if (need0 == 0) return;
+    // digits fixed so far, as (prefix, mask) over the key
+    uint32_t prefix = 0, mask = 0, need = need0;
+    for (int level = 1; level <= 3; ++level) {
+        if (level > 1) {
+            __syncthreads();
+            for (int i = threadIdx.x; i < kRadixBins; i += kFinThreads) hist[i] = 0;
+            __syncthreads();
+            for (int i = threadIdx.x; i < n; i += kFinThreads) {
+                const uint32_t k = keys[i];
+                if (k && (k & mask) == prefix) atomicAdd(&hist[digit(k, level)], 1u);
+            }
+        }
         __syncthreads();
-        uint32_t* gh = wk.hist + ((int64_t)seg * 3 + LEVEL) * kRadixBins;
-        for (int i = threadIdx.x; i < kRadixBins; i += kThreads)
-            if (hnext[i]) atomicAdd(gh + i, hnext[i]);
+        if (threadIdx.x < 32) {
+            const uint2 t = warp_threshold(hist, need);
+            if (threadIdx.x == 0) {
+                s_plan[0] = t.x;
+                s_plan[1] = t.y;
+                s_plan[2] = hist[t.x];
+            }
+        }
+        __syncthreads();
+        const uint32_t c = s_plan[0], above = s_plan[1], eqn = s_plan[2];
+        const uint32_t shift = level == 1 ? 21 : level == 2 ? 10 : 0;
+        const uint32_t dmask = level == 3 ? 0x3FFu : 0x7FFu;
+        const bool all_eq = eqn == need - above;
+        // select the elements of the current prefix whose digit is above c
+        // (and those equal to c when exactly the missing number of them exist)
+        for (int i0 = 0; i0 < n; i0 += kFinThreads) {
+            const int i = i0 + threadIdx.x;
+            const uint32_t k = i < n ? keys[i] : 0u;
+            const bool in = k && (k & mask) == prefix;
+            const uint32_t d = (k >> shift) & dmask;
+            const bool take = in && (d > c || (d == c && all_eq));
+            const uint32_t os = warp_claim(take, &s_cnt[0]);
+            if (take) o[os] = src.ids ? src.ids[seg * src.ids_stride + i] : i;
+        }
+        if (all_eq) break;
+        need -= above;
+        prefix |= c << shift;
+        mask |= dmask << shift;
+        if (level == 3) {
+            // exact ties of the full key: the first `need` claimants win
+            __syncthreads();
+            if (threadIdx.x == 0) s_cnt[1] = 0;
+            __syncthreads();
+            for (int i0 = 0; i0 < n; i0 += kFinThreads) {
+                const int i = i0 + threadIdx.x;
+                const uint32_t k = i < n ? keys[i] : 0u;
+                const bool eq = k && k == prefix;
+                const uint32_t ts = warp_claim(eq, &s_cnt[1]);
+                const bool take = eq && ts < need;
+                const uint32_t os = warp_claim(take, &s_cnt[0]);
+                if (take) o[os] = src.ids ? src.ids[seg * src.ids_stride + i] : i;
+            }
+        }
     }
 }
 
@@ -268,18 +374,28 @@ k_sel_pass(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_t
 cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_out, int32_t* out,
                           int64_t out_stride, cudaStream_t st, bool hist_ready) {
     cudaError_t e;
+    if (src.n <= kSmallMax) {
+        const size_t smem = sizeof(uint32_t) * ((size_t)src.n + kRadixBins);
+        if (smem > 48 * 1024) {
+            e = cudaFuncSetAttribute(k_sel_small, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        k_sel_small<<<nseg, kFinThreads, smem, st>>>(src, n_out, out, out_stride);
+        return cudaGetLastError();
+    }
+    // hist_ready: every level of the histograms was zeroed before the scoring
+    // kernel filled level 1
     if (!hist_ready) {
         e = cudaMemsetAsync(wk.hist, 0, sizeof(uint32_t) * (size_t)nseg * 3 * kRadixBins, st);
         if (e != cudaSuccess) return e;
     }
     e = cudaMemsetAsync(wk.cnt, 0, sizeof(uint32_t) * (size_t)nseg * 4, st);
     if (e != cudaSuccess) return e;
-    const unsigned chunks = (unsigned)((src.n + kChunk - 1) / kChunk);
+    const unsigned chunks = (unsigned)((src.n + kPassChunk - 1) / kPassChunk);
     dim3 grid(chunks ? chunks : 1, (unsigned)nseg);
-    if (!hist_ready) k_sel_hist<<<grid, kThreads, 0, st>>>(src, wk);
-    k_sel_pass<1><<<grid, kThreads, 0, st>>>(src, wk, n_out, out, out_stride);
-    k_sel_pass<2><<<grid, kThreads, 0, st>>>(src, wk, n_out, out, out_stride);
-    k_sel_pass<3><<<grid, kThreads, 0, st>>>(src, wk, n_out, out, out_stride);
+    if (!hist_ready) k_sel_hist<<<grid, kPassThreads, 0, st>>>(src, wk);
+    k_sel_pass1<<<grid, kPassThreads, 0, st>>>(src, wk, n_out, out, out_stride);
+    k_sel_finish<<<nseg, kFinThreads, 0, st>>>(src, wk, n_out, out, out_stride);
     return cudaGetLastError();
 }
 
