@@ -13,6 +13,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kMaxPool = 16384;  // candidate pool bound, tldrocket.com page, paragraph 3
+constexpr int64_t kSmallSelect = 16384;  // selections over at most this many elements run in one CTA
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -70,10 +71,12 @@ int num_sms() {
 }
 
 // Workspace layout (byte offsets, each section 256-byte aligned):
-//   status word | full-layer scores | radix histograms | radix counters |
-//   candidates 1 | candidates 2 | pool scores | attention partials
+//   status word | full-layer scores | radix histograms | scratch histogram |
+//   radix counters | candidates 1 | candidates 2 | pool scores | attention partials
+// The radix histograms and counters are zero between calls: the workspace
+// starts zeroed and every large selection clears what it used.
 struct Layout {
-    size_t status, scores, hist, cnt, cand1, cand2, pscores, part_o, part_ml, total;
+    size_t status, scores, hist, hist_scratch, cnt, cand1, cand2, pscores, part_o, part_ml, total;
     int64_t nseg, cap, cand_stride;
     int nchunk;
 };
@@ -89,9 +92,10 @@ bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int w
     L->status = off; off = align_up(off + 16);
     L->scores = off; off = align_up(off + sizeof(float) * (size_t)(L->nseg * L->cap));
     L->hist = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 3 * kRadixBins);
+    L->hist_scratch = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * kRadixBins);
     L->cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 4);
-    L->cand1 = off; off = align_up(off + sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
-    L->cand2 = off; off = align_up(off + sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
+    L->cand1 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
+    L->cand2 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->pscores = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * pool_k);
     L->part_o = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * c->dim);
     L->part_ml = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * 2);
@@ -205,10 +209,11 @@ csa2_status csa2_index_scores(const csa2_cache* cache, const void* q_idx, csa2_d
     s = check_ws(cache, T, 1, 1, 1, 0, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
     bool fused;
-    // the histogram section is scratch here (the same kernel as in csa2_index_full)
+    // the same kernel as in csa2_index_full; its histogram goes to a scratch
+    // section that no selection reads
     return launch_scores(cache, q_idx, q_dtype, head_w, T, H_I, scores ? scores : at<float>(ws, L.scores),
-                         at<uint32_t>(ws, L.hist), at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream),
-                         &fused);
+                         L.cap > kSmallSelect ? at<uint32_t>(ws, L.hist_scratch) : nullptr,
+                         at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream), &fused);
 }
 
 csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
@@ -221,9 +226,9 @@ csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dty
     s = check_ws(cache, T, 1, pool_k, top_k, 0, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint32_t* hist = at<uint32_t>(ws, L.hist);
-    if (cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)L.nseg * 3 * kRadixBins, st) != cudaSuccess)
-        return CSA2_ERR_CUDA;
+    // a large selection takes its level-1 histogram from the scoring kernel
+    // (the histograms are zero on entry); a small one builds its own
+    uint32_t* hist = L.cap > kSmallSelect ? at<uint32_t>(ws, L.hist) : nullptr;
     // every visible position scored into the workspace
     float* scores = at<float>(ws, L.scores);
     bool fused = false;

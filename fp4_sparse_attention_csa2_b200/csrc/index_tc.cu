@@ -1,27 +1,32 @@
-// Indexer scoring on the 5th-generation tensor cores (tcgen05) for E4M3 index
-// keys:  s_t = sum_h w_h * max(0, q_h . k_t)  for every visible position.
+// Indexer scoring on the 5th-generation tensor cores (tcgen05, kind::f8f6f4)
+// for E4M3 index keys:  s_t = sum_h w_h * max(0, q_h . k_t)  for every
+// visible position.
 //
 // Role of the indexer: tldrocket.com, "DeepSeek AI Released DeepSeek-V4.1-Flash
 // with 1M Context, FP4 KV Cache, and Cross-Layer Attention Reuse", paragraph 3
 // (a Full layer scores the whole context into a candidate pool of <= 16,384
 // positions); hackernews.kjhq.dev post 49735410, key point 3.
 //
-// The key stream is the HBM-bound hot loop (64 B per position, 2*H_I*64 flop
-// per position per query token).  Per 128-position tile:
-//   producer warp   : 1-D bulk copies (TMA engine, no multicast) of the raw
-//                     E4M3 keys, 64 positions (one page run) per copy, into an
-//                     8-stage ring;
-//   converter warps : E4M3 -> fp16 (exact) into a 128-byte-swizzled K-major
-//                     operand tile;
-//   MMA thread      : 4 x tcgen05.mma kind::f16 (M=128 positions, N = T*H_I
-//                     query heads padded to 16, K=16) into a double-buffered
-//                     TMEM accumulator;
-//   epilogue warps  : tcgen05.ld of each position's row, ReLU + head-weighted
-//                     sum, fp32 score store, and the level-1 radix histogram
-//                     of the top-K select in shared memory.
-// Queries go in as fp16 scaled by a power of two per (token, head) so every
-// bf16 query value down to 2^-32 of the row maximum is exact; the scale is
-// folded back into the head weight (exact, a power of two).
+// The key stream is the HBM-bound hot loop (64 B per position).  The E4M3 keys
+// are the MMA's A operand exactly as stored: TMA tensor loads (64 positions =
+// one page run per box, 64-byte swizzle, no multicast) fill a ring of
+// 128-position tiles that tcgen05.mma reads directly.  The bf16 queries become
+// four 8-bit operands whose sum is the query exactly: per (token, head) row the
+// values are scaled by a power of two so the row maximum lies in [128, 256),
+// then q = t1 + t2 + t3 + t4 with t1 = E4M3(q), t2..t4 = E5M2 of the running
+// remainder (round to nearest).  A bf16 value has 8 significant bits; E4M3
+// takes 4 and each E5M2 term 3, so the remainder is 0 for every value at or
+// above 2^-16 of the row maximum (E5M2 reaches down to 2^-16 after scaling).
+// Eight MMAs per tile (4 terms x K=2x32) accumulate q.k in fp32.
+//
+//   producer warp  : TMA loads into the ring (bounded mbarrier waits)
+//   MMA warp       : tcgen05.mma, commits that free ring stages and fill the
+//                    double-buffered TMEM accumulator
+//   epilogue warps : stage the query terms when the sequence changes; per tile
+//                    tcgen05.ld of each position's row, ReLU + head-weighted
+//                    sum, fp32 score store, level-1 radix histogram in smem.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -32,13 +37,12 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kItemTiles = 4;
-constexpr int kRaw = 6;
-constexpr int kA = 2;
-constexpr int kRawBytes = kTile * 64;   // E4M3 keys of one tile
-constexpr int kABytes = kTile * 128;    // 128 rows x 64 fp16
-constexpr int kThreads = 320;
-constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpConv0 = 2, kWarpEpi0 = 6;
-constexpr uint32_t kDrainLimit = 65536;   // tries of the drain waits (x kSuspendNs)
+constexpr int kStages = 8;
+constexpr int kStageBytes = kTile * 64;   // two 64-row boxes of E4M3 keys
+constexpr int kTerms = 4;
+constexpr int kThreads = 192;
+constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;
+constexpr uint32_t kDrainLimit = 65536;
 
 struct Params {
     DevCache c;
@@ -46,11 +50,11 @@ struct Params {
     const float* hw;         // [B][T][H_I]
     int T, H_I, HP, NP;      // HP: H_I rounded up to 16; NP = T * HP (MMA N)
     float* scores;           // [(b*T + j) * cap + t]
-    uint32_t* hist;          // [(b*T + j)][3][kRadixBins], level-1 part accumulated; nullable
+    uint32_t* hist;          // [(b*T + j)][3][kRadixBins]; level 1 accumulated here; nullable
     uint32_t* status;
     int64_t items_per_seq, total_items;
     uint32_t tmem_cols;
-    uint32_t off_b, off_raw, off_hist, off_wq, off_bar;
+    uint32_t off_b, off_hist, off_wq, off_bar;
 };
 
 struct Item {
@@ -70,38 +74,41 @@ __device__ __forceinline__ bool get_item(const Params& p, int64_t item, Item& it
     it.b = b;
     it.t0 = tile0 * kTile;
     it.L = L;
-    it.ntiles = (int)(tiles - tile0 < kItemTiles ? tiles - tile0 : (int64_t)kItemTiles);
+    it.ntiles = (int)(tiles - tile0 < kItemTiles ? tiles - tile0 : kItemTiles);
     return true;
 }
 
 struct Bars {
-    uint64_t raw_full[kRaw], raw_empty[kRaw];
-    uint64_t a_full[kA], a_empty[kA];
+    uint64_t full[kStages], empty[kStages];
     uint64_t acc_full[2], acc_empty[2];
-    uint64_t b_free[2], wq_ready[2], wq_free[2];
+    uint64_t b_ready[2], b_free[2];
     uint64_t hist_done, hist_clear;
     uint64_t drain;
     uint32_t tmem_base;
 };
 
-__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t two_bytes) {
-    uint32_t r;
-    const uint16_t in = (uint16_t)two_bytes;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(in));
-    return r;
+__device__ __forceinline__ float e4m3_round(float x, uint8_t* code) {
+    const uint16_t c = cvt_e4m3x2(0.0f, x);
+    *code = (uint8_t)(c & 0xFF);
+    return e4m3_to_float(*code);
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-    __half2 h = __floats2half2_rn(lo, hi);
-    uint32_t r;
-    memcpy(&r, &h, 4);
-    return r;
+__device__ __forceinline__ float e5m2_round(float x, uint8_t* code) {
+    uint16_t c;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(c) : "f"(0.0f), "f"(x));
+    *code = (uint8_t)(c & 0xFF);
+    uint32_t h;
+    const uint16_t in = c & 0xFF;
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(in));
+    return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFF)));
 }
 
-// Query operand of one sequence: NP rows (column c = token j * HP + head h) of
-// 64 fp16 values, scaled by 2^e per row, and the folded weights w * 2^-e.
+// The four 8-bit query operands of one sequence, NP rows each (row c = token
+// j * HP + head h; padding rows are zero), plus the folded weights
+// w * 2^-e.  4 threads per row, 16 values each.
 __device__ void prepare_queries(const Params& p, int b, uint8_t* bq, float* wq, int tid) {
     const int row_in_pass = tid >> 2, quarter = tid & 3;
+    const int term_bytes = p.NP * 64;
     for (int r0 = 0; r0 < p.NP; r0 += 32) {
         const int c = r0 + row_in_pass;
         const int j = c / p.HP, h = c - j * p.HP;
@@ -129,51 +136,62 @@ __device__ void prepare_queries(const Params& p, int b, uint8_t* bq, float* wq, 
         int e = 0;
         if (m > 0.0f) {
             const int E = (int)((__float_as_uint(m) >> 23) & 0xFF) - 127;
-            e = 14 - E;
+            e = 7 - E;
             e = e < -100 ? -100 : (e > 100 ? 100 : e);
         }
         const float up = __uint_as_float((uint32_t)(127 + e) << 23);
         const float down = __uint_as_float((uint32_t)(127 - e) << 23);
         if (c < p.NP) {
-            uint32_t hv[8];
+            uint8_t t[kTerms][16];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) hv[k] = pack_half2(v[2 * k] * up, v[2 * k + 1] * up);
-            *reinterpret_cast<uint4*>(bq + tc::sw128_offset(c, 2 * quarter)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            *reinterpret_cast<uint4*>(bq + tc::sw128_offset(c, 2 * quarter + 1)) =
-                make_uint4(hv[4], hv[5], hv[6], hv[7]);
+            for (int k = 0; k < 16; ++k) {
+                float r = v[k] * up;                       // exact: a power-of-two scale
+                r -= e4m3_round(r, &t[0][k]);              // exact: both are fp32 values
+                r -= e5m2_round(r, &t[1][k]);
+                r -= e5m2_round(r, &t[2][k]);
+                e5m2_round(r, &t[3][k]);
+            }
+#pragma unroll
+            for (int u = 0; u < kTerms; ++u) {
+                uint32_t wds[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    wds[k] = (uint32_t)t[u][4 * k] | ((uint32_t)t[u][4 * k + 1] << 8) |
+                             ((uint32_t)t[u][4 * k + 2] << 16) | ((uint32_t)t[u][4 * k + 3] << 24);
+                *reinterpret_cast<uint4*>(bq + u * term_bytes + tc::sw64_offset(c, quarter)) =
+                    make_uint4(wds[0], wds[1], wds[2], wds[3]);
+            }
             if (quarter == 0) wq[c] = real ? __ldg(p.hw + ((int64_t)b * p.T + j) * p.H_I + h) * down : 0.0f;
         }
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2) k_score_full_tc(const Params p) {
+__global__ void __launch_bounds__(kThreads, 2)
+k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    // operand tiles need 1024-byte alignment for the 128-byte swizzle
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem;
+    uint8_t* sRing = smem;
     uint8_t* sB = smem + p.off_b;
-    uint8_t* sRaw = smem + p.off_raw;
     uint32_t* sHist = reinterpret_cast<uint32_t*>(smem + p.off_hist);
     float* sWq = reinterpret_cast<float*>(smem + p.off_wq);
     Bars* bars = reinterpret_cast<Bars*>(smem + p.off_bar);
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bq_bytes = kTerms * p.NP * 64;
 
     for (int i = threadIdx.x; i < p.T * kRadixBins; i += kThreads) sHist[i] = 0;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kRaw; ++i) { tc::mbar_init(&bars->raw_full[i], 1); tc::mbar_init(&bars->raw_empty[i], 128); }
-        for (int i = 0; i < kA; ++i) { tc::mbar_init(&bars->a_full[i], 128); tc::mbar_init(&bars->a_empty[i], 1); }
+        for (int i = 0; i < kStages; ++i) { tc::mbar_init(&bars->full[i], 1); tc::mbar_init(&bars->empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars->acc_full[i], 1);
             tc::mbar_init(&bars->acc_empty[i], 128);
+            tc::mbar_init(&bars->b_ready[i], 128);
             tc::mbar_init(&bars->b_free[i], 1);
-            tc::mbar_init(&bars->wq_ready[i], 128);
-            tc::mbar_init(&bars->wq_free[i], 128);
         }
         tc::mbar_init(&bars->hist_done, 128);
         tc::mbar_init(&bars->hist_clear, 128);
         tc::mbar_init(&bars->drain, 1);
         tc::fence_mbar_init();
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
     }
     if (warp == kWarpMma) tc::tmem_alloc(&bars->tmem_base, p.tmem_cols);
     tc::fence_before_sync();
@@ -189,43 +207,42 @@ __global__ void __launch_bounds__(kThreads, 2) k_score_full_tc(const Params p) {
                 Item it;
                 if (!get_item(p, item, it)) continue;
                 for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
-                    const int s = g % kRaw;
-                    if (!tc::mbar_wait(&bars->raw_empty[s], ((g / kRaw) & 1) ^ 1)) { ok = false; break; }
+                    const int s = g % kStages;
+                    if (!tc::mbar_wait(&bars->empty[s], ((g / kStages) & 1) ^ 1)) { ok = false; break; }
                     const int64_t t0 = it.t0 + (int64_t)tl * kTile;
                     int64_t slot[2] = {-1, -1};
-                    int cnt[2] = {0, 0};
                     uint32_t bytes = 0;
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
                         const int64_t p0 = t0 + 64 * r;
-                        { const int64_t rem = it.L - p0; cnt[r] = rem <= 0 ? 0 : (rem > 64 ? 64 : (int)rem); }
-                        if (cnt[r] > 0) {
+                        if (p0 < it.L) {
                             slot[r] = slot_of(p.c, it.b, p0);
                             if (slot[r] < 0) flag(p.status, kStatusBounds);
-                            else bytes += (uint32_t)cnt[r] * 64u;
+                            else bytes += 64u * 64u;
                         }
                     }
                     if (bytes == 0) {
-                        tc::mbar_arrive(&bars->raw_full[s]);
+                        tc::mbar_arrive(&bars->full[s]);
                     } else {
-                        tc::mbar_arrive_expect_tx(&bars->raw_full[s], bytes);
+                        tc::mbar_arrive_expect_tx(&bars->full[s], bytes);
 #pragma unroll
                         for (int r = 0; r < 2; ++r)
-                            if (cnt[r] > 0 && slot[r] >= 0)
-                                tc::bulk_g2s(sRaw + s * kRawBytes + r * 4096,
-                                             static_cast<const uint8_t*>(p.c.keys) + slot[r] * 64,
-                                             (uint32_t)cnt[r] * 64u, &bars->raw_full[s]);
+                            if (slot[r] >= 0)
+                                tc::tma_load_2d(sRing + s * kStageBytes + r * 4096, &tmap, 0, (int32_t)slot[r],
+                                                &bars->full[s]);
                     }
                 }
             }
             if (!ok) flag(p.status, kStatusTimeout);
-            // copies still in flight must land before the CTA's shared memory goes away
-            for (uint32_t k = g > (uint32_t)kRaw ? g - kRaw : 0; k < g; ++k)
-                tc::mbar_wait(&bars->raw_full[k % kRaw], (k / kRaw) & 1, kDrainLimit);
+            // loads still in flight must land before the CTA's shared memory goes away
+            for (uint32_t k = g > (uint32_t)kStages ? g - kStages : 0; k < g; ++k)
+                tc::mbar_wait(&bars->full[k % kStages], (k / kStages) & 1, kDrainLimit);
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = tc::idesc_f16_f32(kTile, p.NP);
+            uint32_t idesc[kTerms];
+#pragma unroll
+            for (int u = 0; u < kTerms; ++u) idesc[u] = tc::idesc_f8_f32(kTile, p.NP, 0u, u == 0 ? 0u : 1u);
             uint32_t g = 0, n = 0;
             int cur_b = -1;
             bool ok = true;
@@ -233,22 +250,25 @@ __global__ void __launch_bounds__(kThreads, 2) k_score_full_tc(const Params p) {
                 Item it;
                 if (!get_item(p, item, it)) continue;
                 if (it.b != cur_b) {
-                    // the query buffer of the previous sequence is free once its MMAs are done
                     if (cur_b >= 0) { tc::mma_commit(&bars->b_free[n & 1]); ++n; }
                     cur_b = it.b;
+                    if (!tc::mbar_wait(&bars->b_ready[n & 1], (n >> 1) & 1)) { ok = false; break; }
                 }
-                const uint32_t bq = tc::smem_u32(sB + (n & 1) * (p.NP * 128));
+                const uint32_t bq = tc::smem_u32(sB + (n & 1) * bq_bytes);
                 for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
-                    const int a = g % kA, acc = g & 1;
-                    if (!tc::mbar_wait(&bars->a_full[a], (g / kA) & 1) ||
+                    const int s = g % kStages, acc = g & 1;
+                    if (!tc::mbar_wait(&bars->full[s], (g / kStages) & 1) ||
                         !tc::mbar_wait(&bars->acc_empty[acc], ((g >> 1) & 1) ^ 1)) { ok = false; break; }
                     tc::fence_after_sync();
-                    const uint32_t aa = tc::smem_u32(sA + a * kABytes);
+                    const uint32_t aa = tc::smem_u32(sRing + s * kStageBytes);
                     const uint32_t d = tmem + (uint32_t)(acc * p.NP);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        tc::mma_f16(d, tc::desc_sw128(aa + 32 * k), tc::desc_sw128(bq + 32 * k), idesc, k > 0);
-                    tc::mma_commit(&bars->a_empty[a]);
+                    for (int u = 0; u < kTerms; ++u)
+#pragma unroll
+                        for (int k = 0; k < 2; ++k)
+                            tc::mma_f8(d, tc::desc_sw64(aa + 32 * k),
+                                       tc::desc_sw64(bq + u * (p.NP * 64) + 32 * k), idesc[u], (u | k) != 0);
+                    tc::mma_commit(&bars->empty[s]);
                     tc::mma_commit(&bars->acc_full[acc]);
                 }
             }
@@ -256,50 +276,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_score_full_tc(const Params p) {
             tc::mma_commit(&bars->drain);
             tc::mbar_wait(&bars->drain, 0, kDrainLimit);
         }
-    } else if (warp < kWarpEpi0) {
-        // converters: 128 threads
-        const int tid = threadIdx.x - kWarpConv0 * 32;
-        uint32_t g = 0, n = 0;
-        int cur_b = -1;
-        bool ok = true;
-        for (int64_t item = blockIdx.x; item < p.total_items && ok; item += gridDim.x) {
-            Item it;
-            if (!get_item(p, item, it)) continue;
-            if (it.b != cur_b) {
-                // a new sequence: stage its queries in the other buffer
-                if (cur_b >= 0) ++n;
-                cur_b = it.b;
-                const int qb = n & 1;
-                if (!tc::mbar_wait(&bars->b_free[qb], ((n >> 1) & 1) ^ 1) ||
-                    !tc::mbar_wait(&bars->wq_free[qb], ((n >> 1) & 1) ^ 1)) { ok = false; break; }
-                prepare_queries(p, it.b, sB + qb * (p.NP * 128), sWq + qb * p.NP, tid);
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(&bars->wq_ready[qb]);
-            }
-            for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
-                const int s = g % kRaw, a = g % kA;
-                if (!tc::mbar_wait(&bars->raw_full[s], (g / kRaw) & 1) ||
-                    !tc::mbar_wait(&bars->a_empty[a], ((g / kA) & 1) ^ 1)) { ok = false; break; }
-                const uint8_t* rs = sRaw + s * kRawBytes;
-                uint8_t* as = sA + a * kABytes;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int cidx = k * 128 + tid;            // 16-byte chunk of the raw tile
-                    const int row = cidx >> 2, quarter = cidx & 3;
-                    const uint4 v = *reinterpret_cast<const uint4*>(rs + cidx * 16);
-                    const uint4 lo = make_uint4(cvt_e4m3x2_f16x2(v.x), cvt_e4m3x2_f16x2(v.x >> 16),
-                                                cvt_e4m3x2_f16x2(v.y), cvt_e4m3x2_f16x2(v.y >> 16));
-                    const uint4 hi = make_uint4(cvt_e4m3x2_f16x2(v.z), cvt_e4m3x2_f16x2(v.z >> 16),
-                                                cvt_e4m3x2_f16x2(v.w), cvt_e4m3x2_f16x2(v.w >> 16));
-                    *reinterpret_cast<uint4*>(as + tc::sw128_offset(row, 2 * quarter)) = lo;
-                    *reinterpret_cast<uint4*>(as + tc::sw128_offset(row, 2 * quarter + 1)) = hi;
-                }
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(&bars->a_full[a]);
-                tc::mbar_arrive(&bars->raw_empty[s]);
-            }
-        }
-        if (!ok) flag(p.status, kStatusTimeout);
     } else {
         // epilogue: 128 threads, thread = TMEM lane = position in the tile
         const int tid = threadIdx.x - kWarpEpi0 * 32;
@@ -310,8 +286,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_score_full_tc(const Params p) {
         int cur_b = -1;
         bool ok = true;
         // Move the shared histogram of sequence b into the global one.  The
-        // 128 epilogue threads meet on two mbarriers (bounded waits, so a
-        // thread that gave up earlier cannot hang the others).
+        // 128 epilogue threads meet on two mbarriers (bounded waits).
         auto flush = [&](int b) -> bool {
             tc::mbar_arrive(&bars->hist_done);
             if (!tc::mbar_wait(&bars->hist_done, nflush & 1)) return false;
@@ -341,12 +316,19 @@ __global__ void __launch_bounds__(kThreads, 2) k_score_full_tc(const Params p) {
             if (it.b != cur_b) {
                 if (cur_b >= 0) {
                     if (!flush(cur_b)) { ok = false; break; }
-                    tc::mbar_arrive(&bars->wq_free[n & 1]);
                     ++n;
                 }
                 cur_b = it.b;
-                if (!warp_wait(&bars->wq_ready[n & 1], (n >> 1) & 1)) { ok = false; break; }
-                wq = sWq + (n & 1) * p.NP;
+                // stage this sequence's query operands once the MMAs of the
+                // sequence that used the buffer before are done
+                const int qb = n & 1;
+                if (!tc::mbar_wait(&bars->b_free[qb], ((n >> 1) & 1) ^ 1)) { ok = false; break; }
+                prepare_queries(p, it.b, sB + qb * bq_bytes, sWq + qb * p.NP, tid);
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(&bars->b_ready[qb]);
+                // the same barrier publishes the weights to the other epilogue threads
+                if (!warp_wait(&bars->b_ready[qb], (n >> 1) & 1)) { ok = false; break; }
+                wq = sWq + qb * p.NP;
             }
             for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                 const int acc = g & 1;
@@ -395,20 +377,49 @@ __global__ void __launch_bounds__(kThreads, 2) k_score_full_tc(const Params p) {
     }
 }
 
-}  // namespace
+struct SmemPlan {
+    uint32_t off_b, off_hist, off_wq, off_bar, total;
+};
 
-namespace {
+SmemPlan smem_plan(int T, int NP) {
+    SmemPlan s;
+    uint32_t off = kStages * kStageBytes;
+    s.off_b = off;
+    off += 2 * kTerms * NP * 64;
+    s.off_hist = off;
+    off += T * kRadixBins * 4;
+    s.off_wq = off;
+    off += 2 * NP * 4;
+    off = (off + 15) / 16 * 16;
+    s.off_bar = off;
+    off += sizeof(Bars);
+    s.total = off + 1024;  // room to align the base to 1024 B
+    return s;
+}
 
-size_t smem_bytes(int T, int NP) {
-    return (size_t)kA * kABytes + 2 * (size_t)NP * 128 + (size_t)kRaw * kRawBytes + (size_t)T * kRadixBins * 4 +
-           2 * (size_t)NP * 4 + sizeof(Bars) + 16 + 1024;
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+    // the driver entry point, resolved through the runtime (no link-time driver dependency)
+    static EncodeTiled fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (EncodeTiled) nullptr;
+        return reinterpret_cast<EncodeTiled>(f);
+    }();
+    return fn;
 }
 
 }  // namespace
 
 bool score_full_tc_supported(const DevCache& c, int T, int H_I) {
     const int HP = (H_I + 15) / 16 * 16;
-    return c.key_dtype == 2 && c.idx_dim == 64 && T * HP <= 256 && smem_bytes(T, T * HP) <= 227 * 1024;
+    return c.key_dtype == 2 && c.idx_dim == 64 && T * HP <= 256 && smem_plan(T, T * HP).total <= 227 * 1024 &&
+           c.n_slots < ((int64_t)1 << 31) && encode_fn() != nullptr;
 }
 
 cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* hw, int T, int H_I, float* scores,
@@ -430,25 +441,31 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
     uint32_t cols = 32;
     while (cols < (uint32_t)(2 * p.NP)) cols <<= 1;
     p.tmem_cols = cols;
-    uint32_t off = kA * kABytes;
-    p.off_b = off;
-    off += 2 * p.NP * 128;
-    p.off_raw = off;
-    off += kRaw * kRawBytes;
-    p.off_hist = off;
-    off += T * kRadixBins * 4;
-    p.off_wq = off;
-    off += 2 * p.NP * 4;
-    off = (off + 15) / 16 * 16;
-    p.off_bar = off;
-    off += sizeof(Bars);
-    const size_t smem = off + 1024;  // room to align the base to 1024 B
-    cudaError_t e = cudaFuncSetAttribute(k_score_full_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const SmemPlan sp = smem_plan(T, p.NP);
+    p.off_b = sp.off_b;
+    p.off_hist = sp.off_hist;
+    p.off_wq = sp.off_wq;
+    p.off_bar = sp.off_bar;
+
+    // keys as a 2-D byte tensor [n_slots][64]: 64-row boxes, 64-byte swizzle
+    CUtensorMap tmap;
+    const cuuint64_t gdim[2] = {64, (cuuint64_t)c.n_slots};
+    const cuuint64_t gstride[1] = {64};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estride[2] = {1, 1};
+    EncodeTiled enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.keys, gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+
+    cudaError_t e = cudaFuncSetAttribute(k_score_full_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
     if (e != cudaSuccess) return e;
     int64_t grid = 2 * (int64_t)num_sms;   // two CTAs per SM
     if (grid > p.total_items) grid = p.total_items;
     if (grid < 1) grid = 1;
-    k_score_full_tc<<<(unsigned)grid, kThreads, smem, st>>>(p);
+    k_score_full_tc<<<(unsigned)grid, kThreads, sp.total, st>>>(tmap, p);
     return cudaGetLastError();
 }
 

@@ -65,6 +65,15 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                  : "memory");
 }
 
+// 2-D tensor-map tile load (TMA, no multicast) into this CTA's shared memory;
+// x is the innermost coordinate (in elements), y the row.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int32_t x, int32_t y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -87,6 +96,17 @@ __device__ __forceinline__ void fence_before_sync() {
 
 __device__ __forceinline__ void fence_after_sync() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (8-bit A and B), one thread.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, kind::f16, issued by one thread.
@@ -132,6 +152,32 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(1) << 46;                   // descriptor version for sm_100
     d |= static_cast<uint64_t>(2) << 61;                   // 128-byte swizzle
     return d;
+}
+
+// Shared-memory operand descriptor, K-major, 64-byte swizzle: rows of 64 B,
+// 8-row groups 512 B apart; the tile base must be 512-byte aligned (the start
+// address may be advanced by 32 B per K step inside the 64 B row).
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1) << 16;
+    d |= static_cast<uint64_t>(512 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(4) << 61;                   // 64-byte swizzle
+    return d;
+}
+
+// Instruction descriptor for kind::f8f6f4: fp32 accumulator, M x N, K-major;
+// format codes: 0 = E4M3, 1 = E5M2.
+__host__ __device__ constexpr uint32_t idesc_f8_f32(int M, int N, uint32_t a_fmt, uint32_t b_fmt) {
+    return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..3) of row `row` in a 64-byte-swizzled
+// K-major tile (rows of 64 B, 512-byte aligned base).
+__device__ __forceinline__ uint32_t sw64_offset(uint32_t row, uint32_t chunk) {
+    return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
 }
 
 // Shared-memory operand descriptor, MN-major, 128-byte swizzle: each 128-B row

@@ -163,7 +163,7 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_
     if (need0 == 0) return;
     const int64_t nvalid = n_valid_positions(src, seg);
     const int64_t n_items = src.ids ? src.n : nvalid;
-    uint32_t* cand = wk.cand1 + seg * wk.cand_stride;
+    uint2* cand = reinterpret_cast<uint2*>(wk.cand1) + seg * wk.cand_stride;
     for (int64_t base = (int64_t)blockIdx.x * kPassChunk; base < n_items; base += (int64_t)gridDim.x * kPassChunk) {
         const int64_t end = min(base + kPassChunk, n_items);
         for (int64_t it0 = base; it0 < end; it0 += kPassThreads) {
@@ -177,7 +177,7 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_
             const bool to_cand = eq && !take_eq;
             const uint32_t cs = warp_claim(to_cand, cnt + 1);
             if (to_cand) {
-                cand[cs] = (uint32_t)i;
+                cand[cs] = make_uint2(e.key, (uint32_t)e.id);
                 atomicAdd(&h2[digit(e.key, 2)], 1u);
             }
             const uint32_t os = warp_claim(take, cnt);
@@ -191,93 +191,122 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_
         if (h2[i]) atomicAdd(gh2 + i, h2[i]);
 }
 
-// Digits 2 and 3 of one segment's candidate list, one CTA.
-__global__ void __launch_bounds__(kFinThreads)
-k_sel_finish(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+// Threshold plan of levels 1 and 2 from the global histograms (one warp).
+// run = 0: level 1 already selected everything.
+struct Plan2 {
+    uint32_t run, c2, need2, n_cand, eq2;
+};
+
+__device__ __forceinline__ Plan2 plan_level2(const uint32_t* h1, const uint32_t* h2, int n_out) {
+    Plan2 pl = {0u, 0u, 0u, 0u, 0u};
+    const uint32_t total = warp_sum_hist(h1);
+    const uint32_t need = total < (uint32_t)n_out ? total : (uint32_t)n_out;
+    if (need > 0) {
+        const uint2 t1 = warp_threshold(h1, need);
+        pl.n_cand = h1[t1.x];
+        const uint32_t need1 = need - t1.y;
+        if (pl.n_cand != need1) {
+            const uint2 t2 = warp_threshold(h2, need1);
+            pl.run = 1;
+            pl.c2 = t2.x;
+            pl.need2 = need1 - t2.y;
+            pl.eq2 = h2[t2.x];
+        }
+    }
+    return pl;
+}
+
+// Digit 2 over the (key, id) candidates of level 1, many CTAs per segment.
+__global__ void __launch_bounds__(kPassThreads)
+k_sel_pass2(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    __shared__ Plan2 s_pl;
     __shared__ uint32_t h3[kRadixBins];
-    __shared__ uint32_t s_plan[6];
-    const int seg = blockIdx.x;
+    const int seg = blockIdx.y;
     const uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
-    const uint32_t* h2 = h1 + kRadixBins;
     uint32_t* cnt = wk.cnt + (int64_t)seg * 4;
-    for (int i = threadIdx.x; i < kRadixBins; i += kFinThreads) h3[i] = 0;
     if (threadIdx.x < 32) {
-        const uint32_t total = warp_sum_hist(h1);
-        const uint32_t need = total < (uint32_t)n_out ? total : (uint32_t)n_out;
-        uint32_t run = 0, c2 = 0, need2 = 0, n_cand = 0;
-        if (need > 0) {
-            const uint2 t1 = warp_threshold(h1, need);
-            n_cand = h1[t1.x];
-            const uint32_t need1 = need - t1.y;
-            if (n_cand != need1) {                // level 1 left candidates
-                const uint2 t2 = warp_threshold(h2, need1);
-                c2 = t2.x;
-                need2 = need1 - t2.y;
-                run = 1;
+        const Plan2 pl = plan_level2(h1, h1 + kRadixBins, n_out);
+        if (threadIdx.x == 0) s_pl = pl;
+    }
+    for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads) h3[i] = 0;
+    __syncthreads();
+    const Plan2 pl = s_pl;
+    if (!pl.run) return;
+    const bool take_eq = pl.eq2 == pl.need2;
+    const uint2* cand = reinterpret_cast<const uint2*>(wk.cand1) + seg * wk.cand_stride;
+    uint2* cand2 = reinterpret_cast<uint2*>(wk.cand2) + seg * wk.cand_stride;
+    int32_t* o = out + (int64_t)seg * out_stride;
+    bool any = false;
+    for (uint32_t base = blockIdx.x * kPassChunk; base < pl.n_cand; base += gridDim.x * kPassChunk) {
+        const uint32_t end = min(base + (uint32_t)kPassChunk, pl.n_cand);
+        for (uint32_t it0 = base; it0 < end; it0 += kPassThreads) {
+            const uint32_t it = it0 + threadIdx.x;
+            const bool in = it < end;
+            const uint2 kv = in ? cand[it] : make_uint2(0u, 0u);
+            const uint32_t d = digit(kv.x, 2);
+            const bool eq = in && d == pl.c2;
+            const bool take = in && (d > pl.c2 || (eq && take_eq));
+            const bool keep = eq && !take_eq;
+            const uint32_t ks = warp_claim(keep, cnt + 2);
+            if (keep) {
+                cand2[ks] = kv;
+                atomicAdd(&h3[digit(kv.x, 3)], 1u);
+                any = true;
+            }
+            const uint32_t os = warp_claim(take, cnt);
+            if (take) o[os] = (int32_t)kv.y;
+        }
+    }
+    if (take_eq || !__syncthreads_or(any)) return;
+    uint32_t* gh3 = wk.hist + ((int64_t)seg * 3 + 2) * kRadixBins;
+    for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads)
+        if (h3[i]) atomicAdd(gh3 + i, h3[i]);
+}
+
+// Digit 3 (exact ties last) of one segment, one CTA; then the histograms and
+// counters of the segment are cleared for the next selection.
+__global__ void __launch_bounds__(kFinThreads)
+k_sel_finish(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    __shared__ Plan2 s_pl;
+    __shared__ uint32_t s_plan[2];
+    const int seg = blockIdx.x;
+    uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
+    uint32_t* cnt = wk.cnt + (int64_t)seg * 4;
+    if (threadIdx.x < 32) {
+        const Plan2 pl = plan_level2(h1, h1 + kRadixBins, n_out);
+        if (threadIdx.x == 0) s_pl = pl;
+    }
+    __syncthreads();
+    const Plan2 pl = s_pl;
+    if (pl.run && pl.eq2 != pl.need2) {
+        const uint32_t* h3 = h1 + 2 * kRadixBins;
+        if (threadIdx.x < 32) {
+            const uint2 t3 = warp_threshold(h3, pl.need2);
+            if (threadIdx.x == 0) {
+                s_plan[0] = t3.x;
+                s_plan[1] = pl.need2 - t3.y;
             }
         }
-        if (threadIdx.x == 0) {
-            s_plan[0] = run;
-            s_plan[1] = c2;
-            s_plan[2] = need2;
-            s_plan[3] = n_cand;
-            s_plan[4] = run ? h2[c2] : 0;
+        __syncthreads();
+        const uint32_t c3 = s_plan[0], need3 = s_plan[1], n2 = pl.eq2;
+        const uint2* cand2 = reinterpret_cast<const uint2*>(wk.cand2) + seg * wk.cand_stride;
+        int32_t* o = out + (int64_t)seg * out_stride;
+        for (uint32_t it0 = 0; it0 < n2; it0 += kFinThreads) {
+            const uint32_t it = it0 + threadIdx.x;
+            const bool in = it < n2;
+            const uint2 kv = in ? cand2[it] : make_uint2(0u, 0u);
+            const uint32_t d = digit(kv.x, 3);
+            const bool eq = in && d == c3;
+            const uint32_t tie = warp_claim(eq, cnt + 3);
+            const bool take = in && (d > c3 || (eq && tie < need3));
+            const uint32_t os = warp_claim(take, cnt);
+            if (take) o[os] = (int32_t)kv.y;
         }
     }
+    // leave the workspace as csa2_workspace_init does: histograms and counters zero
     __syncthreads();
-    if (!s_plan[0]) return;
-    const uint32_t c2 = s_plan[1], need2 = s_plan[2], n_cand = s_plan[3];
-    const bool take_eq2 = s_plan[4] == need2;
-    const uint32_t* cand = wk.cand1 + seg * wk.cand_stride;
-    uint32_t* cand2 = wk.cand2 + seg * wk.cand_stride;
-    int32_t* o = out + (int64_t)seg * out_stride;
-    const int64_t nvalid = n_valid_positions(src, seg);
-    // digit 2: select above c2, keep the digit-c2 candidates for digit 3
-    for (uint32_t it0 = 0; it0 < n_cand; it0 += kFinThreads) {
-        const uint32_t it = it0 + threadIdx.x;
-        Elem e;
-        e.valid = false;
-        uint32_t ci = 0;
-        if (it < n_cand) {
-            ci = cand[it];
-            e = load_elem(src, seg, ci, nvalid);
-        }
-        const uint32_t d = e.valid ? digit(e.key, 2) : 0u;
-        const bool eq = e.valid && d == c2;
-        const bool take = e.valid && (d > c2 || (eq && take_eq2));
-        const bool keep = eq && !take_eq2;
-        const uint32_t ks = warp_claim(keep, cnt + 2);
-        if (keep) {
-            cand2[ks] = ci;
-            atomicAdd(&h3[digit(e.key, 3)], 1u);
-        }
-        const uint32_t os = warp_claim(take, cnt);
-        if (take) o[os] = e.id;
-    }
-    if (take_eq2) return;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        const uint2 t3 = warp_threshold(h3, need2);
-        if (threadIdx.x == 0) {
-            s_plan[1] = t3.x;
-            s_plan[2] = need2 - t3.y;
-            s_plan[3] = h2[c2];
-        }
-    }
-    __syncthreads();
-    const uint32_t c3 = s_plan[1], need3 = s_plan[2], n2 = s_plan[3];
-    for (uint32_t it0 = 0; it0 < n2; it0 += kFinThreads) {
-        const uint32_t it = it0 + threadIdx.x;
-        Elem e;
-        e.valid = false;
-        if (it < n2) e = load_elem(src, seg, cand2[it], nvalid);
-        const uint32_t d = e.valid ? digit(e.key, 3) : 0u;
-        const bool eq = e.valid && d == c3;
-        const uint32_t tie = warp_claim(eq, cnt + 3);
-        const bool take = e.valid && (d > c3 || (eq && tie < need3));
-        const uint32_t os = warp_claim(take, cnt);
-        if (take) o[os] = e.id;
-    }
+    for (int i = threadIdx.x; i < 3 * kRadixBins; i += kFinThreads) h1[i] = 0;
+    if (threadIdx.x < 4) cnt[threadIdx.x] = 0;
 }
 
 // ---------------------------------------------------------------- small segments
@@ -297,11 +326,29 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, int64_t out_stride
     if (threadIdx.x < 2) s_cnt[threadIdx.x] = 0;
     __syncthreads();
     uint32_t mine = 0;
-    for (int i = threadIdx.x; i < n; i += kFinThreads) {
-        Elem e = load_elem(src, seg, i, nvalid);
-        // the ordered key of a finite float is never 0
-        keys[i] = e.valid ? e.key : 0u;
-        if (e.valid) { atomicAdd(&hist[digit(e.key, 1)], 1u); ++mine; }
+    // 16 elements per thread (n <= 16384): ids first, then the values they select
+    constexpr int kPer = kSmallMax / kFinThreads;
+    int32_t ids[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = k * kFinThreads + threadIdx.x;
+        ids[k] = i < n ? (src.ids ? __ldg(src.ids + seg * src.ids_stride + i) : i) : -1;
+    }
+    float vals[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = k * kFinThreads + threadIdx.x;
+        const bool valid = i < n && ids[k] >= 0 && ids[k] < nvalid;
+        vals[k] = valid ? src.vals[seg * src.vals_stride + (src.gather || !src.ids ? (int64_t)ids[k] : i)] : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int i = k * kFinThreads + threadIdx.x;
+        if (i >= n) continue;
+        const bool valid = ids[k] >= 0 && ids[k] < nvalid;
+        const uint32_t key = valid ? ordered_key(vals[k]) : 0u;
+        keys[i] = key;                       // the ordered key of a finite float is never 0
+        if (valid) { atomicAdd(&hist[digit(key, 1)], 1u); ++mine; }
     }
     mine = __reduce_add_sync(0xffffffffu, mine);
     if ((threadIdx.x & 31) == 0 && mine) atomicAdd(&s_cnt[1], mine);
@@ -383,19 +430,17 @@ cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_
         k_sel_small<<<nseg, kFinThreads, smem, st>>>(src, n_out, out, out_stride);
         return cudaGetLastError();
     }
-    // hist_ready: every level of the histograms was zeroed before the scoring
-    // kernel filled level 1
-    if (!hist_ready) {
-        e = cudaMemsetAsync(wk.hist, 0, sizeof(uint32_t) * (size_t)nseg * 3 * kRadixBins, st);
-        if (e != cudaSuccess) return e;
-    }
-    e = cudaMemsetAsync(wk.cnt, 0, sizeof(uint32_t) * (size_t)nseg * 4, st);
-    if (e != cudaSuccess) return e;
+    // the histograms and counters are zero on entry (workspace initialisation,
+    // then every k_sel_finish clears what its selection used); without a
+    // histogram from the scoring kernel, build level 1 here
     const unsigned chunks = (unsigned)((src.n + kPassChunk - 1) / kPassChunk);
     dim3 grid(chunks ? chunks : 1, (unsigned)nseg);
     if (!hist_ready) k_sel_hist<<<grid, kPassThreads, 0, st>>>(src, wk);
     k_sel_pass1<<<grid, kPassThreads, 0, st>>>(src, wk, n_out, out, out_stride);
-    k_sel_finish<<<nseg, kFinThreads, 0, st>>>(src, wk, n_out, out, out_stride);
+    // level-1 candidates: at most the segment size; spread over up to 148 CTAs
+    const unsigned g2 = chunks < 148 ? (chunks ? chunks : 1) : 148;
+    k_sel_pass2<<<dim3(g2, (unsigned)nseg), kPassThreads, 0, st>>>(wk, n_out, out, out_stride);
+    k_sel_finish<<<nseg, kFinThreads, 0, st>>>(wk, n_out, out, out_stride);
     return cudaGetLastError();
 }
 
