@@ -22,9 +22,11 @@
 //   producer warp  : TMA loads into the ring (bounded mbarrier waits)
 //   MMA warp       : tcgen05.mma, commits that free ring stages and fill the
 //                    double-buffered TMEM accumulator
-//   epilogue warps : stage the query terms when the sequence changes; per tile
-//                    tcgen05.ld of each position's row, ReLU + head-weighted
-//                    sum, fp32 score store, level-1 radix histogram in smem.
+//   epilogue warps : two warpgroups, one per TMEM accumulator, so tile g is
+//                    finished by warpgroup g % 2; they stage the query terms
+//                    when the sequence changes; per tile tcgen05.ld of each
+//                    position's row, ReLU + head-weighted sum, fp32 score
+//                    store, level-1 radix histogram in smem.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -40,8 +42,9 @@ constexpr int kItemTiles = 4;
 constexpr int kStages = 8;
 constexpr int kStageBytes = kTile * 64;   // two 64-row boxes of E4M3 keys
 constexpr int kTerms = 4;
-constexpr int kThreads = 192;
-constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;
+constexpr int kThreads = 320;
+constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;   // epilogue: warps 2-9, two warpgroups
+constexpr int kEpiThreads = 256;
 constexpr uint32_t kDrainLimit = 65536;
 
 struct Params {
@@ -184,11 +187,11 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars->acc_full[i], 1);
             tc::mbar_init(&bars->acc_empty[i], 128);
-            tc::mbar_init(&bars->b_ready[i], 128);
+            tc::mbar_init(&bars->b_ready[i], kEpiThreads);
             tc::mbar_init(&bars->b_free[i], 1);
         }
-        tc::mbar_init(&bars->hist_done, 128);
-        tc::mbar_init(&bars->hist_clear, 128);
+        tc::mbar_init(&bars->hist_done, kEpiThreads);
+        tc::mbar_init(&bars->hist_clear, kEpiThreads);
         tc::mbar_init(&bars->drain, 1);
         tc::fence_mbar_init();
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
@@ -277,8 +280,9 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
             tc::mbar_wait(&bars->drain, 0, kDrainLimit);
         }
     } else {
-        // epilogue: 128 threads, thread = TMEM lane = position in the tile
-        const int tid = threadIdx.x - kWarpEpi0 * 32;
+        // epilogue: two warpgroups; thread = TMEM lane = position in the tile
+        const int tid = threadIdx.x - kWarpEpi0 * 32;          // 0..255
+        const int grp = tid >> 7;                               // accumulator this group drains
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
@@ -286,14 +290,14 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
         int cur_b = -1;
         bool ok = true;
         // Move the shared histogram of sequence b into the global one.  The
-        // 128 epilogue threads meet on two mbarriers (bounded waits).
+        // epilogue threads meet on two mbarriers (bounded waits).
         auto flush = [&](int b) -> bool {
             tc::mbar_arrive(&bars->hist_done);
             if (!tc::mbar_wait(&bars->hist_done, nflush & 1)) return false;
             if (p.hist) {
                 for (int j = 0; j < p.T; ++j) {
                     uint32_t* gh = p.hist + ((int64_t)b * p.T + j) * 3 * kRadixBins;
-                    for (int i = tid; i < kRadixBins; i += 128) {
+                    for (int i = tid; i < kRadixBins; i += kEpiThreads) {
                         const uint32_t v = sHist[j * kRadixBins + i];
                         if (v) { atomicAdd(gh + i, v); sHist[j * kRadixBins + i] = 0; }
                     }
@@ -323,31 +327,38 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                 // sequence that used the buffer before are done
                 const int qb = n & 1;
                 if (!tc::mbar_wait(&bars->b_free[qb], ((n >> 1) & 1) ^ 1)) { ok = false; break; }
-                prepare_queries(p, it.b, sB + qb * bq_bytes, sWq + qb * p.NP, tid);
+                if (grp == 0) prepare_queries(p, it.b, sB + qb * bq_bytes, sWq + qb * p.NP, tid);
                 tc::fence_proxy_async_smem();
                 tc::mbar_arrive(&bars->b_ready[qb]);
-                // the same barrier publishes the weights to the other epilogue threads
+                // the same barrier publishes the weights to every epilogue thread
                 if (!warp_wait(&bars->b_ready[qb], (n >> 1) & 1)) { ok = false; break; }
                 wq = sWq + qb * p.NP;
             }
             for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                 const int acc = g & 1;
+                if (acc != grp) continue;                       // the other group's tile
                 if (!warp_wait(&bars->acc_full[acc], (g >> 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
                 const int64_t t = it.t0 + (int64_t)tl * kTile + row;
                 for (int j = 0; j < p.T; ++j) {
                     float s0 = 0.0f, s1 = 0.0f;
-                    for (int c0 = j * p.HP; c0 < (j + 1) * p.HP; c0 += 16) {
-                        float v[16];
-                        tc::tmem_ld16(lane_addr + (uint32_t)(acc * p.NP + c0), v);
+                    for (int c0 = j * p.HP; c0 < (j + 1) * p.HP; c0 += 32) {
+                        // two 16-column loads in flight, one wait
+                        uint32_t r[32];
+                        const bool two = c0 + 16 < (j + 1) * p.HP;
+                        tc::tmem_ld16_nowait(lane_addr + (uint32_t)(acc * p.NP + c0), r);
+                        if (two) tc::tmem_ld16_nowait(lane_addr + (uint32_t)(acc * p.NP + c0 + 16), r + 16);
+                        tc::tmem_ld_wait();
                         const float4* w4 = reinterpret_cast<const float4*>(wq + c0);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 ww = w4[i];
-                            s0 = fmaf(ww.x, fmaxf(v[4 * i], 0.0f), s0);
-                            s1 = fmaf(ww.y, fmaxf(v[4 * i + 1], 0.0f), s1);
-                            s0 = fmaf(ww.z, fmaxf(v[4 * i + 2], 0.0f), s0);
-                            s1 = fmaf(ww.w, fmaxf(v[4 * i + 3], 0.0f), s1);
+                        for (int i = 0; i < 8; ++i) {
+                            if (i < 4 || two) {
+                                const float4 ww = w4[i];
+                                s0 = fmaf(ww.x, fmaxf(__uint_as_float(r[4 * i]), 0.0f), s0);
+                                s1 = fmaf(ww.y, fmaxf(__uint_as_float(r[4 * i + 1]), 0.0f), s1);
+                                s0 = fmaf(ww.z, fmaxf(__uint_as_float(r[4 * i + 2]), 0.0f), s0);
+                                s1 = fmaf(ww.w, fmaxf(__uint_as_float(r[4 * i + 3]), 0.0f), s1);
+                            }
                         }
                     }
                     const float s = s0 + s1;
