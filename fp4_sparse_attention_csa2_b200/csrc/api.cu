@@ -76,7 +76,7 @@ int num_sms() {
 // The radix histograms and counters are zero between calls: the workspace
 // starts zeroed and every large selection clears what it used.
 struct Layout {
-    size_t status, scores, hist, hist_scratch, cnt, cand1, cand2, pscores, part_o, part_ml, total;
+    size_t status, scores, hist, hist_scratch, cnt, cand1, cand2, pscores, part_o, part_ml, qstage, total;
     int64_t nseg, cap, cand_stride;
     int nchunk;
 };
@@ -99,6 +99,7 @@ bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int w
     L->pscores = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * pool_k);
     L->part_o = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * c->dim);
     L->part_ml = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * 2);
+    L->qstage = off; off = align_up(off + (size_t)L->nseg * attn_tc_qstage_bytes(c->dim, H));
     L->total = off;
     return true;
 }
@@ -286,6 +287,7 @@ csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, in
     AttnWork aw;
     aw.part_o = at<float>(ws, L.part_o);
     aw.part_ml = at<float>(ws, L.part_ml);
+    aw.qstage = at<uint8_t>(ws, L.qstage);
     aw.nchunk = L.nchunk;
     return cuda_status(launch_attention(dev_cache(cache), q_bf16, T, H, topk_idx, top_k, window, sm_scale, out, lse,
                                         aw, at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream)));

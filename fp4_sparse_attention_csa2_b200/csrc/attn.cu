@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(kThreads)
 k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, const int32_t* __restrict__ topk,
                int top_k, int window, float scale, float* __restrict__ part_o, float* __restrict__ part_ml,
                int nchunk, uint32_t* status) {
+    pdl_begin();
     extern __shared__ float smem[];
     const int D = c.dim;
     const int DP = D + 4;
@@ -153,6 +154,7 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
 __global__ void __launch_bounds__(128)
 k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk,
                float* __restrict__ out, float* __restrict__ lse) {
+    pdl_begin();
     const int seg = blockIdx.x, h = blockIdx.y;
     __shared__ float s_w[1024];
     __shared__ float s_red[4];
@@ -181,7 +183,22 @@ k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __re
     const float* base = part_o + ((int64_t)seg * nchunk * H + h) * D;
     const int64_t cstride = (int64_t)H * D;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int ch = 0; ch < nchunk; ++ch) {
+    int ch = 0;
+    for (; ch + 4 <= nchunk; ch += 4) {        // 16 independent loads in flight per thread
+        float v[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int d = tid + 128 * k;
+                v[u][k] = d < D ? base[(ch + u) * cstride + d] : 0.0f;
+            }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = fmaf(s_w[ch + u], v[u][k], acc[k]);
+    }
+    for (; ch < nchunk; ++ch) {
         const float w = s_w[ch];
         const float* src = base + ch * cstride;
 #pragma unroll
@@ -204,9 +221,8 @@ int attn_rows_per_chunk() { return kRows; }
 
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st) {
-    k_attn_combine<<<dim3((unsigned)(c.batch * T), (unsigned)H), 128, 0, st>>>(c.dim, H, aw.part_o, aw.part_ml,
-                                                                             aw.nchunk, out, lse);
-    return cudaGetLastError();
+    return launch_pdl(k_attn_combine, dim3((unsigned)(c.batch * T), (unsigned)H), dim3(128), 0, st, c.dim, H, aw.part_o, aw.part_ml,
+                      aw.nchunk, out, lse);
 }
 
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
@@ -228,9 +244,8 @@ cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, con
         e = cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         dim3 grid((unsigned)aw.nchunk, (unsigned)(c.batch * T));
-        k_attn_partial<<<grid, kThreads, smem, st>>>(c, static_cast<const __nv_bfloat16*>(q), T, H, topk, top_k,
+        e = launch_pdl(k_attn_partial, dim3(grid), dim3(kThreads), smem, st, c, static_cast<const __nv_bfloat16*>(q), T, H, topk, top_k,
                                                      window, sm_scale, aw.part_o, aw.part_ml, aw.nchunk, status);
-        e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
     return launch_attn_combine(c, T, H, aw, out, lse, st);

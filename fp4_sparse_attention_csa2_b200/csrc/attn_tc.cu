@@ -40,16 +40,19 @@ struct Params {
     float scale;
     float* part_o;            // [seg][chunk][H][D]
     float* part_ml;           // [seg][chunk][H][2]
+    const uint8_t* qstage;    // [seg][qbytes]: the staged query operand, then H factors
+    uint32_t qbytes;          // bytes of the staged fp16 operand of one segment
     uint32_t* status;
     uint32_t off_q, off_misc, tmem_cols;
 };
 
 struct Misc {
-    uint64_t mma_bar;
-    uint32_t tmem_base;
+    alignas(16) float fac[64];   // per head: softmax scale / query scale (bulk-copied)
+    float red[16][64];           // per head partial max / sum of the threads that share it
     int32_t pos[kRows];
-    float fac[64];            // per head: softmax scale / query scale
-    float red[2][64];         // per head partial max / sum of the two halves
+    uint64_t mma_bar;
+    uint64_t q_bar;
+    uint32_t tmem_base;
 };
 
 __device__ __forceinline__ uint32_t cvt_e2m1x2_f16x2(uint32_t byte) {
@@ -70,6 +73,7 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
+    pdl_begin();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int D = p.c.dim, H = p.H;
@@ -88,7 +92,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
 
     if (tid == 0) {
         tc::mbar_init(&misc->mma_bar, 1);
+        tc::mbar_init(&misc->q_bar, 1);
         tc::fence_mbar_init();
+        // the query operand, staged once per (sequence, token) by k_attn_stage_q,
+        // arrives by bulk copy while the rows are gathered
+        const uint8_t* src = p.qstage + (size_t)seg * (p.qbytes + 256);
+        tc::mbar_arrive_expect_tx(&misc->q_bar, p.qbytes + (uint32_t)H * 4);
+        for (uint32_t off = 0; off < p.qbytes; off += 16384) {
+            const uint32_t n = p.qbytes - off < 16384 ? p.qbytes - off : 16384;
+            tc::bulk_g2s(sQ + off, src + off, n, &misc->q_bar);
+        }
+        tc::bulk_g2s(misc->fac, src + p.qbytes, (uint32_t)H * 4, &misc->q_bar);
     }
     if (warp == 0) tc::tmem_alloc(&misc->tmem_base, p.tmem_cols);
     if (tid < kRows) {
@@ -135,53 +149,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         }
     }
 
-    // ---- queries: fp16 scaled by 2^e per head, K-major swizzled (4 threads per head)
-    for (int w = tid; w < H * 4; w += kThreads) {
-        const int h = w >> 2, part = w & 3;           // part: D/4 consecutive values
-        const int span = D / 4;
-        const __nv_bfloat16* src = p.q + ((int64_t)seg * H + h) * D + part * span;
-        uint4 qv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (8 * i < span) qv[i] = __ldg(reinterpret_cast<const uint4*>(src + 8 * i));
-        float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (8 * i < span) {
-                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[k] << 16)), fabsf(__uint_as_float(wv[k] & 0xFFFF0000u))));
-            }
-        }
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        int e = 0;
-        if (m > 0.0f) {
-            e = 14 - ((int)((__float_as_uint(m) >> 23) & 0xFF) - 127);
-            e = e < -100 ? -100 : (e > 100 ? 100 : e);
-        }
-        const float up = __uint_as_float((uint32_t)(127 + e) << 23);
-        if (part == 0) misc->fac[h] = p.scale * __uint_as_float((uint32_t)(127 - e) << 23);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (8 * i < span) {
-                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
-                uint32_t hv[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    __half2 hh = __floats2half2_rn(__uint_as_float(wv[k] << 16) * up,
-                                                   __uint_as_float(wv[k] & 0xFFFF0000u) * up);
-                    memcpy(&hv[k], &hh, 4);
-                }
-                const int d = part * span + 8 * i;        // 8 values: one 16-byte chunk
-                uint8_t* blk = sQ + (d >> 6) * (H * 128);
-                *reinterpret_cast<uint4*>(blk + tc::sw128_offset(h, (d & 63) >> 3)) =
-                    make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            }
-        }
-    }
-
     // ---- dequantise: value(code) * value(scale), exact in fp16, into the swizzled V tile
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -210,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     __syncthreads();
 
     // ---- S = V Q^T
-    bool ok = true;
-    if (warp == 4 && lane == 0) {
+    bool ok = tc::mbar_wait(&misc->q_bar, 0);   // every thread reads fac[] later
+    if (warp == 4 && lane == 0 && ok) {
         tc::fence_after_sync();
         const uint32_t idesc = tc::idesc_f16_f32(kRows, H);
         const uint32_t v0 = tc::smem_u32(sV), q0 = tc::smem_u32(sQ);
@@ -222,38 +189,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
                             tc::desc_sw128(q0 + kb * (H * 128) + 32 * k), idesc, (kb | k) != 0);
         tc::mma_commit(&misc->mma_bar);
     }
-    ok = tc::mbar_wait(&misc->mma_bar, 0);
+    if (ok) ok = tc::mbar_wait(&misc->mma_bar, 0);
     ok = __syncthreads_and(ok);
     tc::fence_after_sync();
 
-    // ---- logits to shared memory, transposed: z[h][pos] (warps 0-3: lane = position)
-    if (ok && warp < 4) {
-        const int r = warp * 32 + lane;
+    // ---- logits to shared memory, transposed: z[h][pos]; lane = position, the
+    // two warpgroups take one half of the heads each (H >= 32)
+    const int ngrp = H >= 32 ? 2 : 1;
+    const int wgrp = warp >> 2, quad = warp & 3;
+    if (ok && wgrp < ngrp) {
+        const int r = quad * 32 + lane;
         const bool valid = misc->pos[r] >= 0;
-        for (int c0 = 0; c0 < H; c0 += 16) {
+        const int hc = H / ngrp;
+        for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
             float v[16];
-            tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+            tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
 #pragma unroll
             for (int i = 0; i < 16; ++i) sZ[(c0 + i) * kZStride + r] = valid ? v[i] * misc->fac[c0 + i] : -INFINITY;
         }
     }
     __syncthreads();
 
-    // ---- softmax statistics: thread (h, half) over 64 positions
-    const int h = tid % H, half = tid / H;
-    const bool stat = tid < 2 * H;
+    // ---- softmax statistics: nq = 256 / H threads per head, each over 128 / nq positions
+    const int nq = kThreads / H, per = kRows / nq;
+    const int h = tid % H, qt = tid / H;
+    const float* z = sZ + h * kZStride + qt * per;
     float m = -INFINITY, l = 0.0f;
-    if (ok && stat) {
-        const float* z = sZ + h * kZStride + half * 64;
-        for (int i = 0; i < 64; ++i) m = fmaxf(m, z[i]);
-        misc->red[half][h] = m;
+    if (ok) {
+        for (int i = 0; i < per; ++i) m = fmaxf(m, z[i]);
+        misc->red[qt][h] = m;
     }
     __syncthreads();
-    if (ok && stat) {
-        m = fmaxf(misc->red[0][h], misc->red[1][h]);
-        const float* z = sZ + h * kZStride + half * 64;
-        uint8_t* blk = sP + half * (H * 128);
-        for (int c = 0; c < 8; ++c) {
+    if (ok) {
+        for (int k = 0; k < nq; ++k) m = fmaxf(m, misc->red[k][h]);
+        uint8_t* blk = sP + ((qt * per) >> 6) * (H * 128);
+        const int c_first = ((qt * per) & 63) >> 3;
+        for (int c = 0; c < per / 8; ++c) {
             uint32_t hv[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -264,17 +235,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
                 l += back.x + back.y;
                 memcpy(&hv[k], &hh, 4);
             }
-            *reinterpret_cast<uint4*>(blk + tc::sw128_offset(h, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4*>(blk + tc::sw128_offset(h, c_first + c)) =
+                make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
     }
     __syncthreads();   // all reads of red[] (the maxima) are done before it is reused for sums
-    if (ok && stat) misc->red[half][h] = l;
+    if (ok) misc->red[qt][h] = l;
     tc::fence_proxy_async_smem();
     __syncthreads();
     if (ok && tid < H) {
         float* ml = p.part_ml + (((int64_t)seg * p.nchunk + chunk) * H + tid) * 2;
+        float sum = 0.0f;
+        for (int k = 0; k < nq; ++k) sum += misc->red[k][tid];
         ml[0] = m;                                   // thread tid < H holds head tid's maximum
-        ml[1] = misc->red[0][tid] + misc->red[1][tid];
+        ml[1] = sum;
     }
 
     // ---- O^T = V^T P^T, one 128-wide slab of d per accumulator
@@ -293,14 +267,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     ok = __syncthreads_and(ok);
     tc::fence_after_sync();
 
-    // ---- unnormalised partial output (warps 0-3: lane = d within the slab)
-    if (ok && warp < 4) {
+    // ---- unnormalised partial output (lane = d within the slab; the two
+    // warpgroups take one half of the heads each)
+    if (ok && wgrp < ngrp) {
         float* po = p.part_o + ((int64_t)seg * p.nchunk + chunk) * H * D;
-        for (int s = 0; s < D / 128; ++s) {
-            const int d = s * 128 + warp * 32 + lane;
-            for (int c0 = 0; c0 < H; c0 += 16) {
+        const int hc = H / ngrp;
+        for (int s2 = 0; s2 < D / 128; ++s2) {
+            const int d = s2 * 128 + quad * 32 + lane;
+            for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
                 float v[16];
-                tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(H + s * H + c0), v);
+                tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(H + s2 * H + c0), v);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) po[(int64_t)(c0 + i) * D + d] = v[i];
             }
@@ -312,6 +288,65 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     if (warp == 0) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, p.tmem_cols);
+    }
+}
+
+// The query operand of one (sequence, token): H rows of D fp16 values scaled by
+// 2^e per head (the row maximum lands in [2^14, 2^15): every bf16 value down to
+// 2^-32 of it is exact in fp16), laid out exactly as the attention kernel's
+// K-major 128-byte-swizzled operand, followed by the H factors
+// softmax_scale * 2^-e.  grid (B*T), 256 threads, 4 threads per head.
+__global__ void __launch_bounds__(kThreads)
+k_attn_stage_q(const __nv_bfloat16* __restrict__ q, int H, int D, float scale, uint8_t* __restrict__ qstage,
+               uint32_t qbytes) {
+    pdl_begin();
+    const int seg = blockIdx.x, tid = threadIdx.x;
+    uint8_t* dst = qstage + (size_t)seg * (qbytes + 256);
+    float* fac = reinterpret_cast<float*>(dst + qbytes);
+    for (int w = tid; w < H * 4; w += kThreads) {
+        const int h = w >> 2, part = w & 3;           // part: D/4 consecutive values
+        const int span = D / 4;
+        const __nv_bfloat16* src = q + ((int64_t)seg * H + h) * D + part * span;
+        uint4 qv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (8 * i < span) qv[i] = __ldg(reinterpret_cast<const uint4*>(src + 8 * i));
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (8 * i < span) {
+                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[k] << 16)), fabsf(__uint_as_float(wv[k] & 0xFFFF0000u))));
+            }
+        }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        int e = 0;
+        if (m > 0.0f) {
+            e = 14 - ((int)((__float_as_uint(m) >> 23) & 0xFF) - 127);
+            e = e < -100 ? -100 : (e > 100 ? 100 : e);
+        }
+        const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+        if (part == 0) fac[h] = scale * __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (8 * i < span) {
+                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+                uint32_t hv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    __half2 hh = __floats2half2_rn(__uint_as_float(wv[k] << 16) * up,
+                                                   __uint_as_float(wv[k] & 0xFFFF0000u) * up);
+                    memcpy(&hv[k], &hh, 4);
+                }
+                const int d = part * span + 8 * i;        // 8 values: one 16-byte chunk
+                uint8_t* blk = dst + (d >> 6) * (H * 128);
+                *reinterpret_cast<uint4*>(blk + tc::sw128_offset(h, (d & 63) >> 3)) =
+                    make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            }
+        }
     }
 }
 
@@ -329,11 +364,13 @@ size_t attn_tc_smem(int D, int H, uint32_t* off_q, uint32_t* off_misc) {
 
 bool attn_tc_supported(const DevCache& c, int H) {
     uint32_t a, b;
-    return c.dim % 128 == 0 && c.dim <= 512 && H % 16 == 0 && H >= 16 && H <= 64 &&
+    return c.dim % 128 == 0 && c.dim <= 512 && (H == 16 || H == 32 || H == 64) &&
            attn_tc_smem(c.dim, H, &a, &b) <= 227 * 1024;
 }
 
 int attn_tc_rows_per_chunk() { return kRows; }
+
+size_t attn_tc_qstage_bytes(int D, int H) { return (size_t)(D / 64) * H * 128 + 256; }
 
 cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
                                 int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st) {
@@ -349,6 +386,8 @@ cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, 
     p.scale = sm_scale;
     p.part_o = aw.part_o;
     p.part_ml = aw.part_ml;
+    p.qstage = aw.qstage;
+    p.qbytes = (uint32_t)(c.dim / 64) * H * 128;
     p.status = status;
     uint32_t cols = 32;
     while (cols < (uint32_t)(H + (c.dim / 128) * H)) cols <<= 1;
@@ -356,9 +395,10 @@ cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, 
     const size_t smem = attn_tc_smem(c.dim, H, &p.off_q, &p.off_misc);
     cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)aw.nchunk, (unsigned)(c.batch * T));
-    k_attn_tc<<<grid, kThreads, smem, st>>>(p);
-    return cudaGetLastError();
+    e = launch_pdl(k_attn_stage_q, dim3((unsigned)(c.batch * T)), dim3(kThreads), 0, st, p.q, H, c.dim, sm_scale,
+                   aw.qstage, p.qbytes);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_attn_tc, dim3((unsigned)aw.nchunk, (unsigned)(c.batch * T)), dim3(kThreads), smem, st, p);
 }
 
 }  // namespace csa2

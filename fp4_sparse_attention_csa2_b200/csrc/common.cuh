@@ -1,6 +1,7 @@
 // Device-side helpers shared by the libcsa2 kernels (sm_100a).
 #pragma once
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -92,6 +93,33 @@ __device__ __forceinline__ __half2 e2m1x2_to_half2(uint8_t v) {
     __half2 h;
     memcpy(&h, &r, 4);
     return h;
+}
+
+// ---------------------------------------------------------------- launches
+// Programmatic dependent launch: every kernel of the library is launched so
+// that it may start while the previous kernel on the stream finishes; it calls
+// pdl_begin() before touching global memory, which waits until the previous
+// kernel has completed and its writes are visible, and then lets the next
+// kernel launch early.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Monotone map of fp32 onto uint32 (larger float -> larger key); -0 == +0.

@@ -66,6 +66,7 @@ __device__ __forceinline__ float score_one(const float* qs, const float* hw, int
 __global__ void __launch_bounds__(256)
 k_score_full(DevCache c, const void* __restrict__ q, int q_f32, const float* __restrict__ hw, int T, int H_I,
              float* __restrict__ scores, uint32_t* status) {
+    pdl_begin();
     extern __shared__ float smem[];
     float* qs = smem;
     float* ws = smem + T * H_I * kDI;
@@ -91,6 +92,7 @@ k_score_full(DevCache c, const void* __restrict__ q, int q_f32, const float* __r
 __global__ void __launch_bounds__(256)
 k_score_pool(DevCache c, const void* __restrict__ q, int q_f32, const float* __restrict__ hw, int T, int H_I,
              const int32_t* __restrict__ pool, int pool_k, float* __restrict__ scores, uint32_t* status) {
+    pdl_begin();
     extern __shared__ float smem[];
     float* qs = smem;
     float* ws = smem + H_I * kDI;
@@ -122,16 +124,14 @@ cudaError_t launch_score_full(const DevCache& c, const void* q, int q_f32, const
         if (e != cudaSuccess) return e;
     }
     dim3 grid((unsigned)((c.cap + 255) / 256), (unsigned)c.batch);
-    k_score_full<<<grid, 256, smem, st>>>(c, q, q_f32, hw, T, H_I, scores, status);
-    return cudaGetLastError();
+    return launch_pdl(k_score_full, dim3(grid), dim3(256), smem, st, c, q, q_f32, hw, T, H_I, scores, status);
 }
 
 cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
                               const int32_t* pool, int pool_k, float* scores, uint32_t* status, cudaStream_t st) {
     const size_t smem = sizeof(float) * (size_t)H_I * (kDI + 1);
     dim3 grid((unsigned)((pool_k + 255) / 256), (unsigned)(c.batch * T));
-    k_score_pool<<<grid, 256, smem, st>>>(c, q, q_f32, hw, T, H_I, pool, pool_k, scores, status);
-    return cudaGetLastError();
+    return launch_pdl(k_score_pool, dim3(grid), dim3(256), smem, st, c, q, q_f32, hw, T, H_I, pool, pool_k, scores, status);
 }
 
 }  // namespace csa2

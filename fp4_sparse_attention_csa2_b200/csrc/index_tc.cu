@@ -171,6 +171,7 @@ __device__ void prepare_queries(const Params& p, int b, uint8_t* bq, float* wq, 
 
 __global__ void __launch_bounds__(kThreads, 2)
 k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
+    pdl_begin();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sRing = smem;
@@ -476,8 +477,7 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
     int64_t grid = 2 * (int64_t)num_sms;   // two CTAs per SM
     if (grid > p.total_items) grid = p.total_items;
     if (grid < 1) grid = 1;
-    k_score_full_tc<<<(unsigned)grid, kThreads, sp.total, st>>>(tmap, p);
-    return cudaGetLastError();
+    return launch_pdl(k_score_full_tc, dim3((unsigned)grid), dim3(kThreads), sp.total, st, tmap, p);
 }
 
 }  // namespace csa2

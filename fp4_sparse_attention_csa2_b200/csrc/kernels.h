@@ -63,11 +63,13 @@ cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_
 struct AttnWork {
     float* part_o;    // [nseg][nchunk][H][D]
     float* part_ml;   // [nseg][nchunk][H][2]
+    uint8_t* qstage;  // [nseg][attn_tc_qstage_bytes]: staged query operands
     int nchunk;
 };
 int attn_rows_per_chunk();       // smallest chunk of any attention kernel (sizes the workspace)
 bool attn_tc_supported(const DevCache& c, int H);
 int attn_tc_rows_per_chunk();
+size_t attn_tc_qstage_bytes(int D, int H);
 cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
                                 int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st);
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,

@@ -19,6 +19,7 @@ namespace csa2 {
 __global__ void __launch_bounds__(256)
 k_append_quant(DevCache c, const __nv_bfloat16* __restrict__ x, const void* __restrict__ idx_new,
                int idx_new_f32, const int32_t* __restrict__ start_pos, int n_new, uint32_t* status) {
+    pdl_begin();
     const int nblk = c.dim >> 4;
     const int64_t rows_total = (int64_t)c.batch * n_new;
     const int64_t n_row_work = rows_total * nblk;
@@ -111,9 +112,8 @@ cudaError_t launch_append_quant(const DevCache& c, const void* x, const void* id
     const int64_t max_blocks = (int64_t)num_sms * 8;
     if (blocks > max_blocks) blocks = max_blocks;
     if (blocks < 1) blocks = 1;
-    k_append_quant<<<(unsigned)blocks, 256, 0, st>>>(c, static_cast<const __nv_bfloat16*>(x), idx_new, idx_new_f32,
+    return launch_pdl(k_append_quant, dim3((unsigned)blocks), dim3(256), 0, st, c, static_cast<const __nv_bfloat16*>(x), idx_new, idx_new_f32,
                                                       start_pos, n_new, status);
-    return cudaGetLastError();
 }
 
 }  // namespace csa2

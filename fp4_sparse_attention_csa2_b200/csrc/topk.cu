@@ -101,6 +101,13 @@ __device__ __forceinline__ uint32_t warp_sum_hist(const uint32_t* h) {
     return __reduce_add_sync(0xffffffffu, v);
 }
 
+// Histogram increment by a whole warp: lanes with the same bin add once.
+__device__ __forceinline__ void warp_hist_add(uint32_t* hist, bool pred, uint32_t bin) {
+    const uint32_t key = pred ? bin : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, key);
+    if (pred && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(hist + bin, (uint32_t)__popc(peers));
+}
+
 // Warp-aggregated claim: the lanes with `pred` get consecutive values of *counter.
 __device__ __forceinline__ uint32_t warp_claim(bool pred, uint32_t* counter) {
     const int lane = threadIdx.x & 31;
@@ -117,6 +124,7 @@ __device__ __forceinline__ uint32_t warp_claim(bool pred, uint32_t* counter) {
 // ---------------------------------------------------------------- large segments
 // Level-1 histogram, for sources that did not get one from the scoring kernel.
 __global__ void __launch_bounds__(kPassThreads) k_sel_hist(SelSrc src, SelWork wk) {
+    pdl_begin();
     __shared__ uint32_t h[kRadixBins];
     const int seg = blockIdx.y;
     for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads) h[i] = 0;
@@ -137,6 +145,7 @@ __global__ void __launch_bounds__(kPassThreads) k_sel_hist(SelSrc src, SelWork w
 // Level 1 over every element: select digit > c1, compact digit == c1.
 __global__ void __launch_bounds__(kPassThreads)
 k_sel_pass1(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    pdl_begin();
     __shared__ uint32_t s_plan[3];   // c1, elements to select, take every digit-c1 element
     __shared__ uint32_t h2[kRadixBins];
     const int seg = blockIdx.y;
@@ -168,18 +177,15 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_
         const int64_t end = min(base + kPassChunk, n_items);
         for (int64_t it0 = base; it0 < end; it0 += kPassThreads) {
             const int64_t i = it0 + threadIdx.x;
-            Elem e;
-            e.valid = false;
+            Elem e = {false, -1, 0u};
             if (i < end) e = load_elem(src, seg, i, nvalid);
             const uint32_t d = e.valid ? digit(e.key, 1) : 0u;
             const bool eq = e.valid && d == c1;
             const bool take = e.valid && (d > c1 || (eq && take_eq));
             const bool to_cand = eq && !take_eq;
             const uint32_t cs = warp_claim(to_cand, cnt + 1);
-            if (to_cand) {
-                cand[cs] = make_uint2(e.key, (uint32_t)e.id);
-                atomicAdd(&h2[digit(e.key, 2)], 1u);
-            }
+            if (to_cand) cand[cs] = make_uint2(e.key, (uint32_t)e.id);
+            warp_hist_add(h2, to_cand, digit(e.key, 2));
             const uint32_t os = warp_claim(take, cnt);
             if (take) o[os] = e.id;
         }
@@ -219,6 +225,7 @@ __device__ __forceinline__ Plan2 plan_level2(const uint32_t* h1, const uint32_t*
 // Digit 2 over the (key, id) candidates of level 1, many CTAs per segment.
 __global__ void __launch_bounds__(kPassThreads)
 k_sel_pass2(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    pdl_begin();
     __shared__ Plan2 s_pl;
     __shared__ uint32_t h3[kRadixBins];
     const int seg = blockIdx.y;
@@ -250,9 +257,9 @@ k_sel_pass2(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride
             const uint32_t ks = warp_claim(keep, cnt + 2);
             if (keep) {
                 cand2[ks] = kv;
-                atomicAdd(&h3[digit(kv.x, 3)], 1u);
                 any = true;
             }
+            warp_hist_add(h3, keep, digit(kv.x, 3));
             const uint32_t os = warp_claim(take, cnt);
             if (take) o[os] = (int32_t)kv.y;
         }
@@ -267,6 +274,7 @@ k_sel_pass2(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride
 // counters of the segment are cleared for the next selection.
 __global__ void __launch_bounds__(kFinThreads)
 k_sel_finish(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    pdl_begin();
     __shared__ Plan2 s_pl;
     __shared__ uint32_t s_plan[2];
     const int seg = blockIdx.x;
@@ -313,6 +321,7 @@ k_sel_finish(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_strid
 // Whole selection of one segment of at most kSmallMax elements in one CTA.
 __global__ void __launch_bounds__(kFinThreads)
 k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, int64_t out_stride) {
+    pdl_begin();
     extern __shared__ uint32_t sm[];
     uint32_t* keys = sm;                        // [n]; 0 marks an invalid element
     uint32_t* hist = sm + src.n;                // [kRadixBins]
@@ -344,11 +353,11 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, int64_t out_stride
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
         const int i = k * kFinThreads + threadIdx.x;
-        if (i >= n) continue;
-        const bool valid = ids[k] >= 0 && ids[k] < nvalid;
+        const bool valid = i < n && ids[k] >= 0 && ids[k] < nvalid;
         const uint32_t key = valid ? ordered_key(vals[k]) : 0u;
-        keys[i] = key;                       // the ordered key of a finite float is never 0
-        if (valid) { atomicAdd(&hist[digit(key, 1)], 1u); ++mine; }
+        if (i < n) keys[i] = key;            // the ordered key of a finite float is never 0
+        warp_hist_add(hist, valid, digit(key, 1));
+        mine += valid;
     }
     mine = __reduce_add_sync(0xffffffffu, mine);
     if ((threadIdx.x & 31) == 0 && mine) atomicAdd(&s_cnt[1], mine);
@@ -364,9 +373,10 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, int64_t out_stride
             __syncthreads();
             for (int i = threadIdx.x; i < kRadixBins; i += kFinThreads) hist[i] = 0;
             __syncthreads();
-            for (int i = threadIdx.x; i < n; i += kFinThreads) {
-                const uint32_t k = keys[i];
-                if (k && (k & mask) == prefix) atomicAdd(&hist[digit(k, level)], 1u);
+            for (int i0 = 0; i0 < n; i0 += kFinThreads) {
+                const int i = i0 + threadIdx.x;
+                const uint32_t k = i < n ? keys[i] : 0u;
+                warp_hist_add(hist, k && (k & mask) == prefix, digit(k, level));
             }
         }
         __syncthreads();
@@ -427,21 +437,24 @@ cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_
             e = cudaFuncSetAttribute(k_sel_small, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
         }
-        k_sel_small<<<nseg, kFinThreads, smem, st>>>(src, n_out, out, out_stride);
-        return cudaGetLastError();
+        return launch_pdl(k_sel_small, dim3(nseg), dim3(kFinThreads), smem, st, src, n_out, out, out_stride);
     }
     // the histograms and counters are zero on entry (workspace initialisation,
     // then every k_sel_finish clears what its selection used); without a
     // histogram from the scoring kernel, build level 1 here
     const unsigned chunks = (unsigned)((src.n + kPassChunk - 1) / kPassChunk);
     dim3 grid(chunks ? chunks : 1, (unsigned)nseg);
-    if (!hist_ready) k_sel_hist<<<grid, kPassThreads, 0, st>>>(src, wk);
-    k_sel_pass1<<<grid, kPassThreads, 0, st>>>(src, wk, n_out, out, out_stride);
+    if (!hist_ready) {
+        e = launch_pdl(k_sel_hist, dim3(grid), dim3(kPassThreads), 0, st, src, wk);
+        if (e != cudaSuccess) return e;
+    }
+    e = launch_pdl(k_sel_pass1, dim3(grid), dim3(kPassThreads), 0, st, src, wk, n_out, out, out_stride);
+    if (e != cudaSuccess) return e;
     // level-1 candidates: at most the segment size; spread over up to 148 CTAs
     const unsigned g2 = chunks < 148 ? (chunks ? chunks : 1) : 148;
-    k_sel_pass2<<<dim3(g2, (unsigned)nseg), kPassThreads, 0, st>>>(wk, n_out, out, out_stride);
-    k_sel_finish<<<nseg, kFinThreads, 0, st>>>(wk, n_out, out, out_stride);
-    return cudaGetLastError();
+    e = launch_pdl(k_sel_pass2, dim3(g2, (unsigned)nseg), dim3(kPassThreads), 0, st, wk, n_out, out, out_stride);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_sel_finish, dim3(nseg), dim3(kFinThreads), 0, st, wk, n_out, out, out_stride);
 }
 
 }  // namespace csa2
