@@ -11,22 +11,26 @@
 // are the MMA's A operand exactly as stored: TMA tensor loads (64 positions =
 // one page run per box, 64-byte swizzle, no multicast) fill a ring of
 // 128-position tiles that tcgen05.mma reads directly.  The bf16 queries become
-// four 8-bit operands whose sum is the query exactly: per (token, head) row the
-// values are scaled by a power of two so the row maximum lies in [128, 256),
-// then q = t1 + t2 + t3 + t4 with t1 = E4M3(q), t2..t4 = E5M2 of the running
-// remainder (round to nearest).  A bf16 value has 8 significant bits; E4M3
-// takes 4 and each E5M2 term 3, so the remainder is 0 for every value at or
-// above 2^-16 of the row maximum (E5M2 reaches down to 2^-16 after scaling).
-// Eight MMAs per tile (4 terms x K=2x32) accumulate q.k in fp32.
+// U E4M3 operands stacked along N: per (token, head) row the values are scaled
+// by a power of two so the row maximum lies in [128, 256), then
+//     t0 = E4M3(q),  t1 = E4M3(16 (q - t0)),  t2 = E4M3(256 (q - t0 - t1/16))
+// (round to nearest), so q = t0 + t1/16 + t2/256.  A bf16 value has 8
+// significant bits and each term takes 4, so the sum is exact for every value
+// at or above 2^-14 of the row maximum, and off by at most 2^-25 of it below
+// (U = 3; U = 2 when 3 N would not fit: exact above 2^-14, off by at most
+// 2^-21 below).  Two MMAs per tile (K = 2 x 32, N = U x T x H_I) accumulate the
+// term products in fp32; the epilogue adds the term columns with their exact
+// power-of-two weights.
 //
 //   producer warp  : TMA loads into the ring (bounded mbarrier waits)
-//   MMA warp       : tcgen05.mma, commits that free ring stages and fill the
+//   MMA warp       : two tcgen05.mma and one commit per tile into a
 //                    double-buffered TMEM accumulator
-//   epilogue warps : two warpgroups, one per TMEM accumulator, so tile g is
-//                    finished by warpgroup g % 2; they stage the query terms
-//                    when the sequence changes; per tile tcgen05.ld of each
-//                    position's row, ReLU + head-weighted sum, fp32 score
-//                    store, level-1 radix histogram in smem.
+//   epilogue warps : two warpgroups, one per TMEM accumulator (tile g is
+//                    finished by warpgroup g % 2); the first thread to see a
+//                    tile's accumulator releases its ring stage; they stage
+//                    the query terms when the sequence changes; per tile
+//                    tcgen05.ld of each position's row, ReLU + head-weighted
+//                    sum, fp32 score store, level-1 radix histogram in smem.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -41,7 +45,7 @@ constexpr int kTile = 128;
 constexpr int kItemTiles = 4;
 constexpr int kStages = 8;
 constexpr int kStageBytes = kTile * 64;   // two 64-row boxes of E4M3 keys
-constexpr int kTerms = 4;
+constexpr int kMaxTerms = 3;
 constexpr int kThreads = 320;
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;   // epilogue: warps 2-9, two warpgroups
 constexpr int kEpiThreads = 256;
@@ -51,7 +55,8 @@ struct Params {
     DevCache c;
     const __nv_bfloat16* q;  // [B][T][H_I][64]
     const float* hw;         // [B][T][H_I]
-    int T, H_I, HP, NP;      // HP: H_I rounded up to 16; NP = T * HP (MMA N)
+    int T, H_I, HP, NP;      // HP: H_I rounded up to 16; NP = T * HP columns per term
+    int U;                   // query terms stacked along N (MMA N = U * NP)
     float* scores;           // [(b*T + j) * cap + t]
     uint32_t* hist;          // [(b*T + j)][3][kRadixBins]; level 1 accumulated here; nullable
     uint32_t* status;
@@ -82,7 +87,7 @@ __device__ __forceinline__ bool get_item(const Params& p, int64_t item, Item& it
 }
 
 struct Bars {
-    uint64_t full[kStages], empty[kStages];
+    uint64_t full[kStages], empty[kStages];   // empty: released by the epilogue
     uint64_t acc_full[2], acc_empty[2];
     uint64_t b_ready[2], b_free[2];
     uint64_t hist_done, hist_clear;
@@ -96,22 +101,11 @@ __device__ __forceinline__ float e4m3_round(float x, uint8_t* code) {
     return e4m3_to_float(*code);
 }
 
-__device__ __forceinline__ float e5m2_round(float x, uint8_t* code) {
-    uint16_t c;
-    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(c) : "f"(0.0f), "f"(x));
-    *code = (uint8_t)(c & 0xFF);
-    uint32_t h;
-    const uint16_t in = c & 0xFF;
-    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(in));
-    return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFF)));
-}
-
-// The four 8-bit query operands of one sequence, NP rows each (row c = token
-// j * HP + head h; padding rows are zero), plus the folded weights
-// w * 2^-e.  4 threads per row, 16 values each.
+// The U 8-bit query operands of one sequence, stacked: row u * NP + c holds
+// term u of row c (c = token j * HP + head h; padding rows are zero); plus the
+// folded weights w * 2^-e.  4 threads per row, 16 values each.
 __device__ void prepare_queries(const Params& p, int b, uint8_t* bq, float* wq, int tid) {
     const int row_in_pass = tid >> 2, quarter = tid & 3;
-    const int term_bytes = p.NP * 64;
     for (int r0 = 0; r0 < p.NP; r0 += 32) {
         const int c = r0 + row_in_pass;
         const int j = c / p.HP, h = c - j * p.HP;
@@ -145,23 +139,28 @@ __device__ void prepare_queries(const Params& p, int b, uint8_t* bq, float* wq, 
         const float up = __uint_as_float((uint32_t)(127 + e) << 23);
         const float down = __uint_as_float((uint32_t)(127 - e) << 23);
         if (c < p.NP) {
-            uint8_t t[kTerms][16];
+            uint8_t t[kMaxTerms][16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                float r = v[k] * up;                       // exact: a power-of-two scale
-                r -= e4m3_round(r, &t[0][k]);              // exact: both are fp32 values
-                r -= e5m2_round(r, &t[1][k]);
-                r -= e5m2_round(r, &t[2][k]);
-                e5m2_round(r, &t[3][k]);
+                float r = v[k] * up;                        // exact: a power-of-two scale
+#pragma unroll
+                for (int u = 0; u < kMaxTerms; ++u) {
+                    // term u carries the remainder scaled by 16^u (exact); the
+                    // remainder update subtracts its exact value
+                    const float scale = (float)(1 << (4 * u));
+                    const float tv = e4m3_round(r * scale, &t[u][k]);
+                    r -= tv / scale;
+                }
             }
 #pragma unroll
-            for (int u = 0; u < kTerms; ++u) {
+            for (int u = 0; u < kMaxTerms; ++u) {
+                if (u >= p.U) break;
                 uint32_t wds[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     wds[k] = (uint32_t)t[u][4 * k] | ((uint32_t)t[u][4 * k + 1] << 8) |
                              ((uint32_t)t[u][4 * k + 2] << 16) | ((uint32_t)t[u][4 * k + 3] << 24);
-                *reinterpret_cast<uint4*>(bq + u * term_bytes + tc::sw64_offset(c, quarter)) =
+                *reinterpret_cast<uint4*>(bq + tc::sw64_offset(u * p.NP + c, quarter)) =
                     make_uint4(wds[0], wds[1], wds[2], wds[3]);
             }
             if (quarter == 0) wq[c] = real ? __ldg(p.hw + ((int64_t)b * p.T + j) * p.H_I + h) * down : 0.0f;
@@ -180,11 +179,13 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
     float* sWq = reinterpret_cast<float*>(smem + p.off_wq);
     Bars* bars = reinterpret_cast<Bars*>(smem + p.off_bar);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bq_bytes = kTerms * p.NP * 64;
+    const int bq_bytes = p.U * p.NP * 64;
+    const int NA = p.U * p.NP;                  // accumulator columns per tile
 
     for (int i = threadIdx.x; i < p.T * kRadixBins; i += kThreads) sHist[i] = 0;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) { tc::mbar_init(&bars->full[i], 1); tc::mbar_init(&bars->empty[i], 1); }
+        // empty[s] is arrived by the one epilogue thread that first sees the tile's accumulator
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars->acc_full[i], 1);
             tc::mbar_init(&bars->acc_empty[i], 128);
@@ -244,9 +245,7 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            uint32_t idesc[kTerms];
-#pragma unroll
-            for (int u = 0; u < kTerms; ++u) idesc[u] = tc::idesc_f8_f32(kTile, p.NP, 0u, u == 0 ? 0u : 1u);
+            const uint32_t idesc = tc::idesc_f8_f32(kTile, NA, 0u, 0u);
             uint32_t g = 0, n = 0;
             int cur_b = -1;
             bool ok = true;
@@ -265,14 +264,9 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                         !tc::mbar_wait(&bars->acc_empty[acc], ((g >> 1) & 1) ^ 1)) { ok = false; break; }
                     tc::fence_after_sync();
                     const uint32_t aa = tc::smem_u32(sRing + s * kStageBytes);
-                    const uint32_t d = tmem + (uint32_t)(acc * p.NP);
-#pragma unroll
-                    for (int u = 0; u < kTerms; ++u)
-#pragma unroll
-                        for (int k = 0; k < 2; ++k)
-                            tc::mma_f8(d, tc::desc_sw64(aa + 32 * k),
-                                       tc::desc_sw64(bq + u * (p.NP * 64) + 32 * k), idesc[u], (u | k) != 0);
-                    tc::mma_commit(&bars->empty[s]);
+                    const uint32_t d = tmem + (uint32_t)(acc * NA);
+                    tc::mma_f8(d, tc::desc_sw64(aa), tc::desc_sw64(bq), idesc, 0u);
+                    tc::mma_f8(d, tc::desc_sw64(aa + 32), tc::desc_sw64(bq + 32), idesc, 1u);
                     tc::mma_commit(&bars->acc_full[acc]);
                 }
             }
@@ -340,38 +334,40 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                 if (acc != grp) continue;                       // the other group's tile
                 if (!warp_wait(&bars->acc_full[acc], (g >> 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
+                // the MMAs of this tile are complete: its ring stage can be refilled
+                if ((tid & 127) == 0) tc::mbar_arrive(&bars->empty[g % kStages]);
                 const int64_t t = it.t0 + (int64_t)tl * kTile + row;
+                const uint32_t abase = lane_addr + (uint32_t)(acc * NA);
                 for (int j = 0; j < p.T; ++j) {
                     float s0 = 0.0f, s1 = 0.0f;
-                    for (int c0 = j * p.HP; c0 < (j + 1) * p.HP; c0 += 32) {
-                        // two 16-column loads in flight, one wait
-                        uint32_t r[32];
-                        const bool two = c0 + 16 < (j + 1) * p.HP;
-                        tc::tmem_ld16_nowait(lane_addr + (uint32_t)(acc * p.NP + c0), r);
-                        if (two) tc::tmem_ld16_nowait(lane_addr + (uint32_t)(acc * p.NP + c0 + 16), r + 16);
+                    for (int c0 = j * p.HP; c0 < (j + 1) * p.HP; c0 += 16) {
+                        // the 16 heads' columns of every term in flight, one wait
+                        uint32_t r[kMaxTerms][16];
+                        tc::tmem_ld16_nowait(abase + (uint32_t)c0, r[0]);
+                        tc::tmem_ld16_nowait(abase + (uint32_t)(p.NP + c0), r[1]);
+                        if (p.U > 2) tc::tmem_ld16_nowait(abase + (uint32_t)(2 * p.NP + c0), r[2]);
                         tc::tmem_ld_wait();
                         const float4* w4 = reinterpret_cast<const float4*>(wq + c0);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            if (i < 4 || two) {
-                                const float4 ww = w4[i];
-                                s0 = fmaf(ww.x, fmaxf(__uint_as_float(r[4 * i]), 0.0f), s0);
-                                s1 = fmaf(ww.y, fmaxf(__uint_as_float(r[4 * i + 1]), 0.0f), s1);
-                                s0 = fmaf(ww.z, fmaxf(__uint_as_float(r[4 * i + 2]), 0.0f), s0);
-                                s1 = fmaf(ww.w, fmaxf(__uint_as_float(r[4 * i + 3]), 0.0f), s1);
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 ww = w4[i];
+                            float dot[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                float x = fmaf(__uint_as_float(r[1][4 * i + k]), 0.0625f, __uint_as_float(r[0][4 * i + k]));
+                                if (p.U > 2) x = fmaf(__uint_as_float(r[2][4 * i + k]), 0.00390625f, x);
+                                dot[k] = fmaxf(x, 0.0f);
                             }
+                            s0 = fmaf(ww.x, dot[0], s0);
+                            s1 = fmaf(ww.y, dot[1], s1);
+                            s0 = fmaf(ww.z, dot[2], s0);
+                            s1 = fmaf(ww.w, dot[3], s1);
                         }
                     }
                     const float s = s0 + s1;
                     const bool vis = t <= it.L - p.T + j;
                     if (vis) p.scores[((int64_t)it.b * p.T + j) * p.c.cap + t] = s;
-                    if (p.hist) {
-                        // lanes that hit the same bin add once (scores crowd into few bins)
-                        const uint32_t bin = vis ? (ordered_key(s) >> 21) : 0xFFFFFFFFu;
-                        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-                        if (vis && lane == __ffs(peers) - 1)
-                            atomicAdd(&sHist[j * kRadixBins + bin], (uint32_t)__popc(peers));
-                    }
+                    if (p.hist && vis) atomicAdd(&sHist[j * kRadixBins + (ordered_key(s) >> 21)], 1u);
                 }
                 tc::fence_before_sync();
                 tc::mbar_arrive(&bars->acc_empty[acc]);
@@ -393,11 +389,13 @@ struct SmemPlan {
     uint32_t off_b, off_hist, off_wq, off_bar, total;
 };
 
+int n_terms(int NP) { return 3 * NP <= 256 ? 3 : 2; }
+
 SmemPlan smem_plan(int T, int NP) {
     SmemPlan s;
     uint32_t off = kStages * kStageBytes;
     s.off_b = off;
-    off += 2 * kTerms * NP * 64;
+    off += 2 * n_terms(NP) * NP * 64;
     s.off_hist = off;
     off += T * kRadixBins * 4;
     s.off_wq = off;
@@ -430,7 +428,7 @@ EncodeTiled encode_fn() {
 
 bool score_full_tc_supported(const DevCache& c, int T, int H_I) {
     const int HP = (H_I + 15) / 16 * 16;
-    return c.key_dtype == 2 && c.idx_dim == 64 && T * HP <= 256 && smem_plan(T, T * HP).total <= 227 * 1024 &&
+    return c.key_dtype == 2 && c.idx_dim == 64 && 2 * T * HP <= 256 && smem_plan(T, T * HP).total <= 227 * 1024 &&
            c.n_slots < ((int64_t)1 << 31) && encode_fn() != nullptr;
 }
 
@@ -444,6 +442,7 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
     p.H_I = H_I;
     p.HP = (H_I + 15) / 16 * 16;
     p.NP = T * p.HP;
+    p.U = n_terms(p.NP);
     p.scores = scores;
     p.hist = hist;
     p.status = status;
@@ -451,7 +450,7 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
     p.items_per_seq = (tiles_cap + kItemTiles - 1) / kItemTiles;
     p.total_items = p.items_per_seq * c.batch;
     uint32_t cols = 32;
-    while (cols < (uint32_t)(2 * p.NP)) cols <<= 1;
+    while (cols < (uint32_t)(2 * p.U * p.NP)) cols <<= 1;
     p.tmem_cols = cols;
     const SmemPlan sp = smem_plan(T, p.NP);
     p.off_b = sp.off_b;
@@ -474,7 +473,8 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
 
     cudaError_t e = cudaFuncSetAttribute(k_score_full_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
     if (e != cudaSuccess) return e;
-    int64_t grid = 2 * (int64_t)num_sms;   // two CTAs per SM
+    // two CTAs per SM when their accumulators fit in TMEM together
+    int64_t grid = (cols <= 256 ? 2 : 1) * (int64_t)num_sms;
     if (grid > p.total_items) grid = p.total_items;
     if (grid < 1) grid = 1;
     return launch_pdl(k_score_full_tc, dim3((unsigned)grid), dim3(kThreads), sp.total, st, tmap, p);
