@@ -20,8 +20,8 @@ F32, BF16, E4M3 = 0, 1, 2
 
 ABI_FUNCTIONS = (
     "csa2_workspace_bytes", "csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
-    "csa2_index_reindex", "csa2_sparse_swa_attn", "csa2_layer_step", "csa2_read_device_status",
-    "csa2_status_string",
+    "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_sparse_swa_attn", "csa2_layer_step",
+    "csa2_read_device_status", "csa2_status_string",
 )
 
 
@@ -70,13 +70,14 @@ def lib():
         L.csa2_index_scores.argtypes = [cp, vp, i32, vp, i32, i32, vp, vp, sz, vp]
         L.csa2_index_full.argtypes = [cp, vp, i32, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
         L.csa2_index_reindex.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, vp, vp, sz, vp]
+        L.csa2_index_reindex_noalloc.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, vp, vp]
         L.csa2_sparse_swa_attn.argtypes = [cp, vp, i32, i32, vp, i32, i32, ctypes.c_float, vp, vp, vp, sz, vp]
         L.csa2_layer_step.argtypes = [cp, ctypes.POINTER(csa2_layer_args), vp, sz, vp]
         L.csa2_read_device_status.argtypes = [vp, vp]
         L.csa2_status_string.restype = ctypes.c_char_p
         L.csa2_status_string.argtypes = [i32]
         for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
-                     "csa2_index_reindex",
+                     "csa2_index_reindex", "csa2_index_reindex_noalloc",
                      "csa2_sparse_swa_attn", "csa2_layer_step", "csa2_read_device_status"):
             getattr(L, name).restype = i32
         _lib = L
@@ -196,6 +197,15 @@ def index_reindex(cache, q_idx, head_w, pool_idx, top_k, topk_idx, ws, stream=No
     _check(lib().csa2_index_reindex(cache.ref, _p(q_idx), _qdt(q_idx), _p(head_w), T, H_I, _p(pool_idx),
                                     pool_idx.shape[-1], top_k, _p(topk_idx), _p(ws), ws.numel() * ws.element_size(),
                                     _stream(stream)), "index_reindex")
+
+
+def index_reindex_noalloc(cache, q_idx, head_w, pool_idx, top_k, topk_idx, stream=None):
+    """csa2_index_reindex for callers that cannot hand over a workspace: the
+    scratch is a fixed array inside the library (see include/csa2.h)."""
+    B, T, H_I, _ = q_idx.shape
+    _check(lib().csa2_index_reindex_noalloc(cache.ref, _p(q_idx), _qdt(q_idx), _p(head_w), T, H_I, _p(pool_idx),
+                                            pool_idx.shape[-1], top_k, _p(topk_idx), _stream(stream)),
+           "index_reindex_noalloc")
 
 
 def sparse_swa_attn(cache, q, topk_idx, window, out, lse=None, ws=None, sm_scale=0.0, stream=None):

@@ -185,6 +185,29 @@ CSA2_API csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_i
                                void* stream);
 
 /*
+ * csa2_index_reindex without a workspace, for callers that cannot allocate
+ * device memory: code running while a framework captures a CUDA graph under a
+ * no-allocation policy, plugins handed tensors but no allocator, or real-time
+ * paths that cannot pay for cudaMalloc's implicit synchronisation.  The pages
+ * describe no such call; it is a convenience of this library.
+ *
+ * Same arguments and results as csa2_index_reindex, minus ws / ws_bytes.  The
+ * scratch lives in a 4 MiB array inside the library's own device memory (held
+ * by every GPU that loads the library until the process exits), so
+ * batch * T * pool_k must not exceed 1,048,512; larger problems return
+ * CSA2_ERR_UNSUPPORTED before anything is launched.  The first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress, with the
+ * device current), so make the first call on each device before any stream
+ * capture.  Every call on a device shares the one array: calls whose work may
+ * overlap on the GPU (different streams without ordering between them) race
+ * and must not be issued.  Device-detected bound violations are skipped; this
+ * variant has no status word the caller can read.
+ */
+CSA2_API csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
+                                                const float* head_w, int T, int H_I, const int32_t* pool_idx,
+                                                int pool_k, int top_k, int32_t* topk_idx, void* stream);
+
+/*
  * Sparse + sliding-window attention ([HN] key point 2; [TLDR] paragraphs 2-3).
  * For query token j of sequence b at p = seq_lens[b] - T + j, the attended set
  * is S = window ∪ topk without double counting, with window = [max(0, p -
