@@ -278,11 +278,13 @@ csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, in
     if (!q_bf16 || !out || !aligned16(q_bf16) || !aligned16(out) || (lse && !aligned16(lse))) return CSA2_ERR_INVALID_ARG;
     if (T < 1 || H < 1 || top_k < 0 || window < 0 || window > kMaxPool || top_k > kMaxPool) return CSA2_ERR_INVALID_ARG;
     if (top_k > 0 && (!topk_idx || !aligned16(topk_idx))) return CSA2_ERR_INVALID_ARG;
-    if (H > 64) return CSA2_ERR_UNSUPPORTED;
+    if (H > 64 || H % 16) return CSA2_ERR_UNSUPPORTED;
     if (!std::isfinite(sm_scale)) return CSA2_ERR_INVALID_ARG;
     Layout L;
     s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
+    // the split-softmax merge keeps one weight per (chunk, head) in shared memory
+    if ((size_t)L.nchunk * H * sizeof(float) + 2 * H * sizeof(float) > 200 * 1024) return CSA2_ERR_UNSUPPORTED;
     if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
     AttnWork aw;
     aw.part_o = at<float>(ws, L.part_o);

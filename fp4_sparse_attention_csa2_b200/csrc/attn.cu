@@ -111,7 +111,7 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
 #pragma unroll
         for (int i = 0; i < kRows / 4; ++i) {
             const int r = rg + 4 * i;
-            ps[h * kRows + r] = pos[r] >= 0 ? acc[i] * scale : -INFINITY;
+            ps[h * kRows + r] = pos[r] >= 0 ? acc[i] * scale * 1.4426950408889634f : -INFINITY;   // base 2
         }
     }
     __syncthreads();
@@ -123,7 +123,7 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
         for (int r = 0; r < kRows; ++r) m = fmaxf(m, ps[h * kRows + r]);
         float l = 0.0f;
         for (int r = 0; r < kRows; ++r) {
-            const float e = m == -INFINITY ? 0.0f : __expf(ps[h * kRows + r] - m);
+            const float e = m == -INFINITY ? 0.0f : exp2f(ps[h * kRows + r] - m);
             ps[h * kRows + r] = e;
             l += e;
         }
@@ -146,73 +146,75 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
             acc.z = fmaf(e, vv.z, acc.z);
             acc.w = fmaf(e, vv.w, acc.w);
         }
-        *reinterpret_cast<float4*>(po + (int64_t)h * D + d) = acc;
+        po[(int64_t)(d + 0) * H + h] = acc.x;   // partials are [d][head]
+        po[(int64_t)(d + 1) * H + h] = acc.y;
+        po[(int64_t)(d + 2) * H + h] = acc.z;
+        po[(int64_t)(d + 3) * H + h] = acc.w;
     }
 }
 
-// grid (batch*T, H); block 128: merge the chunk partials of one head.
-__global__ void __launch_bounds__(128)
+// Split-softmax merge.  grid (batch*T, D/64), 256 threads; dynamic smem holds
+// the weight of every (chunk, head), 2^(m_c - M) with M the head's maximum
+// over chunks, and the heads' totals.  Thread t covers channel 64*blockIdx.y +
+// t/4 and a quarter of the heads; partials are [chunk][d][head], base 2.
+__global__ void __launch_bounds__(256)
 k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk,
                float* __restrict__ out, float* __restrict__ lse) {
     pdl_begin();
-    const int seg = blockIdx.x, h = blockIdx.y;
-    __shared__ float s_w[1024];
-    __shared__ float s_red[4];
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    float m = -INFINITY;
-    for (int ch = tid; ch < nchunk; ch += 128) m = fmaxf(m, part_ml[(((int64_t)seg * nchunk + ch) * H + h) * 2]);
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) s_red[wid] = m;
-    __syncthreads();
-    m = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-    __syncthreads();
-    float l = 0.0f;
-    for (int ch = tid; ch < nchunk; ch += 128) {
-        const float* ml = part_ml + (((int64_t)seg * nchunk + ch) * H + h) * 2;
-        const float w = (m == -INFINITY || ml[0] == -INFINITY) ? 0.0f : __expf(ml[0] - m);
-        s_w[ch] = w;
-        l += w * ml[1];
+    extern __shared__ float s_w[];             // [nchunk][H], then M[H], L[H]
+    float* s_M = s_w + (size_t)nchunk * H;
+    float* s_L = s_M + H;
+    const int seg = blockIdx.x, tid = threadIdx.x;
+    for (int h = tid; h < H; h += 256) {
+        const float* ml = part_ml + (int64_t)seg * nchunk * H * 2 + h * 2;
+        float m = -INFINITY;
+        for (int c = 0; c < nchunk; ++c) m = fmaxf(m, ml[(int64_t)c * H * 2]);
+        float l = 0.0f;
+        for (int c = 0; c < nchunk; ++c) {
+            const float mc = ml[(int64_t)c * H * 2];
+            const float w = (m == -INFINITY || mc == -INFINITY) ? 0.0f : exp2f(mc - m);
+            s_w[c * H + h] = w;
+            l = fmaf(w, ml[(int64_t)c * H * 2 + 1], l);
+        }
+        s_M[h] = m;
+        s_L[h] = l;
     }
-    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) s_red[wid] = l;
     __syncthreads();
-    l = s_red[0] + s_red[1] + s_red[2] + s_red[3];
-    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-    // every thread owns up to 4 channels; a masked chunk has weight 0 and a
-    // zero partial, so all loads are unconditional and independent
-    const float* base = part_o + ((int64_t)seg * nchunk * H + h) * D;
-    const int64_t cstride = (int64_t)H * D;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    int ch = 0;
-    for (; ch + 4 <= nchunk; ch += 4) {        // 16 independent loads in flight per thread
-        float v[4][4];
+    const int hq = H / 4;                      // heads per thread (H is a multiple of 16 here)
+    const int d = blockIdx.y * 64 + (tid >> 2);
+    const int h0 = (tid & 3) * hq;
+    if (d >= D) return;
+    float acc[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int d = tid + 128 * k;
-                v[u][k] = d < D ? base[(ch + u) * cstride + d] : 0.0f;
-            }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = fmaf(s_w[ch + u], v[u][k], acc[k]);
-    }
-    for (; ch < nchunk; ++ch) {
-        const float w = s_w[ch];
-        const float* src = base + ch * cstride;
+    for (int k = 0; k < 16; ++k) acc[k] = 0.0f;
+    const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h0;
+    const int64_t cstride = (int64_t)D * H;
+    for (int c = 0; c < nchunk; ++c) {
+        const float4* src = reinterpret_cast<const float4*>(base + c * cstride);
+        const float* w = s_w + c * H + h0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int d = tid + 128 * k;
-            if (d < D) acc[k] = fmaf(w, src[d], acc[k]);
+            if (4 * k < hq) {
+                const float4 v = src[k];
+                acc[4 * k] = fmaf(w[4 * k], v.x, acc[4 * k]);
+                acc[4 * k + 1] = fmaf(w[4 * k + 1], v.y, acc[4 * k + 1]);
+                acc[4 * k + 2] = fmaf(w[4 * k + 2], v.z, acc[4 * k + 2]);
+                acc[4 * k + 3] = fmaf(w[4 * k + 3], v.w, acc[4 * k + 3]);
+            }
         }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int d = tid + 128 * k;
-        if (d < D) out[((int64_t)seg * H + h) * D + d] = acc[k] * inv;
+    for (int k = 0; k < 16; ++k) {
+        if (k < hq) {
+            const int h = h0 + k;
+            const float l = s_L[h];
+            out[((int64_t)seg * H + h) * D + d] = l > 0.0f ? acc[k] / l : 0.0f;
+        }
     }
-    if (lse && tid == 0) lse[(int64_t)seg * H + h] = l > 0.0f ? m + logf(l) : -INFINITY;
+    if (lse && blockIdx.y == 0 && tid < H) {
+        const float l = s_L[tid];
+        lse[(int64_t)seg * H + tid] = l > 0.0f ? s_M[tid] * 0.6931471805599453f + logf(l) : -INFINITY;
+    }
 }
 
 }  // namespace
@@ -221,8 +223,13 @@ int attn_rows_per_chunk() { return kRows; }
 
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st) {
-    return launch_pdl(k_attn_combine, dim3((unsigned)(c.batch * T), (unsigned)H), dim3(128), 0, st, c.dim, H, aw.part_o, aw.part_ml,
-                      aw.nchunk, out, lse);
+    const size_t smem = sizeof(float) * ((size_t)aw.nchunk * H + 2 * (size_t)H);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_attn_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(k_attn_combine, dim3((unsigned)(c.batch * T), (unsigned)((c.dim + 63) / 64)), dim3(256), smem, st,
+                      c.dim, H, aw.part_o, aw.part_ml, aw.nchunk, out, lse);
 }
 
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,

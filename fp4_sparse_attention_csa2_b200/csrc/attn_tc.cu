@@ -18,8 +18,8 @@
 //      positions; P (fp16) written K-major;
 //   4. O^T[d, head] = V^T P^T : the same V bytes read through an MN-major
 //      descriptor, one M=128 slab of d per accumulator;
-//   5. unnormalised partial output and (max, sum) per head to the workspace,
-//      merged by the split-softmax combine kernel.
+//   5. unnormalised partial output ([d][head]) and (max, sum) per head in
+//      base-2 units to the workspace, merged by the split-softmax combine kernel.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -228,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
             uint32_t hv[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const float e0 = m == -INFINITY ? 0.0f : __expf(z[8 * c + 2 * k] - m);
-                const float e1 = m == -INFINITY ? 0.0f : __expf(z[8 * c + 2 * k + 1] - m);
+                const float e0 = m == -INFINITY ? 0.0f : exp2f(z[8 * c + 2 * k] - m);
+                const float e1 = m == -INFINITY ? 0.0f : exp2f(z[8 * c + 2 * k + 1] - m);
                 __half2 hh = __floats2half2_rn(e0, e1);
                 const float2 back = __half22float2(hh);   // sum what the MMA will use
                 l += back.x + back.y;
@@ -267,8 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     ok = __syncthreads_and(ok);
     tc::fence_after_sync();
 
-    // ---- unnormalised partial output (lane = d within the slab; the two
-    // warpgroups take one half of the heads each)
+    // ---- unnormalised partial output, [d][head] (lane = d within the slab; the
+    // two warpgroups take one half of the heads each; 16-byte stores)
     if (ok && wgrp < ngrp) {
         float* po = p.part_o + ((int64_t)seg * p.nchunk + chunk) * H * D;
         const int hc = H / ngrp;
@@ -277,8 +277,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
             for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
                 float v[16];
                 tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(H + s2 * H + c0), v);
+                float4* dst = reinterpret_cast<float4*>(po + (int64_t)d * H + c0);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) po[(int64_t)(c0 + i) * D + d] = v[i];
+                for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             }
         }
     }
@@ -329,7 +330,8 @@ k_attn_stage_q(const __nv_bfloat16* __restrict__ q, int H, int D, float scale, u
             e = e < -100 ? -100 : (e > 100 ? 100 : e);
         }
         const float up = __uint_as_float((uint32_t)(127 + e) << 23);
-        if (part == 0) fac[h] = scale * __uint_as_float((uint32_t)(127 - e) << 23);
+        // logits in base-2 units: softmax_scale * log2(e) / 2^e
+        if (part == 0) fac[h] = scale * 1.4426950408889634f * __uint_as_float((uint32_t)(127 - e) << 23);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             if (8 * i < span) {

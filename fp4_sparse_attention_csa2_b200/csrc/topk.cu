@@ -101,6 +101,15 @@ __device__ __forceinline__ uint32_t warp_sum_hist(const uint32_t* h) {
     return __reduce_add_sync(0xffffffffu, v);
 }
 
+// Copy `levels` consecutive 2048-bin histograms from global to shared memory
+// (coalesced, the whole block), so the threshold scans run on shared memory.
+__device__ __forceinline__ void stage_hist(uint32_t* dst, const uint32_t* src, int levels, int nthreads) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (int i = threadIdx.x; i < levels * kRadixBins / 4; i += nthreads) d4[i] = s4[i];
+    __syncthreads();
+}
+
 // Histogram increment by a whole warp: lanes with the same bin add once.
 __device__ __forceinline__ void warp_hist_add(uint32_t* hist, bool pred, uint32_t bin) {
     const uint32_t key = pred ? bin : 0xFFFFFFFFu;
@@ -148,9 +157,10 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_out, int32_t* __restrict__ out, int64_
     pdl_begin();
     __shared__ uint32_t s_plan[3];   // c1, elements to select, take every digit-c1 element
     __shared__ uint32_t h2[kRadixBins];
+    __shared__ __align__(16) uint32_t h1[kRadixBins];
     const int seg = blockIdx.y;
-    const uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
     uint32_t* cnt = wk.cnt + (int64_t)seg * 4;
+    stage_hist(h1, wk.hist + (int64_t)seg * 3 * kRadixBins, 1, kPassThreads);
     if (threadIdx.x < 32) {
         const uint32_t total = warp_sum_hist(h1);
         const uint32_t need = total < (uint32_t)n_out ? total : (uint32_t)n_out;
@@ -228,11 +238,12 @@ k_sel_pass2(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_stride
     pdl_begin();
     __shared__ Plan2 s_pl;
     __shared__ uint32_t h3[kRadixBins];
+    __shared__ __align__(16) uint32_t h12[2 * kRadixBins];
     const int seg = blockIdx.y;
-    const uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
     uint32_t* cnt = wk.cnt + (int64_t)seg * 4;
+    stage_hist(h12, wk.hist + (int64_t)seg * 3 * kRadixBins, 2, kPassThreads);
     if (threadIdx.x < 32) {
-        const Plan2 pl = plan_level2(h1, h1 + kRadixBins, n_out);
+        const Plan2 pl = plan_level2(h12, h12 + kRadixBins, n_out);
         if (threadIdx.x == 0) s_pl = pl;
     }
     for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads) h3[i] = 0;
@@ -277,17 +288,19 @@ k_sel_finish(SelWork wk, int n_out, int32_t* __restrict__ out, int64_t out_strid
     pdl_begin();
     __shared__ Plan2 s_pl;
     __shared__ uint32_t s_plan[2];
+    __shared__ __align__(16) uint32_t hs[3 * kRadixBins];
     const int seg = blockIdx.x;
     uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
     uint32_t* cnt = wk.cnt + (int64_t)seg * 4;
+    stage_hist(hs, h1, 3, kFinThreads);
     if (threadIdx.x < 32) {
-        const Plan2 pl = plan_level2(h1, h1 + kRadixBins, n_out);
+        const Plan2 pl = plan_level2(hs, hs + kRadixBins, n_out);
         if (threadIdx.x == 0) s_pl = pl;
     }
     __syncthreads();
     const Plan2 pl = s_pl;
     if (pl.run && pl.eq2 != pl.need2) {
-        const uint32_t* h3 = h1 + 2 * kRadixBins;
+        const uint32_t* h3 = hs + 2 * kRadixBins;
         if (threadIdx.x < 32) {
             const uint2 t3 = warp_threshold(h3, pl.need2);
             if (threadIdx.x == 0) {
@@ -341,7 +354,7 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, int64_t out_stride
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
         const int i = k * kFinThreads + threadIdx.x;
-        ids[k] = i < n ? (src.ids ? __ldg(src.ids + seg * src.ids_stride + i) : i) : -1;
+        ids[k] = i < n ? (src.ids ? __ldg(src.ids + seg * src.ids_stride + i) : i) : -1;   // the output id
     }
     float vals[kPer];
 #pragma unroll
@@ -395,14 +408,15 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, int64_t out_stride
         const bool all_eq = eqn == need - above;
         // select the elements of the current prefix whose digit is above c
         // (and those equal to c when exactly the missing number of them exist)
-        for (int i0 = 0; i0 < n; i0 += kFinThreads) {
-            const int i = i0 + threadIdx.x;
-            const uint32_t k = i < n ? keys[i] : 0u;
-            const bool in = k && (k & mask) == prefix;
-            const uint32_t d = (k >> shift) & dmask;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int i = k * kFinThreads + threadIdx.x;
+            const uint32_t key = i < n ? keys[i] : 0u;
+            const bool in = key && (key & mask) == prefix;
+            const uint32_t d = (key >> shift) & dmask;
             const bool take = in && (d > c || (d == c && all_eq));
             const uint32_t os = warp_claim(take, &s_cnt[0]);
-            if (take) o[os] = src.ids ? src.ids[seg * src.ids_stride + i] : i;
+            if (take) o[os] = ids[k];
         }
         if (all_eq) break;
         need -= above;
@@ -413,14 +427,15 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, int64_t out_stride
             __syncthreads();
             if (threadIdx.x == 0) s_cnt[1] = 0;
             __syncthreads();
-            for (int i0 = 0; i0 < n; i0 += kFinThreads) {
-                const int i = i0 + threadIdx.x;
-                const uint32_t k = i < n ? keys[i] : 0u;
-                const bool eq = k && k == prefix;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int i = k * kFinThreads + threadIdx.x;
+                const uint32_t key = i < n ? keys[i] : 0u;
+                const bool eq = key && key == prefix;
                 const uint32_t ts = warp_claim(eq, &s_cnt[1]);
                 const bool take = eq && ts < need;
                 const uint32_t os = warp_claim(take, &s_cnt[0]);
-                if (take) o[os] = src.ids ? src.ids[seg * src.ids_stride + i] : i;
+                if (take) o[os] = ids[k];
             }
         }
     }

@@ -217,7 +217,8 @@ CSA2_API csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const v
  *     z_t   = sm_scale * q[b][j][h] . v_t          (sm_scale <= 0: 1/sqrt(dim))
  *     out   = sum_{t in S} softmax(z)_t v_t        fp32 [batch][T][H][dim]
  *     lse   = log sum_{t in S} exp(z_t)            fp32 [batch][T][H], nullable
- * q is bf16 [batch][T][H][dim].  An empty S gives out = 0, lse = -inf.
+ * q is bf16 [batch][T][H][dim] with H a multiple of 16, at most 64.  An empty
+ * S gives out = 0, lse = -inf.
  * topk entries < -1 or >= seq_lens[b] set CSA2_ERR_DEVICE_BOUNDS.
  */
 CSA2_API csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, int T, int H,
