@@ -31,7 +31,8 @@ from fp4_sparse_attention_csa2_b200.runner import Stack, build_replicas  # noqa:
 
 METRIC = "CSA2 decode layer-steps/s at 1M ctx; FP4-KV achieved HBM GB/s vs 8 TB/s"
 PROFILE = os.path.join(ROOT, "profiles", "index_score_ctx1m.md")
-SCORE_SOURCES = ["fp4_sparse_attention_csa2_b200/csrc/index.cu", "fp4_sparse_attention_csa2_b200/csrc/common.cuh"]
+SCORE_SOURCES = ["fp4_sparse_attention_csa2_b200/csrc/index_tc.cu", "fp4_sparse_attention_csa2_b200/csrc/tc.cuh",
+                 "fp4_sparse_attention_csa2_b200/csrc/common.cuh"]
 
 
 def peaks():
