@@ -76,7 +76,7 @@ int num_sms() {
 // The radix histograms and counters are zero between calls: the workspace
 // starts zeroed and every large selection clears what it used.
 struct Layout {
-    size_t status, scores, hist, hist_scratch, cnt, cand1, cand2, pscores, part_o, part_ml, qstage, total;
+    size_t status, scores, hist, hist_scratch, cnt, cand1, cand2, pscores, part_o, part_ml, total;
     int64_t nseg, cap, cand_stride;
     int nchunk;
 };
@@ -99,7 +99,6 @@ bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int w
     L->pscores = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * pool_k);
     L->part_o = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * c->dim);
     L->part_ml = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * 2);
-    L->qstage = off; off = align_up(off + (size_t)L->nseg * attn_tc_qstage_bytes(c->dim, H));
     L->total = off;
     return true;
 }
@@ -246,10 +245,13 @@ csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dty
     src.seq_lens = cache->seq_lens;
     src.T = T;
     src.cap = L.cap;
-    cudaError_t e = launch_select(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, pool_k, st, fused);
+    // the pool's scores come out beside its indices, so the top-k below reads
+    // them contiguously instead of gathering from the full score array
+    float* ps = at<float>(ws, L.pscores);
+    cudaError_t e = launch_select(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, pool_k, st, fused, ps);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
     // this layer's top-k: the top_k best of the same scores, taken from the pool
-    return topk_from_pool(cache, L, ws, scores, L.cap, 1, pool_idx, pool_k, top_k, topk_idx, T, st);
+    return topk_from_pool(cache, L, ws, ps, pool_k, 0, pool_idx, pool_k, top_k, topk_idx, T, st);
 }
 
 csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
@@ -284,15 +286,14 @@ csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, in
     s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
     // the split-softmax merge keeps one weight per (chunk, head) in shared memory
-    if ((size_t)L.nchunk * H * sizeof(float) + 2 * H * sizeof(float) > 200 * 1024) return CSA2_ERR_UNSUPPORTED;
+    if ((size_t)L.nchunk * H * sizeof(float) + 2 * H * sizeof(float) + 1024 > 200 * 1024) return CSA2_ERR_UNSUPPORTED;
     if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
     AttnWork aw;
     aw.part_o = at<float>(ws, L.part_o);
     aw.part_ml = at<float>(ws, L.part_ml);
-    aw.qstage = at<uint8_t>(ws, L.qstage);
     aw.nchunk = L.nchunk;
     return cuda_status(launch_attention(dev_cache(cache), q_bf16, T, H, topk_idx, top_k, window, sm_scale, out, lse,
-                                        aw, at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream)));
+                                        aw, at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream), num_sms()));
 }
 
 csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* a, void* ws, size_t ws_bytes,

@@ -153,67 +153,86 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
     }
 }
 
-// Split-softmax merge.  grid (batch*T, D/64), 256 threads; dynamic smem holds
+// Split-softmax merge.  grid (batch*T, D/16), 256 threads; dynamic smem holds
 // the weight of every (chunk, head), 2^(m_c - M) with M the head's maximum
-// over chunks, and the heads' totals.  Thread t covers channel 64*blockIdx.y +
-// t/4 and a quarter of the heads; partials are [chunk][d][head], base 2.
+// over chunks, and the heads' totals.  Thread t covers channel
+// 16*blockIdx.y + t/16 and heads [4 (t%16), 4 (t%16) + 4); partials are
+// [chunk][d][head], base 2.
 __global__ void __launch_bounds__(256)
 k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk,
                float* __restrict__ out, float* __restrict__ lse) {
     pdl_begin();
-    extern __shared__ float s_w[];             // [nchunk][H], then M[H], L[H]
+    extern __shared__ float s_w[];             // [nchunk][H], then M[H], L[H], per-thread partials [256/H][H]
     float* s_M = s_w + (size_t)nchunk * H;
     float* s_L = s_M + H;
+    float* s_red = s_L + H;
     const int seg = blockIdx.x, tid = threadIdx.x;
-    for (int h = tid; h < H; h += 256) {
-        const float* ml = part_ml + (int64_t)seg * nchunk * H * 2 + h * 2;
-        float m = -INFINITY;
-        for (int c = 0; c < nchunk; ++c) m = fmaxf(m, ml[(int64_t)c * H * 2]);
-        float l = 0.0f;
-        for (int c = 0; c < nchunk; ++c) {
-            const float mc = ml[(int64_t)c * H * 2];
-            const float w = (m == -INFINITY || mc == -INFINITY) ? 0.0f : exp2f(mc - m);
-            s_w[c * H + h] = w;
-            l = fmaf(w, ml[(int64_t)c * H * 2 + 1], l);
-        }
+    const float* ml = part_ml + (int64_t)seg * nchunk * H * 2;
+    // per head, 256/H threads share the chunks: maximum, then weights and total
+    // (threads past per_head * H, which exist when H does not divide 256, idle)
+    const int per_head = 256 / H, h = tid % H, part = tid / H;
+    const int c_end = part < per_head ? nchunk : 0;
+    float m = -INFINITY;
+    for (int c = part; c < c_end; c += per_head) m = fmaxf(m, ml[((int64_t)c * H + h) * 2]);
+    if (part < per_head) s_red[part * H + h] = m;
+    __syncthreads();
+    m = -INFINITY;
+    for (int k = 0; k < per_head; ++k) m = fmaxf(m, s_red[k * H + h]);
+    __syncthreads();
+    float l = 0.0f;
+    for (int c = part; c < c_end; c += per_head) {
+        const float mc = ml[((int64_t)c * H + h) * 2];
+        const float w = (m == -INFINITY || mc == -INFINITY) ? 0.0f : exp2f(mc - m);
+        s_w[c * H + h] = w;
+        l = fmaf(w, ml[((int64_t)c * H + h) * 2 + 1], l);
+    }
+    if (part < per_head) s_red[part * H + h] = l;
+    __syncthreads();
+    if (part == 0) {
+        float tot = 0.0f;
+        for (int k = 0; k < per_head; ++k) tot += s_red[k * H + h];
         s_M[h] = m;
-        s_L[h] = l;
+        s_L[h] = tot;
     }
     __syncthreads();
-    const int hq = H / 4;                      // heads per thread (H is a multiple of 16 here)
-    const int d = blockIdx.y * 64 + (tid >> 2);
-    const int h0 = (tid & 3) * hq;
-    if (d >= D) return;
-    float acc[16];
+    const int d = blockIdx.y * 16 + (tid >> 4);
+    const int h0 = (tid & 15) * 4;
+    if (d < D && h0 < H) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h0;
+        const int64_t cstride = (int64_t)D * H;
+        int c = 0;
+        for (; c + 4 <= nchunk; c += 4) {       // four chunks of loads in flight
+            float4 v[4];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.0f;
-    const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h0;
-    const int64_t cstride = (int64_t)D * H;
-    for (int c = 0; c < nchunk; ++c) {
-        const float4* src = reinterpret_cast<const float4*>(base + c * cstride);
-        const float* w = s_w + c * H + h0;
+            for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const float4*>(base + (c + u) * cstride);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            if (4 * k < hq) {
-                const float4 v = src[k];
-                acc[4 * k] = fmaf(w[4 * k], v.x, acc[4 * k]);
-                acc[4 * k + 1] = fmaf(w[4 * k + 1], v.y, acc[4 * k + 1]);
-                acc[4 * k + 2] = fmaf(w[4 * k + 2], v.z, acc[4 * k + 2]);
-                acc[4 * k + 3] = fmaf(w[4 * k + 3], v.w, acc[4 * k + 3]);
+            for (int u = 0; u < 4; ++u) {
+                const float* w = s_w + (c + u) * H + h0;
+                acc.x = fmaf(w[0], v[u].x, acc.x);
+                acc.y = fmaf(w[1], v[u].y, acc.y);
+                acc.z = fmaf(w[2], v[u].z, acc.z);
+                acc.w = fmaf(w[3], v[u].w, acc.w);
             }
         }
-    }
+        for (; c < nchunk; ++c) {
+            const float4 v = *reinterpret_cast<const float4*>(base + c * cstride);
+            const float* w = s_w + c * H + h0;
+            acc.x = fmaf(w[0], v.x, acc.x);
+            acc.y = fmaf(w[1], v.y, acc.y);
+            acc.z = fmaf(w[2], v.z, acc.z);
+            acc.w = fmaf(w[3], v.w, acc.w);
+        }
+        const float a[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        if (k < hq) {
-            const int h = h0 + k;
-            const float l = s_L[h];
-            out[((int64_t)seg * H + h) * D + d] = l > 0.0f ? acc[k] / l : 0.0f;
+        for (int k = 0; k < 4; ++k) {
+            const float lt = s_L[h0 + k];
+            out[((int64_t)seg * H + h0 + k) * D + d] = lt > 0.0f ? a[k] / lt : 0.0f;
         }
     }
     if (lse && blockIdx.y == 0 && tid < H) {
-        const float l = s_L[tid];
-        lse[(int64_t)seg * H + tid] = l > 0.0f ? s_M[tid] * 0.6931471805599453f + logf(l) : -INFINITY;
+        const float lt = s_L[tid];
+        lse[(int64_t)seg * H + tid] = lt > 0.0f ? s_M[tid] * 0.6931471805599453f + logf(lt) : -INFINITY;
     }
 }
 
@@ -223,25 +242,25 @@ int attn_rows_per_chunk() { return kRows; }
 
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st) {
-    const size_t smem = sizeof(float) * ((size_t)aw.nchunk * H + 2 * (size_t)H);
+    const size_t smem = sizeof(float) * ((size_t)aw.nchunk * H + 2 * (size_t)H + 256);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_attn_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(k_attn_combine, dim3((unsigned)(c.batch * T), (unsigned)((c.dim + 63) / 64)), dim3(256), smem, st,
+    return launch_pdl(k_attn_combine, dim3((unsigned)(c.batch * T), (unsigned)((c.dim + 15) / 16)), dim3(256), smem, st,
                       c.dim, H, aw.part_o, aw.part_ml, aw.nchunk, out, lse);
 }
 
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
                              int window, float sm_scale, float* out, float* lse, const AttnWork& aw_in,
-                             uint32_t* status, cudaStream_t st) {
+                             uint32_t* status, cudaStream_t st, int num_sms) {
     AttnWork aw = aw_in;
     cudaError_t e;
     if (attn_tc_supported(c, H)) {
         const int rows = attn_tc_rows_per_chunk();
         aw.nchunk = (window + top_k + rows - 1) / rows;
         if (aw.nchunk < 1) aw.nchunk = 1;
-        e = launch_attention_tc(c, q, T, H, topk, top_k, window, sm_scale, aw, status, st);
+        e = launch_attention_tc(c, q, T, H, topk, top_k, window, sm_scale, aw, status, st, num_sms);
     } else {
         const int D = c.dim;
         aw.nchunk = (window + top_k + kRows - 1) / kRows;

@@ -8,12 +8,15 @@
 // value of every head).
 //
 // One CTA owns 128 entries of the (window ++ top-k) list of one (sequence,
-// query token) -- a top-k entry that is -1, beyond p or inside the window is
-// masked, so the attended set is window ∪ top-k without double counting:
+// query token) and one group of HG heads (HG = 16, 32 or H: fewer heads per
+// CTA when the (chunk, segment) grid alone would leave SMs idle) -- a top-k
+// entry that is -1, beyond p or inside the window is masked, so the attended
+// set is window ∪ top-k without double counting:
 //   1. gather the FP4 rows (16-byte loads), dequantise exactly to fp16 into a
-//      128 x D tile laid out K-major with the 128-byte swizzle; stage the
-//      queries as fp16 scaled by a power of two per head (exact);
-//   2. S[pos, head] = V Q^T : tcgen05.mma M=128 (positions), N=H, K=D;
+//      128 x D tile laid out K-major with the 128-byte swizzle; meanwhile
+//      convert the group's bf16 queries to fp16 scaled by a power of two per
+//      head (exact) in the same layout;
+//   2. S[pos, head] = V Q^T : tcgen05.mma M=128 (positions), N=HG, K=D;
 //   3. logits to shared memory transposed; per-head max and exp over the 128
 //      positions; P (fp16) written K-major;
 //   4. O^T[d, head] = V^T P^T : the same V bytes read through an MN-major
@@ -36,22 +39,19 @@ struct Params {
     DevCache c;
     const __nv_bfloat16* q;   // [B*T][H][D]
     const int32_t* topk;      // [B*T][top_k]
-    int T, H, top_k, window, nchunk;
+    int T, H, HG, top_k, window, nchunk;
     float scale;
-    float* part_o;            // [seg][chunk][H][D]
+    float* part_o;            // [seg][chunk][D][H]
     float* part_ml;           // [seg][chunk][H][2]
-    const uint8_t* qstage;    // [seg][qbytes]: the staged query operand, then H factors
-    uint32_t qbytes;          // bytes of the staged fp16 operand of one segment
     uint32_t* status;
     uint32_t off_q, off_misc, tmem_cols;
 };
 
 struct Misc {
-    alignas(16) float fac[64];   // per head: softmax scale / query scale (bulk-copied)
+    float fac[64];               // per head of the group: softmax scale * log2(e) / query scale
     float red[16][64];           // per head partial max / sum of the threads that share it
     int32_t pos[kRows];
     uint64_t mma_bar;
-    uint64_t q_bar;
     uint32_t tmem_base;
 };
 
@@ -73,37 +73,28 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
-    pdl_begin();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int D = p.c.dim, H = p.H;
+    const int D = p.c.dim, H = p.H, HG = p.HG;
     const int nkb = D / 64;                     // 64-wide K blocks of the V tile
     uint8_t* sV = smem;                         // nkb x [128 rows x 128 B]
-    uint8_t* sQ = smem + p.off_q;               // nkb x [H rows x 128 B]; later logits + P
-    float* sZ = reinterpret_cast<float*>(sQ);   // [H][kZStride] (after S is computed)
-    uint8_t* sP = sQ + ((H * kZStride * 4 + 1023) & ~1023);   // 2 x [H rows x 128 B]
+    uint8_t* sQ = smem + p.off_q;               // nkb x [HG rows x 128 B]; later logits + P
+    float* sZ = reinterpret_cast<float*>(sQ);   // [HG][kZStride] (after S is computed)
+    uint8_t* sP = sQ + ((HG * kZStride * 4 + 1023) & ~1023);   // 2 x [HG rows x 128 B]
     Misc* misc = reinterpret_cast<Misc*>(smem + p.off_misc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int seg = blockIdx.y, chunk = blockIdx.x;
+    const int chunk = blockIdx.x, seg = blockIdx.y, h_base = blockIdx.z * HG;
+    if (tid == 0) {
+        tc::mbar_init(&misc->mma_bar, 1);
+        tc::fence_mbar_init();
+    }
+    // everything below may read what the preceding kernel wrote (and the
+    // tensor memory is allocated only once that kernel has released its own)
+    pdl_begin();
     const int b = seg / p.T, j = seg % p.T;
     const int64_t L = seq_len(p.c, b, p.status);
     const int64_t pq = L - p.T + j;
-
-    if (tid == 0) {
-        tc::mbar_init(&misc->mma_bar, 1);
-        tc::mbar_init(&misc->q_bar, 1);
-        tc::fence_mbar_init();
-        // the query operand, staged once per (sequence, token) by k_attn_stage_q,
-        // arrives by bulk copy while the rows are gathered
-        const uint8_t* src = p.qstage + (size_t)seg * (p.qbytes + 256);
-        tc::mbar_arrive_expect_tx(&misc->q_bar, p.qbytes + (uint32_t)H * 4);
-        for (uint32_t off = 0; off < p.qbytes; off += 16384) {
-            const uint32_t n = p.qbytes - off < 16384 ? p.qbytes - off : 16384;
-            tc::bulk_g2s(sQ + off, src + off, n, &misc->q_bar);
-        }
-        tc::bulk_g2s(misc->fac, src + p.qbytes, (uint32_t)H * 4, &misc->q_bar);
-    }
     if (warp == 0) tc::tmem_alloc(&misc->tmem_base, p.tmem_cols);
     if (tid < kRows) {
         const int v = chunk * kRows + tid;
@@ -149,6 +140,56 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         }
     }
 
+    // ---- queries of the group (their loads overlap the gathers in flight):
+    // H rows of fp16 scaled by 2^e per head, the row maximum in [2^14, 2^15)
+    // so that every bf16 value down to 2^-32 of it is exact; tph consecutive
+    // threads share one head, D / tph consecutive values each
+    {
+        const int tph = kThreads / HG;               // 4, 8 or 16
+        const int hl = tid / tph, part = tid % tph;
+        const int span = D / tph;                    // a multiple of 8, at most 128
+        const __nv_bfloat16* src = p.q + ((int64_t)seg * H + h_base + hl) * D + part * span;
+        uint4 qv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (8 * i < span) qv[i] = __ldg(reinterpret_cast<const uint4*>(src + 8 * i));
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (8 * i < span) {
+                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[k] << 16)), fabsf(__uint_as_float(wv[k] & 0xFFFF0000u))));
+            }
+        }
+        for (int o = 1; o < tph; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        int e = 0;
+        if (m > 0.0f) {
+            e = 14 - ((int)((__float_as_uint(m) >> 23) & 0xFF) - 127);
+            e = e < -100 ? -100 : (e > 100 ? 100 : e);
+        }
+        const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+        // logits in base-2 units: softmax_scale * log2(e) / 2^e
+        if (part == 0) misc->fac[hl] = p.scale * 1.4426950408889634f * __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (8 * i < span) {
+                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+                uint32_t hv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    __half2 hh = __floats2half2_rn(__uint_as_float(wv[k] << 16) * up,
+                                                   __uint_as_float(wv[k] & 0xFFFF0000u) * up);
+                    memcpy(&hv[k], &hh, 4);
+                }
+                const int d = part * span + 8 * i;        // 8 values: one 16-byte chunk
+                *reinterpret_cast<uint4*>(sQ + (d >> 6) * (HG * 128) + tc::sw128_offset(hl, (d & 63) >> 3)) =
+                    make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            }
+        }
+    }
+
     // ---- dequantise: value(code) * value(scale), exact in fp16, into the swizzled V tile
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -177,30 +218,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     __syncthreads();
 
     // ---- S = V Q^T
-    bool ok = tc::mbar_wait(&misc->q_bar, 0);   // every thread reads fac[] later
-    if (warp == 4 && lane == 0 && ok) {
+    bool ok = true;
+    if (warp == 4 && lane == 0) {
         tc::fence_after_sync();
-        const uint32_t idesc = tc::idesc_f16_f32(kRows, H);
+        const uint32_t idesc = tc::idesc_f16_f32(kRows, HG);
         const uint32_t v0 = tc::smem_u32(sV), q0 = tc::smem_u32(sQ);
         for (int kb = 0; kb < nkb; ++kb)
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 tc::mma_f16(tmem, tc::desc_sw128(v0 + kb * (kRows * 128) + 32 * k),
-                            tc::desc_sw128(q0 + kb * (H * 128) + 32 * k), idesc, (kb | k) != 0);
+                            tc::desc_sw128(q0 + kb * (HG * 128) + 32 * k), idesc, (kb | k) != 0);
         tc::mma_commit(&misc->mma_bar);
     }
-    if (ok) ok = tc::mbar_wait(&misc->mma_bar, 0);
+    ok = tc::mbar_wait(&misc->mma_bar, 0);
     ok = __syncthreads_and(ok);
     tc::fence_after_sync();
 
     // ---- logits to shared memory, transposed: z[h][pos]; lane = position, the
-    // two warpgroups take one half of the heads each (H >= 32)
-    const int ngrp = H >= 32 ? 2 : 1;
+    // two warpgroups take one half of the group's heads each (HG >= 32)
+    const int ngrp = HG >= 32 ? 2 : 1;
     const int wgrp = warp >> 2, quad = warp & 3;
     if (ok && wgrp < ngrp) {
         const int r = quad * 32 + lane;
         const bool valid = misc->pos[r] >= 0;
-        const int hc = H / ngrp;
+        const int hc = HG / ngrp;
         for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
             float v[16];
             tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
@@ -210,9 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     }
     __syncthreads();
 
-    // ---- softmax statistics: nq = 256 / H threads per head, each over 128 / nq positions
-    const int nq = kThreads / H, per = kRows / nq;
-    const int h = tid % H, qt = tid / H;
+    // ---- softmax statistics: nq = 256 / HG threads per head, each over 128 / nq positions
+    const int nq = kThreads / HG, per = kRows / nq;
+    const int h = tid % HG, qt = tid / HG;
     const float* z = sZ + h * kZStride + qt * per;
     float m = -INFINITY, l = 0.0f;
     if (ok) {
@@ -222,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     __syncthreads();
     if (ok) {
         for (int k = 0; k < nq; ++k) m = fmaxf(m, misc->red[k][h]);
-        uint8_t* blk = sP + ((qt * per) >> 6) * (H * 128);
+        uint8_t* blk = sP + ((qt * per) >> 6) * (HG * 128);
         const int c_first = ((qt * per) & 63) >> 3;
         for (int c = 0; c < per / 8; ++c) {
             uint32_t hv[4];
@@ -243,24 +284,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     if (ok) misc->red[qt][h] = l;
     tc::fence_proxy_async_smem();
     __syncthreads();
-    if (ok && tid < H) {
-        float* ml = p.part_ml + (((int64_t)seg * p.nchunk + chunk) * H + tid) * 2;
+    if (ok && tid < HG) {
+        float* ml = p.part_ml + (((int64_t)seg * p.nchunk + chunk) * H + h_base + tid) * 2;
         float sum = 0.0f;
         for (int k = 0; k < nq; ++k) sum += misc->red[k][tid];
-        ml[0] = m;                                   // thread tid < H holds head tid's maximum
+        ml[0] = m;                                   // thread tid < HG holds local head tid's maximum
         ml[1] = sum;
     }
 
     // ---- O^T = V^T P^T, one 128-wide slab of d per accumulator
     if (ok && warp == 4 && lane == 0) {
         tc::fence_after_sync();
-        const uint32_t idesc = tc::idesc_f16_f32(kRows, H, /*a_mn=*/true, /*b_mn=*/false);
+        const uint32_t idesc = tc::idesc_f16_f32(kRows, HG, /*a_mn=*/true, /*b_mn=*/false);
         const uint32_t v0 = tc::smem_u32(sV), p0 = tc::smem_u32(sP);
         for (int s = 0; s < D / 128; ++s)
             for (int ks = 0; ks < kRows / 16; ++ks)
-                tc::mma_f16(tmem + (uint32_t)(H + s * H),
+                tc::mma_f16(tmem + (uint32_t)(HG + s * HG),
                             tc::desc_mn_sw128(v0 + (2 * s) * (kRows * 128) + ks * 2048, kRows * 128, 1024),
-                            tc::desc_sw128(p0 + (ks >> 2) * (H * 128) + 32 * (ks & 3)), idesc, ks != 0);
+                            tc::desc_sw128(p0 + (ks >> 2) * (HG * 128) + 32 * (ks & 3)), idesc, ks != 0);
         tc::mma_commit(&misc->mma_bar);
     }
     if (ok) ok = tc::mbar_wait(&misc->mma_bar, 1);
@@ -268,15 +309,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     tc::fence_after_sync();
 
     // ---- unnormalised partial output, [d][head] (lane = d within the slab; the
-    // two warpgroups take one half of the heads each; 16-byte stores)
+    // two warpgroups take one half of the group's heads each; 16-byte stores)
     if (ok && wgrp < ngrp) {
-        float* po = p.part_o + ((int64_t)seg * p.nchunk + chunk) * H * D;
-        const int hc = H / ngrp;
+        float* po = p.part_o + ((int64_t)seg * p.nchunk + chunk) * H * D + h_base;
+        const int hc = HG / ngrp;
         for (int s2 = 0; s2 < D / 128; ++s2) {
             const int d = s2 * 128 + quad * 32 + lane;
             for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
                 float v[16];
-                tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(H + s2 * H + c0), v);
+                tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(HG + s2 * HG + c0), v);
                 float4* dst = reinterpret_cast<float4*>(po + (int64_t)d * H + c0);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -292,70 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     }
 }
 
-// The query operand of one (sequence, token): H rows of D fp16 values scaled by
-// 2^e per head (the row maximum lands in [2^14, 2^15): every bf16 value down to
-// 2^-32 of it is exact in fp16), laid out exactly as the attention kernel's
-// K-major 128-byte-swizzled operand, followed by the H factors
-// softmax_scale * 2^-e.  grid (B*T), 256 threads, 4 threads per head.
-__global__ void __launch_bounds__(kThreads)
-k_attn_stage_q(const __nv_bfloat16* __restrict__ q, int H, int D, float scale, uint8_t* __restrict__ qstage,
-               uint32_t qbytes) {
-    pdl_begin();
-    const int seg = blockIdx.x, tid = threadIdx.x;
-    uint8_t* dst = qstage + (size_t)seg * (qbytes + 256);
-    float* fac = reinterpret_cast<float*>(dst + qbytes);
-    for (int w = tid; w < H * 4; w += kThreads) {
-        const int h = w >> 2, part = w & 3;           // part: D/4 consecutive values
-        const int span = D / 4;
-        const __nv_bfloat16* src = q + ((int64_t)seg * H + h) * D + part * span;
-        uint4 qv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (8 * i < span) qv[i] = __ldg(reinterpret_cast<const uint4*>(src + 8 * i));
-        float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (8 * i < span) {
-                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[k] << 16)), fabsf(__uint_as_float(wv[k] & 0xFFFF0000u))));
-            }
-        }
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        int e = 0;
-        if (m > 0.0f) {
-            e = 14 - ((int)((__float_as_uint(m) >> 23) & 0xFF) - 127);
-            e = e < -100 ? -100 : (e > 100 ? 100 : e);
-        }
-        const float up = __uint_as_float((uint32_t)(127 + e) << 23);
-        // logits in base-2 units: softmax_scale * log2(e) / 2^e
-        if (part == 0) fac[h] = scale * 1.4426950408889634f * __uint_as_float((uint32_t)(127 - e) << 23);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (8 * i < span) {
-                const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
-                uint32_t hv[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    __half2 hh = __floats2half2_rn(__uint_as_float(wv[k] << 16) * up,
-                                                   __uint_as_float(wv[k] & 0xFFFF0000u) * up);
-                    memcpy(&hv[k], &hh, 4);
-                }
-                const int d = part * span + 8 * i;        // 8 values: one 16-byte chunk
-                uint8_t* blk = dst + (d >> 6) * (H * 128);
-                *reinterpret_cast<uint4*>(blk + tc::sw128_offset(h, (d & 63) >> 3)) =
-                    make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            }
-        }
-    }
-}
-
-size_t attn_tc_smem(int D, int H, uint32_t* off_q, uint32_t* off_misc) {
+size_t attn_tc_smem(int D, int HG, uint32_t* off_q, uint32_t* off_misc) {
     const uint32_t v = (uint32_t)(D / 64) * kRows * 128;
-    const uint32_t qbytes = (uint32_t)(D / 64) * H * 128;
-    const uint32_t zbytes = (((uint32_t)H * kZStride * 4 + 1023) & ~1023u) + 2u * H * 128;
+    const uint32_t qbytes = (uint32_t)(D / 64) * HG * 128;
+    const uint32_t zbytes = (((uint32_t)HG * kZStride * 4 + 1023) & ~1023u) + 2u * HG * 128;
     const uint32_t qreg = ((qbytes > zbytes ? qbytes : zbytes) + 1023) & ~1023u;
     *off_q = v;
     *off_misc = v + qreg;
@@ -372,35 +353,37 @@ bool attn_tc_supported(const DevCache& c, int H) {
 
 int attn_tc_rows_per_chunk() { return kRows; }
 
-size_t attn_tc_qstage_bytes(int D, int H) { return (size_t)(D / 64) * H * 128 + 256; }
+int attn_tc_heads_per_cta(int H, int nchunk, int nseg, int num_sms) {
+    int hg = H;
+    while (hg > 16 && (int64_t)nchunk * nseg * (H / hg) < num_sms) hg >>= 1;
+    return hg;
+}
 
 cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
-                                int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st) {
+                                int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st,
+                                int num_sms) {
     Params p;
     p.c = c;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.topk = topk;
     p.T = T;
     p.H = H;
+    p.HG = attn_tc_heads_per_cta(H, aw.nchunk, c.batch * T, num_sms);
     p.top_k = top_k;
     p.window = window;
     p.nchunk = aw.nchunk;
     p.scale = sm_scale;
     p.part_o = aw.part_o;
     p.part_ml = aw.part_ml;
-    p.qstage = aw.qstage;
-    p.qbytes = (uint32_t)(c.dim / 64) * H * 128;
     p.status = status;
     uint32_t cols = 32;
-    while (cols < (uint32_t)(H + (c.dim / 128) * H)) cols <<= 1;
+    while (cols < (uint32_t)(p.HG + (c.dim / 128) * p.HG)) cols <<= 1;
     p.tmem_cols = cols;
-    const size_t smem = attn_tc_smem(c.dim, H, &p.off_q, &p.off_misc);
+    const size_t smem = attn_tc_smem(c.dim, p.HG, &p.off_q, &p.off_misc);
     cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(k_attn_stage_q, dim3((unsigned)(c.batch * T)), dim3(kThreads), 0, st, p.q, H, c.dim, sm_scale,
-                   aw.qstage, p.qbytes);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(k_attn_tc, dim3((unsigned)aw.nchunk, (unsigned)(c.batch * T)), dim3(kThreads), smem, st, p);
+    return launch_pdl(k_attn_tc, dim3((unsigned)aw.nchunk, (unsigned)(c.batch * T), (unsigned)(H / p.HG)),
+                      dim3(kThreads), smem, st, p);
 }
 
 }  // namespace csa2

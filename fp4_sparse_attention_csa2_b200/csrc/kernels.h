@@ -55,27 +55,29 @@ cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const
 
 // Top-n selection per segment into out[seg * out_stride + 0..n_out) (-1 padded).
 // hist_ready: the level-1 histogram was zeroed and accumulated by the scoring
-// kernel already (the counters are still cleared here).
+// kernel already (the counters are still cleared here).  out_vals (nullable)
+// receives the score of every selected element at the same index.
 cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_out, int32_t* out,
-                          int64_t out_stride, cudaStream_t st, bool hist_ready = false);
+                          int64_t out_stride, cudaStream_t st, bool hist_ready = false, float* out_vals = nullptr);
 
 // Attention partials + combine.
 struct AttnWork {
-    float* part_o;    // [nseg][nchunk][H][D]
+    float* part_o;    // [nseg][nchunk][D][H]
     float* part_ml;   // [nseg][nchunk][H][2]
-    uint8_t* qstage;  // [nseg][attn_tc_qstage_bytes]: staged query operands
     int nchunk;
 };
 int attn_rows_per_chunk();       // smallest chunk of any attention kernel (sizes the workspace)
 bool attn_tc_supported(const DevCache& c, int H);
 int attn_tc_rows_per_chunk();
-size_t attn_tc_qstage_bytes(int D, int H);
+// heads per CTA: H, halved (down to 16) while the grid would leave SMs idle
+int attn_tc_heads_per_cta(int H, int nchunk, int nseg, int num_sms);
 cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
-                                int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st);
+                                int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st,
+                                int num_sms);
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st);
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
                              int window, float sm_scale, float* out, float* lse, const AttnWork& aw,
-                             uint32_t* status, cudaStream_t st);
+                             uint32_t* status, cudaStream_t st, int num_sms);
 
 }  // namespace csa2
