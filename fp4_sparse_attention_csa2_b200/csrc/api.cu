@@ -93,7 +93,7 @@ bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int w
     L->scores = off; off = align_up(off + sizeof(float) * (size_t)(L->nseg * L->cap));
     L->hist = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 3 * kRadixBins);
     L->hist_scratch = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * kRadixBins);
-    L->cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 4);
+    L->cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * kSelCounters);
     L->cand1 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->cand2 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->pscores = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * pool_k);
@@ -245,12 +245,16 @@ csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dty
     src.seq_lens = cache->seq_lens;
     src.T = T;
     src.cap = L.cap;
-    // the pool's scores come out beside its indices, so the top-k below reads
-    // them contiguously instead of gathering from the full score array
     float* ps = at<float>(ws, L.pscores);
+    if (L.cap > kSmallSelect) {
+        // long contexts: the pool and this layer's top-k (the top_k best of the
+        // same scores, a subset of the pool) come out of one selection
+        return cuda_status(launch_select_dual(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, ps, pool_k, top_k,
+                                              topk_idx, top_k, st, fused));
+    }
+    // short contexts: the pool, its scores beside it, then the top-k taken from the pool
     cudaError_t e = launch_select(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, pool_k, st, fused, ps);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
-    // this layer's top-k: the top_k best of the same scores, taken from the pool
     return topk_from_pool(cache, L, ws, ps, pool_k, 0, pool_idx, pool_k, top_k, topk_idx, T, st);
 }
 
@@ -286,7 +290,7 @@ csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, in
     s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
     // the split-softmax merge keeps one weight per (chunk, head) in shared memory
-    if ((size_t)L.nchunk * H * sizeof(float) + 2 * H * sizeof(float) + 1024 > 200 * 1024) return CSA2_ERR_UNSUPPORTED;
+    if (sizeof(float) * ((size_t)L.nchunk * H + 19 * (size_t)H + 256) > 200 * 1024) return CSA2_ERR_UNSUPPORTED;
     if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
     AttnWork aw;
     aw.part_o = at<float>(ws, L.part_o);

@@ -157,16 +157,31 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
 // the weight of every (chunk, head), 2^(m_c - M) with M the head's maximum
 // over chunks, and the heads' totals.  Thread t covers channel
 // 16*blockIdx.y + t/16 and heads [4 (t%16), 4 (t%16) + 4); partials are
-// [chunk][d][head], base 2.
+// [chunk][d][head], base 2.  The first kPre chunks' partials are loaded before
+// the weights are known, so the two memory latencies overlap.
+constexpr int kPre = 8;
+
 __global__ void __launch_bounds__(256)
 k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk,
                float* __restrict__ out, float* __restrict__ lse) {
     pdl_begin();
-    extern __shared__ float s_w[];             // [nchunk][H], then M[H], L[H], per-thread partials [256/H][H]
+    extern __shared__ float s_w[];             // [nchunk][H], M[H], L[H], per-thread partials [256/H][H], out [H][17]
     float* s_M = s_w + (size_t)nchunk * H;
     float* s_L = s_M + H;
     float* s_red = s_L + H;
+    float* s_out = s_red + 256;
     const int seg = blockIdx.x, tid = threadIdx.x;
+    const int d = blockIdx.y * 16 + (tid >> 4);
+    const int h0 = (tid & 15) * 4;
+    const bool mine = d < D && h0 < H;
+    const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h0;
+    const int64_t cstride = (int64_t)D * H;
+    float4 pre[kPre];
+#pragma unroll
+    for (int c = 0; c < kPre; ++c)
+        pre[c] = (mine && c < nchunk) ? *reinterpret_cast<const float4*>(base + c * cstride)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+
     const float* ml = part_ml + (int64_t)seg * nchunk * H * 2;
     // per head, 256/H threads share the chunks: maximum, then weights and total
     // (threads past per_head * H, which exist when H does not divide 256, idle)
@@ -195,13 +210,19 @@ k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __re
         s_L[h] = tot;
     }
     __syncthreads();
-    const int d = blockIdx.y * 16 + (tid >> 4);
-    const int h0 = (tid & 15) * 4;
-    if (d < D && h0 < H) {
+    if (mine) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h0;
-        const int64_t cstride = (int64_t)D * H;
-        int c = 0;
+#pragma unroll
+        for (int c = 0; c < kPre; ++c) {
+            if (c < nchunk) {
+                const float* w = s_w + c * H + h0;
+                acc.x = fmaf(w[0], pre[c].x, acc.x);
+                acc.y = fmaf(w[1], pre[c].y, acc.y);
+                acc.z = fmaf(w[2], pre[c].z, acc.z);
+                acc.w = fmaf(w[3], pre[c].w, acc.w);
+            }
+        }
+        int c = kPre;
         for (; c + 4 <= nchunk; c += 4) {       // four chunks of loads in flight
             float4 v[4];
 #pragma unroll
@@ -227,7 +248,20 @@ k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __re
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const float lt = s_L[h0 + k];
-            out[((int64_t)seg * H + h0 + k) * D + d] = lt > 0.0f ? a[k] / lt : 0.0f;
+            s_out[(h0 + k) * 17 + (tid >> 4)] = lt > 0.0f ? a[k] / lt : 0.0f;
+        }
+    }
+    __syncthreads();
+    // out[seg][h][d]: 16 consecutive channels of every head, 4 per thread
+    const int d_lo = blockIdx.y * 16;
+    for (int i = tid; i < H * 4; i += 256) {
+        const int hh = i >> 2, q = (i & 3) * 4;
+        const float* src = s_out + hh * 17 + q;
+        float* dst = out + ((int64_t)seg * H + hh) * D + d_lo + q;
+        if (d_lo + q + 4 <= D) {
+            *reinterpret_cast<float4*>(dst) = make_float4(src[0], src[1], src[2], src[3]);
+        } else {
+            for (int k = 0; k < 4 && d_lo + q + k < D; ++k) dst[k] = src[k];
         }
     }
     if (lse && blockIdx.y == 0 && tid < H) {
@@ -242,7 +276,7 @@ int attn_rows_per_chunk() { return kRows; }
 
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st) {
-    const size_t smem = sizeof(float) * ((size_t)aw.nchunk * H + 2 * (size_t)H + 256);
+    const size_t smem = sizeof(float) * ((size_t)aw.nchunk * H + 2 * (size_t)H + 256 + 17 * (size_t)H);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_attn_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

@@ -8,14 +8,15 @@
 // value of every head).
 //
 // One CTA owns 128 entries of the (window ++ top-k) list of one (sequence,
-// query token) and one group of HG heads (HG = 16, 32 or H: fewer heads per
-// CTA when the (chunk, segment) grid alone would leave SMs idle) -- a top-k
+// query token) and one group of HG heads (HG = H, or 32 or 16 when the
+// (chunk, segment) grid would otherwise leave SMs idle) -- a top-k
 // entry that is -1, beyond p or inside the window is masked, so the attended
 // set is window ∪ top-k without double counting:
-//   1. gather the FP4 rows (16-byte loads), dequantise exactly to fp16 into a
-//      128 x D tile laid out K-major with the 128-byte swizzle; meanwhile
-//      convert the group's bf16 queries to fp16 scaled by a power of two per
-//      head (exact) in the same layout;
+//   1. fetch each FP4 row with one bulk copy (TMA) into a staging area, and
+//      dequantise exactly to fp16 into a 128 x D tile laid out K-major with
+//      the 128-byte swizzle; while the rows are in flight, convert the
+//      group's bf16 queries to fp16 scaled by a power of two per head (exact)
+//      in the same layout;
 //   2. S[pos, head] = V Q^T : tcgen05.mma M=128 (positions), N=HG, K=D;
 //   3. logits to shared memory transposed; per-head max and exp over the 128
 //      positions; P (fp16) written K-major;
@@ -32,7 +33,8 @@ namespace csa2 {
 namespace {
 
 constexpr int kRows = 128;
-constexpr int kThreads = 256;
+constexpr int kWorkers = 256;               // 8 warps: rows, queries, dequantisation, softmax, stores
+constexpr int kThreads = kWorkers + 32;     // + the warp that allocates TMEM and issues the MMAs
 constexpr int kZStride = kRows + 4;   // padded row of the transposed logits (floats)
 
 struct Params {
@@ -44,14 +46,21 @@ struct Params {
     float* part_o;            // [seg][chunk][D][H]
     float* part_ml;           // [seg][chunk][H][2]
     uint32_t* status;
-    uint32_t off_q, off_misc, tmem_cols;
+    uint32_t row_bytes;       // bytes fetched per row: D/2 codes + D/16 scales, rounded up to 16
+    uint32_t stage_stride;    // row pitch of the staging area: row_bytes, or + 16 to make it an odd multiple of 16
+    uint32_t off_q, off_stage, off_misc, tmem_cols;
 };
 
 struct Misc {
     float fac[64];               // per head of the group: softmax scale * log2(e) / query scale
     float red[16][64];           // per head partial max / sum of the threads that share it
     int32_t pos[kRows];
-    uint64_t mma_bar;
+    uint64_t row_bar;            // the chunk's row copies (one arrival per row)
+    uint64_t kb_bar[8];          // K block k of V written (one arrival per worker)
+    uint64_t s_bar;              // S = V Q^T complete
+    uint64_t p_bar;              // P written (one arrival per worker)
+    uint64_t o_bar[4];           // slab s of O^T complete
+    uint64_t drain_bar;          // every MMA of the CTA complete
     uint32_t tmem_base;
 };
 
@@ -72,6 +81,9 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     return r;
 }
 
+// Named barrier of the kWorkers worker threads (the MMA warp is not part of it).
+__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kWorkers) : "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -81,78 +93,121 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     uint8_t* sQ = smem + p.off_q;               // nkb x [HG rows x 128 B]; later logits + P
     float* sZ = reinterpret_cast<float*>(sQ);   // [HG][kZStride] (after S is computed)
     uint8_t* sP = sQ + ((HG * kZStride * 4 + 1023) & ~1023);   // 2 x [HG rows x 128 B]
+    uint8_t* sStage = smem + p.off_stage;       // [128 rows][stage_stride]: the FP4 rows as fetched (inside sV)
     Misc* misc = reinterpret_cast<Misc*>(smem + p.off_misc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int chunk = blockIdx.x, seg = blockIdx.y, h_base = blockIdx.z * HG;
     if (tid == 0) {
-        tc::mbar_init(&misc->mma_bar, 1);
+        tc::mbar_init(&misc->row_bar, kRows);
+        for (int k = 0; k < 8; ++k) tc::mbar_init(&misc->kb_bar[k], kWorkers);
+        tc::mbar_init(&misc->s_bar, 1);
+        tc::mbar_init(&misc->p_bar, kWorkers);
+        for (int s = 0; s < 4; ++s) tc::mbar_init(&misc->o_bar[s], 1);
+        tc::mbar_init(&misc->drain_bar, 1);
         tc::fence_mbar_init();
     }
+    __syncthreads();
     // everything below may read what the preceding kernel wrote (and the
     // tensor memory is allocated only once that kernel has released its own)
     pdl_begin();
     const int b = seg / p.T, j = seg % p.T;
+
+    if (warp == kWorkers / 32) {
+        // ================= MMA warp: TMEM, then both products as their operands arrive
+        tc::tmem_alloc(&misc->tmem_base, p.tmem_cols);
+        tc::fence_before_sync();
+        __syncthreads();                                  // (1) operands staged, TMEM address published
+        tc::fence_after_sync();
+        const uint32_t tmem = misc->tmem_base;
+        if (lane == 0) {
+            bool ok = true;
+            // S = V Q^T, one 64-wide K block at a time as the workers finish it
+            const uint32_t idesc1 = tc::idesc_f16_f32(kRows, HG);
+            const uint32_t v0 = tc::smem_u32(sV), q0 = tc::smem_u32(sQ), p0 = tc::smem_u32(sP);
+            for (int kb = 0; kb < nkb; ++kb) {
+                ok = ok && tc::mbar_wait(&misc->kb_bar[kb], 0);
+                if (!ok) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    tc::mma_f16(tmem, tc::desc_sw128(v0 + kb * (kRows * 128) + 32 * k),
+                                tc::desc_sw128(q0 + kb * (HG * 128) + 32 * k), idesc1, (kb | k) != 0);
+            }
+            tc::mma_commit(&misc->s_bar);                 // arrives once the issued MMAs are done
+            // O^T = V^T P^T, one 128-wide slab of d per accumulator, each slab committed on its own
+            ok = ok && tc::mbar_wait(&misc->p_bar, 0);
+            if (ok) tc::fence_after_sync();
+            const uint32_t idesc2 = tc::idesc_f16_f32(kRows, HG, /*a_mn=*/true, /*b_mn=*/false);
+            for (int s = 0; s < D / 128; ++s) {
+                if (ok)
+                    for (int ks = 0; ks < kRows / 16; ++ks)
+                        tc::mma_f16(tmem + (uint32_t)(HG + s * HG),
+                                    tc::desc_mn_sw128(v0 + (2 * s) * (kRows * 128) + ks * 2048, kRows * 128, 1024),
+                                    tc::desc_sw128(p0 + (ks >> 2) * (HG * 128) + 32 * (ks & 3)), idesc2, ks != 0);
+                tc::mma_commit(&misc->o_bar[s]);
+            }
+            tc::mma_commit(&misc->drain_bar);
+            ok = tc::mbar_wait(&misc->drain_bar, 0) && ok;   // nothing in flight when TMEM is freed
+            if (!ok) flag(p.status, kStatusTimeout);
+        }
+        __syncwarp();
+        tc::fence_before_sync();
+        __syncthreads();                                  // (2) the workers are done with TMEM
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, p.tmem_cols);
+        return;
+    }
+
+    // ================= workers (8 warps)
+    // loads that do not depend on each other are issued together: this
+    // thread's top-k entry, the group's queries, the sequence length
+    const int v_entry = chunk * kRows + tid;
+    const bool is_topk = tid < kRows && v_entry >= p.window && v_entry < p.window + p.top_k;
+    int32_t t_raw = -1;
+    if (is_topk) t_raw = __ldg(p.topk + (int64_t)seg * p.top_k + (v_entry - p.window));
+    // queries: tph consecutive threads share one head, D / tph consecutive values each
+    const int tph = kWorkers / HG;                   // 4, 8 or 16
+    const int hl = tid / tph, part = tid % tph;
+    const int span = D / tph;                        // a multiple of 8, at most 128
+    uint4 qv[16];
+    {
+        const __nv_bfloat16* src = p.q + ((int64_t)seg * H + h_base + hl) * D + part * span;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (8 * i < span) qv[i] = __ldg(reinterpret_cast<const uint4*>(src + 8 * i));
+    }
     const int64_t L = seq_len(p.c, b, p.status);
     const int64_t pq = L - p.T + j;
-    if (warp == 0) tc::tmem_alloc(&misc->tmem_base, p.tmem_cols);
+
+    // ---- rows: thread r < 128 resolves entry r of the chunk and fetches its
+    // whole FP4 row (codes + scales) with one bulk copy into the staging area
     if (tid < kRows) {
-        const int v = chunk * kRows + tid;
         int32_t t = -1;
-        if (pq >= 0 && v < p.window + p.top_k) {
-            if (v < p.window) {
-                t = pq - v >= 0 ? (int32_t)(pq - v) : -1;
+        if (pq >= 0 && v_entry < p.window + p.top_k) {
+            if (v_entry < p.window) {
+                t = pq - v_entry >= 0 ? (int32_t)(pq - v_entry) : -1;
             } else {
-                t = __ldg(p.topk + (int64_t)seg * p.top_k + (v - p.window));
+                t = t_raw;
                 if (t < -1 || t >= L) { flag(p.status, kStatusBounds); t = -1; }
                 else if (t > pq || t > pq - p.window) t = -1;   // future, or already in the window
             }
         }
+        const int64_t slot = t >= 0 ? slot_of(p.c, b, t) : -1;
+        if (t >= 0 && slot < 0) { flag(p.status, kStatusBounds); t = -1; }
         misc->pos[tid] = t;
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = misc->tmem_base;
-
-    // ---- gather: every load of this thread is issued before any is used
-    // item = (row, 16-byte code chunk = 32 channels); at most 8 items per thread
-    const int nchunk16 = D / 32;
-    const int n_items = kRows * nchunk16 / kThreads;
-    uint4 gcode[8];
-    uint16_t gscale[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        if (k < n_items) {
-            const int w = k * kThreads + tid;
-            const int r = w / nchunk16, cc = w - r * nchunk16;
-            const int32_t t = misc->pos[r];
-            const int64_t slot = t >= 0 ? slot_of(p.c, b, t) : -1;
-            if (t >= 0 && slot < 0) flag(p.status, kStatusBounds);
-            if (slot >= 0) {
-                const uint8_t* row = p.c.rows + slot * p.c.row_stride;
-                gcode[k] = __ldg(reinterpret_cast<const uint4*>(row + cc * 16));
-                gscale[k] = __ldg(reinterpret_cast<const uint16_t*>(row + (D >> 1) + 2 * cc));
-            } else {
-                gcode[k] = make_uint4(0u, 0u, 0u, 0u);
-                gscale[k] = 0;                                  // E4M3 zero scale: the row dequantises to 0
-            }
+        if (t >= 0) {
+            tc::mbar_arrive_expect_tx(&misc->row_bar, p.row_bytes);
+            tc::bulk_g2s(sStage + tid * p.stage_stride, p.c.rows + slot * p.c.row_stride, p.row_bytes,
+                         &misc->row_bar);
+        } else {
+            tc::mbar_arrive(&misc->row_bar);
         }
     }
 
-    // ---- queries of the group (their loads overlap the gathers in flight):
-    // H rows of fp16 scaled by 2^e per head, the row maximum in [2^14, 2^15)
-    // so that every bf16 value down to 2^-32 of it is exact; tph consecutive
-    // threads share one head, D / tph consecutive values each
+    // ---- queries to fp16 scaled by 2^e per head, the row maximum in
+    // [2^14, 2^15) so that every bf16 value down to 2^-32 of it is exact
     {
-        const int tph = kThreads / HG;               // 4, 8 or 16
-        const int hl = tid / tph, part = tid % tph;
-        const int span = D / tph;                    // a multiple of 8, at most 128
-        const __nv_bfloat16* src = p.q + ((int64_t)seg * H + h_base + hl) * D + part * span;
-        uint4 qv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (8 * i < span) qv[i] = __ldg(reinterpret_cast<const uint4*>(src + 8 * i));
         float m = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -189,80 +244,91 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
             }
         }
     }
+    tc::fence_proxy_async_smem();                     // the queries are an MMA operand
+    tc::fence_before_sync();
+    __syncthreads();                                  // (1) pos[], queries, TMEM address
+    tc::fence_after_sync();
+    const uint32_t tmem = misc->tmem_base;
 
-    // ---- dequantise: value(code) * value(scale), exact in fp16, into the swizzled V tile
+    // ---- dequantise: value(code) * value(scale), exact in fp16, into the
+    // swizzled V tile.  Thread t owns row t % 128 and the 32-channel chunks
+    // cc = 2k + t / 128 (k < D / 64), so a warp's 16-byte accesses walk 32
+    // consecutive rows: conflict-free in the staging area (odd 16-byte row
+    // stride) and in the 128-byte-swizzled tile.  The staging area overlaps the
+    // tile, so every read is done before the first write; masked rows become 0.
+    // K block k is handed to the MMA warp as soon as every worker has written it.
+    bool ok = tc::mbar_wait(&misc->row_bar, 0);
+    const bool rows_ok = ok;
+    const int r = tid & (kRows - 1), half = tid >> 7;
+    const int n_own = D / 64;                        // chunks per thread, at most 8
+    const bool live = misc->pos[r] >= 0;
+    uint4 code[8];
+    uint16_t scl[8];
+    {
+        const uint8_t* row = sStage + r * p.stage_stride;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k < n_own) {
+                const int cc = 2 * k + half;
+                code[k] = live ? *reinterpret_cast<const uint4*>(row + cc * 16) : make_uint4(0u, 0u, 0u, 0u);
+                scl[k] = live ? *reinterpret_cast<const uint16_t*>(row + (D >> 1) + 2 * cc) : (uint16_t)0;
+            }
+        }
+    }
+    workers_sync();
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        if (k < n_items) {
-            const int w = k * kThreads + tid;
-            const int r = w / nchunk16, cc = w - r * nchunk16;
+        if (k < n_own) {
             uint32_t s2;
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(gscale[k]));
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(scl[k]));
             const uint32_t s_lo = (s2 & 0xFFFFu) * 0x10001u;            // (s0, s0)
             const uint32_t s_hi = (s2 >> 16) * 0x10001u;                // (s1, s1)
-            const uint32_t cw[4] = {gcode[k].x, gcode[k].y, gcode[k].z, gcode[k].w};
+            const uint32_t cw[4] = {code[k].x, code[k].y, code[k].z, code[k].w};
             uint32_t hv[16];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
                 for (int bb = 0; bb < 4; ++bb)
                     hv[4 * q + bb] = hmul2_u32(cvt_e2m1x2_f16x2(cw[q] >> (8 * bb)), q < 2 ? s_lo : s_hi);
-            uint8_t* blk = sV + (cc >> 1) * (kRows * 128);
+            uint8_t* blk = sV + k * (kRows * 128);               // K block k = cc / 2
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4*>(blk + tc::sw128_offset(r, 4 * (cc & 1) + q)) =
+                *reinterpret_cast<uint4*>(blk + tc::sw128_offset(r, 4 * half + q)) =
                     make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&misc->kb_bar[k]);
         }
     }
-    tc::fence_proxy_async_smem();
-    __syncthreads();
-
-    // ---- S = V Q^T
-    bool ok = true;
-    if (warp == 4 && lane == 0) {
-        tc::fence_after_sync();
-        const uint32_t idesc = tc::idesc_f16_f32(kRows, HG);
-        const uint32_t v0 = tc::smem_u32(sV), q0 = tc::smem_u32(sQ);
-        for (int kb = 0; kb < nkb; ++kb)
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                tc::mma_f16(tmem, tc::desc_sw128(v0 + kb * (kRows * 128) + 32 * k),
-                            tc::desc_sw128(q0 + kb * (HG * 128) + 32 * k), idesc, (kb | k) != 0);
-        tc::mma_commit(&misc->mma_bar);
-    }
-    ok = tc::mbar_wait(&misc->mma_bar, 0);
-    ok = __syncthreads_and(ok);
-    tc::fence_after_sync();
 
     // ---- logits to shared memory, transposed: z[h][pos]; lane = position, the
     // two warpgroups take one half of the group's heads each (HG >= 32)
+    ok = tc::mbar_wait(&misc->s_bar, 0) && ok;
+    tc::fence_after_sync();
     const int ngrp = HG >= 32 ? 2 : 1;
     const int wgrp = warp >> 2, quad = warp & 3;
     if (ok && wgrp < ngrp) {
-        const int r = quad * 32 + lane;
-        const bool valid = misc->pos[r] >= 0;
+        const int rr = quad * 32 + lane;
+        const bool valid = misc->pos[rr] >= 0;
         const int hc = HG / ngrp;
         for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
             float v[16];
             tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sZ[(c0 + i) * kZStride + r] = valid ? v[i] * misc->fac[c0 + i] : -INFINITY;
+            for (int i = 0; i < 16; ++i) sZ[(c0 + i) * kZStride + rr] = valid ? v[i] * misc->fac[c0 + i] : -INFINITY;
         }
     }
-    __syncthreads();
+    workers_sync();
 
     // ---- softmax statistics: nq = 256 / HG threads per head, each over 128 / nq positions
-    const int nq = kThreads / HG, per = kRows / nq;
+    const int nq = kWorkers / HG, per = kRows / nq;
     const int h = tid % HG, qt = tid / HG;
     const float* z = sZ + h * kZStride + qt * per;
     float m = -INFINITY, l = 0.0f;
-    if (ok) {
-        for (int i = 0; i < per; ++i) m = fmaxf(m, z[i]);
-        misc->red[qt][h] = m;
-    }
-    __syncthreads();
-    if (ok) {
-        for (int k = 0; k < nq; ++k) m = fmaxf(m, misc->red[k][h]);
+    for (int i = 0; i < per; ++i) m = fmaxf(m, z[i]);
+    misc->red[qt][h] = m;
+    workers_sync();
+    for (int k = 0; k < nq; ++k) m = fmaxf(m, misc->red[k][h]);
+    {
         uint8_t* blk = sP + ((qt * per) >> 6) * (HG * 128);
         const int c_first = ((qt * per) & 63) >> 3;
         for (int c = 0; c < per / 8; ++c) {
@@ -280,10 +346,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
                 make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
     }
-    __syncthreads();   // all reads of red[] (the maxima) are done before it is reused for sums
-    if (ok) misc->red[qt][h] = l;
-    tc::fence_proxy_async_smem();
-    __syncthreads();
+    tc::fence_proxy_async_smem();                     // P is an MMA operand
+    tc::mbar_arrive(&misc->p_bar);
+    workers_sync();                                   // every read of red[] (the maxima) is done
+    misc->red[qt][h] = l;
+    workers_sync();
     if (ok && tid < HG) {
         float* ml = p.part_ml + (((int64_t)seg * p.nchunk + chunk) * H + h_base + tid) * 2;
         float sum = 0.0f;
@@ -292,28 +359,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         ml[1] = sum;
     }
 
-    // ---- O^T = V^T P^T, one 128-wide slab of d per accumulator
-    if (ok && warp == 4 && lane == 0) {
-        tc::fence_after_sync();
-        const uint32_t idesc = tc::idesc_f16_f32(kRows, HG, /*a_mn=*/true, /*b_mn=*/false);
-        const uint32_t v0 = tc::smem_u32(sV), p0 = tc::smem_u32(sP);
-        for (int s = 0; s < D / 128; ++s)
-            for (int ks = 0; ks < kRows / 16; ++ks)
-                tc::mma_f16(tmem + (uint32_t)(HG + s * HG),
-                            tc::desc_mn_sw128(v0 + (2 * s) * (kRows * 128) + ks * 2048, kRows * 128, 1024),
-                            tc::desc_sw128(p0 + (ks >> 2) * (HG * 128) + 32 * (ks & 3)), idesc, ks != 0);
-        tc::mma_commit(&misc->mma_bar);
-    }
-    if (ok) ok = tc::mbar_wait(&misc->mma_bar, 1);
-    ok = __syncthreads_and(ok);
-    tc::fence_after_sync();
-
-    // ---- unnormalised partial output, [d][head] (lane = d within the slab; the
-    // two warpgroups take one half of the group's heads each; 16-byte stores)
-    if (ok && wgrp < ngrp) {
+    // ---- unnormalised partial output, [d][head], slab by slab as the MMA warp
+    // finishes them (lane = d within the slab; the two warpgroups take one half
+    // of the group's heads each; 16-byte stores)
+    if (wgrp < ngrp) {
         float* po = p.part_o + ((int64_t)seg * p.nchunk + chunk) * H * D + h_base;
         const int hc = HG / ngrp;
         for (int s2 = 0; s2 < D / 128; ++s2) {
+            ok = tc::mbar_wait(&misc->o_bar[s2], 0) && ok;
+            tc::fence_after_sync();
+            if (!ok) continue;
             const int d = s2 * 128 + quad * 32 + lane;
             for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
                 float v[16];
@@ -324,31 +379,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
             }
         }
     }
-    if (!ok && tid == 0) flag(p.status, kStatusTimeout);
+    if (!ok) flag(p.status, kStatusTimeout);
+    if (!rows_ok) tc::mbar_wait(&misc->row_bar, 0);   // no row copy may land after the CTA has left
     tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-        tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, p.tmem_cols);
-    }
+    __syncthreads();                                  // (2) TMEM is released by the MMA warp
 }
 
-size_t attn_tc_smem(int D, int HG, uint32_t* off_q, uint32_t* off_misc) {
+// Bytes of one row the kernel fetches: codes and scales, rounded up to the
+// 16-byte granule of a bulk copy (never past the row: the stride is a
+// multiple of 16 and at least D/2 + D/16).
+int attn_tc_row_bytes(int D) { return (D / 2 + D / 16 + 15) & ~15; }
+
+size_t attn_tc_smem(int D, int HG, uint32_t stage_bytes, uint32_t* off_q, uint32_t* off_stage, uint32_t* off_misc) {
     const uint32_t v = (uint32_t)(D / 64) * kRows * 128;
     const uint32_t qbytes = (uint32_t)(D / 64) * HG * 128;
     const uint32_t zbytes = (((uint32_t)HG * kZStride * 4 + 1023) & ~1023u) + 2u * HG * 128;
     const uint32_t qreg = ((qbytes > zbytes ? qbytes : zbytes) + 1023) & ~1023u;
     *off_q = v;
+    *off_stage = (v - stage_bytes) & ~1023u;   // the tail of the V tile: rows land there before the tile is written
     *off_misc = v + qreg;
     return (size_t)v + qreg + sizeof(Misc) + 1024;
+}
+
+uint32_t attn_tc_stage_stride(int D) {
+    const uint32_t rb = (uint32_t)attn_tc_row_bytes(D);
+    return ((rb / 16) & 1) ? rb : rb + 16;
 }
 
 }  // namespace
 
 bool attn_tc_supported(const DevCache& c, int H) {
-    uint32_t a, b;
+    uint32_t a, b, d;
     return c.dim % 128 == 0 && c.dim <= 512 && (H == 16 || H == 32 || H == 64) &&
-           attn_tc_smem(c.dim, H, &a, &b) <= 227 * 1024;
+           attn_tc_smem(c.dim, H, kRows * attn_tc_stage_stride(c.dim), &a, &b, &d) <= 227 * 1024;
 }
 
 int attn_tc_rows_per_chunk() { return kRows; }
@@ -376,10 +439,12 @@ cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, 
     p.part_o = aw.part_o;
     p.part_ml = aw.part_ml;
     p.status = status;
+    p.row_bytes = (uint32_t)attn_tc_row_bytes(c.dim);
+    p.stage_stride = attn_tc_stage_stride(c.dim);
     uint32_t cols = 32;
     while (cols < (uint32_t)(p.HG + (c.dim / 128) * p.HG)) cols <<= 1;
     p.tmem_cols = cols;
-    const size_t smem = attn_tc_smem(c.dim, p.HG, &p.off_q, &p.off_misc);
+    const size_t smem = attn_tc_smem(c.dim, p.HG, kRows * p.stage_stride, &p.off_q, &p.off_stage, &p.off_misc);
     cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(k_attn_tc, dim3((unsigned)aw.nchunk, (unsigned)(c.batch * T), (unsigned)(H / p.HG)),

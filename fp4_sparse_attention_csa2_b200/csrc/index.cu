@@ -7,9 +7,10 @@
 // point 3.  The scoring function itself is not given by the pages; this is the
 // ReLU-gated, head-weighted dot product.
 //
-// One thread scores one position for every query token of its sequence.  The
-// queries of the sequence sit in shared memory as fp32 and are read as
-// broadcasts; the key (64 values) sits in registers.
+// Full scoring (fp32 keys): one thread scores one position for every query
+// token of its sequence.  Pool scoring (Reindex): four threads share one pool
+// entry, a quarter of the heads each.  The queries sit in shared memory as
+// fp32 and are read as broadcasts; the key (64 values) sits in registers.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -88,30 +89,65 @@ k_score_full(DevCache c, const void* __restrict__ q, int q_f32, const float* __r
     }
 }
 
-// grid (ceil(pool_k / 256), batch * T); dynamic smem: H_I*64 + H_I floats
+// Pool scoring: SPLIT consecutive threads share one pool entry, each taking
+// every SPLIT-th head, and add their parts with shuffles (SPLIT = 4 spreads a
+// single 16,384-entry pool over every SM; SPLIT = 1 when many segments
+// already fill the GPU, so no key is converted twice).  A CTA of 256 threads
+// covers 256 / SPLIT entries.  The queries sit in shared memory with a row
+// pitch of kQPitch floats, so the SPLIT heads read at once fall in different
+// banks.  Dynamic smem: H_I * kQPitch + H_I floats.
+constexpr int kQPitch = kDI + 4;
+
+template <int SPLIT>
 __global__ void __launch_bounds__(256)
 k_score_pool(DevCache c, const void* __restrict__ q, int q_f32, const float* __restrict__ hw, int T, int H_I,
              const int32_t* __restrict__ pool, int pool_k, float* __restrict__ scores, uint32_t* status) {
     pdl_begin();
     extern __shared__ float smem[];
     float* qs = smem;
-    float* ws = smem + H_I * kDI;
+    float* ws = smem + H_I * kQPitch;
     const int seg = blockIdx.y;
     const int b = seg / T, j = seg % T;
-    for (int i = threadIdx.x; i < H_I * kDI; i += blockDim.x) qs[i] = query_value(q, q_f32, (int64_t)seg * H_I * kDI + i);
+    for (int i = threadIdx.x; i < H_I * kDI; i += blockDim.x)
+        qs[(i / kDI) * kQPitch + i % kDI] = query_value(q, q_f32, (int64_t)seg * H_I * kDI + i);
     for (int i = threadIdx.x; i < H_I; i += blockDim.x) ws[i] = hw[(int64_t)seg * H_I + i];
     __syncthreads();
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= pool_k) return;
     const int64_t L = seq_len(c, b, status);
-    const int32_t t = pool[(int64_t)seg * pool_k + i];
-    if (t < 0) return;
-    if (t > L - T + j) { flag(status, kStatusBounds); return; }
-    const int64_t slot = slot_of(c, b, t);
-    if (slot < 0) { flag(status, kStatusBounds); return; }
-    float k[kDI];
-    load_key(c, slot, k);
-    scores[(int64_t)seg * pool_k + i] = score_one(qs, ws, H_I, k);
+    const int part = threadIdx.x % SPLIT;
+    // the SPLIT threads of an entry sit in one warp and stay together to the shuffles
+    const int i = blockIdx.x * (256 / SPLIT) + threadIdx.x / SPLIT;
+    bool live = i < pool_k;
+    int64_t slot = -1;
+    if (live) {
+        const int32_t t = pool[(int64_t)seg * pool_k + i];
+        if (t < 0) {
+            live = false;
+        } else if (t > L - T + j) {
+            if (part == 0) flag(status, kStatusBounds);
+            live = false;
+        } else {
+            slot = slot_of(c, b, t);
+            if (slot < 0) {
+                if (part == 0) flag(status, kStatusBounds);
+                live = false;
+            }
+        }
+    }
+    float s = 0.0f;
+    if (live) {
+        float k[kDI];
+        load_key(c, slot, k);
+        for (int h = part; h < H_I; h += SPLIT) {
+            const float* qh = qs + h * kQPitch;
+            float dot = 0.0f;
+#pragma unroll
+            for (int d = 0; d < kDI; ++d) dot = fmaf(qh[d], k[d], dot);
+            s = fmaf(ws[h], fmaxf(dot, 0.0f), s);
+        }
+    }
+#pragma unroll
+    for (int o = 1; o < SPLIT; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (live && part == 0) scores[(int64_t)seg * pool_k + i] = s;
 }
 
 }  // namespace
@@ -129,9 +165,18 @@ cudaError_t launch_score_full(const DevCache& c, const void* q, int q_f32, const
 
 cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
                               const int32_t* pool, int pool_k, float* scores, uint32_t* status, cudaStream_t st) {
-    const size_t smem = sizeof(float) * (size_t)H_I * (kDI + 1);
-    dim3 grid((unsigned)((pool_k + 255) / 256), (unsigned)(c.batch * T));
-    return launch_pdl(k_score_pool, dim3(grid), dim3(256), smem, st, c, q, q_f32, hw, T, H_I, pool, pool_k, scores, status);
+    const size_t smem = sizeof(float) * (size_t)H_I * (kQPitch + 1);
+    const int64_t nseg = (int64_t)c.batch * T;
+    // four threads per entry while one thread per entry would leave SMs idle
+    // (fewer than about 4 x 148 CTAs of 256 entries)
+    const bool split = nseg * ((pool_k + 255) / 256) < 4 * 148;
+    const int per_cta = split ? 256 / 4 : 256;
+    dim3 grid((unsigned)((pool_k + per_cta - 1) / per_cta), (unsigned)nseg);
+    if (split)
+        return launch_pdl(k_score_pool<4>, dim3(grid), dim3(256), smem, st, c, q, q_f32, hw, T, H_I, pool, pool_k,
+                          scores, status);
+    return launch_pdl(k_score_pool<1>, dim3(grid), dim3(256), smem, st, c, q, q_f32, hw, T, H_I, pool, pool_k, scores,
+                      status);
 }
 
 }  // namespace csa2

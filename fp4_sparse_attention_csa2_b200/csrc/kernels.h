@@ -11,9 +11,10 @@ namespace csa2 {
 // Radix-select state of one workspace (see topk.cu).  Counts and histograms
 // are per segment (one segment = one (sequence, query token)).
 constexpr int kRadixBins = 2048;
+constexpr int kSelCounters = 8;   // per segment: outputs / candidates of two targets, tie ranks
 struct SelWork {
     uint32_t* hist;   // [nseg][3][kRadixBins]
-    uint32_t* cnt;    // [nseg][4]: outputs, level-1 candidates, level-2 candidates, ties
+    uint32_t* cnt;    // [nseg][kSelCounters]: a outputs, a candidates, b outputs, b candidates, a ties, b ties
     uint32_t* cand1;  // [nseg][cand_stride]
     uint32_t* cand2;  // [nseg][cand_stride]
     int64_t cand_stride;
@@ -59,6 +60,12 @@ cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const
 // receives the score of every selected element at the same index.
 cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_out, int32_t* out,
                           int64_t out_stride, cudaStream_t st, bool hist_ready = false, float* out_vals = nullptr);
+// Two selections of the same segments (more than 16,384 elements each): the
+// n_a best into out_a (scores into vals_a, nullable) and the n_b <= n_a best
+// into out_b (n_b == 0: none), out_b a subset of out_a.
+cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, int n_a, int32_t* out_a, float* vals_a,
+                               int64_t stride_a, int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st,
+                               bool hist_ready);
 
 // Attention partials + combine.
 struct AttnWork {

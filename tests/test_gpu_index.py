@@ -95,6 +95,49 @@ def test_all_equal_scores_select_exactly_k():
     for arr, k in ((pool, w.pool_k), (topk, w.top_k)):
         v = arr[0, 0]
         assert np.all(v[:k] >= 0) and np.unique(v).size == k and v.max() < 40000
+    # the top-k is a subset of the pool even when both cut inside one group of ties
+    assert set(topk[0, 0]) <= set(pool[0, 0])
+
+
+@pytest.mark.parametrize("pattern", ["thirds", "two_thirds_top"])
+def test_tied_score_groups_give_nested_sets(pattern):
+    # 40,000 positions whose index keys take three values k0, ~k0 / 2 and 0, so
+    # the scores take three values s0 > s1 > 0 (equal keys give bit-identical
+    # scores); every cutoff falls inside a group of equal scores.  "thirds": the pool takes group 0 whole and part of group 1,
+    # the top-k part of group 0.  "two_thirds_top": group 0 alone is larger
+    # than the pool, so both cut inside the same group of ties.
+    L = 40000
+    w = wl.scaled(wl.WORKLOADS["long64k"], L)
+    slots = (L + 63) // 64 * 64
+    cache = csa2.Cache(1, slots, w.D, 64, w.row_stride, csa2.E4M3, [L], seq_stride_slots=slots)
+    layer = wl.layer_queries(w, 0)
+    q = layer["q_idx"][0, 0].float()                       # [H_I, 64]
+    k0 = q.sum(0)
+    k0 = (k0 / k0.abs().max() * 8).to(torch.bfloat16)     # largest entry 8, inside the E4M3 range
+    keys = torch.zeros((L, 64), dtype=torch.bfloat16)
+    t = torch.arange(L)
+    g = (t % 3) if pattern == "thirds" else torch.where(t % 3 == 2, 2, 0)
+    keys[g == 0] = k0
+    keys[g == 1] = (k0.float() / 2).to(torch.bfloat16)
+    x = torch.zeros((1, L, w.D), dtype=torch.bfloat16, device="cuda")
+    sp = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csa2.kv_append_quant(cache, x, sp, keys[None].cuda())
+    ws = new_ws(cache, w)
+    pool, topk = _run_full(w, layer, cache, ws)
+    assert csa2.read_device_status(ws) == csa2.OK
+    # k0 is along the sum of the indexer queries, so its dot products sum to a
+    # positive number: group 0 scores above group 2 (score 0)
+    s0 = float((layer["w"][0, 0].float() * torch.relu(q @ k0.float())).sum())
+    assert s0 > 0
+    gp, gt = g.numpy()[pool[0, 0]], g.numpy()[topk[0, 0]]
+    n0 = int((g == 0).sum())
+    assert np.unique(pool[0, 0]).size == w.pool_k and np.unique(topk[0, 0]).size == w.top_k
+    assert set(topk[0, 0]) <= set(pool[0, 0])
+    assert np.all(gt == 0)
+    if n0 <= w.pool_k:
+        assert np.sum(gp == 0) == n0 and np.all(gp[gp != 0] == 1)
+    else:
+        assert np.all(gp == 0)
 
 
 def test_reuse_touches_no_index_buffer():
