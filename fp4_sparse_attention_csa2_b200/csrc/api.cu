@@ -72,11 +72,11 @@ int num_sms() {
 
 // Workspace layout (byte offsets, each section 256-byte aligned):
 //   status word | full-layer scores | radix histograms | scratch histogram |
-//   radix counters | candidates 1 | candidates 2 | pool scores | attention partials
+//   radix counters | candidates 1, 2 | survivors 1, 2 | pool scores | attention partials
 // The radix histograms and counters are zero between calls: the workspace
 // starts zeroed and every large selection clears what it used.
 struct Layout {
-    size_t status, scores, hist, hist_scratch, cnt, cand1, cand2, pscores, part_o, part_ml, total;
+    size_t status, scores, hist, hist_scratch, cnt, cand1, cand2, surv1, surv2, pscores, part_o, part_ml, total;
     int64_t nseg, cap, cand_stride;
     int nchunk;
 };
@@ -96,6 +96,8 @@ bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int w
     L->cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * kSelCounters);
     L->cand1 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->cand2 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
+    L->surv1 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
+    L->surv2 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->pscores = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * pool_k);
     L->part_o = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * c->dim);
     L->part_ml = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * 2);
@@ -112,6 +114,8 @@ SelWork sel_work(void* ws, const Layout& L) {
     w.cnt = at<uint32_t>(ws, L.cnt);
     w.cand1 = at<uint32_t>(ws, L.cand1);
     w.cand2 = at<uint32_t>(ws, L.cand2);
+    w.surv1 = at<uint32_t>(ws, L.surv1);
+    w.surv2 = at<uint32_t>(ws, L.surv2);
     w.cand_stride = L.cand_stride;
     return w;
 }

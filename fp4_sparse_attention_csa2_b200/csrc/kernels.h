@@ -14,9 +14,11 @@ constexpr int kRadixBins = 2048;
 constexpr int kSelCounters = 8;   // per segment: outputs / candidates of two targets, tie ranks
 struct SelWork {
     uint32_t* hist;   // [nseg][3][kRadixBins]
-    uint32_t* cnt;    // [nseg][kSelCounters]: a outputs, a candidates, b outputs, b candidates, a ties, b ties
-    uint32_t* cand1;  // [nseg][cand_stride]
-    uint32_t* cand2;  // [nseg][cand_stride]
+    uint32_t* cnt;    // [nseg][kSelCounters]: a outputs, a candidates, b outputs, b candidates, a / b survivors
+    uint32_t* cand1;  // [nseg][cand_stride] (key, id) pairs: level-1 candidates of target a
+    uint32_t* cand2;  // [nseg][cand_stride]: of target b
+    uint32_t* surv1;  // [nseg][cand_stride]: level-2 survivors of target a
+    uint32_t* surv2;  // [nseg][cand_stride]: of target b
     int64_t cand_stride;
 };
 

@@ -15,9 +15,10 @@
 //   large segments (Full layer, up to 1M scores): the level-1 histogram comes
 //     from the scoring kernel; a streaming pass (many CTAs per segment) selects
 //     above each target's level-1 threshold and compacts the elements equal to
-//     it into candidate lists; a cluster of CTAs per segment then resolves
-//     digits 2 and 3 on those lists.  The pool and the layer's top-k are two
-//     targets of the same pass.
+//     it into candidate lists (histogramming their digit 2); a second pass
+//     over the lists (many CTAs) selects above the digit-2 thresholds and keeps
+//     the survivors, and one CTA per segment resolves digit 3 and exact ties.
+//     The pool and the layer's top-k are two targets of the same passes.
 //   small segments (<= 16,384: the top-k of a pool): a cluster of 8 CTAs per
 //     segment keeps every key in registers and resolves all three digits,
 //     summing the CTAs' histograms through distributed shared memory.
@@ -159,6 +160,33 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_wsum
     return before + incl - v;
 }
 
+// Exclusive prefix over the block of four 16-bit counts packed in one 64-bit
+// value (per-block sums must stay below 65,536); *total gets the sums.
+template <int NT>
+__device__ __forceinline__ uint64_t block_excl_scan4(uint64_t v, uint64_t* s_wsum, uint64_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    uint64_t before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        const uint64_t u = s_wsum[w];
+        before += w < warp ? u : 0ull;
+        tot += u;
+    }
+    __syncthreads();   // s_wsum is rewritten by the next call
+    *total = tot;
+    return before + incl - v;
+}
+
+__device__ __forceinline__ uint32_t field16(uint64_t v, int f) { return (uint32_t)(v >> (16 * f)) & 0xFFFFu; }
+
 // Warp-aggregated claim: the lanes with `pred` get consecutive values of *counter.
 __device__ __forceinline__ uint32_t warp_claim(bool pred, uint32_t* counter) {
     const int lane = threadIdx.x & 31;
@@ -258,30 +286,111 @@ __device__ __forceinline__ ClPlan cluster_threshold(cg::cluster_group& cl, uint3
 // Two selections of the same scores at once: target a (the pool, n_a) and
 // target b (the top-k, n_b <= n_a; n_b == 0: none), with b a subset of a.
 // Level-1 plan of one target from the level-1 histogram.
+// Threshold digits of two targets in one 2048-bin histogram (global or shared
+// memory) with one block-wide scan; need_in[t] == 0 asks for
+// min(total, n_out[t]), and a target with need 0 gets no threshold.
+template <int NT>
+__device__ __forceinline__ void block_thresholds2(const uint32_t* h, const uint32_t need_in[2],
+                                                  const uint32_t n_out[2], uint32_t* s_wsum, Thr* s_thr,
+                                                  Thr out[2]) {
+    constexpr int per = kRadixBins / NT;        // 2 or 8: one or two vector loads (many CTAs read one histogram)
+    static_assert(per == 2 || per == 8, "bins per thread");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lo = kRadixBins - per * (tid + 1);
+    uint32_t bins[per];
+    if (per == 8) {
+        const uint4 v0 = reinterpret_cast<const uint4*>(h + lo)[0], v1 = reinterpret_cast<const uint4*>(h + lo)[1];
+        const uint32_t b8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int k = 0; k < per; ++k) bins[k] = b8[k % 8];
+    } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(h + lo);
+        bins[0] = v.x;
+        bins[per - 1] = v.y;
+    }
+    uint32_t sum = 0;
+#pragma unroll
+    for (int k = 0; k < per; ++k) sum += bins[k];
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        const uint32_t v = s_wsum[w];
+        before += w < warp ? v : 0u;
+        total += v;
+    }
+    const uint32_t excl = before + incl - sum;
+    uint32_t need[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        need[t] = need_in[t] ? need_in[t] : (total < n_out[t] ? total : n_out[t]);
+        if (need[t] > 0 && excl < need[t] && need[t] <= excl + sum) {
+            uint32_t above = excl;
+#pragma unroll
+            for (int k = per - 1; k >= 0; --k) {
+                if (need[t] <= above + bins[k]) {
+                    s_thr[t].c = (uint32_t)(lo + k);
+                    s_thr[t].above = above;
+                    s_thr[t].eq = bins[k];
+                    break;
+                }
+                above += bins[k];
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        out[t] = s_thr[t];
+        out[t].need = need[t];
+    }
+    __syncthreads();   // s_wsum and s_thr are rewritten by the next call
+}
+
+// Two selections of the same scores at once: target a (the pool, n_a) and
+// target b (the top-k, n_b <= n_a; n_b == 0: none), with b a subset of a.
+// Level-1 plan of each target from the level-1 histogram.
 struct Plan1 {
     uint32_t need, c, above, eq;   // eq: elements with digit c
     bool take_eq;                  // every digit-c element is needed (or nothing is)
 };
 
 template <int NT>
-__device__ __forceinline__ Plan1 plan_level1(const uint32_t* h1, uint32_t n_out, uint32_t* s_wsum, Thr* s_thr) {
-    Plan1 p = {0u, 0xFFFFFFFFu, 0u, 0u, true};
-    if (n_out == 0) return p;
-    const Thr t = block_threshold<NT>(h1, 0u, n_out, s_wsum, s_thr);
-    p.need = t.need;
-    if (t.need == 0) return p;
-    p.c = t.c;
-    p.above = t.above;
-    p.eq = t.eq;
-    p.take_eq = t.eq == t.need - t.above;
-    return p;
+__device__ __forceinline__ void plans_level1(const uint32_t* h1, uint32_t n_a, uint32_t n_b, uint32_t* s_wsum,
+                                             Thr* s_thr, Plan1& pa, Plan1& pb) {
+    const uint32_t need_in[2] = {0u, 0u}, n_out[2] = {n_a, n_b};
+    Thr t[2];
+    block_thresholds2<NT>(h1, need_in, n_out, s_wsum, s_thr, t);
+    Plan1* pp[2] = {&pa, &pb};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        Plan1 p = {0u, 0xFFFFFFFFu, 0u, 0u, true};
+        if (t[i].need > 0) {
+            p.need = t[i].need;
+            p.c = t[i].c;
+            p.above = t[i].above;
+            p.eq = t[i].eq;
+            p.take_eq = t[i].eq == t[i].need - t[i].above;
+        }
+        *pp[i] = p;
+    }
 }
 
 // Level 1 over every element, both targets: digits above a target's c1 are
 // selected, digit-c1 elements are compacted into that target's candidate list
-// (one list when both thresholds fall on the same digit).  Each CTA claims its
-// output and candidate slots with one atomic per counter (block-wide scans of
-// per-thread counts), so the shared counters see one atomic per CTA and chunk.
+// (one list when both thresholds fall on the same digit that a does not take
+// whole) and their digit 2 is histogrammed in shared memory, then added to the
+// segment's level-2 histogram of that list.  The chunk's scores are loaded
+// before the plan is known.  Each CTA claims its output and candidate slots
+// with one atomic per counter (block-wide scans of per-thread counts; the four
+// atomics issued by four threads).
 constexpr int kPassPer = kPassChunk / kPassThreads;   // elements per thread and chunk
 
 __global__ void __launch_bounds__(kPassThreads)
@@ -289,13 +398,33 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
             int64_t stride_a, int n_b, int32_t* __restrict__ out_b, int64_t stride_b) {
     pdl_begin();
     __shared__ uint32_t s_wsum[kPassThreads / 32];
-    __shared__ Thr s_thr;
+    __shared__ uint64_t s_wsum64[kPassThreads / 32];
+    __shared__ Thr s_thr[2];
     __shared__ uint32_t s_base[4];
+    __shared__ __align__(16) uint32_t h2[2][kRadixBins];   // digit 2 of the candidates of list a, of list b
     const int seg = blockIdx.y, tid = threadIdx.x;
+    for (int i = tid; i < 2 * kRadixBins; i += kPassThreads) (&h2[0][0])[i] = 0;   // ordered by the barriers below
     uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
-    const uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
-    const Plan1 pa = plan_level1<kPassThreads>(h1, (uint32_t)n_a, s_wsum, &s_thr);
-    const Plan1 pb = plan_level1<kPassThreads>(h1, (uint32_t)n_b, s_wsum, &s_thr);
+    const int64_t nvalid = n_valid_positions(src, seg);
+    const int64_t n_items = src.ids ? src.n : nvalid;
+    int64_t base = (int64_t)blockIdx.x * kPassChunk;
+    // the first chunk's elements, in flight while the plan is worked out
+    uint32_t keys[kPassPer];
+    int32_t ids[kPassPer];
+    auto load_chunk = [&](int64_t b0) {
+#pragma unroll
+        for (int k = 0; k < kPassPer; ++k) {
+            const int64_t i = b0 + k * kPassThreads + tid;
+            Elem e = {false, -1, 0u};
+            if (i < n_items) e = load_elem(src, seg, i, nvalid);
+            keys[k] = e.valid ? e.key : 0u;   // a valid key is never 0
+            ids[k] = e.id;
+        }
+    };
+    if (base < n_items) load_chunk(base);
+    Plan1 pa, pb;
+    plans_level1<kPassThreads>(wk.hist + (int64_t)seg * 3 * kRadixBins, (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr,
+                               pa, pb);
     int32_t* oa = out_a + (int64_t)seg * stride_a;
     int32_t* ob = out_b ? out_b + (int64_t)seg * stride_b : nullptr;
     float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
@@ -304,43 +433,32 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
         for (int i = (int)pb.need + tid; i < n_b; i += kPassThreads) ob[i] = -1;
     }
     if (pa.need == 0) return;
-    // b's candidates are a's when both thresholds fall on one digit that a does
-    // not take whole
-    const bool shared = pb.c == pa.c && !pa.take_eq;
-    const int64_t nvalid = n_valid_positions(src, seg);
-    const int64_t n_items = src.ids ? src.n : nvalid;
+    const bool shared = pb.c == pa.c && !pa.take_eq;   // b's candidates are a's
     uint2* cand_a = reinterpret_cast<uint2*>(wk.cand1) + seg * wk.cand_stride;
     uint2* cand_b = reinterpret_cast<uint2*>(wk.cand2) + seg * wk.cand_stride;
-    for (int64_t base = (int64_t)blockIdx.x * kPassChunk; base < n_items; base += (int64_t)gridDim.x * kPassChunk) {
-        uint32_t keys[kPassPer];
-        int32_t ids[kPassPer];
+    for (; base < n_items; base += (int64_t)gridDim.x * kPassChunk) {
+        if (base != (int64_t)blockIdx.x * kPassChunk) load_chunk(base);
         uint32_t na = 0, nca = 0, nb = 0, ncb = 0;
 #pragma unroll
         for (int k = 0; k < kPassPer; ++k) {
-            const int64_t i = base + k * kPassThreads + tid;
-            Elem e = {false, -1, 0u};
-            if (i < n_items) e = load_elem(src, seg, i, nvalid);
-            keys[k] = e.valid ? e.key : 0u;   // a valid key is never 0
-            ids[k] = e.id;
+            const bool valid = keys[k] != 0u;
             const uint32_t d = digit(keys[k], 1);
-            na += e.valid && (d > pa.c || (d == pa.c && pa.take_eq));
-            nca += e.valid && d == pa.c && !pa.take_eq;
-            nb += e.valid && (d > pb.c || (d == pb.c && pb.take_eq));
-            ncb += e.valid && !shared && d == pb.c && !pb.take_eq;
+            na += valid && (d > pa.c || (d == pa.c && pa.take_eq));
+            nca += valid && d == pa.c && !pa.take_eq;
+            nb += valid && (d > pb.c || (d == pb.c && pb.take_eq));
+            ncb += valid && !shared && d == pb.c && !pb.take_eq;
         }
-        // per-thread counts <= 16 and per-block sums <= 4096: two fit one word
-        uint32_t tot_a, tot_b;
-        const uint32_t pre_a = block_excl_scan<kPassThreads>((na << 16) | nca, s_wsum, &tot_a);
-        const uint32_t pre_b = block_excl_scan<kPassThreads>((nb << 16) | ncb, s_wsum, &tot_b);
-        if (tid == 0) {
-            s_base[0] = (tot_a >> 16) ? atomicAdd(cnt + 0, tot_a >> 16) : 0u;
-            s_base[1] = (tot_a & 0xFFFFu) ? atomicAdd(cnt + 1, tot_a & 0xFFFFu) : 0u;
-            s_base[2] = (tot_b >> 16) ? atomicAdd(cnt + 2, tot_b >> 16) : 0u;
-            s_base[3] = (tot_b & 0xFFFFu) ? atomicAdd(cnt + 3, tot_b & 0xFFFFu) : 0u;
+        // per-thread counts <= 16 and per-block sums <= 4096: four fit one 64-bit word
+        uint64_t tot;
+        const uint64_t pre = block_excl_scan4<kPassThreads>(
+            (uint64_t)na | ((uint64_t)nca << 16) | ((uint64_t)nb << 32) | ((uint64_t)ncb << 48), s_wsum64, &tot);
+        if (tid < 4) {   // a outputs, a candidates, b outputs, b candidates
+            const uint32_t v = field16(tot, tid);
+            s_base[tid] = v ? atomicAdd(cnt + tid, v) : 0u;
         }
         __syncthreads();
-        uint32_t os_a = s_base[0] + (pre_a >> 16), cs_a = s_base[1] + (pre_a & 0xFFFFu);
-        uint32_t os_b = s_base[2] + (pre_b >> 16), cs_b = s_base[3] + (pre_b & 0xFFFFu);
+        uint32_t os_a = s_base[0] + field16(pre, 0), cs_a = s_base[1] + field16(pre, 1);
+        uint32_t os_b = s_base[2] + field16(pre, 2), cs_b = s_base[3] + field16(pre, 3);
         __syncthreads();   // s_base is rewritten by the next chunk
 #pragma unroll
         for (int k = 0; k < kPassPer; ++k) {
@@ -360,193 +478,219 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
                 cand_b[cs_b++] = make_uint2(key, (uint32_t)ids[k]);
             }
         }
+        // digit-2 histograms of the candidates just compacted
+#pragma unroll
+        for (int k = 0; k < kPassPer; ++k) {
+            const uint32_t key = keys[k];
+            const uint32_t d = digit(key, 1);
+            if (key && d == pa.c && !pa.take_eq) atomicAdd(&h2[0][digit(key, 2)], 1u);
+            if (key && !shared && d == pb.c && !pb.take_eq) atomicAdd(&h2[1][digit(key, 2)], 1u);
+        }
+    }
+    __syncthreads();
+    uint32_t* gh = wk.hist + (int64_t)seg * 3 * kRadixBins;
+    for (int i = tid; i < 2 * kRadixBins; i += kPassThreads) {
+        const uint32_t v = (&h2[0][0])[i];
+        if (v) atomicAdd(gh + kRadixBins + i, v);   // level-2 histograms of list a, list b
     }
 }
 
-// Digits 2 and 3 of both targets on their candidate lists, one cluster of
-// kClCtas CTAs per segment.  The lists are walked in chunks of kClChunk
-// candidates (chunk n belongs to CTA n % kClCtas); the CTAs' shared-memory
-// histograms are summed through distributed shared memory.  Output slots and
-// tie ranks are claimed once per CTA and chunk (block-wide scans of
-// per-thread counts) on counters in CTA 0's shared memory, after the slots
-// pass 1 filled.  Exact ties at the last digit are ranked by claim order;
-// when both targets cut inside the same group of equal keys, b takes the
-// ranks below its need, which a takes too, so b stays a subset of a.
-// Finally the histograms and counters of the segment are cleared for the
-// next selection.
-constexpr int kClPerItem = 4;                          // candidates per thread and chunk
-constexpr int kClChunk = kClThreads * kClPerItem;
-
-struct Resolve {
-    // per target: digit-2 threshold and whether every digit-c2 element is
-    // taken; digit-3 threshold, and the tie ranks that are taken
-    uint32_t c2[2], c3[2], ties[2];
-    bool eq2[2], lvl3[2];
-    bool coupled;                       // b's ties are ranked with a's
-    uint32_t base[2];                   // slots already filled by pass 1
-    int32_t* out[2];
-    float* vals_a;
+// Digit 2 of both targets over their candidate lists, many CTAs per segment:
+// the lists' chunks of kPassChunk candidates (list a's, then list b's) are
+// spread over the CTAs.  Digit 2 above a target's threshold is selected, the
+// candidates equal to it survive into that target's survivor list.  Slots are
+// claimed once per CTA and chunk, as in pass 1.
+struct Plan2 {
+    Plan1 p[2];
+    bool shared;
+    uint32_t len[2];        // candidate list lengths (0: the target is complete after level 1)
+    uint32_t need2[2];      // still needed from the list
+    Thr q[2];               // digit-2 thresholds
+    bool eq2[2];            // every digit-2 == c2 candidate is needed
 };
 
-// One pass over `list` (len candidates) for the targets in mask (bit t:
-// target t).  level 2: take digit 2 above c2 (or equal, with eq2) and
-// histogram digit 3 of the rest equal to c2 into h3[t]; level 3: among
-// digit-2 == c2, take digit 3 above c3, and ties by rank.
-template <int LEVEL>
-__device__ __forceinline__ void resolve_pass(const Resolve& R, uint32_t mask, const uint2* list, uint32_t len,
-                                             uint32_t rank, uint32_t* ctr, uint32_t (*h3)[kRadixBins],
-                                             uint32_t* s_wsum, uint32_t* s_base) {
-    const int tid = threadIdx.x;
-    const uint32_t nch = (len + kClChunk - 1) / kClChunk;
-    for (uint32_t ch = rank; ch < nch; ch += kClCtas) {        // the same trip count in every thread of a CTA
-        uint2 kv[kClPerItem];
-        bool in2[2][kClPerItem], eqv[2][kClPerItem];
-        uint32_t ne[2] = {0u, 0u};
+template <int NT>
+__device__ __forceinline__ Plan2 plan_level2(const uint32_t* h1, uint32_t n_a, uint32_t n_b, uint32_t* s_wsum,
+                                             Thr* s_thr) {
+    Plan2 P;
+    plans_level1<NT>(h1, n_a, n_b, s_wsum, s_thr, P.p[0], P.p[1]);
+    P.shared = P.p[1].c == P.p[0].c && !P.p[0].take_eq;   // as in k_sel_pass1
+    const uint32_t none[2] = {0u, 0u};
+    for (int t = 0; t < 2; ++t) {
+        P.len[t] = P.p[t].take_eq ? 0u : P.p[t].eq;
+        P.need2[t] = P.len[t] ? P.p[t].need - P.p[t].above : 0u;
+    }
+    if (P.shared) {
+        block_thresholds2<NT>(h1 + kRadixBins, P.need2, none, s_wsum, s_thr, P.q);
+    } else {
+        Thr qa[2], qb[2];
+        const uint32_t na_only[2] = {P.need2[0], 0u}, nb_only[2] = {P.need2[1], 0u};
+        block_thresholds2<NT>(h1 + kRadixBins, na_only, none, s_wsum, s_thr, qa);
+        block_thresholds2<NT>(h1 + 2 * kRadixBins, nb_only, none, s_wsum, s_thr, qb);
+        P.q[0] = qa[0];
+        P.q[1] = qb[0];
+    }
+    for (int t = 0; t < 2; ++t) P.eq2[t] = P.q[t].eq == P.need2[t] - P.q[t].above;
+    return P;
+}
+
+__global__ void __launch_bounds__(kPassThreads)
+k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a,
+            int n_b, int32_t* __restrict__ out_b, int64_t stride_b) {
+    pdl_begin();
+    __shared__ uint32_t s_wsum[kPassThreads / 32];
+    __shared__ uint64_t s_wsum64[kPassThreads / 32];
+    __shared__ Thr s_thr[2];
+    __shared__ uint32_t s_base[4];
+    const int seg = blockIdx.y, tid = threadIdx.x;
+    uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
+    const Plan2 P = plan_level2<kPassThreads>(wk.hist + (int64_t)seg * 3 * kRadixBins, (uint32_t)n_a, (uint32_t)n_b,
+                                              s_wsum, s_thr);
+    const uint2* list[2] = {reinterpret_cast<const uint2*>(wk.cand1) + seg * wk.cand_stride,
+                            reinterpret_cast<const uint2*>(wk.cand2) + seg * wk.cand_stride};
+    uint2* surv[2] = {reinterpret_cast<uint2*>(wk.surv1) + seg * wk.cand_stride,
+                      reinterpret_cast<uint2*>(wk.surv2) + seg * wk.cand_stride};
+    int32_t* out[2] = {out_a + (int64_t)seg * stride_a, out_b ? out_b + (int64_t)seg * stride_b : nullptr};
+    float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
+    // chunks of list a serve b too when shared; list b has chunks of its own otherwise
+    const uint32_t nch_a = (P.len[0] + kPassChunk - 1) / kPassChunk;
+    const uint32_t nch_b = P.shared ? 0u : (P.len[1] + kPassChunk - 1) / kPassChunk;
+    for (uint32_t vc = blockIdx.x; vc < nch_a + nch_b; vc += gridDim.x) {
+        const int li = vc < nch_a ? 0 : 1;
+        const uint32_t c0 = (li == 0 ? vc : vc - nch_a) * kPassChunk;
+        const uint32_t n = li == 0 ? P.len[0] : P.len[1];
+        const uint32_t tmask = li == 1 ? 2u : (P.shared ? 3u : 1u);
+        const uint2* lst = li == 0 ? list[0] : list[1];
+        uint2 kv[kPassPer];
+        uint32_t cn[4] = {0u, 0u, 0u, 0u};   // a taken, a survivors, b taken, b survivors
 #pragma unroll
-        for (int k = 0; k < kClPerItem; ++k) {
-            const uint32_t i = ch * kClChunk + k * kClThreads + tid;
-            const bool in = i < len;
-            kv[k] = in ? list[i] : make_uint2(0u, 0u);
-            const uint32_t d2 = digit(kv[k].x, 2), d3 = digit(kv[k].x, 3);
+        for (int k = 0; k < kPassPer; ++k) {
+            const uint32_t i = c0 + k * kPassThreads + tid;
+            kv[k] = i < n ? lst[i] : make_uint2(0u, 0u);
+            const uint32_t d2 = digit(kv[k].x, 2);
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-                const bool on = in && ((mask >> t) & 1u);
-                in2[t][k] = on && d2 == R.c2[t];
-                eqv[t][k] = LEVEL == 3 && in2[t][k] && d3 == R.c3[t];
-                if (LEVEL == 2 && in2[t][k] && !R.eq2[t]) atomicAdd(&h3[t][d3], 1u);
-                ne[t] += eqv[t][k] && !(t == 1 && R.coupled);
+                const bool on = kv[k].x != 0u && P.len[t] && ((tmask >> t) & 1u);
+                cn[2 * t] += on && (d2 > P.q[t].c || (d2 == P.q[t].c && P.eq2[t]));
+                cn[2 * t + 1] += on && d2 == P.q[t].c && !P.eq2[t];
             }
         }
-        uint32_t rk_next[2] = {0u, 0u};
-        if (LEVEL == 3) {
-            uint32_t tot;
-            const uint32_t pre = block_excl_scan<kClThreads>((ne[0] << 16) | ne[1], s_wsum, &tot);
-            if (tid == 0) {
-                s_base[2] = (tot >> 16) ? atomicAdd(ctr + 2, tot >> 16) : 0u;
-                s_base[3] = (tot & 0xFFFFu) ? atomicAdd(ctr + 3, tot & 0xFFFFu) : 0u;
-            }
-            __syncthreads();
-            rk_next[0] = s_base[2] + (pre >> 16);
-            rk_next[1] = s_base[3] + (pre & 0xFFFFu);
-            __syncthreads();
-        }
-        uint32_t take[2] = {0u, 0u}, nt[2] = {0u, 0u};
-#pragma unroll
-        for (int k = 0; k < kClPerItem; ++k) {
-            const uint32_t d2 = digit(kv[k].x, 2), d3 = digit(kv[k].x, 3);
-            const uint32_t rk_a = eqv[0][k] ? rk_next[0]++ : 0xFFFFFFFFu;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const bool on = ((mask >> t) & 1u) && kv[k].x != 0u;
-                bool tk;
-                if (LEVEL == 2) {
-                    tk = on && (d2 > R.c2[t] || (d2 == R.c2[t] && R.eq2[t]));
-                } else {
-                    const uint32_t rk = t == 0 ? rk_a : (R.coupled ? rk_a : (eqv[1][k] ? rk_next[1]++ : 0xFFFFFFFFu));
-                    tk = in2[t][k] && (d3 > R.c3[t] || (eqv[t][k] && rk < R.ties[t]));
-                }
-                take[t] |= (uint32_t)tk << k;
-                nt[t] += tk;
-            }
-        }
-        uint32_t tot;
-        const uint32_t pre = block_excl_scan<kClThreads>((nt[0] << 16) | nt[1], s_wsum, &tot);
-        if (tid == 0) {
-            s_base[0] = (tot >> 16) ? atomicAdd(ctr + 0, tot >> 16) : 0u;
-            s_base[1] = (tot & 0xFFFFu) ? atomicAdd(ctr + 1, tot & 0xFFFFu) : 0u;
+        uint64_t tot;
+        const uint64_t pre = block_excl_scan4<kPassThreads>(
+            (uint64_t)cn[0] | ((uint64_t)cn[1] << 16) | ((uint64_t)cn[2] << 32) | ((uint64_t)cn[3] << 48), s_wsum64,
+            &tot);
+        if (tid < 4) {   // a outputs, a survivors, b outputs, b survivors
+            const int ctr = tid == 0 ? 0 : tid == 1 ? 4 : tid == 2 ? 2 : 5;
+            const uint32_t v = field16(tot, tid);
+            s_base[tid] = v ? atomicAdd(cnt + ctr, v) : 0u;
         }
         __syncthreads();
-        uint32_t os[2] = {R.base[0] + s_base[0] + (pre >> 16), R.base[1] + s_base[1] + (pre & 0xFFFFu)};
+        uint32_t pos[4];
+#pragma unroll
+        for (int f = 0; f < 4; ++f) pos[f] = s_base[f] + field16(pre, f);
         __syncthreads();   // s_base is rewritten by the next chunk
 #pragma unroll
-        for (int k = 0; k < kClPerItem; ++k) {
-            if ((take[0] >> k) & 1u) {
-                R.out[0][os[0]] = (int32_t)kv[k].y;
-                if (R.vals_a) R.vals_a[os[0]] = key_value(kv[k].x);
-                ++os[0];
+        for (int k = 0; k < kPassPer; ++k) {
+            const uint32_t d2 = digit(kv[k].x, 2);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const bool on = kv[k].x != 0u && P.len[t] && ((tmask >> t) & 1u);
+                if (on && (d2 > P.q[t].c || (d2 == P.q[t].c && P.eq2[t]))) {
+                    out[t][pos[2 * t]] = (int32_t)kv[k].y;
+                    if (t == 0 && va) va[pos[0]] = key_value(kv[k].x);
+                    ++pos[2 * t];
+                } else if (on && d2 == P.q[t].c) {
+                    surv[t][pos[2 * t + 1]++] = kv[k];
+                }
             }
-            if ((take[1] >> k) & 1u) R.out[1][os[1]++] = (int32_t)kv[k].y;
         }
     }
 }
 
-__global__ void __launch_bounds__(kClThreads)
-k_sel_resolve(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a,
-              int n_b, int32_t* __restrict__ out_b, int64_t stride_b) {
-    cg::cluster_group cl = cg::this_cluster();
-    __shared__ __align__(16) uint32_t hist[4][kRadixBins];   // digit 2 of a, of b; digit 3 of a, of b
-    __shared__ uint32_t s_wsum[kClThreads / 32];
-    __shared__ Thr s_thr;
-    __shared__ ClPlan s_cl;
-    __shared__ uint32_t s_ctr[4];     // CTA 0's: a slots, b slots, a tie ranks, b tie ranks
-    __shared__ uint32_t s_base[4];
-    const uint32_t rank = cl.block_rank();
-    const int seg = blockIdx.y, tid = threadIdx.x;
-    for (int i = tid; i < 4 * kRadixBins; i += kClThreads) (&hist[0][0])[i] = 0;
-    if (tid < 4) s_ctr[tid] = 0;
+// Digit 3 and exact ties of both targets among the digit-2 survivors, one CTA
+// of kFinThreads threads per segment (the survivors of smooth score
+// distributions number a few dozen).  Exact ties at the last digit are
+// ranked by claim order; when both targets cut inside the same group of equal
+// keys, b takes the ranks below its need, which a takes too, so b stays a
+// subset of a.  Finally the histograms and counters of the segment are
+// cleared for the next selection.
+constexpr int kFinThreads = 1024;
+
+__global__ void __launch_bounds__(kFinThreads)
+k_sel_finish(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a,
+             int n_b, int32_t* __restrict__ out_b, int64_t stride_b) {
+    __shared__ __align__(16) uint32_t h3[2][kRadixBins];
+    __shared__ uint32_t s_wsum[kFinThreads / 32];
+    __shared__ Thr s_thr[2];
+    __shared__ uint32_t s_ctr[2];     // a tie ranks, b tie ranks
+    const int seg = blockIdx.x, tid = threadIdx.x;
+    for (int i = tid; i < 2 * kRadixBins; i += kFinThreads) (&h3[0][0])[i] = 0;
+    if (tid < 2) s_ctr[tid] = 0;
     pdl_begin();
     uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
     uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
-    const Plan1 pa = plan_level1<kClThreads>(h1, (uint32_t)n_a, s_wsum, &s_thr);
-    const Plan1 pb = plan_level1<kClThreads>(h1, (uint32_t)n_b, s_wsum, &s_thr);
-    const bool shared = pb.c == pa.c && !pa.take_eq;   // as in k_sel_pass1
-    const uint2* list_a = reinterpret_cast<const uint2*>(wk.cand1) + seg * wk.cand_stride;
-    const uint2* list_b = shared ? list_a : reinterpret_cast<const uint2*>(wk.cand2) + seg * wk.cand_stride;
-    const uint32_t len_a = pa.take_eq ? 0u : pa.eq, len_b = pb.take_eq ? 0u : pb.eq;
-    uint32_t* ctr = cl.map_shared_rank(s_ctr, 0);
-    Resolve R;
-    R.base[0] = cnt[0];
-    R.base[1] = cnt[2];
-    R.out[0] = out_a + (int64_t)seg * stride_a;
-    R.out[1] = out_b ? out_b + (int64_t)seg * stride_b : nullptr;
-    R.vals_a = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
-
-    // digit 2 histograms (one for both targets when the list is shared)
-    for (uint32_t i = rank * kClThreads + tid; i < len_a; i += kClCtas * kClThreads)
-        atomicAdd(&hist[0][digit(list_a[i].x, 2)], 1u);
-    if (!shared)
-        for (uint32_t i = rank * kClThreads + tid; i < len_b; i += kClCtas * kClThreads)
-            atomicAdd(&hist[1][digit(list_b[i].x, 2)], 1u);
-    cl.sync();   // histograms complete everywhere; CTA 0's counters are zero
-    const uint32_t need2[2] = {len_a ? pa.need - pa.above : 0u, len_b ? pb.need - pb.above : 0u};
-    ClPlan q[2] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-    if (len_a) q[0] = cluster_threshold(cl, hist[0], need2[0], 0u, s_wsum, &s_cl);
-    if (len_b) q[1] = cluster_threshold(cl, hist[shared ? 0 : 1], need2[1], 0u, s_wsum, &s_cl);
+    const Plan2 P = plan_level2<kFinThreads>(h1, (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr);
+    bool lvl3[2];
+    uint32_t need3[2], ns[2];
     for (int t = 0; t < 2; ++t) {
-        R.c2[t] = q[t].c;
-        R.eq2[t] = q[t].eq == need2[t] - q[t].above;
+        lvl3[t] = P.len[t] && !P.eq2[t];
+        need3[t] = lvl3[t] ? P.need2[t] - P.q[t].above : 0u;
+        ns[t] = cnt[t == 0 ? 4 : 5];                     // survivors
     }
-    const uint32_t act_a = len_a ? 1u : 0u, act_b = len_b ? 2u : 0u;
-    if (shared) {
-        resolve_pass<2>(R, act_a | act_b, list_a, len_a, rank, ctr, &hist[2], s_wsum, s_base);
-    } else {
-        resolve_pass<2>(R, act_a, list_a, len_a, rank, ctr, &hist[2], s_wsum, s_base);
-        resolve_pass<2>(R, act_b, list_b, len_b, rank, ctr, &hist[2], s_wsum, s_base);
+    // with a shared list and one digit-2 threshold both targets have the same survivors
+    const bool one_list = P.shared && lvl3[0] && lvl3[1] && P.q[0].c == P.q[1].c;
+    const uint2* surv[2] = {reinterpret_cast<const uint2*>(wk.surv1) + seg * wk.cand_stride,
+                            reinterpret_cast<const uint2*>(wk.surv2) + seg * wk.cand_stride};
+    for (int t = 0; t < 2; ++t)
+        if (lvl3[t])
+            for (uint32_t i = tid; i < ns[t]; i += kFinThreads) atomicAdd(&h3[t][digit(surv[t][i].x, 3)], 1u);
+    __syncthreads();
+    Thr r3[2];
+    {
+        Thr ra[2], rb[2];
+        const uint32_t none[2] = {0u, 0u};
+        const uint32_t na_only[2] = {need3[0], 0u}, nb_only[2] = {need3[1], 0u};
+        block_thresholds2<kFinThreads>(h3[0], na_only, none, s_wsum, s_thr, ra);
+        block_thresholds2<kFinThreads>(h3[1], nb_only, none, s_wsum, s_thr, rb);
+        r3[0] = ra[0];
+        r3[1] = rb[0];
     }
-    cl.sync();   // digit-3 histograms complete everywhere
-    for (int t = 0; t < 2; ++t) R.lvl3[t] = (t == 0 ? len_a : len_b) && !R.eq2[t];
-    const uint32_t need3[2] = {R.lvl3[0] ? need2[0] - q[0].above : 0u, R.lvl3[1] ? need2[1] - q[1].above : 0u};
-    ClPlan r3[2] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-    if (R.lvl3[0]) r3[0] = cluster_threshold(cl, hist[2], need3[0], 0u, s_wsum, &s_cl);
-    if (R.lvl3[1]) r3[1] = cluster_threshold(cl, hist[3], need3[1], 0u, s_wsum, &s_cl);
+    uint32_t ties[2];
+    for (int t = 0; t < 2; ++t) ties[t] = lvl3[t] ? need3[t] - r3[t].above : 0u;
+    const bool coupled = one_list && r3[0].c == r3[1].c;
+    int32_t* out[2] = {out_a + (int64_t)seg * stride_a, out_b ? out_b + (int64_t)seg * stride_b : nullptr};
+    float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
     for (int t = 0; t < 2; ++t) {
-        R.c3[t] = r3[t].c;
-        R.ties[t] = R.lvl3[t] ? need3[t] - r3[t].above : 0u;
-    }
-    R.coupled = shared && R.lvl3[0] && R.lvl3[1] && R.c2[0] == R.c2[1] && R.c3[0] == R.c3[1];
-    const uint32_t l3_a = R.lvl3[0] ? 1u : 0u, l3_b = R.lvl3[1] ? 2u : 0u;
-    if (shared) {
-        resolve_pass<3>(R, l3_a | l3_b, list_a, len_a, rank, ctr, &hist[2], s_wsum, s_base);
-    } else {
-        resolve_pass<3>(R, l3_a, list_a, len_a, rank, ctr, &hist[2], s_wsum, s_base);
-        resolve_pass<3>(R, l3_b, list_b, len_b, rank, ctr, &hist[2], s_wsum, s_base);
+        if (!lvl3[t] || (one_list && t == 1)) continue;
+        const uint32_t tmask = one_list ? 3u : (1u << t);
+        for (uint32_t i0 = 0; i0 < ns[t]; i0 += kFinThreads) {
+            const uint32_t i = i0 + tid;
+            const bool in = i < ns[t];
+            const uint2 kv = in ? surv[t][i] : make_uint2(0u, 0u);
+            const uint32_t d3 = digit(kv.x, 3);
+            bool on[2], eqv[2];
+            for (int u = 0; u < 2; ++u) {
+                on[u] = in && ((tmask >> u) & 1u);
+                eqv[u] = on[u] && d3 == r3[u].c;
+            }
+            const uint32_t rk_a = warp_claim(eqv[0], &s_ctr[0]);
+            const uint32_t rk_b = coupled ? rk_a : warp_claim(eqv[1], &s_ctr[1]);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t rk = u == 0 ? rk_a : rk_b;
+                const bool tk = on[u] && (d3 > r3[u].c || (eqv[u] && rk < ties[u]));
+                const uint32_t os = warp_claim(tk, cnt + (u == 0 ? 0 : 2));
+                if (tk) {
+                    out[u][os] = (int32_t)kv.y;
+                    if (u == 0 && va) va[os] = key_value(kv.x);
+                }
+            }
+        }
     }
     // leave the workspace as csa2_workspace_init does: histograms and counters zero
-    cl.sync();
-    if (rank == 0) {
-        for (int i = tid; i < 3 * kRadixBins; i += kClThreads) h1[i] = 0;
-        if (tid < kSelCounters) cnt[tid] = 0;
-    }
+    __syncthreads();
+    for (int i = tid; i < 3 * kRadixBins; i += kFinThreads) h1[i] = 0;
+    if (tid < kSelCounters) cnt[tid] = 0;
 }
 
 // ---------------------------------------------------------------- small segments
@@ -662,7 +806,7 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
                                int64_t stride_a, int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st,
                                bool hist_ready) {
     // the histograms and counters are zero on entry (workspace initialisation,
-    // then every k_sel_resolve clears what its selection used); without a
+    // then every k_sel_finish clears what its selection used); without a
     // histogram from the scoring kernel, build level 1 here
     cudaError_t e;
     const unsigned chunks = (unsigned)((src.n + kPassChunk - 1) / kPassChunk);
@@ -674,8 +818,13 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
     e = launch_pdl(k_sel_pass1, dim3(grid), dim3(kPassThreads), 0, st, src, wk, n_a, out_a, vals_a, stride_a, n_b,
                    out_b, stride_b);
     if (e != cudaSuccess) return e;
-    return launch_pdl_cluster(k_sel_resolve, dim3(kClCtas, (unsigned)nseg), dim3(kClThreads), 0, st, kClCtas, wk, n_a,
-                              out_a, vals_a, stride_a, n_b, out_b, stride_b);
+    // candidates: at most the segment size; spread over up to 148 CTAs
+    const unsigned g2 = chunks < 148 ? (chunks ? chunks : 1) : 148;
+    e = launch_pdl(k_sel_pass2, dim3(g2, (unsigned)nseg), dim3(kPassThreads), 0, st, wk, n_a, out_a, vals_a, stride_a,
+                   n_b, out_b, stride_b);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_sel_finish, dim3((unsigned)nseg), dim3(kFinThreads), 0, st, wk, n_a, out_a, vals_a, stride_a,
+                      n_b, out_b, stride_b);
 }
 
 }  // namespace csa2
