@@ -294,7 +294,8 @@ csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, in
     s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
     // the split-softmax merge keeps one weight per (chunk, head) in shared memory
-    if (sizeof(float) * ((size_t)L.nchunk * H + 19 * (size_t)H + 256) > 200 * 1024) return CSA2_ERR_UNSUPPORTED;
+    if (sizeof(float) * ((size_t)L.nchunk * H + 2 * (size_t)H + 256 + (4 * (256 / H) + 1) * (size_t)H) > 200 * 1024)
+        return CSA2_ERR_UNSUPPORTED;
     if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
     AttnWork aw;
     aw.part_o = at<float>(ws, L.part_o);

@@ -153,39 +153,47 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
     }
 }
 
-// Split-softmax merge.  grid (batch*T, D/16), 256 threads; dynamic smem holds
-// the weight of every (chunk, head), 2^(m_c - M) with M the head's maximum
-// over chunks, and the heads' totals.  Thread t covers channel
-// 16*blockIdx.y + t/16 and heads [4 (t%16), 4 (t%16) + 4); partials are
-// [chunk][d][head], base 2.  The first kPre chunks' partials are loaded before
-// the weights are known, so the two memory latencies overlap.
-constexpr int kPre = 8;
+// Split-softmax merge.  grid (batch*T, D / (rows * reps)), 256 threads with
+// rows = 256/H: in round r < reps thread t covers head t % H of channel
+// rows * (reps * blockIdx.y + r) + t / H (threads past rows * H idle).  Dynamic
+// smem holds the weight of every (chunk, head), 2^(m_c - M) with M the head's
+// maximum over chunks, and the heads' totals.  Partials are [chunk][d][head],
+// base 2: a warp's loads are 32 consecutive heads.  The first kPre chunks'
+// partials are loaded before the weights are known, so the two memory
+// latencies overlap.  reps = 1 (many small CTAs, a short chain) for a few
+// sequences; more rounds per CTA when many sequences fill the GPU anyway, so
+// the weights are computed fewer times.
+constexpr int kPre = 20;
 
 __global__ void __launch_bounds__(256)
 k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk,
-               float* __restrict__ out, float* __restrict__ lse) {
+               int reps, float* __restrict__ out, float* __restrict__ lse) {
     pdl_begin();
-    extern __shared__ float s_w[];             // [nchunk][H], M[H], L[H], per-thread partials [256/H][H], out [H][17]
+    extern __shared__ float s_w[];   // [nchunk][H], M[H], L[H], partials [256/H][H], out [H][rows * reps + 1]
     float* s_M = s_w + (size_t)nchunk * H;
     float* s_L = s_M + H;
     float* s_red = s_L + H;
+    const int rows = 256 / H;                  // channels per round
+    const int span = rows * reps;              // channels per CTA
     float* s_out = s_red + 256;
     const int seg = blockIdx.x, tid = threadIdx.x;
-    const int d = blockIdx.y * 16 + (tid >> 4);
-    const int h0 = (tid & 15) * 4;
-    const bool mine = d < D && h0 < H;
-    const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h0;
+    const int d_lo = blockIdx.y * span;
+    const int dr = tid / H, h = tid % H;
     const int64_t cstride = (int64_t)D * H;
-    float4 pre[kPre];
+    // the first round's partials, in flight while the weights are worked out
+    float pre[kPre];
+    {
+        const int d = d_lo + dr;
+        const bool mine = dr < rows && d < D;
+        const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h;
 #pragma unroll
-    for (int c = 0; c < kPre; ++c)
-        pre[c] = (mine && c < nchunk) ? *reinterpret_cast<const float4*>(base + c * cstride)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = 0; c < kPre; ++c) pre[c] = (mine && c < nchunk) ? base[c * cstride] : 0.0f;
+    }
 
     const float* ml = part_ml + (int64_t)seg * nchunk * H * 2;
     // per head, 256/H threads share the chunks: maximum, then weights and total
     // (threads past per_head * H, which exist when H does not divide 256, idle)
-    const int per_head = 256 / H, h = tid % H, part = tid / H;
+    const int per_head = 256 / H, part = tid / H;
     const int c_end = part < per_head ? nchunk : 0;
     float m = -INFINITY;
     for (int c = part; c < c_end; c += per_head) m = fmaxf(m, ml[((int64_t)c * H + h) * 2]);
@@ -210,59 +218,37 @@ k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __re
         s_L[h] = tot;
     }
     __syncthreads();
-    if (mine) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < reps; ++r) {
+        const int d = d_lo + r * rows + dr;
+        const bool mine = dr < rows && d < D;
+        const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h;
+        if (r > 0) {
 #pragma unroll
-        for (int c = 0; c < kPre; ++c) {
-            if (c < nchunk) {
-                const float* w = s_w + c * H + h0;
-                acc.x = fmaf(w[0], pre[c].x, acc.x);
-                acc.y = fmaf(w[1], pre[c].y, acc.y);
-                acc.z = fmaf(w[2], pre[c].z, acc.z);
-                acc.w = fmaf(w[3], pre[c].w, acc.w);
+            for (int c = 0; c < kPre; ++c) pre[c] = (mine && c < nchunk) ? base[c * cstride] : 0.0f;
+        }
+        if (mine) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int c = 0; c < kPre; ++c)
+                if (c < nchunk) acc = fmaf(s_w[c * H + h], pre[c], acc);
+            int c = kPre;
+            for (; c + 4 <= nchunk; c += 4) {       // four chunks of loads in flight
+                float v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) v[u] = base[(c + u) * cstride];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc = fmaf(s_w[(c + u) * H + h], v[u], acc);
             }
-        }
-        int c = kPre;
-        for (; c + 4 <= nchunk; c += 4) {       // four chunks of loads in flight
-            float4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const float4*>(base + (c + u) * cstride);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float* w = s_w + (c + u) * H + h0;
-                acc.x = fmaf(w[0], v[u].x, acc.x);
-                acc.y = fmaf(w[1], v[u].y, acc.y);
-                acc.z = fmaf(w[2], v[u].z, acc.z);
-                acc.w = fmaf(w[3], v[u].w, acc.w);
-            }
-        }
-        for (; c < nchunk; ++c) {
-            const float4 v = *reinterpret_cast<const float4*>(base + c * cstride);
-            const float* w = s_w + c * H + h0;
-            acc.x = fmaf(w[0], v.x, acc.x);
-            acc.y = fmaf(w[1], v.y, acc.y);
-            acc.z = fmaf(w[2], v.z, acc.z);
-            acc.w = fmaf(w[3], v.w, acc.w);
-        }
-        const float a[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float lt = s_L[h0 + k];
-            s_out[(h0 + k) * 17 + (tid >> 4)] = lt > 0.0f ? a[k] / lt : 0.0f;
+            for (; c < nchunk; ++c) acc = fmaf(s_w[c * H + h], base[c * cstride], acc);
+            const float lt = s_L[h];
+            s_out[h * (span + 1) + r * rows + dr] = lt > 0.0f ? acc / lt : 0.0f;
         }
     }
     __syncthreads();
-    // out[seg][h][d]: 16 consecutive channels of every head, 4 per thread
-    const int d_lo = blockIdx.y * 16;
-    for (int i = tid; i < H * 4; i += 256) {
-        const int hh = i >> 2, q = (i & 3) * 4;
-        const float* src = s_out + hh * 17 + q;
-        float* dst = out + ((int64_t)seg * H + hh) * D + d_lo + q;
-        if (d_lo + q + 4 <= D) {
-            *reinterpret_cast<float4*>(dst) = make_float4(src[0], src[1], src[2], src[3]);
-        } else {
-            for (int k = 0; k < 4 && d_lo + q + k < D; ++k) dst[k] = src[k];
-        }
+    // out[seg][h][d]: `span` consecutive channels of every head
+    for (int i = tid; i < H * span; i += 256) {
+        const int hh = i / span, k = i % span;
+        if (d_lo + k < D) out[((int64_t)seg * H + hh) * D + d_lo + k] = s_out[hh * (span + 1) + k];
     }
     if (lse && blockIdx.y == 0 && tid < H) {
         const float lt = s_L[tid];
@@ -276,13 +262,19 @@ int attn_rows_per_chunk() { return kRows; }
 
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st) {
-    const size_t smem = sizeof(float) * ((size_t)aw.nchunk * H + 2 * (size_t)H + 256 + 17 * (size_t)H);
+    const int rows = 256 / H;
+    const int64_t nseg = (int64_t)c.batch * T;
+    // one round per CTA while the grid stays within about four waves of a
+    // 148-SM part, else four rounds (the weights are then computed a quarter as often)
+    const int reps = nseg * ((c.dim + rows - 1) / rows) <= 4 * 148 ? 1 : 4;
+    const int span = rows * reps;
+    const size_t smem = sizeof(float) * ((size_t)aw.nchunk * H + 2 * (size_t)H + 256 + (size_t)(span + 1) * H);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_attn_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(k_attn_combine, dim3((unsigned)(c.batch * T), (unsigned)((c.dim + 15) / 16)), dim3(256), smem, st,
-                      c.dim, H, aw.part_o, aw.part_ml, aw.nchunk, out, lse);
+    return launch_pdl(k_attn_combine, dim3((unsigned)nseg, (unsigned)((c.dim + span - 1) / span)), dim3(256), smem, st,
+                      c.dim, H, aw.part_o, aw.part_ml, aw.nchunk, reps, out, lse);
 }
 
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,

@@ -11,10 +11,11 @@ namespace csa2 {
 // Radix-select state of one workspace (see topk.cu).  Counts and histograms
 // are per segment (one segment = one (sequence, query token)).
 constexpr int kRadixBins = 2048;
-constexpr int kSelCounters = 8;   // per segment: outputs / candidates of two targets, tie ranks
+constexpr int kSelCounters = 32;  // per segment: counters of two targets, an arrival count, the plan
 struct SelWork {
     uint32_t* hist;   // [nseg][3][kRadixBins]
-    uint32_t* cnt;    // [nseg][kSelCounters]: a outputs, a candidates, b outputs, b candidates, a / b survivors
+    uint32_t* cnt;    // [nseg][kSelCounters]: a outputs, a candidates, b outputs, b candidates, a / b survivors,
+                      // -, -, pass-1 arrivals, then the published plan
     uint32_t* cand1;  // [nseg][cand_stride] (key, id) pairs: level-1 candidates of target a
     uint32_t* cand2;  // [nseg][cand_stride]: of target b
     uint32_t* surv1;  // [nseg][cand_stride]: level-2 survivors of target a

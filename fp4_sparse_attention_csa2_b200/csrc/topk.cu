@@ -319,13 +319,15 @@ __device__ __forceinline__ void block_thresholds2(const uint32_t* h, const uint3
     }
     if (lane == 31) s_wsum[warp] = incl;
     __syncthreads();
-    uint32_t before = 0, total = 0;
+    // warp totals: an inclusive scan by every warp over the NT / 32 totals
+    uint32_t wt = lane < NT / 32 ? s_wsum[lane] : 0u;
 #pragma unroll
-    for (int w = 0; w < NT / 32; ++w) {
-        const uint32_t v = s_wsum[w];
-        before += w < warp ? v : 0u;
-        total += v;
+    for (int o = 1; o < NT / 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, wt, o);
+        if (lane >= o) wt += v;
     }
+    const uint32_t total = __shfl_sync(0xffffffffu, wt, NT / 32 - 1);
+    const uint32_t before = warp ? __shfl_sync(0xffffffffu, wt, (warp - 1) & 31) : 0u;
     const uint32_t excl = before + incl - sum;
     uint32_t need[2];
 #pragma unroll
@@ -383,6 +385,71 @@ __device__ __forceinline__ void plans_level1(const uint32_t* h1, uint32_t n_a, u
     }
 }
 
+// Level-2 plan of both targets (digit-2 thresholds on the candidate lists).
+struct Plan2 {
+    Plan1 p[2];
+    bool shared;
+    uint32_t len[2];        // candidate list lengths (0: the target is complete after level 1)
+    uint32_t need2[2];      // still needed from the list
+    Thr q[2];               // digit-2 thresholds
+    bool eq2[2];            // every digit-2 == c2 candidate is needed
+};
+
+// The plan travels from pass 1's last CTA to pass 2 and the finisher as
+// kPlanWords words after the segment's counters.
+constexpr int kPlanWord0 = 9;
+constexpr int kPlanWords = 19;
+static_assert(kPlanWord0 + kPlanWords <= kSelCounters, "plan words");
+
+// Level-1 words (written by k_sel_plan1): both targets' level-1 plans and
+// whether their candidate lists are one.
+__device__ __forceinline__ void plan_write1(uint32_t* w, const Plan1& pa, const Plan1& pb) {
+    const Plan1* pp[2] = {&pa, &pb};
+    for (int t = 0; t < 2; ++t) {
+        w[5 * t + 0] = pp[t]->need;
+        w[5 * t + 1] = pp[t]->c;
+        w[5 * t + 2] = pp[t]->above;
+        w[5 * t + 3] = pp[t]->eq;
+        w[5 * t + 4] = pp[t]->take_eq;
+    }
+    w[18] = pb.c == pa.c && !pa.take_eq;
+}
+
+// Level-2 words (written by pass 1's last CTA): the digit-2 thresholds.
+__device__ __forceinline__ void plan_write2(uint32_t* w, const Plan2& P) {
+    for (int t = 0; t < 2; ++t) {
+        w[10 + 4 * t + 0] = P.q[t].c;
+        w[10 + 4 * t + 1] = P.q[t].above;
+        w[10 + 4 * t + 2] = P.q[t].eq;
+        w[10 + 4 * t + 3] = P.q[t].need;
+    }
+}
+
+// Every thread gets the plan from the words (staged through shared memory).
+__device__ __forceinline__ Plan2 plan_read(const uint32_t* w, uint32_t* s_words) {
+    if (threadIdx.x < kPlanWords) s_words[threadIdx.x] = __ldcg(w + threadIdx.x);
+    __syncthreads();
+    Plan2 P;
+    for (int t = 0; t < 2; ++t) {
+        P.p[t].need = s_words[5 * t + 0];
+        P.p[t].c = s_words[5 * t + 1];
+        P.p[t].above = s_words[5 * t + 2];
+        P.p[t].eq = s_words[5 * t + 3];
+        P.p[t].take_eq = s_words[5 * t + 4] != 0u;
+        P.q[t].c = s_words[10 + 4 * t + 0];
+        P.q[t].above = s_words[10 + 4 * t + 1];
+        P.q[t].eq = s_words[10 + 4 * t + 2];
+        P.q[t].need = s_words[10 + 4 * t + 3];
+    }
+    P.shared = s_words[18] != 0u;
+    for (int t = 0; t < 2; ++t) {
+        P.len[t] = P.p[t].take_eq ? 0u : P.p[t].eq;
+        P.need2[t] = P.len[t] ? P.p[t].need - P.p[t].above : 0u;
+        P.eq2[t] = P.q[t].eq == P.need2[t] - P.q[t].above;
+    }
+    return P;
+}
+
 // Level 1 over every element, both targets: digits above a target's c1 are
 // selected, digit-c1 elements are compacted into that target's candidate list
 // (one list when both thresholds fall on the same digit that a does not take
@@ -408,23 +475,34 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
     const int64_t nvalid = n_valid_positions(src, seg);
     const int64_t n_items = src.ids ? src.n : nvalid;
     int64_t base = (int64_t)blockIdx.x * kPassChunk;
-    // the first chunk's elements, in flight while the plan is worked out
+    // a chunk is fetched in two steps: every load is issued first (the ids, then
+    // the values they select), the keys are formed only when they are needed,
+    // so the first chunk's loads are in flight while the plan is read
     uint32_t keys[kPassPer];
     int32_t ids[kPassPer];
-    auto load_chunk = [&](int64_t b0) {
+    float raw[kPassPer];
+    auto issue_chunk = [&](int64_t b0) {
 #pragma unroll
         for (int k = 0; k < kPassPer; ++k) {
             const int64_t i = b0 + k * kPassThreads + tid;
-            Elem e = {false, -1, 0u};
-            if (i < n_items) e = load_elem(src, seg, i, nvalid);
-            keys[k] = e.valid ? e.key : 0u;   // a valid key is never 0
-            ids[k] = e.id;
+            ids[k] = i < n_items ? (src.ids ? src.ids[seg * src.ids_stride + i] : (int32_t)i) : -1;
+        }
+#pragma unroll
+        for (int k = 0; k < kPassPer; ++k) {
+            const int64_t i = b0 + k * kPassThreads + tid;
+            const bool v = ids[k] >= 0 && ids[k] < nvalid;
+            raw[k] = v ? src.vals[seg * src.vals_stride + (src.gather && src.ids ? (int64_t)ids[k] : i)] : 0.0f;
         }
     };
-    if (base < n_items) load_chunk(base);
-    Plan1 pa, pb;
-    plans_level1<kPassThreads>(wk.hist + (int64_t)seg * 3 * kRadixBins, (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr,
-                               pa, pb);
+    auto form_keys = [&]() {
+#pragma unroll
+        for (int k = 0; k < kPassPer; ++k)   // a valid key is never 0
+            keys[k] = (ids[k] >= 0 && ids[k] < nvalid) ? ordered_key(raw[k]) : 0u;
+    };
+    if (base < n_items) issue_chunk(base);
+    __shared__ uint32_t s_words[kPlanWords];
+    const Plan2 P1w = plan_read(cnt + kPlanWord0, s_words);   // level-1 part (k_sel_plan1)
+    const Plan1 pa = P1w.p[0], pb = P1w.p[1];
     int32_t* oa = out_a + (int64_t)seg * stride_a;
     int32_t* ob = out_b ? out_b + (int64_t)seg * stride_b : nullptr;
     float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
@@ -432,12 +510,13 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
         for (int i = (int)pa.need + tid; i < n_a; i += kPassThreads) oa[i] = -1;
         for (int i = (int)pb.need + tid; i < n_b; i += kPassThreads) ob[i] = -1;
     }
-    if (pa.need == 0) return;
+    if (pa.need == 0) base = n_items;                 // nothing to select (every CTA still reports below)
     const bool shared = pb.c == pa.c && !pa.take_eq;   // b's candidates are a's
     uint2* cand_a = reinterpret_cast<uint2*>(wk.cand1) + seg * wk.cand_stride;
     uint2* cand_b = reinterpret_cast<uint2*>(wk.cand2) + seg * wk.cand_stride;
     for (; base < n_items; base += (int64_t)gridDim.x * kPassChunk) {
-        if (base != (int64_t)blockIdx.x * kPassChunk) load_chunk(base);
+        if (base != (int64_t)blockIdx.x * kPassChunk) issue_chunk(base);
+        form_keys();
         uint32_t na = 0, nca = 0, nb = 0, ncb = 0;
 #pragma unroll
         for (int k = 0; k < kPassPer; ++k) {
@@ -493,6 +572,59 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
         const uint32_t v = (&h2[0][0])[i];
         if (v) atomicAdd(gh + kRadixBins + i, v);   // level-2 histograms of list a, list b
     }
+    // the CTA that reports last sees the complete level-2 histograms and
+    // publishes the plan of both targets for pass 2 and the finisher
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_base[0] = atomicAdd(cnt + 8, 1u) == gridDim.x - 1 ? 1u : 0u;
+    __syncthreads();
+    if (!s_base[0]) return;
+    __threadfence();
+    {
+        // all loads in flight at once (4 x 16 bytes per thread)
+        constexpr int kVec = 2 * kRadixBins / 4 / kPassThreads;
+        uint4 hv[kVec];
+        const uint4* g4 = reinterpret_cast<const uint4*>(gh + kRadixBins);
+#pragma unroll
+        for (int k = 0; k < kVec; ++k) hv[k] = __ldcg(g4 + k * kPassThreads + tid);
+#pragma unroll
+        for (int k = 0; k < kVec; ++k) reinterpret_cast<uint4*>(&h2[0][0])[k * kPassThreads + tid] = hv[k];
+    }
+    __syncthreads();
+    Plan2 P;
+    P.p[0] = pa;
+    P.p[1] = pb;
+    P.shared = shared;
+    const uint32_t none[2] = {0u, 0u};
+    for (int t = 0; t < 2; ++t) {
+        P.len[t] = P.p[t].take_eq ? 0u : P.p[t].eq;
+        P.need2[t] = P.len[t] ? P.p[t].need - P.p[t].above : 0u;
+    }
+    if (shared) {
+        block_thresholds2<kPassThreads>(h2[0], P.need2, none, s_wsum, s_thr, P.q);
+    } else {
+        Thr qa[2], qb[2];
+        const uint32_t na_only[2] = {P.need2[0], 0u}, nb_only[2] = {P.need2[1], 0u};
+        block_thresholds2<kPassThreads>(h2[0], na_only, none, s_wsum, s_thr, qa);
+        block_thresholds2<kPassThreads>(h2[1], nb_only, none, s_wsum, s_thr, qb);
+        P.q[0] = qa[0];
+        P.q[1] = qb[0];
+    }
+    if (tid == 0) plan_write2(cnt + kPlanWord0, P);
+}
+
+// Level-1 plans of both targets from the scorer's histogram, once per segment
+// (every CTA of pass 1 then reads a few words instead of scanning the histogram).
+__global__ void __launch_bounds__(kPassThreads) k_sel_plan1(SelWork wk, int n_a, int n_b) {
+    pdl_begin();
+    __shared__ uint32_t s_wsum[kPassThreads / 32];
+    __shared__ Thr s_thr[2];
+    const int seg = blockIdx.x;
+    uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
+    Plan1 pa, pb;
+    plans_level1<kPassThreads>(wk.hist + (int64_t)seg * 3 * kRadixBins, (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr,
+                               pa, pb);
+    if (threadIdx.x == 0) plan_write1(cnt + kPlanWord0, pa, pb);
 }
 
 // Digit 2 of both targets over their candidate lists, many CTAs per segment:
@@ -500,52 +632,16 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
 // spread over the CTAs.  Digit 2 above a target's threshold is selected, the
 // candidates equal to it survive into that target's survivor list.  Slots are
 // claimed once per CTA and chunk, as in pass 1.
-struct Plan2 {
-    Plan1 p[2];
-    bool shared;
-    uint32_t len[2];        // candidate list lengths (0: the target is complete after level 1)
-    uint32_t need2[2];      // still needed from the list
-    Thr q[2];               // digit-2 thresholds
-    bool eq2[2];            // every digit-2 == c2 candidate is needed
-};
-
-template <int NT>
-__device__ __forceinline__ Plan2 plan_level2(const uint32_t* h1, uint32_t n_a, uint32_t n_b, uint32_t* s_wsum,
-                                             Thr* s_thr) {
-    Plan2 P;
-    plans_level1<NT>(h1, n_a, n_b, s_wsum, s_thr, P.p[0], P.p[1]);
-    P.shared = P.p[1].c == P.p[0].c && !P.p[0].take_eq;   // as in k_sel_pass1
-    const uint32_t none[2] = {0u, 0u};
-    for (int t = 0; t < 2; ++t) {
-        P.len[t] = P.p[t].take_eq ? 0u : P.p[t].eq;
-        P.need2[t] = P.len[t] ? P.p[t].need - P.p[t].above : 0u;
-    }
-    if (P.shared) {
-        block_thresholds2<NT>(h1 + kRadixBins, P.need2, none, s_wsum, s_thr, P.q);
-    } else {
-        Thr qa[2], qb[2];
-        const uint32_t na_only[2] = {P.need2[0], 0u}, nb_only[2] = {P.need2[1], 0u};
-        block_thresholds2<NT>(h1 + kRadixBins, na_only, none, s_wsum, s_thr, qa);
-        block_thresholds2<NT>(h1 + 2 * kRadixBins, nb_only, none, s_wsum, s_thr, qb);
-        P.q[0] = qa[0];
-        P.q[1] = qb[0];
-    }
-    for (int t = 0; t < 2; ++t) P.eq2[t] = P.q[t].eq == P.need2[t] - P.q[t].above;
-    return P;
-}
-
 __global__ void __launch_bounds__(kPassThreads)
 k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a,
             int n_b, int32_t* __restrict__ out_b, int64_t stride_b) {
     pdl_begin();
-    __shared__ uint32_t s_wsum[kPassThreads / 32];
     __shared__ uint64_t s_wsum64[kPassThreads / 32];
-    __shared__ Thr s_thr[2];
     __shared__ uint32_t s_base[4];
     const int seg = blockIdx.y, tid = threadIdx.x;
     uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
-    const Plan2 P = plan_level2<kPassThreads>(wk.hist + (int64_t)seg * 3 * kRadixBins, (uint32_t)n_a, (uint32_t)n_b,
-                                              s_wsum, s_thr);
+    __shared__ uint32_t s_words[kPlanWords];
+    const Plan2 P = plan_read(cnt + kPlanWord0, s_words);
     const uint2* list[2] = {reinterpret_cast<const uint2*>(wk.cand1) + seg * wk.cand_stride,
                             reinterpret_cast<const uint2*>(wk.cand2) + seg * wk.cand_stride};
     uint2* surv[2] = {reinterpret_cast<uint2*>(wk.surv1) + seg * wk.cand_stride,
@@ -564,9 +660,12 @@ k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict_
         uint2 kv[kPassPer];
         uint32_t cn[4] = {0u, 0u, 0u, 0u};   // a taken, a survivors, b taken, b survivors
 #pragma unroll
-        for (int k = 0; k < kPassPer; ++k) {
+        for (int k = 0; k < kPassPer; ++k) {   // every load issued before any is used
             const uint32_t i = c0 + k * kPassThreads + tid;
             kv[k] = i < n ? lst[i] : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < kPassPer; ++k) {
             const uint32_t d2 = digit(kv[k].x, 2);
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
@@ -629,7 +728,8 @@ k_sel_finish(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict
     pdl_begin();
     uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
     uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
-    const Plan2 P = plan_level2<kFinThreads>(h1, (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr);
+    __shared__ uint32_t s_words[kPlanWords];
+    const Plan2 P = plan_read(cnt + kPlanWord0, s_words);
     bool lvl3[2];
     uint32_t need3[2], ns[2];
     for (int t = 0; t < 2; ++t) {
@@ -815,6 +915,8 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
         e = launch_pdl(k_sel_hist, dim3(grid), dim3(kPassThreads), 0, st, src, wk);
         if (e != cudaSuccess) return e;
     }
+    e = launch_pdl(k_sel_plan1, dim3((unsigned)nseg), dim3(kPassThreads), 0, st, wk, n_a, n_b);
+    if (e != cudaSuccess) return e;
     e = launch_pdl(k_sel_pass1, dim3(grid), dim3(kPassThreads), 0, st, src, wk, n_a, out_a, vals_a, stride_a, n_b,
                    out_b, stride_b);
     if (e != cudaSuccess) return e;
