@@ -45,6 +45,12 @@ def peaks():
 
 
 # --------------------------------------------------------------------------- distributed plumbing
+def dist_backend():
+    """NCCL between GPUs; gloo when no GPU is visible (the host-side plumbing
+    is then exercised on CPU processes), or as CSA2_DIST_BACKEND says."""
+    return os.environ.get("CSA2_DIST_BACKEND") or ("nccl" if torch.cuda.is_available() else "gloo")
+
+
 def dist_setup(n_gpus):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -52,9 +58,12 @@ def dist_setup(n_gpus):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if dist_backend() == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -67,12 +76,26 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The slowest rank's value (device times are taken per rank; the job's
+    time is the maximum)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, layers_per_step, steps, ms_max):
+    """Layer executions per second of the whole job: every rank runs its own
+    sequence's steps (weak scaling), over the slowest rank's time."""
+    return world * layers_per_step * steps / (ms_max / 1e3)
+
+
+def rank_seed(seed, rank):
+    """Each rank decodes its own independent sequence."""
+    return seed + rank
 
 
 # --------------------------------------------------------------------------- clocks
@@ -180,7 +203,7 @@ def run_ours(args, world, rank):
     import fp4_sparse_attention_csa2_b200 as csa2
     csa2.lib()
     w = wl.WORKLOADS[args.workload]
-    seed = args.seed + rank
+    seed = rank_seed(args.seed, rank)
     lens = wl.seq_lens(w, seed)
     layers = [wl.layer_queries(w, l, seed) for l in range(len(w.pattern))]
     reps = build_replicas(w, args.replicas, seed, lens)
@@ -228,8 +251,7 @@ def run_ours(args, world, rank):
     st = csa2.read_device_status(ws, stream)
     if st != csa2.OK:
         raise RuntimeError("device status after timing: " + csa2.status_string(st))
-    layer_steps = world * len(w.pattern) * K
-    value = layer_steps / (ms / 1e3)
+    value = job_throughput(world, len(w.pattern), K, ms)
 
     # the dominant kernel (Full-layer scoring over every cached position) timed
     # on its own: a graph of R launches over the rotating replicas
@@ -285,7 +307,7 @@ def run_ours(args, world, rank):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(x0.elapsed_time(x1), world)
-    e2e_value = world * len(w.pattern) * Ke / (e2e_ms / 1e3)
+    e2e_value = job_throughput(world, len(w.pattern), Ke, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
