@@ -469,6 +469,9 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
     __shared__ Thr s_thr[2];
     __shared__ uint32_t s_base[4];
     __shared__ __align__(16) uint32_t h2[2][kRadixBins];   // digit 2 of the candidates of list a, of list b
+    extern __shared__ uint2 stage_dyn[];                      // 2 x kPassChunk: the stages of a and of b
+    uint2* stage_a = stage_dyn;
+    uint2* stage_b = stage_dyn + kPassChunk;
     const int seg = blockIdx.y, tid = threadIdx.x;
     for (int i = tid; i < 2 * kRadixBins; i += kPassThreads) (&h2[0][0])[i] = 0;   // ordered by the barriers below
     uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
@@ -535,28 +538,39 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
             const uint32_t v = field16(tot, tid);
             s_base[tid] = v ? atomicAdd(cnt + tid, v) : 0u;
         }
-        __syncthreads();
-        uint32_t os_a = s_base[0] + field16(pre, 0), cs_a = s_base[1] + field16(pre, 1);
-        uint32_t os_b = s_base[2] + field16(pre, 2), cs_b = s_base[3] + field16(pre, 3);
-        __syncthreads();   // s_base is rewritten by the next chunk
+        // the CTA's outputs are gathered in shared memory first (a's and b's
+        // outputs from the front of their stage, candidates from the back),
+        // then written out as contiguous runs
+        uint32_t os_a = field16(pre, 0), cs_a = field16(pre, 1), os_b = field16(pre, 2), cs_b = field16(pre, 3);
 #pragma unroll
         for (int k = 0; k < kPassPer; ++k) {
             const uint32_t key = keys[k];
             if (!key) continue;
             const uint32_t d = digit(key, 1);
             if (d > pa.c || (d == pa.c && pa.take_eq)) {
-                oa[os_a] = ids[k];
-                if (va) va[os_a] = key_value(key);
-                ++os_a;
+                stage_a[os_a++] = make_uint2((uint32_t)ids[k], key);
             } else if (d == pa.c) {
-                cand_a[cs_a++] = make_uint2(key, (uint32_t)ids[k]);
+                stage_a[kPassChunk - 1 - cs_a++] = make_uint2(key, (uint32_t)ids[k]);
             }
             if (d > pb.c || (d == pb.c && pb.take_eq)) {
-                ob[os_b++] = ids[k];
+                stage_b[os_b++] = make_uint2((uint32_t)ids[k], key);
             } else if (!shared && d == pb.c) {
-                cand_b[cs_b++] = make_uint2(key, (uint32_t)ids[k]);
+                stage_b[kPassChunk - 1 - cs_b++] = make_uint2(key, (uint32_t)ids[k]);
             }
         }
+        __syncthreads();   // the stages are complete; the bases have been claimed
+        {
+            const uint32_t n0 = field16(tot, 0), n1 = field16(tot, 1), n2 = field16(tot, 2), n3 = field16(tot, 3);
+            for (uint32_t i = tid; i < n0; i += kPassThreads) {
+                const uint2 v = stage_a[i];
+                oa[s_base[0] + i] = (int32_t)v.x;
+                if (va) va[s_base[0] + i] = key_value(v.y);
+            }
+            for (uint32_t i = tid; i < n1; i += kPassThreads) cand_a[s_base[1] + i] = stage_a[kPassChunk - 1 - i];
+            for (uint32_t i = tid; i < n2; i += kPassThreads) ob[s_base[2] + i] = (int32_t)stage_b[i].x;
+            for (uint32_t i = tid; i < n3; i += kPassThreads) cand_b[s_base[3] + i] = stage_b[kPassChunk - 1 - i];
+        }
+        __syncthreads();   // s_base and the stages are rewritten by the next chunk
         // digit-2 histograms of the candidates just compacted
 #pragma unroll
         for (int k = 0; k < kPassPer; ++k) {
@@ -638,6 +652,9 @@ k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict_
     pdl_begin();
     __shared__ uint64_t s_wsum64[kPassThreads / 32];
     __shared__ uint32_t s_base[4];
+    extern __shared__ uint2 stage_dyn[];                      // 2 x kPassChunk: the stages of a and of b
+    uint2* stage_a = stage_dyn;
+    uint2* stage_b = stage_dyn + kPassChunk;
     const int seg = blockIdx.y, tid = threadIdx.x;
     uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
     __shared__ uint32_t s_words[kPlanWords];
@@ -683,26 +700,38 @@ k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict_
             const uint32_t v = field16(tot, tid);
             s_base[tid] = v ? atomicAdd(cnt + ctr, v) : 0u;
         }
-        __syncthreads();
+        // outputs gathered in shared memory (front: taken, back: survivors),
+        // then written out as contiguous runs
         uint32_t pos[4];
 #pragma unroll
-        for (int f = 0; f < 4; ++f) pos[f] = s_base[f] + field16(pre, f);
-        __syncthreads();   // s_base is rewritten by the next chunk
+        for (int f = 0; f < 4; ++f) pos[f] = field16(pre, f);
 #pragma unroll
         for (int k = 0; k < kPassPer; ++k) {
             const uint32_t d2 = digit(kv[k].x, 2);
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
+                uint2* stg = t == 0 ? stage_a : stage_b;
                 const bool on = kv[k].x != 0u && P.len[t] && ((tmask >> t) & 1u);
                 if (on && (d2 > P.q[t].c || (d2 == P.q[t].c && P.eq2[t]))) {
-                    out[t][pos[2 * t]] = (int32_t)kv[k].y;
-                    if (t == 0 && va) va[pos[0]] = key_value(kv[k].x);
-                    ++pos[2 * t];
+                    stg[pos[2 * t]++] = kv[k];
                 } else if (on && d2 == P.q[t].c) {
-                    surv[t][pos[2 * t + 1]++] = kv[k];
+                    stg[kPassChunk - 1 - pos[2 * t + 1]++] = kv[k];
                 }
             }
         }
+        __syncthreads();   // the stages are complete; the bases have been claimed
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const uint2* stg = t == 0 ? stage_a : stage_b;
+            const uint32_t nt = field16(tot, 2 * t), ns = field16(tot, 2 * t + 1);
+            for (uint32_t i = tid; i < nt; i += kPassThreads) {
+                const uint2 v = stg[i];
+                out[t][s_base[2 * t] + i] = (int32_t)v.y;
+                if (t == 0 && va) va[s_base[0] + i] = key_value(v.x);
+            }
+            for (uint32_t i = tid; i < ns; i += kPassThreads) surv[t][s_base[2 * t + 1] + i] = stg[kPassChunk - 1 - i];
+        }
+        __syncthreads();   // s_base and the stages are rewritten by the next chunk
     }
 }
 
@@ -917,13 +946,18 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
     }
     e = launch_pdl(k_sel_plan1, dim3((unsigned)nseg), dim3(kPassThreads), 0, st, wk, n_a, n_b);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(k_sel_pass1, dim3(grid), dim3(kPassThreads), 0, st, src, wk, n_a, out_a, vals_a, stride_a, n_b,
-                   out_b, stride_b);
+    constexpr size_t kStageSmem = 2 * kPassChunk * sizeof(uint2);
+    e = cudaFuncSetAttribute(k_sel_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStageSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_sel_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStageSmem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(k_sel_pass1, dim3(grid), dim3(kPassThreads), kStageSmem, st, src, wk, n_a, out_a, vals_a, stride_a,
+                   n_b, out_b, stride_b);
     if (e != cudaSuccess) return e;
     // candidates: at most the segment size; spread over up to 148 CTAs
     const unsigned g2 = chunks < 148 ? (chunks ? chunks : 1) : 148;
-    e = launch_pdl(k_sel_pass2, dim3(g2, (unsigned)nseg), dim3(kPassThreads), 0, st, wk, n_a, out_a, vals_a, stride_a,
-                   n_b, out_b, stride_b);
+    e = launch_pdl(k_sel_pass2, dim3(g2, (unsigned)nseg), dim3(kPassThreads), kStageSmem, st, wk, n_a, out_a, vals_a,
+                   stride_a, n_b, out_b, stride_b);
     if (e != cudaSuccess) return e;
     return launch_pdl(k_sel_finish, dim3((unsigned)nseg), dim3(kFinThreads), 0, st, wk, n_a, out_a, vals_a, stride_a,
                       n_b, out_b, stride_b);
