@@ -42,7 +42,7 @@ namespace csa2 {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kItemTiles = 4;
+constexpr int kItemTiles = 8;
 constexpr int kStages = 8;
 constexpr int kStageBytes = kTile * 64;   // two 64-row boxes of E4M3 keys
 constexpr int kMaxTerms = 3;

@@ -17,7 +17,7 @@
 //     above each target's level-1 threshold and compacts the elements equal to
 //     it into candidate lists (histogramming their digit 2); a second pass
 //     over the lists (many CTAs) selects above the digit-2 thresholds and keeps
-//     the survivors, and one CTA per segment resolves digit 3 and exact ties.
+//     the survivors, and its last CTA resolves digit 3 and exact ties.
 //     The pool and the layer's top-k are two targets of the same passes.
 //   small segments (<= 16,384: the top-k of a pool): a cluster of 8 CTAs per
 //     segment keeps every key in registers and resolves all three digits,
@@ -641,11 +641,92 @@ __global__ void __launch_bounds__(kPassThreads) k_sel_plan1(SelWork wk, int n_a,
     if (threadIdx.x == 0) plan_write1(cnt + kPlanWord0, pa, pb);
 }
 
+// Digit 3 and exact ties of both targets among the digit-2 survivors, run by
+// the CTA of pass 2 that finishes last (the survivors of smooth score
+// distributions number a few dozen).  Exact ties at the last digit are ranked
+// by claim order; when both targets cut inside the same group of equal keys,
+// b takes the ranks below its need, which a takes too, so b stays a subset of
+// a.  Finally the histograms and counters of the segment are cleared for the
+// next selection.  h3: 2 x kRadixBins words of shared memory.
+template <int NT>
+__device__ void finish_level3(const SelWork& wk, int seg, const Plan2& P, int32_t* __restrict__ out_a,
+                              float* __restrict__ vals_a, int64_t stride_a, int32_t* __restrict__ out_b,
+                              int64_t stride_b, uint32_t* h3, uint32_t* s_wsum, Thr* s_thr, uint32_t* s_ctr) {
+    const int tid = threadIdx.x;
+    uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
+    uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
+    for (int i = tid; i < 2 * kRadixBins; i += NT) h3[i] = 0;
+    if (tid < 2) s_ctr[tid] = 0;
+    bool lvl3[2];
+    uint32_t need3[2], ns[2];
+    for (int t = 0; t < 2; ++t) {
+        lvl3[t] = P.len[t] && !P.eq2[t];
+        need3[t] = lvl3[t] ? P.need2[t] - P.q[t].above : 0u;
+        ns[t] = __ldcg(cnt + (t == 0 ? 4 : 5));           // survivors
+    }
+    __syncthreads();
+    // with a shared list and one digit-2 threshold both targets have the same survivors
+    const bool one_list = P.shared && lvl3[0] && lvl3[1] && P.q[0].c == P.q[1].c;
+    const uint2* surv[2] = {reinterpret_cast<const uint2*>(wk.surv1) + seg * wk.cand_stride,
+                            reinterpret_cast<const uint2*>(wk.surv2) + seg * wk.cand_stride};
+    for (int t = 0; t < 2; ++t)
+        if (lvl3[t])
+            for (uint32_t i = tid; i < ns[t]; i += NT) atomicAdd(&h3[t * kRadixBins + digit(__ldcg(surv[t] + i).x, 3)], 1u);
+    __syncthreads();
+    Thr r3[2];
+    {
+        Thr ra[2], rb[2];
+        const uint32_t none[2] = {0u, 0u};
+        const uint32_t na_only[2] = {need3[0], 0u}, nb_only[2] = {need3[1], 0u};
+        block_thresholds2<NT>(h3, na_only, none, s_wsum, s_thr, ra);
+        block_thresholds2<NT>(h3 + kRadixBins, nb_only, none, s_wsum, s_thr, rb);
+        r3[0] = ra[0];
+        r3[1] = rb[0];
+    }
+    uint32_t ties[2];
+    for (int t = 0; t < 2; ++t) ties[t] = lvl3[t] ? need3[t] - r3[t].above : 0u;
+    const bool coupled = one_list && r3[0].c == r3[1].c;
+    int32_t* out[2] = {out_a + (int64_t)seg * stride_a, out_b ? out_b + (int64_t)seg * stride_b : nullptr};
+    float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
+    for (int t = 0; t < 2; ++t) {
+        if (!lvl3[t] || (one_list && t == 1)) continue;
+        const uint32_t tmask = one_list ? 3u : (1u << t);
+        for (uint32_t i0 = 0; i0 < ns[t]; i0 += NT) {
+            const uint32_t i = i0 + tid;
+            const bool in = i < ns[t];
+            const uint2 kv = in ? __ldcg(surv[t] + i) : make_uint2(0u, 0u);
+            const uint32_t d3 = digit(kv.x, 3);
+            bool on[2], eqv[2];
+            for (int u = 0; u < 2; ++u) {
+                on[u] = in && ((tmask >> u) & 1u);
+                eqv[u] = on[u] && d3 == r3[u].c;
+            }
+            const uint32_t rk_a = warp_claim(eqv[0], &s_ctr[0]);
+            const uint32_t rk_b = coupled ? rk_a : warp_claim(eqv[1], &s_ctr[1]);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t rk = u == 0 ? rk_a : rk_b;
+                const bool tk = on[u] && (d3 > r3[u].c || (eqv[u] && rk < ties[u]));
+                const uint32_t os = warp_claim(tk, cnt + (u == 0 ? 0 : 2));
+                if (tk) {
+                    out[u][os] = (int32_t)kv.y;
+                    if (u == 0 && va) va[os] = key_value(kv.x);
+                }
+            }
+        }
+    }
+    // leave the workspace as csa2_workspace_init does: histograms and counters zero
+    __syncthreads();
+    for (int i = tid; i < 3 * kRadixBins; i += NT) h1[i] = 0;
+    if (tid < kSelCounters) cnt[tid] = 0;
+}
+
 // Digit 2 of both targets over their candidate lists, many CTAs per segment:
 // the lists' chunks of kPassChunk candidates (list a's, then list b's) are
 // spread over the CTAs.  Digit 2 above a target's threshold is selected, the
 // candidates equal to it survive into that target's survivor list.  Slots are
-// claimed once per CTA and chunk, as in pass 1.
+// claimed once per CTA and chunk, as in pass 1.  The last CTA to finish
+// resolves digit 3 (finish_level3).
 __global__ void __launch_bounds__(kPassThreads)
 k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a,
             int n_b, int32_t* __restrict__ out_b, int64_t stride_b) {
@@ -733,93 +814,18 @@ k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict_
         }
         __syncthreads();   // s_base and the stages are rewritten by the next chunk
     }
-}
-
-// Digit 3 and exact ties of both targets among the digit-2 survivors, one CTA
-// of kFinThreads threads per segment (the survivors of smooth score
-// distributions number a few dozen).  Exact ties at the last digit are
-// ranked by claim order; when both targets cut inside the same group of equal
-// keys, b takes the ranks below its need, which a takes too, so b stays a
-// subset of a.  Finally the histograms and counters of the segment are
-// cleared for the next selection.
-constexpr int kFinThreads = 1024;
-
-__global__ void __launch_bounds__(kFinThreads)
-k_sel_finish(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a,
-             int n_b, int32_t* __restrict__ out_b, int64_t stride_b) {
-    __shared__ __align__(16) uint32_t h3[2][kRadixBins];
-    __shared__ uint32_t s_wsum[kFinThreads / 32];
+    // the CTA that reports last sees every survivor and finishes the selection
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_base[0] = atomicAdd(cnt + 7, 1u) == gridDim.x - 1 ? 1u : 0u;
+    __syncthreads();
+    if (!s_base[0]) return;
+    __threadfence();
+    __shared__ uint32_t s_wsum[kPassThreads / 32];
     __shared__ Thr s_thr[2];
-    __shared__ uint32_t s_ctr[2];     // a tie ranks, b tie ranks
-    const int seg = blockIdx.x, tid = threadIdx.x;
-    for (int i = tid; i < 2 * kRadixBins; i += kFinThreads) (&h3[0][0])[i] = 0;
-    if (tid < 2) s_ctr[tid] = 0;
-    pdl_begin();
-    uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
-    uint32_t* h1 = wk.hist + (int64_t)seg * 3 * kRadixBins;
-    __shared__ uint32_t s_words[kPlanWords];
-    const Plan2 P = plan_read(cnt + kPlanWord0, s_words);
-    bool lvl3[2];
-    uint32_t need3[2], ns[2];
-    for (int t = 0; t < 2; ++t) {
-        lvl3[t] = P.len[t] && !P.eq2[t];
-        need3[t] = lvl3[t] ? P.need2[t] - P.q[t].above : 0u;
-        ns[t] = cnt[t == 0 ? 4 : 5];                     // survivors
-    }
-    // with a shared list and one digit-2 threshold both targets have the same survivors
-    const bool one_list = P.shared && lvl3[0] && lvl3[1] && P.q[0].c == P.q[1].c;
-    const uint2* surv[2] = {reinterpret_cast<const uint2*>(wk.surv1) + seg * wk.cand_stride,
-                            reinterpret_cast<const uint2*>(wk.surv2) + seg * wk.cand_stride};
-    for (int t = 0; t < 2; ++t)
-        if (lvl3[t])
-            for (uint32_t i = tid; i < ns[t]; i += kFinThreads) atomicAdd(&h3[t][digit(surv[t][i].x, 3)], 1u);
-    __syncthreads();
-    Thr r3[2];
-    {
-        Thr ra[2], rb[2];
-        const uint32_t none[2] = {0u, 0u};
-        const uint32_t na_only[2] = {need3[0], 0u}, nb_only[2] = {need3[1], 0u};
-        block_thresholds2<kFinThreads>(h3[0], na_only, none, s_wsum, s_thr, ra);
-        block_thresholds2<kFinThreads>(h3[1], nb_only, none, s_wsum, s_thr, rb);
-        r3[0] = ra[0];
-        r3[1] = rb[0];
-    }
-    uint32_t ties[2];
-    for (int t = 0; t < 2; ++t) ties[t] = lvl3[t] ? need3[t] - r3[t].above : 0u;
-    const bool coupled = one_list && r3[0].c == r3[1].c;
-    int32_t* out[2] = {out_a + (int64_t)seg * stride_a, out_b ? out_b + (int64_t)seg * stride_b : nullptr};
-    float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
-    for (int t = 0; t < 2; ++t) {
-        if (!lvl3[t] || (one_list && t == 1)) continue;
-        const uint32_t tmask = one_list ? 3u : (1u << t);
-        for (uint32_t i0 = 0; i0 < ns[t]; i0 += kFinThreads) {
-            const uint32_t i = i0 + tid;
-            const bool in = i < ns[t];
-            const uint2 kv = in ? surv[t][i] : make_uint2(0u, 0u);
-            const uint32_t d3 = digit(kv.x, 3);
-            bool on[2], eqv[2];
-            for (int u = 0; u < 2; ++u) {
-                on[u] = in && ((tmask >> u) & 1u);
-                eqv[u] = on[u] && d3 == r3[u].c;
-            }
-            const uint32_t rk_a = warp_claim(eqv[0], &s_ctr[0]);
-            const uint32_t rk_b = coupled ? rk_a : warp_claim(eqv[1], &s_ctr[1]);
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const uint32_t rk = u == 0 ? rk_a : rk_b;
-                const bool tk = on[u] && (d3 > r3[u].c || (eqv[u] && rk < ties[u]));
-                const uint32_t os = warp_claim(tk, cnt + (u == 0 ? 0 : 2));
-                if (tk) {
-                    out[u][os] = (int32_t)kv.y;
-                    if (u == 0 && va) va[os] = key_value(kv.x);
-                }
-            }
-        }
-    }
-    // leave the workspace as csa2_workspace_init does: histograms and counters zero
-    __syncthreads();
-    for (int i = tid; i < 3 * kRadixBins; i += kFinThreads) h1[i] = 0;
-    if (tid < kSelCounters) cnt[tid] = 0;
+    __shared__ uint32_t s_ctr[2];
+    finish_level3<kPassThreads>(wk, seg, P, out_a, vals_a, stride_a, out_b, stride_b,
+                                reinterpret_cast<uint32_t*>(stage_dyn), s_wsum, s_thr, s_ctr);
 }
 
 // ---------------------------------------------------------------- small segments
@@ -935,7 +941,7 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
                                int64_t stride_a, int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st,
                                bool hist_ready) {
     // the histograms and counters are zero on entry (workspace initialisation,
-    // then every k_sel_finish clears what its selection used); without a
+    // then every selection's last CTA clears what it used); without a
     // histogram from the scoring kernel, build level 1 here
     cudaError_t e;
     const unsigned chunks = (unsigned)((src.n + kPassChunk - 1) / kPassChunk);
@@ -956,11 +962,8 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
     if (e != cudaSuccess) return e;
     // candidates: at most the segment size; spread over up to 148 CTAs
     const unsigned g2 = chunks < 148 ? (chunks ? chunks : 1) : 148;
-    e = launch_pdl(k_sel_pass2, dim3(g2, (unsigned)nseg), dim3(kPassThreads), kStageSmem, st, wk, n_a, out_a, vals_a,
-                   stride_a, n_b, out_b, stride_b);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(k_sel_finish, dim3((unsigned)nseg), dim3(kFinThreads), 0, st, wk, n_a, out_a, vals_a, stride_a,
-                      n_b, out_b, stride_b);
+    return launch_pdl(k_sel_pass2, dim3(g2, (unsigned)nseg), dim3(kPassThreads), kStageSmem, st, wk, n_a, out_a,
+                      vals_a, stride_a, n_b, out_b, stride_b);
 }
 
 }  // namespace csa2
