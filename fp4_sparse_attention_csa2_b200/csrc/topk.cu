@@ -836,12 +836,14 @@ k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict_
 // every CTA sums the kClCtas histograms through distributed shared memory and
 // finds the same threshold digit; the following pass selects digits above it
 // and histograms the next digit of the elements equal to it.  Output slots and
-// exact-tie ranks are claimed on counters in CTA 0.
+// exact-tie ranks are claimed on counters in CTA 0, once per CTA and digit.
 __global__ void __launch_bounds__(kClThreads)
 k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, float* __restrict__ out_vals, int64_t out_stride) {
     cg::cluster_group cl = cg::this_cluster();
     __shared__ __align__(16) uint32_t hist[3][kRadixBins];
     __shared__ uint32_t s_wsum[kClThreads / 32];
+    __shared__ uint64_t s_wsum64[kClThreads / 32];
+    __shared__ uint32_t s_base[2];
     __shared__ ClPlan s_plan;
     __shared__ uint32_t s_cnt[2];               // CTA 0's: output slots, exact-tie ranks
     const uint32_t rank = cl.block_rank();
@@ -887,41 +889,60 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, float* __restrict_
         const bool all_eq = pl.eq == need - pl.above;
         // select the elements of the current prefix whose digit is above c (and
         // those equal to c when exactly the missing number of them exist); the
-        // others equal to c go on to the next digit
+        // others equal to c go on to the next digit.  On the last digit the
+        // ones equal to c are exact ties of the full key: the first `need - above`
+        // in claim order win.  Slots and tie ranks are claimed once per CTA
+        // (a block-wide scan, one remote atomic on CTA 0's counters).
+        const bool ties_now = level == 3 && !all_eq;
+        uint32_t take = 0, tie = 0, ntake = 0, ntie = 0;
 #pragma unroll
         for (int k = 0; k < kClPer; ++k) {
             const uint32_t key = keys[k];
             const bool in = key && (key & mask) == prefix;
             const uint32_t d = (key >> shift) & dmask;
-            const bool take = in && (d > pl.c || (d == pl.c && all_eq));
-            if (level < 3 && in && d == pl.c && !all_eq) atomicAdd(&hist[level][digit(key, level + 1)], 1u);
-            const uint32_t os = warp_claim(take, cnt_out);
-            if (take) {
-                o[os] = ids[k];
-                if (ov) ov[os] = key_value(key);
-            }
+            const bool tk = in && (d > pl.c || (d == pl.c && all_eq));
+            const bool eq = in && d == pl.c && !all_eq;
+            if (level < 3 && eq) atomicAdd(&hist[level][digit(key, level + 1)], 1u);
+            take |= (uint32_t)tk << k;
+            ntake += tk;
+            if (ties_now && eq) { tie |= 1u << k; ++ntie; }
         }
-        if (all_eq) {
+        uint32_t tie_rank = 0;
+        const uint32_t need_ties = ties_now ? need - pl.above : 0u;
+        if (ties_now) {
+            uint64_t tot;
+            const uint64_t pre = block_excl_scan4<kClThreads>((uint64_t)ntie, s_wsum64, &tot);
+            if (tid == 0) s_base[1] = field16(tot, 0) ? atomicAdd(cnt_tie, field16(tot, 0)) : 0u;
+            __syncthreads();
+            tie_rank = s_base[1] + field16(pre, 0);
+#pragma unroll
+            for (int k = 0; k < kClPer; ++k)
+                if ((tie >> k) & 1u) {
+                    if (tie_rank < need_ties) { take |= 1u << k; ++ntake; }
+                    ++tie_rank;
+                }
+        }
+        {
+            uint64_t tot;
+            const uint64_t pre = block_excl_scan4<kClThreads>((uint64_t)ntake, s_wsum64, &tot);
+            if (tid == 0) s_base[0] = field16(tot, 0) ? atomicAdd(cnt_out, field16(tot, 0)) : 0u;
+            __syncthreads();
+            uint32_t os = s_base[0] + field16(pre, 0);
+#pragma unroll
+            for (int k = 0; k < kClPer; ++k)
+                if ((take >> k) & 1u) {
+                    o[os] = ids[k];
+                    if (ov) ov[os] = key_value(keys[k]);
+                    ++os;
+                }
+            __syncthreads();   // s_base is rewritten by the next level
+        }
+        if (all_eq || level == 3) {
             done = true;
         } else {
             need -= pl.above;
             prefix |= pl.c << shift;
             mask |= dmask << shift;
-            if (level == 3) {
-                // exact ties of the full key: the first `need` claimants win
-#pragma unroll
-                for (int k = 0; k < kClPer; ++k) {
-                    const uint32_t key = keys[k];
-                    const bool eq = key && key == prefix;
-                    const uint32_t ts = warp_claim(eq, cnt_tie);
-                    const bool take = eq && ts < need;
-                    const uint32_t os = warp_claim(take, cnt_out);
-                    if (take) {
-                        o[os] = ids[k];
-                        if (ov) ov[os] = key_value(key);
-                    }
-                }
-            }
         }
     }
     cl.sync();   // no CTA leaves while another may still read its shared memory
