@@ -401,8 +401,8 @@ constexpr int kPlanWord0 = 9;
 constexpr int kPlanWords = 19;
 static_assert(kPlanWord0 + kPlanWords <= kSelCounters, "plan words");
 
-// Level-1 words (written by k_sel_plan1): both targets' level-1 plans and
-// whether their candidate lists are one.
+// Level-1 words: both targets' level-1 plans and whether their candidate lists
+// are one (written by pass 1's last CTA with the level-2 words).
 __device__ __forceinline__ void plan_write1(uint32_t* w, const Plan1& pa, const Plan1& pb) {
     const Plan1* pp[2] = {&pa, &pb};
     for (int t = 0; t < 2; ++t) {
@@ -503,9 +503,11 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
             keys[k] = (ids[k] >= 0 && ids[k] < nvalid) ? ordered_key(raw[k]) : 0u;
     };
     if (base < n_items) issue_chunk(base);
-    __shared__ uint32_t s_words[kPlanWords];
-    const Plan2 P1w = plan_read(cnt + kPlanWord0, s_words);   // level-1 part (k_sel_plan1)
-    const Plan1 pa = P1w.p[0], pb = P1w.p[1];
+    // level-1 plans of both targets from the scorer's histogram (two 16-byte
+    // loads per thread, one block-wide scan), while the chunk's loads are in flight
+    Plan1 pa, pb;
+    plans_level1<kPassThreads>(wk.hist + (int64_t)seg * 3 * kRadixBins, (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr,
+                               pa, pb);
     int32_t* oa = out_a + (int64_t)seg * stride_a;
     int32_t* ob = out_b ? out_b + (int64_t)seg * stride_b : nullptr;
     float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
@@ -624,21 +626,10 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
         P.q[0] = qa[0];
         P.q[1] = qb[0];
     }
-    if (tid == 0) plan_write2(cnt + kPlanWord0, P);
-}
-
-// Level-1 plans of both targets from the scorer's histogram, once per segment
-// (every CTA of pass 1 then reads a few words instead of scanning the histogram).
-__global__ void __launch_bounds__(kPassThreads) k_sel_plan1(SelWork wk, int n_a, int n_b) {
-    pdl_begin();
-    __shared__ uint32_t s_wsum[kPassThreads / 32];
-    __shared__ Thr s_thr[2];
-    const int seg = blockIdx.x;
-    uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
-    Plan1 pa, pb;
-    plans_level1<kPassThreads>(wk.hist + (int64_t)seg * 3 * kRadixBins, (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr,
-                               pa, pb);
-    if (threadIdx.x == 0) plan_write1(cnt + kPlanWord0, pa, pb);
+    if (tid == 0) {
+        plan_write1(cnt + kPlanWord0, pa, pb);
+        plan_write2(cnt + kPlanWord0, P);
+    }
 }
 
 // Digit 3 and exact ties of both targets among the digit-2 survivors, run by
@@ -971,8 +962,6 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
         e = launch_pdl(k_sel_hist, dim3(grid), dim3(kPassThreads), 0, st, src, wk);
         if (e != cudaSuccess) return e;
     }
-    e = launch_pdl(k_sel_plan1, dim3((unsigned)nseg), dim3(kPassThreads), 0, st, wk, n_a, n_b);
-    if (e != cudaSuccess) return e;
     constexpr size_t kStageSmem = 2 * kPassChunk * sizeof(uint2);
     e = cudaFuncSetAttribute(k_sel_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStageSmem);
     if (e != cudaSuccess) return e;
