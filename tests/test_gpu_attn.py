@@ -54,6 +54,8 @@ def _check(w, ref, dev, q, topk, window=None, sm_scale=0.0):
     ("long64k", 3000, {"T": 4}),
     ("batch32_paged", 20000, {"batch": 4}),
     ("append_mq", 5000, {"batch": 2}),
+    ("long64k", 4000, {"H": 32}),               # tensor-core path with 32 heads
+    ("long64k", 3000, {"H": 48}),               # CUDA-core path; the merge with a head count that does not divide 256
 ])
 def test_attention_on_oracle_topk(name, L, kw):
     w = wl.scaled(wl.WORKLOADS[name], L, **kw)
