@@ -18,8 +18,8 @@
 //      group's bf16 queries to fp16 scaled by a power of two per head (exact)
 //      in the same layout;
 //   2. S[pos, head] = V Q^T : tcgen05.mma M=128 (positions), N=HG, K=D;
-//   3. logits to shared memory transposed; per-head max and exp over the 128
-//      positions; P (fp16) written K-major;
+//   3. softmax read straight from the tensor memory (thread = position):
+//      per-head max and exp over the 128 positions; P (fp16) written K-major;
 //   4. O^T[d, head] = V^T P^T : the same V bytes read through an MN-major
 //      descriptor, one M=128 slab of d per accumulator;
 //   5. unnormalised partial output ([d][head]) and (max, sum) per head in
@@ -35,7 +35,6 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kWorkers = 256;               // 8 warps: rows, queries, dequantisation, softmax, stores
 constexpr int kThreads = kWorkers + 32;     // + the warp that allocates TMEM and issues the MMAs
-constexpr int kZStride = kRows + 4;   // padded row of the transposed logits (floats)
 
 struct Params {
     DevCache c;
@@ -53,7 +52,7 @@ struct Params {
 
 struct Misc {
     float fac[64];               // per head of the group: softmax scale * log2(e) / query scale
-    float red[16][64];           // per head partial max / sum of the threads that share it
+    float red[8][64];            // per head: the four warps' maxima (rows 0-3) and sums (rows 4-7)
     int32_t pos[kRows];
     uint64_t row_bar;            // the chunk's row copies (one arrival per row)
     uint64_t kb_bar[8];          // K block k of V written (one arrival per worker)
@@ -81,6 +80,67 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     return r;
 }
 
+// Named barrier of one worker warpgroup (128 threads; ids 2 and 3).
+__device__ __forceinline__ void group_sync(int wgrp) {
+    asm volatile("bar.sync %0, 128;" ::"r"(2 + wgrp) : "memory");
+}
+
+// The float an order-preserving key came from (-0 comes back as +0).
+__device__ __forceinline__ float key_to_float(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Softmax, first half, for NV heads c0.. of this thread's position: the
+// scaled logits (-inf where the position is empty) into z, and this warp's
+// maximum of each head into red[quad][head].
+template <int NV>
+__device__ __forceinline__ void logits_max(uint32_t trow, int c0, bool valid, Misc* misc, int quad, int lane, float* z) {
+    float v[NV];
+    if constexpr (NV == 8) tc::tmem_ld8(trow + c0, v);
+    else tc::tmem_ld16(trow + c0, v);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        z[i] = valid ? v[i] * misc->fac[c0 + i] : -INFINITY;
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, ordered_key(z[i]));
+        if (lane == i) misc->red[quad][c0 + i] = key_to_float(mk);
+    }
+}
+
+// Softmax, second half: p = 2^(z - m) per head, rounded to fp16 and stored in
+// the K-major P operand (row = head, 64 positions per 128-byte row, chunk pc,
+// element el); this warp's sum of the rounded values into red[4 + quad][head].
+// The sums leave the warp by an exchange that halves the values a lane
+// carries at each step (NV - 1 shuffles for NV heads, not 5 NV); lanes 2 j
+// and 2 j + 1 end with head j mod NV.
+template <int NV>
+__device__ __forceinline__ void probs_sums(uint8_t* prow, int pc, int el, int c0, Misc* misc, int quad, int lane,
+                                           const float* z) {
+    float sv[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int h = c0 + i;
+        const float m = fmaxf(fmaxf(misc->red[0][h], misc->red[1][h]), fmaxf(misc->red[2][h], misc->red[3][h]));
+        const float e = m == -INFINITY ? 0.0f : exp2f(z[i] - m);
+        const __half ph = __float2half_rn(e);
+        *reinterpret_cast<__half*>(prow + tc::sw128_offset(h, pc) + 2 * el) = ph;
+        sv[i] = __half2float(ph);
+    }
+#pragma unroll
+    for (int w = NV / 2; w >= 1; w >>= 1) {
+        const bool up = (lane & (2 * w)) != 0;
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+            const float send = up ? sv[i] : sv[i + w];
+            const float keep = up ? sv[i + w] : sv[i];
+            sv[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2 * w);
+        }
+    }
+    sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], 1);
+#pragma unroll
+    for (int o = 2 * NV; o < 32; o <<= 1) sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], o);
+    if (lane < 2 * NV && (lane & 1) == 0) misc->red[4 + quad][c0 + (lane >> 1)] = sv[0];
+}
+
 // Named barrier of the kWorkers worker threads (the MMA warp is not part of it).
 __device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kWorkers) : "memory"); }
 
@@ -90,9 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     const int D = p.c.dim, H = p.H, HG = p.HG;
     const int nkb = D / 64;                     // 64-wide K blocks of the V tile
     uint8_t* sV = smem;                         // nkb x [128 rows x 128 B]
-    uint8_t* sQ = smem + p.off_q;               // nkb x [HG rows x 128 B]; later logits + P
-    float* sZ = reinterpret_cast<float*>(sQ);   // [HG][kZStride] (after S is computed)
-    uint8_t* sP = sQ + ((HG * kZStride * 4 + 1023) & ~1023);   // 2 x [HG rows x 128 B]
+    uint8_t* sQ = smem + p.off_q;               // nkb x [HG rows x 128 B]; later P
+    uint8_t* sP = sQ;                           // 2 x [HG rows x 128 B] (after S is computed)
     uint8_t* sStage = smem + p.off_stage;       // [128 rows][stage_stride]: the FP4 rows as fetched (inside sV)
     Misc* misc = reinterpret_cast<Misc*>(smem + p.off_misc);
 
@@ -300,82 +359,82 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         }
     }
 
-    // ---- logits to shared memory, transposed: z[h][pos]; lane = position, the
-    // two warpgroups take one half of the group's heads each (HG >= 32)
+    // ---- softmax straight from the tensor memory.  Thread = position (the
+    // TMEM lane of its warp's quarter); each warpgroup takes one half of the
+    // group's heads.  Per head: the maximum over the 128 positions (a
+    // warp-wide max of order-preserving integer keys, then the four warps'
+    // through shared memory); p = 2^(z - m) in fp16, stored straight into the
+    // K-major P operand; the sum of the fp16 values as the MMA will use them.
     ok = tc::mbar_wait(&misc->s_bar, 0) && ok;
     tc::fence_after_sync();
-    const int ngrp = HG >= 32 ? 2 : 1;
     const int wgrp = warp >> 2, quad = warp & 3;
-    if (ok && wgrp < ngrp) {
-        const int rr = quad * 32 + lane;
-        const bool valid = misc->pos[rr] >= 0;
-        const int hc = HG / ngrp;
-        for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
-            float v[16];
-            tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
+    const int hc = HG / 2;                           // heads of a warpgroup: 8, 16 or 32
+    ok = __all_sync(0xffffffffu, ok);                // warp-uniform from here on
+    const int pos = quad * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const bool valid = misc->pos[pos] >= 0;
+    float zz[32];
+    if (ok) {
+        if (hc == 8) {
+            logits_max<8>(trow, wgrp * 8, valid, misc, quad, lane, zz);
+        } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sZ[(c0 + i) * kZStride + rr] = valid ? v[i] * misc->fac[c0 + i] : -INFINITY;
+            for (int blk = 0; blk < 2; ++blk)
+                if (blk * 16 < hc) logits_max<16>(trow, wgrp * hc + blk * 16, valid, misc, quad, lane, zz + 16 * blk);
         }
     }
-    workers_sync();
-
-    // ---- softmax statistics: nq = 256 / HG threads per head, each over 128 / nq positions
-    const int nq = kWorkers / HG, per = kRows / nq;
-    const int h = tid % HG, qt = tid / HG;
-    const float* z = sZ + h * kZStride + qt * per;
-    float m = -INFINITY, l = 0.0f;
-    for (int i = 0; i < per; ++i) m = fmaxf(m, z[i]);
-    misc->red[qt][h] = m;
-    workers_sync();
-    for (int k = 0; k < nq; ++k) m = fmaxf(m, misc->red[k][h]);
-    {
-        uint8_t* blk = sP + ((qt * per) >> 6) * (HG * 128);
-        const int c_first = ((qt * per) & 63) >> 3;
-        for (int c = 0; c < per / 8; ++c) {
-            uint32_t hv[4];
+    group_sync(wgrp);
+    if (ok) {
+        uint8_t* prow = sP + (pos >> 6) * (HG * 128);
+        const int pc = (pos & 63) >> 3, el = pos & 7;
+        if (hc == 8) {
+            probs_sums<8>(prow, pc, el, wgrp * 8, misc, quad, lane, zz);
+        } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float e0 = m == -INFINITY ? 0.0f : exp2f(z[8 * c + 2 * k] - m);
-                const float e1 = m == -INFINITY ? 0.0f : exp2f(z[8 * c + 2 * k + 1] - m);
-                __half2 hh = __floats2half2_rn(e0, e1);
-                const float2 back = __half22float2(hh);   // sum what the MMA will use
-                l += back.x + back.y;
-                memcpy(&hv[k], &hh, 4);
-            }
-            *reinterpret_cast<uint4*>(blk + tc::sw128_offset(h, c_first + c)) =
-                make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            for (int blk = 0; blk < 2; ++blk)
+                if (blk * 16 < hc) probs_sums<16>(prow, pc, el, wgrp * hc + blk * 16, misc, quad, lane, zz + 16 * blk);
         }
     }
     tc::fence_proxy_async_smem();                     // P is an MMA operand
     tc::mbar_arrive(&misc->p_bar);
-    workers_sync();                                   // every read of red[] (the maxima) is done
-    misc->red[qt][h] = l;
-    workers_sync();
-    if (ok && tid < HG) {
-        float* ml = p.part_ml + (((int64_t)seg * p.nchunk + chunk) * H + h_base + tid) * 2;
-        float sum = 0.0f;
-        for (int k = 0; k < nq; ++k) sum += misc->red[k][tid];
-        ml[0] = m;                                   // thread tid < HG holds local head tid's maximum
-        ml[1] = sum;
+    group_sync(wgrp);
+    {
+        const int t = tid & 127;                      // thread of the warpgroup
+        if (ok && t < hc) {
+            const int h = wgrp * hc + t;
+            const float m = fmaxf(fmaxf(misc->red[0][h], misc->red[1][h]), fmaxf(misc->red[2][h], misc->red[3][h]));
+            const float l = (misc->red[4][h] + misc->red[5][h]) + (misc->red[6][h] + misc->red[7][h]);
+            float* ml = p.part_ml + (((int64_t)seg * p.nchunk + chunk) * H + h_base + h) * 2;
+            ml[0] = m;
+            ml[1] = l;
+        }
     }
 
     // ---- unnormalised partial output, [d][head], slab by slab as the MMA warp
-    // finishes them (lane = d within the slab; the two warpgroups take one half
-    // of the group's heads each; 16-byte stores)
-    if (wgrp < ngrp) {
+    // finishes them (lane = d within the slab; each warpgroup takes one half
+    // of the group's heads; 16-byte stores)
+    {
         float* po = p.part_o + ((int64_t)seg * p.nchunk + chunk) * H * D + h_base;
-        const int hc = HG / ngrp;
         for (int s2 = 0; s2 < D / 128; ++s2) {
             ok = tc::mbar_wait(&misc->o_bar[s2], 0) && ok;
             tc::fence_after_sync();
             if (!ok) continue;
             const int d = s2 * 128 + quad * 32 + lane;
-            for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
-                float v[16];
-                tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(HG + s2 * HG + c0), v);
-                float4* dst = reinterpret_cast<float4*>(po + (int64_t)d * H + c0);
+            const uint32_t tcol = trow + (uint32_t)(HG + s2 * HG);
+            if (hc == 8) {
+                float v[8];
+                tc::tmem_ld8(tcol + wgrp * 8, v);
+                float4* dst = reinterpret_cast<float4*>(po + (int64_t)d * H + wgrp * 8);
+                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+            } else {
+                for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
+                    float v[16];
+                    tc::tmem_ld16(tcol + c0, v);
+                    float4* dst = reinterpret_cast<float4*>(po + (int64_t)d * H + c0);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
             }
         }
     }
@@ -393,8 +452,8 @@ int attn_tc_row_bytes(int D) { return (D / 2 + D / 16 + 15) & ~15; }
 size_t attn_tc_smem(int D, int HG, uint32_t stage_bytes, uint32_t* off_q, uint32_t* off_stage, uint32_t* off_misc) {
     const uint32_t v = (uint32_t)(D / 64) * kRows * 128;
     const uint32_t qbytes = (uint32_t)(D / 64) * HG * 128;
-    const uint32_t zbytes = (((uint32_t)HG * kZStride * 4 + 1023) & ~1023u) + 2u * HG * 128;
-    const uint32_t qreg = ((qbytes > zbytes ? qbytes : zbytes) + 1023) & ~1023u;
+    const uint32_t pbytes = 2u * HG * 128;     // P, in the query's place once S is computed
+    const uint32_t qreg = ((qbytes > pbytes ? qbytes : pbytes) + 1023) & ~1023u;
     *off_q = v;
     *off_stage = (v - stage_bytes) & ~1023u;   // the tail of the V tile: rows land there before the tile is written
     *off_misc = v + qreg;
