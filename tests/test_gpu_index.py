@@ -21,6 +21,11 @@ CASES = [
     ("long64k", 5000, {"T": 3}),                # causal among 3 query tokens
     ("batch32_paged", 30000, {"batch": 5}),     # paged, ragged lengths
     ("append_mq", 9000, {"batch": 2}),          # T = 4
+    ("tiny4k", 512, {}),                        # L = K: the pool is every position
+    ("long64k", 16384, {}),                     # L = K = 16,384, the largest pool
+    ("long64k", 16385, {}),                     # one position more than the largest pool
+    ("long64k", 20000, {"pool_k": 2048}),       # k = K: both targets cut at the same place
+    ("long64k", 20000, {"pool_k": 64, "top_k": 1}),   # k = 1
 ]
 
 
