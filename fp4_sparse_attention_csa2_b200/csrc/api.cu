@@ -1,6 +1,7 @@
 // Host side of the libcsa2 C ABI: argument validation, workspace layout and
 // kernel dispatch.  Every entry point validates on the host, then only
 // enqueues work on the caller's stream.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -293,8 +294,12 @@ csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, in
     Layout L;
     s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
-    // the split-softmax merge keeps one weight per (chunk, head) in shared memory
-    if (sizeof(float) * ((size_t)L.nchunk * H + 2 * (size_t)H + 256 + (4 * (256 / H) + 1) * (size_t)H) > 200 * 1024)
+    // the split-softmax merge keeps one weight per (chunk, head) in shared
+    // memory; chunks of the kernel that will run (the workspace is sized for
+    // the smallest chunk of any)
+    const int rows = attn_tc_supported(dev_cache(cache), H) ? attn_tc_rows_per_chunk() : attn_rows_per_chunk();
+    const int64_t nchunk_run = std::max<int64_t>(1, ((int64_t)window + top_k + rows - 1) / rows);
+    if (sizeof(float) * ((size_t)nchunk_run * H + 2 * (size_t)H + 256 + (4 * (256 / H) + 1) * (size_t)H) > 200 * 1024)
         return CSA2_ERR_UNSUPPORTED;
     if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
     AttnWork aw;

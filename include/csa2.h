@@ -218,7 +218,12 @@ CSA2_API csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const v
  *     out   = sum_{t in S} softmax(z)_t v_t        fp32 [batch][T][H][dim]
  *     lse   = log sum_{t in S} exp(z_t)            fp32 [batch][T][H], nullable
  * q is bf16 [batch][T][H][dim] with H a multiple of 16, at most 64.  An empty
- * S gives out = 0, lse = -inf.
+ * S gives out = 0, lse = -inf.  top_k and window are each at most 16,384;
+ * CSA2_ERR_UNSUPPORTED when the split-softmax merge's weights (one float per
+ * (chunk, head); chunks of 128 entries on the tensor-core path -- dim a
+ * multiple of 128 and H in {16, 32, 64} -- else of 32) would not fit in
+ * 200 KiB of shared memory, e.g. H = 64 with window + top_k above 24,864 on
+ * the 32-entry path.
  * topk entries < -1 or >= seq_lens[b] set CSA2_ERR_DEVICE_BOUNDS.
  */
 CSA2_API csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, int T, int H,

@@ -128,3 +128,16 @@ def test_out_of_range_topk_flags_status(small):
                          None, ws)
     assert csa2.read_device_status(ws) == csa2.ERR_DEVICE_BOUNDS
     assert np.all(np.isfinite(out.cpu().numpy()))
+
+
+def test_largest_topk_and_window():
+    # the largest attended set the boundary accepts: top-k 16,384 and window
+    # 16,384 (the pool bound), 257 chunks of 128 entries to merge
+    L = 40000
+    w = wl.scaled(wl.WORKLOADS["long64k"], L, pool_k=16384, top_k=16384, window=16384)
+    l0 = wl.layer_queries(w, 0)
+    ref = build_ref_cache(w, layers=[l0])
+    dev = build_gpu_cache(w, q_idx0=l0["q_idx"])
+    rng = np.random.default_rng(11)
+    topk = rng.choice(L, (1, 1, w.top_k), replace=False).astype(np.int32)   # partly inside the window
+    _check(w, ref, dev, wl.layer_queries(w, 3)["q"], topk)
