@@ -279,14 +279,12 @@ def run_ours(args, world, rank):
     traffic = profiled_traffic(source_hash(SCORE_SOURCES))
 
     # end to end through the public API with host buffers: per step, copy the
-    # queries of every layer from pinned host memory, run the stack, read back
-    # every layer's output and log-sum-exp
-    host_in = [{k: v.pin_memory() for k, v in L.items()} for L in layers]
-    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in stack.out]
-    host_lse = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in stack.lse]
-    h2d = sum(v.numel() * v.element_size() for l, L in enumerate(host_in) for k, v in L.items()
-              if k == "q" or w.pattern[l] != "U")
-    d2h = sum(o.numel() * o.element_size() for o in host_out + host_lse)
+    # step's inputs (every layer's queries; the index queries and head weights
+    # of the Full and Reindex layers) from pinned host memory, run the stack,
+    # read back every layer's output and log-sum-exp: one flat copy each way
+    host_in, host_out = stack.host_buffers(layers)
+    h2d = host_in.numel()
+    d2h = host_out.numel()
     Ke = max(3, min(K, 100))
     barrier(world)
     torch.cuda.synchronize()
@@ -294,14 +292,9 @@ def run_ours(args, world, rank):
     with torch.cuda.stream(stream):
         x0.record(stream)
         for i in range(Ke):
-            for l, L in enumerate(host_in):
-                for k, v in L.items():
-                    if k == "q" or w.pattern[l] != "U":
-                        stack.layers[l][k].copy_(v, non_blocking=True)
+            stack.inputs.copy_(host_in, non_blocking=True)
             stack.step(reps[i % len(reps)])
-            for l in range(len(w.pattern)):
-                host_out[l].copy_(stack.out[l], non_blocking=True)
-                host_lse[l].copy_(stack.lse[l], non_blocking=True)
+            host_out.copy_(stack.outputs, non_blocking=True)
             stream.synchronize()
         x1.record(stream)
     torch.cuda.synchronize()
@@ -336,7 +329,7 @@ def run_ours(args, world, rank):
             "step_bytes_algorithmic": step_bytes(w, lens),
             "e2e": {"value": round(e2e_value, 1), "unit": "layer-steps/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": Ke,
-                    "path": "python binding -> C ABI csa2_layer_step per layer, pinned host buffers, sync per step"},
+                    "path": "python binding -> C ABI csa2_layer_step per layer; one pinned host buffer each way (the inputs, the outputs), sync per step"},
             "gpu_launches": None if launches_per_step is None else launches_per_step * K,
             "gpu_launches_per_step": launches_per_step,
             "clocks": clk.summary(),

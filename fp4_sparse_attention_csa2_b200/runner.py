@@ -38,18 +38,72 @@ def build_replicas(w, n_rep, seed, lens):
     return reps
 
 
+FLAT_ALIGN = 256   # every tensor of a flat buffer starts on this byte boundary (the C ABI wants 16)
+
+
+def flat_views(specs, device, pin=False):
+    """One uint8 buffer holding tensors of the given (shape, dtype) specs, each
+    starting on a FLAT_ALIGN-byte boundary; returns (buffer, [views]).  One
+    copy of the buffer moves all of them (a step's inputs or outputs)."""
+    offs, off = [], 0
+    for shape, dtype in specs:
+        n = 1
+        for d in shape:
+            n *= int(d)
+        offs.append((off, n * torch.empty((), dtype=dtype).element_size()))
+        off = (off + offs[-1][1] + FLAT_ALIGN - 1) // FLAT_ALIGN * FLAT_ALIGN
+    buf = torch.zeros(max(off, 1), dtype=torch.uint8, device=device)
+    if pin:
+        buf = buf.pin_memory()
+    views = [buf[o:o + nb].view(dtype).view(shape) for (o, nb), (shape, dtype) in zip(offs, specs)]
+    return buf, views
+
+
 class Stack:
-    """Device buffers of one decode step and the C-ABI calls that run it."""
+    """Device buffers of one decode step and the C-ABI calls that run it.
+
+    The inputs a step consumes (every layer's q; q_idx and head weights of
+    the Full and Reindex layers) live in one flat device buffer, `inputs`, and
+    every layer's out and lse in another, `outputs`, so a host round trip of a
+    step is one copy each way (`host_buffers` gives matching pinned host
+    buffers)."""
 
     def __init__(self, w, layers, ws):
         self.w, self.ws = w, ws
         B, T = w.batch, w.T
-        self.layers = [{k: v.cuda() for k, v in L.items()} for L in layers]
+        self.modes = [{"F": csa2.FULL, "R": csa2.REINDEX, "U": csa2.REUSE}[m] for m in w.pattern]
+        self.in_keys = [[k for k in L if k == "q" or m != csa2.REUSE] for L, m in zip(layers, self.modes)]
+        in_specs = [(tuple(L[k].shape), L[k].dtype) for L, ks in zip(layers, self.in_keys) for k in ks]
+        self.inputs, views = flat_views(in_specs, "cuda")
+        it = iter(views)
+        self.layers = []
+        for L, ks in zip(layers, self.in_keys):
+            d = {}
+            for k, v in L.items():
+                if k in ks:
+                    d[k] = next(it)
+                    d[k].copy_(v)
+                else:
+                    d[k] = v.cuda()
+            self.layers.append(d)
         self.pool = torch.zeros((B, T, w.pool_k), dtype=torch.int32, device="cuda")
         self.topk = torch.zeros((B, T, w.top_k), dtype=torch.int32, device="cuda")
-        self.out = [torch.empty((B, T, w.H, w.D), dtype=torch.float32, device="cuda") for _ in w.pattern]
-        self.lse = [torch.empty((B, T, w.H), dtype=torch.float32, device="cuda") for _ in w.pattern]
-        self.modes = [{"F": csa2.FULL, "R": csa2.REINDEX, "U": csa2.REUSE}[m] for m in w.pattern]
+        n = len(w.pattern)
+        out_specs = [((B, T, w.H, w.D), torch.float32)] * n + [((B, T, w.H), torch.float32)] * n
+        self.outputs, views = flat_views(out_specs, "cuda")
+        self.out, self.lse = views[:n], views[n:]
+
+    def host_buffers(self, layers):
+        """Pinned host copies of `inputs` (filled from the host-side layers)
+        and of `outputs` (to be read back into)."""
+        in_specs = [(tuple(L[k].shape), L[k].dtype) for L, ks in zip(layers, self.in_keys) for k in ks]
+        h_in, views = flat_views(in_specs, "cpu", pin=True)
+        it = iter(views)
+        for L, ks in zip(layers, self.in_keys):
+            for k in ks:
+                next(it).copy_(L[k])
+        h_out = torch.empty(self.outputs.numel(), dtype=torch.uint8).pin_memory()
+        return h_in, h_out
 
     def step(self, cache):
         for l, m in enumerate(self.modes):
