@@ -94,7 +94,20 @@ def _check(code, what):
 
 
 def _p(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device pointer of a tensor the library reads or writes: a contiguous
+    CUDA tensor (a host tensor would hand the kernels a host address)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libcsa2 takes CUDA tensors; got one on %s" % t.device)
+    if not t.is_contiguous():
+        raise ValueError("libcsa2 takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _addr(t):
+    p = _p(t)
+    return None if p is None else p.value
 
 
 def _stream(stream):
@@ -108,6 +121,8 @@ class Cache:
 
     def __init__(self, batch, n_slots, dim, idx_dim, row_stride, idx_key_dtype, seq_lens, page_table=None,
                  page_size=64, seq_stride_slots=0, device="cuda"):
+        if torch.device(device).type != "cuda":
+            raise ValueError("the cache lives in device memory; got device %s" % device)
         self.rows = torch.zeros((n_slots, row_stride), dtype=torch.uint8, device=device)
         kd = torch.uint8 if idx_key_dtype == E4M3 else torch.float32
         self.idx_keys = torch.zeros((n_slots, idx_dim), dtype=kd, device=device)
@@ -220,12 +235,9 @@ def layer_step(cache, mode, q, topk_idx, out, ws, window, q_idx=None, head_w=Non
                pool_k=0, sm_scale=0.0, stream=None):
     B, T, H, _ = q.shape
     H_I = q_idx.shape[2] if q_idx is not None else 0
-    a = csa2_layer_args(mode, q.data_ptr(), None if q_idx is None else q_idx.data_ptr(),
-                        _qdt(q_idx) if q_idx is not None else BF16,
-                        None if head_w is None else head_w.data_ptr(), T, H, H_I,
-                        pool_k or (pool_idx.shape[-1] if pool_idx is not None else 0), topk_idx.shape[-1], window,
-                        sm_scale, None if pool_idx is None else pool_idx.data_ptr(), topk_idx.data_ptr(),
-                        out.data_ptr(), None if lse is None else lse.data_ptr())
+    a = csa2_layer_args(mode, _addr(q), _addr(q_idx), _qdt(q_idx) if q_idx is not None else BF16, _addr(head_w),
+                        T, H, H_I, pool_k or (pool_idx.shape[-1] if pool_idx is not None else 0), topk_idx.shape[-1],
+                        window, sm_scale, _addr(pool_idx), _addr(topk_idx), _addr(out), _addr(lse))
     _check(lib().csa2_layer_step(cache.ref, ctypes.byref(a), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "layer_step")
 

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import fp4_sparse_attention_csa2_b200 as csa2
 from fp4_sparse_attention_csa2_b200 import build as _build
@@ -86,3 +87,18 @@ def test_bad_pointers_rejected_on_host(lib):
     bad_mode = csa2.csa2_layer_args(mode=7)
     assert lib.csa2_layer_step(ctypes.byref(c), ctypes.byref(bad_mode), 0x80000, 1 << 40, None) == \
         csa2.ERR_INVALID_ARG
+
+
+def test_host_tensors_are_refused_before_any_launch(lib):
+    # no CPU fallback: a host tensor never reaches the library as a pointer
+    with pytest.raises(ValueError):
+        csa2.workspace_init(torch.empty(4096, dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        csa2.Cache(1, 64, 128, 64, 80, csa2.E4M3, [64], seq_stride_slots=64, device="cpu")
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(csa2, "_lib", None)
+    monkeypatch.setattr(csa2, "LIB_PATH", str(tmp_path / "libcsa2.so"))
+    with pytest.raises(RuntimeError):
+        csa2.lib()
