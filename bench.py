@@ -403,18 +403,122 @@ def cpu_baseline(w, seed, layers, budget_s):
             "seconds": round(el, 2)}
 
 
+def oracle_piece_timer(w, seed, layers, budget_s, steps, warmup):
+    """The reference arm: the oracle's decode step of one (sequence, token) cut
+    into pieces -- the Full layer's scoring in slices of positions, then each
+    selection, Reindex and layer attention whole (the calls the step makes) --
+    with the slices sized so that `steps` pieces take about budget_s seconds.  Warm-up steps run pieces untimed; timed step i runs piece
+    (warmup + i) mod P (consecutive pieces are grouped when there are more
+    pieces than steps, so each is timed at least once).  One decode step costs
+    the sum of the pieces' mean times.  Returns (layer-steps per second,
+    seconds of the timed steps, sample description)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from harness import attended_positions, build_ref_cache, fill_ref_rows, host_layer
+    lens = wl.seq_lens(w, seed)
+    ref = build_ref_cache(w, seed=seed, rows=False, layers=layers, batches=[0])
+    hl = [host_layer(L) for L in layers]
+    j = w.T - 1
+    p = int(lens[0]) - w.T + j
+    # the indices every layer attends with, and the rows they need (untimed set-up)
+    topk_of, pools = {}, {}
+    pool = topk = None
+    scores = {}
+    for l, m in enumerate(w.pattern):
+        if m == "F":
+            pool, topk, scores[l] = oracle.index_full(ref, 0, w.T, j, hl[l]["q_idx"][0, j], w.q_idx_dtype,
+                                                      hl[l]["w"][0, j], w.pool_k, w.top_k, want_scores=True)
+            pools[l] = pool
+        elif m == "R":
+            pools[l] = pool
+            topk, _ = oracle.index_reindex(ref, 0, w.T, j, hl[l]["q_idx"][0, j], w.q_idx_dtype, hl[l]["w"][0, j],
+                                           pool, w.top_k)
+        topk_of[l] = topk
+    need = set()
+    for tk in topk_of.values():
+        need |= attended_positions(tk, p, w.window)
+    fill_ref_rows(ref, w, 0, need, wl.latent(w, 0, int(lens[0]), seed))
+    positions = np.arange(p + 1, dtype=np.int32)
+
+    def run(piece):
+        kind, l, a, b = piece
+        if kind == "score":
+            oracle.index_scores(ref, 0, positions[a:b], hl[l]["q_idx"][0, j], w.q_idx_dtype, hl[l]["w"][0, j])
+        elif kind == "select":
+            oracle.select_top(scores[l], None, w.pool_k)
+            oracle.select_top(scores[l], None, w.top_k)
+        elif kind == "reindex":
+            oracle.index_reindex(ref, 0, w.T, j, hl[l]["q_idx"][0, j], w.q_idx_dtype, hl[l]["w"][0, j], pools[l],
+                                 w.top_k)
+        else:
+            oracle.sparse_swa_attn(ref, 0, w.T, j, hl[l]["q"][0, j][a:b], topk_of[l], w.window)
+
+    def timed(piece):
+        t0 = time.perf_counter()
+        run(piece)
+        return time.perf_counter() - t0
+
+    # piece sizes from untimed probes: every piece is a whole oracle call as
+    # the decode step makes it (a layer's attention, a selection, a Reindex),
+    # except the Full scoring, cut into as many position slices as it takes
+    # for `steps` pieces to fit in budget_s
+    probe = min(8192, p + 1)
+    t_pos = timed(("score", 0, 0, probe)) / probe
+    t_rest = sum(timed(("attn", l, 0, w.H)) for l in range(len(w.pattern)))
+    t_rest += sum(timed(("select", l, 0, 0)) for l, m in enumerate(w.pattern) if m == "F")
+    t_rest += sum(timed(("reindex", l, 0, 0)) for l, m in enumerate(w.pattern) if m == "R")
+    n_f = w.pattern.count("F")
+    t_step = n_f * t_pos * (p + 1) + t_rest
+    n_other = len(w.pattern) + n_f + w.pattern.count("R")
+    want = int(np.ceil(max(steps, 1) * t_step / max(budget_s, 1e-9)))
+    n_slices = max(1, -(-max(want - n_other, n_f) // max(n_f, 1)))
+    slice_n = int(max(min(-(-(p + 1) // n_slices), p + 1), min(1024, p + 1)))
+    pieces = []
+    for l, m in enumerate(w.pattern):
+        if m == "F":
+            pieces += [("score", l, a, min(a + slice_n, p + 1)) for a in range(0, p + 1, slice_n)]
+            pieces.append(("select", l, 0, 0))
+        elif m == "R":
+            pieces.append(("reindex", l, 0, 0))
+        pieces.append(("attn", l, 0, w.H))
+    n_groups = min(len(pieces), max(steps, 1))
+    groups = [pieces[g * len(pieces) // n_groups:(g + 1) * len(pieces) // n_groups] for g in range(n_groups)]
+    for i in range(warmup):
+        for pc in groups[i % n_groups]:
+            run(pc)
+    acc = [0.0] * n_groups
+    cnt = [0] * n_groups
+    t_all = time.perf_counter()
+    for i in range(steps):
+        g = (warmup + i) % n_groups
+        t0 = time.perf_counter()
+        for pc in groups[g]:
+            run(pc)
+        acc[g] += time.perf_counter() - t0
+        cnt[g] += 1
+    el = time.perf_counter() - t_all
+    per_seq_token = sum(a / c for a, c in zip(acc, cnt) if c)
+    # one (sequence, token) of the batch; the metric's step covers batch*T of them
+    per_step = per_seq_token * (w.batch * w.T)
+    sample = ("sequence 0, query token %d of the %s stack (%s), single-threaded C oracle, fp64: one decode step cut "
+              "into %d pieces (Full scoring in slices of %d positions; each selection, Reindex and layer attention "
+              "whole), %d timed step(s) of one group of consecutive pieces each, round robin over %d groups; a "
+              "decode step costs the sum of the groups' mean times (%.2f s)"
+              % (j, w.name, w.pattern, len(pieces), slice_n, steps, n_groups, per_seq_token))
+    return len(w.pattern) / per_step, el, sample
+
+
 def run_reference(args, world, rank):
-    """The oracle as the reference arm: full decode steps of the workload on
-    the host cores until the step count or a fixed time budget is reached."""
+    """The oracle as the reference arm (rank 0 only): exactly `warmup` untimed
+    and `steps` timed steps, each a bounded piece of the workload's decode
+    step (see oracle_piece_timer), the value scaled to whole decode steps."""
     if rank != 0:
         return
     w = wl.WORKLOADS[args.workload]
     layers = [wl.layer_queries(w, l, args.seed) for l in range(len(w.pattern))]
-    budget = min(args.ref_budget, 1e9)
-    v, steps, el, sample = oracle_step_timer(w, args.seed, layers, budget_s=budget, max_steps=args.steps,
-                                             warmup=min(args.warmup, 1))
+    v, el, sample = oracle_piece_timer(w, args.seed, layers, args.ref_budget, args.steps, args.warmup)
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "layer-steps/s", "n_gpus": world,
-            "steps": steps, "warmup": min(args.warmup, 1), "ms_per_step": round(el / steps * 1e3, 2),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / max(args.steps, 1) * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded, same generator as the CUDA arm)",
             "config": {"workload": w.name, "context": int(wl.seq_lens(w, args.seed).max()), "layers": w.pattern},
@@ -433,7 +537,7 @@ def main():
     ap.add_argument("--replicas", type=int, default=3)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds of oracle work in the reference arm")
+    ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds of timed oracle work in the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     world, rank, _ = dist_setup(args.gpus)
