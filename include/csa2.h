@@ -30,8 +30,9 @@
  *    sequence longer than the cache, a bounded wait that ran out) never trap:
  *    the kernel skips the bad element and ORs a bit into a sticky status word
  *    in the workspace, read back with csa2_read_device_status.
- *  - The library keeps no mutable global state: calls on different streams
- *    with different workspaces may run concurrently.
+ *  - The library keeps no mutable global state, except the fixed scratch of
+ *    csa2_index_reindex_noalloc (see there): calls on different streams with
+ *    different workspaces may run concurrently.
  *  - Tensors are dense and row-major in the shapes given.  Pointers must be
  *    16-byte aligned, except seq_lens, page_table and start_pos (4-byte):
  *    a cache view of one sequence (page_table + b * max_pages, seq_lens + b)
