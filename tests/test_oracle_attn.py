@@ -133,3 +133,22 @@ def test_paged_equals_contiguous():
         for key in rp[l]:
             assert np.array_equal(rp[l][key][1], rc[l][key][1])
             assert np.array_equal(rp[l][key][2], rc[l][key][2])
+
+
+def test_future_topk_entries_are_not_attended_without_window():
+    # window 0, token 0 of 2: an index of the later token's position (legal,
+    # < L) must be ignored, not clipped onto p; only the past entries count
+    T = 2
+    w, cache, q = _setup(500, T=T)
+    p = 500 - T
+    past = np.array([3, 17, 250, p], dtype=np.int32)
+    topk = np.concatenate([past, np.array([p + 1], dtype=np.int32)])
+    out, lse = oracle.sparse_swa_attn(cache, 0, T, 0, wl.bf16_bits(q[0, 0]), topk, 0, 0.05)
+    V = _decode_rows_lib(cache, 0, sorted(past.tolist()), w.D)
+    nout, nlse = _numpy_attn(q[0, 0], V, 0.05)
+    assert np.allclose(out, nout, atol=1e-12) and np.allclose(lse, nlse, atol=1e-12)
+    # without p itself the set is the three earlier positions only
+    out2, _ = oracle.sparse_swa_attn(cache, 0, T, 0, wl.bf16_bits(q[0, 0]),
+                                     np.array([3, 17, 250, p + 1], dtype=np.int32), 0, 0.05)
+    V2 = _decode_rows_lib(cache, 0, [3, 17, 250], w.D)
+    assert np.allclose(out2, _numpy_attn(q[0, 0], V2, 0.05)[0], atol=1e-12)

@@ -153,3 +153,17 @@ def test_reuse_passes_indices_through_unchanged():
     res = oracle.run_stack(cache, "FRU", layers, 1, w.pool_k, w.top_k, w.window, w.q_idx_dtype)
     assert np.array_equal(res[1][(0, 0)][1], res[2][(0, 0)][1])
     assert res[1][(0, 0)][1].tobytes() == res[2][(0, 0)][1].tobytes()
+
+
+def test_cache_stores_index_keys_as_e4m3_of_the_input():
+    # the oracle cache's index keys equal torch's round-to-nearest-even
+    # float8_e4m3fn conversion of the bf16 key inputs (an encoder other than
+    # the oracle's own; the inputs stay far inside the E4M3 range)
+    w = wl.scaled(wl.WORKLOADS["long64k"], 3000)
+    layers = [wl.layer_queries(w, 0)]
+    cache = build_ref_cache(w, rows=False, layers=layers)
+    keys, _ = wl.index_keys(w, 0, 3000, layers[0]["q_idx"][0, w.T - 1])
+    assert keys.dtype == torch.bfloat16 and float(keys.float().abs().max()) < 448
+    want = keys.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    slots = [cache.slot(0, t) for t in range(3000)]
+    assert np.array_equal(cache.idx_keys[slots], want)
