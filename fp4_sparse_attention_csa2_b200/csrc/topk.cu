@@ -13,15 +13,17 @@
 // win.  Output order is unspecified; -1 pads the tail.
 //
 //   large segments (Full layer, up to 1M scores): the level-1 histogram comes
-//     from the scoring kernel; a streaming pass (many CTAs per segment) selects
-//     above each target's level-1 threshold and compacts the elements equal to
-//     it into candidate lists (histogramming their digit 2); a second pass
-//     over the lists (many CTAs) selects above the digit-2 thresholds and keeps
-//     the survivors, and its last CTA resolves digit 3 and exact ties.
-//     The pool and the layer's top-k are two targets of the same passes.
-//   small segments (<= 16,384: the top-k of a pool): a cluster of 8 CTAs per
-//     segment keeps every key in registers and resolves all three digits,
-//     summing the CTAs' histograms through distributed shared memory.
+//     from the scoring kernel; a streaming pass (many CTAs per segment) works
+//     out each target's level-1 threshold, selects above it and compacts the
+//     elements equal to it into candidate lists (histogramming their digit 2);
+//     the pass's last CTA publishes the digit-2 plan.  A second pass over the
+//     lists (many CTAs) selects above the digit-2 thresholds and keeps the
+//     survivors, and its last CTA resolves digit 3 and exact ties.  The pool
+//     and the layer's top-k are two targets of the same passes.
+//   small segments (<= 16,384: the top-k of a pool, and the pool of a Full
+//     layer over a short context): a cluster of 8 CTAs per segment keeps every
+//     key in registers and resolves all three digits, summing the CTAs'
+//     histograms through distributed shared memory.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
