@@ -9,8 +9,9 @@
 //
 // Full scoring (fp32 keys): one thread scores one position for every query
 // token of its sequence.  Pool scoring (Reindex): four threads share one pool
-// entry, a quarter of the heads each.  The queries sit in shared memory as
-// fp32 and are read as broadcasts; the key (64 values) sits in registers.
+// entry, a quarter of the heads each (one thread per entry when many
+// segments already fill the GPU).  The queries sit in shared memory as fp32
+// and are read as broadcasts; the key (64 values) sits in registers.
 #include "common.cuh"
 #include "kernels.h"
 
