@@ -55,6 +55,8 @@ def lib():
         L.ref_sparse_swa_attn.argtypes = [c_p, i32, i32, i32, i32, c_p, c_p, i32, i32, ctypes.c_double,
                                           c_p, c_p]
         L.ref_dense_attn.argtypes = [c_p, i32, i32, i32, i32, c_p, ctypes.c_double, c_p, c_p]
+        L.ref_sparse_swa_attn_local.argtypes = [c_p, c_p, i64, i32, i32, i32, i32, c_p, c_p, i32, i32,
+                                                ctypes.c_double, c_p, c_p]
         _lib = L
     return _lib
 
@@ -240,6 +242,22 @@ def sparse_swa_attn(cache, b, T, j, q_bf16_u16, topk_idx, window, sm_scale=0.0):
     lse = np.zeros(H, dtype=np.float64)
     _check(lib().ref_sparse_swa_attn(cache.ref, b, T, j, H, _ptr(q), _ptr(tk), tk.size, window, sm_scale,
                                      _ptr(out), _ptr(lse)), "sparse_swa_attn")
+    return out, lse
+
+
+def sparse_swa_attn_local(cache, ring_bf16_u16, b, T, j, q_bf16_u16, topk_idx, window, sm_scale=0.0):
+    """Sparse attention whose window rows come from a layer-local bf16 ring:
+    ring uint16 [batch, ring_len, D] (position t at slot t % ring_len);
+    q uint16 [H, D] -> (out fp64 [H, D], lse fp64 [H])."""
+    ring = np.ascontiguousarray(ring_bf16_u16, dtype=np.uint16)
+    q = np.ascontiguousarray(q_bf16_u16, dtype=np.uint16)
+    H, D = q.shape
+    tk = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    out = np.zeros((H, D), dtype=np.float64)
+    lse = np.zeros(H, dtype=np.float64)
+    _check(lib().ref_sparse_swa_attn_local(cache.ref, _ptr(ring), ring.shape[1], b, T, j, H, _ptr(q), _ptr(tk),
+                                           tk.size, window, sm_scale, _ptr(out), _ptr(lse)),
+           "sparse_swa_attn_local")
     return out, lse
 
 

@@ -442,9 +442,11 @@ int ref_index_reindex(const ref_cache* c, int b, int T, int j, int q_dtype, cons
 /*     lse_h = log sum_{t in S} exp(z_t)                                     */
 /* q is bf16 [H][D]; out is [H][D]; lse is [H] (nullable).                   */
 /* ------------------------------------------------------------------------ */
-int ref_sparse_swa_attn(const ref_cache* c, int b, int T, int j, int H, const uint16_t* q,
-                        const int32_t* topk_idx, int top_k, int window, double sm_scale,
-                        double* out, double* lse)
+/* The window rows come from `ring` when it is given (layer-local window      */
+/* state, see ref_sparse_swa_attn_local), else from the FP4 cache.           */
+static int sparse_swa_attn_rows(const ref_cache* c, const uint16_t* ring, int64_t ring_len, int b, int T, int j,
+                                int H, const uint16_t* q, const int32_t* topk_idx, int top_k, int window,
+                                double sm_scale, double* out, double* lse)
 {
     int D = c->dim;
     int64_t p = query_pos(c, b, T, j);
@@ -473,10 +475,16 @@ int ref_sparse_swa_attn(const ref_cache* c, int b, int T, int j, int H, const ui
     int rc = REF_OK;
     for (int64_t t = 0; t <= p; ++t) {
         if (!in_s[t]) continue;
-        int64_t slot = ref_slot(c, b, t);
-        if (slot < 0) { rc = REF_ERR_BOUNDS; break; }
         S[k] = t;
-        ref_dequant_row(c->rows + slot * c->row_stride, D, v + k * D);
+        if (ring && window > 0 && t >= lo) {
+            /* a window position: its layer-local bf16 row, ring slot t mod ring_len */
+            const uint16_t* r = ring + ((int64_t)b * ring_len + t % ring_len) * D;
+            for (int d = 0; d < D; ++d) v[k * D + d] = (double)bf16_to_f32(r[d]);
+        } else {
+            int64_t slot = ref_slot(c, b, t);
+            if (slot < 0) { rc = REF_ERR_BOUNDS; break; }
+            ref_dequant_row(c->rows + slot * c->row_stride, D, v + k * D);
+        }
         ++k;
     }
     for (int h = 0; h < H && !rc; ++h) {
@@ -504,6 +512,32 @@ int ref_sparse_swa_attn(const ref_cache* c, int b, int T, int j, int H, const ui
     }
     free(in_s); free(S); free(v); free(qd); free(z);
     return rc;
+}
+
+int ref_sparse_swa_attn(const ref_cache* c, int b, int T, int j, int H, const uint16_t* q,
+                        const int32_t* topk_idx, int top_k, int window, double sm_scale,
+                        double* out, double* lse)
+{
+    return sparse_swa_attn_rows(c, NULL, 0, b, T, j, H, q, topk_idx, top_k, window, sm_scale, out, lse);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Sparse attention with layer-local window state ([FANOUT] item 2: the      */
+/* modes share global KV and sparse selections while queries and the        */
+/* sliding-window state stay layer-local; [TLDR] paragraph 2: the window     */
+/* runs in every layer and its states are rebuilt from the last 128          */
+/* tokens).  The attended set S is the one of ref_sparse_swa_attn; a         */
+/* position of the window takes its row from this layer's bf16 ring          */
+/* [batch][ring_len][D] (position t at slot t mod ring_len, ring_len >=      */
+/* window), every other position its dequantised FP4 row from the shared     */
+/* cache.                                                                    */
+/* ------------------------------------------------------------------------ */
+int ref_sparse_swa_attn_local(const ref_cache* c, const uint16_t* ring, int64_t ring_len, int b, int T, int j,
+                              int H, const uint16_t* q, const int32_t* topk_idx, int top_k, int window,
+                              double sm_scale, double* out, double* lse)
+{
+    if (!ring || ring_len < window || ring_len < 1) return REF_ERR_ARG;
+    return sparse_swa_attn_rows(c, ring, ring_len, b, T, j, H, q, topk_idx, top_k, window, sm_scale, out, lse);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -152,3 +152,68 @@ def test_future_topk_entries_are_not_attended_without_window():
                                      np.array([3, 17, 250, p + 1], dtype=np.int32), 0, 0.05)
     V2 = _decode_rows_lib(cache, 0, [3, 17, 250], w.D)
     assert np.allclose(out2, _numpy_attn(q[0, 0], V2, 0.05)[0], atol=1e-12)
+
+
+# ------------------------------------------------------------------ layer-local window state
+# ([FANOUT] item 2: queries and the sliding-window state stay layer-local;
+# [TLDR] paragraph 2: the window runs in every layer)
+
+def _ring(w, L, ring_len, seed):
+    g = torch.Generator().manual_seed(seed)
+    ring = torch.randn((w.batch, ring_len, w.D), generator=g).to(torch.bfloat16)
+    return ring, wl.bf16_bits(ring)
+
+
+def test_local_window_holding_the_cache_rows_equals_shared_rows():
+    # a ring that holds the window positions' dequantised FP4 rows (exact in
+    # bf16) gives exactly the shared-cache result
+    w, cache, q = _setup(900)
+    p, ring_len = 899, 160
+    rows = _decode_rows_lib(cache, 0, range(900), w.D)
+    ring = torch.zeros((1, ring_len, w.D), dtype=torch.float64)
+    for t in range(p - w.window + 1, p + 1):
+        ring[0, t % ring_len] = torch.from_numpy(rows[t])
+    assert torch.equal(ring.to(torch.bfloat16).double(), ring)          # exact in bf16
+    rng = np.random.default_rng(4)
+    topk = rng.choice(900, w.top_k, replace=False).astype(np.int32)
+    a, al = oracle.sparse_swa_attn(cache, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window)
+    b, bl = oracle.sparse_swa_attn_local(cache, wl.bf16_bits(ring.to(torch.bfloat16)), 0, 1, 0,
+                                         wl.bf16_bits(q[0, 0]), topk, w.window)
+    assert np.array_equal(a, b) and np.array_equal(al, bl)
+
+
+def test_local_window_only_is_dense_over_the_ring_rows():
+    w, cache, q = _setup(700)
+    p, ring_len = 699, 200                                               # 700 % 200 != 0: the ring wraps
+    ring, bits = _ring(w, 700, ring_len, 5)
+    topk = np.full(w.top_k, -1, dtype=np.int32)
+    out, lse = oracle.sparse_swa_attn_local(cache, bits, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window, 0.03)
+    V = np.stack([ring[0, t % ring_len].double().numpy() for t in range(p - w.window + 1, p + 1)])
+    nout, nlse = _numpy_attn(q[0, 0], V, 0.03)
+    assert np.allclose(out, nout, atol=1e-12) and np.allclose(lse, nlse, atol=1e-12)
+
+
+def test_local_window_mixed_with_shared_topk_rows():
+    # window rows from the ring, the other attended rows from the FP4 cache; a
+    # top-k entry inside the window uses the ring row once
+    w, cache, q = _setup(900)
+    p, ring_len = 899, 128
+    ring, bits = _ring(w, 900, ring_len, 6)
+    rng = np.random.default_rng(7)
+    topk = rng.choice(700, w.top_k, replace=False).astype(np.int32)
+    topk[:5] = [899, 880, 850, -1, 772]                                  # three of them in the window
+    out, lse = oracle.sparse_swa_attn_local(cache, bits, 0, 1, 0, wl.bf16_bits(q[0, 0]), topk, w.window, 0.04)
+    win = list(range(p - w.window + 1, p + 1))
+    far = sorted(set(int(t) for t in topk if 0 <= t < p - w.window + 1))
+    V = np.concatenate([_decode_rows_lib(cache, 0, far, w.D),
+                        np.stack([ring[0, t % ring_len].double().numpy() for t in win])])
+    nout, nlse = _numpy_attn(q[0, 0], V, 0.04)
+    assert np.allclose(out, nout, atol=1e-12) and np.allclose(lse, nlse, atol=1e-12)
+
+
+def test_local_ring_shorter_than_the_window_is_an_error():
+    w, cache, q = _setup(300)
+    _, bits = _ring(w, 300, w.window - 1, 8)
+    with pytest.raises(RuntimeError):
+        oracle.sparse_swa_attn_local(cache, bits, 0, 1, 0, wl.bf16_bits(q[0, 0]),
+                                     np.full(w.top_k, -1, dtype=np.int32), w.window)

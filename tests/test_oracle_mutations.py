@@ -9,7 +9,8 @@ definitions and round-to-nearest-even encoders, the block quantisation (scale
 the scoring s_t = sum_h w_h max(0, q_h . k_t), the top-n selection, the Full
 and Reindex selections, the paged slot map, the causal query position, and the
 sparse + window attention (window bounds, future entries, scale, softmax
-normaliser, log-sum-exp)."""
+normaliser, log-sum-exp) and its layer-local window rows (ring slot, which
+positions take a ring row)."""
 import os
 import shutil
 import subprocess
@@ -56,6 +57,9 @@ MUTATIONS = [
      "        for (int d = 0; d < D; ++d) qd[d] = (double)bf16_to_f32(q[(int64_t)h * D + (d ^ 1)]);"),
     ("lse_without_max", "        if (lse) lse[h] = m + log(l);\n    }\n    free(in_s);",
      "        if (lse) lse[h] = log(l);\n    }\n    free(in_s);"),
+    ("ring_slot_shifted", "ring + ((int64_t)b * ring_len + t % ring_len) * D;",
+     "ring + ((int64_t)b * ring_len + (t + 1) % ring_len) * D;"),
+    ("ring_rows_for_every_position", "        if (ring && window > 0 && t >= lo) {", "        if (ring && window > 0) {"),
 ]
 
 
