@@ -55,6 +55,7 @@ def lib():
         L.ref_sparse_swa_attn.argtypes = [c_p, i32, i32, i32, i32, c_p, c_p, i32, i32, ctypes.c_double,
                                           c_p, c_p]
         L.ref_dense_attn.argtypes = [c_p, i32, i32, i32, i32, c_p, ctypes.c_double, c_p, c_p]
+        L.ref_index_pool_update.argtypes = [c_p, i32, i32, i32, i32, c_p, c_p, i32, c_p, i32, i64, i32, c_p, c_p]
         L.ref_sparse_swa_attn_local.argtypes = [c_p, c_p, i64, i32, i32, i32, i32, c_p, c_p, i32, i32,
                                                 ctypes.c_double, c_p, c_p]
         _lib = L
@@ -231,6 +232,19 @@ def index_reindex(cache, b, T, j, q, q_dtype, w, pool_idx, top_k, want_scores=Fa
     _check(lib().ref_index_reindex(cache.ref, b, T, j, q_dtype, _ptr(q), _ptr(w), q.shape[0], _ptr(pool),
                                    pool.size, top_k, _ptr(topk), _ptr(scores)), "index_reindex")
     return topk, scores
+
+
+def index_pool_update(cache, b, T, j, q, q_dtype, w, pool_prev, t_new0, top_k):
+    """The pool of an in-flight request after positions t_new0.. were appended:
+    the best of the previous pool and the new positions -> (pool_idx, topk_idx)."""
+    q = _qarr(q, q_dtype)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    prev = np.ascontiguousarray(pool_prev, dtype=np.int32)
+    pool = np.zeros(prev.size, dtype=np.int32)
+    topk = np.zeros(top_k, dtype=np.int32)
+    _check(lib().ref_index_pool_update(cache.ref, b, T, j, q_dtype, _ptr(q), _ptr(w), q.shape[0], _ptr(prev),
+                                       prev.size, t_new0, top_k, _ptr(pool), _ptr(topk)), "index_pool_update")
+    return pool, topk
 
 
 def sparse_swa_attn(cache, b, T, j, q_bf16_u16, topk_idx, window, sm_scale=0.0):

@@ -432,6 +432,40 @@ int ref_index_reindex(const ref_cache* c, int b, int T, int j, int q_dtype, cons
     return rc;
 }
 
+/* Append-time pool maintenance for an in-flight request (the candidate     */
+/* pool of [TLDR] paragraph 3 kept current as tokens are appended): the new  */
+/* pool is the min(pool_k, |candidates|) best of the previous pool's valid   */
+/* entries and the new positions t_new0 .. p, all scored with this query;   */
+/* topk_idx receives the top_k best of the same candidates.  Previous pool   */
+/* entries at or beyond t_new0 (or beyond p) are an argument error.          */
+int ref_index_pool_update(const ref_cache* c, int b, int T, int j, int q_dtype, const void* q, const float* w,
+                          int H_I, const int32_t* pool_prev, int pool_k, int64_t t_new0, int top_k,
+                          int32_t* pool_idx, int32_t* topk_idx)
+{
+    if (top_k > pool_k || pool_k > 16384 || top_k < 0 || t_new0 < 0) return REF_ERR_ARG;
+    int64_t p = query_pos(c, b, T, j);
+    if (p < 0) return REF_ERR_ARG;
+    int64_t n_new = p + 1 > t_new0 ? p + 1 - t_new0 : 0;
+    int64_t cap = pool_k + n_new;
+    int32_t* pos = (int32_t*)malloc(sizeof(int32_t) * (size_t)(cap > 0 ? cap : 1));
+    double* s = (double*)malloc(sizeof(double) * (size_t)(cap > 0 ? cap : 1));
+    if (!pos || !s) { free(pos); free(s); return REF_ERR_ARG; }
+    int64_t n = 0;
+    int rc = REF_OK;
+    for (int i = 0; i < pool_k; ++i) {
+        if (pool_prev[i] < 0) continue;
+        if (pool_prev[i] >= t_new0 || pool_prev[i] > p) { rc = REF_ERR_ARG; break; }
+        pos[n++] = pool_prev[i];
+    }
+    for (int64_t t = t_new0; t <= p && !rc; ++t) pos[n++] = (int32_t)t;
+    if (!rc) rc = ref_index_scores(c, b, n, pos, q_dtype, q, H_I, w, s);
+    if (!rc) rc = ref_select_top(s, pos, n, pool_k, pool_idx);
+    if (!rc) rc = ref_select_top(s, pos, n, top_k, topk_idx);
+    free(pos);
+    free(s);
+    return rc;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Sparse + sliding-window attention ([HN] key point 2, [TLDR] paragraphs 2  */
 /* and 3).  S = window ∪ top-k without double counting, window =             */

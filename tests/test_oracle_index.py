@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from fp4_sparse_attention_csa2_b200 import workloads as wl
-from harness import build_ref_cache, host_layer
+from harness import band_set_check, build_ref_cache, host_layer
 
 
 def _small(name, L, **kw):
@@ -167,3 +167,65 @@ def test_cache_stores_index_keys_as_e4m3_of_the_input():
     want = keys.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     slots = [cache.slot(0, t) for t in range(3000)]
     assert np.array_equal(cache.idx_keys[slots], want)
+
+
+# ------------------------------------------------------------------ append-time pool maintenance
+# (the Full layer's candidate pool of tldrocket.com "DeepSeek AI Released
+# DeepSeek-V4.1-Flash ...", paragraph 3, kept current for an in-flight request)
+
+def _pool_case(L0, L, pool_k=1024, top_k=128):
+    w = wl.scaled(wl.WORKLOADS["long64k"], L, pool_k=pool_k, top_k=top_k)
+    layer = wl.layer_queries(w, 0)
+    cache = build_ref_cache(w, rows=False, layers=[layer])
+    h = host_layer(layer)
+    return w, cache, h["q_idx"][0, 0], h["w"][0, 0]
+
+
+def test_pool_update_equals_full_selection_over_the_longer_context():
+    # top-K(S ∪ N) = top-K(top-K(S) ∪ N): updating the pool of the first L0
+    # positions with the appended ones equals selecting over all L
+    L0, L = 5000, 6000
+    w, cache, q, hw = _pool_case(L0, L)
+    cache.set_seq_lens([L0])
+    prev, _, _ = oracle.index_full(cache, 0, 1, 0, q, w.q_idx_dtype, hw, w.pool_k, w.top_k)
+    cache.set_seq_lens([L])
+    pool, topk = oracle.index_pool_update(cache, 0, 1, 0, q, w.q_idx_dtype, hw, prev, L0, w.top_k)
+    fp, ft, s = oracle.index_full(cache, 0, 1, 0, q, w.q_idx_dtype, hw, w.pool_k, w.top_k, want_scores=True)
+    band_set_check(pool, fp, lambda t: s[t], s.size)
+    band_set_check(topk, ft, lambda t: s[t], s.size)
+    assert set(topk[topk >= 0]) <= set(pool[pool >= 0])
+
+
+def test_pool_update_without_new_positions_keeps_the_pool():
+    w, cache, q, hw = _pool_case(3000, 3000)
+    prev, _, _ = oracle.index_full(cache, 0, 1, 0, q, w.q_idx_dtype, hw, w.pool_k, w.top_k)
+    pool, _ = oracle.index_pool_update(cache, 0, 1, 0, q, w.q_idx_dtype, hw, prev, 3000, w.top_k)
+    assert set(pool.tolist()) == set(prev.tolist())
+
+
+def test_pool_update_from_an_empty_pool_is_the_full_selection():
+    w, cache, q, hw = _pool_case(0, 2500)
+    empty = np.full(w.pool_k, -1, dtype=np.int32)
+    pool, topk = oracle.index_pool_update(cache, 0, 1, 0, q, w.q_idx_dtype, hw, empty, 0, w.top_k)
+    fp, ft, s = oracle.index_full(cache, 0, 1, 0, q, w.q_idx_dtype, hw, w.pool_k, w.top_k, want_scores=True)
+    band_set_check(pool, fp, lambda t: s[t], s.size)
+    band_set_check(topk, ft, lambda t: s[t], s.size)
+
+
+def test_pool_update_rejects_previous_entries_among_the_new_positions():
+    w, cache, q, hw = _pool_case(0, 2000)
+    prev = np.full(w.pool_k, -1, dtype=np.int32)
+    prev[0] = 1500
+    with pytest.raises(RuntimeError):
+        oracle.index_pool_update(cache, 0, 1, 0, q, w.q_idx_dtype, hw, prev, 1200, w.top_k)
+
+
+def test_pool_update_below_the_pool_size_keeps_every_position():
+    # fewer candidates than pool_k: the pool is every position 0..p, the
+    # newest one included
+    w, cache, q, hw = _pool_case(0, 900)
+    prev = np.full(w.pool_k, -1, dtype=np.int32)
+    prev[:600] = np.arange(600)
+    pool, topk = oracle.index_pool_update(cache, 0, 1, 0, q, w.q_idx_dtype, hw, prev, 600, w.top_k)
+    assert set(pool[pool >= 0].tolist()) == set(range(900)) and np.all(pool[900:] == -1)
+    assert np.sum(topk >= 0) == w.top_k

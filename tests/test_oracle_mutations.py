@@ -10,7 +10,7 @@ the scoring s_t = sum_h w_h max(0, q_h . k_t), the top-n selection, the Full
 and Reindex selections, the paged slot map, the causal query position, and the
 sparse + window attention (window bounds, future entries, scale, softmax
 normaliser, log-sum-exp) and its layer-local window rows (ring slot, which
-positions take a ring row)."""
+positions take a ring row), and the append-time pool update."""
 import os
 import shutil
 import subprocess
@@ -41,8 +41,8 @@ MUTATIONS = [
      "    if (x->s < y->s) return -1;\n    if (x->s > y->s) return 1;"),
     ("full_skips_p", "    if (!rc) rc = ref_select_top(s, NULL, n, pool_k, pool_idx);\n    if (!rc) rc = ref_select_top(s, NULL, n, top_k, topk_idx);",
      "    if (!rc) rc = ref_select_top(s, NULL, n - 1, pool_k, pool_idx);\n    if (!rc) rc = ref_select_top(s, NULL, n - 1, top_k, topk_idx);"),
-    ("reindex_returns_ranks", "    if (!rc) rc = ref_select_top(s, pos, n, top_k, topk_idx);",
-     "    if (!rc) rc = ref_select_top(s, NULL, n, top_k, topk_idx);"),
+    ("reindex_returns_ranks", "w, s);\n    if (!rc) rc = ref_select_top(s, pos, n, top_k, topk_idx);",
+     "w, s);\n    if (!rc) rc = ref_select_top(s, NULL, n, top_k, topk_idx);"),
     ("paged_slot_drops_offset", "        slot = (int64_t)phys * c->page_size + t % c->page_size;",
      "        slot = (int64_t)phys * c->page_size;"),
     ("query_position_one_early", "return (int64_t)c->seq_lens[b] - T + j;", "return (int64_t)c->seq_lens[b] - T + j - 1;"),
@@ -60,6 +60,10 @@ MUTATIONS = [
     ("ring_slot_shifted", "ring + ((int64_t)b * ring_len + t % ring_len) * D;",
      "ring + ((int64_t)b * ring_len + (t + 1) % ring_len) * D;"),
     ("ring_rows_for_every_position", "        if (ring && window > 0 && t >= lo) {", "        if (ring && window > 0) {"),
+    ("pool_update_forgets_pool", "        if (pool_prev[i] < 0) continue;\n        if (pool_prev[i] >= t_new0",
+     "        if (pool_prev[i] < 0 || i >= 0) continue;\n        if (pool_prev[i] >= t_new0"),
+    ("pool_update_misses_p", "    for (int64_t t = t_new0; t <= p && !rc; ++t) pos[n++] = (int32_t)t;",
+     "    for (int64_t t = t_new0; t < p && !rc; ++t) pos[n++] = (int32_t)t;"),
 ]
 
 
