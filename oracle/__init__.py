@@ -55,6 +55,7 @@ def lib():
         L.ref_sparse_swa_attn.argtypes = [c_p, i32, i32, i32, i32, c_p, c_p, i32, i32, ctypes.c_double,
                                           c_p, c_p]
         L.ref_dense_attn.argtypes = [c_p, i32, i32, i32, i32, c_p, ctypes.c_double, c_p, c_p]
+        L.ref_lse_merge.argtypes = [i32, i32, i32, c_p, c_p, c_p, c_p]
         L.ref_index_pool_update.argtypes = [c_p, i32, i32, i32, i32, c_p, c_p, i32, c_p, i32, i64, i32, c_p, c_p]
         L.ref_sparse_swa_attn_local.argtypes = [c_p, c_p, i64, i32, i32, i32, i32, c_p, c_p, i32, i32,
                                                 ctypes.c_double, c_p, c_p]
@@ -272,6 +273,18 @@ def sparse_swa_attn_local(cache, ring_bf16_u16, b, T, j, q_bf16_u16, topk_idx, w
     _check(lib().ref_sparse_swa_attn_local(cache.ref, _ptr(ring), ring.shape[1], b, T, j, H, _ptr(q), _ptr(tk),
                                            tk.size, window, sm_scale, _ptr(out), _ptr(lse)),
            "sparse_swa_attn_local")
+    return out, lse
+
+
+def lse_merge(outs, lses):
+    """Merge attention partials over disjoint parts of one attended set:
+    outs [n, H, D], lses [n, H] -> (out [H, D], lse [H])."""
+    outs = np.ascontiguousarray(outs, dtype=np.float64)
+    lses = np.ascontiguousarray(lses, dtype=np.float64)
+    n, H, D = outs.shape
+    out = np.zeros((H, D), dtype=np.float64)
+    lse = np.zeros(H, dtype=np.float64)
+    _check(lib().ref_lse_merge(n, H, D, _ptr(outs), _ptr(lses), _ptr(out), _ptr(lse)), "lse_merge")
     return out, lse
 
 

@@ -575,6 +575,39 @@ int ref_sparse_swa_attn_local(const ref_cache* c, const uint16_t* ring, int64_t 
 }
 
 /* ------------------------------------------------------------------------ */
+/* Merge of attention partials over disjoint parts of one attended set (a    */
+/* context sharded over devices, each attending over its own part): with     */
+/* part i's output O_i and log-sum-exp l_i per head,                         */
+/*     l = log sum_i exp(l_i),   O = sum_i exp(l_i - l) O_i.                 */
+/* A part with l_i = -inf (nothing attended) contributes nothing; if every   */
+/* part is empty the result is O = 0, l = -inf.                              */
+/* outs is [n_parts][H][D], lses is [n_parts][H].                            */
+/* ------------------------------------------------------------------------ */
+int ref_lse_merge(int n_parts, int H, int D, const double* outs, const double* lses, double* out, double* lse)
+{
+    if (n_parts < 1 || H < 1 || D < 1) return REF_ERR_ARG;
+    for (int h = 0; h < H; ++h) {
+        double m = -INFINITY;
+        for (int i = 0; i < n_parts; ++i)
+            if (lses[(int64_t)i * H + h] > m) m = lses[(int64_t)i * H + h];
+        for (int d = 0; d < D; ++d) out[(int64_t)h * D + d] = 0.0;
+        if (m == -INFINITY) {
+            lse[h] = -INFINITY;
+            continue;
+        }
+        double sum = 0.0;
+        for (int i = 0; i < n_parts; ++i) sum += exp(lses[(int64_t)i * H + h] - m);
+        double l = m + log(sum);
+        for (int i = 0; i < n_parts; ++i) {
+            double wgt = exp(lses[(int64_t)i * H + h] - l);
+            for (int d = 0; d < D; ++d) out[(int64_t)h * D + d] += wgt * outs[((int64_t)i * H + h) * D + d];
+        }
+        lse[h] = l;
+    }
+    return REF_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Brute-force dense attention over every visible position 0..p, written     */
 /* separately from the sparse routine (two passes over the cache, no set     */
 /* construction).  When top-k covers the whole visible context the sparse    */

@@ -217,3 +217,38 @@ def test_local_ring_shorter_than_the_window_is_an_error():
     with pytest.raises(RuntimeError):
         oracle.sparse_swa_attn_local(cache, bits, 0, 1, 0, wl.bf16_bits(q[0, 0]),
                                      np.full(w.top_k, -1, dtype=np.int32), w.window)
+
+
+# ------------------------------------------------------------------ partials over disjoint parts
+# (the attention of a context sharded over devices: each attends over its part
+# of S, the parts' (output, log-sum-exp) pairs are merged)
+
+def test_lse_merge_of_disjoint_parts_equals_attention_over_the_union():
+    w, cache, q = _setup(900)
+    rng = np.random.default_rng(9)
+    S = rng.choice(900, 300, replace=False).astype(np.int32)
+    qb = wl.bf16_bits(q[0, 0])
+    full, flse = oracle.sparse_swa_attn(cache, 0, 1, 0, qb, S, 0, 0.05)
+    for n_parts in (2, 3, 5):
+        parts = np.array_split(rng.permutation(S), n_parts)
+        res = [oracle.sparse_swa_attn(cache, 0, 1, 0, qb, part, 0, 0.05) for part in parts]
+        out, lse = oracle.lse_merge(np.stack([r[0] for r in res]), np.stack([r[1] for r in res]))
+        assert np.allclose(out, full, atol=1e-12) and np.allclose(lse, flse, atol=1e-12)
+    # the merge itself against its definition written with numpy
+    outs, lses = np.stack([r[0] for r in res]), np.stack([r[1] for r in res])
+    L = np.logaddexp.reduce(lses, axis=0)
+    assert np.allclose(lse, L, atol=1e-12)
+    assert np.allclose(out, np.einsum("ih,ihd->hd", np.exp(lses - L), outs), atol=1e-12)
+
+
+def test_lse_merge_with_empty_parts():
+    w, cache, q = _setup(600)
+    qb = wl.bf16_bits(q[0, 0])
+    S = np.arange(100, 160, dtype=np.int32)
+    full, flse = oracle.sparse_swa_attn(cache, 0, 1, 0, qb, S, 0)
+    empty = oracle.sparse_swa_attn(cache, 0, 1, 0, qb, np.full(4, -1, dtype=np.int32), 0)
+    assert np.all(np.isneginf(empty[1])) and np.all(empty[0] == 0)
+    out, lse = oracle.lse_merge(np.stack([empty[0], full, empty[0]]), np.stack([empty[1], flse, empty[1]]))
+    assert np.allclose(out, full, atol=1e-15) and np.allclose(lse, flse, atol=1e-15)
+    out, lse = oracle.lse_merge(np.stack([empty[0], empty[0]]), np.stack([empty[1], empty[1]]))
+    assert np.all(out == 0) and np.all(np.isneginf(lse))

@@ -229,3 +229,24 @@ def test_pool_update_below_the_pool_size_keeps_every_position():
     pool, topk = oracle.index_pool_update(cache, 0, 1, 0, q, w.q_idx_dtype, hw, prev, 600, w.top_k)
     assert set(pool[pool >= 0].tolist()) == set(range(900)) and np.all(pool[900:] == -1)
     assert np.sum(topk >= 0) == w.top_k
+
+
+def test_top_k_of_shard_top_ks_is_the_global_top_k():
+    # a context sharded over devices selects globally from the union of the
+    # shards' local selections: top-K(∪ S_g) = top-K(∪ top-K(S_g))
+    w = wl.scaled(wl.WORKLOADS["long64k"], 9000, pool_k=1024, top_k=128)
+    layer = wl.layer_queries(w, 0)
+    cache = build_ref_cache(w, rows=False, layers=[layer])
+    h = host_layer(layer)
+    fp, _, s = oracle.index_full(cache, 0, 1, 0, h["q_idx"][0, 0], w.q_idx_dtype, h["w"][0, 0], w.pool_k, w.top_k,
+                                 want_scores=True)
+    for G in (2, 4, 7):
+        bounds = np.linspace(0, 9000, G + 1).astype(np.int64)
+        cand = []
+        for g in range(G):
+            pos = np.arange(bounds[g], bounds[g + 1], dtype=np.int32)
+            loc = oracle.select_top(s[pos], pos, w.pool_k)
+            cand.append(loc[loc >= 0])
+        cand = np.concatenate(cand)
+        glob = oracle.select_top(s[cand], cand, w.pool_k)
+        band_set_check(glob, fp, lambda t: s[t], s.size)

@@ -10,7 +10,8 @@ the scoring s_t = sum_h w_h max(0, q_h . k_t), the top-n selection, the Full
 and Reindex selections, the paged slot map, the causal query position, and the
 sparse + window attention (window bounds, future entries, scale, softmax
 normaliser, log-sum-exp) and its layer-local window rows (ring slot, which
-positions take a ring row), and the append-time pool update."""
+positions take a ring row), the append-time pool update and the merge of
+attention partials over disjoint parts."""
 import os
 import shutil
 import subprocess
@@ -62,6 +63,8 @@ MUTATIONS = [
     ("ring_rows_for_every_position", "        if (ring && window > 0 && t >= lo) {", "        if (ring && window > 0) {"),
     ("pool_update_forgets_pool", "        if (pool_prev[i] < 0) continue;\n        if (pool_prev[i] >= t_new0",
      "        if (pool_prev[i] < 0 || i >= 0) continue;\n        if (pool_prev[i] >= t_new0"),
+    ("merge_weights_unnormalised", "            double wgt = exp(lses[(int64_t)i * H + h] - l);",
+     "            double wgt = exp(lses[(int64_t)i * H + h] - m);"),
     ("pool_update_misses_p", "    for (int64_t t = t_new0; t <= p && !rc; ++t) pos[n++] = (int32_t)t;",
      "    for (int64_t t = t_new0; t < p && !rc; ++t) pos[n++] = (int32_t)t;"),
 ]
