@@ -411,7 +411,8 @@ def oracle_piece_timer(w, seed, layers, budget_s, steps, warmup):
     (warmup + i) mod P (consecutive pieces are grouped when there are more
     pieces than steps, so each is timed at least once).  One decode step costs
     the sum of the pieces' mean times.  Returns (layer-steps per second,
-    seconds of the timed steps, sample description)."""
+    seconds of the timed steps, sample description, seconds per layer of each
+    type for one (sequence, token) -- None when pieces were grouped)."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import oracle
     from harness import attended_positions, build_ref_cache, fill_ref_rows, host_layer
@@ -498,6 +499,14 @@ def oracle_piece_timer(w, seed, layers, budget_s, steps, warmup):
         cnt[g] += 1
     el = time.perf_counter() - t_all
     per_seq_token = sum(a / c for a, c in zip(acc, cnt) if c)
+    # seconds per layer type (one (sequence, token)), when every piece was timed on its own
+    per_type = None
+    if n_groups == len(pieces) and all(cnt):
+        per_type = {}
+        for m in sorted(set(w.pattern)):
+            layers_m = [l for l, x in enumerate(w.pattern) if x == m]
+            tot = sum(acc[g] / cnt[g] for g in range(n_groups) if groups[g][0][1] in layers_m)
+            per_type[m] = round(tot / len(layers_m), 4)
     # one (sequence, token) of the batch; the metric's step covers batch*T of them
     per_step = per_seq_token * (w.batch * w.T)
     sample = ("sequence 0, query token %d of the %s stack (%s), single-threaded C oracle, fp64: one decode step cut "
@@ -505,7 +514,7 @@ def oracle_piece_timer(w, seed, layers, budget_s, steps, warmup):
               "whole), %d timed step(s) of one group of consecutive pieces each, round robin over %d groups; a "
               "decode step costs the sum of the groups' mean times (%.2f s)"
               % (j, w.name, w.pattern, len(pieces), slice_n, steps, n_groups, per_seq_token))
-    return len(w.pattern) / per_step, el, sample
+    return len(w.pattern) / per_step, el, sample, per_type
 
 
 def run_reference(args, world, rank):
@@ -516,13 +525,14 @@ def run_reference(args, world, rank):
         return
     w = wl.WORKLOADS[args.workload]
     layers = [wl.layer_queries(w, l, args.seed) for l in range(len(w.pattern))]
-    v, el, sample = oracle_piece_timer(w, args.seed, layers, args.ref_budget, args.steps, args.warmup)
+    v, el, sample, per_type = oracle_piece_timer(w, args.seed, layers, args.ref_budget, args.steps, args.warmup)
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "layer-steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / max(args.steps, 1) * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded, same generator as the CUDA arm)",
             "config": {"workload": w.name, "context": int(wl.seq_lens(w, args.seed).max()), "layers": w.pattern},
-            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(v, 4)},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(v, 4),
+                             "seconds_per_layer": per_type},
             "e2e": {"value": round(v, 4), "unit": "layer-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
