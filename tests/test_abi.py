@@ -102,3 +102,18 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(csa2, "LIB_PATH", str(tmp_path / "libcsa2.so"))
     with pytest.raises(RuntimeError):
         csa2.lib()
+
+
+def test_attention_merge_limit_rejected_on_host(lib):
+    # the CUDA-core path (dim not a multiple of 128) merges 32-entry chunks:
+    # 64 heads x (16,384 + 16,384) / 32 chunk weights exceed its 200 KiB of
+    # shared memory, so the call is refused before any launch
+    c = fake_cache(dim=96, row_stride=64)
+    assert lib.csa2_sparse_swa_attn(ctypes.byref(c), 0x40000, 1, 64, 0x60000, 16384, 16384, 0.0, 0x70000, None,
+                                    0x80000, 1 << 40, None) == csa2.ERR_UNSUPPORTED
+    # window or top-k beyond the 16,384 bound: invalid on any path
+    c = fake_cache()
+    assert lib.csa2_sparse_swa_attn(ctypes.byref(c), 0x40000, 1, 64, 0x60000, 2048, 16385, 0.0, 0x70000, None,
+                                    0x80000, 1 << 40, None) == csa2.ERR_INVALID_ARG
+    assert lib.csa2_sparse_swa_attn(ctypes.byref(c), 0x40000, 1, 64, 0x60000, 16385, 128, 0.0, 0x70000, None,
+                                    0x80000, 1 << 40, None) == csa2.ERR_INVALID_ARG
