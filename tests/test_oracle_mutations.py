@@ -16,6 +16,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -76,21 +77,40 @@ def _copy_tree(dst):
         shutil.copytree(os.path.join(ROOT, d), os.path.join(dst, d), ignore=ign)
 
 
+def _run_mutation(base, name, old, new):
+    """Plant one mistake in a copy of the oracle and run the pins on it:
+    (exit status, last line of the pytest report)."""
+    d = os.path.join(base, name)
+    _copy_tree(d)
+    path = os.path.join(d, "oracle", "csa2_ref.c")
+    with open(path) as f:
+        src = f.read()
+    if src.count(old) != 1:
+        return None, "the mutation does not apply"
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    r = subprocess.run([sys.executable, "-m", "pytest", *PIN_TESTS, "-x", "-q", "-p", "no:cacheprovider"],
+                       cwd=d, capture_output=True, text=True, timeout=600)
+    return r.returncode, (r.stdout.strip().splitlines() or [""])[-1]
+
+
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    # every planted mistake in its own copy, several at a time
+    base = str(tmp_path_factory.mktemp("mutations"))
+    with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+        futs = {name: ex.submit(_run_mutation, base, name, old, new) for name, old, new in MUTATIONS}
+        return {name: f.result() for name, f in futs.items()}
+
+
 def test_every_mutation_applies_to_the_current_source():
     src = open(SRC).read()
     for name, old, _ in MUTATIONS:
         assert src.count(old) == 1, name
 
 
-@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_planted_mistake_is_caught(name, old, new, tmp_path):
-    _copy_tree(str(tmp_path))
-    path = tmp_path / "oracle" / "csa2_ref.c"
-    src = path.read_text()
-    assert src.count(old) == 1, name
-    path.write_text(src.replace(old, new))
-    r = subprocess.run([sys.executable, "-m", "pytest", *PIN_TESTS, "-x", "-q", "-p", "no:cacheprovider"],
-                       cwd=str(tmp_path), capture_output=True, text=True, timeout=600)
-    tail = (r.stdout.strip().splitlines() or [""])[-1]
+@pytest.mark.parametrize("name", [m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(name, outcomes):
+    rc, tail = outcomes[name]
     # exit status 1 with a failed test: the copy built and ran, and a pin caught the mistake
-    assert r.returncode == 1 and " failed" in tail, "%s: the pins let the planted mistake through (%s)" % (name, tail)
+    assert rc == 1 and " failed" in tail, "%s: the pins let the planted mistake through (%s)" % (name, tail)
