@@ -250,3 +250,21 @@ def test_top_k_of_shard_top_ks_is_the_global_top_k():
         cand = np.concatenate(cand)
         glob = oracle.select_top(s[cand], cand, w.pool_k)
         band_set_check(glob, fp, lambda t: s[t], s.size)
+
+
+def test_token_j_of_T_equals_a_single_token_at_its_own_length():
+    # causal multi-token decode / prefill: token j of T sees exactly what a
+    # lone query token sees when the sequence ends at p_j = L - T + j
+    T, L = 5, 3000
+    w = wl.scaled(wl.WORKLOADS["long64k"], L, T=T, pool_k=512, top_k=64)
+    layer = wl.layer_queries(w, 0)
+    cache = build_ref_cache(w, rows=False, layers=[layer])
+    h = host_layer(layer)
+    for j in range(T):
+        cache.set_seq_lens([L])
+        pool, topk, _ = oracle.index_full(cache, 0, T, j, h["q_idx"][0, j], w.q_idx_dtype, h["w"][0, j],
+                                          w.pool_k, w.top_k)
+        cache.set_seq_lens([L - T + j + 1])
+        pool1, topk1, _ = oracle.index_full(cache, 0, 1, 0, h["q_idx"][0, j], w.q_idx_dtype, h["w"][0, j],
+                                            w.pool_k, w.top_k)
+        assert np.array_equal(pool, pool1) and np.array_equal(topk, topk1), j
