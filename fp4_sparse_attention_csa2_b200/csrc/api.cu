@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "../../include/csa2.h"
+#include "abi_checks.h"
 #include "kernels.h"
 
 using namespace csa2;
@@ -44,25 +45,6 @@ csa2_status check_cache(const csa2_cache* c) {
     }
     if (capacity(c) > (int64_t)1 << 30) return CSA2_ERR_UNSUPPORTED;
     return CSA2_OK;
-}
-
-DevCache dev_cache(const csa2_cache* c) {
-    DevCache d;
-    d.rows = c->kv_rows;
-    d.keys = c->idx_keys;
-    d.page_table = c->page_table;
-    d.seq_lens = c->seq_lens;
-    d.batch = c->batch;
-    d.max_pages = c->max_pages;
-    d.page_size = c->page_size;
-    d.dim = c->dim;
-    d.idx_dim = c->idx_dim;
-    d.row_stride = c->row_stride;
-    d.seq_stride = c->seq_stride_slots;
-    d.n_slots = c->n_slots;
-    d.cap = capacity(c);
-    d.key_dtype = c->idx_key_dtype == CSA2_E4M3 ? 2 : 0;
-    return d;
 }
 
 int num_sms() {
@@ -177,6 +159,34 @@ csa2_status launch_scores(const csa2_cache* cache, const void* q_idx, csa2_dtype
 
 }  // namespace
 
+DevCache csa2::dev_cache(const csa2_cache* c) {
+    DevCache d;
+    d.rows = c->kv_rows;
+    d.keys = c->idx_keys;
+    d.page_table = c->page_table;
+    d.seq_lens = c->seq_lens;
+    d.batch = c->batch;
+    d.max_pages = c->max_pages;
+    d.page_size = c->page_size;
+    d.dim = c->dim;
+    d.idx_dim = c->idx_dim;
+    d.row_stride = c->row_stride;
+    d.seq_stride = c->seq_stride_slots;
+    d.n_slots = c->n_slots;
+    d.cap = capacity(c);
+    d.key_dtype = c->idx_key_dtype == CSA2_E4M3 ? 2 : 0;
+    return d;
+}
+
+csa2_status csa2::check_reindex_args(const csa2_cache* c, const void* q_idx, csa2_dtype q_dtype,
+                                     const float* head_w, int T, int H_I, const int32_t* pool_idx, int pool_k,
+                                     int top_k, const int32_t* topk_idx) {
+    csa2_status s = check_index_args(c, q_idx, q_dtype, head_w, T, H_I, pool_k, top_k);
+    if (s != CSA2_OK) return s;
+    if (!pool_idx || !topk_idx || !aligned16(pool_idx) || !aligned16(topk_idx)) return CSA2_ERR_INVALID_ARG;
+    return CSA2_OK;
+}
+
 extern "C" {
 
 size_t csa2_workspace_bytes(const csa2_cache* cache, int T, int H, int pool_k, int top_k, int window) {
@@ -266,9 +276,8 @@ csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dty
 csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
                                int T, int H_I, const int32_t* pool_idx, int pool_k, int top_k, int32_t* topk_idx,
                                void* ws, size_t ws_bytes, void* stream) {
-    csa2_status s = check_index_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_k, top_k);
+    csa2_status s = check_reindex_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx);
     if (s != CSA2_OK) return s;
-    if (!pool_idx || !topk_idx || !aligned16(pool_idx) || !aligned16(topk_idx)) return CSA2_ERR_INVALID_ARG;
     Layout L;
     s = check_ws(cache, T, 1, pool_k, top_k, 0, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;

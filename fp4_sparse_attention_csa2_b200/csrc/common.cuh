@@ -150,4 +150,12 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Selection key of a score: 0 (never selected) for an element that is not a
+// candidate or whose score is NaN -- the mark a scorer leaves on a position it
+// had to skip (a page id outside the cache) -- else the ordered key, which is
+// never 0 for a non-NaN float.
+__device__ __forceinline__ uint32_t select_key(float f, bool candidate) {
+    return (candidate && !isnan(f)) ? ordered_key(f) : 0u;
+}
+
 }  // namespace csa2

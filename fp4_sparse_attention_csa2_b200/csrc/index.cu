@@ -81,7 +81,13 @@ k_score_full(DevCache c, const void* __restrict__ q, int q_f32, const float* __r
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= L) return;
     const int64_t slot = slot_of(c, b, t);
-    if (slot < 0) { flag(status, kStatusBounds); return; }
+    if (slot < 0) {
+        // a page outside the cache: the position is skipped (NaN is never selected)
+        flag(status, kStatusBounds);
+        for (int j = 0; j < T; ++j)
+            if (t <= L - T + j) scores[((int64_t)b * T + j) * c.cap + t] = __int_as_float(0x7fc00000);
+        return;
+    }
     float k[kDI];
     load_key(c, slot, k);
     for (int j = 0; j < T; ++j) {
@@ -148,7 +154,9 @@ k_score_pool(DevCache c, const void* __restrict__ q, int q_f32, const float* __r
     }
 #pragma unroll
     for (int o = 1; o < SPLIT; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (live && part == 0) scores[(int64_t)seg * pool_k + i] = s;
+    // every entry gets a value: NaN marks one that is padding or was skipped,
+    // and the selection never takes it (nothing stale from an earlier call is read)
+    if (i < pool_k && part == 0) scores[(int64_t)seg * pool_k + i] = live ? s : __int_as_float(0x7fc00000);
 }
 
 }  // namespace

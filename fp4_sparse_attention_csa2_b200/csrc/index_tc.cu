@@ -332,11 +332,14 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
             for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                 const int acc = g & 1;
                 if (acc != grp) continue;                       // the other group's tile
+                const int64_t t = it.t0 + (int64_t)tl * kTile + row;
+                // a position on a page outside the cache was not loaded (the
+                // producer flagged it): its score is NaN, which is never selected
+                const bool skipped = p.c.page_table != nullptr && t < it.L && slot_of(p.c, it.b, t) < 0;
                 if (!warp_wait(&bars->acc_full[acc], (g >> 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
                 // the MMAs of this tile are complete: its ring stage can be refilled
                 if ((tid & 127) == 0) tc::mbar_arrive(&bars->empty[g % kStages]);
-                const int64_t t = it.t0 + (int64_t)tl * kTile + row;
                 const uint32_t abase = lane_addr + (uint32_t)(acc * NA);
                 for (int j = 0; j < p.T; ++j) {
                     float s0 = 0.0f, s1 = 0.0f;
@@ -364,10 +367,10 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                             s1 = fmaf(ww.w, dot[3], s1);
                         }
                     }
-                    const float s = s0 + s1;
+                    const float s = skipped ? __int_as_float(0x7fc00000) : s0 + s1;
                     const bool vis = t <= it.L - p.T + j;
                     if (vis) p.scores[((int64_t)it.b * p.T + j) * p.c.cap + t] = s;
-                    if (p.hist && vis) atomicAdd(&sHist[j * kRadixBins + (ordered_key(s) >> 21)], 1u);
+                    if (p.hist && vis && !skipped) atomicAdd(&sHist[j * kRadixBins + (ordered_key(s) >> 21)], 1u);
                 }
                 tc::fence_before_sync();
                 tc::mbar_arrive(&bars->acc_empty[acc]);

@@ -10,8 +10,9 @@
 // and outputs.
 #include <mutex>
 
-#include "../../include/csa2.h"
-#include "kernels.h"
+#include <cuda.h>
+
+#include "abi_checks.h"
 
 namespace csa2 {
 namespace {
@@ -20,30 +21,67 @@ namespace {
 // pool, so batch * T * pool_k may not exceed (4 MiB - 256) / 4 = 1,048,512.
 constexpr size_t kScratchBytes = (size_t)4 << 20;
 constexpr size_t kScratchHeader = 256;
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_reindex_scratch[kScratchBytes];
 
-// Device address of g_reindex_scratch per device, looked up once per device.
-// In host code the array's name is only a stand-in for the symbol, never a
-// device address, so the address must come from cudaGetSymbolAddress.
+// Device address of g_reindex_scratch per CUDA context, looked up once per
+// context with that context current.  In host code the array's name is only a
+// stand-in for the symbol, never a device address, so the address must come
+// from cudaGetSymbolAddress.  The address belongs to the context it was looked
+// up in (the module is loaded again into a new context, e.g. after
+// cudaDeviceReset), so the cache is keyed on the current context's unique id
+// (a new context gets a new id even where its handle value is reused).
+using CtxGetCurrent = CUresult (*)(CUcontext*);
+using CtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+void* driver_fn(const char* name) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return f;
+}
+
 std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
+unsigned long long g_ctx[kMaxContexts] = {};
+void* g_addr[kMaxContexts] = {};
+int g_n = 0;
 
 cudaError_t scratch_address(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_reindex_scratch);   // with `dev` current
+    static const CtxGetCurrent get = reinterpret_cast<CtxGetCurrent>(driver_fn("cuCtxGetCurrent"));
+    static const CtxGetId get_id = reinterpret_cast<CtxGetId>(driver_fn("cuCtxGetId"));
+    if (!get || !get_id) return cudaErrorNotSupported;
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    if (!ctx) {
+        // no context bound to this thread yet: bind the current device's
+        // primary context (cudaSetDevice initialises it and makes it current)
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
-        g_addr[dev] = p;
+        e = cudaSetDevice(dev);
+        if (e != cudaSuccess) return e;
+        if (get(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
     }
-    *out = g_addr[dev];
+    unsigned long long id = 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < g_n; ++i)
+        if (g_ctx[i] == id) {
+            *out = g_addr[i];
+            return cudaSuccess;
+        }
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_reindex_scratch);   // in the current context
+    if (e != cudaSuccess) return e;
+    if (g_n < kMaxContexts) {
+        g_ctx[g_n] = id;
+        g_addr[g_n] = p;
+        ++g_n;
+    }
+    *out = p;
     return cudaSuccess;
 }
 
@@ -55,45 +93,24 @@ using namespace csa2;
 extern "C" csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
                                                   const float* head_w, int T, int H_I, const int32_t* pool_idx,
                                                   int pool_k, int top_k, int32_t* topk_idx, void* stream) {
-    if (!cache || !cache->kv_rows || !cache->idx_keys || !cache->seq_lens || !q_idx || !head_w || !pool_idx ||
-        !topk_idx)
-        return CSA2_ERR_INVALID_ARG;
-    if (T < 1 || H_I < 1 || H_I > 64 || T * H_I > 256 || top_k < 1 || top_k > pool_k || pool_k > 16384 ||
-        cache->batch < 1 || cache->idx_dim != 64)
-        return CSA2_ERR_INVALID_ARG;
-    if ((cache->idx_key_dtype == CSA2_E4M3 && q_dtype != CSA2_BF16) ||
-        (cache->idx_key_dtype == CSA2_F32 && q_dtype != CSA2_F32))
-        return CSA2_ERR_INVALID_ARG;
-    // the fixed scratch bounds the problem size
+    // the same checks, in the same order and with the same statuses, as
+    // csa2_index_reindex; only then the bound of the fixed scratch
+    csa2_status s = check_reindex_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx);
+    if (s != CSA2_OK) return s;
     const size_t need = kScratchHeader + sizeof(float) * (size_t)cache->batch * T * pool_k;
     if (need > kScratchBytes) return CSA2_ERR_UNSUPPORTED;
-    // the workspace-based entry point's validation covers the cache itself
-    if (csa2_workspace_bytes(cache, T, 1, pool_k, top_k, 0) == 0) return CSA2_ERR_INVALID_ARG;
 
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return CSA2_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint32_t* status = static_cast<uint32_t*>(scratch);
     float* scores = reinterpret_cast<float*>(static_cast<char*>(scratch) + kScratchHeader);
-    // the status word must start at zero; the scores are all written before they are read
+    // the status word must start at zero; the scorer writes a score for every
+    // pool entry (a NaN marks one it rejected), so nothing stale from an
+    // earlier call is read
     if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return CSA2_ERR_CUDA;
 
-    DevCache d;
-    d.rows = cache->kv_rows;
-    d.keys = cache->idx_keys;
-    d.page_table = cache->page_table;
-    d.seq_lens = cache->seq_lens;
-    d.batch = cache->batch;
-    d.max_pages = cache->max_pages;
-    d.page_size = cache->page_size;
-    d.dim = cache->dim;
-    d.idx_dim = cache->idx_dim;
-    d.row_stride = cache->row_stride;
-    d.seq_stride = cache->seq_stride_slots;
-    d.n_slots = cache->n_slots;
-    d.cap = cache->page_table ? (int64_t)cache->max_pages * cache->page_size : cache->seq_stride_slots;
-    d.key_dtype = cache->idx_key_dtype == CSA2_E4M3 ? 2 : 0;
-
+    const DevCache d = dev_cache(cache);
     cudaError_t e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, pool_idx, pool_k, scores, status,
                                       st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
@@ -107,7 +124,7 @@ extern "C" csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const
     src.seq_lens = cache->seq_lens;
     src.T = T;
     src.cap = d.cap;
-    SelWork unused = {};   // a pool-sized selection runs in one CTA per segment, in shared memory
+    SelWork unused = {};   // a pool-sized selection runs in one cluster per segment, in shared memory
     e = launch_select(src, unused, cache->batch * T, top_k, topk_idx, top_k, st, false);
     return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

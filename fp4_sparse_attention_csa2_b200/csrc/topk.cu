@@ -56,14 +56,15 @@ __device__ __forceinline__ int64_t n_valid_positions(const SelSrc& s, int seg) {
 __device__ __forceinline__ Elem load_elem(const SelSrc& s, int seg, int64_t i, int64_t nvalid) {
     Elem e;
     if (s.ids == nullptr) {
-        e.valid = i < nvalid;
         e.id = (int32_t)i;
-        e.key = e.valid ? ordered_key(s.vals[seg * s.vals_stride + i]) : 0u;
+        e.key = select_key(i < nvalid ? s.vals[seg * s.vals_stride + i] : 0.0f, i < nvalid);
+        e.valid = e.key != 0u;
     } else {
         // entries outside [0, p] are padding or were flagged when scored
         e.id = s.ids[seg * s.ids_stride + i];
-        e.valid = e.id >= 0 && e.id < nvalid;
-        e.key = e.valid ? ordered_key(s.vals[seg * s.vals_stride + (s.gather ? (int64_t)e.id : i)]) : 0u;
+        const bool cand = e.id >= 0 && e.id < nvalid;
+        e.key = select_key(cand ? s.vals[seg * s.vals_stride + (s.gather ? (int64_t)e.id : i)] : 0.0f, cand);
+        e.valid = e.key != 0u;
     }
     return e;
 }
@@ -502,7 +503,7 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
     auto form_keys = [&]() {
 #pragma unroll
         for (int k = 0; k < kPassPer; ++k)   // a valid key is never 0
-            keys[k] = (ids[k] >= 0 && ids[k] < nvalid) ? ordered_key(raw[k]) : 0u;
+            keys[k] = select_key(raw[k], ids[k] >= 0 && ids[k] < nvalid);
     };
     if (base < n_items) issue_chunk(base);
     // level-1 plans of both targets from the scorer's histogram (two 16-byte
@@ -862,9 +863,9 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, float* __restrict_
     for (int k = 0; k < kClPer; ++k) {
         const int i = (k * kClCtas + (int)rank) * kClThreads + tid;
         const bool valid = i < n && ids[k] >= 0 && ids[k] < nvalid;
-        keys[k] = valid ? ordered_key(src.vals[seg * src.vals_stride + (src.gather || !src.ids ? (int64_t)ids[k] : i)])
-                        : 0u;                     // the ordered key of a finite float is never 0
-        if (valid) atomicAdd(&hist[0][digit(keys[k], 1)], 1u);
+        keys[k] = select_key(valid ? src.vals[seg * src.vals_stride + (src.gather || !src.ids ? (int64_t)ids[k] : i)]
+                                   : 0.0f, valid);
+        if (keys[k]) atomicAdd(&hist[0][digit(keys[k], 1)], 1u);
     }
     cl.sync();   // every CTA's level-1 histogram (and CTA 0's zeroed counters) complete
     ClPlan pl = cluster_threshold(cl, hist[0], 0u, (uint32_t)n_out, s_wsum, &s_plan);

@@ -117,3 +117,34 @@ def test_attention_merge_limit_rejected_on_host(lib):
                                     0x80000, 1 << 40, None) == csa2.ERR_INVALID_ARG
     assert lib.csa2_sparse_swa_attn(ctypes.byref(c), 0x40000, 1, 64, 0x60000, 16385, 128, 0.0, 0x70000, None,
                                     0x80000, 1 << 40, None) == csa2.ERR_INVALID_ARG
+
+
+def test_noalloc_reindex_refuses_like_the_workspace_entry_point(lib):
+    # the workspace-free Reindex checks the same arguments as csa2_index_reindex,
+    # in the same order and with the same statuses, before its scratch bound
+    c = fake_cache()
+    args = dict(q=0x40000, dt=csa2.BF16, w=0x50000, T=1, H_I=32, pool=0x60000, pool_k=512, top_k=128, out=0x70000)
+
+    def both(cache=c, **kw):
+        a = dict(args)
+        a.update(kw)
+        r1 = lib.csa2_index_reindex(ctypes.byref(cache), a["q"], a["dt"], a["w"], a["T"], a["H_I"], a["pool"],
+                                    a["pool_k"], a["top_k"], a["out"], 0x80000, 1 << 40, None)
+        r2 = lib.csa2_index_reindex_noalloc(ctypes.byref(cache), a["q"], a["dt"], a["w"], a["T"], a["H_I"],
+                                            a["pool"], a["pool_k"], a["top_k"], a["out"], None)
+        return r1, r2
+
+    for kw, want in [(dict(q=0x40008), csa2.ERR_INVALID_ARG), (dict(w=0x50004), csa2.ERR_INVALID_ARG),
+                     (dict(pool=0x60004), csa2.ERR_INVALID_ARG), (dict(out=0x70008), csa2.ERR_INVALID_ARG),
+                     (dict(pool=None), csa2.ERR_INVALID_ARG), (dict(dt=csa2.F32), csa2.ERR_INVALID_ARG),
+                     (dict(pool_k=16385), csa2.ERR_INVALID_ARG), (dict(top_k=600), csa2.ERR_INVALID_ARG),
+                     (dict(H_I=65), csa2.ERR_INVALID_ARG), (dict(T=9), csa2.ERR_INVALID_ARG)]:
+        assert both(**kw) == (want, want), kw
+    # a malformed cache: the cache's own status, not the scratch bound's
+    for cache, want in [(fake_cache(dim=1024), csa2.ERR_UNSUPPORTED), (fake_cache(idx_dim=32), csa2.ERR_UNSUPPORTED),
+                        (fake_cache(row_stride=280), csa2.ERR_INVALID_ARG)]:
+        assert both(cache=cache, T=8, pool_k=16384, top_k=16) == (want, want)
+    # beyond the fixed scratch (batch * T * pool_k > 1,048,512) once everything else is valid
+    big = fake_cache(batch=80, seq_stride_slots=1 << 14, n_slots=80 << 14)
+    assert lib.csa2_index_reindex_noalloc(ctypes.byref(big), 0x40000, csa2.BF16, 0x50000, 1, 32, 0x60000, 16384, 16,
+                                          0x70000, None) == csa2.ERR_UNSUPPORTED

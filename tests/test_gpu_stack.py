@@ -18,42 +18,47 @@ MAX_ABS, MEAN_ABS = 2e-3, 2e-4
 
 
 def compare_stack(w, ref, got, layers, pairs, latents=None):
-    """Check every layer of `got` (from run_gpu_stack) for the (b, j) pairs.
-    With `latents`, oracle rows are quantised on demand for the attended sets."""
+    """Check every layer of `got` (from run_gpu_stack) for the (b, j) pairs,
+    each step on the GPU's own inputs so that no step's check depends on an
+    earlier step matching exactly: the Full layer's pool and top-k against the
+    oracle's Full selection; the Reindex layer's top-k against the oracle's
+    Reindex of the GPU's pool; Reuse indices byte-identical to the layer
+    before; every layer's out and lse against the oracle's attention over the
+    GPU's own top-k.  With `latents`, oracle rows are quantised on demand for
+    the attended sets.  Returns the number of index differences that lie
+    inside the cutoff band (information only; outside it a check fails)."""
     hl = [host_layer(L) for L in layers]
-    n_exact = 0
+    n_band = 0
     for (b, j) in pairs:
         p = int(ref.seq_lens[b]) - w.T + j
-        pool_ok = True
-        pool = topk = None
+        gpool_cur = None
         for l, mode in enumerate(w.pattern):
             gpool, gtopk, gout, glse = got[l]
             if mode == "F":
                 pool, topk, s = oracle.index_full(ref, b, w.T, j, hl[l]["q_idx"][b, j], w.q_idx_dtype,
                                                   hl[l]["w"][b, j], w.pool_k, w.top_k, want_scores=True)
-                d1 = band_set_check(gpool[b, j], pool, lambda t: s[t], s.size)
-                d2 = band_set_check(gtopk[b, j], topk, lambda t: s[t], s.size)
-                pool_ok = d1 == 0 and d2 == 0
+                n_band += band_set_check(gpool[b, j], pool, lambda t: s[t], s.size)
+                n_band += band_set_check(gtopk[b, j], topk, lambda t: s[t], s.size)
+                gpool_cur = gpool[b, j]
             elif mode == "R":
-                if not pool_ok:
-                    break
+                # the oracle's Reindex of the pool the GPU's Full layer produced
                 topk, s = oracle.index_reindex(ref, b, w.T, j, hl[l]["q_idx"][b, j], w.q_idx_dtype,
-                                               hl[l]["w"][b, j], pool, w.top_k, want_scores=True)
-                by_pos = {int(t): float(v) for t, v in zip(pool, s) if t >= 0}
-                pool_ok = band_set_check(gtopk[b, j], topk, lambda t: by_pos[t], len(by_pos)) == 0
+                                               hl[l]["w"][b, j], gpool_cur, w.top_k, want_scores=True)
+                by_pos = {int(t): float(v) for t, v in zip(gpool_cur, s) if t >= 0}
+                n_band += band_set_check(gtopk[b, j], topk, lambda t: by_pos[t], len(by_pos))
             else:
                 # Reuse: the device passes the indices on unchanged
-                assert np.array_equal(gtopk[b, j], got[l - 1][1][b, j])
-            if not pool_ok:
-                break
+                assert np.array_equal(gtopk[b, j], got[l - 1][1][b, j]), (l, b, j)
+            # this layer's attention over the GPU's own top-k
             if latents is not None:
-                fill_ref_rows(ref, w, b, attended_positions(topk, p, w.window), latents(b))
-            ro, rl = oracle.sparse_swa_attn(ref, b, w.T, j, wl.bf16_bits(layers[l]["q"])[b, j], topk, w.window)
+                fill_ref_rows(ref, w, b, attended_positions(gtopk[b, j], p, w.window), latents(b))
+            ro, rl = oracle.sparse_swa_attn(ref, b, w.T, j, wl.bf16_bits(layers[l]["q"])[b, j], gtopk[b, j],
+                                            w.window)
             mx, mean = attn_errors(gout[b, j], ro)
             assert mx <= MAX_ABS and mean <= MEAN_ABS, (l, b, j, mx, mean)
-            assert np.allclose(glse[b, j], rl, atol=MAX_ABS, rtol=0)
-        n_exact += pool_ok
-    return n_exact
+            lmx, lmean = attn_errors(glse[b, j], rl)
+            assert lmx <= MAX_ABS and lmean <= MEAN_ABS, (l, b, j, "lse", lmx, lmean)
+    return n_band
 
 
 @pytest.mark.parametrize("name,L,kw", [
@@ -71,7 +76,7 @@ def test_stack_small(name, L, kw):
     got, status = run_gpu_stack(dev, w, layers)
     assert status == csa2.OK
     pairs = [(b, j) for b in range(w.batch) for j in range(w.T)]
-    assert compare_stack(w, ref, got, layers, pairs) == len(pairs)
+    compare_stack(w, ref, got, layers, pairs)
 
 
 # ----------------------------------------------------------------------------- full sizes
@@ -91,8 +96,9 @@ def _full_size(name, pairs_of, sample_rows=20000):
             cache_lat[b] = wl.latent(w, b, int(ref.seq_lens[b]))
         return cache_lat[b]
 
-    n_exact = compare_stack(w, ref, got, layers, pairs, latents)
-    assert n_exact >= len(pairs) - 1, "too many (b, j) with index-set differences inside the band"
+    n_band = compare_stack(w, ref, got, layers, pairs, latents)
+    print("%s: %d (b, j) pairs checked at every layer, %d index differences inside the cutoff band"
+          % (name, len(pairs), n_band))
     # a sample of FP4 rows, bit-exact
     rng = np.random.default_rng(1)
     b = pairs[0][0]
@@ -115,7 +121,13 @@ def test_full_size_ctx1m():
 
 
 def test_full_size_batch32_paged():
-    _full_size("batch32_paged", lambda w: [(0, 0), (17, 0), (31, 0)])
+    # eight of the 32 sequences, the shortest and the longest among them
+    def pairs(w):
+        lens = wl.seq_lens(w)
+        order = [int(b) for b in np.argsort(lens)]
+        pick = sorted(set([order[0], order[-1]] + list(range(0, w.batch, 5))))[:8]
+        return [(b, 0) for b in pick]
+    _full_size("batch32_paged", pairs)
 
 
 def test_full_size_append_mq():
@@ -140,8 +152,9 @@ def test_full_size_append_mq():
     # (b) 4 query tokens per sequence through F, R, U, U
     got, status = run_gpu_stack(dev, w, layers)
     assert status == csa2.OK
-    ref = build_ref_cache(w, rows=False, layers=layers, batches=[0, w.batch - 1])
-    pairs = [(b, j) for b in (0, w.batch - 1) for j in range(w.T)]
+    checked = (0, 3, 5, w.batch - 1)
+    ref = build_ref_cache(w, rows=False, layers=layers, batches=list(checked))
+    pairs = [(b, j) for b in checked for j in range(w.T)]
     lat = {}
 
     def latents(b):
@@ -150,5 +163,6 @@ def test_full_size_append_mq():
             lat[b] = wl.latent(w, b, w.lens[1])
         return lat[b]
 
-    n_exact = compare_stack(w, ref, got, layers, pairs, latents)
-    assert n_exact >= len(pairs) - 1
+    n_band = compare_stack(w, ref, got, layers, pairs, latents)
+    print("append_mq: %d (b, j) pairs checked at every layer, %d index differences inside the cutoff band"
+          % (len(pairs), n_band))
