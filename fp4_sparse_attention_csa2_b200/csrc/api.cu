@@ -55,11 +55,12 @@ int num_sms() {
 
 // Workspace layout (byte offsets, each section 256-byte aligned):
 //   status word | full-layer scores | radix histograms | scratch histogram |
-//   radix counters | candidates 1, 2 | survivors 1, 2 | pool scores | attention partials
+//   radix counters | Reindex arrival counters | candidates 1, 2 | survivors 1, 2 |
+//   pool scores | attention partials
 // The radix histograms and counters are zero between calls: the workspace
 // starts zeroed and every large selection clears what it used.
 struct Layout {
-    size_t status, scores, hist, hist_scratch, cnt, cand1, cand2, surv1, surv2, pscores, part_o, part_ml, total;
+    size_t status, scores, hist, hist_scratch, cnt, rx_cnt, cand1, cand2, surv1, surv2, pscores, part_o, part_ml, total;
     int64_t nseg, cap, cand_stride;
     int nchunk;
 };
@@ -77,6 +78,7 @@ bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int w
     L->hist = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 3 * kRadixBins);
     L->hist_scratch = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * kRadixBins);
     L->cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * kSelCounters);
+    L->rx_cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg);
     L->cand1 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->cand2 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->surv1 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
@@ -267,10 +269,10 @@ csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dty
         return cuda_status(launch_select_dual(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, ps, pool_k, top_k,
                                               topk_idx, top_k, st, fused));
     }
-    // short contexts: the pool, its scores beside it, then the top-k taken from the pool
-    cudaError_t e = launch_select(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, pool_k, st, fused, ps);
-    if (e != cudaSuccess) return CSA2_ERR_CUDA;
-    return topk_from_pool(cache, L, ws, ps, pool_k, 0, pool_idx, pool_k, top_k, topk_idx, T, st);
+    // short contexts: the pool and, from it, the top-k, by one CTA per (sequence, token)
+    (void)ps;
+    return cuda_status(launch_select_local(src, (int)L.nseg, pool_k, pool_idx, nullptr, pool_k, top_k, topk_idx, top_k,
+                                           st));
 }
 
 csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
@@ -285,6 +287,9 @@ csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_
     DevCache d = dev_cache(cache);
     uint32_t* status = at<uint32_t>(ws, L.status);
     float* ps = at<float>(ws, L.pscores);
+    if (reindex_tc_supported(d, H_I))
+        return cuda_status(launch_reindex_tc(d, q_idx, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx, ps,
+                                             at<uint32_t>(ws, L.rx_cnt), status, st));
     cudaError_t e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, pool_idx, pool_k, ps, status, st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
     return topk_from_pool(cache, L, ws, ps, pool_k, 0, pool_idx, pool_k, top_k, topk_idx, T, st);
@@ -303,13 +308,6 @@ csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, in
     Layout L;
     s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
-    // the split-softmax merge keeps one weight per (chunk, head) in shared
-    // memory; chunks of the kernel that will run (the workspace is sized for
-    // the smallest chunk of any)
-    const int rows = attn_tc_supported(dev_cache(cache), H) ? attn_tc_rows_per_chunk() : attn_rows_per_chunk();
-    const int64_t nchunk_run = std::max<int64_t>(1, ((int64_t)window + top_k + rows - 1) / rows);
-    if (sizeof(float) * ((size_t)nchunk_run * H + 2 * (size_t)H + 256 + (4 * (256 / H) + 1) * (size_t)H) > 200 * 1024)
-        return CSA2_ERR_UNSUPPORTED;
     if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
     AttnWork aw;
     aw.part_o = at<float>(ws, L.part_o);

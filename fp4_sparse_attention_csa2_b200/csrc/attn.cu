@@ -146,114 +146,59 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
             acc.z = fmaf(e, vv.z, acc.z);
             acc.w = fmaf(e, vv.w, acc.w);
         }
-        po[(int64_t)(d + 0) * H + h] = acc.x;   // partials are [d][head]
-        po[(int64_t)(d + 1) * H + h] = acc.y;
-        po[(int64_t)(d + 2) * H + h] = acc.z;
-        po[(int64_t)(d + 3) * H + h] = acc.w;
+        *reinterpret_cast<float4*>(po + (int64_t)h * D + d) = acc;   // partials are [head][d]
     }
 }
 
-// Split-softmax merge.  grid (batch*T, D / (rows * reps)), 256 threads with
-// rows = 256/H: in round r < reps thread t covers head t % H of channel
-// rows * (reps * blockIdx.y + r) + t / H (threads past rows * H idle).  Dynamic
-// smem holds the weight of every (chunk, head), 2^(m_c - M) with M the head's
-// maximum over chunks, and the heads' totals.  Partials are [chunk][d][head],
-// base 2: a warp's loads are 32 consecutive heads.  The first kPre chunks'
-// partials are loaded before the weights are known, so the two memory
-// latencies overlap.  reps = 1 (many small CTAs, a short chain) for a few
-// sequences; more rounds per CTA when many sequences fill the GPU anyway, so
-// the weights are computed fewer times.
-constexpr int kPre = 20;
+// Split-softmax merge.  One thread per output (head h, channel d) of one
+// (sequence, query token): with chunk c's partial output O_c[h][d] (not
+// normalised) and its per-head (m_c, l_c) in base-2 units,
+//     M = max_c m_c,  L = sum_c 2^(m_c - M) l_c,  out = sum_c 2^(m_c - M) O_c / L,
+// lse = M ln 2 + ln L.  grid (batch*T, ceil(H*D / 256)), 256 threads; a warp's
+// loads of one chunk are 32 consecutive channels of one head, and every load
+// of a batch of kBatch chunks is issued before any is used (the merge runs
+// online over the batches).
+constexpr int kBatch = 24;
 
 __global__ void __launch_bounds__(256)
 k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk,
-               int reps, float* __restrict__ out, float* __restrict__ lse) {
+               float* __restrict__ out, float* __restrict__ lse) {
     pdl_begin();
-    extern __shared__ float s_w[];   // [nchunk][H], M[H], L[H], partials [256/H][H], out [H][rows * reps + 1]
-    float* s_M = s_w + (size_t)nchunk * H;
-    float* s_L = s_M + H;
-    float* s_red = s_L + H;
-    const int rows = 256 / H;                  // channels per round
-    const int span = rows * reps;              // channels per CTA
-    float* s_out = s_red + 256;
-    const int seg = blockIdx.x, tid = threadIdx.x;
-    const int d_lo = blockIdx.y * span;
-    const int dr = tid / H, h = tid % H;
-    const int64_t cstride = (int64_t)D * H;
-    // the first round's partials, in flight while the weights are worked out
-    float pre[kPre];
-    {
-        const int d = d_lo + dr;
-        const bool mine = dr < rows && d < D;
-        const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h;
+    const int seg = blockIdx.x;
+    const int i = blockIdx.y * 256 + threadIdx.x;
+    if (i >= H * D) return;
+    const int h = i / D, d = i - h * D;
+    const int64_t cs_o = (int64_t)H * D, cs_ml = (int64_t)H * 2;
+    const float* po = part_o + (int64_t)seg * nchunk * cs_o + (int64_t)h * D + d;
+    const float* ml = part_ml + (int64_t)seg * nchunk * cs_ml + (int64_t)h * 2;
+    float M = -INFINITY, Lsum = 0.0f, acc = 0.0f;
+    for (int c0 = 0; c0 < nchunk; c0 += kBatch) {
+        float o[kBatch], m[kBatch], l[kBatch];
 #pragma unroll
-        for (int c = 0; c < kPre; ++c) pre[c] = (mine && c < nchunk) ? base[c * cstride] : 0.0f;
-    }
-
-    const float* ml = part_ml + (int64_t)seg * nchunk * H * 2;
-    // per head, 256/H threads share the chunks: maximum, then weights and total
-    // (threads past per_head * H, which exist when H does not divide 256, idle)
-    const int per_head = 256 / H, part = tid / H;
-    const int c_end = part < per_head ? nchunk : 0;
-    float m = -INFINITY;
-    for (int c = part; c < c_end; c += per_head) m = fmaxf(m, ml[((int64_t)c * H + h) * 2]);
-    if (part < per_head) s_red[part * H + h] = m;
-    __syncthreads();
-    m = -INFINITY;
-    for (int k = 0; k < per_head; ++k) m = fmaxf(m, s_red[k * H + h]);
-    __syncthreads();
-    float l = 0.0f;
-    for (int c = part; c < c_end; c += per_head) {
-        const float mc = ml[((int64_t)c * H + h) * 2];
-        const float w = (m == -INFINITY || mc == -INFINITY) ? 0.0f : exp2f(mc - m);
-        s_w[c * H + h] = w;
-        l = fmaf(w, ml[((int64_t)c * H + h) * 2 + 1], l);
-    }
-    if (part < per_head) s_red[part * H + h] = l;
-    __syncthreads();
-    if (part == 0) {
-        float tot = 0.0f;
-        for (int k = 0; k < per_head; ++k) tot += s_red[k * H + h];
-        s_M[h] = m;
-        s_L[h] = tot;
-    }
-    __syncthreads();
-    for (int r = 0; r < reps; ++r) {
-        const int d = d_lo + r * rows + dr;
-        const bool mine = dr < rows && d < D;
-        const float* base = part_o + ((int64_t)seg * nchunk * D + d) * H + h;
-        if (r > 0) {
-#pragma unroll
-            for (int c = 0; c < kPre; ++c) pre[c] = (mine && c < nchunk) ? base[c * cstride] : 0.0f;
+        for (int k = 0; k < kBatch; ++k) {
+            const bool in = c0 + k < nchunk;
+            const float2 v = in ? *reinterpret_cast<const float2*>(ml + (int64_t)(c0 + k) * cs_ml) : make_float2(-INFINITY, 0.0f);
+            m[k] = v.x;
+            l[k] = v.y;
+            o[k] = in ? po[(int64_t)(c0 + k) * cs_o] : 0.0f;
         }
-        if (mine) {
-            float acc = 0.0f;
+        float mb = M;
 #pragma unroll
-            for (int c = 0; c < kPre; ++c)
-                if (c < nchunk) acc = fmaf(s_w[c * H + h], pre[c], acc);
-            int c = kPre;
-            for (; c + 4 <= nchunk; c += 4) {       // four chunks of loads in flight
-                float v[4];
+        for (int k = 0; k < kBatch; ++k) mb = fmaxf(mb, m[k]);
+        if (mb == -INFINITY) continue;                         // nothing attended so far
+        const float rs = M == -INFINITY ? 0.0f : exp2f(M - mb);   // rescale what came before
+        acc *= rs;
+        Lsum *= rs;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) v[u] = base[(c + u) * cstride];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) acc = fmaf(s_w[(c + u) * H + h], v[u], acc);
-            }
-            for (; c < nchunk; ++c) acc = fmaf(s_w[c * H + h], base[c * cstride], acc);
-            const float lt = s_L[h];
-            s_out[h * (span + 1) + r * rows + dr] = lt > 0.0f ? acc / lt : 0.0f;
+        for (int k = 0; k < kBatch; ++k) {
+            const float w = m[k] == -INFINITY ? 0.0f : exp2f(m[k] - mb);
+            acc = fmaf(w, o[k], acc);
+            Lsum = fmaf(w, l[k], Lsum);
         }
+        M = mb;
     }
-    __syncthreads();
-    // out[seg][h][d]: `span` consecutive channels of every head
-    for (int i = tid; i < H * span; i += 256) {
-        const int hh = i / span, k = i % span;
-        if (d_lo + k < D) out[((int64_t)seg * H + hh) * D + d_lo + k] = s_out[hh * (span + 1) + k];
-    }
-    if (lse && blockIdx.y == 0 && tid < H) {
-        const float lt = s_L[tid];
-        lse[(int64_t)seg * H + tid] = lt > 0.0f ? s_M[tid] * 0.6931471805599453f + logf(lt) : -INFINITY;
-    }
+    out[((int64_t)seg * H + h) * D + d] = Lsum > 0.0f ? acc / Lsum : 0.0f;
+    if (lse && d == 0) lse[(int64_t)seg * H + h] = Lsum > 0.0f ? M * 0.6931471805599453f + logf(Lsum) : -INFINITY;
 }
 
 }  // namespace
@@ -262,19 +207,10 @@ int attn_rows_per_chunk() { return kRows; }
 
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st) {
-    const int rows = 256 / H;
     const int64_t nseg = (int64_t)c.batch * T;
-    // one round per CTA while the grid stays within about four waves of a
-    // 148-SM part, else four rounds (the weights are then computed a quarter as often)
-    const int reps = nseg * ((c.dim + rows - 1) / rows) <= 4 * 148 ? 1 : 4;
-    const int span = rows * reps;
-    const size_t smem = sizeof(float) * ((size_t)aw.nchunk * H + 2 * (size_t)H + 256 + (size_t)(span + 1) * H);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_attn_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    return launch_pdl(k_attn_combine, dim3((unsigned)nseg, (unsigned)((c.dim + span - 1) / span)), dim3(256), smem, st,
-                      c.dim, H, aw.part_o, aw.part_ml, aw.nchunk, reps, out, lse);
+    const unsigned blocks = (unsigned)((H * c.dim + 255) / 256);
+    return launch_pdl(k_attn_combine, dim3((unsigned)nseg, blocks), dim3(256), 0, st, c.dim, H, aw.part_o, aw.part_ml,
+                      aw.nchunk, out, lse);
 }
 
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,

@@ -7,22 +7,28 @@
 // layer; E2M1 values with one E4M3 scale per 16 channels, used as key and
 // value of every head).
 //
-// One CTA owns 128 entries of the (window ++ top-k) list of one (sequence,
-// query token) and one group of HG heads (HG = H, or 32 or 16 when the
-// (chunk, segment) grid would otherwise leave SMs idle) -- a top-k
+// The work of one layer is a few hundred kilobytes of rows and well under a
+// GFLOP, so the kernel is built for latency: every CTA runs one short chain
+// and the grid covers the GPU.  One CTA owns 64 entries of the (window ++
+// top-k) list of one (sequence, query token) and a group of HG heads (a top-k
 // entry that is -1, beyond p or inside the window is masked, so the attended
-// set is window ∪ top-k without double counting:
-//   1. fetch each FP4 row with one bulk copy (TMA) into a staging area, and
-//      dequantise exactly to fp16 into a 128 x D tile laid out K-major with
-//      the 128-byte swizzle; while the rows are in flight, convert the
-//      group's bf16 queries to fp16 scaled by a power of two per head (exact)
-//      in the same layout;
-//   2. S[pos, head] = V Q^T : tcgen05.mma M=128 (positions), N=HG, K=D;
-//   3. softmax read straight from the tensor memory (thread = position):
-//      per-head max and exp over the 128 positions; P (fp16) written K-major;
-//   4. O^T[d, head] = V^T P^T : the same V bytes read through an MN-major
-//      descriptor, one M=128 slab of d per accumulator;
-//   5. unnormalised partial output ([d][head]) and (max, sum) per head in
+// set is window ∪ top-k without double counting):
+//   1. 512 worker threads issue every load at once: the group's bf16 queries,
+//      the top-k entries, then each row's codes and scales (8 threads per row,
+//      64 channels each) straight into registers;
+//   2. queries -> fp16 scaled by a power of two per head (exact), rows ->
+//      fp16 by bit placement and two exact fp16 products (see
+//      e2m1x8_to_f16x2_scaled), both stored K-major with the 128-byte swizzle;
+//   3. S[pos, head] = V Q^T on the tensor core (M = 128: rows 64..127 of the
+//      operand are the next K block's rows, their S rows are never used),
+//      its K = D split over four accumulators issued by four warps at once
+//      (one thread issues an MMA every ~70 cycles, and the 32 of one K = 512
+//      product would otherwise be one chain), summed by the softmax;
+//   4. softmax read from the tensor memory by 8 warps (thread = position,
+//      2 warps' maxima and sums per head through shared memory); P in fp16;
+//   5. O^T[d, head] = V^T P^T (K = the 64 positions), one M = 128 slab of d
+//      per accumulator, the slabs issued by the same four warps;
+//   6. the unnormalised partial output [head][d] and (max, sum) per head in
 //      base-2 units to the workspace, merged by the split-softmax combine kernel.
 #include "common.cuh"
 #include "kernels.h"
@@ -32,42 +38,56 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kRows = 128;
-constexpr int kWorkers = 256;               // 8 warps: rows, queries, dequantisation, softmax, stores
+constexpr int kRows = 64;                   // entries per CTA
+constexpr int kWorkers = 512;               // 16 warps
 constexpr int kThreads = kWorkers + 32;     // + the warp that allocates TMEM and issues the MMAs
+constexpr int kBlkBytes = kRows * 128;      // one 64-channel K block of the V tile: 64 rows x 128 B
+constexpr uint32_t kDrainLimit = 65536;
+constexpr int kIssuers = 4;                 // warps 12..15 (lane 0) issue the MMAs, one accumulator each
+constexpr int kIssuer0 = 12;
 
 struct Params {
     DevCache c;
     const __nv_bfloat16* q;   // [B*T][H][D]
     const int32_t* topk;      // [B*T][top_k]
-    int T, H, HG, top_k, window, nchunk;
+    int T, H, top_k, window, nchunk;
     float scale;
-    float* part_o;            // [seg][chunk][D][H]
+    float* part_o;            // [seg][chunk][H][D]
     float* part_ml;           // [seg][chunk][H][2]
     uint32_t* status;
-    uint32_t row_bytes;       // bytes fetched per row: D/2 codes + D/16 scales, rounded up to 16
-    uint32_t stage_stride;    // row pitch of the staging area: row_bytes, or + 16 to make it an odd multiple of 16
-    uint32_t off_q, off_stage, off_misc, tmem_cols;
+    uint32_t off_q, off_p, off_misc, tmem_cols;
 };
 
+template <int HG>
 struct Misc {
-    float fac[64];               // per head of the group: softmax scale * log2(e) / query scale
-    float red[8][64];            // per head: the four warps' maxima (rows 0-3) and sums (rows 4-7)
-    int32_t pos[kRows];
-    uint64_t row_bar;            // the chunk's row copies (one arrival per row)
-    uint64_t kb_bar[8];          // K block k of V written (one arrival per worker)
-    uint64_t s_bar;              // S = V Q^T complete
-    uint64_t p_bar;              // P written (one arrival per worker)
-    uint64_t o_bar[4];           // slab s of O^T complete
-    uint64_t drain_bar;          // every MMA of the CTA complete
+    float fac[HG];               // per head of the group: softmax scale * log2(e) / query scale
+    float red[4][HG];            // per head: maxima of the two row halves (0, 1), sums (2, 3)
+    uint64_t vq_bar;             // V and Q written (one arrival per worker)
+    uint64_t s_bar;              // S = V Q^T complete (one commit per issuing warp)
+    uint64_t p_bar;              // P written (one arrival per softmax thread)
+    uint64_t o_bar;              // O^T complete (one commit per issuing warp)
+    uint64_t drain_bar;          // every MMA of the CTA complete (one commit per issuing warp)
     uint32_t tmem_base;
 };
 
-__device__ __forceinline__ uint32_t cvt_e2m1x2_f16x2(uint32_t byte) {
-    uint32_t r;
-    const uint16_t in = (uint16_t)(byte & 0xFF);
-    asm("{\n\t.reg .b8 b, u;\n\tmov.b16 {b, u}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(r) : "h"(in));
-    return r;
+// Eight E2M1 codes (one 32-bit word, channel 2j in the low nibble of byte j)
+// to four fp16 pairs holding value(code) * 2^-14, by bit placement alone: an
+// E2M1 code s.e1e0.m placed at fp16 bits 15 and 11..9 is the fp16 number
+// 2^(e-15) (1 + m/2) = value * 2^-14 for e > 0, and the subnormal m * 2^-15 =
+// value * 2^-14 for e = 0 (the sign is kept, so -0 stays -0).  Pair k holds
+// channels 2k (low half) and 2k + 1 (high half).  Integer instructions only:
+// several times the throughput of the E2M1 conversion instruction.
+__device__ __forceinline__ void e2m1x8_to_f16x2_scaled(uint32_t w, uint32_t* out) {
+    // per byte: sign << 7 | magnitude << 1 of the byte's low nibble (fe) and high nibble (fo)
+    const uint32_t fe = ((w << 4) & 0x80808080u) | ((w << 1) & 0x0E0E0E0Eu);
+    const uint32_t fo = (w & 0x80808080u) | ((w >> 3) & 0x0E0E0E0Eu);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t r;
+        // high byte of the low half <- byte k of fe, high byte of the high half <- byte k of fo
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(fe), "r"(fo), "r"((uint32_t)(k << 4) | ((uint32_t)(4 + k) << 12)));
+        out[k] = r & 0xFF00FF00u;
+    }
 }
 
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
@@ -80,196 +100,110 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     return r;
 }
 
-// Named barrier of one worker warpgroup (128 threads; ids 2 and 3).
-__device__ __forceinline__ void group_sync(int wgrp) {
-    asm volatile("bar.sync %0, 128;" ::"r"(2 + wgrp) : "memory");
-}
-
 // The float an order-preserving key came from (-0 comes back as +0).
 __device__ __forceinline__ float key_to_float(uint32_t key) {
     return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
-// Softmax, first half, for NV heads c0.. of this thread's position: the
-// scaled logits (-inf where the position is empty) into z, and this warp's
-// maximum of each head into red[quad][head].
-template <int NV>
-__device__ __forceinline__ void logits_max(uint32_t trow, int c0, bool valid, Misc* misc, int quad, int lane, float* z) {
-    float v[NV];
-    if constexpr (NV == 8) tc::tmem_ld8(trow + c0, v);
-    else tc::tmem_ld16(trow + c0, v);
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        z[i] = valid ? v[i] * misc->fac[c0 + i] : -INFINITY;
-        const uint32_t mk = __reduce_max_sync(0xffffffffu, ordered_key(z[i]));
-        if (lane == i) misc->red[quad][c0 + i] = key_to_float(mk);
-    }
-}
+// Named barrier of the softmax warps (the 8 warps that can read TMEM lanes 0..63).
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-// Softmax, second half: p = 2^(z - m) per head, rounded to fp16 and stored in
-// the K-major P operand (row = head, 64 positions per 128-byte row, chunk pc,
-// element el); this warp's sum of the rounded values into red[4 + quad][head].
-// The sums leave the warp by an exchange that halves the values a lane
-// carries at each step (NV - 1 shuffles for NV heads, not 5 NV); lanes 2 j
-// and 2 j + 1 end with head j mod NV.
-template <int NV>
-__device__ __forceinline__ void probs_sums(uint8_t* prow, int pc, int el, int c0, Misc* misc, int quad, int lane,
-                                           const float* z) {
-    float sv[NV];
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int h = c0 + i;
-        const float m = fmaxf(fmaxf(misc->red[0][h], misc->red[1][h]), fmaxf(misc->red[2][h], misc->red[3][h]));
-        const float e = m == -INFINITY ? 0.0f : exp2f(z[i] - m);
-        const __half ph = __float2half_rn(e);
-        *reinterpret_cast<__half*>(prow + tc::sw128_offset(h, pc) + 2 * el) = ph;
-        sv[i] = __half2float(ph);
-    }
-#pragma unroll
-    for (int w = NV / 2; w >= 1; w >>= 1) {
-        const bool up = (lane & (2 * w)) != 0;
-#pragma unroll
-        for (int i = 0; i < w; ++i) {
-            const float send = up ? sv[i] : sv[i + w];
-            const float keep = up ? sv[i + w] : sv[i];
-            sv[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2 * w);
-        }
-    }
-    sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], 1);
-#pragma unroll
-    for (int o = 2 * NV; o < 32; o <<= 1) sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], o);
-    if (lane < 2 * NV && (lane & 1) == 0) misc->red[4 + quad][c0 + (lane >> 1)] = sv[0];
-}
-
-// Named barrier of the kWorkers worker threads (the MMA warp is not part of it).
-__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kWorkers) : "memory"); }
-
+template <int HG>
 __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int D = p.c.dim, H = p.H, HG = p.HG;
-    const int nkb = D / 64;                     // 64-wide K blocks of the V tile
-    uint8_t* sV = smem;                         // nkb x [128 rows x 128 B]
-    uint8_t* sQ = smem + p.off_q;               // nkb x [HG rows x 128 B]; later P
-    uint8_t* sP = sQ;                           // 2 x [HG rows x 128 B] (after S is computed)
-    uint8_t* sStage = smem + p.off_stage;       // [128 rows][stage_stride]: the FP4 rows as fetched (inside sV)
-    Misc* misc = reinterpret_cast<Misc*>(smem + p.off_misc);
+    const int D = p.c.dim, H = p.H;
+    const int nkb = D / 64;                     // 64-channel K blocks
+    uint8_t* sV = smem;                         // (nkb + 1) x [64 rows x 128 B]: M = 128 reads one block past the last
+    uint8_t* sQ = smem + p.off_q;               // nkb x [HG rows x 128 B]
+    uint8_t* sP = smem + p.off_p;               // [HG rows x 128 B]: 64 positions per head
+    Misc<HG>* misc = reinterpret_cast<Misc<HG>*>(smem + p.off_misc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int chunk = blockIdx.x, seg = blockIdx.y, h_base = blockIdx.z * HG;
     if (tid == 0) {
-        tc::mbar_init(&misc->row_bar, kRows);
-        for (int k = 0; k < 8; ++k) tc::mbar_init(&misc->kb_bar[k], kWorkers);
-        tc::mbar_init(&misc->s_bar, 1);
-        tc::mbar_init(&misc->p_bar, kWorkers);
-        for (int s = 0; s < 4; ++s) tc::mbar_init(&misc->o_bar[s], 1);
-        tc::mbar_init(&misc->drain_bar, 1);
+        tc::mbar_init(&misc->vq_bar, kWorkers);
+        tc::mbar_init(&misc->s_bar, kIssuers);
+        tc::mbar_init(&misc->p_bar, 256);
+        tc::mbar_init(&misc->o_bar, kIssuers);
+        tc::mbar_init(&misc->drain_bar, kIssuers);
         tc::fence_mbar_init();
     }
+    if (warp == kWorkers / 32) tc::tmem_alloc(&misc->tmem_base, p.tmem_cols);
+    tc::fence_before_sync();
     __syncthreads();
-    // everything below may read what the preceding kernel wrote (and the
-    // tensor memory is allocated only once that kernel has released its own)
+    tc::fence_after_sync();
+    const uint32_t tmem = misc->tmem_base;
+    // everything below may read what the preceding kernel wrote
     pdl_begin();
     const int b = seg / p.T, j = seg % p.T;
 
     if (warp == kWorkers / 32) {
-        // ================= MMA warp: TMEM, then both products as their operands arrive
-        tc::tmem_alloc(&misc->tmem_base, p.tmem_cols);
-        tc::fence_before_sync();
-        __syncthreads();                                  // (1) operands staged, TMEM address published
-        tc::fence_after_sync();
-        const uint32_t tmem = misc->tmem_base;
-        if (lane == 0) {
-            bool ok = true;
-            // S = V Q^T, one 64-wide K block at a time as the workers finish it
-            const uint32_t idesc1 = tc::idesc_f16_f32(kRows, HG);
-            const uint32_t v0 = tc::smem_u32(sV), q0 = tc::smem_u32(sQ), p0 = tc::smem_u32(sP);
-            for (int kb = 0; kb < nkb; ++kb) {
-                ok = ok && tc::mbar_wait(&misc->kb_bar[kb], 0);
-                if (!ok) break;
-                tc::fence_after_sync();
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    tc::mma_f16(tmem, tc::desc_sw128(v0 + kb * (kRows * 128) + 32 * k),
-                                tc::desc_sw128(q0 + kb * (HG * 128) + 32 * k), idesc1, (kb | k) != 0);
-            }
-            tc::mma_commit(&misc->s_bar);                 // arrives once the issued MMAs are done
-            // O^T = V^T P^T, one 128-wide slab of d per accumulator, each slab committed on its own
-            ok = ok && tc::mbar_wait(&misc->p_bar, 0);
-            if (ok) tc::fence_after_sync();
-            const uint32_t idesc2 = tc::idesc_f16_f32(kRows, HG, /*a_mn=*/true, /*b_mn=*/false);
-            for (int s = 0; s < D / 128; ++s) {
-                if (ok)
-                    for (int ks = 0; ks < kRows / 16; ++ks)
-                        tc::mma_f16(tmem + (uint32_t)(HG + s * HG),
-                                    tc::desc_mn_sw128(v0 + (2 * s) * (kRows * 128) + ks * 2048, kRows * 128, 1024),
-                                    tc::desc_sw128(p0 + (ks >> 2) * (HG * 128) + 32 * (ks & 3)), idesc2, ks != 0);
-                tc::mma_commit(&misc->o_bar[s]);
-            }
-            tc::mma_commit(&misc->drain_bar);
-            ok = tc::mbar_wait(&misc->drain_bar, 0) && ok;   // nothing in flight when TMEM is freed
-            if (!ok) flag(p.status, kStatusTimeout);
-        }
+        // ================= the warp that owns the tensor memory: once every
+        // MMA the issuing warps started is complete, release it
+        bool ok = true;
+        if (lane == 0) ok = tc::mbar_wait(&misc->drain_bar, 0, kDrainLimit);
+        if (!ok) flag(p.status, kStatusTimeout);
         __syncwarp();
         tc::fence_before_sync();
-        __syncthreads();                                  // (2) the workers are done with TMEM
+        __syncthreads();                                  // the workers are done with TMEM
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, p.tmem_cols);
         return;
     }
 
-    // ================= workers (8 warps)
-    // loads that do not depend on each other are issued together: this
-    // thread's top-k entry, the group's queries, the sequence length
-    const int v_entry = chunk * kRows + tid;
-    const bool is_topk = tid < kRows && v_entry >= p.window && v_entry < p.window + p.top_k;
-    int32_t t_raw = -1;
-    if (is_topk) t_raw = __ldg(p.topk + (int64_t)seg * p.top_k + (v_entry - p.window));
-    // queries: tph consecutive threads share one head, D / tph consecutive values each
-    const int tph = kWorkers / HG;                   // 4, 8 or 16
-    const int hl = tid / tph, part = tid % tph;
-    const int span = D / tph;                        // a multiple of 8, at most 128
-    uint4 qv[16];
-    {
-        const __nv_bfloat16* src = p.q + ((int64_t)seg * H + h_base + hl) * D + part * span;
+    // ================= workers (16 warps)
+    // every load that does not depend on another is issued first: the
+    // group's queries (tph threads per head, `span` channels each), the
+    // sequence length, this thread's top-k entry
+    // tph threads per head, at least 8 channels each (one 16-byte load)
+    const int tph = (kWorkers / HG) < (D / 8) ? (kWorkers / HG) : (D / 8);
+    const int hl = tid / tph, qpart = tid % tph;
+    const bool q_thread = hl < HG;
+    const int span = D / tph;                        // 8 .. 64 channels, a multiple of 8
+    uint4 qv[8];
+    if (q_thread) {
+        const __nv_bfloat16* src = p.q + ((int64_t)seg * H + h_base + hl) * D + qpart * span;
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < 8; ++i)
             if (8 * i < span) qv[i] = __ldg(reinterpret_cast<const uint4*>(src + 8 * i));
     }
+    // rows: thread t covers row r = t % 64, channels [64 kp, 64 kp + 64) (K block kp)
+    const int r = tid & (kRows - 1), kp = tid >> 6;
+    const bool row_thread = kp < nkb;
+    const int v_entry = chunk * kRows + r;
+    const bool is_topk = v_entry >= p.window && v_entry < p.window + p.top_k;
+    int32_t t_raw = -1;
+    if (is_topk) t_raw = __ldg(p.topk + (int64_t)seg * p.top_k + (v_entry - p.window));
     const int64_t L = seq_len(p.c, b, p.status);
     const int64_t pq = L - p.T + j;
-
-    // ---- rows: thread r < 128 resolves entry r of the chunk and fetches its
-    // whole FP4 row (codes + scales) with one bulk copy into the staging area
-    if (tid < kRows) {
-        int32_t t = -1;
-        if (pq >= 0 && v_entry < p.window + p.top_k) {
-            if (v_entry < p.window) {
-                t = pq - v_entry >= 0 ? (int32_t)(pq - v_entry) : -1;
-            } else {
-                t = t_raw;
-                if (t < -1 || t >= L) { flag(p.status, kStatusBounds); t = -1; }
-                else if (t > pq || t > pq - p.window) t = -1;   // future, or already in the window
-            }
-        }
-        const int64_t slot = t >= 0 ? slot_of(p.c, b, t) : -1;
-        if (t >= 0 && slot < 0) { flag(p.status, kStatusBounds); t = -1; }
-        misc->pos[tid] = t;
-        if (t >= 0) {
-            tc::mbar_arrive_expect_tx(&misc->row_bar, p.row_bytes);
-            tc::bulk_g2s(sStage + tid * p.stage_stride, p.c.rows + slot * p.c.row_stride, p.row_bytes,
-                         &misc->row_bar);
+    int32_t t = -1;
+    if (pq >= 0 && v_entry < p.window + p.top_k) {
+        if (!is_topk) {
+            t = pq - v_entry >= 0 ? (int32_t)(pq - v_entry) : -1;
         } else {
-            tc::mbar_arrive(&misc->row_bar);
+            t = t_raw;
+            if (t < -1 || t >= L) { if (kp == 0) flag(p.status, kStatusBounds); t = -1; }
+            else if (t > pq || t > pq - p.window) t = -1;   // future, or already in the window
         }
     }
+    const int64_t slot = t >= 0 ? slot_of(p.c, b, t) : -1;
+    if (t >= 0 && slot < 0) { if (kp == 0) flag(p.status, kStatusBounds); t = -1; }
+    uint4 cv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+    uint32_t sv = 0;
+    if (row_thread && t >= 0) {
+        const uint8_t* row = p.c.rows + slot * p.c.row_stride;
+        cv[0] = __ldg(reinterpret_cast<const uint4*>(row + 32 * kp));
+        cv[1] = __ldg(reinterpret_cast<const uint4*>(row + 32 * kp + 16));
+        sv = __ldg(reinterpret_cast<const uint32_t*>(row + (D >> 1) + 4 * kp));
+    }
 
-    // ---- queries to fp16 scaled by 2^e per head, the row maximum in
-    // [2^14, 2^15) so that every bf16 value down to 2^-32 of it is exact
-    {
+    // ---- queries to fp16 scaled by 2^e per head, the head's maximum in
+    // [2^14, 2^15) so that every bf16 value down to 2^-24 of it is exact
+    if (q_thread) {
         float m = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 8; ++i) {
             if (8 * i < span) {
                 const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
 #pragma unroll
@@ -277,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
                     m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[k] << 16)), fabsf(__uint_as_float(wv[k] & 0xFFFF0000u))));
             }
         }
+        // the tph threads of a head are consecutive lanes of one warp (tph a power of two, at most 32)
         for (int o = 1; o < tph; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         int e = 0;
         if (m > 0.0f) {
@@ -285,9 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         }
         const float up = __uint_as_float((uint32_t)(127 + e) << 23);
         // logits in base-2 units: softmax_scale * log2(e) / 2^e
-        if (part == 0) misc->fac[hl] = p.scale * 1.4426950408889634f * __uint_as_float((uint32_t)(127 - e) << 23);
+        if (qpart == 0) misc->fac[hl] = p.scale * 1.4426950408889634f * __uint_as_float((uint32_t)(127 - e) << 23);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 8; ++i) {
             if (8 * i < span) {
                 const uint32_t wv[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
                 uint32_t hv[4];
@@ -297,172 +232,233 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
                                                    __uint_as_float(wv[k] & 0xFFFF0000u) * up);
                     memcpy(&hv[k], &hh, 4);
                 }
-                const int d = part * span + 8 * i;        // 8 values: one 16-byte chunk
+                const int d = qpart * span + 8 * i;       // 8 values: one 16-byte chunk
                 *reinterpret_cast<uint4*>(sQ + (d >> 6) * (HG * 128) + tc::sw128_offset(hl, (d & 63) >> 3)) =
                     make_uint4(hv[0], hv[1], hv[2], hv[3]);
             }
         }
     }
-    tc::fence_proxy_async_smem();                     // the queries are an MMA operand
-    tc::fence_before_sync();
-    __syncthreads();                                  // (1) pos[], queries, TMEM address
-    tc::fence_after_sync();
-    const uint32_t tmem = misc->tmem_base;
 
-    // ---- dequantise: value(code) * value(scale), exact in fp16, into the
-    // swizzled V tile.  Thread t owns row t % 128 and the 32-channel chunks
-    // cc = 2k + t / 128 (k < D / 64), so a warp's 16-byte accesses walk 32
-    // consecutive rows: conflict-free in the staging area (odd 16-byte row
-    // stride) and in the 128-byte-swizzled tile.  The staging area overlaps the
-    // tile, so every read is done before the first write; masked rows become 0.
-    // K block k is handed to the MMA warp as soon as every worker has written it.
-    bool ok = tc::mbar_wait(&misc->row_bar, 0);
-    const bool rows_ok = ok;
-    const int r = tid & (kRows - 1), half = tid >> 7;
-    const int n_own = D / 64;                        // chunks per thread, at most 8
-    const bool live = misc->pos[r] >= 0;
-    uint4 code[8];
-    uint16_t scl[8];
-    {
-        const uint8_t* row = sStage + r * p.stage_stride;
+    // ---- dequantise this thread's 64 channels of its row: value(code) *
+    // value(scale), exact in fp16, into K block kp of the swizzled V tile
+    // (masked rows are 0).  A warp's 16-byte stores walk 32 consecutive rows
+    // of one K block: conflict-free under the 128-byte swizzle.
+    if (row_thread) {
+        uint32_t s2[2];
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2[0]) : "h"((uint16_t)(sv & 0xFFFFu)));
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2[1]) : "h"((uint16_t)(sv >> 16)));
+        const uint32_t two14 = 0x74007400u;                      // (2^14, 2^14) in fp16
+        const uint32_t cw[8] = {cv[0].x, cv[0].y, cv[0].z, cv[0].w, cv[1].x, cv[1].y, cv[1].z, cv[1].w};
+        uint8_t* blk = sV + kp * kBlkBytes;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            if (k < n_own) {
-                const int cc = 2 * k + half;
-                code[k] = live ? *reinterpret_cast<const uint4*>(row + cc * 16) : make_uint4(0u, 0u, 0u, 0u);
-                scl[k] = live ? *reinterpret_cast<const uint16_t*>(row + (D >> 1) + 2 * cc) : (uint16_t)0;
-            }
+        for (int c = 0; c < 8; ++c) {                            // 8 channels per 16-byte chunk c
+            const uint32_t sc = c < 4 ? (c < 2 ? (s2[0] & 0xFFFFu) : (s2[0] >> 16))
+                                      : (c < 6 ? (s2[1] & 0xFFFFu) : (s2[1] >> 16));
+            const uint32_t s_pair = sc * 0x10001u;               // (s, s): scale of channels 16 (c / 2) ..
+            uint32_t hv[4];
+            e2m1x8_to_f16x2_scaled(cw[c], hv);
+            // value * 2^-14 -> value (exact, a normal fp16), then times the
+            // block scale (exact: E2M1 x E4M3 products fit fp16)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) hv[k] = hmul2_u32(hmul2_u32(hv[k], two14), s_pair);
+            *reinterpret_cast<uint4*>(blk + tc::sw128_offset(r, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
     }
-    workers_sync();
+    tc::fence_proxy_async_smem();                     // V and Q are MMA operands
+    tc::mbar_arrive(&misc->vq_bar);
+    // ---- S = V Q^T: M = 128 rows (64 real), N = HG, K = D split in kIssuers
+    // parts; issuer i accumulates K blocks [i nkb / kIssuers, (i + 1) nkb / kIssuers)
+    // into TMEM columns [i HG, (i + 1) HG)
+    const int issuer = warp - kIssuer0;               // 0..3 on the issuing warps
+    const int nacc = nkb < kIssuers ? nkb : kIssuers; // S accumulators in use (D / 64 of them when D < 256)
+    const bool issues = issuer >= 0 && issuer < kIssuers && lane == 0;
+    const uint32_t v0 = tc::smem_u32(sV), q0 = tc::smem_u32(sQ), p0 = tc::smem_u32(sP);
+    bool iss_ok = true;
+    if (issues) {
+        iss_ok = tc::mbar_wait(&misc->vq_bar, 0);
+        if (iss_ok) {
+            tc::fence_after_sync();
+            const uint32_t idesc1 = tc::idesc_f16_f32(128, HG);
+            const uint64_t dv = tc::desc_sw128(v0), dq = tc::desc_sw128(q0);
+            // issuer i < nacc takes K blocks [i nkb / nacc, (i + 1) nkb / nacc); the others none
+            const int kb0 = issuer < nacc ? issuer * nkb / nacc : 0;
+            const int kb1 = issuer < nacc ? (issuer + 1) * nkb / nacc : 0;
+            for (int kb = kb0; kb < kb1; ++kb)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        if (k < n_own) {
-            uint32_t s2;
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(scl[k]));
-            const uint32_t s_lo = (s2 & 0xFFFFu) * 0x10001u;            // (s0, s0)
-            const uint32_t s_hi = (s2 >> 16) * 0x10001u;                // (s1, s1)
-            const uint32_t cw[4] = {code[k].x, code[k].y, code[k].z, code[k].w};
-            uint32_t hv[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int bb = 0; bb < 4; ++bb)
-                    hv[4 * q + bb] = hmul2_u32(cvt_e2m1x2_f16x2(cw[q] >> (8 * bb)), q < 2 ? s_lo : s_hi);
-            uint8_t* blk = sV + k * (kRows * 128);               // K block k = cc / 2
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4*>(blk + tc::sw128_offset(r, 4 * half + q)) =
-                    make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&misc->kb_bar[k]);
+                for (int k = 0; k < 4; ++k)
+                    tc::mma_f16(tmem + (uint32_t)(issuer * HG),
+                                tc::desc_at(dv, (uint32_t)kb * kBlkBytes + 32u * k),
+                                tc::desc_at(dq, (uint32_t)kb * (HG * 128) + 32u * k), idesc1, kb != kb0 || k != 0);
         }
+        tc::mma_commit(&misc->s_bar);                 // arrives once this issuer's MMAs are done
     }
 
-    // ---- softmax straight from the tensor memory.  Thread = position (the
-    // TMEM lane of its warp's quarter); each warpgroup takes one half of the
-    // group's heads.  Per head: the maximum over the 128 positions (a
-    // warp-wide max of order-preserving integer keys, then the four warps'
-    // through shared memory); p = 2^(z - m) in fp16, stored straight into the
-    // K-major P operand; the sum of the fp16 values as the MMA will use them.
+    // ---- softmax straight from the tensor memory.  The 8 warps that can read
+    // TMEM lanes 0..63 (warp % 4 < 2): thread = position (lane group quad),
+    // cg = warp / 4 takes HG / 4 heads.  Per head: the maximum over the 64
+    // positions (a warp-wide max of order-preserving integer keys, then the
+    // two row halves' through shared memory); p = 2^(z - m) in fp16, stored
+    // straight into the K-major P operand; the sum of the fp16 values as the
+    // MMA will use them.
+    constexpr int NV = HG / 4;                       // 4, 8 or 16 heads per softmax thread
+    const int quad = warp & 3, cg = warp >> 2;
+    const bool smx = quad < 2;
+    // (every worker's writes before its vq_bar arrival -- the per-head
+    // factors among them -- are visible once that phase is seen complete)
+    bool ok = tc::mbar_wait(&misc->vq_bar, 0);
     ok = tc::mbar_wait(&misc->s_bar, 0) && ok;
     tc::fence_after_sync();
-    const int wgrp = warp >> 2, quad = warp & 3;
-    const int hc = HG / 2;                           // heads of a warpgroup: 8, 16 or 32
     ok = __all_sync(0xffffffffu, ok);                // warp-uniform from here on
-    const int pos = quad * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const bool valid = misc->pos[pos] >= 0;
-    float zz[32];
-    if (ok) {
-        if (hc == 8) {
-            logits_max<8>(trow, wgrp * 8, valid, misc, quad, lane, zz);
-        } else {
+    if (smx) {
+        // a softmax thread's position is the row r = tid % 64 it loaded: its t says whether it is attended
+        const int pos = quad * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        const bool valid = t >= 0;
+        const int c0 = cg * NV;
+        float z[NV];
+        if (ok) {
+            // S = the sum of the issuers' partial products over K
+            float v[NV];
 #pragma unroll
-            for (int blk = 0; blk < 2; ++blk)
-                if (blk * 16 < hc) logits_max<16>(trow, wgrp * hc + blk * 16, valid, misc, quad, lane, zz + 16 * blk);
-        }
-    }
-    group_sync(wgrp);
-    if (ok) {
-        uint8_t* prow = sP + (pos >> 6) * (HG * 128);
-        const int pc = (pos & 63) >> 3, el = pos & 7;
-        if (hc == 8) {
-            probs_sums<8>(prow, pc, el, wgrp * 8, misc, quad, lane, zz);
-        } else {
+            for (int i = 0; i < NV; ++i) v[i] = 0.0f;
 #pragma unroll
-            for (int blk = 0; blk < 2; ++blk)
-                if (blk * 16 < hc) probs_sums<16>(prow, pc, el, wgrp * hc + blk * 16, misc, quad, lane, zz + 16 * blk);
+            for (int a = 0; a < kIssuers; ++a) {
+                if (a >= nacc) break;
+                float u[NV];
+                const uint32_t col = trow + (uint32_t)(a * HG + c0);
+                if constexpr (NV == 4) {
+                    uint32_t rr[4];
+                    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(rr[0]), "=r"(rr[1]), "=r"(rr[2]), "=r"(rr[3]) : "r"(col));
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) u[i] = __uint_as_float(rr[i]);
+                } else if constexpr (NV == 8) {
+                    tc::tmem_ld8(col, u);
+                } else {
+                    tc::tmem_ld16(col, u);
+                }
+#pragma unroll
+                for (int i = 0; i < NV; ++i) v[i] += u[i];
+            }
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                z[i] = valid ? v[i] * misc->fac[c0 + i] : -INFINITY;
+                const uint32_t mk = __reduce_max_sync(0xffffffffu, ordered_key(z[i]));
+                if (lane == i) misc->red[quad][c0 + i] = key_to_float(mk);
+            }
         }
-    }
-    tc::fence_proxy_async_smem();                     // P is an MMA operand
-    tc::mbar_arrive(&misc->p_bar);
-    group_sync(wgrp);
-    {
-        const int t = tid & 127;                      // thread of the warpgroup
-        if (ok && t < hc) {
-            const int h = wgrp * hc + t;
-            const float m = fmaxf(fmaxf(misc->red[0][h], misc->red[1][h]), fmaxf(misc->red[2][h], misc->red[3][h]));
-            const float l = (misc->red[4][h] + misc->red[5][h]) + (misc->red[6][h] + misc->red[7][h]);
+        softmax_sync();
+        float sums[NV];
+        if (ok) {
+            uint8_t* prow = sP;
+            const int pc = pos >> 3, el = pos & 7;
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                const int h = c0 + i;
+                const float m = fmaxf(misc->red[0][h], misc->red[1][h]);
+                const float e = m == -INFINITY ? 0.0f : exp2f(z[i] - m);
+                const __half ph = __float2half_rn(e);
+                *reinterpret_cast<__half*>(prow + tc::sw128_offset(h, pc) + 2 * el) = ph;
+                sums[i] = __half2float(ph);
+            }
+        }
+        tc::fence_proxy_async_smem();                 // P is an MMA operand
+        tc::mbar_arrive(&misc->p_bar);
+        if (ok) {
+            // per-head warp sums: an exchange that halves the values a lane
+            // carries at each step; lanes 2 j and 2 j + 1 end with head j mod NV
+#pragma unroll
+            for (int w = NV / 2; w >= 1; w >>= 1) {
+                const bool up = (lane & (2 * w)) != 0;
+#pragma unroll
+                for (int i = 0; i < w; ++i) {
+                    const float send = up ? sums[i] : sums[i + w];
+                    const float keep = up ? sums[i + w] : sums[i];
+                    sums[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2 * w);
+                }
+            }
+            sums[0] += __shfl_xor_sync(0xffffffffu, sums[0], 1);
+#pragma unroll
+            for (int o = 2 * NV; o < 32; o <<= 1) sums[0] += __shfl_xor_sync(0xffffffffu, sums[0], o);
+            if (lane < 2 * NV && (lane & 1) == 0) misc->red[2 + quad][c0 + (lane >> 1)] = sums[0];
+        }
+        softmax_sync();
+        if (ok && quad == 0 && lane < NV) {
+            const int h = c0 + lane;
             float* ml = p.part_ml + (((int64_t)seg * p.nchunk + chunk) * H + h_base + h) * 2;
-            ml[0] = m;
-            ml[1] = l;
+            ml[0] = fmaxf(misc->red[0][h], misc->red[1][h]);
+            ml[1] = misc->red[2][h] + misc->red[3][h];
         }
     }
 
-    // ---- unnormalised partial output, [d][head], slab by slab as the MMA warp
-    // finishes them (lane = d within the slab; each warpgroup takes one half
-    // of the group's heads; 16-byte stores)
-    {
-        float* po = p.part_o + ((int64_t)seg * p.nchunk + chunk) * H * D + h_base;
-        for (int s2 = 0; s2 < D / 128; ++s2) {
-            ok = tc::mbar_wait(&misc->o_bar[s2], 0) && ok;
+    // ---- O^T = V^T P^T: M = 128 channels per slab (two K blocks, MN-major),
+    // N = HG, K = 64 positions; issuer i takes slabs i, i + kIssuers, ..
+    if (issues) {
+        bool pok = iss_ok && tc::mbar_wait(&misc->p_bar, 0);
+        if (pok) {
             tc::fence_after_sync();
-            if (!ok) continue;
-            const int d = s2 * 128 + quad * 32 + lane;
-            const uint32_t tcol = trow + (uint32_t)(HG + s2 * HG);
-            if (hc == 8) {
-                float v[8];
-                tc::tmem_ld8(tcol + wgrp * 8, v);
-                float4* dst = reinterpret_cast<float4*>(po + (int64_t)d * H + wgrp * 8);
-                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-            } else {
-                for (int c0 = wgrp * hc; c0 < (wgrp + 1) * hc; c0 += 16) {
-                    float v[16];
-                    tc::tmem_ld16(tcol + c0, v);
-                    float4* dst = reinterpret_cast<float4*>(po + (int64_t)d * H + c0);
+            const uint32_t idesc2 = tc::idesc_f16_f32(128, HG, /*a_mn=*/true, /*b_mn=*/false);
+            const uint64_t dvt = tc::desc_mn_sw128(v0, kBlkBytes, 1024), dp = tc::desc_sw128(p0);
+            for (int s = issuer; s < D / 128; s += kIssuers)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                }
+                for (int ks = 0; ks < kRows / 16; ++ks)
+                    tc::mma_f16(tmem + (uint32_t)(kIssuers * HG + s * HG),
+                                tc::desc_at(dvt, (uint32_t)(2 * s) * kBlkBytes + ks * 2048u), tc::desc_at(dp, 32u * ks),
+                                idesc2, ks != 0);
+        }
+        tc::mma_commit(&misc->o_bar);
+        tc::mma_commit(&misc->drain_bar);
+    }
+
+    // ---- unnormalised partial output, [head][d]: warp w reads slab w / 4,
+    // TMEM lanes of its quad (lane = d within the slab); a warp's stores of
+    // one head are 32 consecutive floats
+    {
+        ok = tc::mbar_wait(&misc->o_bar, 0) && ok;
+        tc::fence_after_sync();
+        ok = __all_sync(0xffffffffu, ok);
+        const int s2 = warp >> 2;
+        if (ok && s2 < D / 128) {
+            const int d = s2 * 128 + quad * 32 + lane;
+            const uint32_t tcol = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(kIssuers * HG + s2 * HG);
+            float* po = p.part_o + (((int64_t)seg * p.nchunk + chunk) * H + h_base) * D + d;
+#pragma unroll
+            for (int c0 = 0; c0 < HG; c0 += 16) {
+                float v[16];
+                tc::tmem_ld16(tcol + c0, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) po[(int64_t)(c0 + i) * D] = v[i];
             }
         }
     }
     if (!ok) flag(p.status, kStatusTimeout);
-    if (!rows_ok) tc::mbar_wait(&misc->row_bar, 0);   // no row copy may land after the CTA has left
     tc::fence_before_sync();
-    __syncthreads();                                  // (2) TMEM is released by the MMA warp
+    __syncthreads();                                  // TMEM is released by the MMA warp
 }
 
-// Bytes of one row the kernel fetches: codes and scales, rounded up to the
-// 16-byte granule of a bulk copy (never past the row: the stride is a
-// multiple of 16 and at least D/2 + D/16).
-int attn_tc_row_bytes(int D) { return (D / 2 + D / 16 + 15) & ~15; }
-
-size_t attn_tc_smem(int D, int HG, uint32_t stage_bytes, uint32_t* off_q, uint32_t* off_stage, uint32_t* off_misc) {
-    const uint32_t v = (uint32_t)(D / 64) * kRows * 128;
-    const uint32_t qbytes = (uint32_t)(D / 64) * HG * 128;
-    const uint32_t pbytes = 2u * HG * 128;     // P, in the query's place once S is computed
-    const uint32_t qreg = ((qbytes > pbytes ? qbytes : pbytes) + 1023) & ~1023u;
+template <int HG>
+size_t attn_tc_smem(int D, uint32_t* off_q, uint32_t* off_p, uint32_t* off_misc) {
+    const uint32_t v = (uint32_t)(D / 64 + 1) * kBlkBytes;           // + one block read past the end by M = 128
+    const uint32_t qbytes = ((uint32_t)(D / 64) * HG * 128 + 1023) & ~1023u;
+    const uint32_t pbytes = ((uint32_t)HG * 128 + 1023) & ~1023u;
     *off_q = v;
-    *off_stage = (v - stage_bytes) & ~1023u;   // the tail of the V tile: rows land there before the tile is written
-    *off_misc = v + qreg;
-    return (size_t)v + qreg + sizeof(Misc) + 1024;
+    *off_p = v + qbytes;
+    *off_misc = v + qbytes + pbytes;
+    return (size_t)v + qbytes + pbytes + sizeof(Misc<HG>) + 1024;
 }
 
-uint32_t attn_tc_stage_stride(int D) {
-    const uint32_t rb = (uint32_t)attn_tc_row_bytes(D);
-    return ((rb / 16) & 1) ? rb : rb + 16;
+template <int HG>
+cudaError_t launch_hg(const DevCache& c, const Params& p0, int nseg, cudaStream_t st) {
+    Params p = p0;
+    uint32_t cols = 32;
+    while (cols < (uint32_t)(kIssuers * HG + (c.dim / 128) * HG)) cols <<= 1;
+    p.tmem_cols = cols;
+    const size_t smem = attn_tc_smem<HG>(c.dim, &p.off_q, &p.off_p, &p.off_misc);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<HG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_attn_tc<HG>, dim3((unsigned)p.nchunk, (unsigned)nseg, (unsigned)(p.H / HG)), dim3(kThreads),
+                      smem, st, p);
 }
 
 }  // namespace
@@ -470,7 +466,7 @@ uint32_t attn_tc_stage_stride(int D) {
 bool attn_tc_supported(const DevCache& c, int H) {
     uint32_t a, b, d;
     return c.dim % 128 == 0 && c.dim <= 512 && (H == 16 || H == 32 || H == 64) &&
-           attn_tc_smem(c.dim, H, kRows * attn_tc_stage_stride(c.dim), &a, &b, &d) <= 227 * 1024;
+           attn_tc_smem<64>(c.dim, &a, &b, &d) <= 227 * 1024;
 }
 
 int attn_tc_rows_per_chunk() { return kRows; }
@@ -490,7 +486,6 @@ cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, 
     p.topk = topk;
     p.T = T;
     p.H = H;
-    p.HG = attn_tc_heads_per_cta(H, aw.nchunk, c.batch * T, num_sms);
     p.top_k = top_k;
     p.window = window;
     p.nchunk = aw.nchunk;
@@ -498,16 +493,11 @@ cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, 
     p.part_o = aw.part_o;
     p.part_ml = aw.part_ml;
     p.status = status;
-    p.row_bytes = (uint32_t)attn_tc_row_bytes(c.dim);
-    p.stage_stride = attn_tc_stage_stride(c.dim);
-    uint32_t cols = 32;
-    while (cols < (uint32_t)(p.HG + (c.dim / 128) * p.HG)) cols <<= 1;
-    p.tmem_cols = cols;
-    const size_t smem = attn_tc_smem(c.dim, p.HG, kRows * p.stage_stride, &p.off_q, &p.off_stage, &p.off_misc);
-    cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(k_attn_tc, dim3((unsigned)aw.nchunk, (unsigned)(c.batch * T), (unsigned)(H / p.HG)),
-                      dim3(kThreads), smem, st, p);
+    const int nseg = c.batch * T;
+    const int hg = attn_tc_heads_per_cta(H, aw.nchunk, nseg, num_sms);
+    if (hg == 16) return launch_hg<16>(c, p, nseg, st);
+    if (hg == 32) return launch_hg<32>(c, p, nseg, st);
+    return launch_hg<64>(c, p, nseg, st);
 }
 
 }  // namespace csa2

@@ -150,6 +150,11 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The score an ordered key came from (-0 comes back as +0).
+__device__ __forceinline__ float key_score(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 // Selection key of a score: 0 (never selected) for an element that is not a
 // candidate or whose score is NaN -- the mark a scorer leaves on a position it
 // had to skip (a page id outside the cache) -- else the ordered key, which is

@@ -246,6 +246,7 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
     } else if (warp == kWarpMma) {
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_f8_f32(kTile, NA, 0u, 0u);
+            const uint64_t dring = tc::desc_sw64(tc::smem_u32(sRing));
             uint32_t g = 0, n = 0;
             int cur_b = -1;
             bool ok = true;
@@ -257,16 +258,16 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                     cur_b = it.b;
                     if (!tc::mbar_wait(&bars->b_ready[n & 1], (n >> 1) & 1)) { ok = false; break; }
                 }
-                const uint32_t bq = tc::smem_u32(sB + (n & 1) * bq_bytes);
+                const uint64_t db = tc::desc_sw64(tc::smem_u32(sB + (n & 1) * bq_bytes));
                 for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                     const int s = g % kStages, acc = g & 1;
                     if (!tc::mbar_wait(&bars->full[s], (g / kStages) & 1) ||
                         !tc::mbar_wait(&bars->acc_empty[acc], ((g >> 1) & 1) ^ 1)) { ok = false; break; }
                     tc::fence_after_sync();
-                    const uint32_t aa = tc::smem_u32(sRing + s * kStageBytes);
+                    const uint64_t da = tc::desc_at(dring, (uint32_t)s * kStageBytes);
                     const uint32_t d = tmem + (uint32_t)(acc * NA);
-                    tc::mma_f8(d, tc::desc_sw64(aa), tc::desc_sw64(bq), idesc, 0u);
-                    tc::mma_f8(d, tc::desc_sw64(aa + 32), tc::desc_sw64(bq + 32), idesc, 1u);
+                    tc::mma_f8(d, da, db, idesc, 0u);
+                    tc::mma_f8(d, tc::desc_at(da, 32), tc::desc_at(db, 32), idesc, 1u);
                     tc::mma_commit(&bars->acc_full[acc]);
                 }
             }

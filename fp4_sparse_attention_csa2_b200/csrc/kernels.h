@@ -53,6 +53,15 @@ bool score_full_tc_supported(const DevCache& c, int T, int H_I);
 cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* hw, int T, int H_I, float* scores,
                                  uint32_t* hist, uint32_t* status, cudaStream_t st, int num_sms);
 
+// Reindex on the tensor cores (E4M3 keys, bf16 queries): pool rescoring into
+// scores[seg * pool_k + i] (NaN for entries that are not candidates) and the
+// top_k of each segment's pool, in one kernel; counters[seg] are zero on entry
+// and on exit.
+bool reindex_tc_supported(const DevCache& c, int H_I);
+cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw, int T, int H_I,
+                              const int32_t* pool, int pool_k, int top_k, int32_t* topk, float* scores,
+                              uint32_t* counters, uint32_t* status, cudaStream_t st);
+
 // Pool rescoring: scores[seg * pool_k + i] for pool entry i of segment seg.
 cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
                               const int32_t* pool, int pool_k, float* scores, uint32_t* status, cudaStream_t st);
@@ -63,6 +72,11 @@ cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const
 // receives the score of every selected element at the same index.
 cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_out, int32_t* out,
                           int64_t out_stride, cudaStream_t st, bool hist_ready = false, float* out_vals = nullptr);
+// One CTA per segment of at most 16,384 elements: the n_a best into out_a
+// (scores into vals_a, nullable) and, with n_b > 0, the n_b best of those
+// into out_b (a subset of out_a).
+cudaError_t launch_select_local(const SelSrc& src, int nseg, int n_a, int32_t* out_a, float* vals_a, int64_t stride_a,
+                                int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st);
 // Two selections of the same segments (more than 16,384 elements each): the
 // n_a best into out_a (scores into vals_a, nullable) and the n_b <= n_a best
 // into out_b (n_b == 0: none), out_b a subset of out_a.

@@ -17,8 +17,9 @@
 namespace csa2 {
 namespace {
 
-// 4 MiB of scratch: 256 bytes of header (status word) followed by the rescored
-// pool, so batch * T * pool_k may not exceed (4 MiB - 256) / 4 = 1,048,512.
+// 4 MiB of scratch: 256 bytes of header (the status word), the per-segment
+// arrival counters of the fused Reindex kernel (rounded up to 256 bytes),
+// then the rescored pool: batch * T * pool_k floats.
 constexpr size_t kScratchBytes = (size_t)4 << 20;
 constexpr size_t kScratchHeader = 256;
 constexpr int kMaxContexts = 64;
@@ -97,20 +98,29 @@ extern "C" csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const
     // csa2_index_reindex; only then the bound of the fixed scratch
     csa2_status s = check_reindex_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx);
     if (s != CSA2_OK) return s;
-    const size_t need = kScratchHeader + sizeof(float) * (size_t)cache->batch * T * pool_k;
+    const size_t nseg = (size_t)cache->batch * T;
+    const size_t cnt_bytes = (sizeof(uint32_t) * nseg + 255) / 256 * 256;
+    const size_t need = kScratchHeader + cnt_bytes + sizeof(float) * nseg * pool_k;
     if (need > kScratchBytes) return CSA2_ERR_UNSUPPORTED;
 
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return CSA2_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint32_t* status = static_cast<uint32_t*>(scratch);
-    float* scores = reinterpret_cast<float*>(static_cast<char*>(scratch) + kScratchHeader);
-    // the status word must start at zero; the scorer writes a score for every
-    // pool entry (a NaN marks one it rejected), so nothing stale from an
-    // earlier call is read
-    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return CSA2_ERR_CUDA;
+    uint32_t* counters = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + kScratchHeader);
+    float* scores = reinterpret_cast<float*>(static_cast<char*>(scratch) + kScratchHeader + cnt_bytes);
+    // the status word and the counters must start at zero (a call cut short
+    // could have left them set); the scorer writes a score for every pool
+    // entry (a NaN marks one it rejected), so nothing stale from an earlier
+    // call is read
+    if (cudaMemsetAsync(status, 0, kScratchHeader + cnt_bytes, st) != cudaSuccess) return CSA2_ERR_CUDA;
 
     const DevCache d = dev_cache(cache);
+    if (reindex_tc_supported(d, H_I)) {
+        const cudaError_t e = launch_reindex_tc(d, q_idx, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx, scores,
+                                                counters, status, st);
+        return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+    }
     cudaError_t e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, pool_idx, pool_k, scores, status,
                                       st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
@@ -124,7 +134,7 @@ extern "C" csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const
     src.seq_lens = cache->seq_lens;
     src.T = T;
     src.cap = d.cap;
-    SelWork unused = {};   // a pool-sized selection runs in one cluster per segment, in shared memory
-    e = launch_select(src, unused, cache->batch * T, top_k, topk_idx, top_k, st, false);
+    // a pool-sized selection runs in one CTA per segment, in shared memory and registers
+    e = launch_select_local(src, (int)nseg, top_k, topk_idx, nullptr, top_k, 0, nullptr, 0, st);
     return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

@@ -109,6 +109,16 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
+// Shared-memory descriptors advance by a byte offset (a multiple of 16) with
+// one add to their start-address field (bits 0..13, in 16-byte units): the
+// descriptor of a tile is built once and every K step or K block is an
+// offset from it, which keeps the issuing thread's per-MMA work to a few
+// instructions (building a descriptor from scratch is a chain of 64-bit
+// operations, and one thread issues every MMA of the CTA).
+__device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t byte_offset) {
+    return desc + (uint64_t)(byte_offset >> 4);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, kind::f16, issued by one thread.
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate) {

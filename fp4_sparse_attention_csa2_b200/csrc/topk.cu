@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "lsel.cuh"
 
 namespace csa2 {
 
@@ -942,13 +943,106 @@ k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, float* __restrict_
     cl.sync();   // no CTA leaves while another may still read its shared memory
 }
 
+// ---------------------------------------------------------------- one CTA per segment
+// Whole selection of one segment of at most 1024 * E elements by one CTA
+// (lsel.cuh): the n_a best into out_a (scores into vals_a, nullable) and,
+// with n_b > 0, the n_b best of those into out_b (a subset of out_a).
+// Element i has value vals[seg * vals_stride + i] and id ids[seg *
+// ids_stride + i] (ids == nullptr: id i, valid for i <= p); VEC: the value
+// and id rows are 16-byte aligned, so four consecutive elements are one load.
+constexpr int kLocalThreads = 1024;
+
+template <int E, bool VEC>
+__global__ void __launch_bounds__(kLocalThreads)
+k_sel_local(SelSrc src, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a, int n_b,
+            int32_t* __restrict__ out_b, int64_t stride_b) {
+    __shared__ lsel::Smem<kLocalThreads> sh;
+    extern __shared__ int32_t s_ids[];               // [1024 * E] when the ids come from memory
+    pdl_begin();
+    const int seg = blockIdx.x;
+    const int64_t nvalid = n_valid_positions(src, seg);
+    const int64_t n = src.ids ? src.n : (src.n < nvalid ? src.n : nvalid);
+    const float* vrow = src.vals + seg * src.vals_stride;
+    const int32_t* irow = src.ids ? src.ids + seg * src.ids_stride : nullptr;
+    uint32_t key[E];
+    int32_t idv[E];
+    // every load issued before any is used (indices clamped to the rows'
+    // allocated length so that no load is conditional; elements at or beyond
+    // n are masked afterwards)
+    const int64_t row_len = irow && src.ids_stride < src.vals_stride ? src.ids_stride : src.vals_stride;
+#pragma unroll
+    for (int g = 0; g < (E + 3) / 4; ++g) {
+        const int i0 = lsel::elem_index<kLocalThreads, E>(4 * g);
+        if (VEC && E % 4 == 0) {
+            const int ic = i0 + 3 < row_len ? i0 : 0;
+            const uint4 v = *reinterpret_cast<const uint4*>(vrow + ic);
+            key[4 * g] = v.x; key[4 * g + 1] = v.y; key[4 * g + 2] = v.z; key[4 * g + 3] = v.w;
+            if (irow) {
+                const int4 d = *reinterpret_cast<const int4*>(irow + ic);
+                idv[4 * g] = d.x; idv[4 * g + 1] = d.y; idv[4 * g + 2] = d.z; idv[4 * g + 3] = d.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (4 * g + k >= E) break;
+                const int i = lsel::elem_index<kLocalThreads, E>(4 * g + k);
+                const int ic = i < row_len ? i : 0;
+                key[4 * g + k] = __float_as_uint(vrow[ic]);
+                if (irow) idv[4 * g + k] = irow[ic];
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int i = lsel::elem_index<kLocalThreads, E>(e);
+        int32_t id = irow ? idv[e] : i;
+        if (i >= n) id = -1;
+        key[e] = select_key(__uint_as_float(key[e]), id >= 0 && id < nvalid);
+        if (irow) s_ids[e * kLocalThreads + threadIdx.x] = id;   // parked in shared memory until the output
+    }
+    auto id_of = [&](int e) -> int32_t {
+        return irow ? s_ids[e * kLocalThreads + threadIdx.x] : lsel::elem_index<kLocalThreads, E>(e);
+    };
+    const uint32_t ta = lsel::select_mask<kLocalThreads, E>(key, (uint32_t)n_a, sh);
+    lsel::write_selected<kLocalThreads, E>(ta, key, id_of, out_a + (int64_t)seg * stride_a,
+                                           vals_a ? vals_a + (int64_t)seg * stride_a : nullptr, n_a, sh);
+    if (n_b > 0) {
+        // the second target chooses among the first one's picks only
+#pragma unroll
+        for (int e = 0; e < E; ++e) key[e] = ((ta >> e) & 1u) ? key[e] : 0u;
+        const uint32_t tb = lsel::select_mask<kLocalThreads, E>(key, (uint32_t)n_b, sh);
+        lsel::write_selected<kLocalThreads, E>(tb, key, id_of, out_b + (int64_t)seg * stride_b, nullptr, n_b, sh);
+    }
+}
+
+template <int E>
+cudaError_t launch_local_e(const SelSrc& src, int nseg, int n_a, int32_t* out_a, float* vals_a, int64_t stride_a,
+                           int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st) {
+    const bool vec = (reinterpret_cast<uintptr_t>(src.vals) & 15u) == 0 && src.vals_stride % 4 == 0 &&
+                     (!src.ids || ((reinterpret_cast<uintptr_t>(src.ids) & 15u) == 0 && src.ids_stride % 4 == 0));
+    const size_t smem = src.ids ? sizeof(int32_t) * kLocalThreads * E : 0;
+    auto kern = vec ? k_sel_local<E, true> : k_sel_local<E, false>;
+    if (smem > 48 * 1024 - sizeof(lsel::Smem<kLocalThreads>)) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(kern, dim3((unsigned)nseg), dim3(kLocalThreads), smem, st, src, n_a, out_a, vals_a, stride_a,
+                      n_b, out_b, stride_b);
+}
+
 }  // namespace
+
+cudaError_t launch_select_local(const SelSrc& src, int nseg, int n_a, int32_t* out_a, float* vals_a, int64_t stride_a,
+                                int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st) {
+    if (src.n <= 1024) return launch_local_e<1>(src, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st);
+    if (src.n <= 4096) return launch_local_e<4>(src, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st);
+    return launch_local_e<16>(src, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st);
+}
 
 cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_out, int32_t* out,
                           int64_t out_stride, cudaStream_t st, bool hist_ready, float* out_vals) {
     if (src.n <= kSmallMax)
-        return launch_pdl_cluster(k_sel_small, dim3(kClCtas, (unsigned)nseg), dim3(kClThreads), 0, st, kClCtas, src,
-                                  n_out, out, out_vals, out_stride);
+        return launch_select_local(src, nseg, n_out, out, out_vals, out_stride, 0, nullptr, 0, st);
     return launch_select_dual(src, wk, nseg, n_out, out, out_vals, out_stride, 0, nullptr, 0, st, hist_ready);
 }
 

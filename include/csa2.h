@@ -192,17 +192,22 @@ CSA2_API csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_i
  * paths that cannot pay for cudaMalloc's implicit synchronisation.  The pages
  * describe no such call; it is a convenience of this library.
  *
- * Same arguments and results as csa2_index_reindex, minus ws / ws_bytes.  The
- * scratch lives in a 4 MiB array inside the library's own device memory (held
- * by every GPU that loads the library until the process exits), so
- * batch * T * pool_k must not exceed 1,048,512; larger problems return
- * CSA2_ERR_UNSUPPORTED before anything is launched.  The first call on a
- * device looks up that array's device address (cudaGetSymbolAddress, with the
- * device current), so make the first call on each device before any stream
- * capture.  Every call on a device shares the one array: calls whose work may
- * overlap on the GPU (different streams without ordering between them) race
- * and must not be issued.  Device-detected bound violations are skipped; this
- * variant has no status word the caller can read.
+ * Same arguments, argument checks and results as csa2_index_reindex, minus
+ * ws / ws_bytes.  The scratch lives in a 4 MiB array inside the library's own
+ * device memory (held by every GPU that loads the library until the process
+ * exits): 256 bytes of status word, one 4-byte counter per (sequence, token)
+ * rounded up to 256 bytes, and batch * T * pool_k floats must fit in it
+ * (e.g. batch * T * pool_k <= 1,048,448 while batch * T <= 64); larger
+ * problems return CSA2_ERR_UNSUPPORTED before anything is launched, after the
+ * other argument checks.  The first call in a CUDA context looks up that
+ * array's device address in that context (cudaGetSymbolAddress), so make the
+ * first call on each device before any stream capture; a new context (e.g.
+ * after cudaDeviceReset) gets a fresh lookup.  Every call on a device shares
+ * the one array, and each call clears its status word and counters with an
+ * asynchronous memset on `stream`: calls whose work may overlap on the GPU
+ * (different streams without ordering between them) race and must not be
+ * issued.  Device-detected bound violations are skipped; this variant has no
+ * status word the caller can read.
  */
 CSA2_API csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
                                                 const float* head_w, int T, int H_I, const int32_t* pool_idx,
@@ -219,12 +224,7 @@ CSA2_API csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const v
  *     out   = sum_{t in S} softmax(z)_t v_t        fp32 [batch][T][H][dim]
  *     lse   = log sum_{t in S} exp(z_t)            fp32 [batch][T][H], nullable
  * q is bf16 [batch][T][H][dim] with H a multiple of 16, at most 64.  An empty
- * S gives out = 0, lse = -inf.  top_k and window are each at most 16,384;
- * CSA2_ERR_UNSUPPORTED when the split-softmax merge's weights (one float per
- * (chunk, head); chunks of 128 entries on the tensor-core path -- dim a
- * multiple of 128 and H in {16, 32, 64} -- else of 32) would not fit in
- * 200 KiB of shared memory, e.g. H = 64 with window + top_k above 24,864 on
- * the 32-entry path.
+ * S gives out = 0, lse = -inf.  top_k and window are each at most 16,384.
  * topk entries < -1 or >= seq_lens[b] set CSA2_ERR_DEVICE_BOUNDS.
  */
 CSA2_API csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, int T, int H,

@@ -104,13 +104,7 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         csa2.lib()
 
 
-def test_attention_merge_limit_rejected_on_host(lib):
-    # the CUDA-core path (dim not a multiple of 128) merges 32-entry chunks:
-    # 64 heads x (16,384 + 16,384) / 32 chunk weights exceed its 200 KiB of
-    # shared memory, so the call is refused before any launch
-    c = fake_cache(dim=96, row_stride=64)
-    assert lib.csa2_sparse_swa_attn(ctypes.byref(c), 0x40000, 1, 64, 0x60000, 16384, 16384, 0.0, 0x70000, None,
-                                    0x80000, 1 << 40, None) == csa2.ERR_UNSUPPORTED
+def test_attention_bounds_rejected_on_host(lib):
     # window or top-k beyond the 16,384 bound: invalid on any path
     c = fake_cache()
     assert lib.csa2_sparse_swa_attn(ctypes.byref(c), 0x40000, 1, 64, 0x60000, 2048, 16385, 0.0, 0x70000, None,
@@ -144,7 +138,7 @@ def test_noalloc_reindex_refuses_like_the_workspace_entry_point(lib):
     for cache, want in [(fake_cache(dim=1024), csa2.ERR_UNSUPPORTED), (fake_cache(idx_dim=32), csa2.ERR_UNSUPPORTED),
                         (fake_cache(row_stride=280), csa2.ERR_INVALID_ARG)]:
         assert both(cache=cache, T=8, pool_k=16384, top_k=16) == (want, want)
-    # beyond the fixed scratch (batch * T * pool_k > 1,048,512) once everything else is valid
+    # beyond the fixed scratch (80 x 16,384 pool scores > 4 MiB) once everything else is valid
     big = fake_cache(batch=80, seq_stride_slots=1 << 14, n_slots=80 << 14)
     assert lib.csa2_index_reindex_noalloc(ctypes.byref(big), 0x40000, csa2.BF16, 0x50000, 1, 32, 0x60000, 16384, 16,
                                           0x70000, None) == csa2.ERR_UNSUPPORTED
