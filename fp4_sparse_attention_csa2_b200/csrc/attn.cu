@@ -150,43 +150,38 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
     }
 }
 
-// Split-softmax merge.  One thread per output (head h, channel d) of one
-// (sequence, query token): with chunk c's partial output O_c[h][d] (not
-// normalised) and its per-head (m_c, l_c) in base-2 units,
+// Split-softmax merge.  Output (head h, channel d) of one (sequence, query
+// token): with chunk c's partial output O_c[h][d] (not normalised) and its
+// per-head (m_c, l_c) in base-2 units,
 //     M = max_c m_c,  L = sum_c 2^(m_c - M) l_c,  out = sum_c 2^(m_c - M) O_c / L,
-// lse = M ln 2 + ln L.  grid (batch*T, ceil(H*D / 256)), 256 threads; a warp's
-// loads of one chunk are 32 consecutive channels of one head, and every load
-// of a batch of kBatch chunks is issued before any is used (the merge runs
-// online over the batches).
-constexpr int kBatch = 24;
+// lse = M ln 2 + ln L.  G consecutive threads share an output, thread `part`
+// taking chunks part, part + G, ..; each thread issues all its loads at once
+// (up to kBatch; indices clamped, so no load is conditional) and the G shares
+// (M, L, acc) are combined by shuffles.  A warp's loads of one chunk are
+// consecutive channels of one head.  grid (batch*T, ceil(H*D*G / 256)).
+constexpr int kBatch = 18;
 
-__global__ void __launch_bounds__(256)
-k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk,
-               float* __restrict__ out, float* __restrict__ lse) {
-    pdl_begin();
-    const int seg = blockIdx.x;
-    const int i = blockIdx.y * 256 + threadIdx.x;
-    if (i >= H * D) return;
-    const int h = i / D, d = i - h * D;
-    const int64_t cs_o = (int64_t)H * D, cs_ml = (int64_t)H * 2;
-    const float* po = part_o + (int64_t)seg * nchunk * cs_o + (int64_t)h * D + d;
-    const float* ml = part_ml + (int64_t)seg * nchunk * cs_ml + (int64_t)h * 2;
-    float M = -INFINITY, Lsum = 0.0f, acc = 0.0f;
-    for (int c0 = 0; c0 < nchunk; c0 += kBatch) {
+__device__ __forceinline__ void merge_part(const float* po, const float* ml, int nchunk, int part, int G, int64_t cs_o,
+                                           int64_t cs_ml, float& M, float& Lsum, float& acc) {
+    M = -INFINITY;
+    Lsum = 0.0f;
+    acc = 0.0f;
+    for (int c0 = part; c0 < nchunk; c0 += kBatch * G) {
         float o[kBatch], m[kBatch], l[kBatch];
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) {
-            const bool in = c0 + k < nchunk;
-            const float2 v = in ? *reinterpret_cast<const float2*>(ml + (int64_t)(c0 + k) * cs_ml) : make_float2(-INFINITY, 0.0f);
-            m[k] = v.x;
+            const int ck = c0 + k * G;
+            const int c = ck < nchunk ? ck : part;
+            const float2 v = *reinterpret_cast<const float2*>(ml + (int64_t)c * cs_ml);
+            o[k] = po[(int64_t)c * cs_o];
+            m[k] = ck < nchunk ? v.x : -INFINITY;
             l[k] = v.y;
-            o[k] = in ? po[(int64_t)(c0 + k) * cs_o] : 0.0f;
         }
         float mb = M;
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) mb = fmaxf(mb, m[k]);
-        if (mb == -INFINITY) continue;                         // nothing attended so far
-        const float rs = M == -INFINITY ? 0.0f : exp2f(M - mb);   // rescale what came before
+        if (mb == -INFINITY) continue;                          // nothing attended so far
+        const float rs = M == -INFINITY ? 0.0f : exp2f(M - mb);
         acc *= rs;
         Lsum *= rs;
 #pragma unroll
@@ -197,8 +192,40 @@ k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __re
         }
         M = mb;
     }
-    out[((int64_t)seg * H + h) * D + d] = Lsum > 0.0f ? acc / Lsum : 0.0f;
-    if (lse && d == 0) lse[(int64_t)seg * H + h] = Lsum > 0.0f ? M * 0.6931471805599453f + logf(Lsum) : -INFINITY;
+}
+
+// Combine two shares (M, L, acc) of one output: both rescaled to the larger maximum.
+__device__ __forceinline__ void merge_pair(float& M, float& Lsum, float& acc, float M2, float L2, float a2) {
+    const float mb = fmaxf(M, M2);
+    if (mb == -INFINITY) return;
+    const float w1 = M == -INFINITY ? 0.0f : exp2f(M - mb), w2 = M2 == -INFINITY ? 0.0f : exp2f(M2 - mb);
+    acc = acc * w1 + a2 * w2;
+    Lsum = Lsum * w1 + L2 * w2;
+    M = mb;
+}
+
+__global__ void __launch_bounds__(256)
+k_attn_combine(int D, int H, const float* __restrict__ part_o, const float* __restrict__ part_ml, int nchunk, int G,
+               float* __restrict__ out, float* __restrict__ lse) {
+    pdl_begin();
+    const int seg = blockIdx.x;
+    const int t = blockIdx.y * 256 + threadIdx.x;
+    const int part = t % G;
+    const int nout = H * D;
+    const int o = t / G;
+    const int oc = o < nout ? o : nout - 1;                 // every lane takes part in the shuffles
+    const int h = oc / D, d = oc - h * D;
+    const int64_t cs_o = (int64_t)H * D, cs_ml = (int64_t)H * 2;
+    float M, Lsum, acc;
+    merge_part(part_o + (int64_t)seg * nchunk * cs_o + (int64_t)h * D + d,
+               part_ml + (int64_t)seg * nchunk * cs_ml + (int64_t)h * 2, nchunk, part, G, cs_o, cs_ml, M, Lsum, acc);
+    for (int x = 1; x < G; x <<= 1)
+        merge_pair(M, Lsum, acc, __shfl_xor_sync(0xffffffffu, M, x), __shfl_xor_sync(0xffffffffu, Lsum, x),
+                   __shfl_xor_sync(0xffffffffu, acc, x));
+    if (o < nout && part == 0) {
+        out[((int64_t)seg * H + h) * D + d] = Lsum > 0.0f ? acc / Lsum : 0.0f;
+        if (lse && d == 0) lse[(int64_t)seg * H + h] = Lsum > 0.0f ? M * 0.6931471805599453f + logf(Lsum) : -INFINITY;
+    }
 }
 
 }  // namespace
@@ -208,9 +235,12 @@ int attn_rows_per_chunk() { return kRows; }
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st) {
     const int64_t nseg = (int64_t)c.batch * T;
-    const unsigned blocks = (unsigned)((H * c.dim + 255) / 256);
+    // threads per output: enough that each thread's chunks are one batch of loads
+    int G = 1;
+    while (G < 32 && aw.nchunk > kBatch * G) G <<= 1;
+    const unsigned blocks = (unsigned)(((int64_t)H * c.dim * G + 255) / 256);
     return launch_pdl(k_attn_combine, dim3((unsigned)nseg, blocks), dim3(256), 0, st, c.dim, H, aw.part_o, aw.part_ml,
-                      aw.nchunk, out, lse);
+                      aw.nchunk, G, out, lse);
 }
 
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,

@@ -119,3 +119,63 @@ def new_workspace(cache, w):
                      device="cuda")
     csa2.workspace_init(ws)
     return ws
+
+
+class E2ERunner:
+    """Decode steps end to end through the public binding, as a serving loop
+    would run them: every step's inputs are copied from pinned host memory and
+    every step's outputs read back into pinned host memory, while the kernels
+    of a step are one CUDA-graph replay.  Two Stacks (two sets of device input
+    and output buffers) alternate, so step i + 1's inputs are on their way in
+    and step i - 1's outputs on their way out while step i computes: the
+    host-to-device copies run on one side stream, the device-to-host copies on
+    another, ordered against the compute stream by events."""
+
+    def __init__(self, w, layers, ws, reps, stream):
+        self.w, self.reps, self.stream = w, reps, stream
+        self.stacks = [Stack(w, layers, ws), Stack(w, layers, ws)]
+        self.h2d = torch.cuda.Stream()
+        self.d2h = torch.cuda.Stream()
+        self.graphs = {}
+        for s, st in enumerate(self.stacks):
+            for r, c in enumerate(reps):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                    st.step(c)
+                self.graphs[(r, s)] = g
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_done = [torch.cuda.Event() for _ in range(2)]
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def bytes_per_step(self):
+        st = self.stacks[0]
+        return st.inputs.numel(), st.outputs.numel()
+
+    def run(self, host_in, host_outs, n, t0=None, t1=None):
+        """n steps; host_in: pinned uint8 copy of a Stack's inputs; host_outs:
+        two pinned uint8 buffers the outputs alternate into.  t0 / t1
+        (optional CUDA events) are recorded before the first copy and after
+        the last read-back."""
+        if t0 is not None:
+            t0.record(self.h2d)
+        for i in range(n):
+            s = i % 2
+            st = self.stacks[s]
+            with torch.cuda.stream(self.h2d):
+                if i >= 2:
+                    self.h2d.wait_event(self.ev_done[s])          # step i - 2 no longer reads these inputs
+                st.inputs.copy_(host_in, non_blocking=True)
+                self.ev_in[s].record(self.h2d)
+            self.stream.wait_event(self.ev_in[s])
+            if i >= 2:
+                self.stream.wait_event(self.ev_out[s])            # step i - 2's outputs have left the device
+            with torch.cuda.stream(self.stream):
+                self.graphs[(i % len(self.reps), s)].replay()
+            self.ev_done[s].record(self.stream)
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(self.ev_done[s])
+                host_outs[s].copy_(st.outputs, non_blocking=True)
+                self.ev_out[s].record(self.d2h)
+        if t1 is not None:
+            self.d2h.wait_stream(self.stream)
+            t1.record(self.d2h)
