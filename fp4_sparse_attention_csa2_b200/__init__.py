@@ -21,7 +21,7 @@ F32, BF16, E4M3 = 0, 1, 2
 ABI_FUNCTIONS = (
     "csa2_workspace_bytes", "csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
     "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_sparse_swa_attn", "csa2_layer_step",
-    "csa2_read_device_status", "csa2_status_string",
+    "csa2_read_device_status", "csa2_status_string", "csa2_debug_set_wait_limit", "csa2_debug_default_wait_limit",
 )
 
 
@@ -76,9 +76,13 @@ def lib():
         L.csa2_read_device_status.argtypes = [vp, vp]
         L.csa2_status_string.restype = ctypes.c_char_p
         L.csa2_status_string.argtypes = [i32]
+        L.csa2_debug_set_wait_limit.argtypes = [ctypes.c_uint32]
+        L.csa2_debug_default_wait_limit.restype = ctypes.c_uint32
+        L.csa2_debug_default_wait_limit.argtypes = []
         for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
                      "csa2_index_reindex", "csa2_index_reindex_noalloc",
-                     "csa2_sparse_swa_attn", "csa2_layer_step", "csa2_read_device_status"):
+                     "csa2_sparse_swa_attn", "csa2_layer_step", "csa2_read_device_status",
+                     "csa2_debug_set_wait_limit"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -245,3 +249,13 @@ def layer_step(cache, mode, q, topk_idx, out, ws, window, q_idx=None, head_w=Non
 def read_device_status(ws, stream=None):
     """Synchronise and return (then clear) the sticky device status code."""
     return lib().csa2_read_device_status(_p(ws), _stream(stream))
+
+
+def debug_set_wait_limit(tries=None):
+    """Diagnostic: tries of the bounded waits that guard work in the tensor-core
+    kernels launched from now on (None restores the default; 0 makes them give
+    up at once and record TIMEOUT).  Returns the default."""
+    L = lib()
+    default = int(L.csa2_debug_default_wait_limit())
+    _check(L.csa2_debug_set_wait_limit(default if tries is None else int(tries)), "debug_set_wait_limit")
+    return default

@@ -2,14 +2,22 @@
 // kernel dispatch.  Every entry point validates on the host, then only
 // enqueues work on the caller's stream.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
 #include "../../include/csa2.h"
 #include "abi_checks.h"
 #include "kernels.h"
+#include "tc.cuh"
 
 using namespace csa2;
+
+namespace {
+std::atomic<uint32_t> g_wait_limit{tc::kWaitLimit};
+}  // namespace
+
+uint32_t csa2::wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
 
 namespace {
 
@@ -347,6 +355,13 @@ csa2_status csa2_read_device_status(void* ws, void* stream) {
     if (word & kStatusBounds) return CSA2_ERR_DEVICE_BOUNDS;
     return CSA2_OK;
 }
+
+csa2_status csa2_debug_set_wait_limit(uint32_t tries) {
+    g_wait_limit.store(tries ? tries : 0u, std::memory_order_relaxed);
+    return CSA2_OK;
+}
+
+uint32_t csa2_debug_default_wait_limit(void) { return tc::kWaitLimit; }
 
 const char* csa2_status_string(csa2_status s) {
     switch (s) {

@@ -55,6 +55,7 @@ struct Params {
     float* part_o;            // [seg][chunk][H][D]
     float* part_ml;           // [seg][chunk][H][2]
     uint32_t* status;
+    uint32_t wait_limit;      // tries of the waits that guard work (not of the drain)
     uint32_t off_q, off_p, off_misc, tmem_cols;
 };
 
@@ -275,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     const uint32_t v0 = tc::smem_u32(sV), q0 = tc::smem_u32(sQ), p0 = tc::smem_u32(sP);
     bool iss_ok = true;
     if (issues) {
-        iss_ok = tc::mbar_wait(&misc->vq_bar, 0);
+        iss_ok = tc::mbar_wait(&misc->vq_bar, 0, p.wait_limit);
         if (iss_ok) {
             tc::fence_after_sync();
             const uint32_t idesc1 = tc::idesc_f16_f32(128, HG);
@@ -305,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     const bool smx = quad < 2;
     // (every worker's writes before its vq_bar arrival -- the per-head
     // factors among them -- are visible once that phase is seen complete)
-    bool ok = tc::mbar_wait(&misc->vq_bar, 0);
-    ok = tc::mbar_wait(&misc->s_bar, 0) && ok;
+    bool ok = tc::mbar_wait(&misc->vq_bar, 0, p.wait_limit);
+    ok = tc::mbar_wait(&misc->s_bar, 0, p.wait_limit) && ok;
     tc::fence_after_sync();
     ok = __all_sync(0xffffffffu, ok);                // warp-uniform from here on
     if (smx) {
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     // ---- O^T = V^T P^T: M = 128 channels per slab (two K blocks, MN-major),
     // N = HG, K = 64 positions; issuer i takes slabs i, i + kIssuers, ..
     if (issues) {
-        bool pok = iss_ok && tc::mbar_wait(&misc->p_bar, 0);
+        bool pok = iss_ok && tc::mbar_wait(&misc->p_bar, 0, p.wait_limit);
         if (pok) {
             tc::fence_after_sync();
             const uint32_t idesc2 = tc::idesc_f16_f32(128, HG, /*a_mn=*/true, /*b_mn=*/false);
@@ -415,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     // TMEM lanes of its quad (lane = d within the slab); a warp's stores of
     // one head are 32 consecutive floats
     {
-        ok = tc::mbar_wait(&misc->o_bar, 0) && ok;
+        ok = tc::mbar_wait(&misc->o_bar, 0, p.wait_limit) && ok;
         tc::fence_after_sync();
         ok = __all_sync(0xffffffffu, ok);
         const int s2 = warp >> 2;
@@ -493,6 +494,7 @@ cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, 
     p.part_o = aw.part_o;
     p.part_ml = aw.part_ml;
     p.status = status;
+    p.wait_limit = wait_limit();
     const int nseg = c.batch * T;
     const int hg = attn_tc_heads_per_cta(H, aw.nchunk, nseg, num_sms);
     if (hg == 16) return launch_hg<16>(c, p, nseg, st);

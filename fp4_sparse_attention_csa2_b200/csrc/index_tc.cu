@@ -60,6 +60,7 @@ struct Params {
     float* scores;           // [(b*T + j) * cap + t]
     uint32_t* hist;          // [(b*T + j)][3][kRadixBins]; level 1 accumulated here; nullable
     uint32_t* status;
+    uint32_t wait_limit;     // tries of the waits that guard work (not of the drains)
     int64_t items_per_seq, total_items;
     uint32_t tmem_cols;
     uint32_t off_b, off_hist, off_wq, off_bar;
@@ -213,7 +214,7 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                 if (!get_item(p, item, it)) continue;
                 for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                     const int s = g % kStages;
-                    if (!tc::mbar_wait(&bars->empty[s], ((g / kStages) & 1) ^ 1)) { ok = false; break; }
+                    if (!tc::mbar_wait(&bars->empty[s], ((g / kStages) & 1) ^ 1, p.wait_limit)) { ok = false; break; }
                     const int64_t t0 = it.t0 + (int64_t)tl * kTile;
                     int64_t slot[2] = {-1, -1};
                     uint32_t bytes = 0;
@@ -256,13 +257,13 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                 if (it.b != cur_b) {
                     if (cur_b >= 0) { tc::mma_commit(&bars->b_free[n & 1]); ++n; }
                     cur_b = it.b;
-                    if (!tc::mbar_wait(&bars->b_ready[n & 1], (n >> 1) & 1)) { ok = false; break; }
+                    if (!tc::mbar_wait(&bars->b_ready[n & 1], (n >> 1) & 1, p.wait_limit)) { ok = false; break; }
                 }
                 const uint64_t db = tc::desc_sw64(tc::smem_u32(sB + (n & 1) * bq_bytes));
                 for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
                     const int s = g % kStages, acc = g & 1;
-                    if (!tc::mbar_wait(&bars->full[s], (g / kStages) & 1) ||
-                        !tc::mbar_wait(&bars->acc_empty[acc], ((g >> 1) & 1) ^ 1)) { ok = false; break; }
+                    if (!tc::mbar_wait(&bars->full[s], (g / kStages) & 1, p.wait_limit) ||
+                        !tc::mbar_wait(&bars->acc_empty[acc], ((g >> 1) & 1) ^ 1, p.wait_limit)) { ok = false; break; }
                     tc::fence_after_sync();
                     const uint64_t da = tc::desc_at(dring, (uint32_t)s * kStageBytes);
                     const uint32_t d = tmem + (uint32_t)(acc * NA);
@@ -289,7 +290,7 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
         // epilogue threads meet on two mbarriers (bounded waits).
         auto flush = [&](int b) -> bool {
             tc::mbar_arrive(&bars->hist_done);
-            if (!tc::mbar_wait(&bars->hist_done, nflush & 1)) return false;
+            if (!tc::mbar_wait(&bars->hist_done, nflush & 1, p.wait_limit)) return false;
             if (p.hist) {
                 for (int j = 0; j < p.T; ++j) {
                     uint32_t* gh = p.hist + ((int64_t)b * p.T + j) * 3 * kRadixBins;
@@ -300,13 +301,13 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                 }
             }
             tc::mbar_arrive(&bars->hist_clear);
-            if (!tc::mbar_wait(&bars->hist_clear, nflush & 1)) return false;
+            if (!tc::mbar_wait(&bars->hist_clear, nflush & 1, p.wait_limit)) return false;
             ++nflush;
             return true;
         };
         // all lanes of a warp take the same decision before tcgen05.ld (.aligned)
         auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-            const bool got = tc::mbar_wait(bar, parity);
+            const bool got = tc::mbar_wait(bar, parity, p.wait_limit);
             return __all_sync(0xffffffffu, got);
         };
         const float* wq = sWq;
@@ -322,7 +323,7 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                 // stage this sequence's query operands once the MMAs of the
                 // sequence that used the buffer before are done
                 const int qb = n & 1;
-                if (!tc::mbar_wait(&bars->b_free[qb], ((n >> 1) & 1) ^ 1)) { ok = false; break; }
+                if (!tc::mbar_wait(&bars->b_free[qb], ((n >> 1) & 1) ^ 1, p.wait_limit)) { ok = false; break; }
                 if (grp == 0) prepare_queries(p, it.b, sB + qb * bq_bytes, sWq + qb * p.NP, tid);
                 tc::fence_proxy_async_smem();
                 tc::mbar_arrive(&bars->b_ready[qb]);
@@ -450,6 +451,7 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
     p.scores = scores;
     p.hist = hist;
     p.status = status;
+    p.wait_limit = wait_limit();
     const int64_t tiles_cap = (c.cap + kTile - 1) / kTile;
     p.items_per_seq = (tiles_cap + kItemTiles - 1) / kItemTiles;
     p.total_items = p.items_per_seq * c.batch;

@@ -8,6 +8,12 @@
 
 namespace csa2 {
 
+// Tries of the bounded mbarrier waits that guard work (not the drains that
+// wait for copies and MMAs already in flight) in the kernels launched from now
+// on; csa2_debug_set_wait_limit sets it (a diagnostic: 0 makes those waits
+// give up at once), the default is tc::kWaitLimit (about two seconds).
+uint32_t wait_limit();
+
 // Radix-select state of one workspace (see topk.cu).  Counts and histograms
 // are per segment (one segment = one (sequence, query token)).
 constexpr int kRadixBins = 2048;

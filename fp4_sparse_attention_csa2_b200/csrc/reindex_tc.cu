@@ -50,6 +50,7 @@ struct Params {
     float* scores;            // [B*T][pool_k] scratch
     uint32_t* counters;       // [B*T] arrival counters, zero between calls
     uint32_t* status;
+    uint32_t wait_limit;      // tries of the wait that guards the epilogue (not of the drain)
     uint32_t tmem_cols;
 };
 
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_reindex_tc(const Params p) {
     }
     bool ok = true;
     if (warp < 4) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm.mma_bar, 0));
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm.mma_bar, 0, p.wait_limit));
         tc::fence_after_sync();
         float s0 = 0.0f, s1 = 0.0f;
         if (ok) {
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_reindex_tc(const Params p) {
     if (warp == 0) {
         // after a wait that gave up, the MMA may still be running: wait for it
         // (again bounded) before the tensor memory is freed
-        if (!ok) tc::mbar_wait(&sm.mma_bar, 0);
+        if (!ok) tc::mbar_wait(&sm.mma_bar, 0, tc::kWaitLimit);
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, p.tmem_cols);
     }
@@ -274,6 +275,7 @@ cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw,
     p.scores = scores;
     p.counters = counters;
     p.status = status;
+    p.wait_limit = wait_limit();
     uint32_t cols = 32;
     while (cols < (uint32_t)(p.U * p.HP)) cols <<= 1;
     p.tmem_cols = cols;

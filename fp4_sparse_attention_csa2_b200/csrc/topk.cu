@@ -21,18 +21,14 @@
 //     survivors, and its last CTA resolves digit 3 and exact ties.  The pool
 //     and the layer's top-k are two targets of the same passes.
 //   small segments (<= 16,384: the top-k of a pool, and the pool of a Full
-//     layer over a short context): a cluster of 8 CTAs per segment keeps every
-//     key in registers and resolves all three digits, summing the CTAs'
-//     histograms through distributed shared memory.
-#include <cooperative_groups.h>
-
+//     layer over a short context): one CTA of 1,024 threads per segment
+//     brackets the cutoff from a sample, compacts the elements inside the
+//     bracket and resolves them by radix select in shared memory (lsel.cuh).
 #include "common.cuh"
 #include "kernels.h"
 #include "lsel.cuh"
 
 namespace csa2 {
-
-namespace cg = cooperative_groups;
 
 namespace {
 
@@ -223,68 +219,6 @@ __global__ void __launch_bounds__(kPassThreads) k_sel_hist(SelSrc src, SelWork w
     uint32_t* gh = wk.hist + (int64_t)seg * 3 * kRadixBins;
     for (int i = threadIdx.x; i < kRadixBins; i += kPassThreads)
         if (h[i]) atomicAdd(gh + i, h[i]);
-}
-
-// Cluster geometry shared by the pool-sized selection and the resolve kernel.
-constexpr int kClCtas = 8;
-constexpr int kClThreads = 512;
-constexpr int kClPer = kSmallMax / (kClCtas * kClThreads);   // elements per thread
-constexpr int kClBinsPer = kRadixBins / kClThreads;          // histogram bins per thread
-
-struct ClPlan {
-    uint32_t c, above, eq, total;
-};
-
-// Threshold of the cluster-wide histogram `h` (this CTA's copy; the others
-// are read through distributed shared memory).  need == 0 asks only for the
-// total (used at level 1, where `need` follows from it).
-__device__ __forceinline__ ClPlan cluster_threshold(cg::cluster_group& cl, uint32_t* h, uint32_t need_in,
-                                                    uint32_t n_out, uint32_t* s_wsum, ClPlan* s_plan) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // thread t owns bins hi - 3 .. hi, hi = 2047 - 4 t: descending bins follow ascending t
-    const int lo = kRadixBins - kClBinsPer * (tid + 1);
-    uint4 g = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int r = 0; r < kClCtas; ++r) {
-        const uint4 v = *reinterpret_cast<const uint4*>(cl.map_shared_rank(h + lo, r));
-        g.x += v.x; g.y += v.y; g.z += v.z; g.w += v.w;
-    }
-    const uint32_t sum = g.x + g.y + g.z + g.w;
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    uint32_t before = 0, total = 0;
-    for (int w = 0; w < kClThreads / 32; ++w) {
-        const uint32_t v = s_wsum[w];
-        before += w < warp ? v : 0u;
-        total += v;
-    }
-    const uint32_t need = need_in ? need_in : (total < n_out ? total : n_out);
-    const uint32_t excl = before + incl - sum;
-    if (need > 0 && excl < need && need <= excl + sum) {
-        const uint32_t b[4] = {g.w, g.z, g.y, g.x};   // bins lo + 3 .. lo, descending
-        uint32_t above = excl;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            if (need <= above + b[k]) {
-                s_plan->c = (uint32_t)(lo + 3 - k);
-                s_plan->above = above;
-                s_plan->eq = b[k];
-                break;
-            }
-            above += b[k];
-        }
-    }
-    if (tid == 0) s_plan->total = total;
-    __syncthreads();
-    const ClPlan pl = *s_plan;
-    __syncthreads();   // s_wsum and s_plan are rewritten by the next call
-    return pl;
 }
 
 // Two selections of the same scores at once: target a (the pool, n_a) and
@@ -567,13 +501,18 @@ k_sel_pass1(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float*
         __syncthreads();   // the stages are complete; the bases have been claimed
         {
             const uint32_t n0 = field16(tot, 0), n1 = field16(tot, 1), n2 = field16(tot, 2), n3 = field16(tot, 3);
+            // outputs stay inside their rows even when the level-1 histogram
+            // undercounts (a scoring kernel whose wait gave up; the status says so)
             for (uint32_t i = tid; i < n0; i += kPassThreads) {
                 const uint2 v = stage_a[i];
-                oa[s_base[0] + i] = (int32_t)v.x;
-                if (va) va[s_base[0] + i] = key_value(v.y);
+                const uint32_t o = s_base[0] + i;
+                if (o >= (uint32_t)n_a) break;
+                oa[o] = (int32_t)v.x;
+                if (va) va[o] = key_value(v.y);
             }
             for (uint32_t i = tid; i < n1; i += kPassThreads) cand_a[s_base[1] + i] = stage_a[kPassChunk - 1 - i];
-            for (uint32_t i = tid; i < n2; i += kPassThreads) ob[s_base[2] + i] = (int32_t)stage_b[i].x;
+            for (uint32_t i = tid; i < n2 && s_base[2] + i < (uint32_t)n_b; i += kPassThreads)
+                ob[s_base[2] + i] = (int32_t)stage_b[i].x;
             for (uint32_t i = tid; i < n3; i += kPassThreads) cand_b[s_base[3] + i] = stage_b[kPassChunk - 1 - i];
         }
         __syncthreads();   // s_base and the stages are rewritten by the next chunk
@@ -703,7 +642,7 @@ __device__ void finish_level3(const SelWork& wk, int seg, const Plan2& P, int32_
                 const uint32_t rk = u == 0 ? rk_a : rk_b;
                 const bool tk = on[u] && (d3 > r3[u].c || (eqv[u] && rk < ties[u]));
                 const uint32_t os = warp_claim(tk, cnt + (u == 0 ? 0 : 2));
-                if (tk) {
+                if (tk && (int64_t)os < (u == 0 ? stride_a : stride_b)) {
                     out[u][os] = (int32_t)kv.y;
                     if (u == 0 && va) va[os] = key_value(kv.x);
                 }
@@ -800,7 +739,8 @@ k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict_
         for (int t = 0; t < 2; ++t) {
             const uint2* stg = t == 0 ? stage_a : stage_b;
             const uint32_t nt = field16(tot, 2 * t), ns = field16(tot, 2 * t + 1);
-            for (uint32_t i = tid; i < nt; i += kPassThreads) {
+            const uint32_t cap = (uint32_t)(t == 0 ? n_a : n_b);
+            for (uint32_t i = tid; i < nt && s_base[2 * t] + i < cap; i += kPassThreads) {
                 const uint2 v = stg[i];
                 out[t][s_base[2 * t] + i] = (int32_t)v.y;
                 if (t == 0 && va) va[s_base[0] + i] = key_value(v.x);
@@ -821,126 +761,6 @@ k_sel_pass2(SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict_
     __shared__ uint32_t s_ctr[2];
     finish_level3<kPassThreads>(wk, seg, P, out_a, vals_a, stride_a, out_b, stride_b,
                                 reinterpret_cast<uint32_t*>(stage_dyn), s_wsum, s_thr, s_ctr);
-}
-
-// ---------------------------------------------------------------- small segments
-// Whole selection of one segment of at most kSmallMax elements by a cluster of
-// kClCtas CTAs.  Element i belongs to CTA (i / kClThreads) % kClCtas, which
-// keeps its key and id in registers.  Each level: every CTA histograms its own
-// elements of the current prefix in shared memory, one cluster barrier, then
-// every CTA sums the kClCtas histograms through distributed shared memory and
-// finds the same threshold digit; the following pass selects digits above it
-// and histograms the next digit of the elements equal to it.  Output slots and
-// exact-tie ranks are claimed on counters in CTA 0, once per CTA and digit.
-__global__ void __launch_bounds__(kClThreads)
-k_sel_small(SelSrc src, int n_out, int32_t* __restrict__ out, float* __restrict__ out_vals, int64_t out_stride) {
-    cg::cluster_group cl = cg::this_cluster();
-    __shared__ __align__(16) uint32_t hist[3][kRadixBins];
-    __shared__ uint32_t s_wsum[kClThreads / 32];
-    __shared__ uint64_t s_wsum64[kClThreads / 32];
-    __shared__ uint32_t s_base[2];
-    __shared__ ClPlan s_plan;
-    __shared__ uint32_t s_cnt[2];               // CTA 0's: output slots, exact-tie ranks
-    const uint32_t rank = cl.block_rank();
-    const int seg = blockIdx.y, tid = threadIdx.x;
-    for (int i = tid; i < 3 * kRadixBins; i += kClThreads) (&hist[0][0])[i] = 0;
-    if (tid < 2) s_cnt[tid] = 0;
-    pdl_begin();
-    const int n = (int)src.n;
-    const int64_t nvalid = n_valid_positions(src, seg);
-    int32_t* o = out + (int64_t)seg * out_stride;
-    float* ov = out_vals ? out_vals + (int64_t)seg * out_stride : nullptr;
-    uint32_t* cnt_out = cl.map_shared_rank(&s_cnt[0], 0);
-    uint32_t* cnt_tie = cl.map_shared_rank(&s_cnt[1], 0);
-
-    int32_t ids[kClPer];
-    uint32_t keys[kClPer];
-#pragma unroll
-    for (int k = 0; k < kClPer; ++k) {
-        const int i = (k * kClCtas + (int)rank) * kClThreads + tid;
-        ids[k] = i < n ? (src.ids ? __ldg(src.ids + seg * src.ids_stride + i) : i) : -1;
-    }
-#pragma unroll
-    for (int k = 0; k < kClPer; ++k) {
-        const int i = (k * kClCtas + (int)rank) * kClThreads + tid;
-        const bool valid = i < n && ids[k] >= 0 && ids[k] < nvalid;
-        keys[k] = select_key(valid ? src.vals[seg * src.vals_stride + (src.gather || !src.ids ? (int64_t)ids[k] : i)]
-                                   : 0.0f, valid);
-        if (keys[k]) atomicAdd(&hist[0][digit(keys[k], 1)], 1u);
-    }
-    cl.sync();   // every CTA's level-1 histogram (and CTA 0's zeroed counters) complete
-    ClPlan pl = cluster_threshold(cl, hist[0], 0u, (uint32_t)n_out, s_wsum, &s_plan);
-    const uint32_t need0 = pl.total < (uint32_t)n_out ? pl.total : (uint32_t)n_out;
-    for (int i = (int)need0 + (int)rank * kClThreads + tid; i < n_out; i += kClCtas * kClThreads) o[i] = -1;
-    uint32_t need = need0, prefix = 0, mask = 0;
-    bool done = need0 == 0;
-    for (int level = 1; level <= 3 && !done; ++level) {
-        if (level > 1) {
-            cl.sync();   // the level's histograms complete in every CTA
-            pl = cluster_threshold(cl, hist[level - 1], need, (uint32_t)n_out, s_wsum, &s_plan);
-        }
-        const uint32_t shift = level == 1 ? 21 : level == 2 ? 10 : 0;
-        const uint32_t dmask = level == 3 ? 0x3FFu : 0x7FFu;
-        const bool all_eq = pl.eq == need - pl.above;
-        // select the elements of the current prefix whose digit is above c (and
-        // those equal to c when exactly the missing number of them exist); the
-        // others equal to c go on to the next digit.  On the last digit the
-        // ones equal to c are exact ties of the full key: the first `need - above`
-        // in claim order win.  Slots and tie ranks are claimed once per CTA
-        // (a block-wide scan, one remote atomic on CTA 0's counters).
-        const bool ties_now = level == 3 && !all_eq;
-        uint32_t take = 0, tie = 0, ntake = 0, ntie = 0;
-#pragma unroll
-        for (int k = 0; k < kClPer; ++k) {
-            const uint32_t key = keys[k];
-            const bool in = key && (key & mask) == prefix;
-            const uint32_t d = (key >> shift) & dmask;
-            const bool tk = in && (d > pl.c || (d == pl.c && all_eq));
-            const bool eq = in && d == pl.c && !all_eq;
-            if (level < 3 && eq) atomicAdd(&hist[level][digit(key, level + 1)], 1u);
-            take |= (uint32_t)tk << k;
-            ntake += tk;
-            if (ties_now && eq) { tie |= 1u << k; ++ntie; }
-        }
-        uint32_t tie_rank = 0;
-        const uint32_t need_ties = ties_now ? need - pl.above : 0u;
-        if (ties_now) {
-            uint64_t tot;
-            const uint64_t pre = block_excl_scan4<kClThreads>((uint64_t)ntie, s_wsum64, &tot);
-            if (tid == 0) s_base[1] = field16(tot, 0) ? atomicAdd(cnt_tie, field16(tot, 0)) : 0u;
-            __syncthreads();
-            tie_rank = s_base[1] + field16(pre, 0);
-#pragma unroll
-            for (int k = 0; k < kClPer; ++k)
-                if ((tie >> k) & 1u) {
-                    if (tie_rank < need_ties) { take |= 1u << k; ++ntake; }
-                    ++tie_rank;
-                }
-        }
-        {
-            uint64_t tot;
-            const uint64_t pre = block_excl_scan4<kClThreads>((uint64_t)ntake, s_wsum64, &tot);
-            if (tid == 0) s_base[0] = field16(tot, 0) ? atomicAdd(cnt_out, field16(tot, 0)) : 0u;
-            __syncthreads();
-            uint32_t os = s_base[0] + field16(pre, 0);
-#pragma unroll
-            for (int k = 0; k < kClPer; ++k)
-                if ((take >> k) & 1u) {
-                    o[os] = ids[k];
-                    if (ov) ov[os] = key_value(keys[k]);
-                    ++os;
-                }
-            __syncthreads();   // s_base is rewritten by the next level
-        }
-        if (all_eq || level == 3) {
-            done = true;
-        } else {
-            need -= pl.above;
-            prefix |= pl.c << shift;
-            mask |= dmask << shift;
-        }
-    }
-    cl.sync();   // no CTA leaves while another may still read its shared memory
 }
 
 // ---------------------------------------------------------------- one CTA per segment

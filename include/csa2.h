@@ -31,7 +31,8 @@
  *    the kernel skips the bad element and ORs a bit into a sticky status word
  *    in the workspace, read back with csa2_read_device_status.
  *  - The library keeps no mutable global state, except the fixed scratch of
- *    csa2_index_reindex_noalloc (see there): calls on different streams with
+ *    csa2_index_reindex_noalloc (see there) and the wait budget of the
+ *    diagnostic csa2_debug_set_wait_limit: calls on different streams with
  *    different workspaces may run concurrently.
  *  - Tensors are dense and row-major in the shapes given.  Pointers must be
  *    16-byte aligned, except seq_lens, page_table and start_pos (4-byte):
@@ -266,6 +267,23 @@ CSA2_API csa2_status csa2_read_device_status(void* ws, void* stream);
 
 /* A static, human-readable name for a status code. */
 CSA2_API const char* csa2_status_string(csa2_status status);
+
+/*
+ * Diagnostic: set how many times the bounded mbarrier waits that guard work in
+ * the tensor-core kernels (scorer, Reindex, attention) try before they give up
+ * and record CSA2_ERR_TIMEOUT, for every launch made after this call returns
+ * (the value is read on the host when a launch is set up; a CUDA graph keeps
+ * the value it was captured with).  A try sleeps for at most about 0.5 us, so
+ * the default, csa2_debug_default_wait_limit(), is about two seconds.  0 makes
+ * those waits give up at once: the kernel then writes no result, flags the
+ * status, waits (bounded) for the copies and MMAs it already issued, frees its
+ * tensor memory and returns, leaving the context usable.  Process-wide; not
+ * meant to be changed while other threads launch.  Always returns CSA2_OK.
+ */
+CSA2_API csa2_status csa2_debug_set_wait_limit(uint32_t tries);
+
+/* The default try count of those waits (the value the library starts with). */
+CSA2_API uint32_t csa2_debug_default_wait_limit(void);
 
 #ifdef __cplusplus
 }
