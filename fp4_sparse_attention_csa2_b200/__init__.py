@@ -20,7 +20,8 @@ F32, BF16, E4M3 = 0, 1, 2
 
 ABI_FUNCTIONS = (
     "csa2_workspace_bytes", "csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
-    "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_sparse_swa_attn", "csa2_layer_step",
+    "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_sparse_swa_attn", "csa2_ring_append",
+    "csa2_sparse_swa_attn_local", "csa2_layer_step",
     "csa2_read_device_status", "csa2_status_string", "csa2_debug_set_wait_limit", "csa2_debug_default_wait_limit",
 )
 
@@ -47,7 +48,7 @@ class csa2_layer_args(ctypes.Structure):
         ("head_w", ctypes.c_void_p), ("T", ctypes.c_int), ("H", ctypes.c_int), ("H_I", ctypes.c_int),
         ("pool_k", ctypes.c_int), ("top_k", ctypes.c_int), ("window", ctypes.c_int), ("sm_scale", ctypes.c_float),
         ("pool_idx", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p), ("out", ctypes.c_void_p),
-        ("lse", ctypes.c_void_p),
+        ("lse", ctypes.c_void_p), ("ring", ctypes.c_void_p), ("ring_len", ctypes.c_int64),
     ]
 
 
@@ -72,6 +73,9 @@ def lib():
         L.csa2_index_reindex.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, vp, vp, sz, vp]
         L.csa2_index_reindex_noalloc.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, vp, vp]
         L.csa2_sparse_swa_attn.argtypes = [cp, vp, i32, i32, vp, i32, i32, ctypes.c_float, vp, vp, vp, sz, vp]
+        L.csa2_ring_append.argtypes = [cp, vp, ctypes.c_int64, vp, vp, i32, vp]
+        L.csa2_sparse_swa_attn_local.argtypes = [cp, vp, ctypes.c_int64, vp, i32, i32, vp, i32, i32, ctypes.c_float,
+                                                 vp, vp, vp, sz, vp]
         L.csa2_layer_step.argtypes = [cp, ctypes.POINTER(csa2_layer_args), vp, sz, vp]
         L.csa2_read_device_status.argtypes = [vp, vp]
         L.csa2_status_string.restype = ctypes.c_char_p
@@ -81,7 +85,8 @@ def lib():
         L.csa2_debug_default_wait_limit.argtypes = []
         for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
                      "csa2_index_reindex", "csa2_index_reindex_noalloc",
-                     "csa2_sparse_swa_attn", "csa2_layer_step", "csa2_read_device_status",
+                     "csa2_sparse_swa_attn", "csa2_ring_append", "csa2_sparse_swa_attn_local",
+                     "csa2_layer_step", "csa2_read_device_status",
                      "csa2_debug_set_wait_limit"):
             getattr(L, name).restype = i32
         _lib = L
@@ -235,13 +240,31 @@ def sparse_swa_attn(cache, q, topk_idx, window, out, lse=None, ws=None, sm_scale
                                       _p(ws), ws.numel() * ws.element_size(), _stream(stream)), "sparse_swa_attn")
 
 
+def ring_append(cache, ring, x, start_pos, stream=None):
+    """Rows x bf16 [B, n_new, dim] of positions start_pos[b] + i into the
+    layer's ring bf16 [B, ring_len, dim] (row t mod ring_len)."""
+    _check(lib().csa2_ring_append(cache.ref, _p(ring), ring.shape[1], _p(x), _p(start_pos), x.shape[1],
+                                  _stream(stream)), "ring_append")
+
+
+def sparse_swa_attn_local(cache, ring, q, topk_idx, window, out, lse=None, ws=None, sm_scale=0.0, stream=None):
+    """sparse_swa_attn with the window rows from the layer's bf16 ring [B, ring_len, dim]."""
+    B, T, H, _ = q.shape
+    top_k = topk_idx.shape[-1] if topk_idx is not None else 0
+    _check(lib().csa2_sparse_swa_attn_local(cache.ref, _p(ring), ring.shape[1], _p(q), T, H, _p(topk_idx), top_k,
+                                            window, sm_scale, _p(out), _p(lse), _p(ws),
+                                            ws.numel() * ws.element_size(), _stream(stream)),
+           "sparse_swa_attn_local")
+
+
 def layer_step(cache, mode, q, topk_idx, out, ws, window, q_idx=None, head_w=None, pool_idx=None, lse=None,
-               pool_k=0, sm_scale=0.0, stream=None):
+               pool_k=0, sm_scale=0.0, ring=None, stream=None):
     B, T, H, _ = q.shape
     H_I = q_idx.shape[2] if q_idx is not None else 0
     a = csa2_layer_args(mode, _addr(q), _addr(q_idx), _qdt(q_idx) if q_idx is not None else BF16, _addr(head_w),
                         T, H, H_I, pool_k or (pool_idx.shape[-1] if pool_idx is not None else 0), topk_idx.shape[-1],
-                        window, sm_scale, _addr(pool_idx), _addr(topk_idx), _addr(out), _addr(lse))
+                        window, sm_scale, _addr(pool_idx), _addr(topk_idx), _addr(out), _addr(lse), _addr(ring),
+                        0 if ring is None else ring.shape[1])
     _check(lib().csa2_layer_step(cache.ref, ctypes.byref(a), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "layer_step")
 

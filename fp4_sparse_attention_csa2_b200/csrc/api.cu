@@ -197,6 +197,41 @@ csa2_status csa2::check_reindex_args(const csa2_cache* c, const void* q_idx, csa
     return CSA2_OK;
 }
 
+namespace {
+
+// Attention with the window rows from the FP4 cache (ring.rows == nullptr) or
+// from a layer-local bf16 ring.
+csa2_status attention(const csa2_cache* cache, const Ring& ring, const void* q_bf16, int T, int H,
+                      const int32_t* topk_idx, int top_k, int window, float sm_scale, float* out, float* lse,
+                      void* ws, size_t ws_bytes, void* stream) {
+    csa2_status s = check_cache(cache);
+    if (s != CSA2_OK) return s;
+    if (!q_bf16 || !out || !aligned16(q_bf16) || !aligned16(out) || (lse && !aligned16(lse))) return CSA2_ERR_INVALID_ARG;
+    if (T < 1 || H < 1 || top_k < 0 || window < 0 || window > kMaxPool || top_k > kMaxPool) return CSA2_ERR_INVALID_ARG;
+    if (top_k > 0 && (!topk_idx || !aligned16(topk_idx))) return CSA2_ERR_INVALID_ARG;
+    if (H > 64 || H % 16) return CSA2_ERR_UNSUPPORTED;
+    if (!std::isfinite(sm_scale)) return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
+    AttnWork aw;
+    aw.part_o = at<float>(ws, L.part_o);
+    aw.part_ml = at<float>(ws, L.part_ml);
+    aw.nchunk = L.nchunk;
+    return cuda_status(launch_attention(dev_cache(cache), q_bf16, T, H, topk_idx, top_k, window, sm_scale, ring, out,
+                                        lse, aw, at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream),
+                                        num_sms()));
+}
+
+// A ring of ring_len rows for T new tokens a step and a window of `window`:
+// the window of the step's first token reaches back T - 1 positions further.
+bool ring_ok(const void* ring, int64_t ring_len, int T, int window) {
+    return ring && aligned16(ring) && ring_len >= 1 && ring_len >= (int64_t)window + T - 1 && ring_len <= ((int64_t)1 << 30);
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t csa2_workspace_bytes(const csa2_cache* cache, int T, int H, int pool_k, int top_k, int window) {
@@ -306,23 +341,32 @@ csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_
 csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, int T, int H, const int32_t* topk_idx,
                                  int top_k, int window, float sm_scale, float* out, float* lse, void* ws,
                                  size_t ws_bytes, void* stream) {
+    return attention(cache, Ring{}, q_bf16, T, H, topk_idx, top_k, window, sm_scale, out, lse, ws, ws_bytes, stream);
+}
+
+csa2_status csa2_sparse_swa_attn_local(const csa2_cache* cache, const void* ring, int64_t ring_len, const void* q_bf16,
+                                       int T, int H, const int32_t* topk_idx, int top_k, int window, float sm_scale,
+                                       float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    if (!ring_ok(ring, ring_len, T, window)) return CSA2_ERR_INVALID_ARG;
+    Ring r;
+    r.rows = static_cast<__nv_bfloat16*>(const_cast<void*>(ring));
+    r.len = ring_len;
+    return attention(cache, r, q_bf16, T, H, topk_idx, top_k, window, sm_scale, out, lse, ws, ws_bytes, stream);
+}
+
+csa2_status csa2_ring_append(const csa2_cache* cache, void* ring, int64_t ring_len, const void* x_bf16,
+                             const int32_t* start_pos, int n_new, void* stream) {
     csa2_status s = check_cache(cache);
     if (s != CSA2_OK) return s;
-    if (!q_bf16 || !out || !aligned16(q_bf16) || !aligned16(out) || (lse && !aligned16(lse))) return CSA2_ERR_INVALID_ARG;
-    if (T < 1 || H < 1 || top_k < 0 || window < 0 || window > kMaxPool || top_k > kMaxPool) return CSA2_ERR_INVALID_ARG;
-    if (top_k > 0 && (!topk_idx || !aligned16(topk_idx))) return CSA2_ERR_INVALID_ARG;
-    if (H > 64 || H % 16) return CSA2_ERR_UNSUPPORTED;
-    if (!std::isfinite(sm_scale)) return CSA2_ERR_INVALID_ARG;
-    Layout L;
-    s = check_ws(cache, T, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
-    if (s != CSA2_OK) return s;
-    if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)cache->dim);
-    AttnWork aw;
-    aw.part_o = at<float>(ws, L.part_o);
-    aw.part_ml = at<float>(ws, L.part_ml);
-    aw.nchunk = L.nchunk;
-    return cuda_status(launch_attention(dev_cache(cache), q_bf16, T, H, topk_idx, top_k, window, sm_scale, out, lse,
-                                        aw, at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream), num_sms()));
+    if (!ring_ok(ring, ring_len, 1, 0) || !x_bf16 || !aligned16(x_bf16) || !start_pos || !aligned4(start_pos) ||
+        n_new < 0 || (int64_t)n_new > ring_len)
+        return CSA2_ERR_INVALID_ARG;
+    if (n_new == 0) return CSA2_OK;
+    Ring r;
+    r.rows = static_cast<__nv_bfloat16*>(ring);
+    r.len = ring_len;
+    return cuda_status(launch_ring_append(r, cache->batch, cache->dim, x_bf16, start_pos, n_new,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* a, void* ws, size_t ws_bytes,
@@ -339,6 +383,9 @@ csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* a, v
         return CSA2_ERR_INVALID_ARG;
     }
     if (s != CSA2_OK) return s;
+    if (a->ring)
+        return csa2_sparse_swa_attn_local(cache, a->ring, a->ring_len, a->q, a->T, a->H, a->topk_idx, a->top_k,
+                                          a->window, a->sm_scale, a->out, a->lse, ws, ws_bytes, stream);
     return csa2_sparse_swa_attn(cache, a->q, a->T, a->H, a->topk_idx, a->top_k, a->window, a->sm_scale, a->out, a->lse,
                                 ws, ws_bytes, stream);
 }
@@ -357,7 +404,7 @@ csa2_status csa2_read_device_status(void* ws, void* stream) {
 }
 
 csa2_status csa2_debug_set_wait_limit(uint32_t tries) {
-    g_wait_limit.store(tries ? tries : 0u, std::memory_order_relaxed);
+    g_wait_limit.store(tries, std::memory_order_relaxed);
     return CSA2_OK;
 }
 

@@ -14,6 +14,8 @@
 // into chunks of kRows entries; one CTA gathers the FP4 rows of its chunk,
 // dequantises them in shared memory and writes a partial (max, sum, unnormalised
 // output) per head.  A second kernel merges the partials (split softmax).
+// With a layer-local bf16 ring ([FANOUT] item 2) the window entries' rows are
+// read from the ring instead (fp32 arithmetic: no range limit beyond fp32's).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -39,8 +41,8 @@ __device__ __forceinline__ int32_t entry_position(const int32_t* topk, int top_k
 // grid (nchunk, batch*T); dynamic smem: H*(D+4) + kRows*(D+4) + H*kRows floats + kRows ints
 __global__ void __launch_bounds__(kThreads)
 k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, const int32_t* __restrict__ topk,
-               int top_k, int window, float scale, float* __restrict__ part_o, float* __restrict__ part_ml,
-               int nchunk, uint32_t* status) {
+               int top_k, int window, float scale, const __nv_bfloat16* __restrict__ ring, int64_t ring_len,
+               float* __restrict__ part_o, float* __restrict__ part_ml, int nchunk, uint32_t* status) {
     pdl_begin();
     extern __shared__ float smem[];
     const int D = c.dim;
@@ -71,6 +73,21 @@ k_attn_partial(DevCache c, const __nv_bfloat16* __restrict__ q, int T, int H, co
         const int r = w / nblk, blk = w % nblk;
         float* dst = vs + r * DP + blk * 16;
         const int32_t t = pos[r];
+        if (ring && t >= 0 && chunk * kRows + r < window) {
+            // a window entry: this layer's bf16 row, ring slot t mod ring_len
+            const uint4* src = reinterpret_cast<const uint4*>(ring + ((int64_t)b * ring_len + t % ring_len) * D + blk * 16);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 u = __ldg(src + h);
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    dst[h * 8 + 2 * k] = __uint_as_float(wv[k] << 16);
+                    dst[h * 8 + 2 * k + 1] = __uint_as_float(wv[k] & 0xFFFF0000u);
+                }
+            }
+            continue;
+        }
         int64_t slot = t >= 0 ? slot_of(c, b, t) : -1;
         if (t >= 0 && slot < 0) flag(status, kStatusBounds);
         if (slot < 0) {
@@ -244,15 +261,15 @@ cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork&
 }
 
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
-                             int window, float sm_scale, float* out, float* lse, const AttnWork& aw_in,
-                             uint32_t* status, cudaStream_t st, int num_sms) {
+                             int window, float sm_scale, const Ring& ring, float* out, float* lse,
+                             const AttnWork& aw_in, uint32_t* status, cudaStream_t st, int num_sms) {
     AttnWork aw = aw_in;
     cudaError_t e;
     if (attn_tc_supported(c, H)) {
         const int rows = attn_tc_rows_per_chunk();
         aw.nchunk = (window + top_k + rows - 1) / rows;
         if (aw.nchunk < 1) aw.nchunk = 1;
-        e = launch_attention_tc(c, q, T, H, topk, top_k, window, sm_scale, aw, status, st, num_sms);
+        e = launch_attention_tc(c, q, T, H, topk, top_k, window, sm_scale, ring, aw, status, st, num_sms);
     } else {
         const int D = c.dim;
         aw.nchunk = (window + top_k + kRows - 1) / kRows;
@@ -262,11 +279,45 @@ cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, con
         e = cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         dim3 grid((unsigned)aw.nchunk, (unsigned)(c.batch * T));
-        e = launch_pdl(k_attn_partial, dim3(grid), dim3(kThreads), smem, st, c, static_cast<const __nv_bfloat16*>(q), T, H, topk, top_k,
-                                                     window, sm_scale, aw.part_o, aw.part_ml, aw.nchunk, status);
+        e = launch_pdl(k_attn_partial, dim3(grid), dim3(kThreads), smem, st, c, static_cast<const __nv_bfloat16*>(q),
+                       T, H, topk, top_k, window, sm_scale, ring.rows, ring.len, aw.part_o, aw.part_ml, aw.nchunk,
+                       status);
     }
     if (e != cudaSuccess) return e;
     return launch_attn_combine(c, T, H, aw, out, lse, st);
+}
+
+}  // namespace csa2
+
+namespace csa2 {
+
+namespace {
+
+// Rows of new tokens into a layer's ring: row i of sequence b (position
+// start_pos[b] + i) to ring row (start_pos[b] + i) mod len.  One warp per row,
+// 16-byte loads and stores.
+__global__ void __launch_bounds__(256)
+k_ring_append(__nv_bfloat16* __restrict__ ring, int64_t len, int batch, int dim, const __nv_bfloat16* __restrict__ x,
+              const int32_t* __restrict__ start_pos, int n_new) {
+    pdl_begin();
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= (int64_t)batch * n_new) return;
+    const int b = (int)(row / n_new), i = (int)(row % n_new);
+    const int64_t pos = (int64_t)__ldg(start_pos + b) + i;
+    if (pos < 0) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x + row * dim);
+    uint4* dst = reinterpret_cast<uint4*>(ring + ((int64_t)b * len + pos % len) * dim);
+    for (int k = threadIdx.x & 31; k < dim / 8; k += 32) dst[k] = __ldg(src + k);
+}
+
+}  // namespace
+
+cudaError_t launch_ring_append(const Ring& ring, int batch, int dim, const void* x, const int32_t* start_pos,
+                               int n_new, cudaStream_t st) {
+    const int64_t rows = (int64_t)batch * n_new;
+    return launch_pdl(k_ring_append, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st,
+                      ring.rows, ring.len, batch, dim,
+                      static_cast<const __nv_bfloat16*>(x), start_pos, n_new);
 }
 
 }  // namespace csa2

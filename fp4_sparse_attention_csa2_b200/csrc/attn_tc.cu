@@ -30,6 +30,12 @@
 //      per accumulator, the slabs issued by the same four warps;
 //   6. the unnormalised partial output [head][d] and (max, sum) per head in
 //      base-2 units to the workspace, merged by the split-softmax combine kernel.
+// With a layer-local bf16 ring ([FANOUT] item 2: the sliding-window state stays
+// with the layer) the window entries' rows are the ring's bf16 rows.  bf16
+// reaches far outside the fp16 range, so a chunk that holds ring rows is scaled
+// by one exact power of two 2^e (its largest magnitude lands in [2^14, 2^15)):
+// e is uniform over the chunk, so it leaves the tensor-core products as they
+// are and comes off as 2^-e on the logits and on the partial output.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -57,6 +63,8 @@ struct Params {
     uint32_t* status;
     uint32_t wait_limit;      // tries of the waits that guard work (not of the drain)
     uint32_t off_q, off_p, off_misc, tmem_cols;
+    const __nv_bfloat16* ring;   // [batch][ring_len][D] or nullptr (window rows from the FP4 cache)
+    int64_t ring_len;
 };
 
 template <int HG>
@@ -69,6 +77,7 @@ struct Misc {
     uint64_t o_bar;              // O^T complete (one commit per issuing warp)
     uint64_t drain_bar;          // every MMA of the CTA complete (one commit per issuing warp)
     uint32_t tmem_base;
+    uint32_t vmax;               // bits of the largest row magnitude of a chunk with ring rows
 };
 
 // Eight E2M1 codes (one 32-bit word, channel 2j in the low nibble of byte j)
@@ -109,7 +118,14 @@ __device__ __forceinline__ float key_to_float(uint32_t key) {
 // Named barrier of the softmax warps (the 8 warps that can read TMEM lanes 0..63).
 __device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-template <int HG>
+// Named barrier of the 16 worker warps.
+__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 2, 512;" ::: "memory"); }
+
+// 2^e as a float, e in [-126, 127].
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+
+// RING: the launch has a layer-local ring (the window entries' rows come from it).
+template <int HG, bool RING>
 __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -128,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         tc::mbar_init(&misc->p_bar, 256);
         tc::mbar_init(&misc->o_bar, kIssuers);
         tc::mbar_init(&misc->drain_bar, kIssuers);
+        misc->vmax = 0u;
         tc::fence_mbar_init();
     }
     if (warp == kWorkers / 32) tc::tmem_alloc(&misc->tmem_base, p.tmem_cols);
@@ -188,11 +205,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
             else if (t > pq || t > pq - p.window) t = -1;   // future, or already in the window
         }
     }
-    const int64_t slot = t >= 0 ? slot_of(p.c, b, t) : -1;
-    if (t >= 0 && slot < 0) { if (kp == 0) flag(p.status, kStatusBounds); t = -1; }
+    // a window entry of a launch with a ring takes its row from the ring (CTA-uniform: ring_chunk)
+    const bool ring_chunk = RING && chunk * kRows < p.window;
+    const bool ring_row = ring_chunk && v_entry < p.window && t >= 0;
+    const int64_t slot = t >= 0 && !ring_row ? slot_of(p.c, b, t) : -1;
+    if (t >= 0 && !ring_row && slot < 0) { if (kp == 0) flag(p.status, kStatusBounds); t = -1; }
     uint4 cv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
     uint32_t sv = 0;
-    if (row_thread && t >= 0) {
+    uint4 rv[RING ? 8 : 1];                          // this thread's 64 bf16 channels of a ring row
+    if (RING && row_thread && ring_row) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.ring + ((int64_t)b * p.ring_len + t % p.ring_len) * D + 64 * kp);
+#pragma unroll
+        for (int i = 0; i < (RING ? 8 : 1); ++i) rv[i] = __ldg(src + i);
+    } else if (row_thread && t >= 0) {
         const uint8_t* row = p.c.rows + slot * p.c.row_stride;
         cv[0] = __ldg(reinterpret_cast<const uint4*>(row + 32 * kp));
         cv[1] = __ldg(reinterpret_cast<const uint4*>(row + 32 * kp + 16));
@@ -240,11 +265,54 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         }
     }
 
+    // ---- the chunk scale of a chunk with ring rows: 2^ec with its largest
+    // magnitude in [2^14, 2^15) (an FP4 row counts as 6 x 448, the largest
+    // E2M1 x E4M3 product); every other chunk has ec = 0
+    int ec = 0;
+    if (RING && ring_chunk) {
+        float am = 0.0f;
+        if (row_thread && ring_row) {
+#pragma unroll
+            for (int i = 0; i < (RING ? 8 : 1); ++i) {
+                const uint32_t wv[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    am = fmaxf(am, fmaxf(fabsf(__uint_as_float(wv[k] << 16)), fabsf(__uint_as_float(wv[k] & 0xFFFF0000u))));
+            }
+        } else if (row_thread && t >= 0) {
+            am = 2688.0f;
+        }
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, __float_as_uint(am));   // non-negative floats order as integers
+        if (lane == 0) atomicMax(&misc->vmax, mk);
+        workers_sync();
+        const uint32_t vm = *reinterpret_cast<volatile uint32_t*>(&misc->vmax);
+        if (vm != 0u) {
+            ec = 14 - ((int)((vm >> 23) & 0xFF) - 127);
+            ec = ec < -100 ? -100 : (ec > 100 ? 100 : ec);
+        }
+    }
+    const float cup = RING ? exp2i(ec) : 1.0f, cdown = RING ? exp2i(-ec) : 1.0f;
+
     // ---- dequantise this thread's 64 channels of its row: value(code) *
     // value(scale), exact in fp16, into K block kp of the swizzled V tile
     // (masked rows are 0).  A warp's 16-byte stores walk 32 consecutive rows
     // of one K block: conflict-free under the 128-byte swizzle.
-    if (row_thread) {
+    if (RING && row_thread && ring_row) {
+        // a ring row: bf16 x 2^ec, rounded once to fp16
+        uint8_t* blk = sV + kp * kBlkBytes;
+#pragma unroll
+        for (int c = 0; c < (RING ? 8 : 1); ++c) {
+            const uint32_t wv[4] = {rv[c].x, rv[c].y, rv[c].z, rv[c].w};
+            uint32_t hv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const __half2 hh = __floats2half2_rn(__uint_as_float(wv[k] << 16) * cup,
+                                                     __uint_as_float(wv[k] & 0xFFFF0000u) * cup);
+                memcpy(&hv[k], &hh, 4);
+            }
+            *reinterpret_cast<uint4*>(blk + tc::sw128_offset(r, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        }
+    } else if (row_thread) {
         uint32_t s2[2];
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2[0]) : "h"((uint16_t)(sv & 0xFFFFu)));
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2[1]) : "h"((uint16_t)(sv >> 16)));
@@ -262,6 +330,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
             // block scale (exact: E2M1 x E4M3 products fit fp16)
 #pragma unroll
             for (int k = 0; k < 4; ++k) hv[k] = hmul2_u32(hmul2_u32(hv[k], two14), s_pair);
+            if (RING && ec != 0) {
+                // an FP4 row in a chunk with ring rows: times 2^ec, rounded once
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    __half2 hh;
+                    memcpy(&hh, &hv[k], 4);
+                    const float2 f = __half22float2(hh);
+                    hh = __floats2half2_rn(f.x * cup, f.y * cup);
+                    memcpy(&hv[k], &hh, 4);
+                }
+            }
             *reinterpret_cast<uint4*>(blk + tc::sw128_offset(r, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
     }
@@ -344,7 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
             }
 #pragma unroll
             for (int i = 0; i < NV; ++i) {
-                z[i] = valid ? v[i] * misc->fac[c0 + i] : -INFINITY;
+                // (the chunk scale comes off last: v * fac alone stays inside the fp32 range)
+                z[i] = valid ? v[i] * misc->fac[c0 + i] * cdown : -INFINITY;
                 const uint32_t mk = __reduce_max_sync(0xffffffffu, ordered_key(z[i]));
                 if (lane == i) misc->red[quad][c0 + i] = key_to_float(mk);
             }
@@ -429,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
                 float v[16];
                 tc::tmem_ld16(tcol + c0, v);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) po[(int64_t)(c0 + i) * D] = v[i];
+                for (int i = 0; i < 16; ++i) po[(int64_t)(c0 + i) * D] = v[i] * cdown;
             }
         }
     }
@@ -449,17 +529,17 @@ size_t attn_tc_smem(int D, uint32_t* off_q, uint32_t* off_p, uint32_t* off_misc)
     return (size_t)v + qbytes + pbytes + sizeof(Misc<HG>) + 1024;
 }
 
-template <int HG>
+template <int HG, bool RING>
 cudaError_t launch_hg(const DevCache& c, const Params& p0, int nseg, cudaStream_t st) {
     Params p = p0;
     uint32_t cols = 32;
     while (cols < (uint32_t)(kIssuers * HG + (c.dim / 128) * HG)) cols <<= 1;
     p.tmem_cols = cols;
     const size_t smem = attn_tc_smem<HG>(c.dim, &p.off_q, &p.off_p, &p.off_misc);
-    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<HG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<HG, RING>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(k_attn_tc<HG>, dim3((unsigned)p.nchunk, (unsigned)nseg, (unsigned)(p.H / HG)), dim3(kThreads),
-                      smem, st, p);
+    return launch_pdl(k_attn_tc<HG, RING>, dim3((unsigned)p.nchunk, (unsigned)nseg, (unsigned)(p.H / HG)),
+                      dim3(kThreads), smem, st, p);
 }
 
 }  // namespace
@@ -479,8 +559,8 @@ int attn_tc_heads_per_cta(int H, int nchunk, int nseg, int num_sms) {
 }
 
 cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
-                                int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st,
-                                int num_sms) {
+                                int window, float sm_scale, const Ring& ring, const AttnWork& aw, uint32_t* status,
+                                cudaStream_t st, int num_sms) {
     Params p;
     p.c = c;
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -495,11 +575,18 @@ cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, 
     p.part_ml = aw.part_ml;
     p.status = status;
     p.wait_limit = wait_limit();
+    p.ring = ring.rows;
+    p.ring_len = ring.len;
     const int nseg = c.batch * T;
     const int hg = attn_tc_heads_per_cta(H, aw.nchunk, nseg, num_sms);
-    if (hg == 16) return launch_hg<16>(c, p, nseg, st);
-    if (hg == 32) return launch_hg<32>(c, p, nseg, st);
-    return launch_hg<64>(c, p, nseg, st);
+    if (ring.rows) {
+        if (hg == 16) return launch_hg<16, true>(c, p, nseg, st);
+        if (hg == 32) return launch_hg<32, true>(c, p, nseg, st);
+        return launch_hg<64, true>(c, p, nseg, st);
+    }
+    if (hg == 16) return launch_hg<16, false>(c, p, nseg, st);
+    if (hg == 32) return launch_hg<32, false>(c, p, nseg, st);
+    return launch_hg<64, false>(c, p, nseg, st);
 }
 
 }  // namespace csa2

@@ -90,6 +90,16 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
                                int64_t stride_a, int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st,
                                bool hist_ready);
 
+// A layer's own window state: bf16 rows [batch][len][dim], position t of
+// sequence b at row t mod len (rows == nullptr: the window comes from the
+// shared FP4 cache).
+struct Ring {
+    __nv_bfloat16* rows = nullptr;
+    int64_t len = 0;
+};
+cudaError_t launch_ring_append(const Ring& ring, int batch, int dim, const void* x, const int32_t* start_pos,
+                               int n_new, cudaStream_t st);
+
 // Attention partials + combine.
 struct AttnWork {
     float* part_o;    // [nseg][nchunk][D][H]
@@ -102,12 +112,12 @@ int attn_tc_rows_per_chunk();
 // heads per CTA: H, halved (down to 16) while the grid would leave SMs idle
 int attn_tc_heads_per_cta(int H, int nchunk, int nseg, int num_sms);
 cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
-                                int window, float sm_scale, const AttnWork& aw, uint32_t* status, cudaStream_t st,
-                                int num_sms);
+                                int window, float sm_scale, const Ring& ring, const AttnWork& aw, uint32_t* status,
+                                cudaStream_t st, int num_sms);
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st);
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
-                             int window, float sm_scale, float* out, float* lse, const AttnWork& aw,
-                             uint32_t* status, cudaStream_t st, int num_sms);
+                             int window, float sm_scale, const Ring& ring, float* out, float* lse,
+                             const AttnWork& aw, uint32_t* status, cudaStream_t st, int num_sms);
 
 }  // namespace csa2

@@ -148,6 +148,14 @@ def latent(w: Workload, b, L, seed=0, t0=0):
     return out
 
 
+def window_rows(w: Workload, l, b, t0, n, seed=0, scale=1.0):
+    """Layer l's own bf16 rows (its layer-local sliding-window state) of
+    positions t0 .. t0 + n - 1 of sequence b: N(0, 1) x scale, rounded to bf16,
+    [n, D].  Drawn per (layer, sequence, t0)."""
+    g = _gen(seed, 70 + l, (b * 131071 + t0) & 0xFFFF)
+    return (torch.randn((n, w.D), generator=g, dtype=torch.float32) * scale).to(torch.bfloat16)
+
+
 def layer_queries(w: Workload, l, seed=0):
     """Layer l's inputs: q bf16 [B, T, H, D], q_idx [B, T, H_I, D_I] (bf16 or
     fp32), head weights w fp32 [B, T, H_I] = 1/H_I."""

@@ -233,12 +233,47 @@ CSA2_API csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q
                                  float* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Layer-local window state ([FANOUT] item 2: the layers share the global KV and
+ * the sparse selections but keep their own queries and sliding-window state;
+ * [TLDR] paragraph 2: the window runs in every layer over the last 128
+ * tokens).  A layer's ring is bf16 [batch][ring_len][dim] in device memory,
+ * owned by the caller; position t of sequence b lives in row t mod ring_len.
+ *
+ * csa2_ring_append writes, for every sequence b and i < n_new, the bf16 row
+ * x_bf16[b][i][0..dim) into ring row (start_pos[b] + i) mod ring_len
+ * (start_pos: device int32 [batch]; a negative start_pos[b] + i is skipped).
+ * Requires 1 <= ring_len <= 2^30, n_new <= ring_len, ring and x_bf16 16-byte
+ * aligned.  Rows must be finite.  The call reads cache->batch and cache->dim
+ * only.
+ *
+ * csa2_sparse_swa_attn_local is csa2_sparse_swa_attn with the rows of the
+ * window positions (p - window < t <= p) taken from the ring, exact bf16,
+ * instead of dequantised from the FP4 cache; top-k positions outside the
+ * window keep their FP4 rows.  The ring must hold the window of every query
+ * token of the call: ring_len >= window + T - 1 (else CSA2_ERR_INVALID_ARG).
+ * Rows may take any finite bf16 value: the tensor-core kernel scales a chunk
+ * of 64 entries that holds ring rows by one exact power of two (its largest
+ * magnitude to [2^14, 2^15)) before its fp16 operands are formed, and takes
+ * the scale off the logits and the partial output (chunks whose largest
+ * magnitude is below 2^-86 keep a scale of 2^100 and lose precision).
+ */
+CSA2_API csa2_status csa2_ring_append(const csa2_cache* cache, void* ring, int64_t ring_len, const void* x_bf16,
+                                      const int32_t* start_pos, int n_new, void* stream);
+
+CSA2_API csa2_status csa2_sparse_swa_attn_local(const csa2_cache* cache, const void* ring, int64_t ring_len,
+                                                const void* q_bf16, int T, int H, const int32_t* topk_idx,
+                                                int top_k, int window, float sm_scale, float* out, float* lse,
+                                                void* ws, size_t ws_bytes, void* stream);
+
+/*
  * One layer of a CSA2 stack ([TLDR] paragraph 3; [FANOUT] item 2):
  *   CSA2_FULL    csa2_index_full (writes pool_idx and topk_idx), then attention
  *   CSA2_REINDEX csa2_index_reindex (reads pool_idx, writes topk_idx), then
  *                attention
  *   CSA2_REUSE   attention only, with topk_idx as given; no index buffer is
  *                read or written other than topk_idx, which is only read.
+ * With ring != NULL the attention is csa2_sparse_swa_attn_local over that
+ * ring (the layer's own window rows, appended by the caller beforehand).
  */
 typedef struct {
     csa2_mode mode;
@@ -252,6 +287,8 @@ typedef struct {
     int32_t* topk_idx;       /* [batch][T][top_k] */
     float* out;              /* [batch][T][H][dim] */
     float* lse;              /* [batch][T][H] or NULL */
+    const void* ring;        /* bf16 [batch][ring_len][dim], this layer's window rows, or NULL */
+    int64_t ring_len;
 } csa2_layer_args;
 
 CSA2_API csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* args, void* ws,

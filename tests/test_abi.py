@@ -142,3 +142,34 @@ def test_noalloc_reindex_refuses_like_the_workspace_entry_point(lib):
     big = fake_cache(batch=80, seq_stride_slots=1 << 14, n_slots=80 << 14)
     assert lib.csa2_index_reindex_noalloc(ctypes.byref(big), 0x40000, csa2.BF16, 0x50000, 1, 32, 0x60000, 16384, 16,
                                           0x70000, None) == csa2.ERR_UNSUPPORTED
+
+
+def test_ring_arguments_rejected_on_host(lib):
+    # the layer-local ring: a ring shorter than window + T - 1, a misaligned or
+    # missing ring, and an append of more rows than the ring holds are refused
+    c = fake_cache()
+    i64 = ctypes.c_int64
+
+    def attn(ring=0x90000, ring_len=128, T=1, window=128):
+        return lib.csa2_sparse_swa_attn_local(ctypes.byref(c), ring, i64(ring_len), 0x40000, T, 64, 0x60000, 2048,
+                                              window, 0.0, 0x70000, None, 0x80000, 1 << 40, None)
+
+    assert attn(ring_len=127) == csa2.ERR_INVALID_ARG
+    assert attn(ring_len=128, T=2) == csa2.ERR_INVALID_ARG
+    assert attn(ring=0x90008) == csa2.ERR_INVALID_ARG
+    assert attn(ring=None) == csa2.ERR_INVALID_ARG
+    assert attn(ring_len=0, window=0) == csa2.ERR_INVALID_ARG
+    # a ring long enough: the call goes on to the attention's own checks (window too large here)
+    assert attn(ring_len=20000, window=16385) == csa2.ERR_INVALID_ARG
+
+    def append(ring=0x90000, ring_len=128, x=0xA0000, sp=0xB0000, n_new=4):
+        return lib.csa2_ring_append(ctypes.byref(c), ring, i64(ring_len), x, sp, n_new, None)
+
+    assert append(n_new=129) == csa2.ERR_INVALID_ARG
+    assert append(x=0xA0002) == csa2.ERR_INVALID_ARG
+    assert append(sp=None) == csa2.ERR_INVALID_ARG
+    assert append(sp=0xB0002) == csa2.ERR_INVALID_ARG
+    assert append(n_new=-1) == csa2.ERR_INVALID_ARG
+    assert append(n_new=0) == csa2.OK                      # nothing to write: nothing launched
+    assert lib.csa2_ring_append(ctypes.byref(fake_cache(dim=100)), 0x90000, i64(128), 0xA0000, 0xB0000, 4,
+                                None) == csa2.ERR_INVALID_ARG
