@@ -444,6 +444,10 @@ def run_ours(args, world, rank):
     del runner, graphs
     torch.cuda.empty_cache()
 
+    # the same step with layer-local window state: every layer appends its T
+    # new bf16 rows to its own ring and attends over the ring's window rows
+    local = local_window_line(w, lens, seed, layers, ws, reps, stream, world, K)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, seed, layers, budget_s=args.cpu_budget)
@@ -493,6 +497,7 @@ def run_ours(args, world, rank):
             "gpu_launches_per_step": launches_per_step,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "local_window": local,
             "workloads": extra,
         }
         line["roofline"]["step_frac_of_8TBps"] = round(line["step_bytes_algorithmic"] / (ms_step / 1e3) / 8e12, 4)
@@ -500,17 +505,63 @@ def run_ours(args, world, rank):
         sys.stdout.flush()
 
 
-def step_bytes(w, lens):
+def local_window_line(w, lens, seed, layers, ws, reps, stream, world, K):
+    """Layer-steps/s of the decode step with a bf16 window ring per layer (the
+    ring append of each layer's T new rows is inside the step), and the
+    attention call over the ring alone."""
+    import fp4_sparse_attention_csa2_b200 as csa2
+    stack = Stack(w, layers, ws)
+    stack.attach_rings(reps, lens, seed)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            stack.step(reps[i % len(reps)])
+    stream.synchronize()
+    st = csa2.read_device_status(ws, stream)
+    if st != csa2.OK:
+        raise RuntimeError("local window: device status after warm-up: " + csa2.status_string(st))
+    graphs, launches = capture_steps(stack, reps, stream)
+    times = replay_regions(graphs, K, stream, world, min_total_s=0.3, min_reps=3)
+    ms = statistics.median(times) / K
+    L0, L1 = stack.layers[0], stack.layers[1]
+    csa2.index_full(reps[0], L0["q_idx"], L0["w"], w.pool_k, w.top_k, stack.pool, stack.topk, ws)
+    attn_ms = timed_launches(lambda c: csa2.sparse_swa_attn_local(c, stack.rings[id(c)][1], L1["q"], stack.topk,
+                                                                  w.window, stack.out[1], stack.lse[1], ws),
+                             reps, stream)
+    st = csa2.read_device_status(ws, stream)
+    if st != csa2.OK:
+        raise RuntimeError("local window: device status after timing: " + csa2.status_string(st))
+    n_q = w.batch * w.T
+    sb = step_bytes(w, lens, local=True)
+    hbm, _ = peaks()
+    del graphs
+    line = {"layer_steps_per_s": round(world * len(w.pattern) / (ms / 1e3), 1), "ms_per_step": round(ms, 5),
+            "ring_rows": stack.ring_len, "ring_bytes_per_layer": w.batch * stack.ring_len * w.D * 2,
+            "gpu_launches_per_step": launches, "attention_ms_per_launch": round(attn_ms, 5),
+            "attention_tflops": round(4.0 * w.H * w.D * n_q * (w.window + w.top_k) / (attn_ms / 1e3) / 1e12, 2),
+            "step_bytes_algorithmic": sb, "step_frac_of_measured_hbm": round(sb / (ms / 1e3) / (hbm * 1e9), 4),
+            "path": "per layer csa2_ring_append of the step's T rows, then csa2_layer_step with the layer's ring "
+                    "(window rows bf16 from the ring, top-k rows FP4 from the shared cache)"}
+    del stack
+    torch.cuda.empty_cache()
+    return line
+
+
+def step_bytes(w, lens, local=False):
     """Algorithmic bytes of one step: index keys scored (every visible key of
     every sequence once: the scorer reads a key once for all of a sequence's
     query tokens), pool keys rescored and FP4 rows attended (upper bound
-    |S| = window + top_k per query token)."""
+    |S| = window + top_k per query token).  local: the window rows are bf16
+    rows of the layer's ring and each layer appends its T new rows."""
     key = 64 if w.idx_key_dtype == wl.E4M3 else 256
     L = lens.astype(np.int64)
     full = int(np.sum(L)) * key
     n_q = w.batch * w.T
     re = n_q * min(w.pool_k, int(L.min())) * key
     S = n_q * (w.window + w.top_k) * (w.D // 2 + w.D // 16)
+    if local:
+        # window rows bf16 from the layer's ring, plus the append of the
+        # step's T rows (read and written)
+        S = n_q * (w.window * 2 * w.D + w.top_k * (w.D // 2 + w.D // 16)) + 2 * n_q * 2 * w.D
     n_f = w.pattern.count("F")
     n_r = w.pattern.count("R")
     return n_f * full + n_r * re + len(w.pattern) * S

@@ -92,6 +92,35 @@ class Stack:
         out_specs = [((B, T, w.H, w.D), torch.float32)] * n + [((B, T, w.H), torch.float32)] * n
         self.outputs, views = flat_views(out_specs, "cuda")
         self.out, self.lse = views[:n], views[n:]
+        self.rings = None
+
+    def attach_rings(self, reps, lens, seed=0):
+        """Give every layer its own bf16 window ring ([B, window + T - 1, D],
+        filled with the layer's rows of the window positions) on every cache
+        replica: each step then appends the layer's T new rows
+        (csa2_ring_append) and attends over the ring's window rows."""
+        w = self.w
+        B, T = w.batch, w.T
+        ring_len = w.window + T - 1
+        self.ring_len = ring_len
+        start = torch.as_tensor(lens, dtype=torch.int32) - ring_len
+        self.fill_start = start.cuda()
+        self.start = (torch.as_tensor(lens, dtype=torch.int32) - T).cuda()
+        self.x_local = []
+        fill = []
+        for l in range(len(self.modes)):
+            rows = torch.stack([wl.window_rows(w, l, b, int(start[b]), ring_len, seed) for b in range(B)])
+            fill.append(rows.cuda())
+            self.x_local.append(rows[:, ring_len - T:].contiguous().cuda())   # the step's own T rows
+        self.rings = {}
+        for c in reps:
+            rl = []
+            for l in range(len(self.modes)):
+                r = torch.zeros((B, ring_len, w.D), dtype=torch.bfloat16, device="cuda")
+                csa2.ring_append(c, r, fill[l], self.fill_start)
+                rl.append(r)
+            self.rings[id(c)] = rl
+        torch.cuda.synchronize()
 
     def host_buffers(self, layers):
         """Pinned host copies of `inputs` (filled from the host-side layers)
@@ -106,12 +135,17 @@ class Stack:
         return h_in, h_out
 
     def step(self, cache):
+        rings = None if self.rings is None else self.rings[id(cache)]
         for l, m in enumerate(self.modes):
             L = self.layers[l]
             idx = m != csa2.REUSE
+            ring = None
+            if rings is not None:
+                ring = rings[l]
+                csa2.ring_append(cache, ring, self.x_local[l], self.start)
             csa2.layer_step(cache, m, L["q"], self.topk, self.out[l], self.ws, self.w.window,
                             q_idx=L["q_idx"] if idx else None, head_w=L["w"] if idx else None, pool_idx=self.pool,
-                            lse=self.lse[l], pool_k=self.w.pool_k)
+                            lse=self.lse[l], pool_k=self.w.pool_k, ring=ring)
 
 
 def new_workspace(cache, w):
