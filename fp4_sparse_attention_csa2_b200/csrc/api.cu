@@ -62,13 +62,14 @@ int num_sms() {
 }
 
 // Workspace layout (byte offsets, each section 256-byte aligned):
-//   status word | full-layer scores | radix histograms | scratch histogram |
+//   status word | full-layer scores | radix histograms | digit-3 histograms | scratch histogram |
 //   radix counters | Reindex arrival counters | candidates 1, 2 | survivors 1, 2 |
 //   pool scores | attention partials
 // The radix histograms and counters are zero between calls: the workspace
 // starts zeroed and every large selection clears what it used.
 struct Layout {
-    size_t status, scores, hist, hist_scratch, cnt, rx_cnt, cand1, cand2, surv1, surv2, pscores, part_o, part_ml, total;
+    size_t status, scores, hist, hist3, hist_scratch, cnt, rx_cnt, cand1, cand2, surv1, surv2, pscores, part_o, part_ml,
+        total;
     int64_t nseg, cap, cand_stride;
     int nchunk;
 };
@@ -84,6 +85,7 @@ bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int w
     L->status = off; off = align_up(off + 16);
     L->scores = off; off = align_up(off + sizeof(float) * (size_t)(L->nseg * L->cap));
     L->hist = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 3 * kRadixBins);
+    L->hist3 = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * 2 * kRadixBins);
     L->hist_scratch = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * kRadixBins);
     L->cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg * kSelCounters);
     L->rx_cnt = off; off = align_up(off + sizeof(uint32_t) * (size_t)L->nseg);
@@ -110,6 +112,8 @@ SelWork sel_work(void* ws, const Layout& L) {
     w.surv1 = at<uint32_t>(ws, L.surv1);
     w.surv2 = at<uint32_t>(ws, L.surv2);
     w.cand_stride = L.cand_stride;
+    w.hist3 = at<uint32_t>(ws, L.hist3);
+    w.status = at<uint32_t>(ws, L.status);
     return w;
 }
 

@@ -27,6 +27,8 @@ struct SelWork {
     uint32_t* surv1;  // [nseg][cand_stride]: level-2 survivors of target a
     uint32_t* surv2;  // [nseg][cand_stride]: of target b
     int64_t cand_stride;
+    uint32_t* hist3 = nullptr;   // [nseg][2][kRadixBins]: digit 3 of both targets (one-grid selection; nullable)
+    uint32_t* status = nullptr;  // sticky device status word
 };
 
 // Where the elements of one selection come from.

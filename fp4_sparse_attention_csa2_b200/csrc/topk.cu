@@ -850,6 +850,263 @@ cudaError_t launch_local_e(const SelSrc& src, int nseg, int n_a, int32_t* out_a,
                       n_b, out_b, stride_b);
 }
 
+// ---------------------------------------------------------------- one grid per selection
+// Both targets of a large segment in one launch, every key held in a register
+// from its load to its decision: C CTAs per segment, each owning
+// kGridThreads x E consecutive elements, meet at barriers (arrival counts in
+// the segment's counters, bounded spins) behind which the segment's digit
+// histograms are complete in global memory:
+//   level 0  (only without the scorer's histogram) digit 1 of every element -> barrier
+//   level 1  the digit-1 histogram -> both targets' (c1, above, eq); the
+//            elements of digit c1 are histogrammed by digit 2          -> barrier A
+//   level 2  the digit-2 histograms -> (c2, above); the elements of digit c2
+//            are histogrammed by digit 3                               -> barrier B
+//   level 3  the digit-3 histograms -> (c3, ties); exact ties at the last
+//            digit are ranked by claim order, one rank shared by both targets
+//            when they cut inside the same group of equal keys (so the top-k
+//            stays inside the pool)
+// then every CTA claims its outputs with one atomic per target, and the last
+// CTA to finish clears the segment's histograms and counters.  All CTAs of a
+// launch must be resident at once: the host launches it only when the whole
+// grid fits on the GPU beside nothing else, and a CTA lets the next kernel
+// launch only after barrier A, when every CTA of the grid has arrived.
+constexpr int kGridThreads = 1024;
+
+// Arrive at the segment barrier (counter ctr) and wait, bounded, until it
+// counts `target` arrivals; false when the wait gave up.
+__device__ __forceinline__ bool seg_barrier(uint32_t* ctr, uint32_t target, uint32_t limit, uint32_t* s_flag) {
+    __threadfence();                                       // this thread's histogram updates, then the arrival
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        atomicAdd(ctr, 1u);
+        uint32_t v = 0;
+        for (uint32_t i = 0;; ++i) {
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+            if (v >= target || i >= limit) break;
+            if (i >= 64) __nanosleep(128);                 // poll back to back at first
+        }
+        *s_flag = v >= target ? 1u : 0u;
+    }
+    __syncthreads();
+    return *s_flag != 0u;
+}
+
+// n words of a histogram written by other CTAs into shared memory (L2 reads).
+__device__ __forceinline__ void load_hist(uint32_t* dst, const uint32_t* src, int n) {
+    for (int i = threadIdx.x; i < n / 4; i += kGridThreads)
+        reinterpret_cast<uint4*>(dst)[i] = __ldcg(reinterpret_cast<const uint4*>(src) + i);
+    __syncthreads();
+}
+
+template <int E>
+__global__ void __launch_bounds__(kGridThreads, 1)
+k_sel_grid(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a,
+           int n_b, int32_t* __restrict__ out_b, int64_t stride_b, int hist_ready, uint32_t wait_limit) {
+    static_assert(E <= 16, "two decision bits per key in one 32-bit word");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ uint32_t s_wsum[kGridThreads / 32];
+    __shared__ uint64_t s_wsum64[kGridThreads / 32];
+    __shared__ Thr s_thr[2];
+    __shared__ uint32_t s_misc[4];
+    __shared__ __align__(16) uint32_t h[2][kRadixBins];    // this CTA's histograms
+    __shared__ __align__(16) uint32_t hc[2][kRadixBins];   // a copy of the segment's
+    const int seg = blockIdx.y, tid = threadIdx.x;
+    const uint32_t C = gridDim.x;
+    uint32_t* cnt = wk.cnt + (int64_t)seg * kSelCounters;
+    uint32_t* h1g = wk.hist + (int64_t)seg * 3 * kRadixBins;
+    uint32_t* h2g = h1g + kRadixBins;                      // [2][kRadixBins]: digit 2 of a's and b's candidates
+    uint32_t* h3g = wk.hist3 + (int64_t)seg * 2 * kRadixBins;
+    uint32_t* bar = cnt + 8;
+    const uint32_t limit = wait_limit * 64u;              // a try sleeps 0.1-0.3 us: a fraction of a second by default
+    const int64_t nvalid = n_valid_positions(src, seg);
+    const int64_t base = (int64_t)blockIdx.x * kGridThreads * E;
+    uint32_t key[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const int64_t i = base + (int64_t)k * kGridThreads + tid;
+        const bool v = i < nvalid;
+        key[k] = select_key(v ? __ldcg(src.vals + seg * src.vals_stride + i) : 0.0f, v);   // a valid key is never 0
+    }
+    for (int i = tid; i < 2 * kRadixBins; i += kGridThreads) (&h[0][0])[i] = 0u;
+    uint32_t nbar = 0;
+    bool ok = true;
+    // flush this CTA's histograms (the nonzero bins) into the segment's and clear them
+    auto flush = [&](uint32_t* dst, int n) {
+        __syncthreads();
+        for (int i = tid; i < n; i += kGridThreads) {
+            const uint32_t v = (&h[0][0])[i];
+            if (v) {
+                atomicAdd(dst + i, v);
+                (&h[0][0])[i] = 0u;
+            }
+        }
+    };
+    if (!hist_ready) {
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < E; ++k)
+            if (key[k]) atomicAdd(&h[0][digit(key[k], 1)], 1u);
+        flush(h1g, kRadixBins);
+        ok = seg_barrier(bar, ++nbar * C, limit, &s_misc[3]) && ok;
+    }
+
+    // ---- level 1
+    load_hist(&hc[0][0], h1g, kRadixBins);
+    Plan1 pa, pb;
+    plans_level1<kGridThreads>(&hc[0][0], (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr, pa, pb);
+    int32_t* oa = out_a + (int64_t)seg * stride_a;
+    int32_t* ob = out_b ? out_b + (int64_t)seg * stride_b : nullptr;
+    float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
+    if (blockIdx.x == 0) {
+        for (int i = (int)pa.need + tid; i < n_a; i += kGridThreads) oa[i] = -1;
+        for (int i = (int)pb.need + tid; i < n_b; i += kGridThreads) ob[i] = -1;
+    }
+    const bool shared = pb.c == pa.c && !pa.take_eq;       // b's candidates are a's
+    const uint32_t c1a = pa.take_eq ? 0xFFFFFFFFu : pa.c, c1b = shared || pb.take_eq ? 0xFFFFFFFFu : pb.c;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const uint32_t d1 = digit(key[k], 1), d2 = digit(key[k], 2);
+        if (key[k] && d1 == c1a) atomicAdd(&h[0][d2], 1u);
+        if (key[k] && d1 == c1b) atomicAdd(&h[1][d2], 1u);
+    }
+    flush(h2g, 2 * kRadixBins);
+    ok = seg_barrier(bar, ++nbar * C, limit, &s_misc[3]) && ok;
+    // every CTA of the grid is resident: the next kernel may launch
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // ---- level 2
+    const Plan1 p1[2] = {pa, pb};
+    uint32_t len[2], need2[2];
+    for (int t = 0; t < 2; ++t) {
+        len[t] = p1[t].take_eq ? 0u : p1[t].eq;
+        need2[t] = len[t] ? p1[t].need - p1[t].above : 0u;
+    }
+    load_hist(&hc[0][0], h2g, 2 * kRadixBins);
+    const uint32_t none[2] = {0u, 0u};
+    Thr q[2];
+    if (shared) {
+        block_thresholds2<kGridThreads>(hc[0], need2, none, s_wsum, s_thr, q);
+    } else {
+        Thr qa[2], qb[2];
+        const uint32_t na_only[2] = {need2[0], 0u}, nb_only[2] = {need2[1], 0u};
+        block_thresholds2<kGridThreads>(hc[0], na_only, none, s_wsum, s_thr, qa);
+        block_thresholds2<kGridThreads>(hc[1], nb_only, none, s_wsum, s_thr, qb);
+        q[0] = qa[0];
+        q[1] = qb[0];
+    }
+    bool eq2[2], lvl3[2];
+    for (int t = 0; t < 2; ++t) {
+        eq2[t] = q[t].eq == need2[t] - q[t].above;
+        lvl3[t] = len[t] && !eq2[t];
+    }
+    // with one list and one digit-2 threshold both targets have the same survivors
+    const bool one_list = shared && lvl3[0] && lvl3[1] && q[0].c == q[1].c;
+    // the survivors of a target share their top 21 bits: (c1, c2)
+    const uint32_t pre_a = lvl3[0] ? (pa.c << 11) | q[0].c : 0xFFFFFFFFu;
+    const uint32_t pre_b = lvl3[1] && !one_list ? (pb.c << 11) | q[1].c : 0xFFFFFFFFu;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const uint32_t top = key[k] >> 10, d3 = digit(key[k], 3);
+        if (key[k] && top == pre_a) atomicAdd(&h[0][d3], 1u);
+        if (key[k] && top == pre_b) atomicAdd(&h[1][d3], 1u);
+    }
+    flush(h3g, 2 * kRadixBins);
+    ok = seg_barrier(bar, ++nbar * C, limit, &s_misc[3]) && ok;
+
+    // ---- level 3
+    load_hist(&hc[0][0], h3g, 2 * kRadixBins);
+    uint32_t need3[2];
+    for (int t = 0; t < 2; ++t) need3[t] = lvl3[t] ? need2[t] - q[t].above : 0u;
+    Thr r3[2];
+    if (one_list) {
+        block_thresholds2<kGridThreads>(hc[0], need3, none, s_wsum, s_thr, r3);
+    } else {
+        Thr ra[2], rb[2];
+        const uint32_t na_only[2] = {need3[0], 0u}, nb_only[2] = {need3[1], 0u};
+        block_thresholds2<kGridThreads>(hc[0], na_only, none, s_wsum, s_thr, ra);
+        block_thresholds2<kGridThreads>(hc[1], nb_only, none, s_wsum, s_thr, rb);
+        r3[0] = ra[0];
+        r3[1] = rb[0];
+    }
+    uint32_t ties[2];
+    for (int t = 0; t < 2; ++t) ties[t] = lvl3[t] ? need3[t] - r3[t].above : 0u;
+    const bool coupled = one_list && r3[0].c == r3[1].c;   // both cut inside one group of equal keys
+
+    // ---- decisions, claims and writes.  Each target's cut as two keys: every
+    // key >= lo is taken; a key equal to tie_key (a cut at the last digit) is
+    // taken by the first `ties` claimants
+    uint32_t lo[2], tie_key[2];
+    for (int t = 0; t < 2; ++t) {
+        const Plan1& p = p1[t];
+        tie_key[t] = 0u;                                   // never a valid key
+        if (p.need == 0) {
+            lo[t] = 0xFFFFFFFFu;                           // above every valid key
+        } else if (p.take_eq) {
+            lo[t] = p.c << 21;
+        } else if (eq2[t]) {
+            lo[t] = (p.c << 21) | (q[t].c << 10);
+        } else {
+            tie_key[t] = (p.c << 21) | (q[t].c << 10) | r3[t].c;
+            lo[t] = tie_key[t] + 1u;
+        }
+    }
+    uint32_t take = 0;                                     // bit 2k: target a takes key k, bit 2k + 1: b
+    uint32_t na = 0, nb = 0;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const bool v = key[k] != 0u;
+        bool sel[2], tie[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            sel[t] = v && key[k] >= lo[t];
+            tie[t] = v && key[k] == tie_key[t];
+        }
+        const uint32_t rk_a = warp_claim(tie[0], cnt + 4);
+        const uint32_t rk_b = coupled ? rk_a : warp_claim(tie[1], cnt + 5);
+        sel[0] = sel[0] || (tie[0] && rk_a < ties[0]);
+        sel[1] = sel[1] || (tie[1] && rk_b < ties[1]);
+        take |= (sel[0] ? 1u : 0u) << (2 * k);
+        take |= (sel[1] ? 2u : 0u) << (2 * k);
+        na += sel[0];
+        nb += sel[1];
+    }
+    uint64_t tot;
+    const uint64_t pre = block_excl_scan4<kGridThreads>((uint64_t)na | ((uint64_t)nb << 16), s_wsum64, &tot);
+    if (tid < 2) {
+        const uint32_t v = field16(tot, tid);
+        s_misc[tid] = v ? atomicAdd(cnt + 2 * tid, v) : 0u;   // a outputs, b outputs
+    }
+    __syncthreads();
+    uint32_t oa_pos = s_misc[0] + field16(pre, 0), ob_pos = s_misc[1] + field16(pre, 1);
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        const int32_t id = (int32_t)(base + (int64_t)k * kGridThreads + tid);
+        if ((take >> (2 * k)) & 1u) {
+            if (oa_pos < (uint32_t)n_a) {
+                oa[oa_pos] = id;
+                if (va) va[oa_pos] = key_value(key[k]);
+            }
+            ++oa_pos;
+        }
+        if ((take >> (2 * k + 1)) & 1u) {
+            if (ob && ob_pos < (uint32_t)n_b) ob[ob_pos] = id;
+            ++ob_pos;
+        }
+    }
+    if (!ok && tid == 0) flag(wk.status, kStatusTimeout);
+
+    // ---- the last CTA leaves the segment's histograms and counters zero
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_misc[2] = atomicAdd(bar, 1u) == (nbar + 1) * C - 1 ? 1u : 0u;
+    __syncthreads();
+    if (!s_misc[2]) return;
+    __threadfence();
+    for (int i = tid; i < 3 * kRadixBins; i += kGridThreads) h1g[i] = 0u;
+    for (int i = tid; i < 2 * kRadixBins; i += kGridThreads) h3g[i] = 0u;
+    if (tid < kSelCounters) cnt[tid] = 0u;
+}
+
 }  // namespace
 
 cudaError_t launch_select_local(const SelSrc& src, int nseg, int n_a, int32_t* out_a, float* vals_a, int64_t stride_a,
@@ -866,13 +1123,54 @@ cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_
     return launch_select_dual(src, wk, nseg, n_out, out, out_vals, out_stride, 0, nullptr, 0, st, hist_ready);
 }
 
+namespace {
+
+// CTAs of k_sel_grid<E> that fit on the device at once (0: unknown).
+template <int E>
+int64_t grid_capacity() {
+    static int64_t cap = -1;
+    if (cap < 0) {
+        int dev = 0, sms = 0, per = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_sel_grid<E>, kGridThreads, 0) != cudaSuccess)
+            return 0;
+        cap = (int64_t)sms * per;
+    }
+    return cap;
+}
+
+template <int E>
+bool try_grid(const SelSrc& src, const SelWork& wk, int nseg, int n_a, int32_t* out_a, float* vals_a, int64_t stride_a,
+              int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st, bool hist_ready, cudaError_t* e) {
+    const int64_t per_cta = (int64_t)kGridThreads * E;
+    const int64_t C = (src.n + per_cta - 1) / per_cta;
+    if (C < 1 || C * nseg > grid_capacity<E>()) return false;
+    *e = launch_pdl(k_sel_grid<E>, dim3((unsigned)C, (unsigned)nseg), dim3(kGridThreads), 0, st, src, wk, n_a, out_a,
+                    vals_a, stride_a, n_b, out_b, stride_b, hist_ready ? 1 : 0, wait_limit());
+    return true;
+}
+
+}  // namespace
+
 cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, int n_a, int32_t* out_a, float* vals_a,
                                int64_t stride_a, int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st,
                                bool hist_ready) {
     // the histograms and counters are zero on entry (workspace initialisation,
-    // then every selection's last CTA clears what it used); without a
-    // histogram from the scoring kernel, build level 1 here
-    cudaError_t e;
+    // then every selection's last CTA clears what it used)
+    cudaError_t e = cudaSuccess;
+    if (src.ids == nullptr && wk.hist3 != nullptr) {
+        // one grid, the keys in registers, when every CTA fits on the GPU at once
+        // the fewest keys per thread (the most CTAs) with which the grid fits
+        if (try_grid<1>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<2>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<4>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<7>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<16>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e))
+            return e;
+    }
+    // otherwise two streaming passes; without a histogram from the scoring
+    // kernel, level 1 is built here
     const unsigned chunks = (unsigned)((src.n + kPassChunk - 1) / kPassChunk);
     dim3 grid(chunks ? chunks : 1, (unsigned)nseg);
     if (!hist_ready) {
