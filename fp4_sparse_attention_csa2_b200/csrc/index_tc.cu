@@ -8,9 +8,10 @@
 // positions); hackernews.kjhq.dev post 49735410, key point 3.
 //
 // The key stream is the HBM-bound hot loop (64 B per position).  The E4M3 keys
-// are the MMA's A operand exactly as stored: TMA tensor loads (64 positions =
-// one page run per box, 64-byte swizzle, no multicast) fill a ring of
-// 128-position tiles that tcgen05.mma reads directly.  The bf16 queries become
+// are the MMA's A operand exactly as stored: TMA tensor loads (64-byte
+// swizzle, no multicast; one 256-row box per stage of a contiguous cache, one
+// 64-row box per page run of a paged one) fill a ring of 256-position stages
+// that tcgen05.mma reads directly, two 128-position tiles per stage.  The bf16 queries become
 // U E4M3 operands stacked along N: per (token, head) row the values are scaled
 // by a power of two so the row maximum lies in [128, 256), then
 //     t0 = E4M3(q),  t1 = E4M3(16 (q - t0)),  t2 = E4M3(256 (q - t0 - t1/16))
@@ -23,11 +24,12 @@
 // power-of-two weights.
 //
 //   producer warp  : TMA loads into the ring (bounded mbarrier waits)
-//   MMA warp       : two tcgen05.mma and one commit per tile into a
-//                    double-buffered TMEM accumulator
-//   epilogue warps : two warpgroups, one per TMEM accumulator (tile g is
-//                    finished by warpgroup g % 2); the first thread to see a
-//                    tile's accumulator releases its ring stage; they stage
+//   MMA warp       : four tcgen05.mma (two per tile) and one commit per stage
+//                    into a double-buffered TMEM accumulator (one buffer
+//                    when two would not fit the 512 columns)
+//   epilogue warps : four warpgroups, one per (buffer, tile); the first
+//                    thread to see a stage's accumulators releases its ring
+//                    stage; they stage
 //                    the query terms when the sequence changes; per tile
 //                    tcgen05.ld of each position's row, ReLU + head-weighted
 //                    sum, fp32 score store, level-1 radix histogram in smem.
@@ -41,14 +43,14 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kTile = 128;
-constexpr int kItemTiles = 8;
+constexpr int kTile = 128;                // positions per MMA (M)
+constexpr int kStagePos = 256;            // positions per ring stage: two tiles, one TMA box when contiguous
 constexpr int kStages = 8;
-constexpr int kStageBytes = kTile * 64;   // two 64-row boxes of E4M3 keys
+constexpr int kStageBytes = kStagePos * 64;
 constexpr int kMaxTerms = 3;
-constexpr int kThreads = 320;
-constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;   // epilogue: warps 2-9, two warpgroups
-constexpr int kEpiThreads = 256;
+constexpr int kThreads = 576;
+constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;   // epilogue: warps 2-17, four warpgroups
+constexpr int kEpiThreads = 512;
 constexpr uint32_t kDrainLimit = 65536;
 
 struct Params {
@@ -61,7 +63,8 @@ struct Params {
     uint32_t* hist;          // [(b*T + j)][3][kRadixBins]; level 1 accumulated here; nullable
     uint32_t* status;
     uint32_t wait_limit;     // tries of the waits that guard work (not of the drains)
-    int64_t items_per_seq, total_items;
+    int64_t items_per_seq, total_items;   // an item is one ring stage of one sequence
+    int nbuf;                // TMEM accumulator buffers of 2 * U * NP columns
     uint32_t tmem_cols;
     uint32_t off_b, off_hist, off_wq, off_bar;
 };
@@ -69,21 +72,37 @@ struct Params {
 struct Item {
     int b;
     int64_t t0, L;
-    int ntiles;
 };
 
-__device__ __forceinline__ bool get_item(const Params& p, int64_t item, Item& it) {
-    const int b = (int)(item / p.items_per_seq);
-    const int64_t k = item - (int64_t)b * p.items_per_seq;
+// The CTA's items blockIdx.x, blockIdx.x + gridDim.x, .. as (sequence, stage)
+// pairs, advanced without a division per item.
+struct ItemCursor {
+    int64_t item, k;
+    int b;
+    __device__ explicit ItemCursor(const Params& p) : item(blockIdx.x) {
+        b = (int)(item / p.items_per_seq);
+        k = item - (int64_t)b * p.items_per_seq;
+    }
+    __device__ void next(const Params& p) {
+        item += gridDim.x;
+        k += gridDim.x;
+        while (k >= p.items_per_seq) {
+            k -= p.items_per_seq;
+            ++b;
+        }
+    }
+};
+
+__device__ __forceinline__ bool get_item(const Params& p, const ItemCursor& cu, Item& it) {
+    const int b = cu.b;
+    const int64_t k = cu.k;
     int64_t L = __ldg(p.c.seq_lens + b);
     L = L < 0 ? 0 : (L > p.c.cap ? p.c.cap : L);
-    const int64_t tiles = (L + kTile - 1) / kTile;
-    const int64_t tile0 = k * kItemTiles;
-    if (tile0 >= tiles) return false;
+    const int64_t t0 = k * kStagePos;
+    if (t0 >= L) return false;
     it.b = b;
-    it.t0 = tile0 * kTile;
+    it.t0 = t0;
     it.L = L;
-    it.ntiles = (int)(tiles - tile0 < kItemTiles ? tiles - tile0 : kItemTiles);
     return true;
 }
 
@@ -169,8 +188,42 @@ __device__ void prepare_queries(const Params& p, int b, uint8_t* bq, float* wq, 
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
-k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
+// Score of one position from its accumulator row (one query token, 32 head
+// columns per term, three terms): x_h = t0 + t1 / 16 + t2 / 256 (the exact
+// term weights), then sum_h w_h max(0, x_h), heads in pairs with f32x2 FMAs.
+__device__ __forceinline__ float score_32x3(uint32_t abase, const float* wq) {
+    const float4* w4 = reinterpret_cast<const float4*>(wq);
+    const float2 k16 = make_float2(0.0625f, 0.0625f), k256 = make_float2(0.00390625f, 0.00390625f);
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {            // heads 16 half .. 16 half + 15
+        uint32_t r[3][16];
+#pragma unroll
+        for (int u = 0; u < 3; ++u) tc::tmem_ld16_nowait(abase + (uint32_t)(32 * u + 16 * half), r[u]);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {                 // heads 16 half + 4 i .. + 3
+            const float4 w = w4[4 * half + i];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int c = 4 * i + 2 * h;
+                float2 x = make_float2(__uint_as_float(r[0][c]), __uint_as_float(r[0][c + 1]));
+                x = __ffma2_rn(make_float2(__uint_as_float(r[1][c]), __uint_as_float(r[1][c + 1])), k16, x);
+                x = __ffma2_rn(make_float2(__uint_as_float(r[2][c]), __uint_as_float(r[2][c + 1])), k256, x);
+                x.x = fmaxf(x.x, 0.0f);
+                x.y = fmaxf(x.y, 0.0f);
+                acc[(2 * i + h) & 3] = __ffma2_rn(h ? make_float2(w.z, w.w) : make_float2(w.x, w.y), x,
+                                                  acc[(2 * i + h) & 3]);
+            }
+        }
+    }
+    return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+}
+
+template <int NBUF>
+__global__ void __launch_bounds__(kThreads, 1)
+k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmap_stage,
+                const Params p) {
     pdl_begin();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -181,15 +234,16 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
     Bars* bars = reinterpret_cast<Bars*>(smem + p.off_bar);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bq_bytes = p.U * p.NP * 64;
-    const int NA = p.U * p.NP;                  // accumulator columns per tile
+    const int NA = p.U * p.NP;                  // accumulator columns per 128-position tile
+    constexpr int nbuf = NBUF;                  // accumulator buffers (a buffer holds a stage's two tiles)
 
     for (int i = threadIdx.x; i < p.T * kRadixBins; i += kThreads) sHist[i] = 0;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) { tc::mbar_init(&bars->full[i], 1); tc::mbar_init(&bars->empty[i], 1); }
-        // empty[s] is arrived by the one epilogue thread that first sees the tile's accumulator
+        // empty[s] is arrived by the one epilogue thread that first sees the stage's accumulators
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars->acc_full[i], 1);
-            tc::mbar_init(&bars->acc_empty[i], 128);
+            tc::mbar_init(&bars->acc_empty[i], 2 * 128);
             tc::mbar_init(&bars->b_ready[i], kEpiThreads);
             tc::mbar_init(&bars->b_free[i], 1);
         }
@@ -198,6 +252,7 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
         tc::mbar_init(&bars->drain, 1);
         tc::fence_mbar_init();
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_stage)) : "memory");
     }
     if (warp == kWarpMma) tc::tmem_alloc(&bars->tmem_base, p.tmem_cols);
     tc::fence_before_sync();
@@ -209,35 +264,39 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
         if (lane == 0) {
             uint32_t g = 0;
             bool ok = true;
-            for (int64_t item = blockIdx.x; item < p.total_items && ok; item += gridDim.x) {
+            for (ItemCursor cu(p); cu.item < p.total_items && ok; cu.next(p)) {
                 Item it;
-                if (!get_item(p, item, it)) continue;
-                for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
-                    const int s = g % kStages;
-                    if (!tc::mbar_wait(&bars->empty[s], ((g / kStages) & 1) ^ 1, p.wait_limit)) { ok = false; break; }
-                    const int64_t t0 = it.t0 + (int64_t)tl * kTile;
-                    int64_t slot[2] = {-1, -1};
+                if (!get_item(p, cu, it)) continue;
+                const int s = g % kStages;
+                if (!tc::mbar_wait(&bars->empty[s], ((g / kStages) & 1) ^ 1, p.wait_limit)) { ok = false; break; }
+                uint8_t* dst = sRing + s * kStageBytes;
+                const int64_t slot0 = p.c.page_table ? -1 : slot_of(p.c, it.b, it.t0);
+                if (slot0 >= 0 && slot0 + kStagePos <= p.c.n_slots) {
+                    // a contiguous cache: the stage is one 256-row box
+                    tc::mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
+                    tc::tma_load_2d(dst, &tmap_stage, 0, (int32_t)slot0, &bars->full[s]);
+                } else {
+                    // a paged cache, or a stage that would reach past the cache:
+                    // one 64-row box per run of 64 positions
+                    int64_t slot[kStagePos / 64];
                     uint32_t bytes = 0;
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const int64_t p0 = t0 + 64 * r;
-                        if (p0 < it.L) {
-                            slot[r] = slot_of(p.c, it.b, p0);
-                            if (slot[r] < 0) flag(p.status, kStatusBounds);
-                            else bytes += 64u * 64u;
-                        }
+                    for (int r = 0; r < kStagePos / 64; ++r) {
+                        const int64_t p0 = it.t0 + 64 * r;
+                        slot[r] = p0 < it.L ? slot_of(p.c, it.b, p0) : -1;
+                        if (p0 < it.L && slot[r] < 0) flag(p.status, kStatusBounds);
+                        if (slot[r] >= 0) bytes += 64u * 64u;
                     }
                     if (bytes == 0) {
                         tc::mbar_arrive(&bars->full[s]);
                     } else {
                         tc::mbar_arrive_expect_tx(&bars->full[s], bytes);
 #pragma unroll
-                        for (int r = 0; r < 2; ++r)
-                            if (slot[r] >= 0)
-                                tc::tma_load_2d(sRing + s * kStageBytes + r * 4096, &tmap, 0, (int32_t)slot[r],
-                                                &bars->full[s]);
+                        for (int r = 0; r < kStagePos / 64; ++r)
+                            if (slot[r] >= 0) tc::tma_load_2d(dst + r * 4096, &tmap, 0, (int32_t)slot[r], &bars->full[s]);
                     }
                 }
+                ++g;
             }
             if (!ok) flag(p.status, kStatusTimeout);
             // loads still in flight must land before the CTA's shared memory goes away
@@ -246,40 +305,49 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = tc::idesc_f8_f32(kTile, NA, 0u, 0u);
+            const uint32_t idesc = tc::idesc_f8_f32(128, NA, 0u, 0u);
             const uint64_t dring = tc::desc_sw64(tc::smem_u32(sRing));
             uint32_t g = 0, n = 0;
             int cur_b = -1;
             bool ok = true;
-            for (int64_t item = blockIdx.x; item < p.total_items && ok; item += gridDim.x) {
+            for (ItemCursor cu(p); cu.item < p.total_items && ok; cu.next(p)) {
                 Item it;
-                if (!get_item(p, item, it)) continue;
+                if (!get_item(p, cu, it)) continue;
                 if (it.b != cur_b) {
                     if (cur_b >= 0) { tc::mma_commit(&bars->b_free[n & 1]); ++n; }
                     cur_b = it.b;
                     if (!tc::mbar_wait(&bars->b_ready[n & 1], (n >> 1) & 1, p.wait_limit)) { ok = false; break; }
                 }
                 const uint64_t db = tc::desc_sw64(tc::smem_u32(sB + (n & 1) * bq_bytes));
-                for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
-                    const int s = g % kStages, acc = g & 1;
-                    if (!tc::mbar_wait(&bars->full[s], (g / kStages) & 1, p.wait_limit) ||
-                        !tc::mbar_wait(&bars->acc_empty[acc], ((g >> 1) & 1) ^ 1, p.wait_limit)) { ok = false; break; }
-                    tc::fence_after_sync();
-                    const uint64_t da = tc::desc_at(dring, (uint32_t)s * kStageBytes);
-                    const uint32_t d = tmem + (uint32_t)(acc * NA);
-                    tc::mma_f8(d, da, db, idesc, 0u);
-                    tc::mma_f8(d, tc::desc_at(da, 32), tc::desc_at(db, 32), idesc, 1u);
-                    tc::mma_commit(&bars->acc_full[acc]);
+                const int s = g % kStages, buf = g % nbuf;
+                const uint32_t use = g / nbuf;            // the buffer's use count
+                if (!tc::mbar_wait(&bars->full[s], (g / kStages) & 1, p.wait_limit) ||
+                    !tc::mbar_wait(&bars->acc_empty[buf], (use & 1) ^ 1, p.wait_limit)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint64_t da = tc::desc_at(dring, (uint32_t)s * kStageBytes);
+                const uint32_t d = tmem + (uint32_t)(buf * 2 * NA);
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {            // the stage's two 128-position tiles
+                    const uint64_t dx = tc::desc_at(da, (uint32_t)x * (kTile * 64));
+                    tc::mma_f8(d + (uint32_t)(x * NA), dx, db, idesc, 0u);
+                    tc::mma_f8(d + (uint32_t)(x * NA), tc::desc_at(dx, 32), tc::desc_at(db, 32), idesc, 1u);
                 }
+                tc::mma_commit(&bars->acc_full[buf]);
+                ++g;
             }
             if (!ok) flag(p.status, kStatusTimeout);
             tc::mma_commit(&bars->drain);
             tc::mbar_wait(&bars->drain, 0, kDrainLimit);
         }
     } else {
-        // epilogue: two warpgroups; thread = TMEM lane = position in the tile
-        const int tid = threadIdx.x - kWarpEpi0 * 32;          // 0..255
-        const int grp = tid >> 7;                               // accumulator this group drains
+        // epilogue: four warpgroups; warpgroup w finishes tile w % 2 of the
+        // stages held in accumulator buffer w / 2 (with one buffer, warpgroups
+        // 2 and 3 only take part in the per-sequence steps); thread = TMEM lane
+        // = position in the tile
+        const int tid = threadIdx.x - kWarpEpi0 * 32;          // 0..511
+        const int grp = tid >> 7;                               // warpgroup
+        const int my_buf = grp >> 1, my_x = grp & 1;
+        const bool works = my_buf < nbuf;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
@@ -311,9 +379,9 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
             return __all_sync(0xffffffffu, got);
         };
         const float* wq = sWq;
-        for (int64_t item = blockIdx.x; item < p.total_items && ok; item += gridDim.x) {
+        for (ItemCursor cu(p); cu.item < p.total_items && ok; cu.next(p)) {
             Item it;
-            if (!get_item(p, item, it)) continue;
+            if (!get_item(p, cu, it)) continue;
             if (it.b != cur_b) {
                 if (cur_b >= 0) {
                     if (!flush(cur_b)) { ok = false; break; }
@@ -331,52 +399,60 @@ k_score_full_tc(const __grid_constant__ CUtensorMap tmap, const Params p) {
                 if (!warp_wait(&bars->b_ready[qb], (n >> 1) & 1)) { ok = false; break; }
                 wq = sWq + qb * p.NP;
             }
-            for (int tl = 0; tl < it.ntiles; ++tl, ++g) {
-                const int acc = g & 1;
-                if (acc != grp) continue;                       // the other group's tile
-                const int64_t t = it.t0 + (int64_t)tl * kTile + row;
-                // a position on a page outside the cache was not loaded (the
-                // producer flagged it): its score is NaN, which is never selected
-                const bool skipped = p.c.page_table != nullptr && t < it.L && slot_of(p.c, it.b, t) < 0;
-                if (!warp_wait(&bars->acc_full[acc], (g >> 1) & 1)) { ok = false; break; }
-                tc::fence_after_sync();
-                // the MMAs of this tile are complete: its ring stage can be refilled
-                if ((tid & 127) == 0) tc::mbar_arrive(&bars->empty[g % kStages]);
-                const uint32_t abase = lane_addr + (uint32_t)(acc * NA);
-                for (int j = 0; j < p.T; ++j) {
-                    float s0 = 0.0f, s1 = 0.0f;
-                    for (int c0 = j * p.HP; c0 < (j + 1) * p.HP; c0 += 16) {
-                        // the 16 heads' columns of every term in flight, one wait
-                        uint32_t r[kMaxTerms][16];
-                        tc::tmem_ld16_nowait(abase + (uint32_t)c0, r[0]);
-                        tc::tmem_ld16_nowait(abase + (uint32_t)(p.NP + c0), r[1]);
-                        if (p.U > 2) tc::tmem_ld16_nowait(abase + (uint32_t)(2 * p.NP + c0), r[2]);
-                        tc::tmem_ld_wait();
-                        const float4* w4 = reinterpret_cast<const float4*>(wq + c0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 ww = w4[i];
-                            float dot[4];
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                float x = fmaf(__uint_as_float(r[1][4 * i + k]), 0.0625f, __uint_as_float(r[0][4 * i + k]));
-                                if (p.U > 2) x = fmaf(__uint_as_float(r[2][4 * i + k]), 0.00390625f, x);
-                                dot[k] = fmaxf(x, 0.0f);
-                            }
-                            s0 = fmaf(ww.x, dot[0], s0);
-                            s1 = fmaf(ww.y, dot[1], s1);
-                            s0 = fmaf(ww.z, dot[2], s0);
-                            s1 = fmaf(ww.w, dot[3], s1);
-                        }
-                    }
-                    const float s = skipped ? __int_as_float(0x7fc00000) : s0 + s1;
-                    const bool vis = t <= it.L - p.T + j;
-                    if (vis) p.scores[((int64_t)it.b * p.T + j) * p.c.cap + t] = s;
-                    if (p.hist && vis && !skipped) atomicAdd(&sHist[j * kRadixBins + (ordered_key(s) >> 21)], 1u);
+            const uint32_t gs = g++;
+            if (!works || (int)(gs % nbuf) != my_buf) continue;   // another warpgroup's stage
+            const uint32_t use = gs / nbuf;
+            const int64_t t = it.t0 + (int64_t)my_x * kTile + row;
+            // a position on a page outside the cache was not loaded (the
+            // producer flagged it): its score is NaN, which is never selected
+            const bool skipped = p.c.page_table != nullptr && t < it.L && slot_of(p.c, it.b, t) < 0;
+            if (!warp_wait(&bars->acc_full[my_buf], use & 1)) { ok = false; break; }
+            tc::fence_after_sync();
+            // the MMAs of this stage are complete: its ring stage can be refilled
+            if (my_x == 0 && (tid & 127) == 0) tc::mbar_arrive(&bars->empty[gs % kStages]);
+            const uint32_t abase = lane_addr + (uint32_t)((my_buf * 2 + my_x) * NA);
+            if (p.T == 1 && p.NP == 32 && p.U == 3) {
+                // one query token, 32 head columns per term: every column of the
+                // three terms in flight at once, the heads in pairs (f32x2)
+                const float sc = skipped ? __int_as_float(0x7fc00000) : score_32x3(abase, wq);
+                if (t <= it.L - 1) {
+                    p.scores[(int64_t)it.b * p.c.cap + t] = sc;
+                    if (p.hist && !skipped) atomicAdd(&sHist[ordered_key(sc) >> 21], 1u);
                 }
-                tc::fence_before_sync();
-                tc::mbar_arrive(&bars->acc_empty[acc]);
+            } else
+            for (int j = 0; j < p.T; ++j) {
+                float s0 = 0.0f, s1 = 0.0f;
+                for (int c0 = j * p.HP; c0 < (j + 1) * p.HP; c0 += 16) {
+                    // the 16 heads' columns of every term in flight, one wait
+                    uint32_t r[kMaxTerms][16];
+                    tc::tmem_ld16_nowait(abase + (uint32_t)c0, r[0]);
+                    tc::tmem_ld16_nowait(abase + (uint32_t)(p.NP + c0), r[1]);
+                    if (p.U > 2) tc::tmem_ld16_nowait(abase + (uint32_t)(2 * p.NP + c0), r[2]);
+                    tc::tmem_ld_wait();
+                    const float4* w4 = reinterpret_cast<const float4*>(wq + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float4 ww = w4[i];
+                        float dot[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            float x = fmaf(__uint_as_float(r[1][4 * i + k]), 0.0625f, __uint_as_float(r[0][4 * i + k]));
+                            if (p.U > 2) x = fmaf(__uint_as_float(r[2][4 * i + k]), 0.00390625f, x);
+                            dot[k] = fmaxf(x, 0.0f);
+                        }
+                        s0 = fmaf(ww.x, dot[0], s0);
+                        s1 = fmaf(ww.y, dot[1], s1);
+                        s0 = fmaf(ww.z, dot[2], s0);
+                        s1 = fmaf(ww.w, dot[3], s1);
+                    }
+                }
+                const float sc = skipped ? __int_as_float(0x7fc00000) : s0 + s1;
+                const bool vis = t <= it.L - p.T + j;
+                if (vis) p.scores[((int64_t)it.b * p.T + j) * p.c.cap + t] = sc;
+                if (p.hist && vis && !skipped) atomicAdd(&sHist[j * kRadixBins + (ordered_key(sc) >> 21)], 1u);
             }
+            tc::fence_before_sync();
+            tc::mbar_arrive(&bars->acc_empty[my_buf]);
         }
         if (ok && cur_b >= 0 && !flush(cur_b)) ok = false;
         if (!ok) flag(p.status, kStatusTimeout);
@@ -452,11 +528,12 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
     p.hist = hist;
     p.status = status;
     p.wait_limit = wait_limit();
-    const int64_t tiles_cap = (c.cap + kTile - 1) / kTile;
-    p.items_per_seq = (tiles_cap + kItemTiles - 1) / kItemTiles;
+    p.items_per_seq = (c.cap + kStagePos - 1) / kStagePos;
     p.total_items = p.items_per_seq * c.batch;
+    // two buffers of a stage's two tiles when they fit in the 512 TMEM columns
+    p.nbuf = 4 * p.U * p.NP <= 512 ? 2 : 1;
     uint32_t cols = 32;
-    while (cols < (uint32_t)(2 * p.U * p.NP)) cols <<= 1;
+    while (cols < (uint32_t)(2 * p.nbuf * p.U * p.NP)) cols <<= 1;
     p.tmem_cols = cols;
     const SmemPlan sp = smem_plan(T, p.NP);
     p.off_b = sp.off_b;
@@ -464,26 +541,31 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
     p.off_wq = sp.off_wq;
     p.off_bar = sp.off_bar;
 
-    // keys as a 2-D byte tensor [n_slots][64]: 64-row boxes, 64-byte swizzle
-    CUtensorMap tmap;
+    // keys as a 2-D byte tensor [n_slots][64], 64-byte swizzle: 64-row boxes
+    // (page runs) and 256-row boxes (a whole stage of a contiguous cache)
+    CUtensorMap tmap, tmap_stage;
     const cuuint64_t gdim[2] = {64, (cuuint64_t)c.n_slots};
     const cuuint64_t gstride[1] = {64};
-    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t box[2] = {64, 64}, box_stage[2] = {64, (cuuint32_t)kStagePos};
     const cuuint32_t estride[2] = {1, 1};
     EncodeTiled enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.keys, gdim, gstride, box, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        enc(&tmap_stage, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.keys, gdim, gstride, box_stage, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
 
-    cudaError_t e = cudaFuncSetAttribute(k_score_full_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+    auto kern = p.nbuf == 2 ? k_score_full_tc<2> : k_score_full_tc<1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
     if (e != cudaSuccess) return e;
-    // two CTAs per SM when their accumulators fit in TMEM together
-    int64_t grid = (cols <= 256 ? 2 : 1) * (int64_t)num_sms;
+    // one CTA per SM (its four epilogue warpgroups and up to 512 TMEM columns)
+    int64_t grid = (int64_t)num_sms;
     if (grid > p.total_items) grid = p.total_items;
     if (grid < 1) grid = 1;
-    return launch_pdl(k_score_full_tc, dim3((unsigned)grid), dim3(kThreads), sp.total, st, tmap, p);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), sp.total, st, tmap, tmap_stage, p);
 }
 
 }  // namespace csa2
