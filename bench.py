@@ -447,6 +447,9 @@ def run_ours(args, world, rank):
     # the same step with layer-local window state: every layer appends its T
     # new bf16 rows to its own ring and attends over the ring's window rows
     local = local_window_line(w, lens, seed, layers, ws, reps, stream, world, K)
+    # the append-time pool update of an in-flight request (its pool kept current
+    # as tokens are appended), for one and for 64 appended positions
+    pool_update = pool_update_line(w, lens, stack, ws, reps, stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -498,6 +501,7 @@ def run_ours(args, world, rank):
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
             "local_window": local,
+            "pool_update": pool_update,
             "workloads": extra,
         }
         line["roofline"]["step_frac_of_8TBps"] = round(line["step_bytes_algorithmic"] / (ms_step / 1e3) / 8e12, 4)
@@ -544,6 +548,35 @@ def local_window_line(w, lens, seed, layers, ws, reps, stream, world, K):
     del stack
     torch.cuda.empty_cache()
     return line
+
+
+def pool_update_line(w, lens, stack, ws, reps, stream):
+    """csa2_index_pool_update timed alone (graph of calls over the replicas):
+    the Full layer's pool, without the positions about to be appended, updated
+    with the last n_new positions under the Reindex layer's query.
+    Algorithmic bytes: the index keys of every candidate (64 B each, E4M3)."""
+    import fp4_sparse_attention_csa2_b200 as csa2
+    L0, L1 = stack.layers[0], stack.layers[1]
+    csa2.index_full(reps[0], L0["q_idx"], L0["w"], w.pool_k, w.top_k, stack.pool, stack.topk, ws)
+    torch.cuda.synchronize()
+    out = {}
+    key = 64 if w.idx_key_dtype == wl.E4M3 else 256
+    for n_new in (1, 64):
+        t_new0 = torch.as_tensor(lens.astype(np.int64) - n_new, device="cuda").view(-1, 1, 1)
+        prev = torch.where(stack.pool >= t_new0, torch.full_like(stack.pool, -1), stack.pool).contiguous()
+        pool = torch.empty_like(prev)
+        topk = torch.empty_like(stack.topk)
+        ms = timed_launches(lambda c: csa2.index_pool_update(c, L1["q_idx"], L1["w"], prev, n_new, w.top_k, pool,
+                                                             topk, ws), reps, stream)
+        st = csa2.read_device_status(ws, stream)
+        if st != csa2.OK:
+            raise RuntimeError("pool update: device status " + csa2.status_string(st))
+        n_q = w.batch * w.T
+        out["n_new_%d" % n_new] = {"us_per_call": round(ms * 1e3, 2),
+                                   "candidates": w.pool_k + n_new,
+                                   "updates_per_s": round(n_q / (ms / 1e3), 1),
+                                   "algorithmic_bytes_per_call": n_q * (w.pool_k + n_new) * key}
+    return out
 
 
 def step_bytes(w, lens, local=False):

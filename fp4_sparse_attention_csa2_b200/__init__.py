@@ -20,7 +20,8 @@ F32, BF16, E4M3 = 0, 1, 2
 
 ABI_FUNCTIONS = (
     "csa2_workspace_bytes", "csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
-    "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_sparse_swa_attn", "csa2_ring_append",
+    "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update", "csa2_sparse_swa_attn",
+    "csa2_ring_append",
     "csa2_sparse_swa_attn_local", "csa2_layer_step",
     "csa2_read_device_status", "csa2_status_string", "csa2_debug_set_wait_limit", "csa2_debug_default_wait_limit",
 )
@@ -72,6 +73,7 @@ def lib():
         L.csa2_index_full.argtypes = [cp, vp, i32, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
         L.csa2_index_reindex.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, vp, vp, sz, vp]
         L.csa2_index_reindex_noalloc.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, vp, vp]
+        L.csa2_index_pool_update.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, sz, vp]
         L.csa2_sparse_swa_attn.argtypes = [cp, vp, i32, i32, vp, i32, i32, ctypes.c_float, vp, vp, vp, sz, vp]
         L.csa2_ring_append.argtypes = [cp, vp, ctypes.c_int64, vp, vp, i32, vp]
         L.csa2_sparse_swa_attn_local.argtypes = [cp, vp, ctypes.c_int64, vp, i32, i32, vp, i32, i32, ctypes.c_float,
@@ -84,7 +86,7 @@ def lib():
         L.csa2_debug_default_wait_limit.restype = ctypes.c_uint32
         L.csa2_debug_default_wait_limit.argtypes = []
         for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
-                     "csa2_index_reindex", "csa2_index_reindex_noalloc",
+                     "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update",
                      "csa2_sparse_swa_attn", "csa2_ring_append", "csa2_sparse_swa_attn_local",
                      "csa2_layer_step", "csa2_read_device_status",
                      "csa2_debug_set_wait_limit"):
@@ -230,6 +232,16 @@ def index_reindex_noalloc(cache, q_idx, head_w, pool_idx, top_k, topk_idx, strea
     _check(lib().csa2_index_reindex_noalloc(cache.ref, _p(q_idx), _qdt(q_idx), _p(head_w), T, H_I, _p(pool_idx),
                                             pool_idx.shape[-1], top_k, _p(topk_idx), _stream(stream)),
            "index_reindex_noalloc")
+
+
+def index_pool_update(cache, q_idx, head_w, pool_prev, n_new, top_k, pool_idx, topk_idx, ws, stream=None):
+    """The pool of an in-flight request after its last n_new positions were
+    appended: the best of pool_prev [B, T, pool_k] and the new positions, into
+    pool_idx [B, T, pool_k] (may be pool_prev) and topk_idx [B, T, top_k]."""
+    B, T, H_I, _ = q_idx.shape
+    _check(lib().csa2_index_pool_update(cache.ref, _p(q_idx), _qdt(q_idx), _p(head_w), T, H_I, _p(pool_prev),
+                                        pool_prev.shape[-1], n_new, top_k, _p(pool_idx), _p(topk_idx), _p(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)), "index_pool_update")
 
 
 def sparse_swa_attn(cache, q, topk_idx, window, out, lse=None, ws=None, sm_scale=0.0, stream=None):

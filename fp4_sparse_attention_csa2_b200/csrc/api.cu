@@ -64,12 +64,12 @@ int num_sms() {
 // Workspace layout (byte offsets, each section 256-byte aligned):
 //   status word | full-layer scores | radix histograms | digit-3 histograms | scratch histogram |
 //   radix counters | Reindex arrival counters | candidates 1, 2 | survivors 1, 2 |
-//   pool scores | attention partials
+//   pool scores | pool-update candidates and their scores | attention partials
 // The radix histograms and counters are zero between calls: the workspace
 // starts zeroed and every large selection clears what it used.
 struct Layout {
-    size_t status, scores, hist, hist3, hist_scratch, cnt, rx_cnt, cand1, cand2, surv1, surv2, pscores, part_o, part_ml,
-        total;
+    size_t status, scores, hist, hist3, hist_scratch, cnt, rx_cnt, cand1, cand2, surv1, surv2, pscores, upd_ids,
+        upd_scores, part_o, part_ml, total;
     int64_t nseg, cap, cand_stride;
     int nchunk;
 };
@@ -94,6 +94,9 @@ bool make_layout(const csa2_cache* c, int T, int H, int pool_k, int top_k, int w
     L->surv1 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->surv2 = off; off = align_up(off + 2 * sizeof(uint32_t) * (size_t)(L->nseg * L->cand_stride));
     L->pscores = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * pool_k);
+    // the candidate list of a pool update: the previous pool and up to kMaxPool appended positions
+    L->upd_ids = off; off = align_up(off + sizeof(int32_t) * (size_t)L->nseg * (pool_k + kMaxPool));
+    L->upd_scores = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * (pool_k + kMaxPool));
     L->part_o = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * c->dim);
     L->part_ml = off; off = align_up(off + sizeof(float) * (size_t)L->nseg * L->nchunk * H * 2);
     L->total = off;
@@ -340,6 +343,43 @@ csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_
     cudaError_t e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, pool_idx, pool_k, ps, status, st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
     return topk_from_pool(cache, L, ws, ps, pool_k, 0, pool_idx, pool_k, top_k, topk_idx, T, st);
+}
+
+csa2_status csa2_index_pool_update(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
+                                   const float* head_w, int T, int H_I, const int32_t* pool_prev, int pool_k, int n_new,
+                                   int top_k, int32_t* pool_idx, int32_t* topk_idx, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    csa2_status s = check_reindex_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_prev, pool_k, top_k, topk_idx);
+    if (s != CSA2_OK) return s;
+    if (!pool_idx || !aligned16(pool_idx) || n_new < 0 || n_new > kMaxPool) return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(cache, T, 1, pool_k, top_k, 0, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevCache d = dev_cache(cache);
+    uint32_t* status = at<uint32_t>(ws, L.status);
+    const int m = pool_k + n_new;                      // candidates per (sequence, token)
+    int32_t* ids = at<int32_t>(ws, L.upd_ids);
+    float* sc = at<float>(ws, L.upd_scores);
+    cudaError_t e = launch_pool_candidates(d, T, pool_prev, pool_k, n_new, ids, status, st);
+    if (e == cudaSuccess) e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, ids, m, sc, status, st);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    SelSrc src;
+    src.vals = sc;
+    src.vals_stride = m;
+    src.ids = ids;
+    src.ids_stride = m;
+    src.gather = 0;
+    src.n = m;
+    src.seq_lens = cache->seq_lens;
+    src.T = T;
+    src.cap = L.cap;
+    // the new pool and this token's top-k (a subset of it) from the same scores
+    if (m <= kSmallSelect)
+        return cuda_status(launch_select_local(src, (int)L.nseg, pool_k, pool_idx, nullptr, pool_k, top_k, topk_idx,
+                                               top_k, st));
+    return cuda_status(launch_select_dual(src, sel_work(ws, L), (int)L.nseg, pool_k, pool_idx, nullptr, pool_k, top_k,
+                                          topk_idx, top_k, st, false));
 }
 
 csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, int T, int H, const int32_t* topk_idx,

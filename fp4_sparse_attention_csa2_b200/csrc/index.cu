@@ -159,7 +159,39 @@ k_score_pool(DevCache c, const void* __restrict__ q, int q_f32, const float* __r
     if (i < pool_k && part == 0) scores[(int64_t)seg * pool_k + i] = live ? s : __int_as_float(0x7fc00000);
 }
 
+// One thread per candidate slot; grid (ceil(m / 256), batch * T).
+__global__ void __launch_bounds__(256)
+k_pool_candidates(DevCache c, int T, const int32_t* __restrict__ pool_prev, int pool_k, int n_new,
+                  int32_t* __restrict__ ids, uint32_t* status) {
+    pdl_begin();
+    const int seg = blockIdx.y, b = seg / T, j = seg % T;
+    const int m = pool_k + n_new;
+    const int i = blockIdx.x * 256 + threadIdx.x;
+    if (i >= m) return;
+    const int64_t L = seq_len(c, b, status);
+    const int64_t p = L - T + j, t_new0 = L - n_new;
+    int32_t t = -1;
+    if (i < pool_k) {
+        t = pool_prev[(int64_t)seg * pool_k + i];
+        if (t < -1 || (t >= 0 && (t >= t_new0 || t > p))) {
+            flag(status, kStatusBounds);
+            t = -1;
+        }
+    } else {
+        const int64_t tn = t_new0 + (i - pool_k);
+        t = tn >= 0 && tn <= p ? (int32_t)tn : -1;
+    }
+    ids[(int64_t)seg * m + i] = t;
+}
+
 }  // namespace
+
+cudaError_t launch_pool_candidates(const DevCache& c, int T, const int32_t* pool_prev, int pool_k, int n_new,
+                                   int32_t* ids, uint32_t* status, cudaStream_t st) {
+    const int m = pool_k + n_new;
+    dim3 grid((unsigned)((m + 255) / 256), (unsigned)(c.batch * T));
+    return launch_pdl(k_pool_candidates, dim3(grid), dim3(256), 0, st, c, T, pool_prev, pool_k, n_new, ids, status);
+}
 
 cudaError_t launch_score_full(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
                               float* scores, uint32_t* status, cudaStream_t st, int /*num_sms*/) {

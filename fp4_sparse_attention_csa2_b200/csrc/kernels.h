@@ -73,6 +73,12 @@ cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw,
 // Pool rescoring: scores[seg * pool_k + i] for pool entry i of segment seg.
 cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
                               const int32_t* pool, int pool_k, float* scores, uint32_t* status, cudaStream_t st);
+// Candidate list of a pool update, ids[seg][0 .. pool_k + n_new): the previous
+// pool's entries (-1 kept; an entry at or beyond the first appended position
+// L - n_new, or beyond the token's position, is flagged and dropped), then the
+// appended positions L - n_new .. L - 1 (those beyond the token's position -1).
+cudaError_t launch_pool_candidates(const DevCache& c, int T, const int32_t* pool_prev, int pool_k, int n_new,
+                                   int32_t* ids, uint32_t* status, cudaStream_t st);
 
 // Top-n selection per segment into out[seg * out_stride + 0..n_out) (-1 padded).
 // hist_ready: the level-1 histogram was zeroed and accumulated by the scoring

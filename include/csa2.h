@@ -187,6 +187,28 @@ CSA2_API csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_i
                                void* stream);
 
 /*
+ * Append-time pool update for an in-flight request ([TLDR] paragraphs 3-4:
+ * the candidate pool kept current as quantised tokens are appended).  The
+ * last n_new positions of every sequence (L - n_new .. L - 1, L =
+ * seq_lens[b]) have just been appended (csa2_kv_append_quant).  For query
+ * token j at p = L - T + j the candidates are the valid entries of
+ * pool_prev[b][j][0..pool_k) (-1 entries are padding; an entry at or beyond
+ * L - n_new, or beyond p, sets CSA2_ERR_DEVICE_BOUNDS and is dropped) and the
+ * new positions L - n_new .. p, all scored with this token's query as in
+ * csa2_index_full:
+ *     pool_idx[b][j]  <- the min(pool_k, |candidates|) best (the new pool),
+ *     topk_idx[b][j]  <- the min(top_k, |candidates|) best (a subset of it),
+ * each a set in unspecified order followed by -1 padding.  Pool entries are
+ * distinct positions.  pool_idx may be pool_prev (an in-place update).
+ * 0 <= n_new <= 16384 (a longer append is a new Full layer); other limits and
+ * layouts as in csa2_index_reindex.
+ */
+CSA2_API csa2_status csa2_index_pool_update(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
+                                            const float* head_w, int T, int H_I, const int32_t* pool_prev,
+                                            int pool_k, int n_new, int top_k, int32_t* pool_idx,
+                                            int32_t* topk_idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * csa2_index_reindex without a workspace, for callers that cannot allocate
  * device memory: code running while a framework captures a CUDA graph under a
  * no-allocation policy, plugins handed tensors but no allocator, or real-time

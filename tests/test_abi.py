@@ -173,3 +173,19 @@ def test_ring_arguments_rejected_on_host(lib):
     assert append(n_new=0) == csa2.OK                      # nothing to write: nothing launched
     assert lib.csa2_ring_append(ctypes.byref(fake_cache(dim=100)), 0x90000, i64(128), 0xA0000, 0xB0000, 4,
                                 None) == csa2.ERR_INVALID_ARG
+
+
+def test_pool_update_arguments_rejected_on_host(lib):
+    c = fake_cache()
+
+    def call(n_new=8, pool_k=512, top_k=64, out=0x90000, prev=0x60000):
+        return lib.csa2_index_pool_update(ctypes.byref(c), 0x40000, csa2.BF16, 0x50000, 1, 32, prev, pool_k, n_new,
+                                          top_k, out, 0x70000, 0x80000, 1 << 40, None)
+
+    assert call(n_new=-1) == csa2.ERR_INVALID_ARG
+    assert call(n_new=16385) == csa2.ERR_INVALID_ARG
+    assert call(out=None) == csa2.ERR_INVALID_ARG
+    assert call(out=0x90008) == csa2.ERR_INVALID_ARG
+    assert call(prev=None) == csa2.ERR_INVALID_ARG
+    assert call(top_k=600) == csa2.ERR_INVALID_ARG
+    assert call(pool_k=16385) == csa2.ERR_INVALID_ARG
