@@ -450,6 +450,8 @@ def run_ours(args, world, rank):
     # the append-time pool update of an in-flight request (its pool kept current
     # as tokens are appended), for one and for 64 appended positions
     pool_update = pool_update_line(w, lens, stack, ws, reps, stream)
+    # prefill / verification of 64 query tokens through the same stack
+    prefill = prefill_line(w, lens, seed, reps, stream, world, T=64)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -502,6 +504,7 @@ def run_ours(args, world, rank):
             "cpu_baseline": cpu,
             "local_window": local,
             "pool_update": pool_update,
+            "prefill": prefill,
             "workloads": extra,
         }
         line["roofline"]["step_frac_of_8TBps"] = round(line["step_bytes_algorithmic"] / (ms_step / 1e3) / 8e12, 4)
@@ -577,6 +580,57 @@ def pool_update_line(w, lens, stack, ws, reps, stream):
                                    "updates_per_s": round(n_q / (ms / 1e3), 1),
                                    "algorithmic_bytes_per_call": n_q * (w.pool_k + n_new) * key}
     return out
+
+
+def prefill_line(w, lens, seed, reps, stream, world, T):
+    """The stack for T query tokens per sequence (the last T positions, as in
+    verifying T drafted tokens or a prefill chunk) through csa2_prefill_layer,
+    one CUDA graph per replica; token-layer steps per second."""
+    import dataclasses
+    import fp4_sparse_attention_csa2_b200 as csa2
+    wt = dataclasses.replace(w, T=T)
+    layers = [{k: v.cuda() for k, v in wl.layer_queries(wt, l, seed).items()} for l in range(len(w.pattern))]
+    B = w.batch
+    n = csa2.prefill_workspace_bytes(reps[0], T, w.H, w.H_I, w.pool_k, w.top_k, w.window)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    csa2.workspace_init(ws)
+    pool = torch.zeros((B, T, w.pool_k), dtype=torch.int32, device="cuda")
+    topk = torch.zeros((B, T, w.top_k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, T, w.H, w.D), dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, T, w.H), dtype=torch.float32, device="cuda")
+    modes = [{"F": csa2.FULL, "R": csa2.REINDEX, "U": csa2.REUSE}[m] for m in w.pattern]
+
+    def step(c):
+        for L, m in zip(layers, modes):
+            idx = m != csa2.REUSE
+            csa2.prefill_layer(c, m, L["q"], topk, out, ws, w.window, q_idx=L["q_idx"] if idx else None,
+                               head_w=L["w"] if idx else None, pool_idx=pool, lse=lse, pool_k=w.pool_k,
+                               H_I=w.H_I)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(reps[i % len(reps)])
+    stream.synchronize()
+    st = csa2.read_device_status(ws, stream)
+    if st != csa2.OK:
+        raise RuntimeError("prefill: device status after warm-up: " + csa2.status_string(st))
+    graphs = []
+    for r in reps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            step(r)
+        graphs.append(g)
+    times = replay_regions(graphs, 3, stream, world, min_total_s=0.3, min_reps=3)
+    ms = statistics.median(times) / 3
+    st = csa2.read_device_status(ws, stream)
+    if st != csa2.OK:
+        raise RuntimeError("prefill: device status after timing: " + csa2.status_string(st))
+    del graphs
+    torch.cuda.empty_cache()
+    return {"query_tokens": T, "ms_per_step": round(ms, 4),
+            "token_layer_steps_per_s": round(world * B * T * len(w.pattern) / (ms / 1e3), 1),
+            "chunk_tokens": min(T, 128 // ((w.H_I + 15) // 16 * 16)),
+            "path": "csa2_prefill_layer per layer: the tokens in chunks through the decode kernels, causal per token"}
 
 
 def step_bytes(w, lens, local=False):

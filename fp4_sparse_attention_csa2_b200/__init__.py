@@ -22,7 +22,7 @@ ABI_FUNCTIONS = (
     "csa2_workspace_bytes", "csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
     "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update", "csa2_sparse_swa_attn",
     "csa2_ring_append",
-    "csa2_sparse_swa_attn_local", "csa2_layer_step",
+    "csa2_sparse_swa_attn_local", "csa2_layer_step", "csa2_prefill_workspace_bytes", "csa2_prefill_layer",
     "csa2_read_device_status", "csa2_status_string", "csa2_debug_set_wait_limit", "csa2_debug_default_wait_limit",
 )
 
@@ -79,6 +79,9 @@ def lib():
         L.csa2_sparse_swa_attn_local.argtypes = [cp, vp, ctypes.c_int64, vp, i32, i32, vp, i32, i32, ctypes.c_float,
                                                  vp, vp, vp, sz, vp]
         L.csa2_layer_step.argtypes = [cp, ctypes.POINTER(csa2_layer_args), vp, sz, vp]
+        L.csa2_prefill_workspace_bytes.restype = sz
+        L.csa2_prefill_workspace_bytes.argtypes = [cp, i32, i32, i32, i32, i32, i32]
+        L.csa2_prefill_layer.argtypes = [cp, ctypes.POINTER(csa2_layer_args), vp, sz, vp]
         L.csa2_read_device_status.argtypes = [vp, vp]
         L.csa2_status_string.restype = ctypes.c_char_p
         L.csa2_status_string.argtypes = [i32]
@@ -88,7 +91,7 @@ def lib():
         for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
                      "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update",
                      "csa2_sparse_swa_attn", "csa2_ring_append", "csa2_sparse_swa_attn_local",
-                     "csa2_layer_step", "csa2_read_device_status",
+                     "csa2_layer_step", "csa2_prefill_layer", "csa2_read_device_status",
                      "csa2_debug_set_wait_limit"):
             getattr(L, name).restype = i32
         _lib = L
@@ -279,6 +282,28 @@ def layer_step(cache, mode, q, topk_idx, out, ws, window, q_idx=None, head_w=Non
                         0 if ring is None else ring.shape[1])
     _check(lib().csa2_layer_step(cache.ref, ctypes.byref(a), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "layer_step")
+
+
+def prefill_workspace_bytes(cache, T, H, H_I, pool_k, top_k, window):
+    n = lib().csa2_prefill_workspace_bytes(cache.ref, T, H, H_I, pool_k, top_k, window)
+    if n == 0:
+        raise CSA2Error(ERR_INVALID_ARG, "prefill_workspace_bytes")
+    return n
+
+
+def prefill_layer(cache, mode, q, topk_idx, out, ws, window, q_idx=None, head_w=None, pool_idx=None, lse=None,
+                  pool_k=0, sm_scale=0.0, ring=None, H_I=None, stream=None):
+    """One layer for all T query tokens of q [B, T, H, dim] (any T), in
+    chunks; arguments as layer_step, plus the stack's indexer head count H_I
+    (taken from q_idx when given; required for Reuse layers)."""
+    B, T, H, _ = q.shape
+    H_I = q_idx.shape[2] if q_idx is not None else H_I
+    a = csa2_layer_args(mode, _addr(q), _addr(q_idx), _qdt(q_idx) if q_idx is not None else BF16, _addr(head_w),
+                        T, H, H_I, pool_k or (pool_idx.shape[-1] if pool_idx is not None else 0), topk_idx.shape[-1],
+                        window, sm_scale, _addr(pool_idx), _addr(topk_idx), _addr(out), _addr(lse), _addr(ring),
+                        0 if ring is None else ring.shape[1])
+    _check(lib().csa2_prefill_layer(cache.ref, ctypes.byref(a), _p(ws), ws.numel() * ws.element_size(),
+                                    _stream(stream)), "prefill_layer")
 
 
 def read_device_status(ws, stream=None):

@@ -237,6 +237,32 @@ bool ring_ok(const void* ring, int64_t ring_len, int T, int window) {
     return ring && aligned16(ring) && ring_len >= 1 && ring_len >= (int64_t)window + T - 1 && ring_len <= ((int64_t)1 << 30);
 }
 
+// Prefill: tokens per chunk, so that every chunk fits the single-step limits
+// (T * H_I <= 256 and the tensor-core scorer's 2 T HP <= 256 columns).
+int prefill_chunk(int T, int H_I) {
+    const int HP = (H_I + 15) / 16 * 16;
+    int c = 128 / (HP > 0 ? HP : 16);
+    if (c * H_I > 256) c = 256 / H_I;
+    if (c < 1) c = 1;
+    return c < T ? c : T;
+}
+
+// A cache view of sequence b whose length is the device int32 at `len`.
+csa2_cache seq_view(const csa2_cache* c, int b, const int32_t* len) {
+    csa2_cache v = *c;
+    v.batch = 1;
+    v.seq_lens = len;
+    if (c->page_table) {
+        v.page_table = c->page_table + (int64_t)b * c->max_pages;
+    } else {
+        const int64_t key_bytes = c->idx_key_dtype == CSA2_E4M3 ? c->idx_dim : 4 * c->idx_dim;
+        v.kv_rows = static_cast<uint8_t*>(c->kv_rows) + (int64_t)b * c->seq_stride_slots * c->row_stride;
+        v.idx_keys = static_cast<uint8_t*>(c->idx_keys) + (int64_t)b * c->seq_stride_slots * key_bytes;
+        v.n_slots = c->seq_stride_slots;
+    }
+    return v;
+}
+
 }  // namespace
 
 extern "C" {
@@ -432,6 +458,68 @@ csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* a, v
                                           a->window, a->sm_scale, a->out, a->lse, ws, ws_bytes, stream);
     return csa2_sparse_swa_attn(cache, a->q, a->T, a->H, a->topk_idx, a->top_k, a->window, a->sm_scale, a->out, a->lse,
                                 ws, ws_bytes, stream);
+}
+
+size_t csa2_prefill_workspace_bytes(const csa2_cache* cache, int T, int H, int H_I, int pool_k, int top_k,
+                                    int window) {
+    if (check_cache(cache) != CSA2_OK || T < 1 || H_I < 1 || H_I > 64) return 0;
+    const csa2_cache v = seq_view(cache, 0, cache->seq_lens);
+    Layout L;
+    if (!make_layout(&v, prefill_chunk(T, H_I), H, pool_k, top_k, window, &L)) return 0;
+    return L.total + 256;                               // + the chunk's sequence length
+}
+
+csa2_status csa2_prefill_layer(const csa2_cache* cache, const csa2_layer_args* a, void* ws, size_t ws_bytes,
+                               void* stream) {
+    csa2_status s = check_cache(cache);
+    if (s != CSA2_OK) return s;
+    if (!a || a->T < 1 || !ws || !aligned16(ws)) return CSA2_ERR_INVALID_ARG;
+    const bool idx = a->mode == CSA2_FULL || a->mode == CSA2_REINDEX;
+    if (!idx && a->mode != CSA2_REUSE) return CSA2_ERR_INVALID_ARG;
+    // the stack's indexer heads set the chunk size, in every mode (a Reuse
+    // layer runs in the same chunks as the index layers, on the same workspace)
+    const int H_I = a->H_I;
+    if (H_I < 1 || H_I > 64 || a->H < 1) return CSA2_ERR_INVALID_ARG;
+    const int T = a->T, tc = prefill_chunk(T, H_I);
+    const csa2_cache v0 = seq_view(cache, 0, cache->seq_lens);
+    Layout L;
+    if (!make_layout(&v0, tc, a->H, idx ? a->pool_k : (a->top_k > 0 ? a->top_k : 1), a->top_k, a->window, &L))
+        return CSA2_ERR_INVALID_ARG;
+    const size_t need = csa2_prefill_workspace_bytes(cache, T, a->H, H_I, idx ? a->pool_k : (a->top_k > 0 ? a->top_k : 1),
+                                                     a->top_k, a->window);
+    if (need == 0 || ws_bytes < need) return CSA2_ERR_INVALID_ARG;
+    int32_t* len = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + need - 256);
+    const size_t chunk_ws = need - 256;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int D = cache->dim;
+    const size_t qi_elem = a->q_idx_dtype == CSA2_F32 ? 4 : 2;
+    for (int b = 0; b < cache->batch; ++b) {
+        for (int k0 = 0; k0 < T; k0 += tc) {
+            // every chunk has tc tokens, so that the workspace layout (and its
+            // sections that stay zero between calls) is the same for all; the
+            // last one is moved back to end at token T - 1 and recomputes a few
+            // tokens with the same inputs
+            const int c = tc;
+            const int j0 = k0 + tc <= T ? k0 : T - tc;
+            // the chunk's tokens are the last c positions of a sequence of length L_b - (T - j0 - c)
+            if (launch_chunk_len(cache->seq_lens + b, T - j0 - c, len, st) != cudaSuccess) return CSA2_ERR_CUDA;
+            const csa2_cache v = seq_view(cache, b, len);
+            const int64_t tok = (int64_t)b * T + j0;     // first (sequence, token) row of the chunk
+            csa2_layer_args ca = *a;
+            ca.T = c;
+            ca.q = static_cast<const uint16_t*>(a->q) + tok * a->H * D;
+            if (a->q_idx) ca.q_idx = static_cast<const char*>(a->q_idx) + tok * H_I * cache->idx_dim * qi_elem;
+            if (a->head_w) ca.head_w = a->head_w + tok * H_I;
+            if (a->pool_idx) ca.pool_idx = a->pool_idx + tok * a->pool_k;
+            ca.topk_idx = a->topk_idx ? a->topk_idx + tok * a->top_k : nullptr;
+            ca.out = a->out + tok * a->H * D;
+            ca.lse = a->lse ? a->lse + tok * a->H : nullptr;
+            if (a->ring) ca.ring = static_cast<const uint16_t*>(a->ring) + (int64_t)b * a->ring_len * D;
+            s = csa2_layer_step(&v, &ca, ws, chunk_ws, stream);
+            if (s != CSA2_OK) return s;
+        }
+    }
+    return CSA2_OK;
 }
 
 csa2_status csa2_read_device_status(void* ws, void* stream) {

@@ -184,7 +184,17 @@ k_pool_candidates(DevCache c, int T, const int32_t* __restrict__ pool_prev, int 
     ids[(int64_t)seg * m + i] = t;
 }
 
+__global__ void k_chunk_len(const int32_t* __restrict__ seq_len, int drop, int32_t* __restrict__ len) {
+    pdl_begin();
+    const int32_t v = *seq_len - drop;
+    *len = v > 0 ? v : 0;
+}
+
 }  // namespace
+
+cudaError_t launch_chunk_len(const int32_t* seq_len, int drop, int32_t* len, cudaStream_t st) {
+    return launch_pdl(k_chunk_len, dim3(1), dim3(1), 0, st, seq_len, drop, len);
+}
 
 cudaError_t launch_pool_candidates(const DevCache& c, int T, const int32_t* pool_prev, int pool_k, int n_new,
                                    int32_t* ids, uint32_t* status, cudaStream_t st) {

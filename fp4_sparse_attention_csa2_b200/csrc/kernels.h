@@ -77,6 +77,8 @@ cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const
 // pool's entries (-1 kept; an entry at or beyond the first appended position
 // L - n_new, or beyond the token's position, is flagged and dropped), then the
 // appended positions L - n_new .. L - 1 (those beyond the token's position -1).
+// *len = max(0, *seq_len - drop): the length of a sequence cut back by `drop` positions.
+cudaError_t launch_chunk_len(const int32_t* seq_len, int drop, int32_t* len, cudaStream_t st);
 cudaError_t launch_pool_candidates(const DevCache& c, int T, const int32_t* pool_prev, int pool_k, int n_new,
                                    int32_t* ids, uint32_t* status, cudaStream_t st);
 

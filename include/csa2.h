@@ -317,6 +317,29 @@ CSA2_API csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_a
                             size_t ws_bytes, void* stream);
 
 /*
+ * Prefill and verification: one layer (as csa2_layer_step) for T query tokens
+ * of every sequence, any T >= 1 ([TLDR] paragraphs 2-3: the layers run over
+ * the prompt as well as over decoded tokens; [HN] summary: prefill compute).
+ * Token j of sequence b sits at p = seq_lens[b] - T + j (its row appended
+ * beforehand) and sees positions <= p only, exactly as in a decode step; the
+ * arguments and output layouts are those of csa2_layer_step with args->T = T
+ * (out [batch][T][H][dim], pool_idx [batch][T][pool_k], ...; a ring is
+ * [batch][ring_len][dim] with ring_len >= window + min(T, chunk) - 1), except
+ * that args->H_I is required in every mode, CSA2_REUSE included: the stack's
+ * indexer heads set the chunk size.  The
+ * tokens run in chunks of min(T, 128 / HP) tokens (HP = H_I rounded up to 16;
+ * 4 for 32 indexer heads), one sequence at a time; the last chunk of a
+ * sequence is moved back to end at token T - 1 and recomputes a few tokens.
+ * ws is a workspace of csa2_prefill_workspace_bytes bytes (0 on invalid
+ * arguments), cleared once with csa2_workspace_init; its status word is read
+ * with csa2_read_device_status as usual.
+ */
+CSA2_API size_t csa2_prefill_workspace_bytes(const csa2_cache* cache, int T, int H, int H_I, int pool_k, int top_k,
+                                             int window);
+CSA2_API csa2_status csa2_prefill_layer(const csa2_cache* cache, const csa2_layer_args* args, void* ws,
+                                        size_t ws_bytes, void* stream);
+
+/*
  * Synchronise `stream`, then return the sticky device status recorded in the
  * workspace (CSA2_OK, CSA2_ERR_DEVICE_BOUNDS or CSA2_ERR_TIMEOUT; the first
  * error class found in that order of severity: TIMEOUT, then BOUNDS) and clear

@@ -189,3 +189,23 @@ def test_pool_update_arguments_rejected_on_host(lib):
     assert call(prev=None) == csa2.ERR_INVALID_ARG
     assert call(top_k=600) == csa2.ERR_INVALID_ARG
     assert call(pool_k=16385) == csa2.ERR_INVALID_ARG
+
+
+def test_prefill_workspace_and_arguments(lib):
+    c = fake_cache()
+    n1 = lib.csa2_prefill_workspace_bytes(ctypes.byref(c), 4, 64, 32, 16384, 2048, 128)
+    n2 = lib.csa2_prefill_workspace_bytes(ctypes.byref(c), 8192, 64, 32, 16384, 2048, 128)
+    # the workspace holds one chunk of four tokens of one sequence, whatever T is
+    assert n1 == n2 > 0
+    assert lib.csa2_prefill_workspace_bytes(ctypes.byref(c), 0, 64, 32, 16384, 2048, 128) == 0
+    assert lib.csa2_prefill_workspace_bytes(ctypes.byref(c), 4, 64, 65, 16384, 2048, 128) == 0
+    a = csa2.csa2_layer_args(mode=csa2.REUSE, q=0x40000, T=0, H=64, H_I=32, top_k=2048, window=128,
+                             topk_idx=0x60000, out=0x70000)
+    assert lib.csa2_prefill_layer(ctypes.byref(c), ctypes.byref(a), 0x80000, n1, None) == csa2.ERR_INVALID_ARG
+    a.T = 16
+    assert lib.csa2_prefill_layer(ctypes.byref(c), ctypes.byref(a), 0x80000, 1024, None) == csa2.ERR_INVALID_ARG
+    a.H_I = 0                                  # the chunk size needs the stack's indexer heads
+    assert lib.csa2_prefill_layer(ctypes.byref(c), ctypes.byref(a), 0x80000, n1, None) == csa2.ERR_INVALID_ARG
+    a.H_I = 32
+    a.mode = 7
+    assert lib.csa2_prefill_layer(ctypes.byref(c), ctypes.byref(a), 0x80000, n1, None) == csa2.ERR_INVALID_ARG
