@@ -397,29 +397,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
         const int c0 = cg * NV;
         float z[NV];
         if (ok) {
-            // S = the sum of the issuers' partial products over K
+            // S = the sum of the issuers' partial products over K: every
+            // accumulator's columns in flight at once, one wait
+            uint32_t rr[kIssuers][NV];
+#pragma unroll
+            for (int a = 0; a < kIssuers; ++a) {
+                if (a >= nacc) break;                    // nacc is uniform over the CTA
+                const uint32_t col = trow + (uint32_t)(a * HG + c0);
+                if constexpr (NV == 4) tc::tmem_ld4_nowait(col, rr[a]);
+                else if constexpr (NV == 8) tc::tmem_ld8_nowait(col, rr[a]);
+                else tc::tmem_ld16_nowait(col, rr[a]);
+            }
+            tc::tmem_ld_wait();
             float v[NV];
 #pragma unroll
             for (int i = 0; i < NV; ++i) v[i] = 0.0f;
 #pragma unroll
             for (int a = 0; a < kIssuers; ++a) {
                 if (a >= nacc) break;
-                float u[NV];
-                const uint32_t col = trow + (uint32_t)(a * HG + c0);
-                if constexpr (NV == 4) {
-                    uint32_t rr[4];
-                    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(rr[0]), "=r"(rr[1]), "=r"(rr[2]), "=r"(rr[3]) : "r"(col));
-                    tc::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) u[i] = __uint_as_float(rr[i]);
-                } else if constexpr (NV == 8) {
-                    tc::tmem_ld8(col, u);
-                } else {
-                    tc::tmem_ld16(col, u);
-                }
-#pragma unroll
-                for (int i = 0; i < NV; ++i) v[i] += u[i];
+                for (int i = 0; i < NV; ++i) v[i] += __uint_as_float(rr[a][i]);
             }
 #pragma unroll
             for (int i = 0; i < NV; ++i) {
