@@ -365,7 +365,8 @@ csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_
     float* ps = at<float>(ws, L.pscores);
     if (reindex_tc_supported(d, H_I))
         return cuda_status(launch_reindex_tc(d, q_idx, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx, ps,
-                                             at<uint32_t>(ws, L.rx_cnt), status, st));
+                                             at<uint32_t>(ws, L.rx_cnt), at<uint32_t>(ws, L.hist),
+                                             at<uint32_t>(ws, L.cnt), status, st));
     cudaError_t e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, pool_idx, pool_k, ps, status, st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
     return topk_from_pool(cache, L, ws, ps, pool_k, 0, pool_idx, pool_k, top_k, topk_idx, T, st);

@@ -66,9 +66,12 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
 // top_k of each segment's pool, in one kernel; counters[seg] are zero on entry
 // and on exit.
 bool reindex_tc_supported(const DevCache& c, int H_I);
+// grid_hist / grid_cnt (nullable): the segment histograms [nseg][3][2048] and
+// counters [nseg][kSelCounters] (zero between calls) of the grid-mode select.
 cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw, int T, int H_I,
                               const int32_t* pool, int pool_k, int top_k, int32_t* topk, float* scores,
-                              uint32_t* counters, uint32_t* status, cudaStream_t st);
+                              uint32_t* counters, uint32_t* grid_hist, uint32_t* grid_cnt, uint32_t* status,
+                              cudaStream_t st);
 
 // Pool rescoring: scores[seg * pool_k + i] for pool entry i of segment seg.
 cudaError_t launch_score_pool(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,

@@ -118,7 +118,7 @@ extern "C" csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const
     const DevCache d = dev_cache(cache);
     if (reindex_tc_supported(d, H_I)) {
         const cudaError_t e = launch_reindex_tc(d, q_idx, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx, scores,
-                                                counters, status, st);
+                                                counters, nullptr, nullptr, status, st);
         return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
     }
     cudaError_t e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, pool_idx, pool_k, scores, status,

@@ -22,10 +22,16 @@
 //   thread 0          two MMAs (K = 2 x 32, M = 128 entries, N = U x HP);
 //   warps 0..3        one entry per thread: read its U x HP columns of the
 //                     accumulator, write the score (NaN when not a candidate).
-// The CTA that finishes its segment last (an arrival counter after a memory
-// fence) reads the segment's pool_k scores back and selects the top_k in one
-// CTA (lsel.cuh), then clears the counter for the next call.
+// Grid mode (when every CTA of the launch fits on the GPU at once): the
+// segment's CTAs select the top_k together, each keeping its 128 keys in
+// registers, through three bounded segment barriers behind which the digit-1,
+// -2 and -3 histograms of the segment are complete (gsel.cuh), then claim
+// their outputs with one atomic per warp; the last CTA clears the histograms
+// and counters.  Otherwise the CTA that finishes its segment last (an arrival
+// counter after a memory fence) reads the segment's pool_k scores back and
+// selects the top_k in one CTA (lsel.cuh), then clears the counter.
 #include "common.cuh"
+#include "gsel.cuh"
 #include "kernels.h"
 #include "lsel.cuh"
 #include "tc.cuh"
@@ -49,6 +55,8 @@ struct Params {
     int32_t* topk;            // [B*T][top_k]
     float* scores;            // [B*T][pool_k] scratch
     uint32_t* counters;       // [B*T] arrival counters, zero between calls
+    uint32_t* grid_hist;      // grid mode: [B*T][3][2048] digit histograms, zero between calls (nullptr: last-CTA mode)
+    uint32_t* grid_cnt;       // grid mode: [B*T][kSelCounters] counters, zero between calls
     uint32_t* status;
     uint32_t wait_limit;      // tries of the wait that guards the epilogue (not of the drain)
     uint32_t tmem_cols;
@@ -62,12 +70,96 @@ struct __align__(1024) Smem {
     uint64_t mma_bar;
     uint32_t tmem_base;
     uint32_t last;
+    uint32_t flag;
+    uint32_t base[4];
+    gsel::Cut cut;
 };
 
 __device__ __forceinline__ float e4m3_round(float x, uint8_t* code) {
     const uint16_t c = cvt_e4m3x2(0.0f, x);
     *code = (uint8_t)(c & 0xFF);
     return e4m3_to_float(*code);
+}
+
+// The top_k of the segment's keys, selected by all its CTAs together; the
+// entry threads (tid < 128) hold one key each (0: not a candidate) and its
+// position `id`.
+__device__ void grid_topk(const Params& p, int seg, uint32_t key, int32_t id, Smem& sm) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const uint32_t C = gridDim.x;
+    uint32_t* h1 = p.grid_hist + (int64_t)seg * 3 * 2048;
+    uint32_t* h2 = h1 + 2048;
+    uint32_t* h3 = h2 + 2048;
+    uint32_t* cnt = p.grid_cnt + (int64_t)seg * kSelCounters;
+    uint32_t* bar = cnt + 8;
+    uint32_t* hc = sm.sel.hist;                     // a copy of one of the segment's histograms
+    const uint32_t limit = p.wait_limit * 64u;
+    uint32_t nbar = 0;
+    bool ok = true;
+    // level 1
+    if (key) atomicAdd(h1 + (key >> 21), 1u);
+    ok = gsel::seg_barrier(bar, ++nbar * C, limit, &sm.flag) && ok;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // every CTA is resident
+    gsel::load_hist<kThreads>(hc, h1, 2048);
+    const gsel::Cut c1 = gsel::threshold<kThreads>(hc, 0u, (uint32_t)p.top_k, sm.sel.wa, &sm.cut);
+    const bool take1 = c1.need == 0 || c1.eq == c1.need - c1.above;
+    if (blockIdx.x == 0)
+        for (int k = (int)c1.need + tid; k < p.top_k; k += kThreads) p.topk[(int64_t)seg * p.top_k + k] = -1;
+    // level 2: the elements of digit c1
+    if (key && !take1 && (key >> 21) == c1.c) atomicAdd(h2 + ((key >> 10) & 0x7FFu), 1u);
+    ok = gsel::seg_barrier(bar, ++nbar * C, limit, &sm.flag) && ok;
+    gsel::load_hist<kThreads>(hc, h2, 2048);
+    const uint32_t need2 = take1 ? 0u : c1.need - c1.above;
+    const gsel::Cut c2 = gsel::threshold<kThreads>(hc, need2, 0u, sm.sel.wa, &sm.cut);
+    const bool take2 = take1 || c2.eq == need2 - c2.above;
+    // level 3: the elements of digits (c1, c2)
+    const uint32_t pre = (c1.c << 11) | c2.c;
+    if (key && !take2 && (key >> 10) == pre) atomicAdd(h3 + (key & 0x3FFu), 1u);
+    ok = gsel::seg_barrier(bar, ++nbar * C, limit, &sm.flag) && ok;
+    gsel::load_hist<kThreads>(hc, h3, 2048);
+    const uint32_t need3 = take2 ? 0u : need2 - c2.above;
+    const gsel::Cut c3 = gsel::threshold<kThreads>(hc, need3, 0u, sm.sel.wa, &sm.cut);
+    // the cut as keys: every key >= lo is taken, and the first `ties` claimants of tie_key
+    uint32_t lo, tie_key = 0u, ties = 0u;
+    if (c1.need == 0) {
+        lo = 0xFFFFFFFFu;
+    } else if (take1) {
+        lo = c1.c << 21;
+    } else if (take2) {
+        lo = (c1.c << 21) | (c2.c << 10);
+    } else {
+        tie_key = (pre << 10) | c3.c;
+        lo = tie_key + 1u;
+        ties = need3 - c3.above;
+    }
+    if (threadIdx.x < kTile) {                       // warps 0..3: the entry threads
+        bool sel = key && key >= lo;
+        const bool tie = key && key == tie_key;
+        const uint32_t m = __ballot_sync(0xffffffffu, tie);
+        if (m) {
+            uint32_t base = 0;
+            const int leader = __ffs(m) - 1;
+            if (lane == leader) base = atomicAdd(cnt + 4, (uint32_t)__popc(m));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            sel = sel || (tie && base + __popc(m & ((1u << lane) - 1u)) < ties);
+        }
+        const uint32_t ms = __ballot_sync(0xffffffffu, sel);
+        uint32_t obase = 0;
+        if (ms && lane == 0) obase = atomicAdd(cnt + 0, (uint32_t)__popc(ms));
+        obase = __shfl_sync(0xffffffffu, obase, 0);
+        const uint32_t pos = obase + __popc(ms & ((1u << lane) - 1u));
+        if (sel && pos < (uint32_t)p.top_k) p.topk[(int64_t)seg * p.top_k + pos] = id;
+    }
+    if (!ok && tid == 0) flag(p.status, kStatusTimeout);
+    // the last CTA leaves the segment's histograms and counters zero
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sm.last = atomicAdd(bar, 1u) == (nbar + 1) * C - 1 ? 1u : 0u;
+    __syncthreads();
+    if (!sm.last) return;
+    __threadfence();
+    for (int k = tid; k < 3 * 2048; k += kThreads) h1[k] = 0u;
+    if (tid < kSelCounters) cnt[tid] = 0u;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) k_reindex_tc(const Params p) {
@@ -85,15 +177,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_reindex_tc(const Params p) {
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = sm.tmem_base;
-    pdl_begin();
+    // in grid mode the next kernel may launch only once every CTA of this one
+    // is resident (after the first segment barrier)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!p.grid_hist) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---- operands
     const int i = blockIdx.x * kTile + tid;         // this thread's pool entry (tid < 128)
     bool live = false;
+    int32_t t = -1;
     if (tid < kTile) {
         const int64_t L = seq_len(p.c, b, p.status);
         const int64_t pq = L - p.T + j;
-        int32_t t = i < p.pool_k ? __ldg(p.pool + (int64_t)seg * p.pool_k + i) : -1;
+        t = i < p.pool_k ? __ldg(p.pool + (int64_t)seg * p.pool_k + i) : -1;
         int64_t slot = -1;
         if (t >= 0) {
             if (t > pq) {
@@ -183,6 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_reindex_tc(const Params p) {
         tc::mma_commit(&sm.mma_bar);
     }
     bool ok = true;
+    uint32_t my_key = 0;                            // grid mode: this entry's key (0: not a candidate)
     if (warp < 4) {
         ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm.mma_bar, 0, p.wait_limit));
         tc::fence_after_sync();
@@ -214,8 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_reindex_tc(const Params p) {
             }
         }
         // every entry of the tile gets a value: NaN marks one that is not a candidate
-        if (i < p.pool_k)
-            p.scores[(int64_t)seg * p.pool_k + i] = (ok && live) ? s0 + s1 : __int_as_float(0x7fc00000);
+        const float sc = (ok && live) ? s0 + s1 : __int_as_float(0x7fc00000);
+        if (p.grid_hist) my_key = select_key(sc, i < p.pool_k && ok && live);
+        else if (i < p.pool_k) p.scores[(int64_t)seg * p.pool_k + i] = sc;
     }
     if (!ok && lane == 0) flag(p.status, kStatusTimeout);
     __threadfence();
@@ -227,6 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_reindex_tc(const Params p) {
         if (!ok) tc::mbar_wait(&sm.mma_bar, 0, tc::kWaitLimit);
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, p.tmem_cols);
+    }
+    if (p.grid_hist) {
+        grid_topk(p, seg, my_key, t, sm);
+        return;
     }
     if (tid == 0) sm.last = atomicAdd(p.counters + seg, 1u) == gridDim.x - 1 ? 1u : 0u;
     __syncthreads();
@@ -259,7 +361,8 @@ bool reindex_tc_supported(const DevCache& c, int H_I) {
 
 cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw, int T, int H_I,
                               const int32_t* pool, int pool_k, int top_k, int32_t* topk, float* scores,
-                              uint32_t* counters, uint32_t* status, cudaStream_t st) {
+                              uint32_t* counters, uint32_t* grid_hist, uint32_t* grid_cnt, uint32_t* status,
+                              cudaStream_t st) {
     Params p;
     p.c = c;
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -274,6 +377,8 @@ cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw,
     p.topk = topk;
     p.scores = scores;
     p.counters = counters;
+    p.grid_hist = nullptr;
+    p.grid_cnt = nullptr;
     p.status = status;
     p.wait_limit = wait_limit();
     uint32_t cols = 32;
@@ -283,6 +388,22 @@ cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw,
     cudaError_t e = cudaFuncSetAttribute(k_reindex_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned tiles = (unsigned)((pool_k + kTile - 1) / kTile);
+    if (grid_hist && grid_cnt) {
+        // grid mode when every CTA of the launch fits on the GPU at once
+        static int64_t cap = -1;
+        if (cap < 0) {
+            int dev = 0, sms = 0, per = 0;
+            cap = 0;
+            if (cudaGetDevice(&dev) == cudaSuccess &&
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_reindex_tc, kThreads, smem) == cudaSuccess)
+                cap = (int64_t)sms * per;
+        }
+        if ((int64_t)tiles * c.batch * T <= cap) {
+            p.grid_hist = grid_hist;
+            p.grid_cnt = grid_cnt;
+        }
+    }
     return launch_pdl(k_reindex_tc, dim3(tiles, (unsigned)(c.batch * T)), dim3(kThreads), smem, st, p);
 }
 

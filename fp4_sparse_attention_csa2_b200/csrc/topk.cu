@@ -25,6 +25,7 @@
 //     brackets the cutoff from a sample, compacts the elements inside the
 //     bracket and resolves them by radix select in shared memory (lsel.cuh).
 #include "common.cuh"
+#include "gsel.cuh"
 #include "kernels.h"
 #include "lsel.cuh"
 
@@ -872,30 +873,10 @@ cudaError_t launch_local_e(const SelSrc& src, int nseg, int n_a, int32_t* out_a,
 // launch only after barrier A, when every CTA of the grid has arrived.
 constexpr int kGridThreads = 1024;
 
-// Arrive at the segment barrier (counter ctr) and wait, bounded, until it
-// counts `target` arrivals; false when the wait gave up.
-__device__ __forceinline__ bool seg_barrier(uint32_t* ctr, uint32_t target, uint32_t limit, uint32_t* s_flag) {
-    __threadfence();                                       // this thread's histogram updates, then the arrival
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        atomicAdd(ctr, 1u);
-        uint32_t v = 0;
-        for (uint32_t i = 0;; ++i) {
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-            if (v >= target || i >= limit) break;
-            if (i >= 64) __nanosleep(128);                 // poll back to back at first
-        }
-        *s_flag = v >= target ? 1u : 0u;
-    }
-    __syncthreads();
-    return *s_flag != 0u;
-}
+using gsel::seg_barrier;
 
-// n words of a histogram written by other CTAs into shared memory (L2 reads).
 __device__ __forceinline__ void load_hist(uint32_t* dst, const uint32_t* src, int n) {
-    for (int i = threadIdx.x; i < n / 4; i += kGridThreads)
-        reinterpret_cast<uint4*>(dst)[i] = __ldcg(reinterpret_cast<const uint4*>(src) + i);
-    __syncthreads();
+    gsel::load_hist<kGridThreads>(dst, src, n);
 }
 
 template <int E>
