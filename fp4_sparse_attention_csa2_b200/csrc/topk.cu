@@ -901,14 +901,25 @@ k_sel_grid(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float* 
     const uint32_t limit = wait_limit * 64u;              // a try sleeps 0.1-0.3 us: a fraction of a second by default
     const int64_t nvalid = n_valid_positions(src, seg);
     const int64_t base = (int64_t)blockIdx.x * kGridThreads * E;
-    uint32_t key[E];
+    // every score load in flight before anything else (clamped, so that no load
+    // is conditional); with the scorer's histogram the level-1 plan is worked
+    // out while they land
+    float raw[E];
 #pragma unroll
     for (int k = 0; k < E; ++k) {
         const int64_t i = base + (int64_t)k * kGridThreads + tid;
-        const bool v = i < nvalid;
-        key[k] = select_key(v ? __ldcg(src.vals + seg * src.vals_stride + i) : 0.0f, v);   // a valid key is never 0
+        raw[k] = __ldcg(src.vals + seg * src.vals_stride + (i < nvalid ? i : 0));
     }
     for (int i = tid; i < 2 * kRadixBins; i += kGridThreads) (&h[0][0])[i] = 0u;
+    Plan1 pa, pb;
+    if (hist_ready) {
+        load_hist(&hc[0][0], h1g, kRadixBins);
+        plans_level1<kGridThreads>(&hc[0][0], (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr, pa, pb);
+    }
+    uint32_t key[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k)   // a valid key is never 0
+        key[k] = select_key(raw[k], base + (int64_t)k * kGridThreads + tid < nvalid);
     uint32_t nbar = 0;
     bool ok = true;
     // flush this CTA's histograms (the nonzero bins) into the segment's and clear them
@@ -929,12 +940,11 @@ k_sel_grid(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float* 
             if (key[k]) atomicAdd(&h[0][digit(key[k], 1)], 1u);
         flush(h1g, kRadixBins);
         ok = seg_barrier(bar, ++nbar * C, limit, &s_misc[3]) && ok;
+        load_hist(&hc[0][0], h1g, kRadixBins);
+        plans_level1<kGridThreads>(&hc[0][0], (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr, pa, pb);
     }
 
     // ---- level 1
-    load_hist(&hc[0][0], h1g, kRadixBins);
-    Plan1 pa, pb;
-    plans_level1<kGridThreads>(&hc[0][0], (uint32_t)n_a, (uint32_t)n_b, s_wsum, s_thr, pa, pb);
     int32_t* oa = out_a + (int64_t)seg * stride_a;
     int32_t* ob = out_b ? out_b + (int64_t)seg * stride_b : nullptr;
     float* va = vals_a ? vals_a + (int64_t)seg * stride_a : nullptr;
