@@ -389,7 +389,10 @@ csa2_status csa2_index_pool_update(const csa2_cache* cache, const void* q_idx, c
     int32_t* ids = at<int32_t>(ws, L.upd_ids);
     float* sc = at<float>(ws, L.upd_scores);
     cudaError_t e = launch_pool_candidates(d, T, pool_prev, pool_k, n_new, ids, status, st);
-    if (e == cudaSuccess) e = launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, ids, m, sc, status, st);
+    if (e == cudaSuccess)
+        e = reindex_tc_supported(d, H_I) ? launch_reindex_tc_scores(d, q_idx, head_w, T, H_I, ids, m, sc, status, st)
+                                         : launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, T, H_I, ids, m, sc,
+                                                             status, st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
     SelSrc src;
     src.vals = sc;

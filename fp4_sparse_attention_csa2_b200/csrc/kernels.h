@@ -66,6 +66,10 @@ cudaError_t launch_score_full_tc(const DevCache& c, const void* q, const float* 
 // top_k of each segment's pool, in one kernel; counters[seg] are zero on entry
 // and on exit.
 bool reindex_tc_supported(const DevCache& c, int H_I);
+// The same kernel's scores alone: scores[seg][i] for the pool entries (NaN
+// for entries that are not candidates), no selection.
+cudaError_t launch_reindex_tc_scores(const DevCache& c, const void* q, const float* hw, int T, int H_I,
+                                     const int32_t* pool, int pool_k, float* scores, uint32_t* status, cudaStream_t st);
 // grid_hist / grid_cnt (nullable): the segment histograms [nseg][3][2048] and
 // counters [nseg][kSelCounters] (zero between calls) of the grid-mode select.
 cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw, int T, int H_I,

@@ -57,6 +57,7 @@ struct Params {
     uint32_t* counters;       // [B*T] arrival counters, zero between calls
     uint32_t* grid_hist;      // grid mode: [B*T][3][2048] digit histograms, zero between calls (nullptr: last-CTA mode)
     uint32_t* grid_cnt;       // grid mode: [B*T][kSelCounters] counters, zero between calls
+    int scores_only;          // write the scores and stop (no selection)
     uint32_t* status;
     uint32_t wait_limit;      // tries of the wait that guards the epilogue (not of the drain)
     uint32_t tmem_cols;
@@ -330,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_reindex_tc(const Params p) {
         grid_topk(p, seg, my_key, t, sm);
         return;
     }
+    if (p.scores_only) return;
     if (tid == 0) sm.last = atomicAdd(p.counters + seg, 1u) == gridDim.x - 1 ? 1u : 0u;
     __syncthreads();
     if (!sm.last) return;
@@ -379,6 +381,7 @@ cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw,
     p.counters = counters;
     p.grid_hist = nullptr;
     p.grid_cnt = nullptr;
+    p.scores_only = 0;
     p.status = status;
     p.wait_limit = wait_limit();
     uint32_t cols = 32;
@@ -404,6 +407,37 @@ cudaError_t launch_reindex_tc(const DevCache& c, const void* q, const float* hw,
             p.grid_cnt = grid_cnt;
         }
     }
+    return launch_pdl(k_reindex_tc, dim3(tiles, (unsigned)(c.batch * T)), dim3(kThreads), smem, st, p);
+}
+
+cudaError_t launch_reindex_tc_scores(const DevCache& c, const void* q, const float* hw, int T, int H_I,
+                                     const int32_t* pool, int pool_k, float* scores, uint32_t* status, cudaStream_t st) {
+    Params p;
+    p.c = c;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.hw = hw;
+    p.T = T;
+    p.H_I = H_I;
+    p.HP = (H_I + 15) / 16 * 16;
+    p.U = 3 * p.HP <= 256 ? 3 : 2;
+    p.pool = pool;
+    p.pool_k = pool_k;
+    p.top_k = 0;
+    p.topk = nullptr;
+    p.scores = scores;
+    p.counters = nullptr;
+    p.grid_hist = nullptr;
+    p.grid_cnt = nullptr;
+    p.scores_only = 1;
+    p.status = status;
+    p.wait_limit = wait_limit();
+    uint32_t cols = 32;
+    while (cols < (uint32_t)(p.U * p.HP)) cols <<= 1;
+    p.tmem_cols = cols;
+    const size_t smem = sizeof(Smem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_reindex_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned tiles = (unsigned)((pool_k + kTile - 1) / kTile);
     return launch_pdl(k_reindex_tc, dim3(tiles, (unsigned)(c.batch * T)), dim3(kThreads), smem, st, p);
 }
 

@@ -879,7 +879,9 @@ __device__ __forceinline__ void load_hist(uint32_t* dst, const uint32_t* src, in
     gsel::load_hist<kGridThreads>(dst, src, n);
 }
 
-template <int E>
+// IDS: the elements are a list of positions (src.ids) with their values at
+// the same index (src.gather == 0), as a pool update's candidates are.
+template <int E, bool IDS>
 __global__ void __launch_bounds__(kGridThreads, 1)
 k_sel_grid(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float* __restrict__ vals_a, int64_t stride_a,
            int n_b, int32_t* __restrict__ out_b, int64_t stride_b, int hist_ready, uint32_t wait_limit) {
@@ -905,10 +907,14 @@ k_sel_grid(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float* 
     // is conditional); with the scorer's histogram the level-1 plan is worked
     // out while they land
     float raw[E];
+    int32_t idv[IDS ? E : 1];
+    const int64_t n_items = IDS ? src.n : nvalid;
 #pragma unroll
     for (int k = 0; k < E; ++k) {
         const int64_t i = base + (int64_t)k * kGridThreads + tid;
-        raw[k] = __ldcg(src.vals + seg * src.vals_stride + (i < nvalid ? i : 0));
+        const int64_t ic = i < n_items ? i : 0;
+        if (IDS) idv[k] = __ldcg(src.ids + seg * src.ids_stride + ic);
+        raw[k] = __ldcg(src.vals + seg * src.vals_stride + ic);
     }
     for (int i = tid; i < 2 * kRadixBins; i += kGridThreads) (&h[0][0])[i] = 0u;
     Plan1 pa, pb;
@@ -918,8 +924,11 @@ k_sel_grid(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float* 
     }
     uint32_t key[E];
 #pragma unroll
-    for (int k = 0; k < E; ++k)   // a valid key is never 0
-        key[k] = select_key(raw[k], base + (int64_t)k * kGridThreads + tid < nvalid);
+    for (int k = 0; k < E; ++k) {   // a valid key is never 0
+        const int64_t i = base + (int64_t)k * kGridThreads + tid;
+        const bool v = IDS ? i < n_items && idv[k] >= 0 && idv[k] < nvalid : i < nvalid;
+        key[k] = select_key(raw[k], v);
+    }
     uint32_t nbar = 0;
     bool ok = true;
     // flush this CTA's histograms (the nonzero bins) into the segment's and clear them
@@ -1071,7 +1080,7 @@ k_sel_grid(SelSrc src, SelWork wk, int n_a, int32_t* __restrict__ out_a, float* 
     uint32_t oa_pos = s_misc[0] + field16(pre, 0), ob_pos = s_misc[1] + field16(pre, 1);
 #pragma unroll
     for (int k = 0; k < E; ++k) {
-        const int32_t id = (int32_t)(base + (int64_t)k * kGridThreads + tid);
+        const int32_t id = IDS ? idv[k] : (int32_t)(base + (int64_t)k * kGridThreads + tid);
         if ((take >> (2 * k)) & 1u) {
             if (oa_pos < (uint32_t)n_a) {
                 oa[oa_pos] = id;
@@ -1117,28 +1126,28 @@ cudaError_t launch_select(const SelSrc& src, const SelWork& wk, int nseg, int n_
 namespace {
 
 // CTAs of k_sel_grid<E> that fit on the device at once (0: unknown).
-template <int E>
+template <int E, bool IDS>
 int64_t grid_capacity() {
     static int64_t cap = -1;
     if (cap < 0) {
         int dev = 0, sms = 0, per = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_sel_grid<E>, kGridThreads, 0) != cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_sel_grid<E, IDS>, kGridThreads, 0) != cudaSuccess)
             return 0;
         cap = (int64_t)sms * per;
     }
     return cap;
 }
 
-template <int E>
+template <int E, bool IDS>
 bool try_grid(const SelSrc& src, const SelWork& wk, int nseg, int n_a, int32_t* out_a, float* vals_a, int64_t stride_a,
               int n_b, int32_t* out_b, int64_t stride_b, cudaStream_t st, bool hist_ready, cudaError_t* e) {
     const int64_t per_cta = (int64_t)kGridThreads * E;
     const int64_t C = (src.n + per_cta - 1) / per_cta;
-    if (C < 1 || C * nseg > grid_capacity<E>()) return false;
-    *e = launch_pdl(k_sel_grid<E>, dim3((unsigned)C, (unsigned)nseg), dim3(kGridThreads), 0, st, src, wk, n_a, out_a,
-                    vals_a, stride_a, n_b, out_b, stride_b, hist_ready ? 1 : 0, wait_limit());
+    if (C < 1 || C * nseg > grid_capacity<E, IDS>()) return false;
+    *e = launch_pdl(k_sel_grid<E, IDS>, dim3((unsigned)C, (unsigned)nseg), dim3(kGridThreads), 0, st, src, wk, n_a,
+                    out_a, vals_a, stride_a, n_b, out_b, stride_b, hist_ready ? 1 : 0, wait_limit());
     return true;
 }
 
@@ -1153,11 +1162,19 @@ cudaError_t launch_select_dual(const SelSrc& src, const SelWork& wk, int nseg, i
     if (src.ids == nullptr && wk.hist3 != nullptr) {
         // one grid, the keys in registers, when every CTA fits on the GPU at once
         // the fewest keys per thread (the most CTAs) with which the grid fits
-        if (try_grid<1>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
-            try_grid<2>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
-            try_grid<4>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
-            try_grid<7>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
-            try_grid<16>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e))
+        if (try_grid<1, false>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<2, false>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<4, false>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<7, false>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<16, false>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e))
+            return e;
+    }
+    if (src.ids != nullptr && src.gather == 0 && wk.hist3 != nullptr) {
+        // a list of positions with their values at the same index
+        if (try_grid<1, true>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<2, true>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<4, true>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e) ||
+            try_grid<7, true>(src, wk, nseg, n_a, out_a, vals_a, stride_a, n_b, out_b, stride_b, st, hist_ready, &e))
             return e;
     }
     // otherwise two streaming passes; without a histogram from the scoring
