@@ -30,6 +30,14 @@
  *    sequence longer than the cache, a bounded wait that ran out) never trap:
  *    the kernel skips the bad element and ORs a bit into a sticky status word
  *    in the workspace, read back with csa2_read_device_status.
+ *  - Some kernels run as one grid whose CTAs wait for each other at bounded
+ *    barriers (the Full layer's selection over more than 16,384 positions,
+ *    the Reindex select and the pool update's large selections, when the
+ *    grid fits on the GPU at once; they fall back to other kernels when it
+ *    does not).  They assume the GPU is not shared with work that keeps its
+ *    SMs busy for seconds; otherwise a barrier can run out and the call
+ *    reports CSA2_ERR_TIMEOUT (results of that call unusable; re-initialise
+ *    the workspace with csa2_workspace_init).
  *  - The library keeps no mutable global state, except the fixed scratch of
  *    csa2_index_reindex_noalloc (see there) and the wait budget of the
  *    diagnostic csa2_debug_set_wait_limit: calls on different streams with
