@@ -19,7 +19,8 @@ FULL, REINDEX, REUSE = 0, 1, 2
 F32, BF16, E4M3 = 0, 1, 2
 
 ABI_FUNCTIONS = (
-    "csa2_workspace_bytes", "csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
+    "csa2_workspace_bytes", "csa2_workspace_init", "csa2_kv_append_quant", "csa2_kv_export_rows",
+    "csa2_kv_import_rows", "csa2_index_scores", "csa2_index_full",
     "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update", "csa2_sparse_swa_attn",
     "csa2_ring_append",
     "csa2_sparse_swa_attn_local", "csa2_layer_step", "csa2_prefill_workspace_bytes", "csa2_prefill_layer",
@@ -69,6 +70,8 @@ def lib():
         L.csa2_workspace_bytes.argtypes = [cp, i32, i32, i32, i32, i32]
         L.csa2_workspace_init.argtypes = [vp, sz, vp]
         L.csa2_kv_append_quant.argtypes = [cp, vp, vp, i32, vp, i32, vp, vp]
+        L.csa2_kv_export_rows.argtypes = [cp, vp, i32, vp, vp, vp, vp]
+        L.csa2_kv_import_rows.argtypes = [cp, vp, i32, vp, vp, vp, vp]
         L.csa2_index_scores.argtypes = [cp, vp, i32, vp, i32, i32, vp, vp, sz, vp]
         L.csa2_index_full.argtypes = [cp, vp, i32, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
         L.csa2_index_reindex.argtypes = [cp, vp, i32, vp, i32, i32, vp, i32, i32, vp, vp, sz, vp]
@@ -88,7 +91,8 @@ def lib():
         L.csa2_debug_set_wait_limit.argtypes = [ctypes.c_uint32]
         L.csa2_debug_default_wait_limit.restype = ctypes.c_uint32
         L.csa2_debug_default_wait_limit.argtypes = []
-        for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_index_scores", "csa2_index_full",
+        for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_kv_export_rows", "csa2_kv_import_rows",
+                     "csa2_index_scores", "csa2_index_full",
                      "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update",
                      "csa2_sparse_swa_attn", "csa2_ring_append", "csa2_sparse_swa_attn_local",
                      "csa2_layer_step", "csa2_prefill_layer", "csa2_read_device_status",
@@ -200,6 +204,19 @@ def kv_append_quant(cache, x, start_pos, idx_new=None, ws=None, stream=None):
     dt = F32 if (idx_new is not None and idx_new.dtype == torch.float32) else BF16
     _check(lib().csa2_kv_append_quant(cache.ref, _p(x), _p(idx_new), dt, _p(start_pos), x.shape[1], _p(ws),
                                       _stream(stream)), "kv_append_quant")
+
+
+def kv_export_rows(cache, start_pos, n, rows, keys=None, ws=None, stream=None):
+    """Stored rows [B, n, dim/2 + dim/16] uint8 (and keys [B, n, key bytes])
+    of positions start_pos[b] + i, copied out of the cache."""
+    _check(lib().csa2_kv_export_rows(cache.ref, _p(start_pos), n, _p(rows), _p(keys), _p(ws), _stream(stream)),
+           "kv_export_rows")
+
+
+def kv_import_rows(cache, start_pos, n, rows, keys=None, ws=None, stream=None):
+    """The inverse of kv_export_rows: the buffers written back into the cache."""
+    _check(lib().csa2_kv_import_rows(cache.ref, _p(start_pos), n, _p(rows), _p(keys), _p(ws), _stream(stream)),
+           "kv_import_rows")
 
 
 def _qdt(q_idx):

@@ -293,6 +293,31 @@ csa2_status csa2_kv_append_quant(const csa2_cache* cache, const void* x_bf16, co
                                            static_cast<cudaStream_t>(stream), num_sms()));
 }
 
+csa2_status csa2_kv_export_rows(const csa2_cache* cache, const int32_t* start_pos, int n, void* rows, void* keys,
+                                void* ws, void* stream) {
+    csa2_status s = check_cache(cache);
+    if (s != CSA2_OK) return s;
+    if (!start_pos || !aligned4(start_pos) || n < 0 || !rows || !aligned4(rows) || (keys && !aligned4(keys)) ||
+        (ws && !aligned16(ws)))
+        return CSA2_ERR_INVALID_ARG;
+    if (n == 0) return CSA2_OK;
+    return cuda_status(launch_rows_io(dev_cache(cache), true, start_pos, n, rows, keys, static_cast<uint32_t*>(ws),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+csa2_status csa2_kv_import_rows(const csa2_cache* cache, const int32_t* start_pos, int n, const void* rows,
+                                const void* keys, void* ws, void* stream) {
+    csa2_status s = check_cache(cache);
+    if (s != CSA2_OK) return s;
+    if (!start_pos || !aligned4(start_pos) || n < 0 || !rows || !aligned4(rows) || (keys && !aligned4(keys)) ||
+        (ws && !aligned16(ws)))
+        return CSA2_ERR_INVALID_ARG;
+    if (n == 0) return CSA2_OK;
+    return cuda_status(launch_rows_io(dev_cache(cache), false, start_pos, n, const_cast<void*>(rows),
+                                      const_cast<void*>(keys), static_cast<uint32_t*>(ws),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 csa2_status csa2_index_scores(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
                               int T, int H_I, float* scores, void* ws, size_t ws_bytes, void* stream) {
     csa2_status s = check_index_args(cache, q_idx, q_dtype, head_w, T, H_I, 1, 1);

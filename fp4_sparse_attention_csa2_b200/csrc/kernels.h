@@ -51,6 +51,11 @@ cudaError_t launch_append_quant(const DevCache& c, const void* x, const void* id
                                 const int32_t* start_pos, int n_new, uint32_t* status, cudaStream_t st,
                                 int num_sms);
 
+// Stored rows and keys of positions start_pos[b] + i between the cache and
+// packed buffers [batch][n][dim / 2 + dim / 16] and [batch][n][key bytes].
+cudaError_t launch_rows_io(const DevCache& c, bool to_buffers, const int32_t* start_pos, int n, void* rows, void* keys,
+                           uint32_t* status, cudaStream_t st);
+
 // Full scoring: scores[(b*T + j) * cap + t] for t <= p_j.
 cudaError_t launch_score_full(const DevCache& c, const void* q, int q_f32, const float* hw, int T, int H_I,
                               float* scores, uint32_t* status, cudaStream_t st, int num_sms);

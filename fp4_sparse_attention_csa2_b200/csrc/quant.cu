@@ -104,6 +104,57 @@ k_append_quant(DevCache c, const __nv_bfloat16* __restrict__ x, const void* __re
     }
 }
 
+namespace {
+
+// Rows (codes then scales, dim / 2 + dim / 16 bytes) and index keys of
+// positions start_pos[b] + i, between the cache and packed buffers
+// [batch][n][...]: one warp per (sequence, position), 2-byte words for rows
+// and 4-byte words for keys.  EXPORT: cache -> buffers (zeros and a bounds
+// flag for a position outside the cache); otherwise buffers -> cache (the
+// position skipped and flagged).
+template <bool EXPORT>
+__global__ void __launch_bounds__(256)
+k_rows_io(DevCache c, const int32_t* __restrict__ start_pos, int n, uint8_t* rows, uint8_t* keys, uint32_t* status) {
+    pdl_begin();
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= (int64_t)c.batch * n) return;
+    const int lane = threadIdx.x & 31;
+    const int b = (int)(r / n), i = (int)(r % n);
+    const int64_t t = (int64_t)__ldg(start_pos + b) + i;
+    const int64_t slot = t >= 0 && t < c.cap ? slot_of(c, b, t) : -1;
+    if (slot < 0 && lane == 0) flag(status, kStatusBounds);
+    const int row_bytes = c.dim / 2 + c.dim / 16;
+    const int key_bytes = c.key_dtype == 2 ? c.idx_dim : 4 * c.idx_dim;
+    uint16_t* brow = reinterpret_cast<uint16_t*>(rows + r * row_bytes);
+    uint32_t* bkey = reinterpret_cast<uint32_t*>(keys + r * key_bytes);
+    if (EXPORT) {
+        const uint16_t* crow = slot >= 0 ? reinterpret_cast<const uint16_t*>(c.rows + slot * c.row_stride) : nullptr;
+        const uint32_t* ckey = slot >= 0 ? reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(c.keys) +
+                                                                             slot * key_bytes) : nullptr;
+        for (int w = lane; w < row_bytes / 2; w += 32) brow[w] = crow ? crow[w] : 0;
+        if (keys)
+            for (int w = lane; w < key_bytes / 4; w += 32) bkey[w] = ckey ? ckey[w] : 0u;
+    } else if (slot >= 0) {
+        uint16_t* crow = reinterpret_cast<uint16_t*>(c.rows + slot * c.row_stride);
+        uint32_t* ckey = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(c.keys) + slot * key_bytes);
+        for (int w = lane; w < row_bytes / 2; w += 32) crow[w] = brow[w];
+        if (keys)
+            for (int w = lane; w < key_bytes / 4; w += 32) ckey[w] = bkey[w];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_rows_io(const DevCache& c, bool to_buffers, const int32_t* start_pos, int n, void* rows, void* keys,
+                           uint32_t* status, cudaStream_t st) {
+    const int64_t r = (int64_t)c.batch * n;
+    const dim3 grid((unsigned)((r + 7) / 8));
+    uint8_t* rb = static_cast<uint8_t*>(rows);
+    uint8_t* kb = static_cast<uint8_t*>(keys);
+    return to_buffers ? launch_pdl(k_rows_io<true>, grid, dim3(256), 0, st, c, start_pos, n, rb, kb, status)
+                      : launch_pdl(k_rows_io<false>, grid, dim3(256), 0, st, c, start_pos, n, rb, kb, status);
+}
+
 cudaError_t launch_append_quant(const DevCache& c, const void* x, const void* idx_new, int idx_new_f32,
                                 const int32_t* start_pos, int n_new, uint32_t* status, cudaStream_t st,
                                 int num_sms) {

@@ -150,6 +150,27 @@ CSA2_API csa2_status csa2_kv_append_quant(const csa2_cache* cache, const void* x
                                  void* ws, void* stream);
 
 /*
+ * The stored form of cached positions, for persistent storage ([TLDR]
+ * paragraph 4: the FP4 rows and E4M3 keys are what the cache holds; [HF]
+ * abstract: the compressed KV as persistent state).  csa2_kv_export_rows
+ * copies, for every sequence b and i < n, position start_pos[b] + i of the
+ * cache into packed device buffers (the caller copies them to the host):
+ *     rows [batch][n][dim/2 + dim/16]  the D/2 code bytes (channel 2j in the
+ *                                       low nibble) then the D/16 E4M3 scales,
+ *     keys [batch][n][idx_dim or 4 * idx_dim]  the index key as stored
+ *                                       (E4M3 bytes or fp32), nullable.
+ * csa2_kv_import_rows writes such buffers back into the cache at the same
+ * positions (seq_lens unchanged), e.g. when a request is restored.  A position
+ * outside the cache is written as zeros (export) or skipped (import), and sets
+ * CSA2_ERR_DEVICE_BOUNDS in ws (nullable).  start_pos is a device int32
+ * [batch]; rows and keys are 4-byte aligned device buffers.
+ */
+CSA2_API csa2_status csa2_kv_export_rows(const csa2_cache* cache, const int32_t* start_pos, int n, void* rows,
+                                         void* keys, void* ws, void* stream);
+CSA2_API csa2_status csa2_kv_import_rows(const csa2_cache* cache, const int32_t* start_pos, int n,
+                                         const void* rows, const void* keys, void* ws, void* stream);
+
+/*
  * Full-layer indexing ([TLDR] paragraph 3; [HN] key point 3).  Query token j
  * of sequence b sits at p = seq_lens[b] - T + j and sees positions t <= p.
  * Every visible position gets the score

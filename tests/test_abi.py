@@ -209,3 +209,14 @@ def test_prefill_workspace_and_arguments(lib):
     a.H_I = 32
     a.mode = 7
     assert lib.csa2_prefill_layer(ctypes.byref(c), ctypes.byref(a), 0x80000, n1, None) == csa2.ERR_INVALID_ARG
+
+
+def test_export_import_arguments_rejected_on_host(lib):
+    c = fake_cache()
+    for fn in (lib.csa2_kv_export_rows, lib.csa2_kv_import_rows):
+        assert fn(ctypes.byref(c), None, 4, 0x40000, 0x50000, None, None) == csa2.ERR_INVALID_ARG
+        assert fn(ctypes.byref(c), 0x30002, 4, 0x40000, 0x50000, None, None) == csa2.ERR_INVALID_ARG
+        assert fn(ctypes.byref(c), 0x30000, -1, 0x40000, 0x50000, None, None) == csa2.ERR_INVALID_ARG
+        assert fn(ctypes.byref(c), 0x30000, 4, None, 0x50000, None, None) == csa2.ERR_INVALID_ARG
+        assert fn(ctypes.byref(c), 0x30000, 4, 0x40002, 0x50000, None, None) == csa2.ERR_INVALID_ARG
+        assert fn(ctypes.byref(c), 0x30000, 0, 0x40000, 0x50000, None, None) == csa2.OK   # nothing to copy
