@@ -12,7 +12,11 @@
 // digit the remaining equal keys are exact ties of which the first claimants
 // win.  Output order is unspecified; -1 pads the tail.
 //
-//   large segments (Full layer, up to 1M scores): the level-1 histogram comes
+//   large segments (Full layer, up to 1M scores), when every CTA of the grid
+//     fits on the GPU at once: one launch, each CTA holding its keys in
+//     registers, two bounded segment barriers between the digit levels
+//     (k_sel_grid; also for a list of positions, as a pool update's).
+//   large segments otherwise: the level-1 histogram comes
 //     from the scoring kernel; a streaming pass (many CTAs per segment) works
 //     out each target's level-1 threshold, selects above it and compacts the
 //     elements equal to it into candidate lists (histogramming their digit 2);
