@@ -24,6 +24,8 @@ ABI_FUNCTIONS = (
     "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update", "csa2_sparse_swa_attn",
     "csa2_ring_append",
     "csa2_sparse_swa_attn_local", "csa2_layer_step", "csa2_prefill_workspace_bytes", "csa2_prefill_layer",
+    "csa2_cp_index_local", "csa2_cp_reindex_local", "csa2_cp_merge_workspace_bytes", "csa2_cp_merge_select",
+    "csa2_cp_sparse_swa_attn", "csa2_lse_merge",
     "csa2_read_device_status", "csa2_status_string", "csa2_debug_set_wait_limit", "csa2_debug_default_wait_limit",
 )
 
@@ -85,6 +87,13 @@ def lib():
         L.csa2_prefill_workspace_bytes.restype = sz
         L.csa2_prefill_workspace_bytes.argtypes = [cp, i32, i32, i32, i32, i32, i32]
         L.csa2_prefill_layer.argtypes = [cp, ctypes.POINTER(csa2_layer_args), vp, sz, vp]
+        L.csa2_cp_index_local.argtypes = [cp, vp, vp, i32, vp, i32, i32, vp, vp, sz, vp]
+        L.csa2_cp_reindex_local.argtypes = [cp, vp, vp, i32, vp, i32, vp, i32, i32, vp, vp, sz, vp]
+        L.csa2_cp_merge_workspace_bytes.restype = sz
+        L.csa2_cp_merge_workspace_bytes.argtypes = [i32, i32, i32]
+        L.csa2_cp_merge_select.argtypes = [vp, i32, i32, i32, vp, i32, vp, i32, vp, vp, sz, vp]
+        L.csa2_cp_sparse_swa_attn.argtypes = [cp, vp, vp, vp, i32, vp, i32, i32, ctypes.c_float, vp, vp, vp, sz, vp]
+        L.csa2_lse_merge.argtypes = [i32, i32, i32, i32, vp, ctypes.c_int64, vp, ctypes.c_int64, vp, vp, vp]
         L.csa2_read_device_status.argtypes = [vp, vp]
         L.csa2_status_string.restype = ctypes.c_char_p
         L.csa2_status_string.argtypes = [i32]
@@ -96,7 +105,8 @@ def lib():
                      "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update",
                      "csa2_sparse_swa_attn", "csa2_ring_append", "csa2_sparse_swa_attn_local",
                      "csa2_layer_step", "csa2_prefill_layer", "csa2_read_device_status",
-                     "csa2_debug_set_wait_limit"):
+                     "csa2_debug_set_wait_limit", "csa2_cp_index_local", "csa2_cp_reindex_local",
+                     "csa2_cp_merge_select", "csa2_cp_sparse_swa_attn", "csa2_lse_merge"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -321,6 +331,81 @@ def prefill_layer(cache, mode, q, topk_idx, out, ws, window, q_idx=None, head_w=
                         0 if ring is None else ring.shape[1])
     _check(lib().csa2_prefill_layer(cache.ref, ctypes.byref(a), _p(ws), ws.numel() * ws.element_size(),
                                     _stream(stream)), "prefill_layer")
+
+
+# ---------------------------------------------------------------- context-parallel decode
+# A candidate (csa2_cand) is held as int32 [..., 2]: the global position and
+# the bits of its fp32 score.
+
+def cand_buffer(batch, n, device="cuda"):
+    """Candidates [batch, n] (int32 pairs: position, score bits)."""
+    return torch.empty((batch, n, 2), dtype=torch.int32, device=device)
+
+
+def cand_scores(cand):
+    """The fp32 scores of a candidate buffer."""
+    return cand.view(torch.float32)[..., 1]
+
+
+def cp_index_local(shard, pos0, q_idx, head_w, pool_k, cand, ws, stream=None):
+    """A Full layer's share on a shard: its pool_k best positions (global,
+    pos0 [B] int32 added) with their scores into cand [B, pool_k, 2].  q_idx
+    [B, 1, H_I, idx_dim]; head_w [B, 1, H_I]."""
+    B, T, H_I, _ = q_idx.shape
+    if T != 1:
+        raise ValueError("context-parallel calls take one query token per sequence")
+    _check(lib().csa2_cp_index_local(shard.ref, _p(pos0), _p(q_idx), _qdt(q_idx), _p(head_w), H_I, pool_k, _p(cand),
+                                     _p(ws), ws.numel() * ws.element_size(), _stream(stream)), "cp_index_local")
+
+
+def cp_reindex_local(shard, pos0, q_idx, head_w, pool_idx, top_k, cand, ws, stream=None):
+    """A Reindex layer's share on a shard: the global pool entries it holds
+    rescored, the top_k best into cand [B, top_k, 2]."""
+    B, T, H_I, _ = q_idx.shape
+    if T != 1:
+        raise ValueError("context-parallel calls take one query token per sequence")
+    _check(lib().csa2_cp_reindex_local(shard.ref, _p(pos0), _p(q_idx), _qdt(q_idx), _p(head_w), H_I, _p(pool_idx),
+                                       pool_idx.shape[-1], top_k, _p(cand), _p(ws), ws.numel() * ws.element_size(),
+                                       _stream(stream)), "cp_reindex_local")
+
+
+def cp_merge_workspace_bytes(R, batch, n_cand):
+    n = lib().csa2_cp_merge_workspace_bytes(R, batch, n_cand)
+    if n == 0:
+        raise CSA2Error(ERR_INVALID_ARG, "cp_merge_workspace_bytes")
+    return n
+
+
+def cp_merge_select(cand, seq_lens_global, n_a, out_a, ws, n_b=0, out_b=None, stream=None):
+    """The selection after the all-gather: cand [R, B, n_cand, 2]; the n_a best
+    positions into out_a [B, n_a] and the n_b best into out_b [B, n_b]."""
+    R, B, n_cand, _ = cand.shape
+    _check(lib().csa2_cp_merge_select(_p(cand), R, B, n_cand, _p(seq_lens_global), n_a, _p(out_a), n_b, _p(out_b),
+                                      _p(ws), ws.numel() * ws.element_size(), _stream(stream)), "cp_merge_select")
+
+
+def cp_sparse_swa_attn(shard, pos0, seq_lens_global, q, topk_idx, window, out, lse, ws, sm_scale=0.0, stream=None):
+    """A layer's attention on a shard: its part of window ∪ top-k (topk_idx
+    global [B, top_k]); out fp32 [B, H, dim], lse fp32 [B, H] of that part."""
+    B, H = q.shape[0], q.shape[-2]
+    top_k = topk_idx.shape[-1] if topk_idx is not None else 0
+    _check(lib().csa2_cp_sparse_swa_attn(shard.ref, _p(pos0), _p(seq_lens_global), _p(q), H, _p(topk_idx), top_k,
+                                         window, sm_scale, _p(out), _p(lse), _p(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream)), "cp_sparse_swa_attn")
+
+
+def lse_merge(outs, lses, out, lse=None, stream=None):
+    """Merge R attention parts: outs [R, B, H, dim] and lses [R, B, H] (views
+    of one buffer allowed: any rank stride) into out [B, H, dim], lse [B, H]."""
+    R, B, H, D = outs.shape
+    for t in (outs, lses):
+        if not t.is_cuda:
+            raise ValueError("libcsa2 takes CUDA tensors; got one on %s" % t.device)
+        if not t[0].is_contiguous():
+            raise ValueError("each part must be contiguous")
+    _check(lib().csa2_lse_merge(R, B, H, D, ctypes.c_void_p(outs.data_ptr()), outs.stride(0),
+                                ctypes.c_void_p(lses.data_ptr()), lses.stride(0), _p(out), _p(lse), _stream(stream)),
+           "lse_merge")
 
 
 def read_device_status(ws, stream=None):

@@ -551,6 +551,210 @@ csa2_status csa2_prefill_layer(const csa2_cache* cache, const csa2_layer_args* a
     return CSA2_OK;
 }
 
+// ---------------------------------------------------------------- context-parallel decode
+// The shard calls run the single-device kernels on the shard's cache (T = 1:
+// every shard position is visible) and use the shard workspace's sections as
+// follows: scores / selection state as csa2_index_full; the shard's pool or
+// top-k ids in upd_ids or upd_scores, their scores in pscores or upd_scores;
+// the attention list in upd_ids.
+
+static_assert(sizeof(csa2_cand) == sizeof(CpCand), "csa2_cand and CpCand must have one layout");
+
+csa2_status csa2_cp_index_local(const csa2_cache* shard, const int32_t* pos0, const void* q_idx, csa2_dtype q_dtype,
+                                const float* head_w, int H_I, int pool_k, csa2_cand* cand, void* ws, size_t ws_bytes,
+                                void* stream) {
+    csa2_status s = check_index_args(shard, q_idx, q_dtype, head_w, 1, H_I, pool_k, 1);
+    if (s != CSA2_OK) return s;
+    if (!pos0 || !aligned4(pos0) || !cand || (reinterpret_cast<uintptr_t>(cand) & 7u)) return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(shard, 1, 1, pool_k, 1, 0, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* hist = L.cap > kSmallSelect ? at<uint32_t>(ws, L.hist) : nullptr;
+    float* scores = at<float>(ws, L.scores);
+    bool fused = false;
+    s = launch_scores(shard, q_idx, q_dtype, head_w, 1, H_I, scores, hist, at<uint32_t>(ws, L.status), st, &fused);
+    if (s != CSA2_OK) return s;
+    SelSrc src;
+    src.vals = scores;
+    src.vals_stride = L.cap;
+    src.ids = nullptr;
+    src.ids_stride = 0;
+    src.gather = 0;
+    src.n = L.cap;
+    src.seq_lens = shard->seq_lens;
+    src.T = 1;
+    src.cap = L.cap;
+    int32_t* ids = at<int32_t>(ws, L.upd_ids);
+    float* vals = at<float>(ws, L.pscores);
+    cudaError_t e = L.cap > kSmallSelect
+                        ? launch_select_dual(src, sel_work(ws, L), (int)L.nseg, pool_k, ids, vals, pool_k, 0, nullptr,
+                                             0, st, fused)
+                        : launch_select_local(src, (int)L.nseg, pool_k, ids, vals, pool_k, 0, nullptr, 0, st);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    return cuda_status(launch_cp_pack(ids, vals, pool_k, pos0, shard->batch, pool_k, reinterpret_cast<CpCand*>(cand),
+                                      st));
+}
+
+csa2_status csa2_cp_reindex_local(const csa2_cache* shard, const int32_t* pos0, const void* q_idx,
+                                  csa2_dtype q_dtype, const float* head_w, int H_I, const int32_t* pool_idx,
+                                  int pool_k, int top_k, csa2_cand* cand, void* ws, size_t ws_bytes, void* stream) {
+    csa2_status s = check_index_args(shard, q_idx, q_dtype, head_w, 1, H_I, pool_k, top_k);
+    if (s != CSA2_OK) return s;
+    if (!pos0 || !aligned4(pos0) || !pool_idx || !aligned16(pool_idx) || !cand ||
+        (reinterpret_cast<uintptr_t>(cand) & 7u))
+        return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(shard, 1, 1, pool_k, top_k, 0, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevCache d = dev_cache(shard);
+    uint32_t* status = at<uint32_t>(ws, L.status);
+    int32_t* local = at<int32_t>(ws, L.upd_ids);           // [batch][pool_k] shard positions or -1
+    float* sc = at<float>(ws, L.pscores);                   // [batch][pool_k]
+    int32_t* ids = at<int32_t>(ws, L.upd_scores);           // [batch][top_k]
+    float* vals = at<float>(ws, L.upd_scores + align_up(sizeof(int32_t) * (size_t)L.nseg * top_k));
+    cudaError_t e = launch_cp_localize(pool_idx, pos0, shard->seq_lens, shard->batch, pool_k, local, st);
+    if (e == cudaSuccess)
+        e = reindex_tc_supported(d, H_I) ? launch_reindex_tc_scores(d, q_idx, head_w, 1, H_I, local, pool_k, sc, status, st)
+                                         : launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, 1, H_I, local, pool_k,
+                                                             sc, status, st);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    SelSrc src;
+    src.vals = sc;
+    src.vals_stride = pool_k;
+    src.ids = local;
+    src.ids_stride = pool_k;
+    src.gather = 0;
+    src.n = pool_k;
+    src.seq_lens = shard->seq_lens;
+    src.T = 1;
+    src.cap = L.cap;
+    e = launch_select_local(src, (int)L.nseg, top_k, ids, vals, top_k, 0, nullptr, 0, st);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    return cuda_status(launch_cp_pack(ids, vals, top_k, pos0, shard->batch, top_k, reinterpret_cast<CpCand*>(cand),
+                                      st));
+}
+
+namespace {
+// Workspace of csa2_cp_merge_select: status | histograms | digit-3 histograms |
+// counters | candidate and survivor buffers | the candidates per sequence.
+struct MergeLayout {
+    size_t status, hist, hist3, cnt, cand1, cand2, surv1, surv2, ids, vals, total;
+    int64_t m;
+};
+
+bool make_merge_layout(int R, int batch, int n_cand, MergeLayout* L) {
+    if (R < 1 || batch < 1 || batch > 65535 || n_cand < 1) return false;
+    L->m = (int64_t)R * n_cand;
+    if (L->m > ((int64_t)1 << 24)) return false;
+    const size_t nseg = (size_t)batch, m = (size_t)L->m;
+    size_t off = 0;
+    L->status = off; off = align_up(off + 16);
+    L->hist = off; off = align_up(off + sizeof(uint32_t) * nseg * 3 * kRadixBins);
+    L->hist3 = off; off = align_up(off + sizeof(uint32_t) * nseg * 2 * kRadixBins);
+    L->cnt = off; off = align_up(off + sizeof(uint32_t) * nseg * kSelCounters);
+    L->cand1 = off; off = align_up(off + 2 * sizeof(uint32_t) * nseg * m);
+    L->cand2 = off; off = align_up(off + 2 * sizeof(uint32_t) * nseg * m);
+    L->surv1 = off; off = align_up(off + 2 * sizeof(uint32_t) * nseg * m);
+    L->surv2 = off; off = align_up(off + 2 * sizeof(uint32_t) * nseg * m);
+    L->ids = off; off = align_up(off + sizeof(int32_t) * nseg * m);
+    L->vals = off; off = align_up(off + sizeof(float) * nseg * m);
+    L->total = off;
+    return true;
+}
+}  // namespace
+
+size_t csa2_cp_merge_workspace_bytes(int R, int batch, int n_cand) {
+    MergeLayout L;
+    return make_merge_layout(R, batch, n_cand, &L) ? L.total : 0;
+}
+
+csa2_status csa2_cp_merge_select(const csa2_cand* cand, int R, int batch, int n_cand, const int32_t* seq_lens_global,
+                                 int n_a, int32_t* out_a, int n_b, int32_t* out_b, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    MergeLayout L;
+    if (!make_merge_layout(R, batch, n_cand, &L)) return CSA2_ERR_INVALID_ARG;
+    if (!cand || (reinterpret_cast<uintptr_t>(cand) & 7u) || !seq_lens_global || !aligned4(seq_lens_global))
+        return CSA2_ERR_INVALID_ARG;
+    if (n_a < 1 || n_a > kMaxPool || !out_a || !aligned16(out_a)) return CSA2_ERR_INVALID_ARG;
+    if (n_b < 0 || n_b > n_a || (n_b > 0 && (!out_b || !aligned16(out_b)))) return CSA2_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws) || ws_bytes < L.total) return CSA2_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* ids = at<int32_t>(ws, L.ids);
+    float* vals = at<float>(ws, L.vals);
+    if (launch_cp_unpack(reinterpret_cast<const CpCand*>(cand), R, batch, n_cand, ids, vals, st) != cudaSuccess)
+        return CSA2_ERR_CUDA;
+    SelSrc src;
+    src.vals = vals;
+    src.vals_stride = L.m;
+    src.ids = ids;
+    src.ids_stride = L.m;
+    src.gather = 0;
+    src.n = L.m;
+    src.seq_lens = seq_lens_global;      // a candidate is valid when 0 <= pos < Lg (T = 1)
+    src.T = 1;
+    src.cap = (int64_t)1 << 31;
+    if (L.m <= kSmallSelect)
+        return cuda_status(launch_select_local(src, batch, n_a, out_a, nullptr, n_a, n_b, n_b > 0 ? out_b : nullptr,
+                                               n_b, st));
+    SelWork w;
+    w.hist = at<uint32_t>(ws, L.hist);
+    w.cnt = at<uint32_t>(ws, L.cnt);
+    w.cand1 = at<uint32_t>(ws, L.cand1);
+    w.cand2 = at<uint32_t>(ws, L.cand2);
+    w.surv1 = at<uint32_t>(ws, L.surv1);
+    w.surv2 = at<uint32_t>(ws, L.surv2);
+    w.cand_stride = L.m;
+    w.hist3 = at<uint32_t>(ws, L.hist3);
+    w.status = at<uint32_t>(ws, L.status);
+    return cuda_status(launch_select_dual(src, w, batch, n_a, out_a, nullptr, n_a, n_b, n_b > 0 ? out_b : nullptr,
+                                          n_b, st, false));
+}
+
+csa2_status csa2_cp_sparse_swa_attn(const csa2_cache* shard, const int32_t* pos0, const int32_t* seq_lens_global,
+                                    const void* q_bf16, int H, const int32_t* topk_idx, int top_k, int window,
+                                    float sm_scale, float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    csa2_status s = check_cache(shard);
+    if (s != CSA2_OK) return s;
+    if (!pos0 || !aligned4(pos0) || !seq_lens_global || !aligned4(seq_lens_global)) return CSA2_ERR_INVALID_ARG;
+    if (!q_bf16 || !out || !lse || !aligned16(q_bf16) || !aligned16(out) || !aligned16(lse)) return CSA2_ERR_INVALID_ARG;
+    if (H < 1 || top_k < 0 || window < 0 || window > kMaxPool || top_k > kMaxPool) return CSA2_ERR_INVALID_ARG;
+    if (top_k > 0 && (!topk_idx || !aligned16(topk_idx))) return CSA2_ERR_INVALID_ARG;
+    if (H > 64 || H % 16) return CSA2_ERR_UNSUPPORTED;
+    if (!std::isfinite(sm_scale)) return CSA2_ERR_INVALID_ARG;
+    Layout L;
+    s = check_ws(shard, 1, H, top_k > 0 ? top_k : 1, top_k, window, ws, ws_bytes, &L);
+    if (s != CSA2_OK) return s;
+    if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)shard->dim);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* status = at<uint32_t>(ws, L.status);
+    // the shard's part of window ∪ top-k as one list of shard positions; the
+    // attention then runs with no window of its own (the list's window part and
+    // top-k part are disjoint)
+    const int n = window + top_k;
+    int32_t* list = at<int32_t>(ws, L.upd_ids);
+    if (n > 0 && launch_cp_attn_list(topk_idx, top_k, window, pos0, shard->seq_lens, seq_lens_global, shard->batch,
+                                     list, status, st) != cudaSuccess)
+        return CSA2_ERR_CUDA;
+    AttnWork aw;
+    aw.part_o = at<float>(ws, L.part_o);
+    aw.part_ml = at<float>(ws, L.part_ml);
+    aw.nchunk = L.nchunk;
+    return cuda_status(launch_attention(dev_cache(shard), q_bf16, 1, H, n > 0 ? list : nullptr, n, 0, sm_scale, Ring{},
+                                        out, lse, aw, status, st, num_sms()));
+}
+
+csa2_status csa2_lse_merge(int R, int batch, int H, int dim, const float* outs, int64_t out_stride,
+                           const float* lses, int64_t lse_stride, float* out, float* lse, void* stream) {
+    if (R < 1 || batch < 1 || H < 1 || dim < 1 || !outs || !lses || !out) return CSA2_ERR_INVALID_ARG;
+    if (!aligned4(outs) || !aligned4(lses) || !aligned4(out) || (lse && !aligned4(lse))) return CSA2_ERR_INVALID_ARG;
+    if (R > 1 && (out_stride < (int64_t)batch * H * dim || lse_stride < (int64_t)batch * H))
+        return CSA2_ERR_INVALID_ARG;
+    return cuda_status(launch_lse_merge(R, batch, H, dim, outs, out_stride, lses, lse_stride, out, lse,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 csa2_status csa2_read_device_status(void* ws, void* stream) {
     if (!ws || !aligned16(ws)) return CSA2_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

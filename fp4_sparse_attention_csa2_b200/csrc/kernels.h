@@ -142,4 +142,26 @@ cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, con
                              int window, float sm_scale, const Ring& ring, float* out, float* lse,
                              const AttnWork& aw, uint32_t* status, cudaStream_t st, int num_sms);
 
+// Context-parallel decode (cp.cu): a candidate is a global position and its
+// score, laid out as csa2_cand.
+struct CpCand {
+    int32_t pos;
+    float score;
+};
+// cand[b][i] <- (ids[b][i] + pos0[b], vals[b][i]), or (-1, 0) for ids < 0.
+cudaError_t launch_cp_pack(const int32_t* ids, const float* vals, int64_t in_stride, const int32_t* pos0, int batch,
+                           int n, CpCand* cand, cudaStream_t st);
+// local[b][i] <- pool[b][i] - pos0[b] when in [0, shard_lens[b]), else -1.
+cudaError_t launch_cp_localize(const int32_t* pool, const int32_t* pos0, const int32_t* shard_lens, int batch, int n,
+                               int32_t* local, cudaStream_t st);
+// [R][batch][n] candidates -> ids / vals [batch][R * n].
+cudaError_t launch_cp_unpack(const CpCand* cand, int R, int batch, int n, int32_t* ids, float* vals,
+                             cudaStream_t st);
+// The shard's part of window ∪ top-k as a list [batch][window + top_k] of shard positions (-1: none).
+cudaError_t launch_cp_attn_list(const int32_t* topk, int top_k, int window, const int32_t* pos0,
+                                const int32_t* shard_lens, const int32_t* lens_global, int batch, int32_t* list,
+                                uint32_t* status, cudaStream_t st);
+cudaError_t launch_lse_merge(int R, int batch, int H, int D, const float* outs, int64_t out_stride, const float* lses,
+                             int64_t lse_stride, float* out, float* lse, cudaStream_t st);
+
 }  // namespace csa2

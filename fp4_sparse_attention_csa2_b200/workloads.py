@@ -216,3 +216,10 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
 def host_array(t: torch.Tensor) -> np.ndarray:
     """bf16 -> uint16 bits, fp32 -> float32 (no conversion of values)."""
     return bf16_bits(t) if t.dtype == torch.bfloat16 else t.contiguous().numpy()
+
+
+def shard_bounds(L, R):
+    """Context-parallel split of one sequence of L positions over R ranks:
+    rank r holds [L r / R, L (r + 1) / R) (floors; ragged when R does not
+    divide L)."""
+    return [(L * r // R, L * (r + 1) // R - L * r // R) for r in range(R)]

@@ -16,6 +16,8 @@
  *   [FANOUT] fanout.sh daily lesson, "What you will learn" item 2 (modes share
  *            global KV and sparse selections; queries and window stay
  *            layer-local).
+ *   [ZH]     zerohour.day item on the same release (a context of one million
+ *            tokens).
  *
  * Conventions for every call:
  *  - All pointers inside csa2_cache and all tensor arguments are DEVICE
@@ -367,6 +369,111 @@ CSA2_API size_t csa2_prefill_workspace_bytes(const csa2_cache* cache, int T, int
                                              int window);
 CSA2_API csa2_status csa2_prefill_layer(const csa2_cache* cache, const csa2_layer_args* args, void* ws,
                                         size_t ws_bytes, void* stream);
+
+/*
+ * Context-parallel decode: the positions of one sequence spread over R
+ * devices ([TLDR] paragraph 1 and [ZH]: contexts of a million tokens; [TLDR]
+ * paragraph 3: pool and top-k are selections by score, so they
+ * split by position).  Rank r keeps positions [pos0[b], pos0[b] + n_r[b]) of
+ * sequence b in a cache of its own, its "shard": there they are positions 0 ..
+ * n_r[b] - 1 and the shard's seq_lens holds n_r.  The shards of a sequence are
+ * disjoint and together hold 0 .. Lg[b] - 1 (Lg: the global lengths).  One
+ * query token per sequence (T = 1) at p = Lg[b] - 1, so every position of every
+ * shard is visible to it.  Two identities make the split exact:
+ *   - the n best positions overall are among the union of every shard's n
+ *     best (a position outside its shard's n best has n better ones there);
+ *   - attention over S is the log-sum-exp merge of attention over the
+ *     disjoint parts S ∩ shard_r.
+ * One layer on every rank:
+ *   FULL     csa2_cp_index_local -> all-gather of the candidates ->
+ *            csa2_cp_merge_select (pool and top-k)
+ *   REINDEX  csa2_cp_reindex_local -> all-gather -> csa2_cp_merge_select
+ *   any      csa2_cp_sparse_swa_attn -> all-gather of (out, lse) ->
+ *            csa2_lse_merge
+ * The all-gathers are the caller's (NCCL over NVLink, a few hundred KB a
+ * layer); every rank ends with the same pool, top-k, output and lse.  The
+ * shard calls share one workspace of csa2_workspace_bytes(shard, 1, H, pool_k,
+ * top_k, window) bytes (cleared once with csa2_workspace_init; its status word
+ * read with csa2_read_device_status); the merge selection has its own.
+ *
+ * A candidate is a global position with its score; position -1 is padding.
+ */
+typedef struct {
+    int32_t pos;
+    float score;
+} csa2_cand;
+
+/*
+ * A Full layer's share on one shard: every shard position scored as
+ * csa2_index_full scores it (T = 1), and cand[b][0..pool_k) <- the
+ * min(pool_k, n_r[b]) best with their scores and global positions (shard
+ * position + pos0[b]), in unspecified order, then (-1, 0) padding.  pos0:
+ * device int32 [batch], >= 0, pos0 + n_r < 2^31; cand: 8-byte aligned device
+ * array [batch][pool_k].  Other arguments and limits as csa2_index_full.
+ */
+CSA2_API csa2_status csa2_cp_index_local(const csa2_cache* shard, const int32_t* pos0, const void* q_idx,
+                                         csa2_dtype q_dtype, const float* head_w, int H_I, int pool_k,
+                                         csa2_cand* cand, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * A Reindex layer's share on one shard: the entries of the global pool
+ * pool_idx[b][0..pool_k) that this shard holds (pos0[b] <= t < pos0[b] +
+ * n_r[b]; the others and -1 padding are skipped) are rescored as
+ * csa2_index_reindex rescores them, and cand[b][0..top_k) <- the min(top_k,
+ * owned) best with their scores and global positions, then (-1, 0) padding.
+ */
+CSA2_API csa2_status csa2_cp_reindex_local(const csa2_cache* shard, const int32_t* pos0, const void* q_idx,
+                                           csa2_dtype q_dtype, const float* head_w, int H_I,
+                                           const int32_t* pool_idx, int pool_k, int top_k, csa2_cand* cand,
+                                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The selection after the all-gather: cand is [R][batch][n_cand] (rank r's
+ * candidates of sequence b at cand + (r * batch + b) * n_cand).  For each b, of
+ * the candidates with 0 <= pos < seq_lens_global[b] (device int32 [batch]),
+ *     out_a[b][0..n_a) <- the min(n_a, count) best positions,
+ *     out_b[b][0..n_b) <- the min(n_b, count) best (a subset of out_a; n_b = 0
+ *                         and out_b = NULL for none),
+ * each a set in unspecified order followed by -1 padding, ties at the cutoff
+ * broken arbitrarily.  Positions must be distinct.  1 <= n_b <= n_a <= 16384
+ * (or n_b = 0), R * n_cand <= 2^24.  ws is a separate workspace of
+ * csa2_cp_merge_workspace_bytes(R, batch, n_cand) bytes (0 on invalid
+ * arguments), cleared once with csa2_workspace_init.
+ */
+CSA2_API size_t csa2_cp_merge_workspace_bytes(int R, int batch, int n_cand);
+CSA2_API csa2_status csa2_cp_merge_select(const csa2_cand* cand, int R, int batch, int n_cand,
+                                          const int32_t* seq_lens_global, int n_a, int32_t* out_a, int n_b,
+                                          int32_t* out_b, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * A layer's attention on one shard: with the global attended set S of
+ * csa2_sparse_swa_attn (T = 1, p = seq_lens_global[b] - 1, window ∪ the
+ * top-k entries topk_idx[b][0..top_k) that are global positions), this shard
+ * attends over S ∩ shard and writes that part's normalised output and
+ * log-sum-exp: out fp32 [batch][H][dim], lse fp32 [batch][H] (required; an
+ * empty part gives out = 0, lse = -inf).  Top-k entries must be distinct;
+ * entries < -1 or >= seq_lens_global[b] set CSA2_ERR_DEVICE_BOUNDS.  The
+ * window rows come from the FP4 cache.  Other arguments as
+ * csa2_sparse_swa_attn.
+ */
+CSA2_API csa2_status csa2_cp_sparse_swa_attn(const csa2_cache* shard, const int32_t* pos0,
+                                             const int32_t* seq_lens_global, const void* q_bf16, int H,
+                                             const int32_t* topk_idx, int top_k, int window, float sm_scale,
+                                             float* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The merge of R attention parts over disjoint parts of one attended set:
+ * part r's output at outs + r * out_stride (fp32 [batch][H][dim]) and its lse
+ * at lses + r * lse_stride (fp32 [batch][H]); strides in floats, so that both
+ * may sit in one all-gathered buffer.  Per (b, h):
+ *     lse = log sum_r exp(lse_r),   out = sum_r exp(lse_r - lse) out_r,
+ * a part with lse_r = -inf contributing nothing (all empty: out = 0, lse =
+ * -inf).  out fp32 [batch][H][dim]; lse nullable.  R >= 1; with R > 1,
+ * out_stride >= batch * H * dim and lse_stride >= batch * H.  Pointers 4-byte
+ * aligned.
+ */
+CSA2_API csa2_status csa2_lse_merge(int R, int batch, int H, int dim, const float* outs, int64_t out_stride,
+                                    const float* lses, int64_t lse_stride, float* out, float* lse, void* stream);
 
 /*
  * Synchronise `stream`, then return the sticky device status recorded in the

@@ -69,3 +69,34 @@ def run_gpu_stack(cache, w, layers, ws=None):
 def attn_errors(got, want):
     d = np.abs(np.asarray(got, dtype=np.float64) - want)
     return float(d.max()), float(d.mean())
+
+
+def build_gpu_shards(w, R, seed=0, lens=None, q_idx0=None):
+    """The cache of every rank of an R-way context-parallel split: shard r of
+    sequence b holds positions wl.shard_bounds(L_b, R)[r] of the seeded inputs
+    (written through csa2_kv_append_quant into a contiguous cache of its own).
+    Returns [(cache, pos0 int32 [B] on the device)] per rank."""
+    lens = wl.seq_lens(w, seed) if lens is None else np.asarray(lens, dtype=np.int32)
+    if q_idx0 is None:
+        q_idx0 = wl.layer_queries(w, 0, seed)["q_idx"]
+    bounds = [wl.shard_bounds(int(lens[b]), R) for b in range(w.batch)]
+    xs = [wl.latent(w, b, int(lens[b]), seed) for b in range(w.batch)]
+    ks = [wl.index_keys(w, b, int(lens[b]), q_idx0[b, w.T - 1], seed)[0] for b in range(w.batch)]
+    shards = []
+    sp = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for r in range(R):
+        n = [bounds[b][r][1] for b in range(w.batch)]
+        cap = max(64, (max(n) + 63) // 64 * 64)
+        cache = csa2.Cache(w.batch, w.batch * cap, w.D, w.D_I, w.row_stride, w.idx_key_dtype, n, None, w.page_size,
+                           cap)
+        for b in range(w.batch):
+            p0, nb = bounds[b][r]
+            v = cache.view(b)
+            for t0 in range(0, nb, APPEND_CHUNK):
+                t1 = min(nb, t0 + APPEND_CHUNK)
+                sp.fill_(t0)
+                csa2.kv_append_quant(v, xs[b][p0 + t0:p0 + t1][None].cuda(), sp, ks[b][p0 + t0:p0 + t1][None].cuda())
+        pos0 = torch.tensor([bounds[b][r][0] for b in range(w.batch)], dtype=torch.int32, device="cuda")
+        shards.append((cache, pos0))
+    torch.cuda.synchronize()
+    return shards

@@ -220,3 +220,64 @@ def test_export_import_arguments_rejected_on_host(lib):
         assert fn(ctypes.byref(c), 0x30000, 4, None, 0x50000, None, None) == csa2.ERR_INVALID_ARG
         assert fn(ctypes.byref(c), 0x30000, 4, 0x40002, 0x50000, None, None) == csa2.ERR_INVALID_ARG
         assert fn(ctypes.byref(c), 0x30000, 0, 0x40000, 0x50000, None, None) == csa2.OK   # nothing to copy
+
+
+def test_context_parallel_arguments_rejected_on_host(lib):
+    c = fake_cache()
+    big = 1 << 40
+
+    def local(pos0=0x30100, cand=0x90000, pool_k=16384, H_I=32):
+        return lib.csa2_cp_index_local(ctypes.byref(c), pos0, 0x40000, csa2.BF16, 0x50000, H_I, pool_k, cand, 0x80000,
+                                       big, None)
+
+    assert local(pos0=None) == csa2.ERR_INVALID_ARG
+    assert local(pos0=0x30102) == csa2.ERR_INVALID_ARG
+    assert local(cand=None) == csa2.ERR_INVALID_ARG
+    assert local(cand=0x90004) == csa2.ERR_INVALID_ARG          # candidates are 8-byte pairs
+    assert local(pool_k=16385) == csa2.ERR_INVALID_ARG
+    assert local(H_I=65) == csa2.ERR_INVALID_ARG
+
+    def reindex(pool=0x60000, pool_k=16384, top_k=2048, cand=0x90000):
+        return lib.csa2_cp_reindex_local(ctypes.byref(c), 0x30100, 0x40000, csa2.BF16, 0x50000, 32, pool, pool_k,
+                                         top_k, cand, 0x80000, big, None)
+
+    assert reindex(pool=None) == csa2.ERR_INVALID_ARG
+    assert reindex(pool=0x60004) == csa2.ERR_INVALID_ARG
+    assert reindex(top_k=16385) == csa2.ERR_INVALID_ARG
+    assert reindex(cand=0x90004) == csa2.ERR_INVALID_ARG
+
+    # the merge workspace: histograms, four candidate buffers and the per-sequence candidates
+    n = lib.csa2_cp_merge_workspace_bytes(8, 1, 16384)
+    assert n >= 8 * 16384 * (4 * 8 + 8) and n % 256 == 0
+    assert lib.csa2_cp_merge_workspace_bytes(0, 1, 16384) == 0
+    assert lib.csa2_cp_merge_workspace_bytes(8, 1, 0) == 0
+    assert lib.csa2_cp_merge_workspace_bytes(1025, 1, 16384) == 0     # more than 2^24 candidates
+
+    def merge(cand=0x90000, n_a=16384, out_a=0xA0000, n_b=2048, out_b=0xB0000, ws_bytes=n, lens=0x30000):
+        return lib.csa2_cp_merge_select(cand, 8, 1, 16384, lens, n_a, out_a, n_b, out_b, 0x80000, ws_bytes, None)
+
+    assert merge(cand=0x90004) == csa2.ERR_INVALID_ARG
+    assert merge(lens=None) == csa2.ERR_INVALID_ARG
+    assert merge(n_a=0) == csa2.ERR_INVALID_ARG
+    assert merge(n_a=16385) == csa2.ERR_INVALID_ARG
+    assert merge(n_b=16384 + 1) == csa2.ERR_INVALID_ARG
+    assert merge(out_b=None) == csa2.ERR_INVALID_ARG
+    assert merge(out_a=0xA0004) == csa2.ERR_INVALID_ARG
+    assert merge(ws_bytes=n - 1) == csa2.ERR_INVALID_ARG
+
+    def attn(lse=0x70000, H=64, top_k=2048, window=128, topk=0x60000, glens=0x30000):
+        return lib.csa2_cp_sparse_swa_attn(ctypes.byref(c), 0x30100, glens, 0x40000, H, topk, top_k, window, 0.0,
+                                           0xA0000, lse, 0x80000, big, None)
+
+    assert attn(lse=None) == csa2.ERR_INVALID_ARG                  # the merge needs every part's lse
+    assert attn(glens=None) == csa2.ERR_INVALID_ARG
+    assert attn(topk=None) == csa2.ERR_INVALID_ARG
+    assert attn(window=16385) == csa2.ERR_INVALID_ARG
+    assert attn(H=24) == csa2.ERR_UNSUPPORTED
+
+    def merge_attn(R=2, out_stride=64 * 512, lse_stride=64):
+        return lib.csa2_lse_merge(R, 1, 64, 512, 0x90000, out_stride, 0xA0000, lse_stride, 0xB0000, None, None)
+
+    assert merge_attn(R=0) == csa2.ERR_INVALID_ARG
+    assert merge_attn(out_stride=64 * 512 - 1) == csa2.ERR_INVALID_ARG
+    assert merge_attn(lse_stride=63) == csa2.ERR_INVALID_ARG
