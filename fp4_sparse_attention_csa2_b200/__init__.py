@@ -27,6 +27,7 @@ ABI_FUNCTIONS = (
     "csa2_cp_index_local", "csa2_cp_reindex_local", "csa2_cp_merge_workspace_bytes", "csa2_cp_merge_select",
     "csa2_cp_sparse_swa_attn", "csa2_lse_merge",
     "csa2_read_device_status", "csa2_status_string", "csa2_debug_set_wait_limit", "csa2_debug_default_wait_limit",
+    "csa2_debug_encode",
 )
 
 
@@ -100,13 +101,15 @@ def lib():
         L.csa2_debug_set_wait_limit.argtypes = [ctypes.c_uint32]
         L.csa2_debug_default_wait_limit.restype = ctypes.c_uint32
         L.csa2_debug_default_wait_limit.argtypes = []
+        L.csa2_debug_encode.argtypes = [i32, vp, ctypes.c_int64, vp, vp]
         for name in ("csa2_workspace_init", "csa2_kv_append_quant", "csa2_kv_export_rows", "csa2_kv_import_rows",
                      "csa2_index_scores", "csa2_index_full",
                      "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update",
                      "csa2_sparse_swa_attn", "csa2_ring_append", "csa2_sparse_swa_attn_local",
                      "csa2_layer_step", "csa2_prefill_layer", "csa2_read_device_status",
                      "csa2_debug_set_wait_limit", "csa2_cp_index_local", "csa2_cp_reindex_local",
-                     "csa2_cp_merge_select", "csa2_cp_sparse_swa_attn", "csa2_lse_merge"):
+                     "csa2_cp_merge_select", "csa2_cp_sparse_swa_attn", "csa2_lse_merge",
+                     "csa2_debug_encode"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -185,6 +188,34 @@ class Cache:
                              c.max_pages, c.page_size, c.dim, c.idx_dim, c.row_stride, 0, c.n_slots,
                              c.idx_key_dtype)
         v.owner = self
+        return v
+
+    def shard_view(self, b, pos0, n):
+        """A batch-1 cache whose positions 0 .. n-1 are positions pos0 ..
+        pos0 + n - 1 of sequence b of this cache (sharing its memory; its own
+        seq_lens = [n]): one rank's shard for the context-parallel calls.
+        pos0 must be a multiple of 64 (of the page size when paged)."""
+        c = self.c
+        v = _View()
+        v.lens = torch.tensor([n], dtype=torch.int32, device=self.rows.device)
+        if self.page_table is None:
+            if pos0 % 64 or pos0 + n > self.seq_stride_slots:
+                raise ValueError("shard outside the sequence or not 64-aligned")
+            st = self.seq_stride_slots - pos0
+            base = b * self.seq_stride_slots + pos0
+            v.c = csa2_cache(c.kv_rows + base * self.row_stride,
+                             c.idx_keys + base * self.idx_dim * self.idx_keys.element_size(), None,
+                             v.lens.data_ptr(), 1, 0, c.page_size, c.dim, c.idx_dim, c.row_stride, st,
+                             self.n_slots - base, c.idx_key_dtype)
+        else:
+            if pos0 % self.page_size:
+                raise ValueError("a paged shard starts on a page boundary")
+            first = pos0 // self.page_size
+            v.c = csa2_cache(c.kv_rows, c.idx_keys, c.page_table + 4 * (b * c.max_pages + first), v.lens.data_ptr(),
+                             1, c.max_pages - first, c.page_size, c.dim, c.idx_dim, c.row_stride, 0, c.n_slots,
+                             c.idx_key_dtype)
+        v.owner = self
+        v.batch, v.dim = 1, self.dim
         return v
 
     @property
@@ -406,6 +437,12 @@ def lse_merge(outs, lses, out, lse=None, stream=None):
     _check(lib().csa2_lse_merge(R, B, H, D, ctypes.c_void_p(outs.data_ptr()), outs.stride(0),
                                 ctypes.c_void_p(lses.data_ptr()), lses.stride(0), _p(out), _p(lse), _stream(stream)),
            "lse_merge")
+
+
+def debug_encode(x, codes, fmt, stream=None):
+    """Diagnostic: the quantiser's E2M1 (fmt 0) or E4M3 (fmt 1) conversion of
+    every fp32 value of x into codes (uint8, same length)."""
+    _check(lib().csa2_debug_encode(fmt, _p(x), x.numel(), _p(codes), _stream(stream)), "debug_encode")
 
 
 def read_device_status(ws, stream=None):

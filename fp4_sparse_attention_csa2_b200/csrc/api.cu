@@ -775,6 +775,13 @@ csa2_status csa2_debug_set_wait_limit(uint32_t tries) {
 
 uint32_t csa2_debug_default_wait_limit(void) { return tc::kWaitLimit; }
 
+csa2_status csa2_debug_encode(int format, const float* x, int64_t n, uint8_t* codes, void* stream) {
+    if ((format != 0 && format != 1) || n < 0 || (n > 0 && (!x || !codes || !aligned4(x))))
+        return CSA2_ERR_INVALID_ARG;
+    if (n == 0) return CSA2_OK;
+    return cuda_status(launch_debug_encode(format, x, n, codes, static_cast<cudaStream_t>(stream), num_sms()));
+}
+
 const char* csa2_status_string(csa2_status s) {
     switch (s) {
         case CSA2_OK: return "CSA2_OK";

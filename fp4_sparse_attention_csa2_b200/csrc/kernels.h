@@ -51,6 +51,10 @@ cudaError_t launch_append_quant(const DevCache& c, const void* x, const void* id
                                 const int32_t* start_pos, int n_new, uint32_t* status, cudaStream_t st,
                                 int num_sms);
 
+// Diagnostic: the quantiser's conversions on arbitrary fp32 values (format 0:
+// E2M1 codes, 1: E4M3 codes), one code per byte.
+cudaError_t launch_debug_encode(int format, const float* x, int64_t n, uint8_t* out, cudaStream_t st, int num_sms);
+
 // Stored rows and keys of positions start_pos[b] + i between the cache and
 // packed buffers [batch][n][dim / 2 + dim / 16] and [batch][n][key bytes].
 cudaError_t launch_rows_io(const DevCache& c, bool to_buffers, const int32_t* start_pos, int n, void* rows, void* keys,

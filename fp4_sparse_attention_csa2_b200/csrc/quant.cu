@@ -143,7 +143,49 @@ k_rows_io(DevCache c, const int32_t* __restrict__ start_pos, int n, uint8_t* row
     }
 }
 
+// Diagnostic: the quantiser's own conversions (cvt_e2m1x8 for the codes,
+// cvt_e4m3x2 for the scales and index keys) applied to arbitrary fp32 values,
+// one code per output byte (E2M1 in the low nibble).  A thread takes 8
+// consecutive values; a tail shorter than 8 is padded with zeros that are not
+// written back.
+__global__ void __launch_bounds__(256)
+k_debug_encode(int format, const float* __restrict__ x, int64_t n, uint8_t* __restrict__ out) {
+    pdl_begin();
+    const int64_t groups = (n + 7) / 8;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i0 = g * 8;
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = i0 + k < n ? x[i0 + k] : 0.0f;
+        uint8_t c[8];
+        if (format == 0) {
+            const uint32_t w = cvt_e2m1x8(v);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                c[2 * k] = (uint8_t)((w >> (8 * k)) & 0xF);
+                c[2 * k + 1] = (uint8_t)((w >> (8 * k + 4)) & 0xF);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint16_t h = cvt_e4m3x2(v[2 * k + 1], v[2 * k]);
+                c[2 * k] = (uint8_t)(h & 0xFF);
+                c[2 * k + 1] = (uint8_t)(h >> 8);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (i0 + k < n) out[i0 + k] = c[k];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_debug_encode(int format, const float* x, int64_t n, uint8_t* out, cudaStream_t st, int num_sms) {
+    int64_t blocks = (n / 8 + 255) / 256 + 1;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    return launch_pdl(k_debug_encode, dim3((unsigned)blocks), dim3(256), 0, st, format, x, n, out);
+}
 
 cudaError_t launch_rows_io(const DevCache& c, bool to_buffers, const int32_t* start_pos, int n, void* rows, void* keys,
                            uint32_t* status, cudaStream_t st) {

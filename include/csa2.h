@@ -503,6 +503,19 @@ CSA2_API csa2_status csa2_debug_set_wait_limit(uint32_t tries);
 /* The default try count of those waits (the value the library starts with). */
 CSA2_API uint32_t csa2_debug_default_wait_limit(void);
 
+/*
+ * Diagnostic: the conversions csa2_kv_append_quant uses, applied to n
+ * arbitrary fp32 values x (device, 4-byte aligned), one code per byte into
+ * codes (device): format 0 gives the E2M1 code of each value (round to
+ * nearest, ties to even, saturating at 6, sign kept; the low nibble), format
+ * 1 its E4M3 code (the same rules, saturating at 448), as the quantiser forms
+ * FP4 codes from quotients x / s and E4M3 scales and keys ([TLDR] paragraph
+ * 4).  It lets a test check those conversions on every fp32 input, not only
+ * on the quotients that bf16 inputs reach.  Non-finite inputs give whatever
+ * the conversion instruction gives.
+ */
+CSA2_API csa2_status csa2_debug_encode(int format, const float* x, int64_t n, uint8_t* codes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

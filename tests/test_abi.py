@@ -281,3 +281,11 @@ def test_context_parallel_arguments_rejected_on_host(lib):
     assert merge_attn(R=0) == csa2.ERR_INVALID_ARG
     assert merge_attn(out_stride=64 * 512 - 1) == csa2.ERR_INVALID_ARG
     assert merge_attn(lse_stride=63) == csa2.ERR_INVALID_ARG
+
+
+def test_debug_encode_arguments_rejected_on_host(lib):
+    assert lib.csa2_debug_encode(2, 0x10000, 8, 0x20000, None) == csa2.ERR_INVALID_ARG
+    assert lib.csa2_debug_encode(0, 0x10000, -1, 0x20000, None) == csa2.ERR_INVALID_ARG
+    assert lib.csa2_debug_encode(1, 0x10002, 8, 0x20000, None) == csa2.ERR_INVALID_ARG
+    assert lib.csa2_debug_encode(0, None, 8, 0x20000, None) == csa2.ERR_INVALID_ARG
+    assert lib.csa2_debug_encode(0, None, 0, None, None) == csa2.OK      # nothing to convert

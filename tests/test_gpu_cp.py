@@ -71,6 +71,7 @@ def run_cp_stack(w, shards, layers, lens):
 
 @pytest.mark.parametrize("name,L,R,kw", [
     ("long64k", 20000, 2, {}),                                   # 20,000 merged candidates: the two-pass select
+    ("long64k", 50000, 2, {}),                                   # shards over 16,384 positions: two-pass shard pools
     ("long64k", 50000, 3, {"pool_k": 4096, "top_k": 512}),       # 12,288 candidates: the one-CTA select
     ("tiny4k", 4096, 4, {}),                                     # fp32 keys (CUDA-core scoring), 16 x 128 heads
     ("batch32_paged", 30000, 2, {"batch": 3}),                   # ragged sequences, each split over the ranks
@@ -225,3 +226,27 @@ def test_stack_class_on_one_rank():
         compare_stack(w, ref, got, layers, [(0, 0)])
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name,L,R,kw", [
+    ("long64k", 50000, 3, {}),                                   # contiguous cache
+    ("batch32_paged", 40000, 2, {"batch": 1, "lens": ("fixed", 40000)}),   # paged cache, page-aligned shards
+])
+def test_cp_on_shard_views_of_one_cache(name, L, R, kw):
+    # the shards as views of one cache (Cache.shard_view): the same results
+    # as the oracle on the whole sequence
+    from gpu_harness import build_gpu_cache
+    w = wl.scaled(wl.WORKLOADS[name], L, T=1, **kw)
+    layers = [wl.layer_queries(w, l) for l in range(len(w.pattern))]
+    lens = wl.seq_lens(w)
+    ref = build_ref_cache(w, layers=layers)
+    dev = build_gpu_cache(w, q_idx0=layers[0]["q_idx"])
+    step = (L + R - 1) // R // 64 * 64 + 64
+    shards = []
+    for r in range(R):
+        p0 = min(r * step, L)
+        v = dev.shard_view(0, p0, min(step, L - p0))
+        shards.append((v, torch.tensor([p0], dtype=torch.int32, device="cuda")))
+    got, status = run_cp_stack(w, shards, layers, lens)
+    assert all(s == csa2.OK for s in status), status
+    compare_stack(w, ref, got, layers, [(0, 0)])

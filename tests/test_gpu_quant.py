@@ -2,6 +2,9 @@
 csa2_kv_append_quant are bit-exact with the oracle on the same seeded inputs
 (format: tldrocket.com "DeepSeek AI Released DeepSeek-V4.1-Flash ...",
 paragraph 4)."""
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -140,3 +143,28 @@ def test_out_of_range_append_flags_status():
     assert csa2.read_device_status(ws) == csa2.ERR_DEVICE_BOUNDS
     rows = cache.rows.cpu().numpy()
     assert np.all(rows[60:64, :72] != 0) and csa2.read_device_status(ws) == csa2.OK
+
+
+def _sums_on_device(codes, bits, fin):
+    """Per block: the two position-weighted sums of tests/golden/make_encoder_sweep.py."""
+    c = codes.to(torch.int64) * fin
+    w1 = (((bits * 2654435761) & 0xFFFFFFFF) >> 12) + 1      # int64 products wrap: the low 32 bits are exact
+    w2 = (((bits * 40503) & 0xFFFFFFFF) >> 12) + 1
+    return [int((c * w1).sum()), int((c * w2).sum()), int(fin.sum())]
+
+
+@pytest.mark.parametrize("fmt,name", [(0, "e2m1"), (1, "e4m3")])
+def test_encoders_every_fp32_input(fmt, name):
+    # the quantiser's conversions on all 2^32 fp32 bit patterns against the
+    # oracle's encoders (tests/golden/encoder_sweep.json, written by
+    # tests/golden/make_encoder_sweep.py from the oracle alone), block by block
+    with open(os.path.join(os.path.dirname(__file__), "golden", "encoder_sweep.json")) as f:
+        golden = json.load(f)
+    nb = 1 << golden["block_bits"]
+    codes = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    for blk, want in enumerate(golden[name]):
+        bits = torch.arange(blk * nb, (blk + 1) * nb, dtype=torch.int64, device="cuda")
+        x = torch.where(bits >= (1 << 31), bits - (1 << 32), bits).to(torch.int32).view(torch.float32)
+        csa2.debug_encode(x, codes, fmt)
+        fin = torch.isfinite(x).to(torch.int64)
+        assert _sums_on_device(codes, bits, fin) == list(want), (name, blk)

@@ -160,3 +160,24 @@ def test_dequant_is_code_times_scale():
             s = torch.tensor([rows[r][32 + blk]], dtype=torch.uint8).view(torch.float8_e4m3fn).double().item()
             err = np.abs(deq[blk * 16:(blk + 1) * 16] - xd[blk * 16:(blk + 1) * 16])
             assert np.all(err <= 1.0 * s + 1e-12)
+
+
+def test_encoder_sweep_golden_is_the_oracles():
+    # the stored per-block sums of the exhaustive encoder sweep are the oracle's
+    # own (recomputed here for one block of values in [2^-7, 2) and one of
+    # negative values), and every block counts its finite patterns
+    import json
+    import os
+    import sys
+    here = os.path.join(os.path.dirname(__file__), "golden")
+    sys.path.insert(0, here)
+    import make_encoder_sweep as mk
+    with open(os.path.join(here, "encoder_sweep.json")) as f:
+        g = json.load(f)
+    assert g["block_bits"] == mk.BLOCK_BITS and len(g["e2m1"]) == len(g["e4m3"]) == mk.N_BLOCKS
+    for blk in (15, 48):
+        _, sums = mk._work(blk)
+        assert [list(sums["e2m1"]), list(sums["e4m3"])] == [g["e2m1"][blk], g["e4m3"][blk]]
+    # the 2 x 2^23 patterns with exponent 255 (Inf / NaN) are the only ones left out
+    n_fin = [g["e4m3"][b][2] for b in range(mk.N_BLOCKS)]
+    assert sum(n_fin) == (1 << 32) - 2 * (1 << 23)
