@@ -638,113 +638,43 @@ def prefill_line(w, lens, seed, reps, stream, world, T):
 
 def cp_decode_line(w, lens, layers, reps, stream, R=8):
     """One rank's device work in an R-way context-parallel decode step of the
-    stack (the sequence's positions split into R shards of L / R): its shard
-    calls, the merge selections over all R ranks' candidates and the
-    log-sum-exp merges of all R attention parts.  The ranks' candidates and
-    parts are computed once beforehand from the real shards (shard views of
-    the replicas); the all-gathers between ranks are not in the timed region
-    (one GPU here).  The timed steps rotate over every shard of every replica
-    (R x replicas shards, more key bytes than the L2 holds)."""
-    import fp4_sparse_attention_csa2_b200 as csa2
-    L = int(lens[0])
-    n = L // R
-    if w.batch != 1 or w.T != 1 or w.paged or n % 64 or n * R != L:
+    stack (runner.CpRankStep: the sequence's positions in R shards of L / R;
+    its shard calls, the merge selections over all R ranks' candidates and the
+    log-sum-exp merges of all R attention parts).  The all-gathers between
+    ranks are not in the timed region (one GPU here).  The timed steps rotate
+    over every shard of every replica (R x replicas shards, more key bytes than
+    the L2 holds)."""
+    from fp4_sparse_attention_csa2_b200.runner import CpRankStep
+    try:
+        cp = CpRankStep(w, lens, layers, reps, R)
+    except ValueError:
         return None
-    B, H, D = 1, w.H, w.D
-    shards = [(c.shard_view(0, r * n, n), r) for c in reps for r in range(R)]
-    pos0 = [torch.tensor([r * n], dtype=torch.int32, device="cuda") for r in range(R)]
-    glens = torch.as_tensor(lens.astype(np.int32)).cuda()
-    ws = torch.empty(csa2.workspace_bytes(shards[0][0], 1, H, w.pool_k, w.top_k, w.window), dtype=torch.uint8,
-                     device="cuda")
-    csa2.workspace_init(ws)
-    mws = torch.empty(csa2.cp_merge_workspace_bytes(R, B, w.pool_k), dtype=torch.uint8, device="cuda")
-    csa2.workspace_init(mws)
-    dl = [{k: v.cuda() for k, v in L_.items()} for L_ in layers]
-    pool = torch.empty((B, w.pool_k), dtype=torch.int32, device="cuda")
-    topk = torch.empty((B, w.top_k), dtype=torch.int32, device="cuda")
-    gpool = torch.empty((R, B, w.pool_k, 2), dtype=torch.int32, device="cuda")
-    gtopk = torch.empty((R, B, w.top_k, 2), dtype=torch.int32, device="cuda")
-    gout = torch.empty((len(w.pattern), R, B, H, D), dtype=torch.float32, device="cuda")
-    glse = torch.empty((len(w.pattern), R, B, H), dtype=torch.float32, device="cuda")
-    cand_pool = torch.empty((B, w.pool_k, 2), dtype=torch.int32, device="cuda")
-    cand_topk = torch.empty((B, w.top_k, 2), dtype=torch.int32, device="cuda")
-    part_o = torch.empty((B, H, D), dtype=torch.float32, device="cuda")
-    part_l = torch.empty((B, H), dtype=torch.float32, device="cuda")
-    out = torch.empty((B, H, D), dtype=torch.float32, device="cuda")
-    lse = torch.empty((B, H), dtype=torch.float32, device="cuda")
-    # every rank's candidates and attention parts, from the first replica's shards
     with torch.cuda.stream(stream):
-        for l, m in enumerate(w.pattern):
-            if m == "F":
-                for r in range(R):
-                    csa2.cp_index_local(shards[r][0], pos0[r], dl[l]["q_idx"], dl[l]["w"], w.pool_k, gpool[r], ws)
-                csa2.cp_merge_select(gpool, glens, w.pool_k, pool, mws, n_b=w.top_k, out_b=topk)
-            elif m == "R":
-                for r in range(R):
-                    csa2.cp_reindex_local(shards[r][0], pos0[r], dl[l]["q_idx"], dl[l]["w"], pool, w.top_k,
-                                          gtopk[r], ws)
-                csa2.cp_merge_select(gtopk, glens, w.top_k, topk, mws)
-            for r in range(R):
-                csa2.cp_sparse_swa_attn(shards[r][0], pos0[r], glens, dl[l]["q"], topk, w.window, gout[l, r],
-                                        glse[l, r], ws)
-    stream.synchronize()
-    for x in (ws, mws):
-        st = csa2.read_device_status(x, stream)
-        if st != csa2.OK:
-            raise RuntimeError("context parallel: device status " + csa2.status_string(st))
-
-    def step(sh):
-        shard, r = sh
-        for l, m in enumerate(w.pattern):
-            if m == "F":
-                csa2.cp_index_local(shard, pos0[r], dl[l]["q_idx"], dl[l]["w"], w.pool_k, cand_pool, ws)
-                csa2.cp_merge_select(gpool, glens, w.pool_k, pool, mws, n_b=w.top_k, out_b=topk)
-            elif m == "R":
-                csa2.cp_reindex_local(shard, pos0[r], dl[l]["q_idx"], dl[l]["w"], pool, w.top_k, cand_topk, ws)
-                csa2.cp_merge_select(gtopk, glens, w.top_k, topk, mws)
-            csa2.cp_sparse_swa_attn(shard, pos0[r], glens, dl[l]["q"], topk, w.window, part_o, part_l, ws)
-            csa2.lse_merge(gout[l], glse[l], out, lse)
-
-    ms = timed_launches(step, shards, stream, calls_per_rep=1, replays=5)
-    # the step's pieces: a Full layer's indexing share (shard scoring and pool,
-    # merge of all ranks' pools), a Reindex layer's, and one layer's attention
-    lf, lr = w.pattern.index("F"), w.pattern.index("R") if "R" in w.pattern else None
-    lu = len(w.pattern) - 1
-
-    def full_part(sh):
-        csa2.cp_index_local(sh[0], pos0[sh[1]], dl[lf]["q_idx"], dl[lf]["w"], w.pool_k, cand_pool, ws)
-        csa2.cp_merge_select(gpool, glens, w.pool_k, pool, mws, n_b=w.top_k, out_b=topk)
-
-    def reindex_part(sh):
-        csa2.cp_reindex_local(sh[0], pos0[sh[1]], dl[lr]["q_idx"], dl[lr]["w"], pool, w.top_k, cand_topk, ws)
-        csa2.cp_merge_select(gtopk, glens, w.top_k, topk, mws)
-
-    def attn_part(sh):
-        csa2.cp_sparse_swa_attn(sh[0], pos0[sh[1]], glens, dl[lu]["q"], topk, w.window, part_o, part_l, ws)
-        csa2.lse_merge(gout[lu], glse[lu], out, lse)
-
-    f_ms = timed_launches(full_part, shards, stream, calls_per_rep=1, replays=5)
-    r_ms = timed_launches(reindex_part, shards, stream, calls_per_rep=1, replays=5) if lr is not None else None
-    a_ms = timed_launches(attn_part, shards, stream, calls_per_rep=1, replays=5)
-    for x in (ws, mws):
-        st = csa2.read_device_status(x, stream)
-        if st != csa2.OK:
-            raise RuntimeError("context parallel: device status after timing " + csa2.status_string(st))
+        ms = timed_launches(cp.step, cp.shards, stream, calls_per_rep=1, replays=5)
+        # the step's pieces: a Full layer's indexing share (shard scoring and
+        # pool, merge of all ranks' pools), a Reindex layer's, one layer's attention
+        f_ms = timed_launches(cp.full_part, cp.shards, stream, calls_per_rep=1, replays=5)
+        r_ms = timed_launches(cp.reindex_part, cp.shards, stream, calls_per_rep=1, replays=5) \
+            if "R" in w.pattern else None
+        a_ms = timed_launches(cp.attn_part, cp.shards, stream, calls_per_rep=1, replays=5)
+    cp.check("after timing")
     key = 64 if w.idx_key_dtype == wl.E4M3 else 256
-    n_f = w.pattern.count("F")
-    n_r = w.pattern.count("R")
-    gathered = R * (n_f * w.pool_k * 8 + n_r * w.top_k * 8 + len(w.pattern) * H * (D + 1) * 4)
-    return {"ranks": R, "shard_positions": n, "us_per_step_rank": round(ms * 1e3, 2),
+    n_f, n_r = w.pattern.count("F"), w.pattern.count("R")
+    gathered = R * (n_f * w.pool_k * 8 + n_r * w.top_k * 8 + len(w.pattern) * w.H * (w.D + 1) * 4)
+    line = {"ranks": R, "shard_positions": cp.n, "us_per_step_rank": round(ms * 1e3, 2),
             "us_full_index_share": round(f_ms * 1e3, 2),
             "us_reindex_share": None if r_ms is None else round(r_ms * 1e3, 2),
             "us_attention_layer": round(a_ms * 1e3, 2),
             "layer_steps_per_s_compute": round(len(w.pattern) / (ms / 1e3), 1),
-            "shard_key_bytes_per_step": n * key * n_f,
+            "shard_key_bytes_per_step": cp.n * key * n_f,
             "allgather_bytes_per_step_rank": gathered,
             "allgathers_per_step": 2 * n_f + 2 * n_r + len(w.pattern) - n_f - n_r,
             "path": "per rank: csa2_cp_index_local / csa2_cp_reindex_local on its shard, csa2_cp_merge_select over "
                     "all ranks' candidates, csa2_cp_sparse_swa_attn on its shard, csa2_lse_merge of all parts; "
                     "the NCCL all-gathers between these are not timed (one GPU)"}
+    del cp
+    torch.cuda.empty_cache()
+    return line
 
 
 def step_bytes(w, lens, local=False):

@@ -213,3 +213,94 @@ class E2ERunner:
         if t1 is not None:
             self.d2h.wait_stream(self.stream)
             t1.record(self.d2h)
+
+
+class CpRankStep:
+    """One rank's device work in an R-way context-parallel decode step of the
+    stack, on one GPU: the sequence (batch 1, one query token) is split into R
+    shards of L / R positions, taken as shard views of the given caches.  The
+    candidates and attention parts of all R ranks are computed once from the
+    first cache's shards; step(shard) then runs one rank's calls of a step --
+    its shard calls, the merge selections over all ranks' candidates, the
+    log-sum-exp merges of all ranks' parts -- with no exchange in between."""
+
+    def __init__(self, w, lens, layers, caches, R=8):
+        L = int(lens[0])
+        n = L // R
+        if w.batch != 1 or w.T != 1 or w.paged or n % 64 or n * R != L:
+            raise ValueError("an even split of one contiguous sequence into 64-aligned shards")
+        self.w, self.R, self.n = w, R, n
+        H, D, B = w.H, w.D, 1
+        dev = "cuda"
+        self.shards = [(c.shard_view(0, r * n, n), r) for c in caches for r in range(R)]
+        self.pos0 = [torch.tensor([r * n], dtype=torch.int32, device=dev) for r in range(R)]
+        self.glens = torch.tensor([L], dtype=torch.int32, device=dev)
+        self.ws = torch.empty(csa2.workspace_bytes(self.shards[0][0], 1, H, w.pool_k, w.top_k, w.window),
+                              dtype=torch.uint8, device=dev)
+        csa2.workspace_init(self.ws)
+        self.mws = torch.empty(csa2.cp_merge_workspace_bytes(R, B, w.pool_k), dtype=torch.uint8, device=dev)
+        csa2.workspace_init(self.mws)
+        self.dl = [{k: v.cuda() for k, v in x.items()} for x in layers]
+        self.pool = torch.empty((B, w.pool_k), dtype=torch.int32, device=dev)
+        self.topk = torch.empty((B, w.top_k), dtype=torch.int32, device=dev)
+        self.gpool = torch.empty((R, B, w.pool_k, 2), dtype=torch.int32, device=dev)
+        self.gtopk = torch.empty((R, B, w.top_k, 2), dtype=torch.int32, device=dev)
+        self.gout = torch.empty((len(w.pattern), R, B, H, D), dtype=torch.float32, device=dev)
+        self.glse = torch.empty((len(w.pattern), R, B, H), dtype=torch.float32, device=dev)
+        self.cand_pool = torch.empty((B, w.pool_k, 2), dtype=torch.int32, device=dev)
+        self.cand_topk = torch.empty((B, w.top_k, 2), dtype=torch.int32, device=dev)
+        self.part_o = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+        self.part_l = torch.empty((B, H), dtype=torch.float32, device=dev)
+        self.out = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+        # every rank's candidates and attention parts, from the first cache's shards
+        for l, m in enumerate(w.pattern):
+            q = self.dl[l]
+            if m == "F":
+                for r in range(R):
+                    csa2.cp_index_local(self.shards[r][0], self.pos0[r], q["q_idx"], q["w"], w.pool_k, self.gpool[r],
+                                        self.ws)
+                csa2.cp_merge_select(self.gpool, self.glens, w.pool_k, self.pool, self.mws, n_b=w.top_k,
+                                     out_b=self.topk)
+            elif m == "R":
+                for r in range(R):
+                    csa2.cp_reindex_local(self.shards[r][0], self.pos0[r], q["q_idx"], q["w"], self.pool, w.top_k,
+                                          self.gtopk[r], self.ws)
+                csa2.cp_merge_select(self.gtopk, self.glens, w.top_k, self.topk, self.mws)
+            for r in range(R):
+                csa2.cp_sparse_swa_attn(self.shards[r][0], self.pos0[r], self.glens, q["q"], self.topk, w.window,
+                                        self.gout[l, r], self.glse[l, r], self.ws)
+        torch.cuda.synchronize()
+        self.check("after the set-up")
+
+    def check(self, when):
+        for x in (self.ws, self.mws):
+            st = csa2.read_device_status(x)
+            if st != csa2.OK:
+                raise RuntimeError("context parallel %s: device status %s" % (when, csa2.status_string(st)))
+
+    def full_part(self, sh, l=None):
+        w, q = self.w, self.dl[self.w.pattern.index("F") if l is None else l]
+        csa2.cp_index_local(sh[0], self.pos0[sh[1]], q["q_idx"], q["w"], w.pool_k, self.cand_pool, self.ws)
+        csa2.cp_merge_select(self.gpool, self.glens, w.pool_k, self.pool, self.mws, n_b=w.top_k, out_b=self.topk)
+
+    def reindex_part(self, sh, l=None):
+        w, q = self.w, self.dl[self.w.pattern.index("R") if l is None else l]
+        csa2.cp_reindex_local(sh[0], self.pos0[sh[1]], q["q_idx"], q["w"], self.pool, w.top_k, self.cand_topk,
+                              self.ws)
+        csa2.cp_merge_select(self.gtopk, self.glens, w.top_k, self.topk, self.mws)
+
+    def attn_part(self, sh, l=None):
+        w = self.w
+        l = len(w.pattern) - 1 if l is None else l
+        csa2.cp_sparse_swa_attn(sh[0], self.pos0[sh[1]], self.glens, self.dl[l]["q"], self.topk, w.window,
+                                self.part_o, self.part_l, self.ws)
+        csa2.lse_merge(self.gout[l], self.glse[l], self.out, self.lse)
+
+    def step(self, sh):
+        for l, m in enumerate(self.w.pattern):
+            if m == "F":
+                self.full_part(sh, l)
+            elif m == "R":
+                self.reindex_part(sh, l)
+            self.attn_part(sh, l)
