@@ -97,7 +97,11 @@ k_cp_attn_list(const int32_t* __restrict__ topk, int top_k, int window, const in
 }
 
 // out[b][h][d] = sum_r exp(lse_r - lse) out_r[b][h][d], lse = log sum_r
-// exp(lse_r), one thread per output element.
+// exp(lse_r), one thread per output element.  The parts are taken kMergeU at a
+// time, every load of a group issued before any is used, and merged online
+// (running maximum m, sum and accumulator rescaled by exp(m_old - m_new)).
+constexpr int kMergeU = 8;
+
 __global__ void __launch_bounds__(kThreads)
 k_lse_merge(int R, int batch, int H, int D, const float* __restrict__ outs, int64_t out_stride,
             const float* __restrict__ lses, int64_t lse_stride, float* __restrict__ out, float* __restrict__ lse) {
@@ -106,23 +110,32 @@ k_lse_merge(int R, int batch, int H, int D, const float* __restrict__ outs, int6
     if (e >= (int64_t)batch * H * D) return;
     const int64_t bh = e / D;
     const int d = (int)(e % D);
-    float m = -INFINITY;
-    for (int r = 0; r < R; ++r) m = fmaxf(m, lses[r * lse_stride + bh]);
-    if (m == -INFINITY) {
-        out[e] = 0.0f;
-        if (lse && d == 0) lse[bh] = -INFINITY;
-        return;
+    float m = -INFINITY, sum = 0.0f, acc = 0.0f;
+    for (int r0 = 0; r0 < R; r0 += kMergeU) {
+        float l[kMergeU], o[kMergeU];
+#pragma unroll
+        for (int k = 0; k < kMergeU; ++k) {
+            const bool in = r0 + k < R;
+            l[k] = in ? lses[(r0 + k) * lse_stride + bh] : -INFINITY;
+            o[k] = in ? outs[(r0 + k) * out_stride + e] : 0.0f;
+        }
+        float mn = m;
+#pragma unroll
+        for (int k = 0; k < kMergeU; ++k) mn = fmaxf(mn, l[k]);
+        if (mn == -INFINITY) continue;                 // nothing attended so far
+        const float c = expf(m - mn);                  // 0 while m is -inf
+        sum *= c;
+        acc *= c;
+#pragma unroll
+        for (int k = 0; k < kMergeU; ++k) {
+            const float wk = expf(l[k] - mn);          // 0 for an empty part
+            sum += wk;
+            acc += wk * o[k];
+        }
+        m = mn;
     }
-    float sum = 0.0f, acc = 0.0f;
-    for (int r = 0; r < R; ++r) {
-        const float l = lses[r * lse_stride + bh];
-        if (l == -INFINITY) continue;
-        const float w = expf(l - m);
-        sum += w;
-        acc += w * outs[r * out_stride + e];
-    }
-    out[e] = acc / sum;
-    if (lse && d == 0) lse[bh] = m + logf(sum);
+    out[e] = m == -INFINITY ? 0.0f : acc / sum;
+    if (lse && d == 0) lse[bh] = m == -INFINITY ? -INFINITY : m + logf(sum);
 }
 
 }  // namespace
