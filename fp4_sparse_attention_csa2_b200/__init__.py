@@ -12,7 +12,9 @@ import os
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libcsa2.so")
+# CSA2_LIBRARY=debug selects the debug build (NVTX ranges, device-side bounds
+# checks); it is never loaded otherwise
+LIB_PATH = os.path.join(HERE, "libcsa2_debug.so" if os.environ.get("CSA2_LIBRARY") == "debug" else "libcsa2.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_BOUNDS = range(6)
 FULL, REINDEX, REUSE = 0, 1, 2
@@ -65,7 +67,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError("libcsa2.so is not built; run `python -m fp4_sparse_attention_csa2_b200.build`")
+            raise RuntimeError("%s is not built; run `python -m fp4_sparse_attention_csa2_b200.build%s`"
+                               % (os.path.basename(LIB_PATH), " --debug" if "debug" in LIB_PATH else ""))
         L = ctypes.CDLL(LIB_PATH)
         vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         cp = ctypes.POINTER(csa2_cache)

@@ -5,6 +5,24 @@
 #include "../../include/csa2.h"
 #include "kernels.h"
 
+// NVTX ranges, one per C-ABI call (built with -DCSA2_NVTX, the debug build):
+// a profiler's timeline shows each call and the kernels it enqueued.  NVTX
+// is header-only and costs a branch per call when no tool is attached.
+#ifdef CSA2_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace csa2 {
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+}  // namespace csa2
+#define CSA2_RANGE(name) ::csa2::NvtxRange csa2_nvtx_range_(name)
+#else
+#define CSA2_RANGE(name) ((void)0)
+#endif
+
 namespace csa2 {
 
 // CSA2_OK, or the status csa2_index_reindex returns for these arguments

@@ -268,12 +268,14 @@ csa2_cache seq_view(const csa2_cache* c, int b, const int32_t* len) {
 extern "C" {
 
 size_t csa2_workspace_bytes(const csa2_cache* cache, int T, int H, int pool_k, int top_k, int window) {
+    CSA2_RANGE("csa2_workspace_bytes");
     Layout L;
     if (!make_layout(cache, T, H, pool_k, top_k, window, &L)) return 0;
     return L.total;
 }
 
 csa2_status csa2_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    CSA2_RANGE("csa2_workspace_init");
     if (!ws || !aligned16(ws) || ws_bytes < 16) return CSA2_ERR_INVALID_ARG;
     return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
 }
@@ -281,6 +283,7 @@ csa2_status csa2_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 csa2_status csa2_kv_append_quant(const csa2_cache* cache, const void* x_bf16, const void* idx_new,
                                  csa2_dtype idx_new_dtype, const int32_t* start_pos, int n_new, void* ws,
                                  void* stream) {
+    CSA2_RANGE("csa2_kv_append_quant");
     csa2_status s = check_cache(cache);
     if (s != CSA2_OK) return s;
     if (!x_bf16 || !start_pos || !aligned16(x_bf16) || !aligned4(start_pos) || n_new < 0) return CSA2_ERR_INVALID_ARG;
@@ -295,6 +298,7 @@ csa2_status csa2_kv_append_quant(const csa2_cache* cache, const void* x_bf16, co
 
 csa2_status csa2_kv_export_rows(const csa2_cache* cache, const int32_t* start_pos, int n, void* rows, void* keys,
                                 void* ws, void* stream) {
+    CSA2_RANGE("csa2_kv_export_rows");
     csa2_status s = check_cache(cache);
     if (s != CSA2_OK) return s;
     if (!start_pos || !aligned4(start_pos) || n < 0 || !rows || !aligned4(rows) || (keys && !aligned4(keys)) ||
@@ -307,6 +311,7 @@ csa2_status csa2_kv_export_rows(const csa2_cache* cache, const int32_t* start_po
 
 csa2_status csa2_kv_import_rows(const csa2_cache* cache, const int32_t* start_pos, int n, const void* rows,
                                 const void* keys, void* ws, void* stream) {
+    CSA2_RANGE("csa2_kv_import_rows");
     csa2_status s = check_cache(cache);
     if (s != CSA2_OK) return s;
     if (!start_pos || !aligned4(start_pos) || n < 0 || !rows || !aligned4(rows) || (keys && !aligned4(keys)) ||
@@ -320,6 +325,7 @@ csa2_status csa2_kv_import_rows(const csa2_cache* cache, const int32_t* start_po
 
 csa2_status csa2_index_scores(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
                               int T, int H_I, float* scores, void* ws, size_t ws_bytes, void* stream) {
+    CSA2_RANGE("csa2_index_scores");
     csa2_status s = check_index_args(cache, q_idx, q_dtype, head_w, T, H_I, 1, 1);
     if (s != CSA2_OK) return s;
     if (scores && !aligned16(scores)) return CSA2_ERR_INVALID_ARG;
@@ -337,6 +343,7 @@ csa2_status csa2_index_scores(const csa2_cache* cache, const void* q_idx, csa2_d
 csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
                             int T, int H_I, int pool_k, int top_k, int32_t* pool_idx, int32_t* topk_idx, void* ws,
                             size_t ws_bytes, void* stream) {
+    CSA2_RANGE("csa2_index_full");
     csa2_status s = check_index_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_k, top_k);
     if (s != CSA2_OK) return s;
     if (!pool_idx || !topk_idx || !aligned16(pool_idx) || !aligned16(topk_idx)) return CSA2_ERR_INVALID_ARG;
@@ -379,6 +386,7 @@ csa2_status csa2_index_full(const csa2_cache* cache, const void* q_idx, csa2_dty
 csa2_status csa2_index_reindex(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype, const float* head_w,
                                int T, int H_I, const int32_t* pool_idx, int pool_k, int top_k, int32_t* topk_idx,
                                void* ws, size_t ws_bytes, void* stream) {
+    CSA2_RANGE("csa2_index_reindex");
     csa2_status s = check_reindex_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx);
     if (s != CSA2_OK) return s;
     Layout L;
@@ -401,6 +409,7 @@ csa2_status csa2_index_pool_update(const csa2_cache* cache, const void* q_idx, c
                                    const float* head_w, int T, int H_I, const int32_t* pool_prev, int pool_k, int n_new,
                                    int top_k, int32_t* pool_idx, int32_t* topk_idx, void* ws, size_t ws_bytes,
                                    void* stream) {
+    CSA2_RANGE("csa2_index_pool_update");
     csa2_status s = check_reindex_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_prev, pool_k, top_k, topk_idx);
     if (s != CSA2_OK) return s;
     if (!pool_idx || !aligned16(pool_idx) || n_new < 0 || n_new > kMaxPool) return CSA2_ERR_INVALID_ARG;
@@ -440,12 +449,14 @@ csa2_status csa2_index_pool_update(const csa2_cache* cache, const void* q_idx, c
 csa2_status csa2_sparse_swa_attn(const csa2_cache* cache, const void* q_bf16, int T, int H, const int32_t* topk_idx,
                                  int top_k, int window, float sm_scale, float* out, float* lse, void* ws,
                                  size_t ws_bytes, void* stream) {
+    CSA2_RANGE("csa2_sparse_swa_attn");
     return attention(cache, Ring{}, q_bf16, T, H, topk_idx, top_k, window, sm_scale, out, lse, ws, ws_bytes, stream);
 }
 
 csa2_status csa2_sparse_swa_attn_local(const csa2_cache* cache, const void* ring, int64_t ring_len, const void* q_bf16,
                                        int T, int H, const int32_t* topk_idx, int top_k, int window, float sm_scale,
                                        float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    CSA2_RANGE("csa2_sparse_swa_attn_local");
     if (!ring_ok(ring, ring_len, T, window)) return CSA2_ERR_INVALID_ARG;
     Ring r;
     r.rows = static_cast<__nv_bfloat16*>(const_cast<void*>(ring));
@@ -455,6 +466,7 @@ csa2_status csa2_sparse_swa_attn_local(const csa2_cache* cache, const void* ring
 
 csa2_status csa2_ring_append(const csa2_cache* cache, void* ring, int64_t ring_len, const void* x_bf16,
                              const int32_t* start_pos, int n_new, void* stream) {
+    CSA2_RANGE("csa2_ring_append");
     csa2_status s = check_cache(cache);
     if (s != CSA2_OK) return s;
     if (!ring_ok(ring, ring_len, 1, 0) || !x_bf16 || !aligned16(x_bf16) || !start_pos || !aligned4(start_pos) ||
@@ -470,6 +482,7 @@ csa2_status csa2_ring_append(const csa2_cache* cache, void* ring, int64_t ring_l
 
 csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* a, void* ws, size_t ws_bytes,
                             void* stream) {
+    CSA2_RANGE("csa2_layer_step");
     if (!a) return CSA2_ERR_INVALID_ARG;
     csa2_status s = CSA2_OK;
     if (a->mode == CSA2_FULL) {
@@ -491,6 +504,7 @@ csa2_status csa2_layer_step(const csa2_cache* cache, const csa2_layer_args* a, v
 
 size_t csa2_prefill_workspace_bytes(const csa2_cache* cache, int T, int H, int H_I, int pool_k, int top_k,
                                     int window) {
+    CSA2_RANGE("csa2_prefill_workspace_bytes");
     if (check_cache(cache) != CSA2_OK || T < 1 || H_I < 1 || H_I > 64) return 0;
     const csa2_cache v = seq_view(cache, 0, cache->seq_lens);
     Layout L;
@@ -500,6 +514,7 @@ size_t csa2_prefill_workspace_bytes(const csa2_cache* cache, int T, int H, int H
 
 csa2_status csa2_prefill_layer(const csa2_cache* cache, const csa2_layer_args* a, void* ws, size_t ws_bytes,
                                void* stream) {
+    CSA2_RANGE("csa2_prefill_layer");
     csa2_status s = check_cache(cache);
     if (s != CSA2_OK) return s;
     if (!a || a->T < 1 || !ws || !aligned16(ws)) return CSA2_ERR_INVALID_ARG;
@@ -563,6 +578,7 @@ static_assert(sizeof(csa2_cand) == sizeof(CpCand), "csa2_cand and CpCand must ha
 csa2_status csa2_cp_index_local(const csa2_cache* shard, const int32_t* pos0, const void* q_idx, csa2_dtype q_dtype,
                                 const float* head_w, int H_I, int pool_k, csa2_cand* cand, void* ws, size_t ws_bytes,
                                 void* stream) {
+    CSA2_RANGE("csa2_cp_index_local");
     csa2_status s = check_index_args(shard, q_idx, q_dtype, head_w, 1, H_I, pool_k, 1);
     if (s != CSA2_OK) return s;
     if (!pos0 || !aligned4(pos0) || !cand || (reinterpret_cast<uintptr_t>(cand) & 7u)) return CSA2_ERR_INVALID_ARG;
@@ -599,6 +615,7 @@ csa2_status csa2_cp_index_local(const csa2_cache* shard, const int32_t* pos0, co
 csa2_status csa2_cp_reindex_local(const csa2_cache* shard, const int32_t* pos0, const void* q_idx,
                                   csa2_dtype q_dtype, const float* head_w, int H_I, const int32_t* pool_idx,
                                   int pool_k, int top_k, csa2_cand* cand, void* ws, size_t ws_bytes, void* stream) {
+    CSA2_RANGE("csa2_cp_reindex_local");
     csa2_status s = check_index_args(shard, q_idx, q_dtype, head_w, 1, H_I, pool_k, top_k);
     if (s != CSA2_OK) return s;
     if (!pos0 || !aligned4(pos0) || !pool_idx || !aligned16(pool_idx) || !cand ||
@@ -666,6 +683,7 @@ bool make_merge_layout(int R, int batch, int n_cand, MergeLayout* L) {
 }  // namespace
 
 size_t csa2_cp_merge_workspace_bytes(int R, int batch, int n_cand) {
+    CSA2_RANGE("csa2_cp_merge_workspace_bytes");
     MergeLayout L;
     return make_merge_layout(R, batch, n_cand, &L) ? L.total : 0;
 }
@@ -673,6 +691,7 @@ size_t csa2_cp_merge_workspace_bytes(int R, int batch, int n_cand) {
 csa2_status csa2_cp_merge_select(const csa2_cand* cand, int R, int batch, int n_cand, const int32_t* seq_lens_global,
                                  int n_a, int32_t* out_a, int n_b, int32_t* out_b, void* ws, size_t ws_bytes,
                                  void* stream) {
+    CSA2_RANGE("csa2_cp_merge_select");
     MergeLayout L;
     if (!make_merge_layout(R, batch, n_cand, &L)) return CSA2_ERR_INVALID_ARG;
     if (!cand || (reinterpret_cast<uintptr_t>(cand) & 7u) || !seq_lens_global || !aligned4(seq_lens_global))
@@ -715,6 +734,7 @@ csa2_status csa2_cp_merge_select(const csa2_cand* cand, int R, int batch, int n_
 csa2_status csa2_cp_sparse_swa_attn(const csa2_cache* shard, const int32_t* pos0, const int32_t* seq_lens_global,
                                     const void* q_bf16, int H, const int32_t* topk_idx, int top_k, int window,
                                     float sm_scale, float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    CSA2_RANGE("csa2_cp_sparse_swa_attn");
     csa2_status s = check_cache(shard);
     if (s != CSA2_OK) return s;
     if (!pos0 || !aligned4(pos0) || !seq_lens_global || !aligned4(seq_lens_global)) return CSA2_ERR_INVALID_ARG;
@@ -747,6 +767,7 @@ csa2_status csa2_cp_sparse_swa_attn(const csa2_cache* shard, const int32_t* pos0
 
 csa2_status csa2_lse_merge(int R, int batch, int H, int dim, const float* outs, int64_t out_stride,
                            const float* lses, int64_t lse_stride, float* out, float* lse, void* stream) {
+    CSA2_RANGE("csa2_lse_merge");
     if (R < 1 || batch < 1 || H < 1 || dim < 1 || !outs || !lses || !out) return CSA2_ERR_INVALID_ARG;
     if (!aligned4(outs) || !aligned4(lses) || !aligned4(out) || (lse && !aligned4(lse))) return CSA2_ERR_INVALID_ARG;
     if (R > 1 && (out_stride < (int64_t)batch * H * dim || lse_stride < (int64_t)batch * H))
@@ -756,6 +777,7 @@ csa2_status csa2_lse_merge(int R, int batch, int H, int dim, const float* outs, 
 }
 
 csa2_status csa2_read_device_status(void* ws, void* stream) {
+    CSA2_RANGE("csa2_read_device_status");
     if (!ws || !aligned16(ws)) return CSA2_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint32_t word = 0;
@@ -769,6 +791,7 @@ csa2_status csa2_read_device_status(void* ws, void* stream) {
 }
 
 csa2_status csa2_debug_set_wait_limit(uint32_t tries) {
+    CSA2_RANGE("csa2_debug_set_wait_limit");
     g_wait_limit.store(tries, std::memory_order_relaxed);
     return CSA2_OK;
 }
@@ -776,6 +799,7 @@ csa2_status csa2_debug_set_wait_limit(uint32_t tries) {
 uint32_t csa2_debug_default_wait_limit(void) { return tc::kWaitLimit; }
 
 csa2_status csa2_debug_encode(int format, const float* x, int64_t n, uint8_t* codes, void* stream) {
+    CSA2_RANGE("csa2_debug_encode");
     if ((format != 0 && format != 1) || n < 0 || (n > 0 && (!x || !codes || !aligned4(x))))
         return CSA2_ERR_INVALID_ARG;
     if (n == 0) return CSA2_OK;
@@ -783,6 +807,7 @@ csa2_status csa2_debug_encode(int format, const float* x, int64_t n, uint8_t* co
 }
 
 const char* csa2_status_string(csa2_status s) {
+    CSA2_RANGE("csa2_status_string");
     switch (s) {
         case CSA2_OK: return "CSA2_OK";
         case CSA2_ERR_INVALID_ARG: return "CSA2_ERR_INVALID_ARG";

@@ -27,16 +27,30 @@ __device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
     if (status) atomicOr(status, bit);
 }
 
+// The debug build (-DCSA2_DEBUG_BOUNDS) checks every position and page where
+// it becomes a cache slot (slot_of, the one place all kernels translate
+// positions): t outside [0, cap) and a contiguous slot beyond the cache give
+// -1, which every caller flags in the status word and skips.  Indices taken
+// from caller buffers (top-k, pool and candidate entries, page ids) are
+// checked in every build.
+#ifdef CSA2_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+
 // Slot of position t of sequence b, or -1 when the page table points outside
-// the cache.  The caller guarantees 0 <= t < cap.
+// the cache.  The caller guarantees 0 <= t < cap (checked in the debug build).
 __device__ __forceinline__ int64_t slot_of(const DevCache& c, int b, int64_t t) {
+    if (kDebugBounds && (t < 0 || t >= c.cap || b < 0 || b >= c.batch)) return -1;
     if (c.page_table) {
         int64_t pg = t / c.page_size;
         int32_t phys = __ldg(c.page_table + (int64_t)b * c.max_pages + pg);
         int64_t s = (int64_t)phys * c.page_size + (t - pg * c.page_size);
         return (phys < 0 || s >= c.n_slots) ? -1 : s;
     }
-    return (int64_t)b * c.seq_stride + t;
+    const int64_t s = (int64_t)b * c.seq_stride + t;
+    return (kDebugBounds && s >= c.n_slots) ? -1 : s;
 }
 
 // Valid length of sequence b clamped to the capacity (flags a longer one).

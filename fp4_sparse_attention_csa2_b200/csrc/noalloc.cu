@@ -94,6 +94,7 @@ using namespace csa2;
 extern "C" csa2_status csa2_index_reindex_noalloc(const csa2_cache* cache, const void* q_idx, csa2_dtype q_dtype,
                                                   const float* head_w, int T, int H_I, const int32_t* pool_idx,
                                                   int pool_k, int top_k, int32_t* topk_idx, void* stream) {
+    CSA2_RANGE("csa2_index_reindex_noalloc");
     // the same checks, in the same order and with the same statuses, as
     // csa2_index_reindex; only then the bound of the fixed scratch
     csa2_status s = check_reindex_args(cache, q_idx, q_dtype, head_w, T, H_I, pool_idx, pool_k, top_k, topk_idx);

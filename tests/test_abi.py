@@ -34,6 +34,14 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(handle, n), n
 
 
+def test_debug_build_exports_every_symbol():
+    # the debug variant (NVTX ranges, device-side bounds checks) has the same ABI
+    path = _build.build(debug=True)
+    handle = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(handle, n), n
+
+
 def test_status_strings(lib):
     for code, name in enumerate(["CSA2_OK", "CSA2_ERR_INVALID_ARG", "CSA2_ERR_UNSUPPORTED", "CSA2_ERR_CUDA",
                                  "CSA2_ERR_TIMEOUT", "CSA2_ERR_DEVICE_BOUNDS"]):
