@@ -660,7 +660,8 @@ def cp_decode_line(w, lens, layers, reps, stream, R=8):
     cp.check("after timing")
     key = 64 if w.idx_key_dtype == wl.E4M3 else 256
     n_f, n_r = w.pattern.count("F"), w.pattern.count("R")
-    gathered = R * (n_f * w.pool_k * 8 + n_r * w.top_k * 8 + len(w.pattern) * w.H * (w.D + 1) * 4)
+    gathered = R * (n_f * w.pool_k * 8 + len(w.pattern) * w.H * (w.D + 1) * 4)    # all-gathers
+    reduced = n_r * w.pool_k * 4                                                   # the Reindex all-reduce
     line = {"ranks": R, "shard_positions": cp.n, "us_per_step_rank": round(ms * 1e3, 2),
             "us_full_index_share": round(f_ms * 1e3, 2),
             "us_reindex_share": None if r_ms is None else round(r_ms * 1e3, 2),
@@ -668,10 +669,12 @@ def cp_decode_line(w, lens, layers, reps, stream, R=8):
             "layer_steps_per_s_compute": round(len(w.pattern) / (ms / 1e3), 1),
             "shard_key_bytes_per_step": cp.n * key * n_f,
             "allgather_bytes_per_step_rank": gathered,
-            "allgathers_per_step": 2 * n_f + 2 * n_r + len(w.pattern) - n_f - n_r,
-            "path": "per rank: csa2_cp_index_local / csa2_cp_reindex_local on its shard, csa2_cp_merge_select over "
-                    "all ranks' candidates, csa2_cp_sparse_swa_attn on its shard, csa2_lse_merge of all parts; "
-                    "the NCCL all-gathers between these are not timed (one GPU)"}
+            "allreduce_bytes_per_step": reduced,
+            "collectives_per_step": n_f + n_r + len(w.pattern),
+            "path": "per rank: csa2_cp_index_local on its shard + csa2_cp_merge_select over all ranks' candidates "
+                    "(Full), csa2_cp_reindex_local + csa2_cp_reindex_select on the summed pool scores (Reindex), "
+                    "csa2_cp_sparse_swa_attn on its shard + csa2_lse_merge of all parts (every layer); the NCCL "
+                    "collectives between these are not timed (one GPU)"}
     del cp
     torch.cuda.empty_cache()
     return line

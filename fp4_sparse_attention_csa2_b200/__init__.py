@@ -26,7 +26,8 @@ ABI_FUNCTIONS = (
     "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update", "csa2_sparse_swa_attn",
     "csa2_ring_append",
     "csa2_sparse_swa_attn_local", "csa2_layer_step", "csa2_prefill_workspace_bytes", "csa2_prefill_layer",
-    "csa2_cp_index_local", "csa2_cp_reindex_local", "csa2_cp_merge_workspace_bytes", "csa2_cp_merge_select",
+    "csa2_cp_index_local", "csa2_cp_reindex_local", "csa2_cp_reindex_select", "csa2_cp_merge_workspace_bytes",
+    "csa2_cp_merge_select",
     "csa2_cp_sparse_swa_attn", "csa2_lse_merge",
     "csa2_read_device_status", "csa2_status_string", "csa2_debug_set_wait_limit", "csa2_debug_default_wait_limit",
     "csa2_debug_encode",
@@ -92,7 +93,8 @@ def lib():
         L.csa2_prefill_workspace_bytes.argtypes = [cp, i32, i32, i32, i32, i32, i32]
         L.csa2_prefill_layer.argtypes = [cp, ctypes.POINTER(csa2_layer_args), vp, sz, vp]
         L.csa2_cp_index_local.argtypes = [cp, vp, vp, i32, vp, i32, i32, vp, vp, sz, vp]
-        L.csa2_cp_reindex_local.argtypes = [cp, vp, vp, i32, vp, i32, vp, i32, i32, vp, vp, sz, vp]
+        L.csa2_cp_reindex_local.argtypes = [cp, vp, vp, i32, vp, i32, vp, i32, vp, vp, sz, vp]
+        L.csa2_cp_reindex_select.argtypes = [vp, vp, i32, i32, vp, i32, vp, vp]
         L.csa2_cp_merge_workspace_bytes.restype = sz
         L.csa2_cp_merge_workspace_bytes.argtypes = [i32, i32, i32]
         L.csa2_cp_merge_select.argtypes = [vp, i32, i32, i32, vp, i32, vp, i32, vp, vp, sz, vp]
@@ -110,7 +112,7 @@ def lib():
                      "csa2_index_reindex", "csa2_index_reindex_noalloc", "csa2_index_pool_update",
                      "csa2_sparse_swa_attn", "csa2_ring_append", "csa2_sparse_swa_attn_local",
                      "csa2_layer_step", "csa2_prefill_layer", "csa2_read_device_status",
-                     "csa2_debug_set_wait_limit", "csa2_cp_index_local", "csa2_cp_reindex_local",
+                     "csa2_debug_set_wait_limit", "csa2_cp_index_local", "csa2_cp_reindex_local", "csa2_cp_reindex_select",
                      "csa2_cp_merge_select", "csa2_cp_sparse_swa_attn", "csa2_lse_merge",
                      "csa2_debug_encode"):
             getattr(L, name).restype = i32
@@ -392,15 +394,24 @@ def cp_index_local(shard, pos0, q_idx, head_w, pool_k, cand, ws, stream=None):
                                      _p(ws), ws.numel() * ws.element_size(), _stream(stream)), "cp_index_local")
 
 
-def cp_reindex_local(shard, pos0, q_idx, head_w, pool_idx, top_k, cand, ws, stream=None):
-    """A Reindex layer's share on a shard: the global pool entries it holds
-    rescored, the top_k best into cand [B, top_k, 2]."""
+def cp_reindex_local(shard, pos0, q_idx, head_w, pool_idx, pool_scores, ws, stream=None):
+    """A Reindex layer's share on a shard: pool_scores fp32 [B, pool_k] <- the
+    scores of the global pool entries it holds, 0 for the others (summed over
+    the ranks, every entry carries its owner's score)."""
     B, T, H_I, _ = q_idx.shape
     if T != 1:
         raise ValueError("context-parallel calls take one query token per sequence")
     _check(lib().csa2_cp_reindex_local(shard.ref, _p(pos0), _p(q_idx), _qdt(q_idx), _p(head_w), H_I, _p(pool_idx),
-                                       pool_idx.shape[-1], top_k, _p(cand), _p(ws), ws.numel() * ws.element_size(),
+                                       pool_idx.shape[-1], _p(pool_scores), _p(ws), ws.numel() * ws.element_size(),
                                        _stream(stream)), "cp_reindex_local")
+
+
+def cp_reindex_select(pool_idx, pool_scores, seq_lens_global, top_k, topk_idx, stream=None):
+    """The top_k best entries of pool_idx [B, pool_k] by the summed
+    pool_scores into topk_idx [B, top_k]."""
+    B, pool_k = pool_idx.shape[0], pool_idx.shape[-1]
+    _check(lib().csa2_cp_reindex_select(_p(pool_idx), _p(pool_scores), B, pool_k, _p(seq_lens_global), top_k,
+                                        _p(topk_idx), _stream(stream)), "cp_reindex_select")
 
 
 def cp_merge_workspace_bytes(R, batch, n_cand):

@@ -11,13 +11,14 @@ calls; the exchanges between them are all-gathers over the process group
 
     Full     cp_index_local -> all-gather (pool_k candidates a rank) ->
              cp_merge_select (pool and top-k, the same on every rank)
-    Reindex  cp_reindex_local -> all-gather (top_k candidates a rank) ->
-             cp_merge_select (top-k)
+    Reindex  cp_reindex_local -> all-reduce (sum) of the pool's scores (each
+             entry is scored by its one owner, the other ranks add zeros) ->
+             cp_reindex_select (top-k)
     every    cp_sparse_swa_attn -> all-gather of (out, lse) -> lse_merge
 
-Per layer that is pool_k * 8 B (Full) or top_k * 8 B (Reindex) of candidates
-and H * (dim + 1) * 4 B of attention part per rank and sequence; every rank
-then holds the whole layer's output.  The library's calls are the only
+Per layer and sequence that is pool_k * 8 B of candidates a rank (Full),
+pool_k * 4 B of scores (Reindex) and H * (dim + 1) * 4 B of attention part a
+rank; every rank then holds the whole layer's output.  The library's calls are the only
 compute; this module only sequences them and the collectives.
 """
 import torch
@@ -53,9 +54,8 @@ class ContextParallelStack:
         o.workspace_init(self.mws)
         B, R = self.B, self.R
         self.cand_pool = torch.empty((B, pool_k, 2), dtype=torch.int32, device=device)
-        self.cand_topk = torch.empty((B, top_k, 2), dtype=torch.int32, device=device)
+        self.pool_scores = torch.empty((B, pool_k), dtype=torch.float32, device=device)
         self.gath_pool = torch.empty((R, B, pool_k, 2), dtype=torch.int32, device=device)
-        self.gath_topk = torch.empty((R, B, top_k, 2), dtype=torch.int32, device=device)
         # a rank's attention part as one buffer: out [B][H][D] then lse [B][H]
         self.n_out = B * H * self.D
         self.part = torch.empty(self.n_out + B * H, dtype=torch.float32, device=device)
@@ -78,9 +78,9 @@ class ContextParallelStack:
             o.cp_merge_select(self.gath_pool, self.lens_global, self.pool_k, pool, self.mws, n_b=self.top_k,
                               out_b=topk)
         elif mode == csa2.REINDEX:
-            o.cp_reindex_local(self.shard, self.pos0, q_idx, head_w, pool, self.top_k, self.cand_topk, self.ws)
-            self._gather(self.gath_topk, self.cand_topk)
-            o.cp_merge_select(self.gath_topk, self.lens_global, self.top_k, topk, self.mws)
+            o.cp_reindex_local(self.shard, self.pos0, q_idx, head_w, pool, self.pool_scores, self.ws)
+            dist.all_reduce(self.pool_scores, op=dist.ReduceOp.SUM, group=self.group)
+            o.cp_reindex_select(pool, self.pool_scores, self.lens_global, self.top_k, topk)
         elif mode != csa2.REUSE:
             raise ValueError("mode must be FULL, REINDEX or REUSE")
         part_out = self.part[:self.n_out].view(B, self.H, self.D)

@@ -614,43 +614,49 @@ csa2_status csa2_cp_index_local(const csa2_cache* shard, const int32_t* pos0, co
 
 csa2_status csa2_cp_reindex_local(const csa2_cache* shard, const int32_t* pos0, const void* q_idx,
                                   csa2_dtype q_dtype, const float* head_w, int H_I, const int32_t* pool_idx,
-                                  int pool_k, int top_k, csa2_cand* cand, void* ws, size_t ws_bytes, void* stream) {
+                                  int pool_k, float* pool_scores, void* ws, size_t ws_bytes, void* stream) {
     CSA2_RANGE("csa2_cp_reindex_local");
-    csa2_status s = check_index_args(shard, q_idx, q_dtype, head_w, 1, H_I, pool_k, top_k);
+    csa2_status s = check_index_args(shard, q_idx, q_dtype, head_w, 1, H_I, pool_k, 1);
     if (s != CSA2_OK) return s;
-    if (!pos0 || !aligned4(pos0) || !pool_idx || !aligned16(pool_idx) || !cand ||
-        (reinterpret_cast<uintptr_t>(cand) & 7u))
+    if (!pos0 || !aligned4(pos0) || !pool_idx || !aligned16(pool_idx) || !pool_scores || !aligned16(pool_scores))
         return CSA2_ERR_INVALID_ARG;
     Layout L;
-    s = check_ws(shard, 1, 1, pool_k, top_k, 0, ws, ws_bytes, &L);
+    s = check_ws(shard, 1, 1, pool_k, 1, 0, ws, ws_bytes, &L);
     if (s != CSA2_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     DevCache d = dev_cache(shard);
     uint32_t* status = at<uint32_t>(ws, L.status);
     int32_t* local = at<int32_t>(ws, L.upd_ids);           // [batch][pool_k] shard positions or -1
     float* sc = at<float>(ws, L.pscores);                   // [batch][pool_k]
-    int32_t* ids = at<int32_t>(ws, L.upd_scores);           // [batch][top_k]
-    float* vals = at<float>(ws, L.upd_scores + align_up(sizeof(int32_t) * (size_t)L.nseg * top_k));
     cudaError_t e = launch_cp_localize(pool_idx, pos0, shard->seq_lens, shard->batch, pool_k, local, st);
     if (e == cudaSuccess)
         e = reindex_tc_supported(d, H_I) ? launch_reindex_tc_scores(d, q_idx, head_w, 1, H_I, local, pool_k, sc, status, st)
                                          : launch_score_pool(d, q_idx, q_dtype == CSA2_F32, head_w, 1, H_I, local, pool_k,
                                                              sc, status, st);
-    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    if (e == cudaSuccess) e = launch_cp_owned_scores(local, sc, (int64_t)shard->batch * pool_k, pool_scores, st);
+    return cuda_status(e);
+}
+
+csa2_status csa2_cp_reindex_select(const int32_t* pool_idx, const float* pool_scores, int batch, int pool_k,
+                                   const int32_t* seq_lens_global, int top_k, int32_t* topk_idx, void* stream) {
+    CSA2_RANGE("csa2_cp_reindex_select");
+    if (batch < 1 || batch > 65535 || pool_k < 1 || pool_k > kMaxPool || top_k < 1 || top_k > pool_k)
+        return CSA2_ERR_INVALID_ARG;
+    if (!pool_idx || !aligned16(pool_idx) || !pool_scores || !aligned16(pool_scores) || !topk_idx ||
+        !aligned16(topk_idx) || !seq_lens_global || !aligned4(seq_lens_global))
+        return CSA2_ERR_INVALID_ARG;
     SelSrc src;
-    src.vals = sc;
+    src.vals = pool_scores;
     src.vals_stride = pool_k;
-    src.ids = local;
+    src.ids = pool_idx;
     src.ids_stride = pool_k;
     src.gather = 0;
     src.n = pool_k;
-    src.seq_lens = shard->seq_lens;
+    src.seq_lens = seq_lens_global;      // an entry is valid when 0 <= pos < Lg (T = 1) and its score is a number
     src.T = 1;
-    src.cap = L.cap;
-    e = launch_select_local(src, (int)L.nseg, top_k, ids, vals, top_k, 0, nullptr, 0, st);
-    if (e != cudaSuccess) return CSA2_ERR_CUDA;
-    return cuda_status(launch_cp_pack(ids, vals, top_k, pos0, shard->batch, top_k, reinterpret_cast<CpCand*>(cand),
-                                      st));
+    src.cap = (int64_t)1 << 31;
+    return cuda_status(launch_select_local(src, batch, top_k, topk_idx, nullptr, top_k, 0, nullptr, 0,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 namespace {
@@ -749,20 +755,34 @@ csa2_status csa2_cp_sparse_swa_attn(const csa2_cache* shard, const int32_t* pos0
     if (sm_scale <= 0.0f) sm_scale = 1.0f / std::sqrt((float)shard->dim);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint32_t* status = at<uint32_t>(ws, L.status);
-    // the shard's part of window ∪ top-k as one list of shard positions; the
-    // attention then runs with no window of its own (the list's window part and
-    // top-k part are disjoint)
+    AttnWork aw;
+    aw.part_o = at<float>(ws, L.part_o);
+    aw.part_ml = at<float>(ws, L.part_ml);
+    aw.nchunk = L.nchunk;
+    DevCache d = dev_cache(shard);
+    if (attn_tc_supported(d, H)) {
+        // the tensor-core kernel maps the global window and top-k entries to the
+        // shard's positions itself
+        CpShard cp;
+        cp.pos0 = pos0;
+        cp.glens = seq_lens_global;
+        aw.nchunk = (window + top_k + attn_tc_rows_per_chunk() - 1) / attn_tc_rows_per_chunk();
+        if (aw.nchunk < 1) aw.nchunk = 1;
+        cudaError_t e = launch_attention_tc(d, q_bf16, 1, H, top_k > 0 ? topk_idx : nullptr, top_k, window, sm_scale,
+                                            Ring{}, aw, status, st, num_sms(), cp);
+        if (e == cudaSuccess) e = launch_attn_combine(d, 1, H, aw, out, lse, st);
+        return cuda_status(e);
+    }
+    // otherwise the shard's part of window ∪ top-k as one list of shard
+    // positions, attended with no window of its own (the list's window part
+    // and top-k part are disjoint)
     const int n = window + top_k;
     int32_t* list = at<int32_t>(ws, L.upd_ids);
     if (n > 0 && launch_cp_attn_list(topk_idx, top_k, window, pos0, shard->seq_lens, seq_lens_global, shard->batch,
                                      list, status, st) != cudaSuccess)
         return CSA2_ERR_CUDA;
-    AttnWork aw;
-    aw.part_o = at<float>(ws, L.part_o);
-    aw.part_ml = at<float>(ws, L.part_ml);
-    aw.nchunk = L.nchunk;
-    return cuda_status(launch_attention(dev_cache(shard), q_bf16, 1, H, n > 0 ? list : nullptr, n, 0, sm_scale, Ring{},
-                                        out, lse, aw, status, st, num_sms()));
+    return cuda_status(launch_attention(d, q_bf16, 1, H, n > 0 ? list : nullptr, n, 0, sm_scale, Ring{}, out, lse, aw,
+                                        status, st, num_sms()));
 }
 
 csa2_status csa2_lse_merge(int R, int batch, int H, int dim, const float* outs, int64_t out_stride,

@@ -65,6 +65,11 @@ struct Params {
     uint32_t off_q, off_p, off_misc, tmem_cols;
     const __nv_bfloat16* ring;   // [batch][ring_len][D] or nullptr (window rows from the FP4 cache)
     int64_t ring_len;
+    // a context-parallel shard (T = 1): the cache holds positions [cp_pos0[b],
+    // cp_pos0[b] + L) of a sequence of cp_glens[b] positions; window and top-k
+    // are global positions and only the shard's are attended (nullptr: off)
+    const int32_t* cp_pos0;
+    const int32_t* cp_glens;
 };
 
 template <int HG>
@@ -194,16 +199,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const Params p) {
     int32_t t_raw = -1;
     if (is_topk) t_raw = __ldg(p.topk + (int64_t)seg * p.top_k + (v_entry - p.window));
     const int64_t L = seq_len(p.c, b, p.status);
-    const int64_t pq = L - p.T + j;
+    // on a context-parallel shard the query sits at the sequence's last
+    // position and the entries are the sequence's positions; the shard's own
+    // ones are mapped to its positions below, the others masked
+    const bool cp = p.cp_pos0 != nullptr;
+    const int64_t Lg = cp ? (int64_t)__ldg(p.cp_glens + b) : L;
+    const int64_t pq = cp ? Lg - 1 : L - p.T + j;
     int32_t t = -1;
     if (pq >= 0 && v_entry < p.window + p.top_k) {
         if (!is_topk) {
             t = pq - v_entry >= 0 ? (int32_t)(pq - v_entry) : -1;
         } else {
             t = t_raw;
-            if (t < -1 || t >= L) { if (kp == 0) flag(p.status, kStatusBounds); t = -1; }
+            if (t < -1 || t >= Lg) { if (kp == 0) flag(p.status, kStatusBounds); t = -1; }
             else if (t > pq || t > pq - p.window) t = -1;   // future, or already in the window
         }
+    }
+    if (cp && t >= 0) {
+        const int64_t ts = (int64_t)t - __ldg(p.cp_pos0 + b);
+        t = ts >= 0 && ts < L ? (int32_t)ts : -1;
     }
     // a window entry of a launch with a ring takes its row from the ring (CTA-uniform: ring_chunk)
     const bool ring_chunk = RING && chunk * kRows < p.window;
@@ -557,8 +571,11 @@ int attn_tc_heads_per_cta(int H, int nchunk, int nseg, int num_sms) {
 
 cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
                                 int window, float sm_scale, const Ring& ring, const AttnWork& aw, uint32_t* status,
-                                cudaStream_t st, int num_sms) {
+                                cudaStream_t st, int num_sms, const CpShard& cp) {
+    if (cp.pos0 && (T != 1 || ring.rows)) return cudaErrorInvalidValue;
     Params p;
+    p.cp_pos0 = cp.pos0;
+    p.cp_glens = cp.glens;
     p.c = c;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.topk = topk;

@@ -49,6 +49,20 @@ k_cp_localize(const int32_t* __restrict__ pool, const int32_t* __restrict__ pos0
     local[e] = (pool[e] >= 0 && t >= 0 && t < __ldg(shard_lens + b)) ? (int32_t)t : -1;
 }
 
+// A Reindex layer's share of the pool scores: out[b][i] <- the score of pool
+// entry i when this shard holds it (NaN when the shard could not score it),
+// 0 when another shard holds it or it is padding.  Summed over the ranks (an
+// all-reduce), every entry then carries its owner's score exactly: the other
+// terms are zeros.
+__global__ void __launch_bounds__(kThreads)
+k_cp_owned_scores(const int32_t* __restrict__ local, const float* __restrict__ sc, int64_t n,
+                  float* __restrict__ out) {
+    pdl_begin();
+    const int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (e >= n) return;
+    out[e] = local[e] >= 0 ? sc[e] : 0.0f;
+}
+
 // All-gathered candidates [R][batch][n] -> per sequence [batch][R * n]: ids
 // and scores in the layout the selection kernels read.
 __global__ void __launch_bounds__(kThreads)
@@ -150,6 +164,10 @@ cudaError_t launch_cp_localize(const int32_t* pool, const int32_t* pos0, const i
                                int32_t* local, cudaStream_t st) {
     return launch_pdl(k_cp_localize, dim3(blocks_for((int64_t)batch * n)), dim3(kThreads), 0, st, pool, pos0,
                       shard_lens, batch, n, local);
+}
+
+cudaError_t launch_cp_owned_scores(const int32_t* local, const float* sc, int64_t n, float* out, cudaStream_t st) {
+    return launch_pdl(k_cp_owned_scores, dim3(blocks_for(n)), dim3(kThreads), 0, st, local, sc, n, out);
 }
 
 cudaError_t launch_cp_unpack(const CpCand* cand, int R, int batch, int n, int32_t* ids, float* vals,

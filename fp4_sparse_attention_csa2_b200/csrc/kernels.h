@@ -137,9 +137,14 @@ bool attn_tc_supported(const DevCache& c, int H);
 int attn_tc_rows_per_chunk();
 // heads per CTA: H, halved (down to 16) while the grid would leave SMs idle
 int attn_tc_heads_per_cta(int H, int nchunk, int nseg, int num_sms);
+// A context-parallel shard's place in its sequence (pos0 == nullptr: not a shard).
+struct CpShard {
+    const int32_t* pos0 = nullptr;   // [batch] the sequence position of the shard's position 0
+    const int32_t* glens = nullptr;  // [batch] the sequences' lengths
+};
 cudaError_t launch_attention_tc(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
                                 int window, float sm_scale, const Ring& ring, const AttnWork& aw, uint32_t* status,
-                                cudaStream_t st, int num_sms);
+                                cudaStream_t st, int num_sms, const CpShard& cp = CpShard{});
 cudaError_t launch_attn_combine(const DevCache& c, int T, int H, const AttnWork& aw, float* out, float* lse,
                                 cudaStream_t st);
 cudaError_t launch_attention(const DevCache& c, const void* q, int T, int H, const int32_t* topk, int top_k,
@@ -158,6 +163,8 @@ cudaError_t launch_cp_pack(const int32_t* ids, const float* vals, int64_t in_str
 // local[b][i] <- pool[b][i] - pos0[b] when in [0, shard_lens[b]), else -1.
 cudaError_t launch_cp_localize(const int32_t* pool, const int32_t* pos0, const int32_t* shard_lens, int batch, int n,
                                int32_t* local, cudaStream_t st);
+// out[e] <- sc[e] where local[e] >= 0 (this shard's pool entries), else 0.
+cudaError_t launch_cp_owned_scores(const int32_t* local, const float* sc, int64_t n, float* out, cudaStream_t st);
 // [R][batch][n] candidates -> ids / vals [batch][R * n].
 cudaError_t launch_cp_unpack(const CpCand* cand, int R, int batch, int n, int32_t* ids, float* vals,
                              cudaStream_t st);

@@ -221,8 +221,9 @@ class CpRankStep:
     shards of L / R positions, taken as shard views of the given caches.  The
     candidates and attention parts of all R ranks are computed once from the
     first cache's shards; step(shard) then runs one rank's calls of a step --
-    its shard calls, the merge selections over all ranks' candidates, the
-    log-sum-exp merges of all ranks' parts -- with no exchange in between."""
+    its shard calls, the selections over all ranks' candidates (Full) and
+    summed pool scores (Reindex), the log-sum-exp merges of all ranks' parts
+    -- with no exchange in between."""
 
     def __init__(self, w, lens, layers, caches, R=8):
         L = int(lens[0])
@@ -244,11 +245,12 @@ class CpRankStep:
         self.pool = torch.empty((B, w.pool_k), dtype=torch.int32, device=dev)
         self.topk = torch.empty((B, w.top_k), dtype=torch.int32, device=dev)
         self.gpool = torch.empty((R, B, w.pool_k, 2), dtype=torch.int32, device=dev)
-        self.gtopk = torch.empty((R, B, w.top_k, 2), dtype=torch.int32, device=dev)
+        self.rscores = torch.empty((R, B, w.pool_k), dtype=torch.float32, device=dev)
+        self.gscores = torch.empty((B, w.pool_k), dtype=torch.float32, device=dev)
         self.gout = torch.empty((len(w.pattern), R, B, H, D), dtype=torch.float32, device=dev)
         self.glse = torch.empty((len(w.pattern), R, B, H), dtype=torch.float32, device=dev)
         self.cand_pool = torch.empty((B, w.pool_k, 2), dtype=torch.int32, device=dev)
-        self.cand_topk = torch.empty((B, w.top_k, 2), dtype=torch.int32, device=dev)
+        self.pool_scores = torch.empty((B, w.pool_k), dtype=torch.float32, device=dev)
         self.part_o = torch.empty((B, H, D), dtype=torch.float32, device=dev)
         self.part_l = torch.empty((B, H), dtype=torch.float32, device=dev)
         self.out = torch.empty((B, H, D), dtype=torch.float32, device=dev)
@@ -264,9 +266,10 @@ class CpRankStep:
                                      out_b=self.topk)
             elif m == "R":
                 for r in range(R):
-                    csa2.cp_reindex_local(self.shards[r][0], self.pos0[r], q["q_idx"], q["w"], self.pool, w.top_k,
-                                          self.gtopk[r], self.ws)
-                csa2.cp_merge_select(self.gtopk, self.glens, w.top_k, self.topk, self.mws)
+                    csa2.cp_reindex_local(self.shards[r][0], self.pos0[r], q["q_idx"], q["w"], self.pool,
+                                          self.rscores[r], self.ws)
+                torch.sum(self.rscores, dim=0, out=self.gscores)      # the all-reduce
+                csa2.cp_reindex_select(self.pool, self.gscores, self.glens, w.top_k, self.topk)
             for r in range(R):
                 csa2.cp_sparse_swa_attn(self.shards[r][0], self.pos0[r], self.glens, q["q"], self.topk, w.window,
                                         self.gout[l, r], self.glse[l, r], self.ws)
@@ -286,9 +289,8 @@ class CpRankStep:
 
     def reindex_part(self, sh, l=None):
         w, q = self.w, self.dl[self.w.pattern.index("R") if l is None else l]
-        csa2.cp_reindex_local(sh[0], self.pos0[sh[1]], q["q_idx"], q["w"], self.pool, w.top_k, self.cand_topk,
-                              self.ws)
-        csa2.cp_merge_select(self.gtopk, self.glens, w.top_k, self.topk, self.mws)
+        csa2.cp_reindex_local(sh[0], self.pos0[sh[1]], q["q_idx"], q["w"], self.pool, self.pool_scores, self.ws)
+        csa2.cp_reindex_select(self.pool, self.gscores, self.glens, w.top_k, self.topk)
 
     def attn_part(self, sh, l=None):
         w = self.w

@@ -387,11 +387,12 @@ CSA2_API csa2_status csa2_prefill_layer(const csa2_cache* cache, const csa2_laye
  * One layer on every rank:
  *   FULL     csa2_cp_index_local -> all-gather of the candidates ->
  *            csa2_cp_merge_select (pool and top-k)
- *   REINDEX  csa2_cp_reindex_local -> all-gather -> csa2_cp_merge_select
+ *   REINDEX  csa2_cp_reindex_local -> all-reduce (sum) of the pool's scores ->
+ *            csa2_cp_reindex_select
  *   any      csa2_cp_sparse_swa_attn -> all-gather of (out, lse) ->
  *            csa2_lse_merge
- * The all-gathers are the caller's (NCCL over NVLink, a few hundred KB a
- * layer); every rank ends with the same pool, top-k, output and lse.  The
+ * The collectives are the caller's (NCCL over NVLink, at most a few hundred KB
+ * a layer); every rank ends with the same pool, top-k, output and lse.  The
  * shard calls share one workspace of csa2_workspace_bytes(shard, 1, H, pool_k,
  * top_k, window) bytes (cleared once with csa2_workspace_init; its status word
  * read with csa2_read_device_status); the merge selection has its own.
@@ -418,14 +419,33 @@ CSA2_API csa2_status csa2_cp_index_local(const csa2_cache* shard, const int32_t*
 /*
  * A Reindex layer's share on one shard: the entries of the global pool
  * pool_idx[b][0..pool_k) that this shard holds (pos0[b] <= t < pos0[b] +
- * n_r[b]; the others and -1 padding are skipped) are rescored as
- * csa2_index_reindex rescores them, and cand[b][0..top_k) <- the min(top_k,
- * owned) best with their scores and global positions, then (-1, 0) padding.
+ * n_r[b]) are rescored as csa2_index_reindex rescores them, and
+ *     pool_scores[b][i] <- that score for an entry this shard holds (NaN if it
+ *                          could not be scored: CSA2_ERR_DEVICE_BOUNDS),
+ *                          0 for an entry another shard holds and for -1
+ *                          padding.
+ * Every pool entry has exactly one owner, so the sum of the ranks'
+ * pool_scores (an all-reduce, exact: the other terms are zeros) holds every
+ * entry's score; csa2_cp_reindex_select then picks the top-k.  pool_scores is
+ * fp32 [batch][pool_k], 16-byte aligned.  Other arguments as
+ * csa2_cp_index_local and csa2_index_reindex.
  */
 CSA2_API csa2_status csa2_cp_reindex_local(const csa2_cache* shard, const int32_t* pos0, const void* q_idx,
                                            csa2_dtype q_dtype, const float* head_w, int H_I,
-                                           const int32_t* pool_idx, int pool_k, int top_k, csa2_cand* cand,
-                                           void* ws, size_t ws_bytes, void* stream);
+                                           const int32_t* pool_idx, int pool_k, float* pool_scores, void* ws,
+                                           size_t ws_bytes, void* stream);
+
+/*
+ * The Reindex top-k after the all-reduce: topk_idx[b][0..top_k) <- the
+ * min(top_k, valid) best entries of pool_idx[b] by pool_scores[b] (summed over
+ * the ranks), an entry being valid when 0 <= pos < seq_lens_global[b] and its
+ * score is a number; a set in unspecified order, -1 padding last, ties at the
+ * cutoff broken arbitrarily.  1 <= top_k <= pool_k <= 16384; pool_idx,
+ * pool_scores and topk_idx 16-byte aligned.  Needs no workspace.
+ */
+CSA2_API csa2_status csa2_cp_reindex_select(const int32_t* pool_idx, const float* pool_scores, int batch,
+                                            int pool_k, const int32_t* seq_lens_global, int top_k,
+                                            int32_t* topk_idx, void* stream);
 
 /*
  * The selection after the all-gather: cand is [R][batch][n_cand] (rank r's

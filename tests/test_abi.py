@@ -245,14 +245,26 @@ def test_context_parallel_arguments_rejected_on_host(lib):
     assert local(pool_k=16385) == csa2.ERR_INVALID_ARG
     assert local(H_I=65) == csa2.ERR_INVALID_ARG
 
-    def reindex(pool=0x60000, pool_k=16384, top_k=2048, cand=0x90000):
+    def reindex(pool=0x60000, pool_k=16384, scores=0x90000):
         return lib.csa2_cp_reindex_local(ctypes.byref(c), 0x30100, 0x40000, csa2.BF16, 0x50000, 32, pool, pool_k,
-                                         top_k, cand, 0x80000, big, None)
+                                         scores, 0x80000, big, None)
 
     assert reindex(pool=None) == csa2.ERR_INVALID_ARG
     assert reindex(pool=0x60004) == csa2.ERR_INVALID_ARG
-    assert reindex(top_k=16385) == csa2.ERR_INVALID_ARG
-    assert reindex(cand=0x90004) == csa2.ERR_INVALID_ARG
+    assert reindex(pool_k=16385) == csa2.ERR_INVALID_ARG
+    assert reindex(scores=None) == csa2.ERR_INVALID_ARG
+    assert reindex(scores=0x90004) == csa2.ERR_INVALID_ARG
+
+    def rselect(pool_k=16384, top_k=2048, topk=0xA0000, lens=0x30000, batch=1):
+        return lib.csa2_cp_reindex_select(0x60000, 0x90000, batch, pool_k, lens, top_k, topk, None)
+
+    assert rselect(top_k=0) == csa2.ERR_INVALID_ARG
+    assert rselect(top_k=16385, pool_k=16385) == csa2.ERR_INVALID_ARG
+    assert rselect(top_k=4096, pool_k=2048) == csa2.ERR_INVALID_ARG
+    assert rselect(topk=None) == csa2.ERR_INVALID_ARG
+    assert rselect(topk=0xA0004) == csa2.ERR_INVALID_ARG
+    assert rselect(lens=None) == csa2.ERR_INVALID_ARG
+    assert rselect(batch=0) == csa2.ERR_INVALID_ARG
 
     # the merge workspace: histograms, four candidate buffers and the per-sequence candidates
     n = lib.csa2_cp_merge_workspace_bytes(8, 1, 16384)

@@ -92,18 +92,24 @@ class OracleOps:
             pool = pool[pool >= 0]
             self._put(cand, b, pool + int(pos0[b]), s[pool])
 
-    def cp_reindex_local(self, shard, pos0, q_idx, head_w, pool, top_k, cand, ws):
+    def cp_reindex_local(self, shard, pos0, q_idx, head_w, pool, pool_scores, ws):
         import oracle
         from fp4_sparse_attention_csa2_b200 import workloads as wl
         for b in range(shard.batch):
             p0, nb = shard.bounds[b]
             g = pool[b].numpy()
             local = np.where((g >= p0) & (g < p0 + nb), g - p0, -1).astype(np.int32)
-            tk, s = oracle.index_reindex(shard.ref, b, 1, 0, wl.host_array(q_idx)[b, 0], self.w.q_idx_dtype,
-                                         head_w[b, 0].numpy(), local, top_k, want_scores=True)
-            by_pos = {int(t): float(v) for t, v in zip(local, s) if t >= 0}
-            tk = tk[tk >= 0]
-            self._put(cand, b, tk + p0, [by_pos[int(t)] for t in tk])
+            _, s = oracle.index_reindex(shard.ref, b, 1, 0, wl.host_array(q_idx)[b, 0], self.w.q_idx_dtype,
+                                        head_w[b, 0].numpy(), local, 1, want_scores=True)
+            pool_scores[b] = torch.from_numpy(np.where(local >= 0, s, 0.0).astype(np.float32))
+
+    def cp_reindex_select(self, pool, pool_scores, lens_global, top_k, topk):
+        import oracle
+        for b in range(pool.shape[0]):
+            pos = pool[b].numpy()
+            sc = pool_scores[b].numpy().astype(np.float64)
+            ok = (pos >= 0) & (pos < int(lens_global[b])) & ~np.isnan(sc)
+            topk[b] = torch.from_numpy(oracle.select_top(sc[ok], pos[ok], top_k))
 
     def cp_merge_select(self, cand, lens_global, n_a, out_a, ws, n_b=0, out_b=None):
         import oracle

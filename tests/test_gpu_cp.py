@@ -1,7 +1,9 @@
 """Context-parallel decode on the GPU: the shard calls (csa2_cp_index_local,
-csa2_cp_reindex_local, csa2_cp_sparse_swa_attn), the merge selection and the
-log-sum-exp merge, with R ranks emulated one after another on one GPU (each
-rank's shard is a cache of its own; the all-gathers become stacked buffers).
+csa2_cp_reindex_local, csa2_cp_sparse_swa_attn), the selections after the
+exchange (csa2_cp_merge_select, csa2_cp_reindex_select) and the log-sum-exp
+merge, with R ranks emulated one after another on one GPU (each rank's shard
+is a cache of its own; the all-gathers become stacked buffers, the all-reduce
+a sum).
 The merged results are checked against the oracle run on the whole sequence
 (tldrocket.com "DeepSeek AI Released DeepSeek-V4.1-Flash ...", paragraphs 1
 and 3; zerohour.day: a context of one million tokens): the Full layer's pool
@@ -44,7 +46,7 @@ def run_cp_stack(w, shards, layers, lens):
     pool = torch.full((B, w.pool_k), -7, dtype=torch.int32, device="cuda")
     topk = torch.full((B, w.top_k), -7, dtype=torch.int32, device="cuda")
     cand_pool = torch.empty((R, B, w.pool_k, 2), dtype=torch.int32, device="cuda")
-    cand_topk = torch.empty((R, B, w.top_k, 2), dtype=torch.int32, device="cuda")
+    pool_scores = torch.empty((R, B, w.pool_k), dtype=torch.float32, device="cuda")
     res = []
     for l, mode in enumerate(w.pattern):
         L = device_layer(layers[l])
@@ -54,8 +56,10 @@ def run_cp_stack(w, shards, layers, lens):
             csa2.cp_merge_select(cand_pool, glens, w.pool_k, pool, mws, n_b=w.top_k, out_b=topk)
         elif mode == "R":
             for r, (cache, pos0) in enumerate(shards):
-                csa2.cp_reindex_local(cache, pos0, L["q_idx"], L["w"], pool, w.top_k, cand_topk[r], wss[r])
-            csa2.cp_merge_select(cand_topk, glens, w.top_k, topk, mws)
+                csa2.cp_reindex_local(cache, pos0, L["q_idx"], L["w"], pool, pool_scores[r], wss[r])
+            # the all-reduce: each entry's owner adds its score, every other rank a zero
+            summed = pool_scores.sum(dim=0).contiguous()
+            csa2.cp_reindex_select(pool, summed, glens, w.top_k, topk)
         outs = torch.empty((R, B, w.H, w.D), dtype=torch.float32, device="cuda")
         lses = torch.empty((R, B, w.H), dtype=torch.float32, device="cuda")
         for r, (cache, pos0) in enumerate(shards):
@@ -104,10 +108,13 @@ def test_cp_full_size_ctx1m_eight_ranks():
     print("ctx1m over 8 ranks: %d index differences inside the cutoff band" % n_band)
 
 
-def test_cp_parts_are_attention_over_each_shards_share():
+@pytest.mark.parametrize("H", [64, 48])
+def test_cp_parts_are_attention_over_each_shards_share(H):
     # each rank's (out, lse) is the attention over S ∩ shard: the oracle's
-    # attention over that explicit set (no window of its own)
-    w = wl.scaled(wl.WORKLOADS["long64k"], 9000, T=1)
+    # attention over that explicit set (no window of its own); 64 heads run the
+    # tensor-core kernel with the shard mapping inside it, 48 heads the
+    # CUDA-core kernel over the shard's list
+    w = wl.scaled(wl.WORKLOADS["long64k"], 9000, T=1, H=H)
     R = 3
     lens = wl.seq_lens(w)
     l0 = wl.layer_queries(w, 0)
