@@ -1,5 +1,5 @@
 """The context-parallel driver (fp4_sparse_attention_csa2_b200.cp) on CPU
-processes: two ranks over gloo, each holding half of every sequence, run a
+processes: two or three ranks over gloo, each holding a shard of every sequence, run a
 Full, Reindex, Reuse stack through ContextParallelStack with the library's
 shard calls replaced by oracle stand-ins of the same names.  This covers the
 exchange plumbing with no GPU: the order of the all-gathers, the candidate and
@@ -13,6 +13,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -20,7 +21,6 @@ ROOT = os.path.dirname(HERE)
 
 WORKLOAD = ("long64k", 3000, dict(batch=2, pool_k=1024, top_k=128, T=1, lens=("uniform", 2000, 3000),
                                   pattern="FRUU"))
-R = 2
 
 
 def _free_port():
@@ -42,7 +42,7 @@ def _setup():
 class ShardRef:
     """A rank's shard for the stand-ins: the oracle's cache of its positions."""
 
-    def __init__(self, w, layers, lens, r):
+    def __init__(self, w, layers, lens, r, R):
         import oracle
         from fp4_sparse_attention_csa2_b200 import workloads as wl
         self.bounds = [wl.shard_bounds(int(lens[b]), R)[r] for b in range(w.batch)]
@@ -147,26 +147,26 @@ class OracleOps:
                 lse[b] = torch.from_numpy(l)
 
 
-def _worker(rank, port, q):
+def _worker(rank, R, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
     import traceback
     import torch.distributed as dist
     dist.init_process_group("gloo", rank=rank, world_size=R, timeout=datetime.timedelta(seconds=60))
     try:
-        _run(rank, q)
+        _run(rank, R, q)
     except Exception:
         q.put((rank, traceback.format_exc()))
     finally:
         dist.destroy_process_group()
 
 
-def _run(rank, q):
+def _run(rank, R, q):
     if True:
         w, layers, lens = _setup()
         import fp4_sparse_attention_csa2_b200 as csa2
         from fp4_sparse_attention_csa2_b200.cp import ContextParallelStack
-        shard = ShardRef(w, layers, lens, rank)
+        shard = ShardRef(w, layers, lens, rank, R)
         pos0 = torch.tensor([p0 for p0, _ in shard.bounds], dtype=torch.int32)
         st = ContextParallelStack(shard, pos0, torch.as_tensor(lens), w.H, w.pool_k, w.top_k, w.window,
                                   ops=OracleOps(w), device="cpu")
@@ -185,11 +185,12 @@ def _run(rank, q):
         q.put((rank, res))
 
 
-def test_two_ranks_match_the_whole_sequence():
+@pytest.mark.parametrize("R", [2, 3])
+def test_ranks_match_the_whole_sequence(R):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, port, q)) for r in range(R)]
+    procs = [ctx.Process(target=_worker, args=(r, R, port, q)) for r in range(R)]
     for p in procs:
         p.start()
     got = dict(q.get(timeout=300) for _ in procs)
@@ -200,9 +201,10 @@ def test_two_ranks_match_the_whole_sequence():
     for p in procs:
         assert p.exitcode == 0
     # every rank holds the same results
-    for a, b in zip(got[0], got[1]):
-        for x, y in zip(a, b):
-            assert np.array_equal(x, y)
+    for r in range(1, R):
+        for a, b in zip(got[0], got[r]):
+            for x, y in zip(a, b):
+                assert np.array_equal(x, y)
     sys.path.insert(0, HERE)
     import oracle
     from harness import band_set_check, build_ref_cache, host_layer
