@@ -213,8 +213,8 @@ class Cache:
                              v.lens.data_ptr(), 1, 0, c.page_size, c.dim, c.idx_dim, c.row_stride, st,
                              self.n_slots - base, c.idx_key_dtype)
         else:
-            if pos0 % self.page_size:
-                raise ValueError("a paged shard starts on a page boundary")
+            if pos0 % self.page_size or pos0 + n > self.capacity:
+                raise ValueError("a paged shard starts on a page boundary and ends within the sequence's pages")
             first = pos0 // self.page_size
             v.c = csa2_cache(c.kv_rows, c.idx_keys, c.page_table + 4 * (b * c.max_pages + first), v.lens.data_ptr(),
                              1, c.max_pages - first, c.page_size, c.dim, c.idx_dim, c.row_stride, 0, c.n_slots,

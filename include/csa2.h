@@ -458,7 +458,9 @@ CSA2_API csa2_status csa2_cp_reindex_select(const int32_t* pool_idx, const float
  * broken arbitrarily.  Positions must be distinct.  1 <= n_b <= n_a <= 16384
  * (or n_b = 0), R * n_cand <= 2^24.  ws is a separate workspace of
  * csa2_cp_merge_workspace_bytes(R, batch, n_cand) bytes (0 on invalid
- * arguments), cleared once with csa2_workspace_init.
+ * arguments), cleared once with csa2_workspace_init; its status word (a
+ * selection's bounded barrier that ran out: CSA2_ERR_TIMEOUT) is read with
+ * csa2_read_device_status.
  */
 CSA2_API size_t csa2_cp_merge_workspace_bytes(int R, int batch, int n_cand);
 CSA2_API csa2_status csa2_cp_merge_select(const csa2_cand* cand, int R, int batch, int n_cand,
